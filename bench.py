@@ -1,0 +1,450 @@
+"""Benchmark of the frame-wise GDN frame scan on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                [--config NAME] [--e2e-steps K2] [--no-cpu-baseline]
+
+One step = one full pass of the scan (contraction, chunk composition, prefix,
+replay, readout) over one batch of the workload, inputs resident in HBM. The
+default workload is the 60 s 720p rollout, one GDN layer: B=1, H=16, D=128,
+S=80x45=3600 tokens per latent frame, T=121 latent frames, bf16 q/k/v, fp32
+state, chunk-parallel scan (8-frame spans).
+
+Metric: frame·head·tokens/s = B*H*T*S / step time, and the fraction of the
+HBM roofline. Under torchrun (N>1) every rank runs its own copy of the
+workload on its own GPU (the heads shard with no data-path collective: weak
+scaling); NCCL carries only the barrier and the max-over-ranks timing.
+
+--impl reference times the float64 CPU oracle (the reference implementation
+of this build) on a bounded sample of the same workload, on rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from frame_wise_gated_b200 import synth  # noqa: E402
+
+METRIC = "GDN frame-scan frame·head·tokens/s (% of HBM roofline), 1xB200"
+UNIT = "frame·head·tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+def algorithmic_bytes(cfg, step=True):
+    """Bytes the method must move per step: q, k, v in and o out (raw q, k
+    plus two outputs for the bidirectional prologue workload), beta and gamma,
+    and the per-head state in/out."""
+    e = 2 if cfg.bf16 else 4
+    n_t = 5 if cfg.prologue else 4
+    per_fh = cfg.S * (n_t * cfg.D * e + 4) + 4
+    state = 2 * cfg.D * cfg.D * 4
+    return cfg.frame_heads * per_fh + cfg.B * cfg.H * state
+
+
+def phase_bytes(cfg):
+    """Algorithmic bytes per launch of each kernel phase (per frame-head
+    figure x frame-heads)."""
+    e = 2 if cfg.bf16 else 4
+    fh = cfg.frame_heads
+    nro = 2 if cfg.bidir_block else 1
+    return {
+        "contract": fh * cfg.S * (2 * cfg.D * e + 4),          # K, V, beta
+        "readout": fh * cfg.S * 2 * cfg.D * e,                  # Q in, O out
+        "prologue": fh * cfg.S * 4 * cfg.D * e,                 # raw q, k in; q^, k^ out
+        "_readout_launches_per_step": nro,
+    }
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("hbm_gbs", FALLBACK_HBM_GBS), d.get("bf16_tflops", FALLBACK_BF16_TFLOPS), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def csrc_digest():
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "frame_wise_gated_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_phase, cfg_name):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources and this workload; else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+    except ValueError:
+        return None
+    ent = d.get(kernel_phase)
+    if not ent or ent.get("csrc_sha") != csrc_digest() or ent.get("workload") != cfg_name:
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_sample(cfg, frames=None, slab=(0, 0)):
+    """Times the float64 oracle on one (b, h) slab (first `frames` frames).
+    Returns (tokens per second, seconds, tokens, description)."""
+    from oracle import gdn_oracle as O
+    b, h = slab
+    sl = synth.make_slab(cfg, b, h)
+    T = cfg.T if frames is None else min(frames, cfg.T)
+    wid = (lambda x: synth.bf16_bits_to_f32(x[:T]).astype(np.float64)) if cfg.bf16 else \
+        (lambda x: x[:T].astype(np.float64))
+    q, k, v = wid(sl["q"]), wid(sl["k"]), wid(sl["v"])
+    beta = sl["beta"][:T].astype(np.float64)
+    gamma = sl["gamma"][:T].astype(np.float64)
+    st = synth.make_state(cfg)
+    s0 = None if st is None else st[b, h]
+    t0 = time.perf_counter()
+    if cfg.prologue:
+        wq, wk = synth.make_weights(cfg)
+        qh, kh = O.qk_prologue(q, k, wq, wk, cfg.grid_w)
+        O.frame_scan(qh, kh, v, beta, gamma, s0, keys_scaled=True)
+        O.frame_scan(qh, kh, v, beta, gamma, s0, reverse=True, block=cfg.bidir_block,
+                     keys_scaled=True)
+    else:
+        O.frame_scan(q, k, v, beta, gamma, s0)
+    dt = time.perf_counter() - t0
+    toks = T * cfg.S
+    return toks / dt, dt, toks, f"one (b,h) slab, {T} of {cfg.T} frames x {cfg.S} tokens"
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, cfg):
+    rank = env_int("RANK", 0)
+    if rank != 0:
+        return 0
+    frames = max(1, min(cfg.T, args.ref_frames))
+    times = []
+    for i in range(args.warmup + args.steps):
+        _, dt, toks, desc = cpu_oracle_sample(cfg, frames=frames, slab=(0, i % cfg.H))
+        if i >= args.warmup:
+            times.append(dt)
+    tot = sum(times)
+    value = toks * len(times) / tot
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "T": cfg.T, "S": cfg.S,
+                   "D": cfg.D, "sample_per_step": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
+                         "sample": f"{desc} per step; float64 NumPy oracle as it stands"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, cfg):
+    import torch
+    from frame_wise_gated_b200 import api, build
+
+    world = env_int("WORLD_SIZE", 1)
+    rank = env_int("RANK", 0)
+    local = env_int("LOCAL_RANK", 0)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    build.build()
+    api.lib()
+
+    # ---- inputs (seeded, synthetic), resident in HBM ----
+    arr = synth.make_inputs(cfg)
+    et = torch.bfloat16 if cfg.bf16 else torch.float32
+
+    def dev_t(x):
+        t = torch.from_numpy(x)
+        if cfg.bf16 and x.dtype == np.uint16:
+            t = t.view(torch.bfloat16)
+        return t.to(dev)
+
+    q, k, v = dev_t(arr["q"]), dev_t(arr["k"]), dev_t(arr["v"])
+    beta = torch.from_numpy(arr["beta"]).to(dev)
+    gamma = torch.from_numpy(arr["gamma"]).to(dev)
+    s0 = None if arr["state"] is None else torch.from_numpy(arr["state"]).to(dev)
+    pro = None
+    if cfg.prologue:
+        pro = dict(w_q=torch.from_numpy(arr["w_q"]).to(dev), w_k=torch.from_numpy(arr["w_k"]).to(dev),
+                   grid_h=cfg.grid_h, grid_w=cfg.grid_w)
+    kw = dict(prologue=pro, bidir=bool(cfg.bidir_block), block_reset=bool(cfg.bidir_block),
+              block=cfg.bidir_block or 3, sequential=args.sequential)
+    out = torch.empty_like(q)
+    out_rev = torch.empty_like(q) if cfg.bidir_block else None
+    st_out = torch.empty((cfg.B, cfg.H, cfg.D, cfg.D), device=dev, dtype=torch.float32)
+    st_rev = torch.empty_like(st_out) if cfg.bidir_block else None
+    flags = api.scan_flags(bf16=cfg.bf16, prologue=pro is not None, bidir=bool(cfg.bidir_block),
+                           block_reset=bool(cfg.bidir_block), block=cfg.bidir_block or 3,
+                           sequential=args.sequential)
+    ws = torch.empty(api.workspace_bytes(cfg.B, cfg.H, cfg.T, cfg.S, cfg.D, flags),
+                     device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        api.frame_scan_fwd_ex(q, k, v, beta, gamma, s0, out=out, state_out=st_out,
+                              out_rev=out_rev, state_out_rev=st_rev, workspace=ws, **kw)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    api.check_device_status()
+
+    # ---- timed region: K steps, CUDA events on the launch stream ----
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    api.launch_count(reset=True)
+    api.profile_enable(True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    launches = api.launch_count(reset=True)
+    phases = api.profile_read()
+    api.profile_enable(False)
+    clk = clocks.stop()
+    api.check_device_status()
+    ms = ev0.elapsed_time(ev1)
+    if dist is not None:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    tokens_all = cfg.tokens * world
+    value = tokens_all / (ms_step * 1e-3)
+
+    # ---- dominant kernel roofline (live per-kernel events over the timed region) ----
+    hbm, bf16_tf, peak_kind = peaks()
+    pb = phase_bytes(cfg)
+    dom = max((p for p in phases if phases[p][1] > 0), key=lambda p: phases[p][0])
+    dom_ms = phases[dom][0] / phases[dom][1]
+    alg = pb.get(dom)
+    if dom == "readout":
+        alg = pb["readout"]
+    roof = None
+    if alg is not None:
+        ach = alg / (dom_ms * 1e-3) / 1e9
+        traffic = ncu_traffic(dom, cfg.name)
+        roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
+                "frac": ach / hbm, "traffic": traffic, "peak_source": peak_kind,
+                "alg_bytes_per_launch": alg, "ms_per_launch": dom_ms}
+    step_bytes = algorithmic_bytes(cfg)
+    step_roof = {"alg_bytes_per_step": step_bytes, "achieved_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
+                 "frac": step_bytes / (ms_step * 1e-3) / 1e9 / hbm}
+
+    # ---- end to end through the C ABI with host buffers ----
+    e2e = None
+    if args.e2e_steps > 0:
+        e2e = run_e2e(args, cfg, arr, dev, api, barrier, dist, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        frames = max(1, min(cfg.T, args.ref_frames_baseline))
+        val, dt, toks, desc = cpu_oracle_sample(cfg, frames=frames)
+        cpu = {"value": val, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
+               "sample": f"{desc}; {dt:.1f} s of float64 NumPy oracle"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if cfg.bf16 else "f32", "data": "synthetic",
+            "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "T": cfg.T, "S": cfg.S,
+                       "D": cfg.D, "grid": f"{cfg.grid_w}x{cfg.grid_h}",
+                       "scan": "sequential" if args.sequential else "chunked (8-frame spans)",
+                       "prologue": cfg.prologue, "bidir_block": cfg.bidir_block,
+                       "l2": f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB algorithmic per step)",
+                       "parallelism": f"replica x{world} (heads shard, no collective)"},
+            "roofline": roof, "step_roofline": step_roof,
+            "phases_ms_per_step": {p: phases[p][0] / args.steps for p in phases if phases[p][1]},
+            "gpu_launches": launches, "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(args, cfg, arr, dev, api, barrier, dist, world):
+    """Same metric through the plain C-ABI entry (gdn_frame_scan_fwd, library
+    scratch) with host buffers: every step copies the inputs from pinned host
+    memory to the device and the outputs back, inside the timed region."""
+    import torch
+    if cfg.prologue:
+        return None  # the fused prologue is reachable only through the _ex entry
+    et = torch.bfloat16 if cfg.bf16 else torch.float32
+
+    def pinned(x):
+        t = torch.from_numpy(x)
+        if cfg.bf16 and x.dtype == np.uint16:
+            t = t.view(torch.bfloat16)
+        return t.pin_memory()
+
+    hq, hk, hv = pinned(arr["q"]), pinned(arr["k"]), pinned(arr["v"])
+    hb, hg = pinned(arr["beta"]), pinned(arr["gamma"])
+    hs0 = None if arr["state"] is None else pinned(arr["state"])
+    dq, dk, dv = (torch.empty(x.shape, dtype=x.dtype, device=dev) for x in (hq, hk, hv))
+    db, dg = torch.empty(hb.shape, device=dev), torch.empty(hg.shape, device=dev)
+    ds0 = None if hs0 is None else torch.empty(hs0.shape, device=dev)
+    hout = torch.empty(hq.shape, dtype=hq.dtype).pin_memory()
+    hst = torch.empty((cfg.B, cfg.H, cfg.D, cfg.D), dtype=torch.float32).pin_memory()
+    dout = torch.empty_like(dq)
+    dst = torch.empty((cfg.B, cfg.H, cfg.D, cfg.D), device=dev)
+    h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hb, hg) + ((hs0,) if hs0 is not None else ()))
+    d2h = hout.numel() * hout.element_size() + hst.numel() * 4
+
+    def step():
+        for d_, h_ in ((dq, hq), (dk, hk), (dv, hv), (db, hb), (dg, hg)):
+            d_.copy_(h_, non_blocking=True)
+        if ds0 is not None:
+            ds0.copy_(hs0, non_blocking=True)
+        api.frame_scan_fwd(dq, dk, dv, db, dg, ds0, out=dout, state_out=dst,
+                           sequential=args.sequential)
+        hout.copy_(dout, non_blocking=True)
+        hst.copy_(dst, non_blocking=True)
+
+    for _ in range(1):
+        step()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.e2e_steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    if dist is not None:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.e2e_steps
+    return {"value": cfg.tokens * world / (ms_step * 1e-3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_step,
+            "steps": args.e2e_steps, "entry": "gdn_frame_scan_fwd (host buffers, pinned)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="rollout60s_720p", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--sequential", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-frames", type=int, default=6,
+                    help="frames of one slab per reference step")
+    ap.add_argument("--ref-frames-baseline", type=int, default=40,
+                    help="frames of one slab for the cpu_baseline sample")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    cfg = synth.CONFIGS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+    return run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,489 @@
+// C ABI of libgdnscan.so: argument checks, workspace layout and the launch plan.
+//
+// The plan for one call (SANA-WM blog, blog.hotdry.top: recurrence in section
+// 混合线性注意力, span composition and prologue order in the Context-Parallel
+// section; reverse scan with block resets per the hyper.ai summary, 方法):
+//   [prologue]  RMSNorm -> ReLU -> key scale -> RoPE on raw q, k   (a1)
+//   contract    A_t, U_t for every frame-head                     (a2)
+//   per direction:
+//     chunked:    compose (E_p, H_p, g_p) per span                (a3)
+//                 prefix over spans -> span start states          (a4)
+//                 replay each span from its start state           (a5)
+//     sequential: one chain over T                                (a4+a5)
+//     blocks:     one chain per reset block                       (a5)
+//     readout     O_t = Q_t S_t^T                                 (a6)
+#include <stdio.h>
+#include <string.h>
+
+#include <cmath>
+#include <string>
+#include <vector>
+
+#include "gdn_internal.cuh"
+
+namespace gdn {
+
+static thread_local std::string t_last_error;
+static thread_local long long t_launches = 0;
+
+void count_launch(int n) { t_launches += n; }
+
+// ---- phase timing with CUDA events (gdn_profile_enable / gdn_profile_read) ----
+enum Phase { PH_PROLOGUE = 0, PH_CONTRACT, PH_COMPOSE, PH_PREFIX, PH_SCAN, PH_READOUT, PH_COUNT };
+struct ProfRec {
+  int phase;
+  cudaEvent_t a, b;
+};
+struct Profiler {
+  bool on = false;
+  std::vector<ProfRec> recs;
+  std::vector<cudaEvent_t> pool;
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+  void recycle() {
+    for (auto& r : recs) {
+      pool.push_back(r.a);
+      pool.push_back(r.b);
+    }
+    recs.clear();
+  }
+};
+static thread_local Profiler t_prof;
+
+struct PhaseScope {
+  cudaStream_t st;
+  int idx = -1;
+  PhaseScope(int phase, cudaStream_t s) : st(s) {
+    if (!t_prof.on) return;
+    ProfRec r{phase, t_prof.get(), t_prof.get()};
+    cudaEventRecord(r.a, st);
+    t_prof.recs.push_back(r);
+    idx = (int)t_prof.recs.size() - 1;
+  }
+  ~PhaseScope() {
+    if (idx >= 0) cudaEventRecord(t_prof.recs[idx].b, st);
+  }
+};
+
+static int fail(int status, const char* fmt, const char* detail = "") {
+  char buf[512];
+  snprintf(buf, sizeof(buf), fmt, detail);
+  t_last_error = buf;
+  return status;
+}
+
+static int cuda_fail(cudaError_t e, const char* where) {
+  char buf[512];
+  snprintf(buf, sizeof(buf), "%s: %s", where, cudaGetErrorString(e));
+  t_last_error = buf;
+  return GDN_ERR_CUDA;
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static bool valid_D(int D) { return D == 16 || D == 32 || D == 64 || D == 128 || D == 256; }
+
+static int block_len(unsigned flags) {
+  int b = (int)GDN_BLOCK(flags);
+  return b ? b : 3;
+}
+static int chunk_len(unsigned flags) {
+  int c = (int)GDN_CHUNK(flags);
+  return c ? c : 8;
+}
+
+Layout make_layout(int B, int H, int T, int S, int D, unsigned flags) {
+  Layout L;
+  const size_t heads = (size_t)B * H;
+  const size_t frames = heads * T;
+  const size_t mat = (size_t)D * D * sizeof(float);
+  const int nchunk = (T + chunk_len(flags) - 1) / chunk_len(flags);
+  const int nblock = (T + block_len(flags) - 1) / block_len(flags);
+  L.nseg_max = nchunk > nblock ? nchunk : nblock;
+  size_t off = 0;
+  L.A = off;
+  off = align256(off + frames * mat);
+  L.U = off;
+  off = align256(off + frames * mat);
+  L.Sfr = off;
+  off = align256(off + frames * mat);  // fp32, or bf16 hi+lo: the same bytes
+  L.E = off;
+  off = align256(off + heads * L.nseg_max * mat);
+  L.Hc = off;
+  off = align256(off + heads * L.nseg_max * mat);
+  L.Sst = off;
+  off = align256(off + heads * L.nseg_max * mat);
+  L.g = off;
+  off = align256(off + heads * L.nseg_max * sizeof(float));
+  L.qh = L.kh = off;
+  if (flags & GDN_FUSED_PROLOGUE) {
+    const size_t elt = (flags & GDN_BF16) ? 2 : 4;
+    const size_t tens = frames * (size_t)S * D * elt;
+    L.qh = off;
+    off = align256(off + tens);
+    L.kh = off;
+    off = align256(off + tens);
+  }
+  L.total = off;
+  return L;
+}
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+static int device_cc_major() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return 0;
+  return major;
+}
+
+static int check_sizes(int B, int H, int T, int S, int D) {
+  if (B < 1 || H < 1 || T < 1 || S < 1)
+    return fail(GDN_ERR_INVALID, "sizes must be >= 1%s");
+  if (!valid_D(D)) return fail(GDN_ERR_UNSUPPORTED, "D must be 16, 32, 64, 128 or 256%s");
+  if (S > 65535 * 64) return fail(GDN_ERR_UNSUPPORTED, "S above 4194240%s");
+  const long long frames = (long long)B * H * T;
+  if (frames > (1LL << 31) - 1) return fail(GDN_ERR_UNSUPPORTED, "B*H*T too large%s");
+  return GDN_OK;
+}
+
+// Runs one direction of the scan from A, U already in the workspace.
+static int run_direction(const gdn_params& p, const Layout& L, char* ws, bool reverse,
+                         bool block_reset, const void* q, void* out, float* state_out,
+                         bool use_tc_chain, bool use_tc_readout, cudaStream_t st) {
+  const bool bf16 = (p.flags & GDN_BF16) != 0;
+  const long long frames = (long long)p.B * p.H * p.T;
+  ChainArgs a;
+  memset(&a, 0, sizeof(a));
+  a.D = p.D;
+  a.T = p.T;
+  a.L = chunk_len(p.flags);
+  a.block = block_len(p.flags);
+  a.reverse = reverse ? 1 : 0;
+  a.heads = p.B * p.H;
+  a.A = (const float*)(ws + L.A);
+  a.U = (const float*)(ws + L.U);
+  a.gamma = p.gamma;
+  a.state_in = p.state_in;
+  a.state_out = state_out;
+  a.Sfr = (float*)(ws + L.Sfr);
+  a.sfr_hilo = use_tc_readout ? 1 : 0;
+  a.E = (float*)(ws + L.E);
+  a.Hc = (float*)(ws + L.Hc);
+  a.g = (float*)(ws + L.g);
+  a.Sst = (float*)(ws + L.Sst);
+
+  auto chain = [&](const ChainArgs& c, int n) -> cudaError_t {
+    PhaseScope ps(c.mode == CHAIN_COMPOSE ? PH_COMPOSE : c.mode == CHAIN_PREFIX ? PH_PREFIX : PH_SCAN,
+                  st);
+    return use_tc_chain ? tc_chain(c, n, st) : simt_chain(c, n, st);
+  };
+  cudaError_t e;
+  if (p.flags & GDN_SEQUENTIAL) {
+    a.seg = SEG_SEQUENTIAL;
+    a.seq_reset = block_reset ? 1 : 0;
+    a.nseg = 1;
+    a.mode = CHAIN_SCAN;
+    if ((e = chain(a, a.heads)) != cudaSuccess) return cuda_fail(e, "scan chain");
+  } else if (block_reset) {
+    a.seg = SEG_BLOCKS;
+    a.nseg = (p.T + a.block - 1) / a.block;
+    a.mode = CHAIN_SCAN;
+    if ((e = chain(a, a.heads * a.nseg)) != cudaSuccess) return cuda_fail(e, "block chains");
+  } else {
+    a.seg = SEG_CHUNKS;
+    a.nseg = (p.T + a.L - 1) / a.L;
+    if (a.nseg == 1) {
+      a.mode = CHAIN_SCAN;
+      if ((e = chain(a, a.heads)) != cudaSuccess) return cuda_fail(e, "scan chain");
+    } else {
+      a.mode = CHAIN_COMPOSE;
+      if ((e = chain(a, 2 * a.heads * a.nseg)) != cudaSuccess) return cuda_fail(e, "compose");
+      a.mode = CHAIN_PREFIX;
+      if ((e = chain(a, a.heads)) != cudaSuccess) return cuda_fail(e, "prefix");
+      a.mode = CHAIN_SCAN;
+      if ((e = chain(a, a.heads * a.nseg)) != cudaSuccess) return cuda_fail(e, "replay");
+    }
+  }
+  {
+    PhaseScope ps(PH_READOUT, st);
+    if (use_tc_readout)
+      e = tc_readout(q, ws + L.Sfr, out, frames, p.S, p.D, st);
+    else
+      e = simt_readout(bf16, q, (const float*)(ws + L.Sfr), out, frames, p.S, p.D, st);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "readout");
+  return GDN_OK;
+}
+
+static int scan_ex(const gdn_params& p, cudaStream_t st) {
+  int rc = check_sizes(p.B, p.H, p.T, p.S, p.D);
+  if (rc) return rc;
+  const unsigned f = p.flags;
+  if (!p.q || !p.k || !p.v || !p.beta || !p.gamma || !p.out)
+    return fail(GDN_ERR_INVALID, "null q/k/v/beta/gamma/out%s");
+  if (!aligned16(p.q) || !aligned16(p.k) || !aligned16(p.v) || !aligned16(p.out) ||
+      !aligned16(p.beta) || !aligned16(p.gamma))
+    return fail(GDN_ERR_INVALID, "pointers must be 16-byte aligned%s");
+  if (p.out == p.q || p.out == p.k || p.out == p.v)
+    return fail(GDN_ERR_INVALID, "out must not alias q, k or v%s");
+  if ((f & GDN_BIDIR) && (!p.out_rev || p.out_rev == p.out || !aligned16(p.out_rev)))
+    return fail(GDN_ERR_INVALID, "GDN_BIDIR needs a separate, aligned out_rev%s");
+  if ((f & GDN_BIDIR) && (f & GDN_REVERSE))
+    return fail(GDN_ERR_INVALID, "GDN_BIDIR and GDN_REVERSE are exclusive%s");
+  if (f & GDN_FUSED_PROLOGUE) {
+    if (!p.w_q || !p.w_k) return fail(GDN_ERR_INVALID, "prologue needs w_q and w_k%s");
+    if (p.grid_h < 1 || p.grid_w < 1 || (long long)p.grid_h * p.grid_w != p.S)
+      return fail(GDN_ERR_INVALID, "prologue needs grid_h * grid_w == S%s");
+    if (f & GDN_KEYS_SCALED)
+      return fail(GDN_ERR_INVALID, "GDN_FUSED_PROLOGUE applies the key scale itself%s");
+  }
+  const Layout L = make_layout(p.B, p.H, p.T, p.S, p.D, f);
+  if (!p.workspace || p.workspace_bytes < L.total)
+    return fail(GDN_ERR_WORKSPACE, "workspace missing or smaller than gdn_workspace_bytes%s");
+  if (((uintptr_t)p.workspace & 255u) != 0)
+    return fail(GDN_ERR_INVALID, "workspace must be 256-byte aligned%s");
+
+  const bool bf16 = (f & GDN_BF16) != 0;
+  const bool sm100 = device_cc_major() == 10;
+  const bool simt = (f & GDN_FORCE_SIMT) || !bf16 || !sm100;
+  const bool tc_contract_ok = !simt && tc_contract_supported(p.D);
+  const bool tc_readout_ok = !simt && tc_readout_supported(p.D);
+  const bool tc_chain_ok = !simt && tc_chain_supported(p.D);
+  char* ws = (char*)p.workspace;
+  const long long frames = (long long)p.B * p.H * p.T;
+  cudaError_t e;
+
+  const void* q = p.q;
+  const void* k = p.k;
+  bool keys_scaled = (f & GDN_KEYS_SCALED) != 0;
+  if (f & GDN_FUSED_PROLOGUE) {
+    const float eps = p.eps > 0.f ? p.eps : 1e-6f;
+    const float base = p.rope_base > 0.f ? p.rope_base : 10000.f;
+    const float ks = (float)(1.0 / std::sqrt((double)p.D * (double)p.S));
+    {
+      PhaseScope ps(PH_PROLOGUE, st);
+      e = simt_prologue(bf16, p.q, p.k, p.w_q, p.w_k, ws + L.qh, ws + L.kh, frames, p.S,
+                        p.grid_w, p.D, eps, base, ks, st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "prologue");
+    q = ws + L.qh;
+    k = ws + L.kh;
+    keys_scaled = true;
+  }
+  const double c = keys_scaled ? 1.0 : 1.0 / std::sqrt((double)p.D * (double)p.S);
+  float* A = (float*)(ws + L.A);
+  float* U = (float*)(ws + L.U);
+  {
+    PhaseScope ps(PH_CONTRACT, st);
+    if (tc_contract_ok)
+      e = tc_contract(k, p.v, p.beta, A, U, frames, p.S, p.D, (float)(c * c), (float)c, st);
+    else
+      e = simt_contract(bf16, k, p.v, p.beta, A, U, frames, p.S, p.D, (float)(c * c), (float)c,
+                        st);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "contract");
+
+  const bool block_reset = (f & GDN_BLOCK_RESET) != 0;
+  if (f & GDN_BIDIR) {
+    rc = run_direction(p, L, ws, false, false, q, p.out, p.state_out, tc_chain_ok,
+                       tc_readout_ok, st);
+    if (rc) return rc;
+    return run_direction(p, L, ws, true, block_reset, q, p.out_rev, p.state_out_rev,
+                         tc_chain_ok, tc_readout_ok, st);
+  }
+  return run_direction(p, L, ws, (f & GDN_REVERSE) != 0, block_reset, q, p.out, p.state_out,
+                       tc_chain_ok, tc_readout_ok, st);
+}
+
+}  // namespace gdn
+
+using namespace gdn;
+
+extern "C" {
+
+int gdn_version(void) { return 100; }
+
+const char* gdn_status_string(int s) {
+  switch (s) {
+    case GDN_OK: return "ok";
+    case GDN_ERR_INVALID: return "invalid argument";
+    case GDN_ERR_UNSUPPORTED: return "unsupported size";
+    case GDN_ERR_CUDA: return "CUDA error";
+    case GDN_ERR_TIMEOUT: return "device wait timed out";
+    case GDN_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+const char* gdn_last_error(void) { return t_last_error.c_str(); }
+
+long long gdn_launch_count(int reset) {
+  long long n = t_launches;
+  if (reset) t_launches = 0;
+  return n;
+}
+
+size_t gdn_workspace_bytes(int B, int H, int T, int S, int D, unsigned flags) {
+  if (B < 1 || H < 1 || T < 1 || S < 1 || !valid_D(D)) return 0;
+  return make_layout(B, H, T, S, D, flags).total;
+}
+
+int gdn_frame_scan_fwd_ex(const gdn_params* p, gdn_stream_t stream) {
+  t_last_error.clear();
+  if (!p) return fail(GDN_ERR_INVALID, "null params%s");
+  return scan_ex(*p, (cudaStream_t)stream);
+}
+
+int gdn_frame_scan_fwd(const void* q, const void* k, const void* v, const float* beta,
+                       const float* gamma, const float* state_in, void* out, float* state_out,
+                       int B, int H, int T, int S, int D, unsigned flags, gdn_stream_t stream) {
+  t_last_error.clear();
+  if (flags & (GDN_FUSED_PROLOGUE | GDN_BIDIR))
+    return fail(GDN_ERR_INVALID, "GDN_FUSED_PROLOGUE / GDN_BIDIR need gdn_frame_scan_fwd_ex%s");
+  int rc = check_sizes(B, H, T, S, D);
+  if (rc) return rc;
+  gdn_params p;
+  memset(&p, 0, sizeof(p));
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.beta = beta;
+  p.gamma = gamma;
+  p.state_in = state_in;
+  p.out = out;
+  p.state_out = state_out;
+  p.B = B;
+  p.H = H;
+  p.T = T;
+  p.S = S;
+  p.D = D;
+  p.flags = flags;
+  p.workspace_bytes = make_layout(B, H, T, S, D, flags).total;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMallocAsync(&p.workspace, p.workspace_bytes, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+  rc = scan_ex(p, st);
+  e = cudaFreeAsync(p.workspace, st);
+  if (rc == GDN_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(workspace)");
+  return rc;
+}
+
+int gdn_qk_prologue(const void* q_raw, const void* k_raw, const float* w_q, const float* w_k,
+                    void* q_out, void* k_out, int B, int H, int T, int grid_h, int grid_w, int D,
+                    float eps, float rope_base, unsigned flags, gdn_stream_t stream) {
+  t_last_error.clear();
+  if (grid_h < 1 || grid_w < 1) return fail(GDN_ERR_INVALID, "grid must be >= 1%s");
+  const long long S = (long long)grid_h * grid_w;
+  if (S > 65535 * 64) return fail(GDN_ERR_UNSUPPORTED, "S above 4194240%s");
+  int rc = check_sizes(B, H, T, (int)S, D);
+  if (rc) return rc;
+  if (!q_raw || !k_raw || !w_q || !w_k || !q_out || !k_out)
+    return fail(GDN_ERR_INVALID, "null pointer%s");
+  if (q_out == q_raw || q_out == k_raw || k_out == q_raw || k_out == k_raw || q_out == k_out)
+    return fail(GDN_ERR_INVALID, "outputs must not alias inputs%s");
+  const float ks = (float)(1.0 / std::sqrt((double)D * (double)S));
+  cudaError_t e = simt_prologue((flags & GDN_BF16) != 0, q_raw, k_raw, w_q, w_k, q_out, k_out,
+                                (long long)B * H * T, (int)S, grid_w, D,
+                                eps > 0.f ? eps : 1e-6f, rope_base > 0.f ? rope_base : 10000.f,
+                                ks, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "prologue");
+  return GDN_OK;
+}
+
+int gdn_frame_contract(const void* k, const void* v, const float* beta, float* A, float* U,
+                       int N, int S, int D, unsigned flags, gdn_stream_t stream) {
+  t_last_error.clear();
+  int rc = check_sizes(1, 1, N, S, D);
+  if (rc) return rc;
+  if (!k || !v || !beta || !A || !U) return fail(GDN_ERR_INVALID, "null pointer%s");
+  const bool bf16 = (flags & GDN_BF16) != 0;
+  const double c = (flags & GDN_KEYS_SCALED) ? 1.0 : 1.0 / std::sqrt((double)D * (double)S);
+  const bool tc = bf16 && !(flags & GDN_FORCE_SIMT) && device_cc_major() == 10 &&
+                  tc_contract_supported(D);
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = tc ? tc_contract(k, v, beta, A, U, N, S, D, (float)(c * c), (float)c, st)
+                     : simt_contract(bf16, k, v, beta, A, U, N, S, D, (float)(c * c),
+                                     (float)c, st);
+  if (e != cudaSuccess) return cuda_fail(e, "contract");
+  return GDN_OK;
+}
+
+int gdn_chunk_composites(const float* A, const float* U, const float* gamma, float* E, float* Hc,
+                         float* g, int N, int L, int D, unsigned flags, gdn_stream_t stream) {
+  t_last_error.clear();
+  int rc = check_sizes(1, N, L, 1, D);
+  if (rc) return rc;
+  if (!A || !U || !gamma || !E || !Hc || !g) return fail(GDN_ERR_INVALID, "null pointer%s");
+  ChainArgs a;
+  memset(&a, 0, sizeof(a));
+  a.mode = CHAIN_COMPOSE;
+  a.seg = SEG_CHUNKS;
+  a.D = D;
+  a.T = L;
+  a.L = L;
+  a.block = 3;
+  a.nseg = 1;
+  a.heads = N;
+  a.A = A;
+  a.U = U;
+  a.gamma = gamma;
+  a.E = E;
+  a.Hc = Hc;
+  a.g = g;
+  const bool tc = !(flags & GDN_FORCE_SIMT) && device_cc_major() == 10 && tc_chain_supported(D);
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = tc ? tc_chain(a, 2 * N, st) : simt_chain(a, 2 * N, st);
+  if (e != cudaSuccess) return cuda_fail(e, "compose");
+  return GDN_OK;
+}
+
+int gdn_profile_enable(int enable) {
+  if (enable) t_prof.recycle();
+  t_prof.on = enable != 0;
+  return GDN_OK;
+}
+
+int gdn_profile_read(double* ms, long long* counts, int n) {
+  if (!ms || !counts || n < 1) return fail(GDN_ERR_INVALID, "null or empty output%s");
+  const int np = n < PH_COUNT ? n : PH_COUNT;
+  for (int i = 0; i < np; ++i) {
+    ms[i] = 0.0;
+    counts[i] = 0;
+  }
+  for (auto& r : t_prof.recs) {
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e != cudaSuccess) return cuda_fail(e, "profile event");
+    float t = 0.f;
+    e = cudaEventElapsedTime(&t, r.a, r.b);
+    if (e != cudaSuccess) return cuda_fail(e, "profile elapsed");
+    if (r.phase < np) {
+      ms[r.phase] += t;
+      counts[r.phase] += 1;
+    }
+  }
+  return np;
+}
+
+int gdn_check_device_status(gdn_stream_t stream) {
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  int status = 0;
+  e = tc_read_status(&status, st);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (status) return fail(GDN_ERR_TIMEOUT, "a device-side wait ran out (code %s)",
+                          status == 1 ? "mbarrier" : "other");
+  return GDN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,130 @@
+// Internal declarations shared by the kernels and the C ABI of libgdnscan.so.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "gdn.h"
+
+namespace gdn {
+
+// ---- scalar load/store by element type -------------------------------------
+template <typename T>
+__device__ __forceinline__ float ldf(const T* p);
+template <>
+__device__ __forceinline__ float ldf<float>(const float* p) { return *p; }
+template <>
+__device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(*p);
+}
+template <typename T>
+__device__ __forceinline__ void stf(T* p, float x);
+template <>
+__device__ __forceinline__ void stf<float>(float* p, float x) { *p = x; }
+template <>
+__device__ __forceinline__ void stf<__nv_bfloat16>(__nv_bfloat16* p, float x) {
+  *p = __float2bfloat16_rn(x);
+}
+
+// ---- scan plan ---------------------------------------------------------------
+// How the frames of one direction are cut into chains of the recurrence.
+enum SegMode : int {
+  SEG_SEQUENTIAL = 0,  // one chain over all T frames (block resets inside it)
+  SEG_CHUNKS = 1,      // uniform spans of L frames in scan order, composed
+  SEG_BLOCKS = 2,      // one chain per reset block (blocks are independent)
+};
+
+enum ChainMode : int {
+  CHAIN_SCAN = 0,     // S <- gamma (S - S A) + U per frame, store S_t
+  CHAIN_COMPOSE = 1,  // per span: E <- E + A - E A and H <- gamma (H - H A) + U
+  CHAIN_PREFIX = 2,   // per head: S_start(p+1) = g_p (S_start(p) - S_start(p) E_p) + H_p
+};
+
+// Everything the chain kernels need; pointers are device pointers.
+struct ChainArgs {
+  int mode;       // ChainMode
+  int seg;        // SegMode
+  int D, T;
+  int L;          // chunk length (SEG_CHUNKS)
+  int block;      // reset block length (SEG_BLOCKS, or resets inside SEG_SEQUENTIAL)
+  int seq_reset;  // SEG_SEQUENTIAL: zero the state on entering a new block
+  int reverse;
+  int nseg;       // chains per head: 1, ceil(T/L) or ceil(T/block)
+  int heads;      // B*H
+  const float* A;         // [heads*T, D, D]
+  const float* U;         // [heads*T, D, D]
+  const float* gamma;     // [heads*T]
+  const float* state_in;  // [heads, D, D] or null
+  float* state_out;       // [heads, D, D] or null
+  float* Sfr;             // per-frame states [heads*T, D, D] fp32, or bf16 hi/lo pairs
+  int sfr_hilo;           // 1: Sfr holds [heads*T][2][D][D] bf16 (hi, lo)
+  float* E;               // [heads*nseg, D, D]
+  float* Hc;              // [heads*nseg, D, D]
+  float* g;               // [heads*nseg]
+  float* Sst;             // [heads*nseg, D, D] span start states
+};
+
+// Scan-order helpers (host and device).
+__host__ __device__ __forceinline__ int frame_at(int j, int T, int reverse) {
+  return reverse ? T - 1 - j : j;
+}
+// Range [j0, j1) of scan positions covered by chain p.
+__host__ __device__ __forceinline__ void seg_range(const ChainArgs& a, int p, int* j0, int* j1) {
+  if (a.seg == SEG_SEQUENTIAL) {
+    *j0 = 0;
+    *j1 = a.T;
+  } else if (a.seg == SEG_CHUNKS) {
+    *j0 = p * a.L;
+    *j1 = min(*j0 + a.L, a.T);
+  } else {
+    int nb = (a.T + a.block - 1) / a.block;
+    int blk = a.reverse ? nb - 1 - p : p;
+    int t0 = blk * a.block, t1 = min(t0 + a.block, a.T);
+    if (a.reverse) {
+      *j0 = a.T - t1;
+      *j1 = a.T - t0;
+    } else {
+      *j0 = t0;
+      *j1 = t1;
+    }
+  }
+}
+
+// ---- workspace layout ---------------------------------------------------------
+struct Layout {
+  size_t A, U, Sfr, E, Hc, g, Sst, qh, kh, total;
+  int nseg_max;
+};
+
+Layout make_layout(int B, int H, int T, int S, int D, unsigned flags);
+
+// ---- launch bookkeeping --------------------------------------------------------
+void count_launch(int n = 1);
+
+// ---- SIMT (CUDA-core) kernels: any D in {16..256}, fp32 or bf16 -----------------
+cudaError_t simt_prologue(bool bf16, const void* q_raw, const void* k_raw, const float* w_q,
+                          const float* w_k, void* q_out, void* k_out, long long frames, int S,
+                          int grid_w, int D, float eps, float base, float kscale,
+                          cudaStream_t st);
+cudaError_t simt_contract(bool bf16, const void* k, const void* v, const float* beta, float* A,
+                          float* U, long long N, int S, int D, float cA, float cU,
+                          cudaStream_t st);
+cudaError_t simt_chain(const ChainArgs& a, int nchains, cudaStream_t st);
+cudaError_t simt_readout(bool bf16, const void* q, const float* Sfr, void* out, long long N,
+                         int S, int D, cudaStream_t st);
+
+// ---- tensor-core (tcgen05) kernels, bf16, sm_100a -------------------------------
+bool tc_contract_supported(int D);
+cudaError_t tc_contract(const void* k, const void* v, const float* beta, float* A, float* U,
+                        long long N, int S, int D, float cA, float cU, cudaStream_t st);
+bool tc_readout_supported(int D);
+cudaError_t tc_readout(const void* q, const void* Sfr_hilo, void* out, long long N, int S, int D,
+                       cudaStream_t st);
+bool tc_chain_supported(int D);
+cudaError_t tc_chain(const ChainArgs& a, int nchains, cudaStream_t st);
+// Reads and clears the device status word of the tensor-core kernels.
+cudaError_t tc_read_status(int* status, cudaStream_t st);
+
+}  // namespace gdn

@@ -1,0 +1,413 @@
+// CUDA-core (SIMT) kernels of the frame-wise GDN scan.
+//
+// These carry the fp32 dtype path, every head dimension D in {16, ..., 256},
+// and serve as the in-library cross-check of the tensor-core kernels. All
+// arithmetic is fp32 with fp32 accumulation.
+//
+// Recurrence (SANA-WM blog, blog.hotdry.top, section 混合线性注意力):
+//   A_t = K^^T diag(beta) K^,  U_t = V^T diag(beta) K^,  K^ = K / sqrt(D*S)
+//   S_t = gamma_t (S_{t-1} - S_{t-1} A_t) + U_t,  O_t = Q_t S_t^T.
+// Span composition (same page, Context-Parallel section): S_end = S_start C + H.
+#include "gdn_internal.cuh"
+
+namespace gdn {
+
+// ----------------------------------------------------------------------------
+// Prologue: RMSNorm -> ReLU -> key scale -> 2-D spatial RoPE, one warp per token
+// (SANA-WM blog, Context-Parallel section, the fused-op order).
+// ----------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256)
+    k_prologue(const T* __restrict__ qin, const T* __restrict__ kin, const float* __restrict__ wq,
+               const float* __restrict__ wk, T* __restrict__ qout, T* __restrict__ kout,
+               long long ntok, int S, int grid_w, int D, float eps, float base, float kscale) {
+  const long long tok = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (tok >= ntok) return;
+  const int which = blockIdx.y;  // 0: q, 1: k
+  const T* in = which ? kin : qin;
+  T* out = which ? kout : qout;
+  const float* w = which ? wk : wq;
+  const float scale = which ? kscale : 1.0f;
+  const size_t off = (size_t)tok * D;
+  const int s = (int)(tok % S);
+  const int py = s / grid_w, px = s % grid_w;
+  const int npairs = D >> 1, quarter = D >> 2, half = D >> 1;
+
+  float a[4], b[4];
+  float ss = 0.f;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int p = lane + 32 * m;
+    a[m] = b[m] = 0.f;
+    if (p < npairs) {
+      a[m] = ldf(in + off + 2 * p);
+      b[m] = ldf(in + off + 2 * p + 1);
+      ss += a[m] * a[m] + b[m] * b[m];
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = 1.0f / sqrtf(ss / (float)D + eps);
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int p = lane + 32 * m;
+    if (p < npairs) {
+      const float x0 = fmaxf(a[m] * inv * w[2 * p], 0.f) * scale;
+      const float x1 = fmaxf(b[m] * inv * w[2 * p + 1], 0.f) * scale;
+      const int hsel = p / quarter, i = p % quarter;
+      const float pos = hsel ? (float)px : (float)py;
+      const float theta = powf(base, -2.0f * (float)i / (float)half);
+      float sn, cs;
+      sincosf(pos * theta, &sn, &cs);
+      stf(out + off + 2 * p, x0 * cs - x1 * sn);
+      stf(out + off + 2 * p + 1, x0 * sn + x1 * cs);
+    }
+  }
+}
+
+cudaError_t simt_prologue(bool bf16, const void* q_raw, const void* k_raw, const float* w_q,
+                          const float* w_k, void* q_out, void* k_out, long long frames, int S,
+                          int grid_w, int D, float eps, float base, float kscale,
+                          cudaStream_t st) {
+  const long long ntok = frames * S;
+  dim3 grid((unsigned)((ntok + 7) / 8), 2);
+  if (bf16)
+    k_prologue<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        (const __nv_bfloat16*)q_raw, (const __nv_bfloat16*)k_raw, w_q, w_k,
+        (__nv_bfloat16*)q_out, (__nv_bfloat16*)k_out, ntok, S, grid_w, D, eps, base, kscale);
+  else
+    k_prologue<float><<<grid, 256, 0, st>>>((const float*)q_raw, (const float*)k_raw, w_q, w_k,
+                                            (float*)q_out, (float*)k_out, ntok, S, grid_w, D,
+                                            eps, base, kscale);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ----------------------------------------------------------------------------
+// Per-frame contraction (step a2): A = cA K^T diag(beta) K, U = cU V^T diag(beta) K.
+// One CTA per (frame, TILE x TILE output tile); tokens streamed 32 at a time.
+// ----------------------------------------------------------------------------
+template <typename T, int TILE>
+__global__ void __launch_bounds__(256)
+    k_contract_simt(const T* __restrict__ k, const T* __restrict__ v,
+                    const float* __restrict__ beta, float* __restrict__ A, float* __restrict__ U,
+                    int S, int D, float cA, float cU) {
+  constexpr int R = TILE / 16;
+  constexpr int KC = 32;
+  __shared__ float Ki[KC][TILE];
+  __shared__ float Kj[KC][TILE];  // beta * k, columns of the tile
+  __shared__ float Vi[KC][TILE];
+  const long long n = blockIdx.x;
+  const int nt = D / TILE;
+  const int ti = blockIdx.y / nt, tj = blockIdx.y % nt;
+  const T* kf = k + (size_t)n * S * D;
+  const T* vf = v + (size_t)n * S * D;
+  const float* bf = beta + (size_t)n * S;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float accA[R][R], accU[R][R];
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int j = 0; j < R; ++j) accA[i][j] = accU[i][j] = 0.f;
+
+  for (int s0 = 0; s0 < S; s0 += KC) {
+    for (int e = threadIdx.x; e < KC * TILE; e += 256) {
+      const int r = e / TILE, c = e % TILE, s = s0 + r;
+      float ki = 0.f, kj = 0.f, vi = 0.f;
+      if (s < S) {
+        ki = ldf(kf + (size_t)s * D + ti * TILE + c);
+        kj = ldf(kf + (size_t)s * D + tj * TILE + c) * bf[s];
+        vi = ldf(vf + (size_t)s * D + ti * TILE + c);
+      }
+      Ki[r][c] = ki;
+      Kj[r][c] = kj;
+      Vi[r][c] = vi;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int r = 0; r < KC; ++r) {
+      float a[R], vv[R], bb[R];
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        a[i] = Ki[r][ty * R + i];
+        vv[i] = Vi[r][ty * R + i];
+        bb[i] = Kj[r][tx * R + i];
+      }
+#pragma unroll
+      for (int i = 0; i < R; ++i)
+#pragma unroll
+        for (int j = 0; j < R; ++j) {
+          accA[i][j] = fmaf(a[i], bb[j], accA[i][j]);
+          accU[i][j] = fmaf(vv[i], bb[j], accU[i][j]);
+        }
+    }
+    __syncthreads();
+  }
+  float* An = A + (size_t)n * D * D;
+  float* Un = U + (size_t)n * D * D;
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+      const size_t idx = (size_t)(ti * TILE + ty * R + i) * D + tj * TILE + tx * R + j;
+      An[idx] = accA[i][j] * cA;
+      Un[idx] = accU[i][j] * cU;
+    }
+}
+
+template <typename T>
+static cudaError_t contract_t(const void* k, const void* v, const float* beta, float* A,
+                              float* U, long long N, int S, int D, float cA, float cU,
+                              cudaStream_t st) {
+  const int tile = D < 64 ? D : 64;
+  dim3 grid((unsigned)N, (D / tile) * (D / tile));
+  switch (tile) {
+    case 16:
+      k_contract_simt<T, 16><<<grid, 256, 0, st>>>((const T*)k, (const T*)v, beta, A, U, S, D,
+                                                   cA, cU);
+      break;
+    case 32:
+      k_contract_simt<T, 32><<<grid, 256, 0, st>>>((const T*)k, (const T*)v, beta, A, U, S, D,
+                                                   cA, cU);
+      break;
+    default:
+      k_contract_simt<T, 64><<<grid, 256, 0, st>>>((const T*)k, (const T*)v, beta, A, U, S, D,
+                                                   cA, cU);
+  }
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t simt_contract(bool bf16, const void* k, const void* v, const float* beta, float* A,
+                          float* U, long long N, int S, int D, float cA, float cU,
+                          cudaStream_t st) {
+  return bf16 ? contract_t<__nv_bfloat16>(k, v, beta, A, U, N, S, D, cA, cU, st)
+              : contract_t<float>(k, v, beta, A, U, N, S, D, cA, cU, st);
+}
+
+// ----------------------------------------------------------------------------
+// Chains of the recurrence X <- alpha (X - X Y) + Z (steps a3, a4, a5).
+// Each state row evolves on its own (row i of X Y needs only row i of X), so a
+// CTA owns 16 rows of one chain; Y is streamed through shared memory 16 rows
+// of k at a time. Thread (r, l): row r = tid / 16, columns l + 16 m.
+// ----------------------------------------------------------------------------
+constexpr int kChainRows = 16;
+
+__device__ __forceinline__ void chain_step(float* X, float* Yc, const float* __restrict__ Y,
+                                           const float* __restrict__ Z, float alpha, int D,
+                                           int row0, float* acc) {
+  const int r = threadIdx.x >> 4, l = threadIdx.x & 15;
+  const int nm = D >> 4;
+  for (int m = 0; m < nm; ++m) acc[m] = 0.f;
+  for (int k0 = 0; k0 < D; k0 += 16) {
+    for (int e = threadIdx.x; e < 16 * D; e += 256) Yc[e] = Y[(size_t)k0 * D + e];
+    __syncthreads();
+#pragma unroll 4
+    for (int kk = 0; kk < 16; ++kk) {
+      const float x = X[r * D + k0 + kk];
+      for (int m = 0; m < nm; ++m) acc[m] = fmaf(x, Yc[kk * D + l + 16 * m], acc[m]);
+    }
+    __syncthreads();
+  }
+  const int row = row0 + r;
+  if (row < D) {
+    for (int m = 0; m < nm; ++m) {
+      const int c = l + 16 * m;
+      X[r * D + c] = alpha * (X[r * D + c] - acc[m]) + Z[(size_t)row * D + c];
+    }
+  }
+  __syncthreads();
+}
+
+__device__ __forceinline__ void rows_store(const float* X, float* dst, int D, int row0) {
+  const int r = threadIdx.x >> 4, l = threadIdx.x & 15;
+  const int row = row0 + r;
+  if (row < D)
+    for (int c = l; c < D; c += 16) dst[(size_t)row * D + c] = X[r * D + c];
+}
+
+__device__ __forceinline__ void rows_store_hilo(const float* X, __nv_bfloat16* dst, int D,
+                                                int row0) {
+  const int r = threadIdx.x >> 4, l = threadIdx.x & 15;
+  const int row = row0 + r;
+  if (row < D)
+    for (int c = l; c < D; c += 16) {
+      const float x = X[r * D + c];
+      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+      dst[(size_t)row * D + c] = hi;
+      dst[(size_t)D * D + (size_t)row * D + c] = __float2bfloat16_rn(x - __bfloat162float(hi));
+    }
+}
+
+__device__ __forceinline__ void rows_load(float* X, const float* src, int D, int row0) {
+  const int r = threadIdx.x >> 4, l = threadIdx.x & 15;
+  const int row = row0 + r;
+  for (int c = l; c < D; c += 16) X[r * D + c] = (src && row < D) ? src[(size_t)row * D + c] : 0.f;
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(256) k_chain_simt(ChainArgs a) {
+  extern __shared__ float smem[];
+  const int D = a.D, T = a.T;
+  float* X = smem;                    // [16][D]
+  float* Yc = smem + kChainRows * D;  // [16][D]
+  float acc[16];
+  const int row0 = blockIdx.y * kChainRows;
+  const int c = blockIdx.x;
+
+  if (a.mode == CHAIN_SCAN) {
+    const int bh = c / a.nseg, p = c % a.nseg;
+    int j0, j1;
+    seg_range(a, p, &j0, &j1);
+    const float* init = nullptr;
+    if (p == 0) {
+      init = a.state_in ? a.state_in + (size_t)bh * D * D : nullptr;
+    } else if (a.seg == SEG_CHUNKS) {
+      init = a.Sst + ((size_t)bh * a.nseg + p) * D * D;
+    }
+    rows_load(X, init, D, row0);
+    int tprev = -1;
+    for (int j = j0; j < j1; ++j) {
+      const int t = frame_at(j, T, a.reverse);
+      if (a.seg == SEG_SEQUENTIAL && a.seq_reset && j > 0 && (t / a.block) != (tprev / a.block))
+        rows_load(X, nullptr, D, row0);
+      tprev = t;
+      const size_t fi = (size_t)bh * T + t;
+      chain_step(X, Yc, a.A + fi * D * D, a.U + fi * D * D, a.gamma[fi], D, row0, acc);
+      if (a.sfr_hilo)
+        rows_store_hilo(X, (__nv_bfloat16*)a.Sfr + fi * 2 * D * D, D, row0);
+      else
+        rows_store(X, a.Sfr + fi * D * D, D, row0);
+      if (j == T - 1 && a.state_out) rows_store(X, a.state_out + (size_t)bh * D * D, D, row0);
+    }
+  } else if (a.mode == CHAIN_COMPOSE) {
+    const int half = a.heads * a.nseg;
+    const int which = c >= half;  // 0: E, 1: H
+    const int cc = which ? c - half : c;
+    const int bh = cc / a.nseg, p = cc % a.nseg;
+    int j0, j1;
+    seg_range(a, p, &j0, &j1);
+    rows_load(X, nullptr, D, row0);
+    float gp = 1.f;
+    for (int j = j0; j < j1; ++j) {
+      const int t = frame_at(j, T, a.reverse);
+      const size_t fi = (size_t)bh * T + t;
+      const float* Af = a.A + fi * D * D;
+      if (which)
+        chain_step(X, Yc, Af, a.U + fi * D * D, a.gamma[fi], D, row0, acc);
+      else
+        chain_step(X, Yc, Af, Af, 1.0f, D, row0, acc);
+      gp *= a.gamma[fi];
+    }
+    const size_t si = (size_t)bh * a.nseg + p;
+    rows_store(X, (which ? a.Hc : a.E) + si * D * D, D, row0);
+    if (!which && blockIdx.y == 0 && threadIdx.x == 0) a.g[si] = gp;
+  } else {  // CHAIN_PREFIX
+    const int bh = c;
+    rows_load(X, a.state_in ? a.state_in + (size_t)bh * D * D : nullptr, D, row0);
+    for (int p = 0; p < a.nseg; ++p) {
+      const size_t si = (size_t)bh * a.nseg + p;
+      rows_store(X, a.Sst + si * D * D, D, row0);
+      if (p + 1 < a.nseg) chain_step(X, Yc, a.E + si * D * D, a.Hc + si * D * D, a.g[si], D, row0, acc);
+    }
+  }
+}
+
+cudaError_t simt_chain(const ChainArgs& a, int nchains, cudaStream_t st) {
+  const size_t smem = 2 * kChainRows * a.D * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k_chain_simt, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid((unsigned)nchains, (a.D + kChainRows - 1) / kChainRows);
+  k_chain_simt<<<grid, 256, smem, st>>>(a);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ----------------------------------------------------------------------------
+// Readout (step a6): O[s, i] = sum_k Q[s, k] S_t[i, k]. CTA = 64 tokens x TILE
+// output columns of one frame; each thread owns 4 tokens x (TILE/16) columns.
+// ----------------------------------------------------------------------------
+template <typename T, int TILE>
+__global__ void __launch_bounds__(256)
+    k_readout_simt(const T* __restrict__ q, const float* __restrict__ Sfr, T* __restrict__ out,
+                   int S, int D) {
+  constexpr int R = TILE / 16;
+  constexpr int TS = 64;
+  constexpr int KC = 16;
+  __shared__ float Qs[KC][TS + 1];
+  __shared__ float Ss[KC][TILE + 1];
+  const long long n = blockIdx.x;
+  const int s0 = blockIdx.y * TS;
+  const int i0 = blockIdx.z * TILE;
+  const T* qf = q + (size_t)n * S * D;
+  const float* Sn = Sfr + (size_t)n * D * D;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][R];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < R; ++b) acc[a][b] = 0.f;
+  for (int k0 = 0; k0 < D; k0 += KC) {
+    for (int e = threadIdx.x; e < KC * TS; e += 256) {
+      const int tok = e / KC, kk = e % KC, s = s0 + tok;
+      Qs[kk][tok] = s < S ? ldf(qf + (size_t)s * D + k0 + kk) : 0.f;
+    }
+    for (int e = threadIdx.x; e < KC * TILE; e += 256) {
+      const int ii = e / KC, kk = e % KC;
+      Ss[kk][ii] = Sn[(size_t)(i0 + ii) * D + k0 + kk];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < KC; ++kk) {
+      float qa[4], sb[R];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) qa[a] = Qs[kk][ty * 4 + a];
+#pragma unroll
+      for (int b = 0; b < R; ++b) sb[b] = Ss[kk][tx * R + b];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < R; ++b) acc[a][b] = fmaf(qa[a], sb[b], acc[a][b]);
+    }
+    __syncthreads();
+  }
+  T* of = out + (size_t)n * S * D;
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int s = s0 + ty * 4 + a;
+    if (s < S)
+#pragma unroll
+      for (int b = 0; b < R; ++b) stf(of + (size_t)s * D + i0 + tx * R + b, acc[a][b]);
+  }
+}
+
+template <typename T>
+static cudaError_t readout_t(const void* q, const float* Sfr, void* out, long long N, int S,
+                             int D, cudaStream_t st) {
+  const int tile = D < 64 ? D : 64;
+  dim3 grid((unsigned)N, (S + 63) / 64, D / tile);
+  switch (tile) {
+    case 16:
+      k_readout_simt<T, 16><<<grid, 256, 0, st>>>((const T*)q, Sfr, (T*)out, S, D);
+      break;
+    case 32:
+      k_readout_simt<T, 32><<<grid, 256, 0, st>>>((const T*)q, Sfr, (T*)out, S, D);
+      break;
+    default:
+      k_readout_simt<T, 64><<<grid, 256, 0, st>>>((const T*)q, Sfr, (T*)out, S, D);
+  }
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t simt_readout(bool bf16, const void* q, const float* Sfr, void* out, long long N,
+                         int S, int D, cudaStream_t st) {
+  return bf16 ? readout_t<__nv_bfloat16>(q, Sfr, out, N, S, D, st)
+              : readout_t<float>(q, Sfr, out, N, S, D, st);
+}
+
+}  // namespace gdn

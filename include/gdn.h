@@ -1,0 +1,229 @@
+/*
+ * gdn.h — C ABI of libgdnscan.so, a B200 (sm_100a) implementation of the
+ * frame-wise Gated DeltaNet (GDN) frame scan.
+ *
+ * What it computes. For every batch b, head h and latent frame t, with the S
+ * spatial tokens of the frame stored token-major (Q_t, K_t, V_t are S x D):
+ *
+ *     K^_t = K_t / sqrt(D*S)                       key scale
+ *     A_t  = K^_t^T diag(beta_t) K^_t              D x D, symmetric PSD
+ *     U_t  = V_t^T  diag(beta_t) K^_t              D x D
+ *     S_t  = gamma_t (S_{t-1} - S_{t-1} A_t) + U_t   (= S_{t-1} M_t + U_t)
+ *     O_t  = Q_t S_t^T                             token s: o_s = S_t q_s
+ *
+ * Sources (web pages on SANA-WM, cited by title and section):
+ *  - "SANA-WM：2.6B 参数分布式 Diffusion Transformer 实现消费级 GPU 分钟级 720p
+ *    视频生成" (blog.hotdry.top), section "混合线性注意力：长上下文的内存破局点":
+ *    the recurrence S_t = S_{t-1} M_t + U_t, M_t = gamma_t (I - K^ beta K^^T),
+ *    U_t = V beta K^^T, one D x D state update per frame, beta per token, and
+ *    the key scale 1/sqrt(D*S). Section "显存分片：Context-Parallel 的工程实现":
+ *    S_end = S_start C_p + H_p per span of frames (used here to run time
+ *    chunks in parallel on one GPU), and the fused prologue order RMSNorm ->
+ *    ReLU -> key scale -> RoPE -> scan.
+ *  - "Jiayun's Blog", post on SANA-WM, section 2.1: the same frame-wise form,
+ *    S = 80 x 45 = 3600 tokens per 720p latent frame.
+ *  - hyper.ai summary of the SANA-WM paper, section "方法": the chunk-causal
+ *    variant resets the reverse-time scan at chunk boundaries.
+ *  - "SANA-WM 世界模型实战指南" (trdm.cn), section 七: chunk_size: 3.
+ * The readout O_t = S_t Q_t with the post-update state is not written out on
+ * the pages; it is the plain reading, matching token-wise GDN's o_i = S_i q_i.
+ *
+ * Conventions shared by every entry point.
+ *  - Layouts: q, k, v, out are [B, H, T, S, D] contiguous (D innermost),
+ *    bf16 when GDN_BF16 is set, else fp32; beta is [B, H, T, S] fp32; gamma
+ *    is [B, H, T] fp32; states are [B, H, D, D] fp32 row-major, row = value
+ *    channel, column = key channel.
+ *  - All pointers are DEVICE pointers, owned by the caller, 16-byte aligned.
+ *    Outputs must not alias inputs.
+ *  - Shapes: D in {16, 32, 64, 128, 256}; S >= 1; T >= 1; B, H >= 1.
+ *  - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream); no entry point synchronises the host except
+ *    gdn_check_device_status.
+ *  - Errors: argument errors return GDN_ERR_INVALID / GDN_ERR_UNSUPPORTED
+ *    before anything is launched; a failed launch returns GDN_ERR_CUDA; a
+ *    device-side bounded wait that ran out is reported by
+ *    gdn_check_device_status as GDN_ERR_TIMEOUT. gdn_last_error() gives a
+ *    one-line description of the last failure on the calling host thread.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+typedef struct CUstream_st* gdn_stream_t; /* identical to cudaStream_t */
+
+enum {
+  GDN_OK = 0,
+  GDN_ERR_INVALID = -1,     /* null/misaligned pointer, bad size or flag combination */
+  GDN_ERR_UNSUPPORTED = -2, /* D outside {16,32,64,128,256}, or sizes past index limits */
+  GDN_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed */
+  GDN_ERR_TIMEOUT = -4,     /* a device-side bounded wait expired */
+  GDN_ERR_WORKSPACE = -5    /* workspace missing or smaller than gdn_workspace_bytes */
+};
+
+/* flags */
+#define GDN_BF16 0x1u           /* q/k/v/out are bf16, else fp32 */
+#define GDN_REVERSE 0x2u        /* reverse-time scan: frames T-1 .. 0 */
+#define GDN_BLOCK_RESET 0x4u    /* zero the state on entering each block (scan order) */
+#define GDN_SEQUENTIAL 0x8u     /* one chain over T, no span composition */
+#define GDN_FUSED_PROLOGUE 0x10u /* _ex only: q, k are raw; apply the prologue */
+#define GDN_KEYS_SCALED 0x20u   /* k already carries 1/sqrt(D*S): do not scale again */
+#define GDN_FORCE_SIMT 0x40u    /* use the CUDA-core kernels even where tensor-core ones exist */
+#define GDN_BIDIR 0x80u         /* _ex only: forward scan -> out, reverse scan -> out_rev */
+#define GDN_BLOCK(f) (((f) >> 8) & 0xffu)  /* reset block length; 0 means 3 */
+#define GDN_CHUNK(f) (((f) >> 16) & 0xffu) /* time-chunk length; 0 means 8 */
+#define GDN_MAKE_BLOCK(n) ((((unsigned)(n)) & 0xffu) << 8)
+#define GDN_MAKE_CHUNK(n) ((((unsigned)(n)) & 0xffu) << 16)
+
+/*
+ * gdn_frame_scan_fwd — the whole frame scan for [B, H] heads over T frames.
+ *
+ *   q, k, v     [B,H,T,S,D]  bf16 (GDN_BF16) or fp32, device
+ *   beta        [B,H,T,S]    fp32 per-token update gate
+ *   gamma       [B,H,T]      fp32 per-frame decay
+ *   state_in    [B,H,D,D]    fp32 state entering the first frame in scan
+ *                            order; NULL means zeros. With GDN_BLOCK_RESET it
+ *                            seeds only the first block in scan order.
+ *   out         [B,H,T,S,D]  same dtype as q: O_t = Q_t S_t^T
+ *   state_out   [B,H,D,D]    fp32 state after the last frame in scan order
+ *                            (frame T-1 forward, frame 0 reversed); NULL = not written
+ *   flags       GDN_BF16 | GDN_REVERSE | GDN_BLOCK_RESET | GDN_SEQUENTIAL |
+ *               GDN_KEYS_SCALED | GDN_FORCE_SIMT | GDN_MAKE_BLOCK(n) | GDN_MAKE_CHUNK(n)
+ *
+ * Blocks for GDN_BLOCK_RESET are floor(t / block) counted from t = 0 in both
+ * directions. Without GDN_SEQUENTIAL the scan runs as time chunks composed
+ * through S_end = S_start C_p + H_p (equal to the sequential scan up to
+ * rounding). Scratch comes from a stream-ordered allocation (cudaMallocAsync)
+ * made and freed inside the call; use gdn_frame_scan_fwd_ex to pass your own.
+ * Returns GDN_OK or a negative status.
+ */
+GDN_API int gdn_frame_scan_fwd(const void* q, const void* k, const void* v, const float* beta,
+                       const float* gamma, const float* state_in, void* out, float* state_out,
+                       int B, int H, int T, int S, int D, unsigned flags, gdn_stream_t stream);
+
+/*
+ * gdn_qk_prologue — the per-token prologue ahead of the scan, in the pages'
+ * order (SANA-WM blog, Context-Parallel section: RMSNorm -> ReLU -> key scale
+ * -> RoPE), on raw q and k:
+ *     x <- x / sqrt(mean_D(x^2) + eps) * w        (w_q for q, w_k for k)
+ *     x <- max(x, 0)
+ *     k <- k / sqrt(D*S)                           (keys only; S = grid_h*grid_w)
+ *     x <- RoPE2D(x): token s at (y, x) = (s / grid_w, s % grid_w); channels
+ *          [0, D/2) turn with y, [D/2, D) with x; pair (2i, 2i+1) of a half,
+ *          i < D/4, turns by pos * rope_base^(-2i/(D/2)).
+ *   q_raw, k_raw    [B,H,T,S,D] bf16 or fp32 (GDN_BF16), device
+ *   w_q, w_k        [D] fp32
+ *   q_out, k_out    [B,H,T,S,D] same dtype; k_out carries the key scale, so a
+ *                   following gdn_frame_scan_fwd takes GDN_KEYS_SCALED.
+ * Only GDN_BF16 is read from flags. Returns GDN_OK or a negative status.
+ */
+GDN_API int gdn_qk_prologue(const void* q_raw, const void* k_raw, const float* w_q, const float* w_k,
+                    void* q_out, void* k_out, int B, int H, int T, int grid_h, int grid_w, int D,
+                    float eps, float rope_base, unsigned flags, gdn_stream_t stream);
+
+/* Everything gdn_frame_scan_fwd takes, plus the prologue, the second
+ * direction and caller-owned scratch. Zero-initialise and fill. */
+typedef struct gdn_params {
+  const void* q;          /* [B,H,T,S,D]; raw when GDN_FUSED_PROLOGUE */
+  const void* k;          /* [B,H,T,S,D]; raw when GDN_FUSED_PROLOGUE */
+  const void* v;          /* [B,H,T,S,D] */
+  const float* beta;      /* [B,H,T,S] */
+  const float* gamma;     /* [B,H,T] */
+  const float* state_in;  /* [B,H,D,D] or NULL; seeds each direction's first frame */
+  void* out;              /* [B,H,T,S,D] forward (or GDN_REVERSE) output */
+  float* state_out;       /* [B,H,D,D] or NULL */
+  void* out_rev;          /* GDN_BIDIR: [B,H,T,S,D] reverse-scan output */
+  float* state_out_rev;   /* GDN_BIDIR: [B,H,D,D] or NULL */
+  const float* w_q;       /* GDN_FUSED_PROLOGUE: [D] RMSNorm weight of q */
+  const float* w_k;       /* GDN_FUSED_PROLOGUE: [D] RMSNorm weight of k */
+  int B, H, T, S, D;
+  int grid_h, grid_w;     /* GDN_FUSED_PROLOGUE: latent grid, grid_h*grid_w == S */
+  float eps;              /* RMSNorm epsilon (0 means 1e-6) */
+  float rope_base;        /* RoPE base (0 means 10000) */
+  unsigned flags;
+  void* workspace;        /* device scratch, 256-byte aligned */
+  size_t workspace_bytes; /* >= gdn_workspace_bytes(B,H,T,S,D,flags) */
+} gdn_params;
+
+/*
+ * gdn_frame_scan_fwd_ex — the scan with the options of gdn_params.
+ * With GDN_BIDIR the forward scan (never reset) writes out/state_out and the
+ * reverse-time scan writes out_rev/state_out_rev; GDN_BLOCK_RESET then applies
+ * to the reverse scan only (the chunk-causal variant of the hyper.ai summary,
+ * "方法"); A_t and U_t are computed once and shared by both directions.
+ * Returns GDN_OK or a negative status (GDN_ERR_WORKSPACE if scratch is short).
+ */
+GDN_API int gdn_frame_scan_fwd_ex(const gdn_params* p, gdn_stream_t stream);
+
+/* Bytes of scratch gdn_frame_scan_fwd_ex needs for these sizes and flags
+ * (0 on invalid sizes). */
+GDN_API size_t gdn_workspace_bytes(int B, int H, int T, int S, int D, unsigned flags);
+
+/*
+ * gdn_frame_contract — step a2 alone: for every frame-head n in [0, N),
+ *   A[n] = K^_n^T diag(beta_n) K^_n,  U[n] = V_n^T diag(beta_n) K^_n
+ * with K^ = k / sqrt(D*S) (or k as given under GDN_KEYS_SCALED).
+ *   k, v   [N,S,D] bf16/fp32;  beta [N,S] fp32;  A, U [N,D,D] fp32 row-major
+ * Honours GDN_BF16, GDN_KEYS_SCALED, GDN_FORCE_SIMT. Returns a status.
+ */
+GDN_API int gdn_frame_contract(const void* k, const void* v, const float* beta, float* A, float* U,
+                       int N, int S, int D, unsigned flags, gdn_stream_t stream);
+
+/*
+ * gdn_chunk_composites — step a3 alone: for each span n of L consecutive
+ * frames (in the order given) with inputs A, U [n*L + j] and gamma[n*L + j],
+ * j < L, the span's affine map S_start -> S_start C_n + H_n in the form
+ *   C_n = g_n (I - E_n),  g_n = prod_j gamma_j
+ * (E_n and H_n start at 0; each frame does E <- E + A - E A and
+ *  H <- gamma (H - H A) + U). Writes E [n,D,D], H [n,D,D], g [n] fp32.
+ *   A, U  [N*L,D,D] fp32;  gamma [N*L] fp32
+ * Honours GDN_FORCE_SIMT. Returns a status.
+ */
+GDN_API int gdn_chunk_composites(const float* A, const float* U, const float* gamma, float* E, float* Hc,
+                         float* g, int N, int L, int D, unsigned flags, gdn_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the library's device status
+ * word: GDN_OK, GDN_ERR_TIMEOUT if a kernel's bounded wait expired since the
+ * last check, or GDN_ERR_CUDA if the stream reports an error. */
+GDN_API int gdn_check_device_status(gdn_stream_t stream);
+
+/* Static description of a status code. */
+GDN_API const char* gdn_status_string(int status);
+
+/* One-line description of the last failure on this host thread ("" if none). */
+GDN_API const char* gdn_last_error(void);
+
+/* Kernel launches made by this host thread's gdn_* calls since the last reset;
+ * reset = 1 clears the counter after reading it. */
+GDN_API long long gdn_launch_count(int reset);
+
+/* Phase timing: while enabled, every kernel the library launches from this
+ * host thread is bracketed by two CUDA events recorded on its launch stream
+ * (instrumentation for benchmarks; no host synchronisation). enable = 1
+ * starts a fresh record, enable = 0 stops recording. Returns GDN_OK. */
+GDN_API int gdn_profile_enable(int enable);
+
+/* Sums the recorded kernel durations per phase, waiting on the events:
+ * ms[i] and counts[i] for phase i < n, with phases 0 prologue, 1 contract,
+ * 2 compose, 3 prefix, 4 scan/replay, 5 readout. Returns the number of
+ * phases written, or a negative status. */
+GDN_API int gdn_profile_read(double* ms, long long* counts, int n);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+GDN_API int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

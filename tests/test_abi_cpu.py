@@ -1,0 +1,74 @@
+"""The C-ABI library builds, loads and exports every declared entry point;
+host-side argument checks answer without a GPU (no compute is launched)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from frame_wise_gated_b200 import api, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return api.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "gdn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in api.SIGNATURES, n
+
+
+def test_version_and_status_strings(lib):
+    assert lib.gdn_version() >= 100
+    assert lib.gdn_status_string(0) == b"ok"
+    assert lib.gdn_status_string(-4) == b"device wait timed out"
+
+
+def test_workspace_bytes(lib):
+    f = api.scan_flags(bf16=True)
+    n = api.workspace_bytes(1, 16, 121, 3600, 128, f)
+    # A, U and per-frame states (3 x 64 KiB per frame-head) plus span scratch
+    assert n >= 3 * 1936 * 128 * 128 * 4
+    assert api.workspace_bytes(1, 1, 1, 1, 17, f) == 0
+    assert api.workspace_bytes(1, 16, 121, 3600, 128, f | api.FUSED_PROLOGUE) > n
+
+
+def test_argument_errors_without_gpu(lib):
+    null = None
+    rc = lib.gdn_frame_scan_fwd(null, null, null, null, null, null, null, null,
+                                1, 1, 4, 16, 17, api.BF16, null)
+    assert rc == api.GDN_ERR_UNSUPPORTED
+    rc = lib.gdn_frame_scan_fwd(null, null, null, null, null, null, null, null,
+                                1, 1, 0, 16, 16, 0, null)
+    assert rc == api.GDN_ERR_INVALID
+    p = api.GdnParams()
+    p.B, p.H, p.T, p.S, p.D = 1, 1, 2, 4, 16
+    assert lib.gdn_frame_scan_fwd_ex(ctypes.byref(p), null) == api.GDN_ERR_INVALID
+    assert b"null" in lib.gdn_last_error()
+    assert lib.gdn_frame_scan_fwd_ex(None, null) == api.GDN_ERR_INVALID
+    rc = lib.gdn_frame_scan_fwd(null, null, null, null, null, null, null, null,
+                                1, 1, 4, 16, 16, api.FUSED_PROLOGUE, null)
+    assert rc == api.GDN_ERR_INVALID
+
+
+def test_product_path_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "frame_wise_gated_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert "import oracle" not in txt and "from oracle" not in txt, f
