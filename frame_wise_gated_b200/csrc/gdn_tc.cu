@@ -1,20 +1,545 @@
-// Tensor-core (tcgen05) kernels: placeholder until the sm_100a kernels land.
+// Tensor-core (tcgen05 / TMEM / TMA) kernels of the frame-wise GDN scan, sm_100a.
+//
+// Recurrence (SANA-WM blog, blog.hotdry.top, section 混合线性注意力):
+//   A_t = K^^T diag(beta_t) K^,  U_t = V_t^T diag(beta_t) K^,  K^ = K / sqrt(D*S)
+//   S_t = gamma_t (S_{t-1} - S_{t-1} A_t) + U_t,  O_t = Q_t S_t^T.
+//
+// k_contract_tc (step a2), D = 128. One CTA per SM, persistent over
+// frame-heads. Per 64-token stage, TMA brings K and V tiles ([64 tokens][64 D]
+// boxes, 128-byte swizzle) into shared memory; four scaler warps write
+// beta * K next to them in the same layout; one thread issues, per 16 tokens,
+//   A_acc += K^T (beta K)   and   U_acc += V^T (beta K)
+// as two 128x128x16 bf16 MMAs sharing the B operand. K^T and V^T are read as
+// MN-major operands straight from the token-major tiles: no transposes. The
+// fp32 accumulators live in TMEM (2 x 256 columns, double-buffered so the
+// epilogue of one frame-head overlaps the MMAs of the next); four epilogue
+// warps scale them (1/(D S) and 1/sqrt(D S)) and store A_t, U_t in fp32.
+//
+// k_readout_tc (step a6), D = 128. Per 128-token tile of a frame-head,
+//   O_tile = Q_tile S_t^T = Q_tile S_hi^T + Q_tile S_lo^T
+// with S_t held as a bf16 (hi, lo) pair (the pair carries ~16 bits of the
+// fp32 state). Q tiles stream through a 3-stage TMA ring, the accumulator is
+// double-buffered in TMEM, and the epilogue converts to bf16 into a swizzled
+// staging tile that one thread writes back with a TMA store.
+//
+// Every wait is bounded (see sm100::mbar_wait); a wait that runs out records
+// a status the host reads with gdn_check_device_status.
+#include <cuda.h>
+
+#include <mutex>
+
 #include "gdn_internal.cuh"
+#include "gdn_sm100.cuh"
 
 namespace gdn {
 
 static __device__ int g_tc_status = 0;
 
-bool tc_contract_supported(int) { return false; }
-bool tc_readout_supported(int) { return false; }
+using namespace sm100;
+
+// ----------------------------------------------------------------------------
+// host: tensor maps through the driver entry point (no link-time libcuda)
+// ----------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor [d2][d1][d0] (d0 innermost), box {b0, b1, 1}, 128-byte swizzle.
+static cudaError_t make_map_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1,
+                                    uint64_t d2, uint32_t b0, uint32_t b1) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+static int num_sms() {
+  int dev = 0, n = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return (uint8_t*)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
+}
+
+// ============================================================================
+// Contraction (a2)
+// ============================================================================
+namespace ctr {
+constexpr int D = 128;
+constexpr int TOK = 64;                 // tokens per stage
+constexpr int NST = 4;                  // pipeline stages
+constexpr int BOX = TOK * 128;          // one [64 tokens][64 channels] bf16 box: 8 KiB
+constexpr int TILE = 2 * BOX;           // one tensor's stage tile: 16 KiB
+constexpr int OFF_K = 0;
+constexpr int OFF_V = OFF_K + NST * TILE;
+constexpr int OFF_BK = OFF_V + NST * TILE;
+constexpr int OFF_BETA = OFF_BK + NST * TILE;
+constexpr int OFF_BAR = OFF_BETA + NST * TOK * 4;
+constexpr int NBAR = 3 * NST + 5;       // full, bk_full, empty, acc_full[2], acc_empty[2], fin
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+constexpr int THREADS = 320;            // producer, MMA, 4 scaler warps, 4 epilogue warps
+constexpr uint32_t TMEM_COLS = 512;
+}  // namespace ctr
+
+__global__ void __launch_bounds__(ctr::THREADS, 1)
+    k_contract_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const float* __restrict__ beta, float* __restrict__ A, float* __restrict__ U,
+                  int N, int S, float cA, float cU) {
+  using namespace ctr;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar_full = sb + OFF_BAR;
+  const uint32_t bar_bk = bar_full + 8 * NST;
+  const uint32_t bar_empty = bar_bk + 8 * NST;
+  const uint32_t bar_accf = bar_empty + 8 * NST;
+  const uint32_t bar_acce = bar_accf + 16;
+  const uint32_t bar_fin = bar_acce + 16;
+  uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bar_full + 8 * s, 2);      // expect_tx arrival + beta arrival
+      mbar_init(bar_bk + 8 * s, 128);      // every scaler thread
+      mbar_init(bar_empty + 8 * s, 1);     // MMA commit
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_accf + 8 * b, 1);
+      mbar_init(bar_acce + 8 * b, 128);
+    }
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int nst_frame = (S + TOK - 1) / TOK;
+  const int my_count = (int)blockIdx.x < N ? (N - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+  if (warp == 0) {
+    // ---- TMA producer (lane 0 issues; the warp loads beta) ----
+    int g = 0;
+    bool ok = true;
+    for (int i = 0; i < my_count && ok; ++i) {
+      const int n = blockIdx.x + i * gridDim.x;
+      for (int st = 0; st < nst_frame; ++st, ++g) {
+        const int s = g % NST;
+        const uint32_t u = (uint32_t)(g / NST);
+        ok = mbar_wait(bar_empty + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 1);
+        if (!ok) break;
+        if (lane == 0) {
+          const uint32_t kd = sb + OFF_K + s * TILE, vd = sb + OFF_V + s * TILE;
+          mbar_arrive_expect_tx(bar_full + 8 * s, 2 * TILE);
+          tma_load_3d(kd, &tmK, bar_full + 8 * s, 0, st * TOK, n);
+          tma_load_3d(kd + BOX, &tmK, bar_full + 8 * s, 64, st * TOK, n);
+          tma_load_3d(vd, &tmV, bar_full + 8 * s, 0, st * TOK, n);
+          tma_load_3d(vd + BOX, &tmV, bar_full + 8 * s, 64, st * TOK, n);
+        }
+        float* bs = (float*)(smem + OFF_BETA) + s * TOK;
+        for (int r = lane; r < TOK; r += 32) {
+          const int tok = st * TOK + r;
+          bs[r] = tok < S ? __ldg(beta + (size_t)n * S + tok) : 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_full + 8 * s);
+      }
+    }
+    // Drain: every TMA this CTA issued has landed before teardown.
+    if (lane == 0) {
+      for (int gg = (g > NST ? g - NST : 0); gg < g; ++gg)
+        mbar_wait(bar_full + 8 * (gg % NST), (uint32_t)(gg / NST) & 1, abort_flag, &g_tc_status, 2);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---- MMA issuer ----
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, true, true);
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; i < my_count && ok; ++i) {
+        const int b = i & 1;
+        const uint32_t ub = (uint32_t)(i >> 1);
+        ok = mbar_wait(bar_acce + 8 * b, (ub & 1) ^ 1, abort_flag, &g_tc_status, 3);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t dA = tmem + b * 256, dU = dA + 128;
+        for (int st = 0; st < nst_frame; ++st, ++g) {
+          const int s = g % NST;
+          const uint32_t u = (uint32_t)(g / NST);
+          ok = mbar_wait(bar_bk + 8 * s, u & 1, abort_flag, &g_tc_status, 4);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t ka = sb + OFF_K + s * TILE, va = sb + OFF_V + s * TILE,
+                         ba = sb + OFF_BK + s * TILE;
+#pragma unroll
+          for (int kk = 0; kk < TOK / 16; ++kk) {
+            // 16 tokens = two 8-row groups of 1024 B
+            const uint64_t dk = smem_desc_sw128(ka + kk * 2048, BOX, 1024);
+            const uint64_t dv = smem_desc_sw128(va + kk * 2048, BOX, 1024);
+            const uint64_t db = smem_desc_sw128(ba + kk * 2048, BOX, 1024);
+            const uint32_t acc = (st > 0 || kk > 0) ? 1u : 0u;
+            mma_bf16(dA, dk, db, idesc, acc);
+            mma_bf16(dU, dv, db, idesc, acc);
+          }
+          mma_commit(bar_empty + 8 * s);
+        }
+        if (!ok) break;
+        mma_commit(bar_accf + 8 * b);
+      }
+      mma_commit(bar_fin);
+      mbar_wait(bar_fin, 0, abort_flag, &g_tc_status, 5);
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ---- beta * K into the B operand tile (same swizzled layout as K) ----
+    const int t = threadIdx.x - 64;
+    int g = 0;
+    bool ok = true;
+    for (int i = 0; i < my_count && ok; ++i) {
+      for (int st = 0; st < nst_frame; ++st, ++g) {
+        const int s = g % NST;
+        const uint32_t u = (uint32_t)(g / NST);
+        ok = mbar_wait(bar_full + 8 * s, u & 1, abort_flag, &g_tc_status, 6);
+        if (!ok) break;
+        const uint8_t* kt = smem + OFF_K + s * TILE;
+        uint8_t* bt = smem + OFF_BK + s * TILE;
+        const float* bs = (const float*)(smem + OFF_BETA) + s * TOK;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const int c = t + 128 * m;          // 16-byte chunk of the 16 KiB tile
+          const float bv = bs[(c >> 3) & (TOK - 1)];  // 8 chunks per 128-byte token row
+          uint4 x = *(const uint4*)(kt + c * 16);
+          uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&w[e]);
+            float2 f = __bfloat1622float2(h);
+            w[e] = pack_bf16x2(f.x * bv, f.y * bv);
+          }
+          *(uint4*)(bt + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async();
+        mbar_arrive(bar_bk + 8 * s);
+      }
+    }
+  } else {
+    // ---- epilogue: TMEM -> scale -> fp32 A_t, U_t rows ----
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    for (int i = 0; i < my_count; ++i) {
+      const int b = i & 1;
+      const uint32_t ub = (uint32_t)(i >> 1);
+      if (!mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 7)) break;
+      tc_fence_after();
+      const int n = blockIdx.x + i * gridDim.x;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float* dst = (half ? U : A) + ((size_t)n * D + row) * D;
+        const float sc = half ? cU : cA;
+#pragma unroll
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 256 + half * 128 + c0, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float4 v = make_float4(__uint_as_float(r[4 * j]) * sc, __uint_as_float(r[4 * j + 1]) * sc,
+                                   __uint_as_float(r[4 * j + 2]) * sc,
+                                   __uint_as_float(r[4 * j + 3]) * sc);
+            *(float4*)(dst + c0 + 4 * j) = v;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_acce + 8 * b);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+bool tc_contract_supported(int D) { return D == 128; }
+
+cudaError_t tc_contract(const void* k, const void* v, const float* beta, float* A, float* U,
+                        long long N, int S, int D, float cA, float cU, cudaStream_t st) {
+  if (D != 128) return cudaErrorNotSupported;
+  CUtensorMap mk, mv;
+  cudaError_t e = make_map_bf16_3d(&mk, k, D, S, N, 64, ctr::TOK);
+  if (e != cudaSuccess) return e;
+  e = make_map_bf16_3d(&mv, v, D, S, N, 64, ctr::TOK);
+  if (e != cudaSuccess) return e;
+  static bool attr = false;
+  if (!attr) {
+    e = cudaFuncSetAttribute(k_contract_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, ctr::SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int grid = (int)(N < num_sms() ? N : num_sms());
+  k_contract_tc<<<grid, ctr::THREADS, ctr::SMEM, st>>>(mk, mv, beta, A, U, (int)N, S, cA, cU);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ============================================================================
+// Readout (a6)
+// ============================================================================
+namespace rdo {
+constexpr int D = 128;
+constexpr int TOK = 128;                // tokens per tile (MMA M)
+constexpr int NQ = 3;                   // Q ring stages
+constexpr int BOX = TOK * 128;          // [128 rows][64 channels] bf16: 16 KiB
+constexpr int QT = 2 * BOX;             // one Q tile: 32 KiB
+constexpr int OFF_Q = 0;
+constexpr int OFF_S = OFF_Q + NQ * QT;  // S hi (2 boxes) then S lo (2 boxes): 64 KiB
+constexpr int OFF_O = OFF_S + 4 * BOX;  // output staging, 2 boxes: 32 KiB
+constexpr int OFF_BAR = OFF_O + 2 * BOX;
+constexpr int NBAR = 2 * NQ + 2 + 4 + 1;  // q_full, q_empty, s_full, s_empty, acc f/e x2, fin
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+constexpr int THREADS = 192;            // producer, MMA, 4 epilogue warps
+constexpr uint32_t TMEM_COLS = 256;
+}  // namespace rdo
+
+__global__ void __launch_bounds__(rdo::THREADS, 1)
+    k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
+                 const __grid_constant__ CUtensorMap tmO, int N, int S) {
+  using namespace rdo;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar_qf = sb + OFF_BAR;
+  const uint32_t bar_qe = bar_qf + 8 * NQ;
+  const uint32_t bar_sf = bar_qe + 8 * NQ;
+  const uint32_t bar_se = bar_sf + 8;
+  const uint32_t bar_accf = bar_se + 8;
+  const uint32_t bar_acce = bar_accf + 16;
+  const uint32_t bar_fin = bar_acce + 16;
+  uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NQ; ++s) {
+      mbar_init(bar_qf + 8 * s, 1);
+      mbar_init(bar_qe + 8 * s, 1);
+    }
+    mbar_init(bar_sf, 1);
+    mbar_init(bar_se, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_accf + 8 * b, 1);
+      mbar_init(bar_acce + 8 * b, 128);
+    }
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int ntile = (S + TOK - 1) / TOK;
+  const int my_count = (int)blockIdx.x < N ? (N - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; i < my_count && ok; ++i) {
+        const int n = blockIdx.x + i * gridDim.x;
+        ok = mbar_wait(bar_se, ((uint32_t)i & 1) ^ 1, abort_flag, &g_tc_status, 11);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar_sf, 4 * BOX);
+        const uint32_t sd = sb + OFF_S;
+        tma_load_3d(sd, &tmS, bar_sf, 0, 0, 2 * n);
+        tma_load_3d(sd + BOX, &tmS, bar_sf, 64, 0, 2 * n);
+        tma_load_3d(sd + 2 * BOX, &tmS, bar_sf, 0, 0, 2 * n + 1);
+        tma_load_3d(sd + 3 * BOX, &tmS, bar_sf, 64, 0, 2 * n + 1);
+        for (int tl = 0; tl < ntile; ++tl, ++g) {
+          const int s = g % NQ;
+          const uint32_t u = (uint32_t)(g / NQ);
+          ok = mbar_wait(bar_qe + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 12);
+          if (!ok) break;
+          const uint32_t qd = sb + OFF_Q + s * QT;
+          mbar_arrive_expect_tx(bar_qf + 8 * s, QT);
+          tma_load_3d(qd, &tmQ, bar_qf + 8 * s, 0, tl * TOK, n);
+          tma_load_3d(qd + BOX, &tmQ, bar_qf + 8 * s, 64, tl * TOK, n);
+        }
+      }
+      for (int gg = (g > NQ ? g - NQ : 0); gg < g; ++gg)
+        mbar_wait(bar_qf + 8 * (gg % NQ), (uint32_t)(gg / NQ) & 1, abort_flag, &g_tc_status, 13);
+      if (my_count > 0) mbar_wait(bar_sf, (uint32_t)(my_count - 1) & 1, abort_flag, &g_tc_status, 14);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; i < my_count && ok; ++i) {
+        ok = mbar_wait(bar_sf, (uint32_t)i & 1, abort_flag, &g_tc_status, 15);
+        if (!ok) break;
+        tc_fence_after();
+        for (int tl = 0; tl < ntile; ++tl, ++g) {
+          const int s = g % NQ;
+          const uint32_t u = (uint32_t)(g / NQ);
+          const int b = g & 1;
+          const uint32_t ub = (uint32_t)(g >> 1);
+          ok = mbar_wait(bar_acce + 8 * b, (ub & 1) ^ 1, abort_flag, &g_tc_status, 16);
+          if (!ok) break;
+          ok = mbar_wait(bar_qf + 8 * s, u & 1, abort_flag, &g_tc_status, 17);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t qa = sb + OFF_Q + s * QT, sh = sb + OFF_S, sl = sb + OFF_S + 2 * BOX;
+          const uint32_t d = tmem + b * 128;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            // K-major: 16 channels = 32 bytes inside a 128-byte swizzled row
+            const uint32_t off = (kk >> 2) * BOX + (kk & 3) * 32;
+            const uint64_t dq = smem_desc_sw128(qa + off, 16, 1024);
+            const uint64_t dh = smem_desc_sw128(sh + off, 16, 1024);
+            const uint64_t dl = smem_desc_sw128(sl + off, 16, 1024);
+            mma_bf16(d, dq, dh, idesc, kk > 0 ? 1u : 0u);
+            mma_bf16(d, dq, dl, idesc, 1u);
+          }
+          mma_commit(bar_qe + 8 * s);
+          mma_commit(bar_accf + 8 * b);
+        }
+        if (!ok) break;
+        mma_commit(bar_se);
+      }
+      mma_commit(bar_fin);
+      mbar_wait(bar_fin, 0, abort_flag, &g_tc_status, 18);
+    }
+    __syncwarp();
+  } else {
+    // ---- epilogue: TMEM -> bf16 -> swizzled staging -> TMA store ----
+    const int q = warp & 3;
+    const int row = q * 32 + lane;  // token within the tile
+    const int et = threadIdx.x - 64;
+    uint8_t* ost = smem + OFF_O;
+    const uint32_t ost_a = sb + OFF_O;
+    int g = 0;
+    bool ok = true;
+    for (int i = 0; i < my_count && ok; ++i) {
+      const int n = blockIdx.x + i * gridDim.x;
+      for (int tl = 0; tl < ntile; ++tl, ++g) {
+        const int b = g & 1;
+        const uint32_t ub = (uint32_t)(g >> 1);
+        ok = mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 19);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t packed[64];
+#pragma unroll
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 128 + c0, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            packed[c0 / 2 + j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+        }
+        tc_fence_before();
+        mbar_arrive(bar_acce + 8 * b);
+        // the previous tile's TMA store has finished reading the staging tile
+        if (et == 0) bulk_wait_read0();
+        named_bar_sync(1, 128);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int box = j >> 3, chunk = j & 7;
+          uint8_t* dst = ost + box * BOX + row * 128 + ((chunk ^ (row & 7)) << 4);
+          *(uint4*)dst = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
+                                    packed[4 * j + 3]);
+        }
+        fence_proxy_async();
+        named_bar_sync(1, 128);
+        if (et == 0) {
+          tma_store_3d(&tmO, ost_a, 0, tl * TOK, n);
+          tma_store_3d(&tmO, ost_a + BOX, 64, tl * TOK, n);
+          bulk_commit();
+        }
+      }
+    }
+    if (et == 0) bulk_wait0();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+bool tc_readout_supported(int D) { return D == 128; }
+
+cudaError_t tc_readout(const void* q, const void* Sfr_hilo, void* out, long long N, int S, int D,
+                       cudaStream_t st) {
+  if (D != 128) return cudaErrorNotSupported;
+  CUtensorMap mq, ms, mo;
+  cudaError_t e = make_map_bf16_3d(&mq, q, D, S, N, 64, rdo::TOK);
+  if (e != cudaSuccess) return e;
+  e = make_map_bf16_3d(&ms, Sfr_hilo, D, D, 2 * N, 64, 128);
+  if (e != cudaSuccess) return e;
+  e = make_map_bf16_3d(&mo, out, D, S, N, 64, rdo::TOK);
+  if (e != cudaSuccess) return e;
+  static bool attr = false;
+  if (!attr) {
+    e = cudaFuncSetAttribute(k_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, rdo::SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int grid = (int)(N < num_sms() ? N : num_sms());
+  k_readout_tc<<<grid, rdo::THREADS, rdo::SMEM, st>>>(mq, ms, mo, (int)N, S);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ============================================================================
+// Chain kernels on tensor cores: not yet; the CUDA-core chains carry the scan.
+// ============================================================================
 bool tc_chain_supported(int) { return false; }
-cudaError_t tc_contract(const void*, const void*, const float*, float*, float*, long long, int,
-                        int, float, float, cudaStream_t) {
-  return cudaErrorNotSupported;
-}
-cudaError_t tc_readout(const void*, const void*, void*, long long, int, int, cudaStream_t) {
-  return cudaErrorNotSupported;
-}
 cudaError_t tc_chain(const ChainArgs&, int, cudaStream_t) { return cudaErrorNotSupported; }
 
 cudaError_t tc_read_status(int* status, cudaStream_t st) {
