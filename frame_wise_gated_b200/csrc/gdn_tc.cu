@@ -158,7 +158,8 @@ __global__ void __launch_bounds__(ctr::THREADS, 1)
       for (int st = 0; st < nst_frame; ++st, ++g) {
         const int s = g % NST;
         const uint32_t u = (uint32_t)(g / NST);
-        ok = mbar_wait(bar_empty + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 1);
+        if (lane == 0) ok = mbar_wait(bar_empty + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 1);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         if (lane == 0) {
           const uint32_t kd = sb + OFF_K + s * TILE, vd = sb + OFF_V + s * TILE;
@@ -467,8 +468,7 @@ __global__ void __launch_bounds__(rdo::THREADS, 1)
       for (int tl = 0; tl < ntile; ++tl, ++g) {
         const int b = g & 1;
         const uint32_t ub = (uint32_t)(g >> 1);
-        ok = mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 19);
-        if (!ok) break;
+        mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 19);
         tc_fence_after();
         uint32_t packed[64];
 #pragma unroll
@@ -485,6 +485,10 @@ __global__ void __launch_bounds__(rdo::THREADS, 1)
         // the previous tile's TMA store has finished reading the staging tile
         if (et == 0) bulk_wait_read0();
         named_bar_sync(1, 128);
+        if (*abort_flag) {  // uniform across the four epilogue warps
+          ok = false;
+          break;
+        }
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int box = j >> 3, chunk = j & 7;
@@ -537,10 +541,324 @@ cudaError_t tc_readout(const void* q, const void* Sfr_hilo, void* out, long long
 }
 
 // ============================================================================
-// Chain kernels on tensor cores: not yet; the CUDA-core chains carry the scan.
+// Chains of the recurrence on tensor cores (steps a3, a4, a5), D = 128.
+//
+// One CTA runs one chain X <- alpha (X - X Y) + Z (the state update; the span
+// composites E <- E + A - E A and H <- gamma (H - H A) + U; the prefix over
+// spans S <- g (S - S E) + H). The 128 x 128 fp32 X lives in registers: warp
+// w holds rows 32 (w % 4) .. +31 (its TMEM lane quadrant), columns
+// 64 (w / 4) .. +63. Each step writes X as a bf16 (hi, lo) pair into a K-major
+// operand tile and one thread issues
+//     P = X_hi Y_hi + X_lo Y_hi + X_hi Y_lo      (fp32 in TMEM)
+// which carries ~16 mantissa bits of both factors. Y (fp32 in global memory)
+// is split into bf16 (hi, lo) MN-major tiles for the next step while the
+// current step's MMAs run (two Y buffers).
 // ============================================================================
-bool tc_chain_supported(int) { return false; }
-cudaError_t tc_chain(const ChainArgs&, int, cudaStream_t) { return cudaErrorNotSupported; }
+namespace chn {
+constexpr int D = 128;
+constexpr int HALF = 64 * 128 * 2 * 2;  // one bf16 128x128 operand tile: 32 KiB
+constexpr int ATOM = 128 * 128;         // 16 KiB: 128 rows x 128 bytes
+constexpr int OFF_XH = 0;
+constexpr int OFF_XL = OFF_XH + HALF;
+constexpr int OFF_Y = OFF_XL + HALF;     // Y[b] hi at OFF_Y + b*2*HALF, lo at + HALF
+constexpr int OFF_BAR = OFF_Y + 4 * HALF;
+constexpr int OFF_MISC = OFF_BAR + 16;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+constexpr int THREADS = 256;
+constexpr uint32_t TMEM_COLS = 128;
+}  // namespace chn
+
+struct ChainStep {
+  const float* Y;
+  const float* Z;
+  float alpha;
+  int reset;  // zero X before this step
+  int t;      // frame (scan/compose) or span (prefix)
+};
+
+// Program of chain c: number of steps and, for step s, its operands.
+struct ChainProg {
+  int mode, which, bh, p, j0, n;
+  const float* init;
+};
+
+__device__ __forceinline__ ChainProg chain_prog(const ChainArgs& a, int c) {
+  ChainProg g;
+  g.mode = a.mode;
+  g.which = 0;
+  g.init = nullptr;
+  if (a.mode == CHAIN_SCAN) {
+    g.bh = c / a.nseg;
+    g.p = c % a.nseg;
+    int j0, j1;
+    seg_range(a, g.p, &j0, &j1);
+    g.j0 = j0;
+    g.n = j1 - j0;
+    if (g.p == 0)
+      g.init = a.state_in ? a.state_in + (size_t)g.bh * a.D * a.D : nullptr;
+    else if (a.seg == SEG_CHUNKS)
+      g.init = a.Sst + ((size_t)g.bh * a.nseg + g.p) * a.D * a.D;
+  } else if (a.mode == CHAIN_COMPOSE) {
+    const int half = a.heads * a.nseg;
+    g.which = c >= half;
+    const int cc = g.which ? c - half : c;
+    g.bh = cc / a.nseg;
+    g.p = cc % a.nseg;
+    int j0, j1;
+    seg_range(a, g.p, &j0, &j1);
+    g.j0 = j0;
+    g.n = j1 - j0;
+  } else {
+    g.bh = c;
+    g.p = 0;
+    g.j0 = 0;
+    g.n = a.nseg - 1;
+    g.init = a.state_in ? a.state_in + (size_t)g.bh * a.D * a.D : nullptr;
+  }
+  return g;
+}
+
+__device__ __forceinline__ ChainStep chain_step_at(const ChainArgs& a, const ChainProg& g, int s) {
+  ChainStep st;
+  const size_t DD = (size_t)a.D * a.D;
+  if (g.mode == CHAIN_PREFIX) {
+    const size_t si = (size_t)g.bh * a.nseg + s;
+    st.Y = a.E + si * DD;
+    st.Z = a.Hc + si * DD;
+    st.alpha = a.g[si];
+    st.reset = 0;
+    st.t = s;
+    return st;
+  }
+  const int j = g.j0 + s;
+  const int t = frame_at(j, a.T, a.reverse);
+  const size_t fi = (size_t)g.bh * a.T + t;
+  st.t = t;
+  st.Y = a.A + fi * DD;
+  st.reset = 0;
+  if (g.mode == CHAIN_SCAN) {
+    st.Z = a.U + fi * DD;
+    st.alpha = a.gamma[fi];
+    if (a.seg == SEG_SEQUENTIAL && a.seq_reset && j > 0) {
+      const int tp = frame_at(j - 1, a.T, a.reverse);
+      st.reset = (t / a.block) != (tp / a.block);
+    }
+  } else {
+    st.Z = g.which ? a.U + fi * DD : st.Y;
+    st.alpha = g.which ? a.gamma[fi] : 1.0f;
+  }
+  return st;
+}
+
+// Y (fp32 row-major [k][n]) -> bf16 hi/lo MN-major swizzled tiles.
+__device__ __forceinline__ void chain_load_y(const float* __restrict__ Y, uint8_t* yh, uint8_t* yl) {
+  using namespace chn;
+#pragma unroll 2
+  for (int m = 0; m < 8; ++m) {
+    const int cid = threadIdx.x + THREADS * m;  // 2048 chunks of 8 values
+    const int k = cid >> 4, nc = cid & 15;
+    const float4 f0 = __ldg((const float4*)(Y + k * D + nc * 8));
+    const float4 f1 = __ldg((const float4*)(Y + k * D + nc * 8 + 4));
+    const float v[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * e]), h1 = __float2bfloat16_rn(v[2 * e + 1]);
+      hw[e] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
+      lw[e] = pack_bf16x2(v[2 * e] - __bfloat162float(h0), v[2 * e + 1] - __bfloat162float(h1));
+    }
+    const int off = (nc >> 3) * ATOM + k * 128 + (((nc & 7) ^ (k & 7)) << 4);
+    *(uint4*)(yh + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *(uint4*)(yl + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
+}
+
+// X row slice (64 values of row `row`, columns 64h..) -> K-major hi/lo tiles.
+__device__ __forceinline__ void chain_store_x(const float* x, uint8_t* xh, uint8_t* xl, int row,
+                                              int h) {
+  using namespace chn;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float a0 = x[8 * c + 2 * e], a1 = x[8 * c + 2 * e + 1];
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(a0), h1 = __float2bfloat16_rn(a1);
+      hw[e] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
+      lw[e] = pack_bf16x2(a0 - __bfloat162float(h0), a1 - __bfloat162float(h1));
+    }
+    const int off = h * ATOM + row * 128 + ((c ^ (row & 7)) << 4);
+    *(uint4*)(xh + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *(uint4*)(xl + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
+}
+
+__device__ __forceinline__ void store_row_f32(float* dst, const float* x) {
+#pragma unroll
+  for (int c = 0; c < 64; c += 4) *(float4*)(dst + c) = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
+}
+
+__device__ __forceinline__ void store_row_hilo(__nv_bfloat16* hi, __nv_bfloat16* lo, const float* x) {
+#pragma unroll
+  for (int c = 0; c < 64; c += 8) {
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float a0 = x[c + 2 * e], a1 = x[c + 2 * e + 1];
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(a0), h1 = __float2bfloat16_rn(a1);
+      hw[e] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
+      lw[e] = pack_bf16x2(a0 - __bfloat162float(h0), a1 - __bfloat162float(h1));
+    }
+    *(uint4*)(hi + c) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *(uint4*)(lo + c) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
+}
+
+__global__ void __launch_bounds__(chn::THREADS, 1) k_chain_tc(ChainArgs a) {
+  using namespace chn;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q = warp & 3, h = warp >> 2;
+  const int row = q * 32 + lane;
+  const uint32_t bar_mma = sb + OFF_BAR;
+  uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
+  const size_t DD = (size_t)D * D;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_mma, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  const ChainProg g = chain_prog(a, blockIdx.x);
+  float x[64];
+  if (g.init) {
+    const float* src = g.init + (size_t)row * D + h * 64;
+#pragma unroll
+    for (int c = 0; c < 64; c += 4) {
+      const float4 f = __ldg((const float4*)(src + c));
+      x[c] = f.x; x[c + 1] = f.y; x[c + 2] = f.z; x[c + 3] = f.w;
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 64; ++c) x[c] = 0.f;
+  }
+  float gprod = 1.f;
+  if (g.n > 0) chain_load_y(chain_step_at(a, g, 0).Y, smem + OFF_Y, smem + OFF_Y + HALF);
+
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, true);
+  for (int s = 0; s < g.n; ++s) {
+    const ChainStep st = chain_step_at(a, g, s);
+    if (g.mode == CHAIN_PREFIX) store_row_f32(a.Sst + ((size_t)g.bh * a.nseg + s) * DD + (size_t)row * D + h * 64, x);
+    if (st.reset) {
+#pragma unroll
+      for (int c = 0; c < 64; ++c) x[c] = 0.f;
+    }
+    chain_store_x(x, smem + OFF_XH, smem + OFF_XL, row, h);
+    fence_proxy_async();
+    __syncthreads();
+    if (*abort_flag) break;  // uniform: read after the barrier
+    const int yb = s & 1;
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      const uint32_t yh = sb + OFF_Y + yb * 2 * HALF, yl = yh + HALF;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t xo = (kk >> 2) * ATOM + (kk & 3) * 32;
+        const uint64_t dxh = smem_desc_sw128(sb + OFF_XH + xo, 16, 1024);
+        const uint64_t dxl = smem_desc_sw128(sb + OFF_XL + xo, 16, 1024);
+        const uint64_t dyh = smem_desc_sw128(yh + kk * 2048, ATOM, 1024);
+        const uint64_t dyl = smem_desc_sw128(yl + kk * 2048, ATOM, 1024);
+        mma_bf16(tmem, dxh, dyh, idesc, kk > 0 ? 1u : 0u);
+        mma_bf16(tmem, dxl, dyh, idesc, 1u);
+        mma_bf16(tmem, dxh, dyl, idesc, 1u);
+      }
+      mma_commit(bar_mma);
+    }
+    if (s + 1 < g.n) {
+      uint8_t* yn = smem + OFF_Y + (yb ^ 1) * 2 * HALF;
+      chain_load_y(chain_step_at(a, g, s + 1).Y, yn, yn + HALF);
+    }
+    float z[64];
+    {
+      const float* zr = st.Z + (size_t)row * D + h * 64;
+#pragma unroll
+      for (int c = 0; c < 64; c += 4) {
+        const float4 f = __ldg((const float4*)(zr + c));
+        z[c] = f.x; z[c + 1] = f.y; z[c + 2] = f.z; z[c + 3] = f.w;
+      }
+    }
+    // On a timeout the flag is set; the step finishes on stale values and
+    // every thread leaves at the next barrier.
+    mbar_wait(bar_mma, (uint32_t)s & 1, abort_flag, &g_tc_status, 21);
+    tc_fence_after();
+#pragma unroll
+    for (int c0 = 0; c0 < 64; c0 += 32) {
+      uint32_t r[32];
+      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + h * 64 + c0, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        x[c0 + c] = st.alpha * (x[c0 + c] - __uint_as_float(r[c])) + z[c0 + c];
+    }
+    tc_fence_before();
+    if (g.mode == CHAIN_COMPOSE) gprod *= a.gamma[(size_t)g.bh * a.T + st.t];
+    if (g.mode == CHAIN_SCAN) {
+      const size_t fi = (size_t)g.bh * a.T + st.t;
+      if (a.sfr_hilo) {
+        __nv_bfloat16* base = (__nv_bfloat16*)a.Sfr + fi * 2 * DD + (size_t)row * D + h * 64;
+        store_row_hilo(base, base + DD, x);
+      } else {
+        store_row_f32(a.Sfr + fi * DD + (size_t)row * D + h * 64, x);
+      }
+      if (g.j0 + s == a.T - 1 && a.state_out)
+        store_row_f32(a.state_out + (size_t)g.bh * DD + (size_t)row * D + h * 64, x);
+    }
+  }
+  __syncthreads();
+  if (!*abort_flag) {
+    if (g.mode == CHAIN_COMPOSE) {
+      const size_t si = (size_t)g.bh * a.nseg + g.p;
+      store_row_f32((g.which ? a.Hc : a.E) + si * DD + (size_t)row * D + h * 64, x);
+      if (!g.which && threadIdx.x == 0) a.g[si] = gprod;
+    } else if (g.mode == CHAIN_PREFIX) {
+      store_row_f32(a.Sst + ((size_t)g.bh * a.nseg + g.n) * DD + (size_t)row * D + h * 64, x);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+bool tc_chain_supported(int D) { return D == 128; }
+
+cudaError_t tc_chain(const ChainArgs& a, int nchains, cudaStream_t st) {
+  if (a.D != 128) return cudaErrorNotSupported;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e =
+        cudaFuncSetAttribute(k_chain_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, chn::SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  k_chain_tc<<<nchains, chn::THREADS, chn::SMEM, st>>>(a);
+  count_launch();
+  return cudaGetLastError();
+}
 
 cudaError_t tc_read_status(int* status, cudaStream_t st) {
   int zero = 0;
