@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(ctr::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
-      mbar_init(bar_full + 8 * s, 2);      // expect_tx arrival + beta arrival
+      mbar_init(bar_full + 8 * s, 33);     // expect_tx arrival + 32 lanes' beta copies
       mbar_init(bar_bk + 8 * s, 128);      // every scaler thread
       mbar_init(bar_empty + 8 * s, 1);     // MMA commit
     }
@@ -169,13 +169,16 @@ __global__ void __launch_bounds__(ctr::THREADS, 1)
           tma_load_3d(vd, &tmV, bar_full + 8 * s, 0, st * TOK, n);
           tma_load_3d(vd + BOX, &tmV, bar_full + 8 * s, 64, st * TOK, n);
         }
-        float* bs = (float*)(smem + OFF_BETA) + s * TOK;
+        // beta of the stage's tokens: asynchronous 4-byte copies (zeros past S)
+        // that arrive on the same barrier, so the loop never waits on them.
+        const uint32_t bsa = sb + OFF_BETA + s * TOK * 4;
+#pragma unroll
         for (int r = lane; r < TOK; r += 32) {
           const int tok = st * TOK + r;
-          bs[r] = tok < S ? __ldg(beta + (size_t)n * S + tok) : 0.f;
+          const bool in = tok < S;
+          cp_async_4(bsa + r * 4, beta + (size_t)n * S + (in ? tok : 0), in ? 4u : 0u);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_full + 8 * s);
+        cp_async_arrive_noinc(bar_full + 8 * s);
       }
     }
     // Drain: every TMA this CTA issued has landed before teardown.
