@@ -181,6 +181,8 @@ static int run_direction(const gdn_params& p, const Layout& L, char* ws, bool re
   a.Hc = (float*)(ws + L.Hc);
   a.g = (float*)(ws + L.g);
   a.Sst = (float*)(ws + L.Sst);
+  a.y_image = use_tc_chain ? 1 : 0;  // the tensor-core chains read A and E as operand images
+  a.e_image = a.y_image;
 
   auto chain = [&](const ChainArgs& c, int n) -> cudaError_t {
     PhaseScope ps(c.mode == CHAIN_COMPOSE ? PH_COMPOSE : c.mode == CHAIN_PREFIX ? PH_PREFIX : PH_SCAN,
@@ -286,7 +288,8 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
   {
     PhaseScope ps(PH_CONTRACT, st);
     if (tc_contract_ok)
-      e = tc_contract(k, p.v, p.beta, A, U, frames, p.S, p.D, (float)(c * c), (float)c, st);
+      e = tc_contract(k, p.v, p.beta, A, U, frames, p.S, p.D, (float)(c * c), (float)c,
+                      tc_chain_ok ? 1 : 0, st);
     else
       e = simt_contract(bf16, k, p.v, p.beta, A, U, frames, p.S, p.D, (float)(c * c), (float)c,
                         st);
@@ -411,7 +414,7 @@ int gdn_frame_contract(const void* k, const void* v, const float* beta, float* A
   const bool tc = bf16 && !(flags & GDN_FORCE_SIMT) && device_cc_major() == 10 &&
                   tc_contract_supported(D);
   cudaStream_t st = (cudaStream_t)stream;
-  cudaError_t e = tc ? tc_contract(k, v, beta, A, U, N, S, D, (float)(c * c), (float)c, st)
+  cudaError_t e = tc ? tc_contract(k, v, beta, A, U, N, S, D, (float)(c * c), (float)c, 0, st)
                      : simt_contract(bf16, k, v, beta, A, U, N, S, D, (float)(c * c),
                                      (float)c, st);
   if (e != cudaSuccess) return cuda_fail(e, "contract");
@@ -442,7 +445,24 @@ int gdn_chunk_composites(const float* A, const float* U, const float* gamma, flo
   a.g = g;
   const bool tc = !(flags & GDN_FORCE_SIMT) && device_cc_major() == 10 && tc_chain_supported(D);
   cudaStream_t st = (cudaStream_t)stream;
-  cudaError_t e = tc ? tc_chain(a, 2 * N, st) : simt_chain(a, 2 * N, st);
+  cudaError_t e;
+  if (tc) {
+    // The tensor-core chains read A as operand images: convert into scratch.
+    void* img = nullptr;
+    e = cudaMallocAsync(&img, (size_t)N * L * kImageBytes, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(images)");
+    e = tc_to_image(A, img, (long long)N * L, st);
+    if (e == cudaSuccess) {
+      a.A = (const float*)img;
+      a.y_image = 1;
+      a.e_image = 0;
+      e = tc_chain(a, 2 * N, st);
+    }
+    cudaError_t e2 = cudaFreeAsync(img, st);
+    if (e == cudaSuccess) e = e2;
+  } else {
+    e = simt_chain(a, 2 * N, st);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "compose");
   return GDN_OK;
 }

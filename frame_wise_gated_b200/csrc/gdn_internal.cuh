@@ -64,7 +64,18 @@ struct ChainArgs {
   float* Hc;              // [heads*nseg, D, D]
   float* g;               // [heads*nseg]
   float* Sst;             // [heads*nseg, D, D] span start states
+  int y_image;            // A (and E for the prefix) are stored as bf16 operand images
+  int e_image;            // the compose chain writes E as an operand image
 };
+
+// An "operand image" of a D x D fp32 matrix M (D = 128) is the exact
+// shared-memory tile the tensor-core chain kernel uses as its B operand
+// B[k][n] = M[k][n]: a bf16 (hi, lo) pair, hi = bf16(M), lo = bf16(M - hi),
+// each as two 64-column blocks of 128 rows x 128 bytes in the 128-byte
+// swizzled MN-major layout (hi: bytes [0, 32K), lo: [32K, 64K)). It occupies
+// the same 64 KiB as the fp32 matrix and is copied into shared memory with a
+// single bulk copy.
+constexpr int kImageBytes = 128 * 128 * 4;
 
 // Scan-order helpers (host and device).
 __host__ __device__ __forceinline__ int frame_at(int j, int T, int reverse) {
@@ -118,7 +129,10 @@ cudaError_t simt_readout(bool bf16, const void* q, const float* Sfr, void* out, 
 // ---- tensor-core (tcgen05) kernels, bf16, sm_100a -------------------------------
 bool tc_contract_supported(int D);
 cudaError_t tc_contract(const void* k, const void* v, const float* beta, float* A, float* U,
-                        long long N, int S, int D, float cA, float cU, cudaStream_t st);
+                        long long N, int S, int D, float cA, float cU, int a_image,
+                        cudaStream_t st);
+// fp32 D x D matrices -> operand images (D = 128).
+cudaError_t tc_to_image(const float* src, void* dst, long long n, cudaStream_t st);
 bool tc_readout_supported(int D);
 cudaError_t tc_readout(const void* q, const void* Sfr_hilo, void* out, long long N, int S, int D,
                        cudaStream_t st);

@@ -109,7 +109,7 @@ constexpr uint32_t TMEM_COLS = 512;
 __global__ void __launch_bounds__(ctr::THREADS, 1)
     k_contract_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const float* __restrict__ beta, float* __restrict__ A, float* __restrict__ U,
-                  int N, int S, float cA, float cU) {
+                  int N, int S, float cA, float cU, int a_image) {
   using namespace ctr;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -272,18 +272,39 @@ __global__ void __launch_bounds__(ctr::THREADS, 1)
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         float* dst = (half ? U : A) + ((size_t)n * D + row) * D;
+        uint8_t* img = (uint8_t*)A + (size_t)n * kImageBytes;
         const float sc = half ? cU : cA;
 #pragma unroll
         for (int c0 = 0; c0 < 128; c0 += 32) {
           uint32_t r[32];
           tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 256 + half * 128 + c0, r);
           tmem_wait_ld();
+          if (half == 0 && a_image) {
+            // A_t row `row` as the B-operand image (row k = row, columns c0..c0+31)
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            float4 v = make_float4(__uint_as_float(r[4 * j]) * sc, __uint_as_float(r[4 * j + 1]) * sc,
-                                   __uint_as_float(r[4 * j + 2]) * sc,
-                                   __uint_as_float(r[4 * j + 3]) * sc);
-            *(float4*)(dst + c0 + 4 * j) = v;
+            for (int j = 0; j < 4; ++j) {
+              const int col = c0 + 8 * j;
+              uint32_t hw[4], lw[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float a0 = __uint_as_float(r[8 * j + 2 * e]) * sc;
+                const float a1 = __uint_as_float(r[8 * j + 2 * e + 1]) * sc;
+                const __nv_bfloat16 h0 = __float2bfloat16_rn(a0), h1 = __float2bfloat16_rn(a1);
+                hw[e] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
+                lw[e] = pack_bf16x2(a0 - __bfloat162float(h0), a1 - __bfloat162float(h1));
+              }
+              const int off = (col >> 6) * (128 * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4);
+              *(uint4*)(img + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+              *(uint4*)(img + 32768 + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              float4 v = make_float4(__uint_as_float(r[4 * j]) * sc, __uint_as_float(r[4 * j + 1]) * sc,
+                                     __uint_as_float(r[4 * j + 2]) * sc,
+                                     __uint_as_float(r[4 * j + 3]) * sc);
+              *(float4*)(dst + c0 + 4 * j) = v;
+            }
           }
         }
       }
@@ -303,7 +324,8 @@ __global__ void __launch_bounds__(ctr::THREADS, 1)
 bool tc_contract_supported(int D) { return D == 128; }
 
 cudaError_t tc_contract(const void* k, const void* v, const float* beta, float* A, float* U,
-                        long long N, int S, int D, float cA, float cU, cudaStream_t st) {
+                        long long N, int S, int D, float cA, float cU, int a_image,
+                        cudaStream_t st) {
   if (D != 128) return cudaErrorNotSupported;
   CUtensorMap mk, mv;
   cudaError_t e = make_map_bf16_3d(&mk, k, D, S, N, 64, ctr::TOK);
@@ -317,7 +339,8 @@ cudaError_t tc_contract(const void* k, const void* v, const float* beta, float* 
     attr = true;
   }
   const int grid = (int)(N < num_sms() ? N : num_sms());
-  k_contract_tc<<<grid, ctr::THREADS, ctr::SMEM, st>>>(mk, mv, beta, A, U, (int)N, S, cA, cU);
+  k_contract_tc<<<grid, ctr::THREADS, ctr::SMEM, st>>>(mk, mv, beta, A, U, (int)N, S, cA, cU,
+                                                        a_image);
   count_launch();
   return cudaGetLastError();
 }
@@ -563,20 +586,20 @@ constexpr int HALF = 64 * 128 * 2 * 2;  // one bf16 128x128 operand tile: 32 KiB
 constexpr int ATOM = 128 * 128;         // 16 KiB: 128 rows x 128 bytes
 constexpr int OFF_XH = 0;
 constexpr int OFF_XL = OFF_XH + HALF;
-constexpr int OFF_Y = OFF_XL + HALF;     // Y[b] hi at OFF_Y + b*2*HALF, lo at + HALF
-constexpr int OFF_BAR = OFF_Y + 4 * HALF;
-constexpr int OFF_MISC = OFF_BAR + 16;
+constexpr int OFF_Y = OFF_XL + HALF;     // Y image b at OFF_Y + b * kImageBytes (hi, then lo)
+constexpr int OFF_BAR = OFF_Y + 2 * kImageBytes;  // bar_mma, bar_y[2]
+constexpr int OFF_MISC = OFF_BAR + 32;
 constexpr int SMEM = OFF_MISC + 16 + 1024;
 constexpr int THREADS = 256;
 constexpr uint32_t TMEM_COLS = 128;
 }  // namespace chn
 
 struct ChainStep {
-  const float* Y;
-  const float* Z;
+  const void* Y;    // operand image of Y
+  const float* Z;   // fp32 Z, or null: Z = Y (span composite E)
   float alpha;
-  int reset;  // zero X before this step
-  int t;      // frame (scan/compose) or span (prefix)
+  int reset;        // zero X before this step
+  int t;            // frame (scan/compose) or span (prefix)
 };
 
 // Program of chain c: number of steps and, for step s, its operands.
@@ -647,52 +670,52 @@ __device__ __forceinline__ ChainStep chain_step_at(const ChainArgs& a, const Cha
       st.reset = (t / a.block) != (tp / a.block);
     }
   } else {
-    st.Z = g.which ? a.U + fi * DD : st.Y;
+    st.Z = g.which ? a.U + fi * DD : nullptr;
     st.alpha = g.which ? a.gamma[fi] : 1.0f;
   }
   return st;
 }
 
-// Y (fp32 row-major [k][n]) -> bf16 hi/lo MN-major swizzled tiles.
-__device__ __forceinline__ void chain_load_y(const float* __restrict__ Y, uint8_t* yh, uint8_t* yl) {
-  using namespace chn;
-#pragma unroll 2
-  for (int m = 0; m < 8; ++m) {
-    const int cid = threadIdx.x + THREADS * m;  // 2048 chunks of 8 values
-    const int k = cid >> 4, nc = cid & 15;
-    const float4 f0 = __ldg((const float4*)(Y + k * D + nc * 8));
-    const float4 f1 = __ldg((const float4*)(Y + k * D + nc * 8 + 4));
-    const float v[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-    uint32_t hw[4], lw[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * e]), h1 = __float2bfloat16_rn(v[2 * e + 1]);
-      hw[e] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
-      lw[e] = pack_bf16x2(v[2 * e] - __bfloat162float(h0), v[2 * e + 1] - __bfloat162float(h1));
-    }
-    const int off = (nc >> 3) * ATOM + k * 128 + (((nc & 7) ^ (k & 7)) << 4);
-    *(uint4*)(yh + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-    *(uint4*)(yl + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-  }
+// Bulk copy of one operand image (64 KiB) into shared memory; one thread.
+__device__ __forceinline__ void chain_fetch_y(uint32_t dst, const void* src, uint32_t bar) {
+  mbar_arrive_expect_tx(bar, kImageBytes);
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"((uint32_t)kImageBytes), "r"(bar)
+      : "memory");
 }
 
-// X row slice (64 values of row `row`, columns 64h..) -> K-major hi/lo tiles.
+// X row slice (64 values of row `row`, columns 64h..) -> hi/lo 16-byte chunks
+// at `off(c)` of tiles xh / xl (c = chunk 0..7 of the slice).
+__device__ __forceinline__ void split_chunk(const float* v, uint4* hi, uint4* lo) {
+  uint32_t hw[4], lw[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float a0 = v[2 * e], a1 = v[2 * e + 1];
+    const __nv_bfloat16 h0 = __float2bfloat16_rn(a0), h1 = __float2bfloat16_rn(a1);
+    hw[e] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
+    lw[e] = pack_bf16x2(a0 - __bfloat162float(h0), a1 - __bfloat162float(h1));
+  }
+  *hi = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  *lo = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+}
+
+// Same swizzled position for K-major X tiles (rows = state rows, 64 columns per
+// 128-byte row of atom h) and for MN-major operand images (rows = k, 64
+// columns n per 128-byte row of block h).
+__device__ __forceinline__ int tile_off(int row, int h, int c) {
+  return h * chn::ATOM + row * 128 + ((c ^ (row & 7)) << 4);
+}
+
 __device__ __forceinline__ void chain_store_x(const float* x, uint8_t* xh, uint8_t* xl, int row,
                                               int h) {
-  using namespace chn;
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
-    uint32_t hw[4], lw[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float a0 = x[8 * c + 2 * e], a1 = x[8 * c + 2 * e + 1];
-      const __nv_bfloat16 h0 = __float2bfloat16_rn(a0), h1 = __float2bfloat16_rn(a1);
-      hw[e] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
-      lw[e] = pack_bf16x2(a0 - __bfloat162float(h0), a1 - __bfloat162float(h1));
-    }
-    const int off = h * ATOM + row * 128 + ((c ^ (row & 7)) << 4);
-    *(uint4*)(xh + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-    *(uint4*)(xl + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    uint4 hi, lo;
+    split_chunk(x + 8 * c, &hi, &lo);
+    *(uint4*)(xh + tile_off(row, h, c)) = hi;
+    *(uint4*)(xl + tile_off(row, h, c)) = lo;
   }
 }
 
@@ -703,18 +726,14 @@ __device__ __forceinline__ void store_row_f32(float* dst, const float* x) {
 
 __device__ __forceinline__ void store_row_hilo(__nv_bfloat16* hi, __nv_bfloat16* lo, const float* x) {
 #pragma unroll
-  for (int c = 0; c < 64; c += 8) {
-    uint32_t hw[4], lw[4];
+  for (int c = 0; c < 64; c += 8) split_chunk(x + c, (uint4*)(hi + c), (uint4*)(lo + c));
+}
+
+__device__ __forceinline__ void store_row_image(uint8_t* img, const float* x, int row, int h) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float a0 = x[c + 2 * e], a1 = x[c + 2 * e + 1];
-      const __nv_bfloat16 h0 = __float2bfloat16_rn(a0), h1 = __float2bfloat16_rn(a1);
-      hw[e] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
-      lw[e] = pack_bf16x2(a0 - __bfloat162float(h0), a1 - __bfloat162float(h1));
-    }
-    *(uint4*)(hi + c) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-    *(uint4*)(lo + c) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-  }
+  for (int c = 0; c < 8; ++c)
+    split_chunk(x + 8 * c, (uint4*)(img + tile_off(row, h, c)),
+                (uint4*)(img + 2 * chn::ATOM + tile_off(row, h, c)));
 }
 
 __global__ void __launch_bounds__(chn::THREADS, 1) k_chain_tc(ChainArgs a) {
@@ -726,12 +745,16 @@ __global__ void __launch_bounds__(chn::THREADS, 1) k_chain_tc(ChainArgs a) {
   const int q = warp & 3, h = warp >> 2;
   const int row = q * 32 + lane;
   const uint32_t bar_mma = sb + OFF_BAR;
+  const uint32_t bar_y = bar_mma + 8;  // two, one per Y buffer
   uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
   volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
   const size_t DD = (size_t)D * D;
+  const ChainProg g = chain_prog(a, blockIdx.x);
 
   if (threadIdx.x == 0) {
     mbar_init(bar_mma, 1);
+    mbar_init(bar_y, 1);
+    mbar_init(bar_y + 8, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -743,8 +766,13 @@ __global__ void __launch_bounds__(chn::THREADS, 1) k_chain_tc(ChainArgs a) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  int fetched = 0;  // Y images requested so far (thread 0)
+  if (threadIdx.x == 0) {
+    for (; fetched < 2 && fetched < g.n; ++fetched)
+      chain_fetch_y(sb + OFF_Y + fetched * kImageBytes, chain_step_at(a, g, fetched).Y,
+                    bar_y + 8 * fetched);
+  }
 
-  const ChainProg g = chain_prog(a, blockIdx.x);
   float x[64];
   if (g.init) {
     const float* src = g.init + (size_t)row * D + h * 64;
@@ -758,24 +786,26 @@ __global__ void __launch_bounds__(chn::THREADS, 1) k_chain_tc(ChainArgs a) {
     for (int c = 0; c < 64; ++c) x[c] = 0.f;
   }
   float gprod = 1.f;
-  if (g.n > 0) chain_load_y(chain_step_at(a, g, 0).Y, smem + OFF_Y, smem + OFF_Y + HALF);
 
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, true);
   for (int s = 0; s < g.n; ++s) {
     const ChainStep st = chain_step_at(a, g, s);
-    if (g.mode == CHAIN_PREFIX) store_row_f32(a.Sst + ((size_t)g.bh * a.nseg + s) * DD + (size_t)row * D + h * 64, x);
+    const int yb = s & 1;
+    if (g.mode == CHAIN_PREFIX)
+      store_row_f32(a.Sst + ((size_t)g.bh * a.nseg + s) * DD + (size_t)row * D + h * 64, x);
     if (st.reset) {
 #pragma unroll
       for (int c = 0; c < 64; ++c) x[c] = 0.f;
     }
     chain_store_x(x, smem + OFF_XH, smem + OFF_XL, row, h);
     fence_proxy_async();
+    // Y_s has landed (every thread observes the copy's completion)
+    mbar_wait(bar_y + 8 * yb, (uint32_t)(s >> 1) & 1, abort_flag, &g_tc_status, 22);
     __syncthreads();
     if (*abort_flag) break;  // uniform: read after the barrier
-    const int yb = s & 1;
     if (threadIdx.x == 0) {
       tc_fence_after();
-      const uint32_t yh = sb + OFF_Y + yb * 2 * HALF, yl = yh + HALF;
+      const uint32_t yh = sb + OFF_Y + yb * kImageBytes, yl = yh + 2 * ATOM;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t xo = (kk >> 2) * ATOM + (kk & 3) * 32;
@@ -789,17 +819,29 @@ __global__ void __launch_bounds__(chn::THREADS, 1) k_chain_tc(ChainArgs a) {
       }
       mma_commit(bar_mma);
     }
-    if (s + 1 < g.n) {
-      uint8_t* yn = smem + OFF_Y + (yb ^ 1) * 2 * HALF;
-      chain_load_y(chain_step_at(a, g, s + 1).Y, yn, yn + HALF);
-    }
     float z[64];
-    {
+    if (st.Z) {
       const float* zr = st.Z + (size_t)row * D + h * 64;
 #pragma unroll
       for (int c = 0; c < 64; c += 4) {
         const float4 f = __ldg((const float4*)(zr + c));
         z[c] = f.x; z[c + 1] = f.y; z[c + 2] = f.z; z[c + 3] = f.w;
+      }
+    } else {
+      // Z = Y: read this row's slice back from the image (hi + lo)
+      const uint8_t* yi = smem + OFF_Y + yb * kImageBytes;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 hi = *(const uint4*)(yi + tile_off(row, h, c));
+        const uint4 lo = *(const uint4*)(yi + 2 * ATOM + tile_off(row, h, c));
+        const uint32_t hw[4] = {hi.x, hi.y, hi.z, hi.w}, lw[4] = {lo.x, lo.y, lo.z, lo.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 fh = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hw[e]));
+          const float2 fl = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lw[e]));
+          z[8 * c + 2 * e] = fh.x + fl.x;
+          z[8 * c + 2 * e + 1] = fh.y + fl.y;
+        }
       }
     }
     // On a timeout the flag is set; the step finishes on stale values and
@@ -816,6 +858,13 @@ __global__ void __launch_bounds__(chn::THREADS, 1) k_chain_tc(ChainArgs a) {
         x[c0 + c] = st.alpha * (x[c0 + c] - __uint_as_float(r[c])) + z[c0 + c];
     }
     tc_fence_before();
+    // Every thread is past its reads of Y buffer yb (the Z = Y read) and the
+    // MMA reading it has completed: refill it with Y_{s+2}.
+    __syncthreads();
+    if (threadIdx.x == 0 && s + 2 < g.n) {
+      chain_fetch_y(sb + OFF_Y + yb * kImageBytes, chain_step_at(a, g, s + 2).Y, bar_y + 8 * yb);
+      ++fetched;
+    }
     if (g.mode == CHAIN_COMPOSE) gprod *= a.gamma[(size_t)g.bh * a.T + st.t];
     if (g.mode == CHAIN_SCAN) {
       const size_t fi = (size_t)g.bh * a.T + st.t;
@@ -831,13 +880,23 @@ __global__ void __launch_bounds__(chn::THREADS, 1) k_chain_tc(ChainArgs a) {
   }
   __syncthreads();
   if (!*abort_flag) {
+    const size_t si = (size_t)g.bh * a.nseg + g.p;
     if (g.mode == CHAIN_COMPOSE) {
-      const size_t si = (size_t)g.bh * a.nseg + g.p;
-      store_row_f32((g.which ? a.Hc : a.E) + si * DD + (size_t)row * D + h * 64, x);
+      if (g.which)
+        store_row_f32(a.Hc + si * DD + (size_t)row * D + h * 64, x);
+      else if (a.e_image)
+        store_row_image((uint8_t*)a.E + si * kImageBytes, x, row, h);
+      else
+        store_row_f32(a.E + si * DD + (size_t)row * D + h * 64, x);
       if (!g.which && threadIdx.x == 0) a.g[si] = gprod;
     } else if (g.mode == CHAIN_PREFIX) {
       store_row_f32(a.Sst + ((size_t)g.bh * a.nseg + g.n) * DD + (size_t)row * D + h * 64, x);
     }
+  }
+  // Drain: wait (bounded) for any Y copy still in flight before teardown.
+  if (threadIdx.x == 0) {
+    for (int s = (fetched > 2 ? fetched - 2 : 0); s < fetched; ++s)
+      mbar_wait(bar_y + 8 * (s & 1), (uint32_t)(s >> 1) & 1, abort_flag, &g_tc_status, 23);
   }
   tc_fence_before();
   __syncthreads();
@@ -847,10 +906,30 @@ __global__ void __launch_bounds__(chn::THREADS, 1) k_chain_tc(ChainArgs a) {
   }
 }
 
+// fp32 matrix -> operand image; one CTA of 256 threads per matrix.
+__global__ void __launch_bounds__(256) k_to_image(const float* __restrict__ src, uint8_t* __restrict__ dst) {
+  const float* m = src + (size_t)blockIdx.x * 128 * 128;
+  uint8_t* img = dst + (size_t)blockIdx.x * kImageBytes;
+  for (int cid = threadIdx.x; cid < 128 * 16; cid += 256) {
+    const int k = cid >> 4, nc = cid & 15;
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = m[k * 128 + nc * 8 + e];
+    split_chunk(v, (uint4*)(img + tile_off(k, nc >> 3, nc & 7)),
+                (uint4*)(img + 2 * chn::ATOM + tile_off(k, nc >> 3, nc & 7)));
+  }
+}
+
+cudaError_t tc_to_image(const float* src, void* dst, long long n, cudaStream_t st) {
+  k_to_image<<<(unsigned)n, 256, 0, st>>>(src, (uint8_t*)dst);
+  count_launch();
+  return cudaGetLastError();
+}
+
 bool tc_chain_supported(int D) { return D == 128; }
 
 cudaError_t tc_chain(const ChainArgs& a, int nchains, cudaStream_t st) {
-  if (a.D != 128) return cudaErrorNotSupported;
+  if (a.D != 128 || !a.y_image) return cudaErrorNotSupported;
   static bool attr = false;
   if (!attr) {
     cudaError_t e =
