@@ -72,6 +72,7 @@ SIGNATURES = {
     "gdn_frame_scan_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _U, _P]),
     "gdn_qk_prologue": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _F, _U, _P]),
     "gdn_frame_scan_fwd_ex": (_I, [ctypes.POINTER(GdnParams), _P]),
+    "gdn_frame_scan_fwd_static": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _U, _P]),
     "gdn_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _U]),
     "gdn_frame_contract": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _U, _P]),
     "gdn_chunk_composites": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _U, _P]),
@@ -224,6 +225,36 @@ def frame_scan_fwd(q, k, v, beta, gamma, state_in=None, *, reverse=False, block_
     _check(lib().gdn_frame_scan_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(gamma),
                                     _ptr(state_in), _ptr(out), _ptr(state_out),
                                     B, H, T, S, D, flags, _stream(stream)), "gdn_frame_scan_fwd")
+    return out, state_out
+
+
+STATIC_SCRATCH_BYTES = 32 << 20
+
+
+def frame_scan_fwd_static(q, k, v, beta, gamma, state_in=None, *, reverse=False,
+                          block_reset=False, block=3, chunk=8, sequential=False,
+                          keys_scaled=False, force_simt=False, out=None, state_out=None,
+                          stream=None):
+    """The frame scan through gdn_frame_scan_fwd_static: for callers that must
+    not allocate device memory per call (e.g. a streaming loop running one
+    short block of frames at a time). Scratch is the library's fixed 32 MiB
+    device array; outputs are allocated here only when not passed in.
+    Returns (out, state_out)."""
+    B, H, T, S, D = q.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _want(t, n, q.dtype, (B, H, T, S, D))
+    _want(beta, "beta", torch.float32, (B, H, T, S))
+    _want(gamma, "gamma", torch.float32, (B, H, T))
+    flags = scan_flags(bf16=q.dtype == torch.bfloat16, reverse=reverse, block_reset=block_reset,
+                       block=block, chunk=chunk, sequential=sequential,
+                       keys_scaled=keys_scaled, force_simt=force_simt)
+    out = torch.empty_like(q) if out is None else out
+    state_out = torch.empty((B, H, D, D), device=q.device, dtype=torch.float32) \
+        if state_out is None else state_out
+    _check(lib().gdn_frame_scan_fwd_static(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(gamma),
+                                           _ptr(state_in), _ptr(out), _ptr(state_out),
+                                           B, H, T, S, D, flags, _stream(stream)),
+           "gdn_frame_scan_fwd_static")
     return out, state_out
 
 

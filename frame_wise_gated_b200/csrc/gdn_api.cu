@@ -308,6 +308,16 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
                        tc_chain_ok, tc_readout_ok, st);
 }
 
+int scan_ex_entry(const gdn_params& p, cudaStream_t st) {
+  t_last_error.clear();
+  return scan_ex(p, st);
+}
+
+int set_last_error(int status, const char* msg) {
+  t_last_error = msg;
+  return status;
+}
+
 }  // namespace gdn
 
 using namespace gdn;

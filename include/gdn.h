@@ -165,6 +165,33 @@ typedef struct gdn_params {
  */
 GDN_API int gdn_frame_scan_fwd_ex(const gdn_params* p, gdn_stream_t stream);
 
+/*
+ * gdn_frame_scan_fwd_static — gdn_frame_scan_fwd for callers that cannot
+ * allocate device memory at call time. (The pages have no counterpart: this
+ * is a deployment entry point.) Streaming loops that run one short block of
+ * frames per call, hosts whose device memory is all held by their own pooling
+ * allocator, and plugin contexts that get no workspace pointer all fall in
+ * this group: cudaMalloc / cudaFree can synchronise the device, can fail
+ * while a pool owns the memory, or may be forbidden outright.
+ *
+ * Same arguments, results and flags as gdn_frame_scan_fwd (GDN_FUSED_PROLOGUE
+ * and GDN_BIDIR are rejected). Scratch is a fixed 32 MiB array in device
+ * memory inside the library, held on every GPU that loads it until the process
+ * exits; nothing is allocated or freed. Sizes whose gdn_workspace_bytes exceeds
+ * 32 MiB (e.g. one 3-frame block of 16 heads at 720p needs about 13 MB; a full
+ * 121-frame rollout does not fit) return GDN_ERR_WORKSPACE before any launch.
+ * The first call on each device looks up the array's device address (a
+ * one-time runtime query); make that first call before any stream capture.
+ * All calls share the array: calls ordered on one stream are safe, calls that
+ * overlap on the GPU (other streams, unordered host threads) race. No part of
+ * the scratch has to start at zero: a call writes every byte it reads.
+ */
+GDN_API int gdn_frame_scan_fwd_static(const void* q, const void* k, const void* v,
+                                      const float* beta, const float* gamma,
+                                      const float* state_in, void* out, float* state_out, int B,
+                                      int H, int T, int S, int D, unsigned flags,
+                                      gdn_stream_t stream);
+
 /* Bytes of scratch gdn_frame_scan_fwd_ex needs for these sizes and flags
  * (0 on invalid sizes). */
 GDN_API size_t gdn_workspace_bytes(int B, int H, int T, int S, int D, unsigned flags);
