@@ -123,8 +123,10 @@ Layout make_layout(int B, int H, int T, int S, int D, unsigned flags) {
   off = align256(off + heads * L.nseg_max * mat);
   L.g = off;
   off = align256(off + heads * L.nseg_max * sizeof(float));
-  L.qh = L.kh = off;
+  L.qh = L.kh = L.rope = off;
   if (flags & GDN_FUSED_PROLOGUE) {
+    L.rope = off;  // (cos, sin) table: positions [0, S) x pairs [0, D/4)
+    off = align256(off + (size_t)S * (D / 4) * 8);
     const size_t elt = (flags & GDN_BF16) ? 2 : 4;
     const size_t tens = frames * (size_t)S * D * elt;
     L.qh = off;
@@ -159,7 +161,8 @@ static int check_sizes(int B, int H, int T, int S, int D) {
 // Runs one direction of the scan from A, U already in the workspace.
 static int run_direction(const gdn_params& p, const Layout& L, char* ws, bool reverse,
                          bool block_reset, const void* q, void* out, float* state_out,
-                         bool use_tc_chain, bool use_tc_readout, cudaStream_t st) {
+                         bool use_tc_chain, bool use_tc_readout, const ProArgs* pro_q,
+                         cudaStream_t st) {
   const bool bf16 = (p.flags & GDN_BF16) != 0;
   const long long frames = (long long)p.B * p.H * p.T;
   ChainArgs a;
@@ -219,7 +222,7 @@ static int run_direction(const gdn_params& p, const Layout& L, char* ws, bool re
   {
     PhaseScope ps(PH_READOUT, st);
     if (use_tc_readout)
-      e = tc_readout(q, ws + L.Sfr, out, frames, p.S, p.D, st);
+      e = tc_readout(q, ws + L.Sfr, out, frames, p.S, p.D, pro_q, st);
     else
       e = simt_readout(bf16, q, (const float*)(ws + L.Sfr), out, frames, p.S, p.D, st);
   }
@@ -268,19 +271,40 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
   const void* q = p.q;
   const void* k = p.k;
   bool keys_scaled = (f & GDN_KEYS_SCALED) != 0;
+  ProArgs pro_k = {}, pro_q = {};
+  const ProArgs* ppk = nullptr;
+  const ProArgs* ppq = nullptr;
   if (f & GDN_FUSED_PROLOGUE) {
     const float eps = p.eps > 0.f ? p.eps : 1e-6f;
     const float base = p.rope_base > 0.f ? p.rope_base : 10000.f;
-    const float ks = (float)(1.0 / std::sqrt((double)p.D * (double)p.S));
-    {
-      PhaseScope ps(PH_PROLOGUE, st);
-      e = simt_prologue(bf16, p.q, p.k, p.w_q, p.w_k, ws + L.qh, ws + L.kh, frames, p.S,
-                        p.grid_w, p.D, eps, base, ks, st);
+    const int npos_max = p.grid_h > p.grid_w ? p.grid_h : p.grid_w;
+    if (tc_contract_ok && tc_readout_ok && npos_max <= tc_prologue_max_positions()) {
+      // Fused: the tensor-core loaders apply RMSNorm, ReLU and RoPE to the raw
+      // tiles in shared memory; the key scale goes into the contraction's
+      // epilogue constants (RoPE is linear, so the order does not matter).
+      const int npos = p.grid_h > p.grid_w ? p.grid_h : p.grid_w;
+      float2* cs = (float2*)(ws + L.rope);
+      {
+        PhaseScope ps(PH_PROLOGUE, st);
+        e = rope_table(cs, npos, p.D, base, st);
+      }
+      if (e != cudaSuccess) return cuda_fail(e, "rope table");
+      pro_k = ProArgs{p.w_k, cs, p.grid_w, eps, npos};
+      pro_q = ProArgs{p.w_q, cs, p.grid_w, eps, npos};
+      ppk = &pro_k;
+      ppq = &pro_q;
+    } else {
+      const float ks = (float)(1.0 / std::sqrt((double)p.D * (double)p.S));
+      {
+        PhaseScope ps(PH_PROLOGUE, st);
+        e = simt_prologue(bf16, p.q, p.k, p.w_q, p.w_k, ws + L.qh, ws + L.kh, frames, p.S,
+                          p.grid_w, p.D, eps, base, ks, st);
+      }
+      if (e != cudaSuccess) return cuda_fail(e, "prologue");
+      q = ws + L.qh;
+      k = ws + L.kh;
+      keys_scaled = true;
     }
-    if (e != cudaSuccess) return cuda_fail(e, "prologue");
-    q = ws + L.qh;
-    k = ws + L.kh;
-    keys_scaled = true;
   }
   const double c = keys_scaled ? 1.0 : 1.0 / std::sqrt((double)p.D * (double)p.S);
   float* A = (float*)(ws + L.A);
@@ -289,7 +313,7 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
     PhaseScope ps(PH_CONTRACT, st);
     if (tc_contract_ok)
       e = tc_contract(k, p.v, p.beta, A, U, frames, p.S, p.D, (float)(c * c), (float)c,
-                      tc_chain_ok ? 1 : 0, st);
+                      tc_chain_ok ? 1 : 0, ppk, st);
     else
       e = simt_contract(bf16, k, p.v, p.beta, A, U, frames, p.S, p.D, (float)(c * c), (float)c,
                         st);
@@ -299,13 +323,13 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
   const bool block_reset = (f & GDN_BLOCK_RESET) != 0;
   if (f & GDN_BIDIR) {
     rc = run_direction(p, L, ws, false, false, q, p.out, p.state_out, tc_chain_ok,
-                       tc_readout_ok, st);
+                       tc_readout_ok, ppq, st);
     if (rc) return rc;
     return run_direction(p, L, ws, true, block_reset, q, p.out_rev, p.state_out_rev,
-                         tc_chain_ok, tc_readout_ok, st);
+                         tc_chain_ok, tc_readout_ok, ppq, st);
   }
   return run_direction(p, L, ws, (f & GDN_REVERSE) != 0, block_reset, q, p.out, p.state_out,
-                       tc_chain_ok, tc_readout_ok, st);
+                       tc_chain_ok, tc_readout_ok, ppq, st);
 }
 
 int scan_ex_entry(const gdn_params& p, cudaStream_t st) {
@@ -424,7 +448,8 @@ int gdn_frame_contract(const void* k, const void* v, const float* beta, float* A
   const bool tc = bf16 && !(flags & GDN_FORCE_SIMT) && device_cc_major() == 10 &&
                   tc_contract_supported(D);
   cudaStream_t st = (cudaStream_t)stream;
-  cudaError_t e = tc ? tc_contract(k, v, beta, A, U, N, S, D, (float)(c * c), (float)c, 0, st)
+  cudaError_t e = tc ? tc_contract(k, v, beta, A, U, N, S, D, (float)(c * c), (float)c, 0,
+                                   nullptr, st)
                      : simt_contract(bf16, k, v, beta, A, U, N, S, D, (float)(c * c),
                                      (float)c, st);
   if (e != cudaSuccess) return cuda_fail(e, "contract");

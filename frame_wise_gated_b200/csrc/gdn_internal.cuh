@@ -105,7 +105,7 @@ __host__ __device__ __forceinline__ void seg_range(const ChainArgs& a, int p, in
 
 // ---- workspace layout ---------------------------------------------------------
 struct Layout {
-  size_t A, U, Sfr, E, Hc, g, Sst, qh, kh, total;
+  size_t A, U, Sfr, E, Hc, g, Sst, qh, kh, rope, total;
   int nseg_max;
 };
 
@@ -127,15 +127,30 @@ cudaError_t simt_readout(bool bf16, const void* q, const float* Sfr, void* out, 
                          int S, int D, cudaStream_t st);
 
 // ---- tensor-core (tcgen05) kernels, bf16, sm_100a -------------------------------
+// Prologue applied inside the tensor-core loaders (RMSNorm -> ReLU -> 2-D RoPE;
+// the key scale is folded into the contraction's epilogue constants).
+struct ProArgs {
+  const float* w;    // [D] RMSNorm weight
+  const float2* cs;  // [D/4][npos] (cos, sin) of pos * base^(-2i/(D/2)), pair-major
+  int grid_w;
+  float eps;
+  int npos;
+};
+// (cos, sin) table, pair-major: cs[i * npos + pos], pos < npos, i < D/4
+// (consecutive tokens of a row read consecutive entries).
+cudaError_t rope_table(float2* cs, int npos, int D, float base, cudaStream_t st);
+
+// Largest max(grid_h, grid_w) the fused prologue's shared-memory table holds (D = 128).
+int tc_prologue_max_positions();
 bool tc_contract_supported(int D);
 cudaError_t tc_contract(const void* k, const void* v, const float* beta, float* A, float* U,
                         long long N, int S, int D, float cA, float cU, int a_image,
-                        cudaStream_t st);
+                        const ProArgs* pro, cudaStream_t st);
 // fp32 D x D matrices -> operand images (D = 128).
 cudaError_t tc_to_image(const float* src, void* dst, long long n, cudaStream_t st);
 bool tc_readout_supported(int D);
 cudaError_t tc_readout(const void* q, const void* Sfr_hilo, void* out, long long N, int S, int D,
-                       cudaStream_t st);
+                       const ProArgs* pro, cudaStream_t st);
 bool tc_chain_supported(int D);
 cudaError_t tc_chain(const ChainArgs& a, int nchains, cudaStream_t st);
 // Reads and clears the device status word of the tensor-core kernels.

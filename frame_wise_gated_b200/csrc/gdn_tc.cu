@@ -85,6 +85,79 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return (uint8_t*)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
 }
 
+// ----------------------------------------------------------------------------
+// Prologue inside the loaders (SANA-WM blog, Context-Parallel section: the
+// fused op runs RMSNorm -> ReLU -> key scale -> RoPE ahead of the scan). A
+// group of 16 / NCH threads (consecutive lanes) handles one token row of a
+// tile made of two [rows][64] bf16 boxes with the 128-byte swizzle; each
+// thread owns NCH 16-byte chunks (8 * NCH channels starting at channel c0) and
+// the group combines its sums of squares. Since the RMSNorm factor
+// inv = 1/sqrt(mean(x^2) + eps) is positive and RoPE is linear,
+//     RoPE(max(x * inv * w, 0)) = inv * RoPE(max(x * w, 0)),
+// which saves a multiply per element. The row is written back in place and
+// returned in f (fp32). Pair p of the thread is channel pair c0/2 + p of the
+// token; inside its half (y for channels < 64, x above) that is pair index
+// (c0 % 64)/2 + p of the (cos, sin) table row of the token's position.
+// ----------------------------------------------------------------------------
+template <int NCH>
+__device__ __forceinline__ void pro_row_part(uint8_t* tile, int box_bytes, int r, int c0, int D,
+                                             int tok, bool valid, const ProArgs& pro,
+                                             const float* w, const float2* tab, float* f) {
+  const int box = c0 >> 6, ch0 = (c0 & 63) >> 3;
+  uint8_t* rowp = tile + box * box_bytes + r * 128;
+  float ssp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    const uint4 v = *(const uint4*)(rowp + (((ch0 + c) ^ (r & 7)) << 4));
+    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wd[e]));
+      f[8 * c + 2 * e] = x.x;
+      f[8 * c + 2 * e + 1] = x.y;
+      ssp[e] = fmaf(x.x, x.x, fmaf(x.y, x.y, ssp[e]));
+    }
+  }
+  float ss = (ssp[0] + ssp[1]) + (ssp[2] + ssp[3]);
+#pragma unroll
+  for (int o = 1; o < 16 / NCH; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = 1.0f / sqrtf(ss / (float)D + pro.eps);
+  const int pos = valid ? (box ? tok % pro.grid_w : tok / pro.grid_w) : 0;
+  const float2* cs = tab + ((c0 & 63) >> 1) * pro.npos + pos;
+#pragma unroll
+  for (int j = 0; j < 4 * NCH; ++j) {
+    const float a = fmaxf(f[2 * j] * w[2 * j], 0.f);
+    const float b = fmaxf(f[2 * j + 1] * w[2 * j + 1], 0.f);
+    const float2 t = cs[j * pro.npos];
+    f[2 * j] = inv * (a * t.x - b * t.y);
+    f[2 * j + 1] = inv * (a * t.y + b * t.x);
+  }
+#pragma unroll
+  for (int c = 0; c < NCH; ++c)
+    *(uint4*)(rowp + (((ch0 + c) ^ (r & 7)) << 4)) =
+        make_uint4(pack_bf16x2(f[8 * c], f[8 * c + 1]), pack_bf16x2(f[8 * c + 2], f[8 * c + 3]),
+                   pack_bf16x2(f[8 * c + 4], f[8 * c + 5]), pack_bf16x2(f[8 * c + 6], f[8 * c + 7]));
+}
+
+// (cos, sin) of pos * base^(-2i/(D/2)) for pos < npos, i < D/4, at cs[i * npos + pos].
+__global__ void k_rope_table(float2* cs, int npos, int D, float base) {
+  const int n = npos * (D / 4);
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += gridDim.x * blockDim.x) {
+    const int i = e / npos, pos = e % npos;
+    const float theta = powf(base, -2.0f * (float)i / (float)(D / 2));
+    float sn, c;
+    sincosf((float)pos * theta, &sn, &c);
+    cs[e] = make_float2(c, sn);
+  }
+}
+
+cudaError_t rope_table(float2* cs, int npos, int D, float base, cudaStream_t st) {
+  const int n = npos * (D / 4);
+  k_rope_table<<<(n + 255) / 256, 256, 0, st>>>(cs, npos, D, base);
+  count_launch();
+  return cudaGetLastError();
+}
+
 // ============================================================================
 // Contraction (a2)
 // ============================================================================
@@ -101,15 +174,18 @@ constexpr int OFF_BETA = OFF_BK + NST * TILE;
 constexpr int OFF_BAR = OFF_BETA + NST * TOK * 4;
 constexpr int NBAR = 3 * NST + 5;       // full, bk_full, empty, acc_full[2], acc_empty[2], fin
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr int SMEM = OFF_MISC + 16 + 1024;
-constexpr int THREADS = 320;            // producer, MMA, 4 scaler warps, 4 epilogue warps
+constexpr int OFF_TAB = OFF_MISC + 16;  // prologue (cos, sin) table copy
+constexpr int TAB_MAX = 80 * 32;        // entries: positions x pairs (D/4 = 32)
+constexpr int SMEM = OFF_TAB + TAB_MAX * 8 + 1024;
+constexpr int NSC = 256;                // scaler threads (8 warps)
+constexpr int THREADS = 64 + NSC + 128;  // producer, MMA, 8 scaler warps, 4 epilogue warps
 constexpr uint32_t TMEM_COLS = 512;
 }  // namespace ctr
 
 __global__ void __launch_bounds__(ctr::THREADS, 1)
     k_contract_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const float* __restrict__ beta, float* __restrict__ A, float* __restrict__ U,
-                  int N, int S, float cA, float cU, int a_image) {
+                  int N, int S, float cA, float cU, int a_image, ProArgs pro) {
   using namespace ctr;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -127,7 +203,7 @@ __global__ void __launch_bounds__(ctr::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(bar_full + 8 * s, 33);     // expect_tx arrival + 32 lanes' beta copies
-      mbar_init(bar_bk + 8 * s, 128);      // every scaler thread
+      mbar_init(bar_bk + 8 * s, NSC);      // every scaler thread
       mbar_init(bar_empty + 8 * s, 1);     // MMA commit
     }
     for (int b = 0; b < 2; ++b) {
@@ -138,6 +214,9 @@ __global__ void __launch_bounds__(ctr::THREADS, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  float2* tab = (float2*)(smem + OFF_TAB);
+  if (pro.w)
+    for (int e = threadIdx.x; e < pro.npos * (D / 4); e += THREADS) tab[e] = pro.cs[e];
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
     tmem_relinquish();
@@ -227,9 +306,16 @@ __global__ void __launch_bounds__(ctr::THREADS, 1)
       mbar_wait(bar_fin, 0, abort_flag, &g_tc_status, 5);
     }
     __syncwarp();
-  } else if (warp < 6) {
+  } else if (warp < 2 + NSC / 32) {
     // ---- beta * K into the B operand tile (same swizzled layout as K) ----
     const int t = threadIdx.x - 64;
+    // prologue: four threads per token (r = t / 4), 32 channels each
+    const int pr = t >> 2, pc0 = (t & 3) * 32;
+    float wreg[32];
+    if (pro.w) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) wreg[j] = __ldg(pro.w + pc0 + j);
+    }
     int g = 0;
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
@@ -238,12 +324,29 @@ __global__ void __launch_bounds__(ctr::THREADS, 1)
         const uint32_t u = (uint32_t)(g / NST);
         ok = mbar_wait(bar_full + 8 * s, u & 1, abort_flag, &g_tc_status, 6);
         if (!ok) break;
-        const uint8_t* kt = smem + OFF_K + s * TILE;
+        uint8_t* kt = smem + OFF_K + s * TILE;
         uint8_t* bt = smem + OFF_BK + s * TILE;
         const float* bs = (const float*)(smem + OFF_BETA) + s * TOK;
+        if (pro.w) {
+          // raw k -> K^ in place (RMSNorm, ReLU, RoPE), then beta * K^
+          const int tok = st * TOK + pr;
+          float f[32];
+          pro_row_part<4>(kt, BOX, pr, pc0, D, tok, tok < S, pro, wreg, tab, f);
+          const float bv = bs[pr];
+          uint8_t* rowp = bt + (pc0 >> 6) * BOX + pr * 128;
+          const int ch0 = (pc0 & 63) >> 3;
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const int c = t + 128 * m;          // 16-byte chunk of the 16 KiB tile
+          for (int c = 0; c < 4; ++c)
+            *(uint4*)(rowp + (((ch0 + c) ^ (pr & 7)) << 4)) = make_uint4(
+                pack_bf16x2(f[8 * c] * bv, f[8 * c + 1] * bv), pack_bf16x2(f[8 * c + 2] * bv, f[8 * c + 3] * bv),
+                pack_bf16x2(f[8 * c + 4] * bv, f[8 * c + 5] * bv), pack_bf16x2(f[8 * c + 6] * bv, f[8 * c + 7] * bv));
+          fence_proxy_async();
+          mbar_arrive(bar_bk + 8 * s);
+          continue;
+        }
+#pragma unroll
+        for (int m = 0; m < 1024 / NSC; ++m) {
+          const int c = t + NSC * m;          // 16-byte chunk of the 16 KiB tile
           const float bv = bs[(c >> 3) & (TOK - 1)];  // 8 chunks per 128-byte token row
           uint4 x = *(const uint4*)(kt + c * 16);
           uint32_t w[4] = {x.x, x.y, x.z, x.w};
@@ -322,11 +425,15 @@ __global__ void __launch_bounds__(ctr::THREADS, 1)
 }
 
 bool tc_contract_supported(int D) { return D == 128; }
+int tc_prologue_max_positions() { return ctr::TAB_MAX / 32; }
 
 cudaError_t tc_contract(const void* k, const void* v, const float* beta, float* A, float* U,
                         long long N, int S, int D, float cA, float cU, int a_image,
-                        cudaStream_t st) {
+                        const ProArgs* pro, cudaStream_t st) {
   if (D != 128) return cudaErrorNotSupported;
+  if (pro && pro->npos * (D / 4) > ctr::TAB_MAX) return cudaErrorNotSupported;
+  ProArgs pa = {};
+  if (pro) pa = *pro;
   CUtensorMap mk, mv;
   cudaError_t e = make_map_bf16_3d(&mk, k, D, S, N, 64, ctr::TOK);
   if (e != cudaSuccess) return e;
@@ -340,7 +447,7 @@ cudaError_t tc_contract(const void* k, const void* v, const float* beta, float* 
   }
   const int grid = (int)(N < num_sms() ? N : num_sms());
   k_contract_tc<<<grid, ctr::THREADS, ctr::SMEM, st>>>(mk, mv, beta, A, U, (int)N, S, cA, cU,
-                                                        a_image);
+                                                        a_image, pa);
   count_launch();
   return cudaGetLastError();
 }
@@ -358,23 +465,29 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_S = OFF_Q + NQ * QT;  // S hi (2 boxes) then S lo (2 boxes): 64 KiB
 constexpr int OFF_O = OFF_S + 4 * BOX;  // output staging, 2 boxes: 32 KiB
 constexpr int OFF_BAR = OFF_O + 2 * BOX;
-constexpr int NBAR = 2 * NQ + 2 + 4 + 1;  // q_full, q_empty, s_full, s_empty, acc f/e x2, fin
+constexpr int NBAR = 3 * NQ + 2 + 4 + 1;  // q_full, q_ready, q_empty, s_full, s_empty, acc f/e x2, fin
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr int SMEM = OFF_MISC + 16 + 1024;
-constexpr int THREADS = 192;            // producer, MMA, 4 epilogue warps
+constexpr int OFF_W = OFF_MISC + 16;    // prologue weights [D] fp32
+constexpr int OFF_TAB = OFF_W + D * 4;  // prologue (cos, sin) table copy
+constexpr int TAB_MAX = 80 * 32;
+constexpr int SMEM = OFF_TAB + TAB_MAX * 8 + 1024;
+// producer, MMA, 4 epilogue warps (+ 8 warps applying the prologue to Q tiles)
+constexpr int threads(bool pro) { return pro ? 448 : 192; }
 constexpr uint32_t TMEM_COLS = 256;
 }  // namespace rdo
 
-__global__ void __launch_bounds__(rdo::THREADS, 1)
+template <bool PRO>
+__global__ void __launch_bounds__(rdo::threads(PRO), 1)
     k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
-                 const __grid_constant__ CUtensorMap tmO, int N, int S) {
+                 const __grid_constant__ CUtensorMap tmO, int N, int S, ProArgs pro) {
   using namespace rdo;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t bar_qf = sb + OFF_BAR;
-  const uint32_t bar_qe = bar_qf + 8 * NQ;
+  const uint32_t bar_qr = bar_qf + 8 * NQ;  // Q tile transformed by the prologue warps
+  const uint32_t bar_qe = bar_qr + 8 * NQ;
   const uint32_t bar_sf = bar_qe + 8 * NQ;
   const uint32_t bar_se = bar_sf + 8;
   const uint32_t bar_accf = bar_se + 8;
@@ -386,6 +499,7 @@ __global__ void __launch_bounds__(rdo::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NQ; ++s) {
       mbar_init(bar_qf + 8 * s, 1);
+      mbar_init(bar_qr + 8 * s, 256);
       mbar_init(bar_qe + 8 * s, 1);
     }
     mbar_init(bar_sf, 1);
@@ -398,6 +512,10 @@ __global__ void __launch_bounds__(rdo::THREADS, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if (PRO && threadIdx.x < D) ((float*)(smem + OFF_W))[threadIdx.x] = pro.w[threadIdx.x];
+  if (PRO)
+    for (int e = threadIdx.x; e < pro.npos * (D / 4); e += (int)blockDim.x)
+      ((float2*)(smem + OFF_TAB))[e] = pro.cs[e];
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
     tmem_relinquish();
@@ -455,7 +573,7 @@ __global__ void __launch_bounds__(rdo::THREADS, 1)
           const uint32_t ub = (uint32_t)(g >> 1);
           ok = mbar_wait(bar_acce + 8 * b, (ub & 1) ^ 1, abort_flag, &g_tc_status, 16);
           if (!ok) break;
-          ok = mbar_wait(bar_qf + 8 * s, u & 1, abort_flag, &g_tc_status, 17);
+          ok = mbar_wait((PRO ? bar_qr : bar_qf) + 8 * s, u & 1, abort_flag, &g_tc_status, 17);
           if (!ok) break;
           tc_fence_after();
           const uint32_t qa = sb + OFF_Q + s * QT, sh = sb + OFF_S, sl = sb + OFF_S + 2 * BOX;
@@ -480,7 +598,7 @@ __global__ void __launch_bounds__(rdo::THREADS, 1)
       mbar_wait(bar_fin, 0, abort_flag, &g_tc_status, 18);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 6) {
     // ---- epilogue: TMEM -> bf16 -> swizzled staging -> TMA store ----
     const int q = warp & 3;
     const int row = q * 32 + lane;  // token within the tile
@@ -496,18 +614,6 @@ __global__ void __launch_bounds__(rdo::THREADS, 1)
         const uint32_t ub = (uint32_t)(g >> 1);
         mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 19);
         tc_fence_after();
-        uint32_t packed[64];
-#pragma unroll
-        for (int c0 = 0; c0 < 128; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 128 + c0, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            packed[c0 / 2 + j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-        }
-        tc_fence_before();
-        mbar_arrive(bar_acce + 8 * b);
         // the previous tile's TMA store has finished reading the staging tile
         if (et == 0) bulk_wait_read0();
         named_bar_sync(1, 128);
@@ -516,12 +622,26 @@ __global__ void __launch_bounds__(rdo::THREADS, 1)
           break;
         }
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int box = j >> 3, chunk = j & 7;
-          uint8_t* dst = ost + box * BOX + row * 128 + ((chunk ^ (row & 7)) << 4);
-          *(uint4*)dst = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2],
-                                    packed[4 * j + 3]);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t packed[32];
+#pragma unroll
+          for (int c0 = 0; c0 < 64; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 128 + half * 64 + c0, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              packed[c0 / 2 + j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+          }
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint8_t* dst = ost + half * BOX + row * 128 + ((c ^ (row & 7)) << 4);
+            *(uint4*)dst = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2],
+                                      packed[4 * c + 3]);
+          }
         }
+        tc_fence_before();
+        mbar_arrive(bar_acce + 8 * b);
         fence_proxy_async();
         named_bar_sync(1, 128);
         if (et == 0) {
@@ -532,6 +652,26 @@ __global__ void __launch_bounds__(rdo::THREADS, 1)
       }
     }
     if (et == 0) bulk_wait0();
+  } else if (PRO) {
+    // ---- prologue on each raw Q tile, in place (two threads per token) ----
+    const int t = threadIdx.x - 192;
+    const int r = t >> 1, h = t & 1;
+    int g = 0;
+    bool ok = true;
+    for (int i = 0; i < my_count && ok; ++i) {
+      for (int tl = 0; tl < ntile; ++tl, ++g) {
+        const int s = g % NQ;
+        const uint32_t u = (uint32_t)(g / NQ);
+        ok = mbar_wait(bar_qf + 8 * s, u & 1, abort_flag, &g_tc_status, 20);
+        if (!ok) break;
+        const int tok = tl * TOK + r;
+        float f[64];
+        pro_row_part<8>(smem + OFF_Q + s * QT, BOX, r, 64 * h, D, tok, tok < S, pro,
+                        (const float*)(smem + OFF_W) + 64 * h, (const float2*)(smem + OFF_TAB), f);
+        fence_proxy_async();
+        mbar_arrive(bar_qr + 8 * s);
+      }
+    }
   }
 
   tc_fence_before();
@@ -544,9 +684,26 @@ __global__ void __launch_bounds__(rdo::THREADS, 1)
 
 bool tc_readout_supported(int D) { return D == 128; }
 
+template <bool PRO>
+static cudaError_t launch_readout(const CUtensorMap& mq, const CUtensorMap& ms, const CUtensorMap& mo,
+                                  long long N, int S, const ProArgs& pa, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_readout_tc<PRO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         rdo::SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int grid = (int)(N < num_sms() ? N : num_sms());
+  k_readout_tc<PRO><<<grid, rdo::threads(PRO), rdo::SMEM, st>>>(mq, ms, mo, (int)N, S, pa);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t tc_readout(const void* q, const void* Sfr_hilo, void* out, long long N, int S, int D,
-                       cudaStream_t st) {
+                       const ProArgs* pro, cudaStream_t st) {
   if (D != 128) return cudaErrorNotSupported;
+  if (pro && pro->npos * (D / 4) > rdo::TAB_MAX) return cudaErrorNotSupported;
   CUtensorMap mq, ms, mo;
   cudaError_t e = make_map_bf16_3d(&mq, q, D, S, N, 64, rdo::TOK);
   if (e != cudaSuccess) return e;
@@ -554,16 +711,12 @@ cudaError_t tc_readout(const void* q, const void* Sfr_hilo, void* out, long long
   if (e != cudaSuccess) return e;
   e = make_map_bf16_3d(&mo, out, D, S, N, 64, rdo::TOK);
   if (e != cudaSuccess) return e;
-  static bool attr = false;
-  if (!attr) {
-    e = cudaFuncSetAttribute(k_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, rdo::SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
+  ProArgs pa = {};
+  if (pro) {
+    pa = *pro;
+    return launch_readout<true>(mq, ms, mo, N, S, pa, st);
   }
-  const int grid = (int)(N < num_sms() ? N : num_sms());
-  k_readout_tc<<<grid, rdo::THREADS, rdo::SMEM, st>>>(mq, ms, mo, (int)N, S);
-  count_launch();
-  return cudaGetLastError();
+  return launch_readout<false>(mq, ms, mo, N, S, pa, st);
 }
 
 // ============================================================================

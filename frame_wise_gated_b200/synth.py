@@ -58,6 +58,8 @@ CONFIGS = {
     "rollout60s_720p": Config("rollout60s_720p", 1, 16, 121, 3600, 128, 45, 80, True, 3),
     "prologue_bidir_720p": Config("prologue_bidir_720p", 1, 16, 121, 3600, 128, 45, 80, True, 4,
                                   prologue=True, bidir_block=3),
+    "prologue_bidir_clip5s_720p": Config("prologue_bidir_clip5s_720p", 1, 16, 21, 3600, 128, 45,
+                                         80, True, 7, prologue=True, bidir_block=3),
     "sweep_d64": Config("sweep_d64", 4, 32, 61, 3600, 64, 45, 80, True, 5,
                         beta_dist="beta22", gamma_lo=0.8, state_sigma=0.1),
     "sweep_d256": Config("sweep_d256", 4, 8, 61, 3600, 256, 45, 80, True, 6,
