@@ -70,6 +70,7 @@ def phase_bytes(cfg):
     return {
         "contract": fh * cfg.S * (2 * cfg.D * e + 4),          # K, V, beta
         "readout": fh * cfg.S * 2 * cfg.D * e,                  # Q in, O out
+        "scan_readout": fh * cfg.S * 2 * cfg.D * e,             # Q in, O out (replay fused)
         "prologue": fh * cfg.S * 4 * cfg.D * e,                 # raw q, k in; q^, k^ out
         "_readout_launches_per_step": nro,
     }
@@ -269,14 +270,15 @@ def run_ours(args, cfg):
         pro = dict(w_q=torch.from_numpy(arr["w_q"]).to(dev), w_k=torch.from_numpy(arr["w_k"]).to(dev),
                    grid_h=cfg.grid_h, grid_w=cfg.grid_w)
     kw = dict(prologue=pro, bidir=bool(cfg.bidir_block), block_reset=bool(cfg.bidir_block),
-              block=cfg.bidir_block or 3, sequential=args.sequential)
+              block=cfg.bidir_block or 3, sequential=args.sequential,
+              fused_replay=args.fused_replay)
     out = torch.empty_like(q)
     out_rev = torch.empty_like(q) if cfg.bidir_block else None
     st_out = torch.empty((cfg.B, cfg.H, cfg.D, cfg.D), device=dev, dtype=torch.float32)
     st_rev = torch.empty_like(st_out) if cfg.bidir_block else None
     flags = api.scan_flags(bf16=cfg.bf16, prologue=pro is not None, bidir=bool(cfg.bidir_block),
                            block_reset=bool(cfg.bidir_block), block=cfg.bidir_block or 3,
-                           sequential=args.sequential)
+                           sequential=args.sequential, fused_replay=args.fused_replay)
     ws = torch.empty(api.workspace_bytes(cfg.B, cfg.H, cfg.T, cfg.S, cfg.D, flags),
                      device=dev, dtype=torch.uint8)
     stream = torch.cuda.current_stream(dev)
@@ -445,6 +447,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="rollout60s_720p", choices=sorted(synth.CONFIGS))
     ap.add_argument("--sequential", action="store_true")
+    ap.add_argument("--fused-replay", action="store_true",
+                    help="replay spans inside the readout kernel")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-frames", type=int, default=6,

@@ -32,6 +32,7 @@ FUSED_PROLOGUE = 0x10
 KEYS_SCALED = 0x20
 FORCE_SIMT = 0x40
 BIDIR = 0x80
+FUSED_REPLAY = 0x1000000
 
 
 def make_block(n: int) -> int:
@@ -85,7 +86,7 @@ SIGNATURES = {
     "gdn_profile_read": (_I, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong), _I]),
 }
 
-PHASES = ("prologue", "contract", "compose", "prefix", "scan", "readout")
+PHASES = ("prologue", "contract", "compose", "prefix", "scan", "readout", "scan_readout")
 
 _lib = None
 
@@ -135,8 +136,9 @@ def _want(t: torch.Tensor, name: str, dtype=None, shape=None):
 
 def scan_flags(*, bf16: bool, reverse=False, block_reset=False, block=3, chunk=8,
                sequential=False, keys_scaled=False, force_simt=False, prologue=False,
-               bidir=False) -> int:
+               bidir=False, fused_replay=False) -> int:
     f = (BF16 if bf16 else 0) | make_block(block) | make_chunk(chunk)
+    f |= FUSED_REPLAY if fused_replay else 0
     f |= REVERSE if reverse else 0
     f |= BLOCK_RESET if block_reset else 0
     f |= SEQUENTIAL if sequential else 0
@@ -153,8 +155,8 @@ def workspace_bytes(B, H, T, S, D, flags) -> int:
 
 def frame_scan_fwd_ex(q, k, v, beta, gamma, state_in=None, *, reverse=False, block_reset=False,
                       block=3, chunk=8, sequential=False, keys_scaled=False, force_simt=False,
-                      prologue=None, bidir=False, out=None, state_out=None, out_rev=None,
-                      state_out_rev=None, workspace=None, stream=None):
+                      prologue=None, bidir=False, fused_replay=False, out=None, state_out=None,
+                      out_rev=None, state_out_rev=None, workspace=None, stream=None):
     """The frame scan through gdn_frame_scan_fwd_ex.
 
     q, k, v [B,H,T,S,D] (bf16 or fp32); beta [B,H,T,S] fp32; gamma [B,H,T]
@@ -174,7 +176,8 @@ def frame_scan_fwd_ex(q, k, v, beta, gamma, state_in=None, *, reverse=False, blo
         _want(state_in, "state_in", torch.float32, (B, H, D, D))
     flags = scan_flags(bf16=bf16, reverse=reverse, block_reset=block_reset, block=block,
                        chunk=chunk, sequential=sequential, keys_scaled=keys_scaled,
-                       force_simt=force_simt, prologue=prologue is not None, bidir=bidir)
+                       force_simt=force_simt, prologue=prologue is not None, bidir=bidir,
+                       fused_replay=fused_replay)
     out = torch.empty_like(q) if out is None else out
     state_out = torch.empty((B, H, D, D), device=q.device, dtype=torch.float32) \
         if state_out is None else state_out

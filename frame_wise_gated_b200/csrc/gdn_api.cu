@@ -29,7 +29,10 @@ static thread_local long long t_launches = 0;
 void count_launch(int n) { t_launches += n; }
 
 // ---- phase timing with CUDA events (gdn_profile_enable / gdn_profile_read) ----
-enum Phase { PH_PROLOGUE = 0, PH_CONTRACT, PH_COMPOSE, PH_PREFIX, PH_SCAN, PH_READOUT, PH_COUNT };
+enum Phase {
+  PH_PROLOGUE = 0, PH_CONTRACT, PH_COMPOSE, PH_PREFIX, PH_SCAN, PH_READOUT, PH_SCAN_READOUT,
+  PH_COUNT
+};
 struct ProfRec {
   int phase;
   cudaEvent_t a, b;
@@ -193,6 +196,33 @@ static int run_direction(const gdn_params& p, const Layout& L, char* ws, bool re
     return use_tc_chain ? tc_chain(c, n, st) : simt_chain(c, n, st);
   };
   cudaError_t e;
+  // Replay fused with the readout: spans or reset blocks, tensor-core path, no prologue.
+  const bool fused = (p.flags & GDN_FUSED_REPLAY) && use_tc_chain && use_tc_readout && !pro_q &&
+                     (p.flags & GDN_BF16) &&
+                     !(p.flags & GDN_SEQUENTIAL) && tc_scan_readout_supported(p.D);
+  auto scan_readout = [&](const ChainArgs& c, int n) -> int {
+    PhaseScope ps(PH_SCAN_READOUT, st);
+    cudaError_t er = tc_scan_readout(c, n, q, out, p.S, st);
+    return er == cudaSuccess ? GDN_OK : cuda_fail(er, "scan+readout");
+  };
+  if (fused) {
+    a.mode = CHAIN_SCAN;
+    if (block_reset) {
+      a.seg = SEG_BLOCKS;
+      a.nseg = (p.T + a.block - 1) / a.block;
+      return scan_readout(a, a.heads * a.nseg);
+    }
+    a.seg = SEG_CHUNKS;
+    a.nseg = (p.T + a.L - 1) / a.L;
+    if (a.nseg > 1) {
+      a.mode = CHAIN_COMPOSE;
+      if ((e = chain(a, 2 * a.heads * a.nseg)) != cudaSuccess) return cuda_fail(e, "compose");
+      a.mode = CHAIN_PREFIX;
+      if ((e = chain(a, a.heads)) != cudaSuccess) return cuda_fail(e, "prefix");
+      a.mode = CHAIN_SCAN;
+    }
+    return scan_readout(a, a.heads * a.nseg);
+  }
   if (p.flags & GDN_SEQUENTIAL) {
     a.seg = SEG_SEQUENTIAL;
     a.seq_reset = block_reset ? 1 : 0;

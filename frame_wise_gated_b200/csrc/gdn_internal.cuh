@@ -151,6 +151,10 @@ cudaError_t tc_to_image(const float* src, void* dst, long long n, cudaStream_t s
 bool tc_readout_supported(int D);
 cudaError_t tc_readout(const void* q, const void* Sfr_hilo, void* out, long long N, int S, int D,
                        const ProArgs* pro, cudaStream_t st);
+// Replay of CHAIN_SCAN chains fused with the readout (bf16 out, no prologue).
+bool tc_scan_readout_supported(int D);
+cudaError_t tc_scan_readout(const ChainArgs& a, int nchains, const void* q, void* out, int S,
+                            cudaStream_t st);
 bool tc_chain_supported(int D);
 cudaError_t tc_chain(const ChainArgs& a, int nchains, cudaStream_t st);
 // Reads and clears the device status word of the tensor-core kernels.

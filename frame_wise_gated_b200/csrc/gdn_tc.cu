@@ -739,8 +739,9 @@ constexpr int HALF = 64 * 128 * 2 * 2;  // one bf16 128x128 operand tile: 32 KiB
 constexpr int ATOM = 128 * 128;         // 16 KiB: 128 rows x 128 bytes
 constexpr int OFF_XH = 0;
 constexpr int OFF_XL = OFF_XH + HALF;
-constexpr int OFF_Y = OFF_XL + HALF;     // Y image b at OFF_Y + b * kImageBytes (hi, then lo)
-constexpr int OFF_BAR = OFF_Y + 2 * kImageBytes;  // bar_mma, bar_y[2]
+constexpr int OFF_Y = OFF_XL + HALF;     // Y operand image (hi, then lo)
+constexpr int OFF_Z = OFF_Y + kImageBytes;  // Z fp32: 4 boxes of [128 rows][32 fp32], swizzled
+constexpr int OFF_BAR = OFF_Z + kImageBytes;  // bar_mma, bar_y, bar_z
 constexpr int OFF_MISC = OFF_BAR + 32;
 constexpr int SMEM = OFF_MISC + 16 + 1024;
 constexpr int THREADS = 256;
@@ -889,7 +890,9 @@ __device__ __forceinline__ void store_row_image(uint8_t* img, const float* x, in
                 (uint4*)(img + 2 * chn::ATOM + tile_off(row, h, c)));
 }
 
-__global__ void __launch_bounds__(chn::THREADS, 1) k_chain_tc(ChainArgs a) {
+__global__ void __launch_bounds__(chn::THREADS, 1)
+    k_chain_tc(ChainArgs a, const __grid_constant__ CUtensorMap tmZ,
+               const __grid_constant__ CUtensorMap tmSfr) {
   using namespace chn;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -897,17 +900,23 @@ __global__ void __launch_bounds__(chn::THREADS, 1) k_chain_tc(ChainArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = warp & 3, h = warp >> 2;
   const int row = q * 32 + lane;
+  const bool leader = threadIdx.x == 0;
   const uint32_t bar_mma = sb + OFF_BAR;
-  const uint32_t bar_y = bar_mma + 8;  // two, one per Y buffer
+  const uint32_t bar_y = bar_mma + 8;
+  const uint32_t bar_z = bar_mma + 16;
   uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
   volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
   const size_t DD = (size_t)D * D;
   const ChainProg g = chain_prog(a, blockIdx.x);
+  // Z comes from global memory (TMA) except for the span composite E, whose
+  // Z is its own Y (read back from the Y image).
+  const bool z_global = !(g.mode == CHAIN_COMPOSE && g.which == 0);
+  const bool store_sfr = g.mode == CHAIN_SCAN;
 
-  if (threadIdx.x == 0) {
+  if (leader) {
     mbar_init(bar_mma, 1);
     mbar_init(bar_y, 1);
-    mbar_init(bar_y + 8, 1);
+    mbar_init(bar_z, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -919,11 +928,23 @@ __global__ void __launch_bounds__(chn::THREADS, 1) k_chain_tc(ChainArgs a) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  int fetched = 0;  // Y images requested so far (thread 0)
-  if (threadIdx.x == 0) {
-    for (; fetched < 2 && fetched < g.n; ++fetched)
-      chain_fetch_y(sb + OFF_Y + fetched * kImageBytes, chain_step_at(a, g, fetched).Y,
-                    bar_y + 8 * fetched);
+  // Z of step s: matrix index for the tensor map (frame for U, span for H).
+  auto z_index = [&](const ChainStep& st) -> int {
+    return g.mode == CHAIN_PREFIX ? g.bh * a.nseg + st.t : g.bh * a.T + st.t;
+  };
+  auto fetch_z = [&](int zi) {
+    mbar_arrive_expect_tx(bar_z, kImageBytes);
+#pragma unroll
+    for (int b = 0; b < 4; ++b) tma_load_3d(sb + OFF_Z + b * ATOM, &tmZ, bar_z, 32 * b, 0, zi);
+  };
+  int nz = 0, ny = 0, nstore = 0;  // copies issued (leader)
+  if (leader && g.n > 0) {
+    chain_fetch_y(sb + OFF_Y, chain_step_at(a, g, 0).Y, bar_y);
+    ++ny;
+    if (z_global) {
+      fetch_z(z_index(chain_step_at(a, g, 0)));
+      ++nz;
+    }
   }
 
   float x[64];
@@ -939,50 +960,25 @@ __global__ void __launch_bounds__(chn::THREADS, 1) k_chain_tc(ChainArgs a) {
     for (int c = 0; c < 64; ++c) x[c] = 0.f;
   }
   float gprod = 1.f;
+  int tprev = -1;  // frame whose state sits in the X tile, to be stored
 
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, true);
   for (int s = 0; s < g.n; ++s) {
     const ChainStep st = chain_step_at(a, g, s);
-    const int yb = s & 1;
     if (g.mode == CHAIN_PREFIX)
       store_row_f32(a.Sst + ((size_t)g.bh * a.nseg + s) * DD + (size_t)row * D + h * 64, x);
-    if (st.reset) {
-#pragma unroll
-      for (int c = 0; c < 64; ++c) x[c] = 0.f;
-    }
+    // A reset (zero state entering this step) is applied in the update below
+    // (x <- Z), so the tile still carries the previous frame's state to store.
+    // The X tile is free once the previous state store has read it.
+    if (leader && nstore > 0) bulk_wait_read0();
+    __syncthreads();
     chain_store_x(x, smem + OFF_XH, smem + OFF_XL, row, h);
     fence_proxy_async();
-    // Y_s has landed (every thread observes the copy's completion)
-    mbar_wait(bar_y + 8 * yb, (uint32_t)(s >> 1) & 1, abort_flag, &g_tc_status, 22);
-    __syncthreads();
-    if (*abort_flag) break;  // uniform: read after the barrier
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-      const uint32_t yh = sb + OFF_Y + yb * kImageBytes, yl = yh + 2 * ATOM;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t xo = (kk >> 2) * ATOM + (kk & 3) * 32;
-        const uint64_t dxh = smem_desc_sw128(sb + OFF_XH + xo, 16, 1024);
-        const uint64_t dxl = smem_desc_sw128(sb + OFF_XL + xo, 16, 1024);
-        const uint64_t dyh = smem_desc_sw128(yh + kk * 2048, ATOM, 1024);
-        const uint64_t dyl = smem_desc_sw128(yl + kk * 2048, ATOM, 1024);
-        mma_bf16(tmem, dxh, dyh, idesc, kk > 0 ? 1u : 0u);
-        mma_bf16(tmem, dxl, dyh, idesc, 1u);
-        mma_bf16(tmem, dxh, dyl, idesc, 1u);
-      }
-      mma_commit(bar_mma);
-    }
+    mbar_wait(bar_y, (uint32_t)s & 1, abort_flag, &g_tc_status, 22);
     float z[64];
-    if (st.Z) {
-      const float* zr = st.Z + (size_t)row * D + h * 64;
-#pragma unroll
-      for (int c = 0; c < 64; c += 4) {
-        const float4 f = __ldg((const float4*)(zr + c));
-        z[c] = f.x; z[c + 1] = f.y; z[c + 2] = f.z; z[c + 3] = f.w;
-      }
-    } else {
-      // Z = Y: read this row's slice back from the image (hi + lo)
-      const uint8_t* yi = smem + OFF_Y + yb * kImageBytes;
+    if (!z_global) {
+      // Z = Y: this row's slice of the image (hi + lo), read before the buffer is refilled
+      const uint8_t* yi = smem + OFF_Y;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const uint4 hi = *(const uint4*)(yi + tile_off(row, h, c));
@@ -997,10 +993,52 @@ __global__ void __launch_bounds__(chn::THREADS, 1) k_chain_tc(ChainArgs a) {
         }
       }
     }
+    __syncthreads();
+    if (*abort_flag) break;  // uniform: read after the barrier
+    if (leader) {
+      if (store_sfr && tprev >= 0) {
+        // the tile holds S of frame tprev: store its hi/lo pair for the readout
+        const int zz = 2 * (g.bh * a.T + tprev);
+        tma_store_3d(&tmSfr, sb + OFF_XH, 0, 0, zz);
+        tma_store_3d(&tmSfr, sb + OFF_XH + ATOM, 64, 0, zz);
+        tma_store_3d(&tmSfr, sb + OFF_XL, 0, 0, zz + 1);
+        tma_store_3d(&tmSfr, sb + OFF_XL + ATOM, 64, 0, zz + 1);
+        bulk_commit();
+        ++nstore;
+      }
+      tc_fence_after();
+      const uint32_t yh = sb + OFF_Y, yl = yh + 2 * ATOM;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t xo = (kk >> 2) * ATOM + (kk & 3) * 32;
+        const uint64_t dxh = smem_desc_sw128(sb + OFF_XH + xo, 16, 1024);
+        const uint64_t dxl = smem_desc_sw128(sb + OFF_XL + xo, 16, 1024);
+        const uint64_t dyh = smem_desc_sw128(yh + kk * 2048, ATOM, 1024);
+        const uint64_t dyl = smem_desc_sw128(yl + kk * 2048, ATOM, 1024);
+        mma_bf16(tmem, dxh, dyh, idesc, kk > 0 ? 1u : 0u);
+        mma_bf16(tmem, dxl, dyh, idesc, 1u);
+        mma_bf16(tmem, dxh, dyl, idesc, 1u);
+      }
+      mma_commit(bar_mma);
+    }
     // On a timeout the flag is set; the step finishes on stale values and
     // every thread leaves at the next barrier.
     mbar_wait(bar_mma, (uint32_t)s & 1, abort_flag, &g_tc_status, 21);
     tc_fence_after();
+    if (leader && s + 1 < g.n) {  // the Y buffer is free: next step's Y
+      chain_fetch_y(sb + OFF_Y, chain_step_at(a, g, s + 1).Y, bar_y);
+      ++ny;
+    }
+    if (z_global) {
+      mbar_wait(bar_z, (uint32_t)s & 1, abort_flag, &g_tc_status, 24);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        // columns 64h + 4c .. +3 sit in box (2h + c/8), 16-byte chunk c % 8
+        const int box = 2 * h + (c >> 3), ch = c & 7;
+        const float4 f = *(const float4*)(smem + OFF_Z + box * ATOM + row * 128 + ((ch ^ (row & 7)) << 4));
+        z[4 * c] = f.x; z[4 * c + 1] = f.y; z[4 * c + 2] = f.z; z[4 * c + 3] = f.w;
+      }
+    }
 #pragma unroll
     for (int c0 = 0; c0 < 64; c0 += 32) {
       uint32_t r[32];
@@ -1008,27 +1046,42 @@ __global__ void __launch_bounds__(chn::THREADS, 1) k_chain_tc(ChainArgs a) {
       tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 32; ++c)
-        x[c0 + c] = st.alpha * (x[c0 + c] - __uint_as_float(r[c])) + z[c0 + c];
+        x[c0 + c] = st.reset ? z[c0 + c]
+                             : st.alpha * (x[c0 + c] - __uint_as_float(r[c])) + z[c0 + c];
     }
     tc_fence_before();
-    // Every thread is past its reads of Y buffer yb (the Z = Y read) and the
-    // MMA reading it has completed: refill it with Y_{s+2}.
-    __syncthreads();
-    if (threadIdx.x == 0 && s + 2 < g.n) {
-      chain_fetch_y(sb + OFF_Y + yb * kImageBytes, chain_step_at(a, g, s + 2).Y, bar_y + 8 * yb);
-      ++fetched;
+    if (z_global) {
+      // every thread has read Z: fetch the next step's
+      __syncthreads();
+      if (leader && s + 1 < g.n) {
+        fetch_z(z_index(chain_step_at(a, g, s + 1)));
+        ++nz;
+      }
     }
     if (g.mode == CHAIN_COMPOSE) gprod *= a.gamma[(size_t)g.bh * a.T + st.t];
     if (g.mode == CHAIN_SCAN) {
-      const size_t fi = (size_t)g.bh * a.T + st.t;
-      if (a.sfr_hilo) {
-        __nv_bfloat16* base = (__nv_bfloat16*)a.Sfr + fi * 2 * DD + (size_t)row * D + h * 64;
-        store_row_hilo(base, base + DD, x);
-      } else {
-        store_row_f32(a.Sfr + fi * DD + (size_t)row * D + h * 64, x);
-      }
+      tprev = st.t;
       if (g.j0 + s == a.T - 1 && a.state_out)
         store_row_f32(a.state_out + (size_t)g.bh * DD + (size_t)row * D + h * 64, x);
+    }
+  }
+  // the last state of a scan chain: through the X tile to its hi/lo store
+  if (store_sfr && tprev >= 0) {
+    if (leader && nstore > 0) bulk_wait_read0();
+    __syncthreads();
+    if (!*abort_flag) {
+      chain_store_x(x, smem + OFF_XH, smem + OFF_XL, row, h);
+      fence_proxy_async();
+    }
+    __syncthreads();
+    if (leader && !*abort_flag) {
+      const int zz = 2 * (g.bh * a.T + tprev);
+      tma_store_3d(&tmSfr, sb + OFF_XH, 0, 0, zz);
+      tma_store_3d(&tmSfr, sb + OFF_XH + ATOM, 64, 0, zz);
+      tma_store_3d(&tmSfr, sb + OFF_XL, 0, 0, zz + 1);
+      tma_store_3d(&tmSfr, sb + OFF_XL + ATOM, 64, 0, zz + 1);
+      bulk_commit();
+      ++nstore;
     }
   }
   __syncthreads();
@@ -1046,10 +1099,11 @@ __global__ void __launch_bounds__(chn::THREADS, 1) k_chain_tc(ChainArgs a) {
       store_row_f32(a.Sst + ((size_t)g.bh * a.nseg + g.n) * DD + (size_t)row * D + h * 64, x);
     }
   }
-  // Drain: wait (bounded) for any Y copy still in flight before teardown.
-  if (threadIdx.x == 0) {
-    for (int s = (fetched > 2 ? fetched - 2 : 0); s < fetched; ++s)
-      mbar_wait(bar_y + 8 * (s & 1), (uint32_t)(s >> 1) & 1, abort_flag, &g_tc_status, 23);
+  // Drain (bounded): copies in flight land before teardown.
+  if (leader) {
+    if (nstore > 0) bulk_wait0();
+    if (ny > 0) mbar_wait(bar_y, (uint32_t)(ny - 1) & 1, abort_flag, &g_tc_status, 23);
+    if (nz > 0) mbar_wait(bar_z, (uint32_t)(nz - 1) & 1, abort_flag, &g_tc_status, 25);
   }
   tc_fence_before();
   __syncthreads();
@@ -1079,10 +1133,336 @@ cudaError_t tc_to_image(const float* src, void* dst, long long n, cudaStream_t s
   return cudaGetLastError();
 }
 
+// ============================================================================
+// Replay fused with the readout (steps a5 + a6), D = 128.
+//
+// One CTA takes one chain of CHAIN_SCAN (a span of frames, or a reset block)
+// and, frame by frame, first advances the state on tensor cores
+//     P = S_{f-1} A_t (3 bf16 products),  S_f = gamma_t (S_{f-1} - P) + U_t
+// then streams the frame's Q tiles through
+//     O_tile = Q_tile S_f^T = Q_tile S_hi^T + Q_tile S_lo^T.
+// The bf16 (hi, lo) state tile in shared memory is at once the A operand of
+// the next state step and the B operand of this frame's readout, so S_t never
+// goes to HBM. While the readout of frame f streams, the next state step's
+// MMA already runs; the state warps write S_{f+1} into the tile as soon as the
+// last readout MMA of frame f has drained.
+// Roles: warp 0 TMA producer of Q tiles; warp 1 MMA issuer; warps 2-9 hold
+// the state (row 32 (w % 4) + lane, columns 64 ((w - 2) / 4) ..) and run the
+// readout epilogue (token row 32 (w % 4) + lane of the tile, same columns),
+// writing O straight to global memory.
+// ============================================================================
+namespace sro {
+constexpr int D = 128;
+constexpr int TOK = 128;
+constexpr int NQ = 3;
+constexpr int BOX = TOK * 128;          // [128 rows][64 channels] bf16: 16 KiB
+constexpr int QT = 2 * BOX;
+constexpr int OFF_Q = 0;
+constexpr int OFF_X = OFF_Q + NQ * QT;  // state tile: hi (2 atoms) then lo (2 atoms)
+constexpr int OFF_Y = OFF_X + 4 * BOX;  // A_t operand image
+constexpr int OFF_BAR = OFF_Y + kImageBytes;
+constexpr int NBAR = 2 * NQ + 4 + 4 + 1;  // q_full, q_empty, y_full, x_full, p_full, r_done, acc f/e x2, fin
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+constexpr int THREADS = 320;
+constexpr uint32_t TMEM_COLS = 512;    // two readout accumulators + the state product
+constexpr uint32_t P_COL = 256;
+}  // namespace sro
+
+__global__ void __launch_bounds__(sro::THREADS, 1)
+    k_scan_readout_tc(ChainArgs a, const __grid_constant__ CUtensorMap tmQ,
+                      __nv_bfloat16* __restrict__ out, int S, int nchains) {
+  using namespace sro;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar_qf = sb + OFF_BAR;
+  const uint32_t bar_qe = bar_qf + 8 * NQ;
+  const uint32_t bar_yf = bar_qe + 8 * NQ;
+  const uint32_t bar_xf = bar_yf + 8;
+  const uint32_t bar_pf = bar_xf + 8;
+  const uint32_t bar_rd = bar_pf + 8;
+  const uint32_t bar_accf = bar_rd + 8;
+  const uint32_t bar_acce = bar_accf + 16;
+  const uint32_t bar_fin = bar_acce + 16;
+  uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
+  const size_t DD = (size_t)D * D;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NQ; ++s) {
+      mbar_init(bar_qf + 8 * s, 1);
+      mbar_init(bar_qe + 8 * s, 1);
+    }
+    mbar_init(bar_yf, 1);
+    mbar_init(bar_xf, 256);
+    mbar_init(bar_pf, 1);
+    mbar_init(bar_rd, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_accf + 8 * b, 1);
+      mbar_init(bar_acce + 8 * b, 256);
+    }
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int ntile = (S + TOK - 1) / TOK;
+
+  if (warp == 0) {
+    // ---- Q tiles of every frame of every chain, in order ----
+    if (lane == 0) {
+      int g = 0;
+      bool ok = true;
+      for (int c = blockIdx.x; c < nchains && ok; c += gridDim.x) {
+        const ChainProg pg = chain_prog(a, c);
+        for (int f = 0; f < pg.n && ok; ++f) {
+          const int n = pg.bh * a.T + frame_at(pg.j0 + f, a.T, a.reverse);
+          for (int tl = 0; tl < ntile; ++tl, ++g) {
+            const int s = g % NQ;
+            const uint32_t u = (uint32_t)(g / NQ);
+            ok = mbar_wait(bar_qe + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 31);
+            if (!ok) break;
+            const uint32_t qd = sb + OFF_Q + s * QT;
+            mbar_arrive_expect_tx(bar_qf + 8 * s, QT);
+            tma_load_3d(qd, &tmQ, bar_qf + 8 * s, 0, tl * TOK, n);
+            tma_load_3d(qd + BOX, &tmQ, bar_qf + 8 * s, 64, tl * TOK, n);
+          }
+        }
+      }
+      for (int gg = (g > NQ ? g - NQ : 0); gg < g; ++gg)
+        mbar_wait(bar_qf + 8 * (gg % NQ), (uint32_t)(gg / NQ) & 1, abort_flag, &g_tc_status, 32);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---- MMA issuer: state step, then the frame's readout tiles ----
+    if (lane == 0) {
+      constexpr uint32_t id_chain = idesc_bf16_f32(128, 128, false, true);
+      constexpr uint32_t id_read = idesc_bf16_f32(128, 128, false, false);
+      const uint32_t xh = sb + OFF_X, xl = sb + OFF_X + 2 * BOX;
+      int cidx = 0, xidx = 0, g = 0;
+      bool ok = true;
+      auto chain_mma = [&]() {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t xo = (kk >> 2) * BOX + (kk & 3) * 32;
+          const uint64_t dxh = smem_desc_sw128(xh + xo, 16, 1024);
+          const uint64_t dxl = smem_desc_sw128(xl + xo, 16, 1024);
+          const uint64_t dyh = smem_desc_sw128(sb + OFF_Y + kk * 2048, BOX, 1024);
+          const uint64_t dyl = smem_desc_sw128(sb + OFF_Y + 2 * BOX + kk * 2048, BOX, 1024);
+          mma_bf16(tmem + P_COL, dxh, dyh, id_chain, kk > 0 ? 1u : 0u);
+          mma_bf16(tmem + P_COL, dxl, dyh, id_chain, 1u);
+          mma_bf16(tmem + P_COL, dxh, dyl, id_chain, 1u);
+        }
+        mma_commit(bar_pf);
+      };
+      for (int c = blockIdx.x; c < nchains && ok; c += gridDim.x) {
+        const ChainProg pg = chain_prog(a, c);
+        // S_init in the tile -> first state step
+        ok = mbar_wait(bar_xf, (uint32_t)(xidx++) & 1, abort_flag, &g_tc_status, 33);
+        if (!ok) break;
+        ok = mbar_wait(bar_yf, (uint32_t)(cidx++) & 1, abort_flag, &g_tc_status, 34);
+        if (!ok) break;
+        tc_fence_after();
+        chain_mma();
+        for (int f = 0; f < pg.n && ok; ++f) {
+          ok = mbar_wait(bar_xf, (uint32_t)(xidx++) & 1, abort_flag, &g_tc_status, 35);  // S_f
+          if (!ok) break;
+          tc_fence_after();
+          if (f + 1 < pg.n) {
+            ok = mbar_wait(bar_yf, (uint32_t)(cidx++) & 1, abort_flag, &g_tc_status, 36);
+            if (!ok) break;
+            tc_fence_after();
+            chain_mma();
+          }
+          for (int tl = 0; tl < ntile; ++tl, ++g) {
+            const int s = g % NQ;
+            const uint32_t u = (uint32_t)(g / NQ);
+            const int b = g & 1;
+            const uint32_t ub = (uint32_t)(g >> 1);
+            ok = mbar_wait(bar_acce + 8 * b, (ub & 1) ^ 1, abort_flag, &g_tc_status, 37);
+            if (!ok) break;
+            ok = mbar_wait(bar_qf + 8 * s, u & 1, abort_flag, &g_tc_status, 38);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t qa = sb + OFF_Q + s * QT;
+            const uint32_t d = tmem + b * 128;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * BOX + (kk & 3) * 32;
+              const uint64_t dq = smem_desc_sw128(qa + off, 16, 1024);
+              const uint64_t dh = smem_desc_sw128(xh + off, 16, 1024);
+              const uint64_t dl = smem_desc_sw128(xl + off, 16, 1024);
+              mma_bf16(d, dq, dh, id_read, kk > 0 ? 1u : 0u);
+              mma_bf16(d, dq, dl, id_read, 1u);
+            }
+            mma_commit(bar_qe + 8 * s);
+            mma_commit(bar_accf + 8 * b);
+          }
+          mma_commit(bar_rd);
+        }
+      }
+      mma_commit(bar_fin);
+      mbar_wait(bar_fin, 0, abort_flag, &g_tc_status, 39);
+    }
+    __syncwarp();
+  } else {
+    // ---- state + readout epilogue (256 threads) ----
+    const int q = warp & 3, h = (warp - 2) >> 2;
+    const int row = q * 32 + lane;
+    const bool leader = threadIdx.x == 64;
+    uint8_t* xtile = smem + OFF_X;
+    int pidx = 0, ridx = 0, g = 0, fetched = 0;
+    float x[64];
+    auto fetch_y = [&](const void* src) {
+      if (leader) {
+        chain_fetch_y(sb + OFF_Y, src, bar_yf);
+        ++fetched;
+      }
+    };
+    auto write_x = [&]() {
+      chain_store_x(x, xtile, xtile + 2 * BOX, row, h);
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(bar_xf);
+    };
+    for (int c = blockIdx.x; c < nchains; c += gridDim.x) {
+      const ChainProg pg = chain_prog(a, c);
+      if (*abort_flag) break;
+      // the previous readout (if any) has drained the tile
+      if (ridx > 0) mbar_wait(bar_rd, (uint32_t)(ridx - 1) & 1, abort_flag, &g_tc_status, 40);
+      if (pg.init) {
+        const float* src = pg.init + (size_t)row * D + h * 64;
+#pragma unroll
+        for (int cc = 0; cc < 64; cc += 4) {
+          const float4 v = __ldg((const float4*)(src + cc));
+          x[cc] = v.x; x[cc + 1] = v.y; x[cc + 2] = v.z; x[cc + 3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < 64; ++cc) x[cc] = 0.f;
+      }
+      fetch_y(chain_step_at(a, pg, 0).Y);
+      write_x();
+      for (int f = 0; f < pg.n; ++f) {
+        const ChainStep st = chain_step_at(a, pg, f);
+        const int n = pg.bh * a.T + st.t;
+        float z[64];
+        {
+          const float* zr = st.Z + (size_t)row * D + h * 64;
+#pragma unroll
+          for (int cc = 0; cc < 64; cc += 4) {
+            const float4 v = __ldg((const float4*)(zr + cc));
+            z[cc] = v.x; z[cc + 1] = v.y; z[cc + 2] = v.z; z[cc + 3] = v.w;
+          }
+        }
+        mbar_wait(bar_pf, (uint32_t)(pidx++) & 1, abort_flag, &g_tc_status, 41);
+        tc_fence_after();
+        if (f + 1 < pg.n) fetch_y(chain_step_at(a, pg, f + 1).Y);  // Y buffer is free again
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + P_COL + h * 64 + c0, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc)
+            x[c0 + cc] = st.alpha * (x[c0 + cc] - __uint_as_float(r[cc])) + z[c0 + cc];
+        }
+        if (ridx > 0) mbar_wait(bar_rd, (uint32_t)(ridx - 1) & 1, abort_flag, &g_tc_status, 42);
+        write_x();  // S_f: readout B operand and the next step's A operand
+        if (pg.j0 + f == a.T - 1 && a.state_out)
+          store_row_f32(a.state_out + (size_t)pg.bh * DD + (size_t)row * D + h * 64, x);
+        // readout epilogue of frame f
+        for (int tl = 0; tl < ntile; ++tl, ++g) {
+          const int b = g & 1;
+          const uint32_t ub = (uint32_t)(g >> 1);
+          mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 43);
+          tc_fence_after();
+          const int tok = tl * TOK + row;
+          __nv_bfloat16* orow = out + ((size_t)n * S + tok) * D + h * 64;
+#pragma unroll
+          for (int c0 = 0; c0 < 64; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 128 + h * 64 + c0, r);
+            tmem_wait_ld();
+            if (tok < S) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                *(uint4*)(orow + c0 + 8 * j) = make_uint4(
+                    pack_bf16x2(__uint_as_float(r[8 * j]), __uint_as_float(r[8 * j + 1])),
+                    pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3])),
+                    pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5])),
+                    pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7])));
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(bar_acce + 8 * b);
+        }
+        ++ridx;
+      }
+    }
+    // drain: the last Y copy has landed (its chain MMA normally waited on it)
+    if (leader && fetched > 0)
+      mbar_wait(bar_yf, (uint32_t)(fetched - 1) & 1, abort_flag, &g_tc_status, 44);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+bool tc_scan_readout_supported(int D) { return D == 128; }
+
+cudaError_t tc_scan_readout(const ChainArgs& a, int nchains, const void* q, void* out, int S,
+                            cudaStream_t st) {
+  if (a.D != 128 || !a.y_image) return cudaErrorNotSupported;
+  CUtensorMap mq;
+  const long long N = (long long)a.heads * a.T;
+  cudaError_t e = make_map_bf16_3d(&mq, q, 128, S, N, 64, sro::TOK);
+  if (e != cudaSuccess) return e;
+  static bool attr = false;
+  if (!attr) {
+    e = cudaFuncSetAttribute(k_scan_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             sro::SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int grid = nchains < num_sms() ? nchains : num_sms();
+  k_scan_readout_tc<<<grid, sro::THREADS, sro::SMEM, st>>>(a, mq, (__nv_bfloat16*)out, S, nchains);
+  count_launch();
+  return cudaGetLastError();
+}
+
 bool tc_chain_supported(int D) { return D == 128; }
+
+// 3-D fp32 tensor of D x D matrices, box {32 columns, 128 rows}, 128-byte swizzle.
+static cudaError_t make_map_f32_mats(CUtensorMap* m, const void* base, uint64_t n) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t dims[3] = {128, 128, n};
+  cuuint64_t strides[2] = {128 * 4, 128 * 128 * 4};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
 
 cudaError_t tc_chain(const ChainArgs& a, int nchains, cudaStream_t st) {
   if (a.D != 128 || !a.y_image) return cudaErrorNotSupported;
+  if (a.mode == CHAIN_SCAN && !a.sfr_hilo) return cudaErrorNotSupported;
   static bool attr = false;
   if (!attr) {
     cudaError_t e =
@@ -1090,7 +1470,19 @@ cudaError_t tc_chain(const ChainArgs& a, int nchains, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  k_chain_tc<<<nchains, chn::THREADS, chn::SMEM, st>>>(a);
+  const long long frames = (long long)a.heads * a.T;
+  CUtensorMap mz, ms;
+  cudaError_t e;
+  if (a.mode == CHAIN_PREFIX)
+    e = make_map_f32_mats(&mz, a.Hc, (uint64_t)a.heads * a.nseg);
+  else
+    e = make_map_f32_mats(&mz, a.U, (uint64_t)frames);
+  if (e != cudaSuccess) return e;
+  // per-frame states: bf16 hi/lo pairs [2 * frames][128][128]
+  e = make_map_bf16_3d(&ms, a.mode == CHAIN_SCAN ? (const void*)a.Sfr : (const void*)a.U, 128, 128,
+                       2 * frames, 64, 128);
+  if (e != cudaSuccess) return e;
+  k_chain_tc<<<nchains, chn::THREADS, chn::SMEM, st>>>(a, mz, ms);
   count_launch();
   return cudaGetLastError();
 }

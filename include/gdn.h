@@ -80,6 +80,8 @@ enum {
 #define GDN_KEYS_SCALED 0x20u   /* k already carries 1/sqrt(D*S): do not scale again */
 #define GDN_FORCE_SIMT 0x40u    /* use the CUDA-core kernels even where tensor-core ones exist */
 #define GDN_BIDIR 0x80u         /* _ex only: forward scan -> out, reverse scan -> out_rev */
+#define GDN_FUSED_REPLAY 0x1000000u /* tensor-core path: replay each span inside the readout
+                                       kernel instead of storing S_t (spans/blocks, no prologue) */
 #define GDN_BLOCK(f) (((f) >> 8) & 0xffu)  /* reset block length; 0 means 3 */
 #define GDN_CHUNK(f) (((f) >> 16) & 0xffu) /* time-chunk length; 0 means 8 */
 #define GDN_MAKE_BLOCK(n) ((((unsigned)(n)) & 0xffu) << 8)
@@ -98,7 +100,8 @@ enum {
  *   state_out   [B,H,D,D]    fp32 state after the last frame in scan order
  *                            (frame T-1 forward, frame 0 reversed); NULL = not written
  *   flags       GDN_BF16 | GDN_REVERSE | GDN_BLOCK_RESET | GDN_SEQUENTIAL |
- *               GDN_KEYS_SCALED | GDN_FORCE_SIMT | GDN_MAKE_BLOCK(n) | GDN_MAKE_CHUNK(n)
+ *               GDN_KEYS_SCALED | GDN_FORCE_SIMT | GDN_FUSED_REPLAY |
+ *               GDN_MAKE_BLOCK(n) | GDN_MAKE_CHUNK(n)
  *
  * Blocks for GDN_BLOCK_RESET are floor(t / block) counted from t = 0 in both
  * directions. Without GDN_SEQUENTIAL the scan runs as time chunks composed
@@ -242,8 +245,8 @@ GDN_API int gdn_profile_enable(int enable);
 
 /* Sums the recorded kernel durations per phase, waiting on the events:
  * ms[i] and counts[i] for phase i < n, with phases 0 prologue, 1 contract,
- * 2 compose, 3 prefix, 4 scan/replay, 5 readout. Returns the number of
- * phases written, or a negative status. */
+ * 2 compose, 3 prefix, 4 scan/replay, 5 readout, 6 replay fused with the
+ * readout. Returns the number of phases written, or a negative status. */
 GDN_API int gdn_profile_read(double* ms, long long* counts, int n);
 
 /* ABI version: major * 10000 + minor * 100 + patch. */

@@ -101,6 +101,8 @@ MODES = {
     "reverse_block": dict(reverse=True, block_reset=True),
     "forward_block": dict(block_reset=True, block=4),
     "reverse_block_seq": dict(reverse=True, block_reset=True, sequential=True),
+    "fused_replay": dict(fused_replay=True),
+    "fused_replay_rev_block": dict(fused_replay=True, reverse=True, block_reset=True),
 }
 
 
@@ -232,6 +234,7 @@ def test_fused_prologue_bidirectional(D, path):
 
 FULL = [
     ("clip5s_720p", {}),
+    ("clip5s_720p", {"fused_replay": True}),
     ("rollout60s_720p", {}),
     ("rollout60s_720p", {"sequential": True}),
     ("prologue_bidir_720p", {}),
@@ -240,7 +243,7 @@ FULL = [
 ]
 
 
-@pytest.mark.parametrize("name,kw", FULL, ids=[f"{n}{'-seq' if k else ''}" for n, k in FULL])
+@pytest.mark.parametrize("name,kw", FULL, ids=[n + "".join("-" + k for k in kw) for n, kw in FULL])
 def test_full_size_sampled(name, kw):
     cfg = synth.CONFIGS[name]
     arr = synth.make_inputs(cfg)
