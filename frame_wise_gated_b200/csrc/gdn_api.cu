@@ -189,6 +189,7 @@ static int run_direction(const gdn_params& p, const Layout& L, char* ws, bool re
   a.Sst = (float*)(ws + L.Sst);
   a.y_image = use_tc_chain ? 1 : 0;  // the tensor-core chains read A and E as operand images
   a.e_image = a.y_image;
+  a.sst_hilo = a.y_image;
 
   auto chain = [&](const ChainArgs& c, int n) -> cudaError_t {
     PhaseScope ps(c.mode == CHAIN_COMPOSE ? PH_COMPOSE : c.mode == CHAIN_PREFIX ? PH_PREFIX : PH_SCAN,

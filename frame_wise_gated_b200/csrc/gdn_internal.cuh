@@ -66,6 +66,7 @@ struct ChainArgs {
   float* Sst;             // [heads*nseg, D, D] span start states
   int y_image;            // A (and E for the prefix) are stored as bf16 operand images
   int e_image;            // the compose chain writes E as an operand image
+  int sst_hilo;           // Sst holds [heads*nseg][2][D][D] bf16 (hi, lo) pairs
 };
 
 // An "operand image" of a D x D fp32 matrix M (D = 128) is the exact

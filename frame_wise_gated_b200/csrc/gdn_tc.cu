@@ -760,6 +760,7 @@ struct ChainStep {
 struct ChainProg {
   int mode, which, bh, p, j0, n;
   const float* init;
+  int init_hilo;  // init points at a bf16 (hi, lo) pair
 };
 
 __device__ __forceinline__ ChainProg chain_prog(const ChainArgs& a, int c) {
@@ -767,6 +768,7 @@ __device__ __forceinline__ ChainProg chain_prog(const ChainArgs& a, int c) {
   g.mode = a.mode;
   g.which = 0;
   g.init = nullptr;
+  g.init_hilo = 0;
   if (a.mode == CHAIN_SCAN) {
     g.bh = c / a.nseg;
     g.p = c % a.nseg;
@@ -776,8 +778,10 @@ __device__ __forceinline__ ChainProg chain_prog(const ChainArgs& a, int c) {
     g.n = j1 - j0;
     if (g.p == 0)
       g.init = a.state_in ? a.state_in + (size_t)g.bh * a.D * a.D : nullptr;
-    else if (a.seg == SEG_CHUNKS)
+    else if (a.seg == SEG_CHUNKS) {
       g.init = a.Sst + ((size_t)g.bh * a.nseg + g.p) * a.D * a.D;
+      g.init_hilo = a.sst_hilo;
+    }
   } else if (a.mode == CHAIN_COMPOSE) {
     const int half = a.heads * a.nseg;
     g.which = c >= half;
@@ -873,6 +877,39 @@ __device__ __forceinline__ void chain_store_x(const float* x, uint8_t* xh, uint8
   }
 }
 
+// 64 values of row `row`, columns 64h.., of an initial state: fp32, or a bf16
+// (hi, lo) pair whose hi matrix starts at `init` (lo follows D*D values later).
+__device__ __forceinline__ void load_init_slice(const float* init, int hilo, int row, int h,
+                                                float* x) {
+  constexpr int D = chn::D;
+  if (!init) {
+#pragma unroll
+    for (int c = 0; c < 64; ++c) x[c] = 0.f;
+  } else if (hilo) {
+    const __nv_bfloat16* hi = (const __nv_bfloat16*)init + (size_t)row * D + h * 64;
+    const __nv_bfloat16* lo = hi + (size_t)D * D;
+#pragma unroll
+    for (int c = 0; c < 64; c += 8) {
+      const uint4 a4 = __ldg((const uint4*)(hi + c)), b4 = __ldg((const uint4*)(lo + c));
+      const uint32_t aw[4] = {a4.x, a4.y, a4.z, a4.w}, bw[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&aw[e]));
+        const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bw[e]));
+        x[c + 2 * e] = fa.x + fb.x;
+        x[c + 2 * e + 1] = fa.y + fb.y;
+      }
+    }
+  } else {
+    const float* src = init + (size_t)row * D + h * 64;
+#pragma unroll
+    for (int c = 0; c < 64; c += 4) {
+      const float4 f = __ldg((const float4*)(src + c));
+      x[c] = f.x; x[c + 1] = f.y; x[c + 2] = f.z; x[c + 3] = f.w;
+    }
+  }
+}
+
 __device__ __forceinline__ void store_row_f32(float* dst, const float* x) {
 #pragma unroll
   for (int c = 0; c < 64; c += 4) *(float4*)(dst + c) = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
@@ -948,24 +985,26 @@ __global__ void __launch_bounds__(chn::THREADS, 1)
   }
 
   float x[64];
-  if (g.init) {
-    const float* src = g.init + (size_t)row * D + h * 64;
-#pragma unroll
-    for (int c = 0; c < 64; c += 4) {
-      const float4 f = __ldg((const float4*)(src + c));
-      x[c] = f.x; x[c + 1] = f.y; x[c + 2] = f.z; x[c + 3] = f.w;
-    }
-  } else {
-#pragma unroll
-    for (int c = 0; c < 64; ++c) x[c] = 0.f;
-  }
+  load_init_slice(g.init, g.init_hilo, row, h, x);
   float gprod = 1.f;
-  int tprev = -1;  // frame whose state sits in the X tile, to be stored
+  // Tile states to store (hi/lo pairs, by TMA): a scan stores each frame's
+  // state (the tile at step s holds the state after frame t_{s-1}); the prefix
+  // stores each span's start state (the tile at step s holds S_start(s)).
+  const bool store_sst = g.mode == CHAIN_PREFIX && a.sst_hilo;
+  int tprev = -1;
+  auto store_tile = [&](int pair) {
+    tma_store_3d(&tmSfr, sb + OFF_XH, 0, 0, 2 * pair);
+    tma_store_3d(&tmSfr, sb + OFF_XH + ATOM, 64, 0, 2 * pair);
+    tma_store_3d(&tmSfr, sb + OFF_XL, 0, 0, 2 * pair + 1);
+    tma_store_3d(&tmSfr, sb + OFF_XL + ATOM, 64, 0, 2 * pair + 1);
+    bulk_commit();
+    ++nstore;
+  };
 
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, true);
   for (int s = 0; s < g.n; ++s) {
     const ChainStep st = chain_step_at(a, g, s);
-    if (g.mode == CHAIN_PREFIX)
+    if (g.mode == CHAIN_PREFIX && !store_sst)
       store_row_f32(a.Sst + ((size_t)g.bh * a.nseg + s) * DD + (size_t)row * D + h * 64, x);
     // A reset (zero state entering this step) is applied in the update below
     // (x <- Z), so the tile still carries the previous frame's state to store.
@@ -996,16 +1035,8 @@ __global__ void __launch_bounds__(chn::THREADS, 1)
     __syncthreads();
     if (*abort_flag) break;  // uniform: read after the barrier
     if (leader) {
-      if (store_sfr && tprev >= 0) {
-        // the tile holds S of frame tprev: store its hi/lo pair for the readout
-        const int zz = 2 * (g.bh * a.T + tprev);
-        tma_store_3d(&tmSfr, sb + OFF_XH, 0, 0, zz);
-        tma_store_3d(&tmSfr, sb + OFF_XH + ATOM, 64, 0, zz);
-        tma_store_3d(&tmSfr, sb + OFF_XL, 0, 0, zz + 1);
-        tma_store_3d(&tmSfr, sb + OFF_XL + ATOM, 64, 0, zz + 1);
-        bulk_commit();
-        ++nstore;
-      }
+      if (store_sfr && tprev >= 0) store_tile(g.bh * a.T + tprev);  // S after frame tprev
+      if (store_sst) store_tile(g.bh * a.nseg + s);                  // S_start(s)
       tc_fence_after();
       const uint32_t yh = sb + OFF_Y, yl = yh + 2 * ATOM;
 #pragma unroll
@@ -1065,8 +1096,9 @@ __global__ void __launch_bounds__(chn::THREADS, 1)
         store_row_f32(a.state_out + (size_t)g.bh * DD + (size_t)row * D + h * 64, x);
     }
   }
-  // the last state of a scan chain: through the X tile to its hi/lo store
-  if (store_sfr && tprev >= 0) {
+  // the last state of a scan chain (or the last span start of the prefix):
+  // through the X tile to its hi/lo store
+  if ((store_sfr && tprev >= 0) || store_sst) {
     if (leader && nstore > 0) bulk_wait_read0();
     __syncthreads();
     if (!*abort_flag) {
@@ -1074,15 +1106,7 @@ __global__ void __launch_bounds__(chn::THREADS, 1)
       fence_proxy_async();
     }
     __syncthreads();
-    if (leader && !*abort_flag) {
-      const int zz = 2 * (g.bh * a.T + tprev);
-      tma_store_3d(&tmSfr, sb + OFF_XH, 0, 0, zz);
-      tma_store_3d(&tmSfr, sb + OFF_XH + ATOM, 64, 0, zz);
-      tma_store_3d(&tmSfr, sb + OFF_XL, 0, 0, zz + 1);
-      tma_store_3d(&tmSfr, sb + OFF_XL + ATOM, 64, 0, zz + 1);
-      bulk_commit();
-      ++nstore;
-    }
+    if (leader && !*abort_flag) store_tile(store_sst ? g.bh * a.nseg + g.n : g.bh * a.T + tprev);
   }
   __syncthreads();
   if (!*abort_flag) {
@@ -1095,7 +1119,7 @@ __global__ void __launch_bounds__(chn::THREADS, 1)
       else
         store_row_f32(a.E + si * DD + (size_t)row * D + h * 64, x);
       if (!g.which && threadIdx.x == 0) a.g[si] = gprod;
-    } else if (g.mode == CHAIN_PREFIX) {
+    } else if (g.mode == CHAIN_PREFIX && !store_sst) {
       store_row_f32(a.Sst + ((size_t)g.bh * a.nseg + g.n) * DD + (size_t)row * D + h * 64, x);
     }
   }
@@ -1339,17 +1363,7 @@ __global__ void __launch_bounds__(sro::THREADS, 1)
       if (*abort_flag) break;
       // the previous readout (if any) has drained the tile
       if (ridx > 0) mbar_wait(bar_rd, (uint32_t)(ridx - 1) & 1, abort_flag, &g_tc_status, 40);
-      if (pg.init) {
-        const float* src = pg.init + (size_t)row * D + h * 64;
-#pragma unroll
-        for (int cc = 0; cc < 64; cc += 4) {
-          const float4 v = __ldg((const float4*)(src + cc));
-          x[cc] = v.x; x[cc + 1] = v.y; x[cc + 2] = v.z; x[cc + 3] = v.w;
-        }
-      } else {
-#pragma unroll
-        for (int cc = 0; cc < 64; ++cc) x[cc] = 0.f;
-      }
+      load_init_slice(pg.init, pg.init_hilo, row, h, x);
       fetch_y(chain_step_at(a, pg, 0).Y);
       write_x();
       for (int f = 0; f < pg.n; ++f) {
@@ -1478,9 +1492,12 @@ cudaError_t tc_chain(const ChainArgs& a, int nchains, cudaStream_t st) {
   else
     e = make_map_f32_mats(&mz, a.U, (uint64_t)frames);
   if (e != cudaSuccess) return e;
-  // per-frame states: bf16 hi/lo pairs [2 * frames][128][128]
-  e = make_map_bf16_3d(&ms, a.mode == CHAIN_SCAN ? (const void*)a.Sfr : (const void*)a.U, 128, 128,
-                       2 * frames, 64, 128);
+  // stored tile states, bf16 hi/lo pairs: per frame (scan) or per span (prefix)
+  if (a.mode == CHAIN_PREFIX && a.sst_hilo)
+    e = make_map_bf16_3d(&ms, a.Sst, 128, 128, 2 * (uint64_t)a.heads * a.nseg, 64, 128);
+  else
+    e = make_map_bf16_3d(&ms, a.mode == CHAIN_SCAN ? (const void*)a.Sfr : (const void*)a.U, 128,
+                         128, 2 * frames, 64, 128);
   if (e != cudaSuccess) return e;
   k_chain_tc<<<nchains, chn::THREADS, chn::SMEM, st>>>(a, mz, ms);
   count_launch();
