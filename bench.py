@@ -231,6 +231,22 @@ def run_reference(args, cfg):
     return 0
 
 
+def reduce_step_time(ms, dist=None, device=None):
+    """Max over ranks of a per-rank elapsed time (ms); identity on one rank."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(ms)
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(tokens_per_rank, world, ms_per_step):
+    """Whole-job throughput: the units all ranks processed / the slowest rank's time."""
+    return tokens_per_rank * world / (ms_per_step * 1e-3)
+
+
 def run_ours(args, cfg):
     import torch
     from frame_wise_gated_b200 import api, build
@@ -316,14 +332,9 @@ def run_ours(args, cfg):
     api.profile_enable(False)
     clk = clocks.stop()
     api.check_device_status()
-    ms = ev0.elapsed_time(ev1)
-    if dist is not None:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_step_time(ev0.elapsed_time(ev1), dist, dev)
     ms_step = ms / args.steps
-    tokens_all = cfg.tokens * world
-    value = tokens_all / (ms_step * 1e-3)
+    value = whole_job_value(cfg.tokens, world, ms_step)
 
     # ---- dominant kernel roofline (live per-kernel events over the timed region) ----
     hbm, bf16_tf, peak_kind = peaks()
@@ -428,13 +439,9 @@ def run_e2e(args, cfg, arr, dev, api, barrier, dist, world):
     ev1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    ms = ev0.elapsed_time(ev1)
-    if dist is not None:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_step_time(ev0.elapsed_time(ev1), dist, dev)
     ms_step = ms / args.e2e_steps
-    return {"value": cfg.tokens * world / (ms_step * 1e-3), "unit": UNIT,
+    return {"value": whole_job_value(cfg.tokens, world, ms_step), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_step,
             "steps": args.e2e_steps, "entry": "gdn_frame_scan_fwd (host buffers, pinned)"}
 

@@ -78,6 +78,7 @@ SIGNATURES = {
     "gdn_frame_contract": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _U, _P]),
     "gdn_chunk_composites": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _U, _P]),
     "gdn_check_device_status": (_I, [_P]),
+    "gdn_selftest_wait": (_I, [_I, ctypes.c_longlong, _P]),
     "gdn_status_string": (ctypes.c_char_p, [_I]),
     "gdn_last_error": (ctypes.c_char_p, []),
     "gdn_launch_count": (ctypes.c_longlong, [_I]),
@@ -329,3 +330,9 @@ def profile_read() -> dict:
     if r < 0:
         _check(r, "gdn_profile_read")
     return {PHASES[i]: (ms[i], cnt[i]) for i in range(r)}
+
+
+def selftest_wait(arrive: bool, limit_ns: int = 1_000_000, stream=None) -> None:
+    """Launches the bounded-wait self test (see gdn_selftest_wait)."""
+    _check(lib().gdn_selftest_wait(1 if arrive else 0, int(limit_ns), _stream(stream)),
+           "gdn_selftest_wait")

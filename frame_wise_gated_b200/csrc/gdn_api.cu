@@ -560,6 +560,15 @@ int gdn_profile_read(double* ms, long long* counts, int n) {
   return np;
 }
 
+int gdn_selftest_wait(int arrive, long long limit_ns, gdn_stream_t stream) {
+  t_last_error.clear();
+  if (limit_ns < 0 || limit_ns > 1000000000LL)
+    return fail(GDN_ERR_INVALID, "limit_ns must be in [0, 1e9]%s");
+  cudaError_t e = tc_selftest_wait(arrive, limit_ns, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+  return GDN_OK;
+}
+
 int gdn_check_device_status(gdn_stream_t stream) {
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = cudaStreamSynchronize(st);

@@ -158,6 +158,7 @@ cudaError_t tc_scan_readout(const ChainArgs& a, int nchains, const void* q, void
                             cudaStream_t st);
 bool tc_chain_supported(int D);
 cudaError_t tc_chain(const ChainArgs& a, int nchains, cudaStream_t st);
+cudaError_t tc_selftest_wait(int arrive, long long limit_ns, cudaStream_t st);
 // Reads and clears the device status word of the tensor-core kernels.
 cudaError_t tc_read_status(int* status, cudaStream_t st);
 

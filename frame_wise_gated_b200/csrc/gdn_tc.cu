@@ -1504,6 +1504,30 @@ cudaError_t tc_chain(const ChainArgs& a, int nchains, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// Failure-path self test: one block waits (bounded by limit_ns) on an mbarrier
+// that completes only if `arrive`; a wait that runs out is recorded in the
+// status word with code 99 and the kernel returns normally.
+__global__ void k_selftest_wait(int arrive, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (arrive && threadIdx.x == 0) mbar_arrive(b);
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_limit(b, 0, &abort_flag, &g_tc_status, 99, limit_ns);
+}
+
+cudaError_t tc_selftest_wait(int arrive, long long limit_ns, cudaStream_t st) {
+  k_selftest_wait<<<1, 32, 0, st>>>(arrive, (unsigned long long)limit_ns);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t tc_read_status(int* status, cudaStream_t st) {
   int zero = 0;
   cudaError_t e = cudaMemcpyFromSymbolAsync(status, g_tc_status, sizeof(int), 0,

@@ -227,6 +227,14 @@ GDN_API int gdn_chunk_composites(const float* A, const float* U, const float* ga
  * last check, or GDN_ERR_CUDA if the stream reports an error. */
 GDN_API int gdn_check_device_status(gdn_stream_t stream);
 
+/* gdn_selftest_wait — exercises the device-side failure path without any
+ * fault: one block waits on an mbarrier that is completed only when `arrive`
+ * is non-zero, bounded by limit_ns nanoseconds (at most 1e9). When the wait
+ * runs out the kernel records the timeout in the library's status word and
+ * returns normally, so the next gdn_check_device_status reports
+ * GDN_ERR_TIMEOUT and the context stays usable. Returns the launch status. */
+GDN_API int gdn_selftest_wait(int arrive, long long limit_ns, gdn_stream_t stream);
+
 /* Static description of a status code. */
 GDN_API const char* gdn_status_string(int status);
 
