@@ -309,7 +309,7 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
     const float eps = p.eps > 0.f ? p.eps : 1e-6f;
     const float base = p.rope_base > 0.f ? p.rope_base : 10000.f;
     const int npos_max = p.grid_h > p.grid_w ? p.grid_h : p.grid_w;
-    if (tc_contract_ok && tc_readout_ok && npos_max <= tc_prologue_max_positions()) {
+    if (tc_contract_ok && tc_readout_ok && p.D == 128 && npos_max <= tc_prologue_max_positions()) {
       // Fused: the tensor-core loaders apply RMSNorm, ReLU and RoPE to the raw
       // tiles in shared memory; the key scale goes into the contraction's
       // epilogue constants (RoPE is linear, so the order does not matter).
@@ -515,9 +515,9 @@ int gdn_chunk_composites(const float* A, const float* U, const float* gamma, flo
   if (tc) {
     // The tensor-core chains read A as operand images: convert into scratch.
     void* img = nullptr;
-    e = cudaMallocAsync(&img, (size_t)N * L * kImageBytes, st);
+    e = cudaMallocAsync(&img, (size_t)N * L * D * D * 4, st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(images)");
-    e = tc_to_image(A, img, (long long)N * L, st);
+    e = tc_to_image(A, img, (long long)N * L, D, st);
     if (e == cudaSuccess) {
       a.A = (const float*)img;
       a.y_image = 1;

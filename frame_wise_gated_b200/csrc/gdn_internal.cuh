@@ -147,8 +147,8 @@ bool tc_contract_supported(int D);
 cudaError_t tc_contract(const void* k, const void* v, const float* beta, float* A, float* U,
                         long long N, int S, int D, float cA, float cU, int a_image,
                         const ProArgs* pro, cudaStream_t st);
-// fp32 D x D matrices -> operand images (D = 128).
-cudaError_t tc_to_image(const float* src, void* dst, long long n, cudaStream_t st);
+// fp32 D x D matrices -> operand images (D = 64 or 128).
+cudaError_t tc_to_image(const float* src, void* dst, long long n, int D, cudaStream_t st);
 bool tc_readout_supported(int D);
 cudaError_t tc_readout(const void* q, const void* Sfr_hilo, void* out, long long N, int S, int D,
                        const ProArgs* pro, cudaStream_t st);

@@ -424,12 +424,12 @@ __global__ void __launch_bounds__(ctr::THREADS, 1)
   }
 }
 
-bool tc_contract_supported(int D) { return D == 128; }
+bool tc_contract_supported(int D) { return D == 128 || D == 64; }
 int tc_prologue_max_positions() { return ctr::TAB_MAX / 32; }
 
-cudaError_t tc_contract(const void* k, const void* v, const float* beta, float* A, float* U,
-                        long long N, int S, int D, float cA, float cU, int a_image,
-                        const ProArgs* pro, cudaStream_t st) {
+static cudaError_t tc_contract128(const void* k, const void* v, const float* beta, float* A,
+                                  float* U, long long N, int S, int D, float cA, float cU,
+                                  int a_image, const ProArgs* pro, cudaStream_t st) {
   if (D != 128) return cudaErrorNotSupported;
   if (pro && pro->npos * (D / 4) > ctr::TAB_MAX) return cudaErrorNotSupported;
   ProArgs pa = {};
@@ -682,7 +682,7 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
   }
 }
 
-bool tc_readout_supported(int D) { return D == 128; }
+bool tc_readout_supported(int D) { return D == 128 || D == 64; }
 
 template <bool PRO>
 static cudaError_t launch_readout(const CUtensorMap& mq, const CUtensorMap& ms, const CUtensorMap& mo,
@@ -700,8 +700,8 @@ static cudaError_t launch_readout(const CUtensorMap& mq, const CUtensorMap& ms, 
   return cudaGetLastError();
 }
 
-cudaError_t tc_readout(const void* q, const void* Sfr_hilo, void* out, long long N, int S, int D,
-                       const ProArgs* pro, cudaStream_t st) {
+static cudaError_t tc_readout128(const void* q, const void* Sfr_hilo, void* out, long long N,
+                                 int S, int D, const ProArgs* pro, cudaStream_t st) {
   if (D != 128) return cudaErrorNotSupported;
   if (pro && pro->npos * (D / 4) > rdo::TAB_MAX) return cudaErrorNotSupported;
   CUtensorMap mq, ms, mo;
@@ -1138,21 +1138,25 @@ __global__ void __launch_bounds__(chn::THREADS, 1)
 }
 
 // fp32 matrix -> operand image; one CTA of 256 threads per matrix.
-__global__ void __launch_bounds__(256) k_to_image(const float* __restrict__ src, uint8_t* __restrict__ dst) {
-  const float* m = src + (size_t)blockIdx.x * 128 * 128;
-  uint8_t* img = dst + (size_t)blockIdx.x * kImageBytes;
-  for (int cid = threadIdx.x; cid < 128 * 16; cid += 256) {
-    const int k = cid >> 4, nc = cid & 15;
+// An image of a D x D matrix (D = 64 or 128): hi = D/64 blocks of
+// [D rows][128 B] (block b holds columns 64b..64b+63), then lo likewise.
+__global__ void __launch_bounds__(256) k_to_image(const float* __restrict__ src, uint8_t* __restrict__ dst,
+                                                  int D) {
+  const float* m = src + (size_t)blockIdx.x * D * D;
+  uint8_t* img = dst + (size_t)blockIdx.x * D * D * 4;
+  const int cpr = D / 8;  // 16-byte chunks per row
+  for (int cid = threadIdx.x; cid < D * cpr; cid += 256) {
+    const int k = cid / cpr, nc = cid % cpr;
     float v[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = m[k * 128 + nc * 8 + e];
-    split_chunk(v, (uint4*)(img + tile_off(k, nc >> 3, nc & 7)),
-                (uint4*)(img + 2 * chn::ATOM + tile_off(k, nc >> 3, nc & 7)));
+    for (int e = 0; e < 8; ++e) v[e] = m[k * D + nc * 8 + e];
+    const int off = (nc >> 3) * D * 128 + k * 128 + (((nc & 7) ^ (k & 7)) << 4);
+    split_chunk(v, (uint4*)(img + off), (uint4*)(img + D * D * 2 + off));
   }
 }
 
-cudaError_t tc_to_image(const float* src, void* dst, long long n, cudaStream_t st) {
-  k_to_image<<<(unsigned)n, 256, 0, st>>>(src, (uint8_t*)dst);
+cudaError_t tc_to_image(const float* src, void* dst, long long n, int D, cudaStream_t st) {
+  k_to_image<<<(unsigned)n, 256, 0, st>>>(src, (uint8_t*)dst, D);
   count_launch();
   return cudaGetLastError();
 }
@@ -1458,7 +1462,7 @@ cudaError_t tc_scan_readout(const ChainArgs& a, int nchains, const void* q, void
   return cudaGetLastError();
 }
 
-bool tc_chain_supported(int D) { return D == 128; }
+bool tc_chain_supported(int D) { return D == 128 || D == 64; }
 
 // 3-D fp32 tensor of D x D matrices, box {32 columns, 128 rows}, 128-byte swizzle.
 static cudaError_t make_map_f32_mats(CUtensorMap* m, const void* base, uint64_t n) {
@@ -1474,7 +1478,7 @@ static cudaError_t make_map_f32_mats(CUtensorMap* m, const void* base, uint64_t 
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t tc_chain(const ChainArgs& a, int nchains, cudaStream_t st) {
+static cudaError_t tc_chain128(const ChainArgs& a, int nchains, cudaStream_t st) {
   if (a.D != 128 || !a.y_image) return cudaErrorNotSupported;
   if (a.mode == CHAIN_SCAN && !a.sfr_hilo) return cudaErrorNotSupported;
   static bool attr = false;
@@ -1502,6 +1506,740 @@ cudaError_t tc_chain(const ChainArgs& a, int nchains, cudaStream_t st) {
   k_chain_tc<<<nchains, chn::THREADS, chn::SMEM, st>>>(a, mz, ms);
   count_launch();
   return cudaGetLastError();
+}
+
+// ============================================================================
+// D = 64 tensor-core kernels.
+//
+// Contraction: [K^T; V^T] is one M = 128 MN-major operand (the K and V boxes
+// of a stage sit next to each other, LBO = one box) against beta*K (N = 64),
+// so one 128x64x16 MMA per 16 tokens yields [A_t; U_t] in TMEM rows 0-63 /
+// 64-127. Readout: M = 128 tokens, N = 64, one 128-byte swizzle atom wide.
+// Chains: the state is 64 x 64; a span's E and H chains share Y = A_t and run
+// stacked in one CTA (E in rows 0-63, H in rows 64-127); a scan or prefix chain
+// uses rows 0-63 only. Operand images for D = 64: hi [64 rows][128 B] then lo.
+// ============================================================================
+namespace c64 {
+constexpr int D = 64;
+constexpr int TOK = 64;
+constexpr int NST = 6;
+constexpr int BOX = TOK * 128;        // [64 tokens][64 channels] bf16: 8 KiB
+constexpr int KV = 2 * BOX;           // K box, then V box: the stacked A operand
+constexpr int OFF_KV = 0;
+constexpr int OFF_BK = OFF_KV + NST * KV;
+constexpr int OFF_BETA = OFF_BK + NST * BOX;
+constexpr int OFF_BAR = OFF_BETA + NST * TOK * 4;
+constexpr int NBAR = 3 * NST + 5;
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+constexpr int NSC = 128;
+constexpr int THREADS = 64 + NSC + 128;
+constexpr uint32_t TMEM_COLS = 128;
+constexpr int IMG = D * D * 4;        // operand image bytes
+}  // namespace c64
+
+__global__ void __launch_bounds__(c64::THREADS, 1)
+    k_contract64_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const float* __restrict__ beta, float* __restrict__ A, float* __restrict__ U,
+                    int N, int S, float cA, float cU, int a_image) {
+  using namespace c64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar_full = sb + OFF_BAR;
+  const uint32_t bar_bk = bar_full + 8 * NST;
+  const uint32_t bar_empty = bar_bk + 8 * NST;
+  const uint32_t bar_accf = bar_empty + 8 * NST;
+  const uint32_t bar_acce = bar_accf + 16;
+  const uint32_t bar_fin = bar_acce + 16;
+  uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bar_full + 8 * s, 33);
+      mbar_init(bar_bk + 8 * s, NSC);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_accf + 8 * b, 1);
+      mbar_init(bar_acce + 8 * b, 128);
+    }
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int nst_frame = (S + TOK - 1) / TOK;
+  const int my_count = (int)blockIdx.x < N ? (N - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+  if (warp == 0) {
+    int g = 0;
+    bool ok = true;
+    for (int i = 0; i < my_count && ok; ++i) {
+      const int n = blockIdx.x + i * gridDim.x;
+      for (int st = 0; st < nst_frame; ++st, ++g) {
+        const int s = g % NST;
+        const uint32_t u = (uint32_t)(g / NST);
+        if (lane == 0) ok = mbar_wait(bar_empty + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 51);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane == 0) {
+          const uint32_t kd = sb + OFF_KV + s * KV;
+          mbar_arrive_expect_tx(bar_full + 8 * s, KV);
+          tma_load_3d(kd, &tmK, bar_full + 8 * s, 0, st * TOK, n);
+          tma_load_3d(kd + BOX, &tmV, bar_full + 8 * s, 0, st * TOK, n);
+        }
+        const uint32_t bsa = sb + OFF_BETA + s * TOK * 4;
+#pragma unroll
+        for (int r = lane; r < TOK; r += 32) {
+          const int tok = st * TOK + r;
+          const bool in = tok < S;
+          cp_async_4(bsa + r * 4, beta + (size_t)n * S + (in ? tok : 0), in ? 4u : 0u);
+        }
+        cp_async_arrive_noinc(bar_full + 8 * s);
+      }
+    }
+    if (lane == 0) {
+      for (int gg = (g > NST ? g - NST : 0); gg < g; ++gg)
+        mbar_wait(bar_full + 8 * (gg % NST), (uint32_t)(gg / NST) & 1, abort_flag, &g_tc_status, 52);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 64, true, true);
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; i < my_count && ok; ++i) {
+        const int b = i & 1;
+        const uint32_t ub = (uint32_t)(i >> 1);
+        ok = mbar_wait(bar_acce + 8 * b, (ub & 1) ^ 1, abort_flag, &g_tc_status, 53);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t d = tmem + b * 64;
+        for (int st = 0; st < nst_frame; ++st, ++g) {
+          const int s = g % NST;
+          const uint32_t u = (uint32_t)(g / NST);
+          ok = mbar_wait(bar_bk + 8 * s, u & 1, abort_flag, &g_tc_status, 54);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t kva = sb + OFF_KV + s * KV, ba = sb + OFF_BK + s * BOX;
+#pragma unroll
+          for (int kk = 0; kk < TOK / 16; ++kk) {
+            const uint64_t da = smem_desc_sw128(kva + kk * 2048, BOX, 1024);  // [K^T; V^T]
+            const uint64_t db = smem_desc_sw128(ba + kk * 2048, BOX, 1024);
+            mma_bf16(d, da, db, idesc, (st > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(bar_empty + 8 * s);
+        }
+        if (!ok) break;
+        mma_commit(bar_accf + 8 * b);
+      }
+      mma_commit(bar_fin);
+      mbar_wait(bar_fin, 0, abort_flag, &g_tc_status, 55);
+    }
+    __syncwarp();
+  } else if (warp < 2 + NSC / 32) {
+    const int t = threadIdx.x - 64;
+    int g = 0;
+    bool ok = true;
+    for (int i = 0; i < my_count && ok; ++i) {
+      for (int st = 0; st < nst_frame; ++st, ++g) {
+        const int s = g % NST;
+        const uint32_t u = (uint32_t)(g / NST);
+        ok = mbar_wait(bar_full + 8 * s, u & 1, abort_flag, &g_tc_status, 56);
+        if (!ok) break;
+        const uint8_t* kt = smem + OFF_KV + s * KV;
+        uint8_t* bt = smem + OFF_BK + s * BOX;
+        const float* bs = (const float*)(smem + OFF_BETA) + s * TOK;
+#pragma unroll
+        for (int m = 0; m < (BOX / 16) / NSC; ++m) {
+          const int c = t + NSC * m;
+          const float bv = bs[c >> 3];
+          uint4 x = *(const uint4*)(kt + c * 16);
+          uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
+            w[e] = pack_bf16x2(f.x * bv, f.y * bv);
+          }
+          *(uint4*)(bt + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async();
+        mbar_arrive(bar_bk + 8 * s);
+      }
+    }
+  } else {
+    // TMEM rows 0-63 hold A_t, rows 64-127 U_t
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const bool isA = row < 64;
+    const int r = isA ? row : row - 64;
+    for (int i = 0; i < my_count; ++i) {
+      const int b = i & 1;
+      const uint32_t ub = (uint32_t)(i >> 1);
+      if (!mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 57)) break;
+      tc_fence_after();
+      const int n = blockIdx.x + i * gridDim.x;
+      const float sc = isA ? cA : cU;
+#pragma unroll
+      for (int c0 = 0; c0 < 64; c0 += 32) {
+        uint32_t rr[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 64 + c0, rr);
+        tmem_wait_ld();
+        if (isA && a_image) {
+          uint8_t* img = (uint8_t*)A + (size_t)n * IMG;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(rr[8 * j + e]) * sc;
+            const int off = r * 128 + ((((c0 >> 3) + j) ^ (r & 7)) << 4);
+            split_chunk(v, (uint4*)(img + off), (uint4*)(img + D * D * 2 + off));
+          }
+        } else {
+          float* dst = (isA ? A : U) + ((size_t)n * D + r) * D + c0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *(float4*)(dst + 4 * j) =
+                make_float4(__uint_as_float(rr[4 * j]) * sc, __uint_as_float(rr[4 * j + 1]) * sc,
+                            __uint_as_float(rr[4 * j + 2]) * sc, __uint_as_float(rr[4 * j + 3]) * sc);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_acce + 8 * b);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+namespace r64 {
+constexpr int D = 64;
+constexpr int TOK = 128;
+constexpr int NQ = 4;
+constexpr int QBOX = TOK * 128;          // [128 tokens][64 channels] bf16: 16 KiB
+constexpr int SBOX = 64 * 128;           // [64 rows][64] bf16: 8 KiB
+constexpr int OFF_Q = 0;
+constexpr int OFF_S = OFF_Q + NQ * QBOX; // S hi, then S lo
+constexpr int OFF_O = OFF_S + 2 * SBOX;  // output staging: one box
+constexpr int OFF_BAR = OFF_O + QBOX;
+constexpr int NBAR = 2 * NQ + 2 + 4 + 1;
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 128;
+}  // namespace r64
+
+__global__ void __launch_bounds__(r64::THREADS, 1)
+    k_readout64_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
+                   const __grid_constant__ CUtensorMap tmO, int N, int S) {
+  using namespace r64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar_qf = sb + OFF_BAR;
+  const uint32_t bar_qe = bar_qf + 8 * NQ;
+  const uint32_t bar_sf = bar_qe + 8 * NQ;
+  const uint32_t bar_se = bar_sf + 8;
+  const uint32_t bar_accf = bar_se + 8;
+  const uint32_t bar_acce = bar_accf + 16;
+  const uint32_t bar_fin = bar_acce + 16;
+  uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NQ; ++s) {
+      mbar_init(bar_qf + 8 * s, 1);
+      mbar_init(bar_qe + 8 * s, 1);
+    }
+    mbar_init(bar_sf, 1);
+    mbar_init(bar_se, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_accf + 8 * b, 1);
+      mbar_init(bar_acce + 8 * b, 128);
+    }
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int ntile = (S + TOK - 1) / TOK;
+  const int my_count = (int)blockIdx.x < N ? (N - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; i < my_count && ok; ++i) {
+        const int n = blockIdx.x + i * gridDim.x;
+        ok = mbar_wait(bar_se, ((uint32_t)i & 1) ^ 1, abort_flag, &g_tc_status, 61);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar_sf, 2 * SBOX);
+        tma_load_3d(sb + OFF_S, &tmS, bar_sf, 0, 0, 2 * n);
+        tma_load_3d(sb + OFF_S + SBOX, &tmS, bar_sf, 0, 0, 2 * n + 1);
+        for (int tl = 0; tl < ntile; ++tl, ++g) {
+          const int s = g % NQ;
+          const uint32_t u = (uint32_t)(g / NQ);
+          ok = mbar_wait(bar_qe + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 62);
+          if (!ok) break;
+          mbar_arrive_expect_tx(bar_qf + 8 * s, QBOX);
+          tma_load_3d(sb + OFF_Q + s * QBOX, &tmQ, bar_qf + 8 * s, 0, tl * TOK, n);
+        }
+      }
+      for (int gg = (g > NQ ? g - NQ : 0); gg < g; ++gg)
+        mbar_wait(bar_qf + 8 * (gg % NQ), (uint32_t)(gg / NQ) & 1, abort_flag, &g_tc_status, 63);
+      if (my_count > 0) mbar_wait(bar_sf, (uint32_t)(my_count - 1) & 1, abort_flag, &g_tc_status, 64);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 64, false, false);
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; i < my_count && ok; ++i) {
+        ok = mbar_wait(bar_sf, (uint32_t)i & 1, abort_flag, &g_tc_status, 65);
+        if (!ok) break;
+        tc_fence_after();
+        for (int tl = 0; tl < ntile; ++tl, ++g) {
+          const int s = g % NQ;
+          const uint32_t u = (uint32_t)(g / NQ);
+          const int b = g & 1;
+          const uint32_t ub = (uint32_t)(g >> 1);
+          ok = mbar_wait(bar_acce + 8 * b, (ub & 1) ^ 1, abort_flag, &g_tc_status, 66);
+          if (!ok) break;
+          ok = mbar_wait(bar_qf + 8 * s, u & 1, abort_flag, &g_tc_status, 67);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t qa = sb + OFF_Q + s * QBOX;
+          const uint32_t d = tmem + b * 64;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t dq = smem_desc_sw128(qa + kk * 32, 16, 1024);
+            const uint64_t dh = smem_desc_sw128(sb + OFF_S + kk * 32, 16, 1024);
+            const uint64_t dl = smem_desc_sw128(sb + OFF_S + SBOX + kk * 32, 16, 1024);
+            mma_bf16(d, dq, dh, idesc, kk > 0 ? 1u : 0u);
+            mma_bf16(d, dq, dl, idesc, 1u);
+          }
+          mma_commit(bar_qe + 8 * s);
+          mma_commit(bar_accf + 8 * b);
+        }
+        if (!ok) break;
+        mma_commit(bar_se);
+      }
+      mma_commit(bar_fin);
+      mbar_wait(bar_fin, 0, abort_flag, &g_tc_status, 68);
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int et = threadIdx.x - 64;
+    uint8_t* ost = smem + OFF_O;
+    int g = 0;
+    bool ok = true;
+    for (int i = 0; i < my_count && ok; ++i) {
+      const int n = blockIdx.x + i * gridDim.x;
+      for (int tl = 0; tl < ntile; ++tl, ++g) {
+        const int b = g & 1;
+        const uint32_t ub = (uint32_t)(g >> 1);
+        mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 69);
+        tc_fence_after();
+        if (et == 0) bulk_wait_read0();
+        named_bar_sync(1, 128);
+        if (*abort_flag) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 32) {
+          uint32_t rr[32];
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 64 + c0, rr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *(uint4*)(ost + row * 128 + ((((c0 >> 3) + j) ^ (row & 7)) << 4)) = make_uint4(
+                pack_bf16x2(__uint_as_float(rr[8 * j]), __uint_as_float(rr[8 * j + 1])),
+                pack_bf16x2(__uint_as_float(rr[8 * j + 2]), __uint_as_float(rr[8 * j + 3])),
+                pack_bf16x2(__uint_as_float(rr[8 * j + 4]), __uint_as_float(rr[8 * j + 5])),
+                pack_bf16x2(__uint_as_float(rr[8 * j + 6]), __uint_as_float(rr[8 * j + 7])));
+        }
+        tc_fence_before();
+        mbar_arrive(bar_acce + 8 * b);
+        fence_proxy_async();
+        named_bar_sync(1, 128);
+        if (et == 0) {
+          tma_store_3d(&tmO, sb + OFF_O, 0, tl * TOK, n);
+          bulk_commit();
+        }
+      }
+    }
+    if (et == 0) bulk_wait0();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+namespace h64 {
+constexpr int D = 64;
+constexpr int XT = 128 * 128;            // X tile: 128 rows x 64 bf16 (one atom): 16 KiB
+constexpr int OFF_XH = 0;
+constexpr int OFF_XL = OFF_XH + XT;
+constexpr int OFF_Y = OFF_XL + XT;       // operand image (hi 8 KiB, lo 8 KiB)
+constexpr int OFF_Z = OFF_Y + c64::IMG;  // Z fp32: 2 boxes of [64 rows][32 fp32]
+constexpr int OFF_BAR = OFF_Z + c64::IMG;
+constexpr int OFF_MISC = OFF_BAR + 32;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+constexpr int THREADS = 256;
+constexpr uint32_t TMEM_COLS = 64;
+}  // namespace h64
+
+// Rows 0-63 run the chain; for a span composite they run E and rows 64-127 run
+// H of the same span (same Y). Each thread: row 32 (w % 4) + lane, columns
+// 32 (w / 4) .. +31.
+__global__ void __launch_bounds__(h64::THREADS)
+    k_chain64_tc(ChainArgs a, const __grid_constant__ CUtensorMap tmZ,
+                 const __grid_constant__ CUtensorMap tmSt) {
+  using namespace h64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q = warp & 3, h = warp >> 2;
+  const int row = q * 32 + lane;
+  const bool top = row < 64;
+  const int r = top ? row : row - 64;
+  const bool leader = threadIdx.x == 0;
+  const uint32_t bar_mma = sb + OFF_BAR;
+  const uint32_t bar_y = bar_mma + 8;
+  const uint32_t bar_z = bar_mma + 16;
+  uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
+  const size_t DD = (size_t)D * D;
+  const bool compose = a.mode == CHAIN_COMPOSE;
+  // one CTA per span for the composites: E (rows 0-63) and H (rows 64-127)
+  ChainProg g = chain_prog(a, blockIdx.x);
+  const bool active = compose || top;                 // rows that carry a chain
+  const bool zy = compose && top;                     // E rows: Z = Y
+  const bool store_sfr = g.mode == CHAIN_SCAN;
+  const bool store_sst = g.mode == CHAIN_PREFIX && a.sst_hilo;
+  if (leader) {
+    mbar_init(bar_mma, 1);
+    mbar_init(bar_y, 1);
+    mbar_init(bar_z, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  auto z_index = [&](const ChainStep& st) -> int {
+    return g.mode == CHAIN_PREFIX ? g.bh * a.nseg + st.t : g.bh * a.T + st.t;
+  };
+  auto fetch_y = [&](const void* src) {
+    mbar_arrive_expect_tx(bar_y, c64::IMG);
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            sb + OFF_Y),
+        "l"(src), "r"((uint32_t)c64::IMG), "r"(bar_y)
+        : "memory");
+  };
+  auto fetch_z = [&](int zi) {
+    mbar_arrive_expect_tx(bar_z, c64::IMG);
+    tma_load_3d(sb + OFF_Z, &tmZ, bar_z, 0, 0, zi);
+    tma_load_3d(sb + OFF_Z + 64 * 128, &tmZ, bar_z, 32, 0, zi);
+  };
+  int nz = 0, ny = 0, nstore = 0;
+  if (leader && g.n > 0) {
+    fetch_y(chain_step_at(a, g, 0).Y);
+    ++ny;
+    fetch_z(z_index(chain_step_at(a, g, 0)));
+    ++nz;
+  }
+  float x[32];
+  {
+    const bool has_init = top && g.init;
+    if (!has_init) {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) x[c] = 0.f;
+    } else if (g.init_hilo) {
+      const __nv_bfloat16* hi = (const __nv_bfloat16*)g.init + (size_t)r * D + h * 32;
+      const __nv_bfloat16* lo = hi + DD;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) x[c] = __bfloat162float(hi[c]) + __bfloat162float(lo[c]);
+    } else {
+#pragma unroll
+      for (int c = 0; c < 32; ++c) x[c] = g.init[(size_t)r * D + h * 32 + c];
+    }
+  }
+  float gprod = 1.f;
+  int tprev = -1;
+  auto store_tile = [&](int pair) {  // rows 0-63 of the X tile: S hi/lo, one [64][64] box each
+    tma_store_3d(&tmSt, sb + OFF_XH, 0, 0, 2 * pair);
+    tma_store_3d(&tmSt, sb + OFF_XL, 0, 0, 2 * pair + 1);
+    bulk_commit();
+    ++nstore;
+  };
+  auto write_x = [&]() {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint4 hi, lo;
+      split_chunk(x + 8 * c, &hi, &lo);
+      const int off = row * 128 + (((4 * h + c) ^ (row & 7)) << 4);
+      *(uint4*)(smem + OFF_XH + off) = hi;
+      *(uint4*)(smem + OFF_XL + off) = lo;
+    }
+  };
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 64, false, true);
+  for (int s = 0; s < g.n; ++s) {
+    const ChainStep st = chain_step_at(a, g, s);
+    if (g.mode == CHAIN_PREFIX && !store_sst && top)
+      for (int c = 0; c < 32; ++c) a.Sst[((size_t)g.bh * a.nseg + s) * DD + (size_t)r * D + h * 32 + c] = x[c];
+    if (leader && nstore > 0) bulk_wait_read0();
+    __syncthreads();
+    write_x();
+    fence_proxy_async();
+    mbar_wait(bar_y, (uint32_t)s & 1, abort_flag, &g_tc_status, 71);
+    float z[32];
+    if (zy) {
+      const uint8_t* yi = smem + OFF_Y;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int off = r * 128 + (((4 * h + c) ^ (r & 7)) << 4);
+        const uint4 hi = *(const uint4*)(yi + off), lo = *(const uint4*)(yi + D * D * 2 + off);
+        const uint32_t hw[4] = {hi.x, hi.y, hi.z, hi.w}, lw[4] = {lo.x, lo.y, lo.z, lo.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 fh = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hw[e]));
+          const float2 fl = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lw[e]));
+          z[8 * c + 2 * e] = fh.x + fl.x;
+          z[8 * c + 2 * e + 1] = fh.y + fl.y;
+        }
+      }
+    }
+    __syncthreads();
+    if (*abort_flag) break;
+    if (leader) {
+      if (store_sfr && tprev >= 0) store_tile(g.bh * a.T + tprev);
+      if (store_sst) store_tile(g.bh * a.nseg + s);
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t dxh = smem_desc_sw128(sb + OFF_XH + kk * 32, 16, 1024);
+        const uint64_t dxl = smem_desc_sw128(sb + OFF_XL + kk * 32, 16, 1024);
+        const uint64_t dyh = smem_desc_sw128(sb + OFF_Y + kk * 2048, D * 128, 1024);
+        const uint64_t dyl = smem_desc_sw128(sb + OFF_Y + D * D * 2 + kk * 2048, D * 128, 1024);
+        mma_bf16(tmem, dxh, dyh, idesc, kk > 0 ? 1u : 0u);
+        mma_bf16(tmem, dxl, dyh, idesc, 1u);
+        mma_bf16(tmem, dxh, dyl, idesc, 1u);
+      }
+      mma_commit(bar_mma);
+    }
+    mbar_wait(bar_mma, (uint32_t)s & 1, abort_flag, &g_tc_status, 72);
+    tc_fence_after();
+    if (leader && s + 1 < g.n) {
+      fetch_y(chain_step_at(a, g, s + 1).Y);
+      ++ny;
+    }
+    mbar_wait(bar_z, (uint32_t)s & 1, abort_flag, &g_tc_status, 73);
+    if (!zy) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float4 f = *(const float4*)(smem + OFF_Z + h * 8192 + r * 128 + ((c ^ (r & 7)) << 4));
+        z[4 * c] = f.x; z[4 * c + 1] = f.y; z[4 * c + 2] = f.z; z[4 * c + 3] = f.w;
+      }
+    }
+    {
+      uint32_t rr[32];
+      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + h * 32, rr);
+      tmem_wait_ld();
+      const float alpha = zy ? 1.0f : compose ? a.gamma[(size_t)g.bh * a.T + st.t] : st.alpha;
+      if (active) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          x[c] = st.reset ? z[c] : alpha * (x[c] - __uint_as_float(rr[c])) + z[c];
+      }
+    }
+    tc_fence_before();
+    __syncthreads();  // every thread has read Z
+    if (leader && s + 1 < g.n) {
+      fetch_z(z_index(chain_step_at(a, g, s + 1)));
+      ++nz;
+    }
+    if (compose) gprod *= a.gamma[(size_t)g.bh * a.T + st.t];
+    if (store_sfr) {
+      tprev = st.t;
+      if (g.j0 + s == a.T - 1 && a.state_out && top)
+        for (int c = 0; c < 32; ++c) a.state_out[(size_t)g.bh * DD + (size_t)r * D + h * 32 + c] = x[c];
+    }
+  }
+  if ((store_sfr && tprev >= 0) || store_sst) {
+    if (leader && nstore > 0) bulk_wait_read0();
+    __syncthreads();
+    if (!*abort_flag) {
+      write_x();
+      fence_proxy_async();
+    }
+    __syncthreads();
+    if (leader && !*abort_flag) store_tile(store_sst ? g.bh * a.nseg + g.n : g.bh * a.T + tprev);
+  }
+  __syncthreads();
+  if (!*abort_flag) {
+    const size_t si = (size_t)g.bh * a.nseg + g.p;
+    if (compose) {
+      if (!top) {
+        for (int c = 0; c < 32; ++c) a.Hc[si * DD + (size_t)r * D + h * 32 + c] = x[c];
+      } else if (a.e_image) {
+        uint8_t* img = (uint8_t*)a.E + si * c64::IMG;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int off = r * 128 + (((4 * h + c) ^ (r & 7)) << 4);
+          split_chunk(x + 8 * c, (uint4*)(img + off), (uint4*)(img + D * D * 2 + off));
+        }
+      } else {
+        for (int c = 0; c < 32; ++c) a.E[si * DD + (size_t)r * D + h * 32 + c] = x[c];
+      }
+      if (threadIdx.x == 0) a.g[si] = gprod;
+    } else if (g.mode == CHAIN_PREFIX && !store_sst && top) {
+      for (int c = 0; c < 32; ++c)
+        a.Sst[((size_t)g.bh * a.nseg + g.n) * DD + (size_t)r * D + h * 32 + c] = x[c];
+    }
+  }
+  if (leader) {
+    if (nstore > 0) bulk_wait0();
+    if (ny > 0) mbar_wait(bar_y, (uint32_t)(ny - 1) & 1, abort_flag, &g_tc_status, 74);
+    if (nz > 0) mbar_wait(bar_z, (uint32_t)(nz - 1) & 1, abort_flag, &g_tc_status, 75);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// 3-D fp32 tensor of 64 x 64 matrices, box {32 columns, 64 rows}, 128-byte swizzle.
+static cudaError_t make_map_f32_mats64(CUtensorMap* m, const void* base, uint64_t n) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t dims[3] = {64, 64, n};
+  cuuint64_t strides[2] = {64 * 4, 64 * 64 * 4};
+  cuuint32_t box[3] = {32, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+static cudaError_t tc_chain64(const ChainArgs& a, int nchains, cudaStream_t st) {
+  if (a.mode == CHAIN_SCAN && !a.sfr_hilo) return cudaErrorNotSupported;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_chain64_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         h64::SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const long long frames = (long long)a.heads * a.T;
+  CUtensorMap mz, ms;
+  cudaError_t e = a.mode == CHAIN_PREFIX ? make_map_f32_mats64(&mz, a.Hc, (uint64_t)a.heads * a.nseg)
+                                         : make_map_f32_mats64(&mz, a.U, (uint64_t)frames);
+  if (e != cudaSuccess) return e;
+  if (a.mode == CHAIN_PREFIX && a.sst_hilo)
+    e = make_map_bf16_3d(&ms, a.Sst, 64, 64, 2 * (uint64_t)a.heads * a.nseg, 64, 64);
+  else
+    e = make_map_bf16_3d(&ms, a.mode == CHAIN_SCAN ? (const void*)a.Sfr : (const void*)a.U, 64, 64,
+                         2 * frames, 64, 64);
+  if (e != cudaSuccess) return e;
+  // span composites run E and H stacked in one CTA per span
+  const int grid = a.mode == CHAIN_COMPOSE ? nchains / 2 : nchains;
+  k_chain64_tc<<<grid, h64::THREADS, h64::SMEM, st>>>(a, mz, ms);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ---- public entry points of the tensor-core kernels (dispatch on D) ----
+cudaError_t tc_contract(const void* k, const void* v, const float* beta, float* A, float* U,
+                        long long N, int S, int D, float cA, float cU, int a_image,
+                        const ProArgs* pro, cudaStream_t st) {
+  if (D == 64) {
+    if (pro) return cudaErrorNotSupported;
+    CUtensorMap mk, mv;
+    cudaError_t e = make_map_bf16_3d(&mk, k, 64, S, N, 64, c64::TOK);
+    if (e != cudaSuccess) return e;
+    e = make_map_bf16_3d(&mv, v, 64, S, N, 64, c64::TOK);
+    if (e != cudaSuccess) return e;
+    static bool attr64 = false;
+    if (!attr64) {
+      e = cudaFuncSetAttribute(k_contract64_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, c64::SMEM);
+      if (e != cudaSuccess) return e;
+      attr64 = true;
+    }
+    const int grid = (int)(N < num_sms() ? N : num_sms());
+    k_contract64_tc<<<grid, c64::THREADS, c64::SMEM, st>>>(mk, mv, beta, A, U, (int)N, S, cA, cU,
+                                                            a_image);
+    count_launch();
+    return cudaGetLastError();
+  }
+  return tc_contract128(k, v, beta, A, U, N, S, D, cA, cU, a_image, pro, st);
+}
+
+cudaError_t tc_readout(const void* q, const void* Sfr_hilo, void* out, long long N, int S, int D,
+                       const ProArgs* pro, cudaStream_t st) {
+  if (D == 64) {
+    if (pro) return cudaErrorNotSupported;
+    CUtensorMap mq, ms, mo;
+    cudaError_t e = make_map_bf16_3d(&mq, q, 64, S, N, 64, r64::TOK);
+    if (e != cudaSuccess) return e;
+    e = make_map_bf16_3d(&ms, Sfr_hilo, 64, 64, 2 * N, 64, 64);
+    if (e != cudaSuccess) return e;
+    e = make_map_bf16_3d(&mo, out, 64, S, N, 64, r64::TOK);
+    if (e != cudaSuccess) return e;
+    static bool attr64 = false;
+    if (!attr64) {
+      e = cudaFuncSetAttribute(k_readout64_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, r64::SMEM);
+      if (e != cudaSuccess) return e;
+      attr64 = true;
+    }
+    const int grid = (int)(N < num_sms() ? N : num_sms());
+    k_readout64_tc<<<grid, r64::THREADS, r64::SMEM, st>>>(mq, ms, mo, (int)N, S);
+    count_launch();
+    return cudaGetLastError();
+  }
+  return tc_readout128(q, Sfr_hilo, out, N, S, D, pro, st);
+}
+
+cudaError_t tc_chain(const ChainArgs& a, int nchains, cudaStream_t st) {
+  if (a.D == 64 && a.y_image) return tc_chain64(a, nchains, st);
+  return tc_chain128(a, nchains, st);
 }
 
 // Failure-path self test: one block waits (bounded by limit_ns) on an mbarrier
