@@ -69,7 +69,7 @@ def phase_bytes(cfg):
     nro = 2 if cfg.bidir_block else 1
     return {
         "contract": fh * cfg.S * (2 * cfg.D * e + 4),          # K, V, beta
-        "readout": fh * cfg.S * 2 * cfg.D * e,                  # Q in, O out
+        "readout": fh * cfg.S * (2 + (1 if cfg.bidir_block else 0)) * cfg.D * e,  # Q in, O (and O_rev) out
         "scan_readout": fh * cfg.S * 2 * cfg.D * e,             # Q in, O out (replay fused)
         "prologue": fh * cfg.S * 4 * cfg.D * e,                 # raw q, k in; q^, k^ out
         "_readout_launches_per_step": nro,

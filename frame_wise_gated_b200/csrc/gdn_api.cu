@@ -118,6 +118,11 @@ Layout make_layout(int B, int H, int T, int S, int D, unsigned flags) {
   off = align256(off + frames * mat);
   L.Sfr = off;
   off = align256(off + frames * mat);  // fp32, or bf16 hi+lo: the same bytes
+  L.Sfr2 = L.Sfr;
+  if (flags & GDN_BIDIR) {             // the reverse direction's per-frame states
+    L.Sfr2 = off;
+    off = align256(off + frames * mat);
+  }
   L.E = off;
   off = align256(off + heads * L.nseg_max * mat);
   L.Hc = off;
@@ -165,7 +170,7 @@ static int check_sizes(int B, int H, int T, int S, int D) {
 static int run_direction(const gdn_params& p, const Layout& L, char* ws, bool reverse,
                          bool block_reset, const void* q, void* out, float* state_out,
                          bool use_tc_chain, bool use_tc_readout, const ProArgs* pro_q,
-                         cudaStream_t st) {
+                         cudaStream_t st, size_t sfr_off, bool do_readout) {
   const bool bf16 = (p.flags & GDN_BF16) != 0;
   const long long frames = (long long)p.B * p.H * p.T;
   ChainArgs a;
@@ -181,7 +186,7 @@ static int run_direction(const gdn_params& p, const Layout& L, char* ws, bool re
   a.gamma = p.gamma;
   a.state_in = p.state_in;
   a.state_out = state_out;
-  a.Sfr = (float*)(ws + L.Sfr);
+  a.Sfr = (float*)(ws + sfr_off);
   a.sfr_hilo = use_tc_readout ? 1 : 0;
   a.E = (float*)(ws + L.E);
   a.Hc = (float*)(ws + L.Hc);
@@ -198,8 +203,8 @@ static int run_direction(const gdn_params& p, const Layout& L, char* ws, bool re
   };
   cudaError_t e;
   // Replay fused with the readout: spans or reset blocks, tensor-core path, no prologue.
-  const bool fused = (p.flags & GDN_FUSED_REPLAY) && use_tc_chain && use_tc_readout && !pro_q &&
-                     (p.flags & GDN_BF16) &&
+  const bool fused = do_readout && (p.flags & GDN_FUSED_REPLAY) && use_tc_chain && use_tc_readout &&
+                     !pro_q && (p.flags & GDN_BF16) &&
                      !(p.flags & GDN_SEQUENTIAL) && tc_scan_readout_supported(p.D);
   auto scan_readout = [&](const ChainArgs& c, int n) -> int {
     PhaseScope ps(PH_SCAN_READOUT, st);
@@ -250,12 +255,13 @@ static int run_direction(const gdn_params& p, const Layout& L, char* ws, bool re
       if ((e = chain(a, a.heads * a.nseg)) != cudaSuccess) return cuda_fail(e, "replay");
     }
   }
+  if (!do_readout) return GDN_OK;
   {
     PhaseScope ps(PH_READOUT, st);
     if (use_tc_readout)
-      e = tc_readout(q, ws + L.Sfr, out, frames, p.S, p.D, pro_q, st);
+      e = tc_readout(q, ws + sfr_off, out, frames, p.S, p.D, pro_q, st);
     else
-      e = simt_readout(bf16, q, (const float*)(ws + L.Sfr), out, frames, p.S, p.D, st);
+      e = simt_readout(bf16, q, (const float*)(ws + sfr_off), out, frames, p.S, p.D, st);
   }
   if (e != cudaSuccess) return cuda_fail(e, "readout");
   return GDN_OK;
@@ -353,14 +359,22 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
 
   const bool block_reset = (f & GDN_BLOCK_RESET) != 0;
   if (f & GDN_BIDIR) {
+    // Both directions' states first, then (tensor-core path) one readout that
+    // reads each Q tile once for both outputs.
+    const bool both = tc_readout_ok && tc_chain_ok && tc_readout2_supported(p.D);
     rc = run_direction(p, L, ws, false, false, q, p.out, p.state_out, tc_chain_ok,
-                       tc_readout_ok, ppq, st);
+                       tc_readout_ok, ppq, st, L.Sfr, !both);
     if (rc) return rc;
-    return run_direction(p, L, ws, true, block_reset, q, p.out_rev, p.state_out_rev,
-                         tc_chain_ok, tc_readout_ok, ppq, st);
+    rc = run_direction(p, L, ws, true, block_reset, q, p.out_rev, p.state_out_rev, tc_chain_ok,
+                       tc_readout_ok, ppq, st, L.Sfr2, !both);
+    if (rc || !both) return rc;
+    PhaseScope ps(PH_READOUT, st);
+    e = tc_readout2(q, ws + L.Sfr, ws + L.Sfr2, p.out, p.out_rev, frames, p.S, p.D, ppq, st);
+    if (e != cudaSuccess) return cuda_fail(e, "bidirectional readout");
+    return GDN_OK;
   }
   return run_direction(p, L, ws, (f & GDN_REVERSE) != 0, block_reset, q, p.out, p.state_out,
-                       tc_chain_ok, tc_readout_ok, ppq, st);
+                       tc_chain_ok, tc_readout_ok, ppq, st, L.Sfr, true);
 }
 
 int scan_ex_entry(const gdn_params& p, cudaStream_t st) {

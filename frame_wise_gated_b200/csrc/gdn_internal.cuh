@@ -106,7 +106,7 @@ __host__ __device__ __forceinline__ void seg_range(const ChainArgs& a, int p, in
 
 // ---- workspace layout ---------------------------------------------------------
 struct Layout {
-  size_t A, U, Sfr, E, Hc, g, Sst, qh, kh, rope, total;
+  size_t A, U, Sfr, Sfr2, E, Hc, g, Sst, qh, kh, rope, total;
   int nseg_max;
 };
 
@@ -156,6 +156,11 @@ cudaError_t tc_readout(const void* q, const void* Sfr_hilo, void* out, long long
 bool tc_scan_readout_supported(int D);
 cudaError_t tc_scan_readout(const ChainArgs& a, int nchains, const void* q, void* out, int S,
                             cudaStream_t st);
+// Both directions' readouts in one pass over Q (bf16 out, D = 128).
+bool tc_readout2_supported(int D);
+cudaError_t tc_readout2(const void* q, const void* sfr_f, const void* sfr_r, void* out_f,
+                        void* out_r, long long N, int S, int D, const ProArgs* pro,
+                        cudaStream_t st);
 bool tc_chain_supported(int D);
 cudaError_t tc_chain(const ChainArgs& a, int nchains, cudaStream_t st);
 cudaError_t tc_selftest_wait(int arrive, long long limit_ns, cudaStream_t st);

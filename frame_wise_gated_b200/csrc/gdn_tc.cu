@@ -2186,6 +2186,274 @@ static cudaError_t tc_chain64(const ChainArgs& a, int nchains, cudaStream_t st) 
   return cudaGetLastError();
 }
 
+// ============================================================================
+// Bidirectional readout (a6 for both directions, a1 fused), D = 128.
+// Each raw Q tile is loaded once (and, with the prologue, transformed once)
+// and multiplied with both directions' states:
+//   O_fwd = Q S_fwd_hi^T + Q S_fwd_lo^T,   O_rev = Q S_rev_hi^T + Q S_rev_lo^T
+// (four fp32 TMEM accumulators: two tiles in flight x two directions). Both
+// outputs leave through two 16 KiB swizzled staging buffers and TMA stores.
+// The prologue's (cos, sin) table is read through L1 (no room in smem).
+// ============================================================================
+namespace rd2 {
+constexpr int D = 128;
+constexpr int TOK = 128;
+constexpr int NQ = 2;
+constexpr int BOX = TOK * 128;           // [128 rows][64 channels] bf16: 16 KiB
+constexpr int QT = 2 * BOX;
+constexpr int OFF_Q = 0;
+constexpr int OFF_SF = OFF_Q + NQ * QT;  // forward state: hi (2 boxes), lo (2 boxes)
+constexpr int OFF_SR = OFF_SF + 4 * BOX; // reverse state
+constexpr int OFF_O = OFF_SR + 4 * BOX;  // two staging boxes
+constexpr int OFF_W = OFF_O + 2 * BOX;   // prologue weights
+constexpr int OFF_BAR = OFF_W + D * 4;
+constexpr int NBAR = 3 * NQ + 2 + 4 + 1;
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+constexpr int threads(bool pro) { return pro ? 448 : 192; }
+constexpr uint32_t TMEM_COLS = 512;
+}  // namespace rd2
+
+template <bool PRO>
+__global__ void __launch_bounds__(rd2::threads(PRO), 1)
+    k_readout2_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmSF,
+                  const __grid_constant__ CUtensorMap tmSR, const __grid_constant__ CUtensorMap tmOF,
+                  const __grid_constant__ CUtensorMap tmOR, int N, int S, ProArgs pro) {
+  using namespace rd2;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar_qf = sb + OFF_BAR;
+  const uint32_t bar_qr = bar_qf + 8 * NQ;
+  const uint32_t bar_qe = bar_qr + 8 * NQ;
+  const uint32_t bar_sf = bar_qe + 8 * NQ;
+  const uint32_t bar_se = bar_sf + 8;
+  const uint32_t bar_accf = bar_se + 8;
+  const uint32_t bar_acce = bar_accf + 16;
+  const uint32_t bar_fin = bar_acce + 16;
+  uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NQ; ++s) {
+      mbar_init(bar_qf + 8 * s, 1);
+      mbar_init(bar_qr + 8 * s, 256);
+      mbar_init(bar_qe + 8 * s, 1);
+    }
+    mbar_init(bar_sf, 1);
+    mbar_init(bar_se, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_accf + 8 * b, 1);
+      mbar_init(bar_acce + 8 * b, 128);
+    }
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (PRO && threadIdx.x < D) ((float*)(smem + OFF_W))[threadIdx.x] = pro.w[threadIdx.x];
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int ntile = (S + TOK - 1) / TOK;
+  const int my_count = (int)blockIdx.x < N ? (N - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; i < my_count && ok; ++i) {
+        const int n = blockIdx.x + i * gridDim.x;
+        ok = mbar_wait(bar_se, ((uint32_t)i & 1) ^ 1, abort_flag, &g_tc_status, 81);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar_sf, 8 * BOX);
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            tma_load_3d(sb + OFF_SF + (2 * hl + x) * BOX, &tmSF, bar_sf, 64 * x, 0, 2 * n + hl);
+            tma_load_3d(sb + OFF_SR + (2 * hl + x) * BOX, &tmSR, bar_sf, 64 * x, 0, 2 * n + hl);
+          }
+        for (int tl = 0; tl < ntile; ++tl, ++g) {
+          const int s = g % NQ;
+          const uint32_t u = (uint32_t)(g / NQ);
+          ok = mbar_wait(bar_qe + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 82);
+          if (!ok) break;
+          const uint32_t qd = sb + OFF_Q + s * QT;
+          mbar_arrive_expect_tx(bar_qf + 8 * s, QT);
+          tma_load_3d(qd, &tmQ, bar_qf + 8 * s, 0, tl * TOK, n);
+          tma_load_3d(qd + BOX, &tmQ, bar_qf + 8 * s, 64, tl * TOK, n);
+        }
+      }
+      for (int gg = (g > NQ ? g - NQ : 0); gg < g; ++gg)
+        mbar_wait(bar_qf + 8 * (gg % NQ), (uint32_t)(gg / NQ) & 1, abort_flag, &g_tc_status, 83);
+      if (my_count > 0) mbar_wait(bar_sf, (uint32_t)(my_count - 1) & 1, abort_flag, &g_tc_status, 84);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; i < my_count && ok; ++i) {
+        ok = mbar_wait(bar_sf, (uint32_t)i & 1, abort_flag, &g_tc_status, 85);
+        if (!ok) break;
+        tc_fence_after();
+        for (int tl = 0; tl < ntile; ++tl, ++g) {
+          const int s = g % NQ;
+          const uint32_t u = (uint32_t)(g / NQ);
+          const int b = g & 1;
+          const uint32_t ub = (uint32_t)(g >> 1);
+          ok = mbar_wait(bar_acce + 8 * b, (ub & 1) ^ 1, abort_flag, &g_tc_status, 86);
+          if (!ok) break;
+          ok = mbar_wait((PRO ? bar_qr : bar_qf) + 8 * s, u & 1, abort_flag, &g_tc_status, 87);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t qa = sb + OFF_Q + s * QT;
+#pragma unroll
+          for (int dir = 0; dir < 2; ++dir) {
+            const uint32_t sh = sb + (dir ? OFF_SR : OFF_SF), sl = sh + 2 * BOX;
+            const uint32_t d = tmem + b * 256 + dir * 128;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * BOX + (kk & 3) * 32;
+              const uint64_t dq = smem_desc_sw128(qa + off, 16, 1024);
+              mma_bf16(d, dq, smem_desc_sw128(sh + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+              mma_bf16(d, dq, smem_desc_sw128(sl + off, 16, 1024), idesc, 1u);
+            }
+          }
+          mma_commit(bar_qe + 8 * s);
+          mma_commit(bar_accf + 8 * b);
+        }
+        if (!ok) break;
+        mma_commit(bar_se);
+      }
+      mma_commit(bar_fin);
+      mbar_wait(bar_fin, 0, abort_flag, &g_tc_status, 88);
+    }
+    __syncwarp();
+  } else if (warp < 6) {
+    // ---- epilogue: four 64-column rounds per tile (fwd lo/hi half, rev ...) ----
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int et = threadIdx.x - 64;
+    int g = 0, nstores = 0;
+    bool ok = true;
+    for (int i = 0; i < my_count && ok; ++i) {
+      const int n = blockIdx.x + i * gridDim.x;
+      for (int tl = 0; tl < ntile; ++tl, ++g) {
+        const int b = g & 1;
+        const uint32_t ub = (uint32_t)(g >> 1);
+        mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 89);
+        tc_fence_after();
+#pragma unroll
+        for (int rnd = 0; rnd < 4; ++rnd) {
+          const int dir = rnd >> 1, half = rnd & 1, buf = nstores & 1;
+          // the store that last used this staging buffer has read it
+          if (et == 0 && nstores >= 2) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+          named_bar_sync(1, 128);
+          if (*abort_flag) {
+            ok = false;
+            break;
+          }
+          uint8_t* ost = smem + OFF_O + buf * BOX;
+#pragma unroll
+          for (int c0 = 0; c0 < 64; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 256 + dir * 128 + half * 64 + c0, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              *(uint4*)(ost + row * 128 + ((((c0 >> 3) + j) ^ (row & 7)) << 4)) = make_uint4(
+                  pack_bf16x2(__uint_as_float(r[8 * j]), __uint_as_float(r[8 * j + 1])),
+                  pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3])),
+                  pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5])),
+                  pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7])));
+          }
+          fence_proxy_async();
+          named_bar_sync(1, 128);
+          if (et == 0) {
+            tma_store_3d(dir ? &tmOR : &tmOF, sb + OFF_O + buf * BOX, 64 * half, tl * TOK, n);
+            bulk_commit();
+          }
+          ++nstores;
+        }
+        if (!ok) break;
+        tc_fence_before();
+        mbar_arrive(bar_acce + 8 * b);
+      }
+    }
+    if (et == 0) bulk_wait0();
+  } else if (PRO) {
+    const int t = threadIdx.x - 192;
+    const int r = t >> 1, h = t & 1;
+    int g = 0;
+    bool ok = true;
+    for (int i = 0; i < my_count && ok; ++i) {
+      for (int tl = 0; tl < ntile; ++tl, ++g) {
+        const int s = g % NQ;
+        const uint32_t u = (uint32_t)(g / NQ);
+        ok = mbar_wait(bar_qf + 8 * s, u & 1, abort_flag, &g_tc_status, 90);
+        if (!ok) break;
+        const int tok = tl * TOK + r;
+        float f[64];
+        pro_row_part<8>(smem + OFF_Q + s * QT, BOX, r, 64 * h, D, tok, tok < S, pro,
+                        (const float*)(smem + OFF_W) + 64 * h, pro.cs, f);
+        fence_proxy_async();
+        mbar_arrive(bar_qr + 8 * s);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+template <bool PRO>
+static cudaError_t launch_readout2(const CUtensorMap* m, long long N, int S, const ProArgs& pa,
+                                   cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_readout2_tc<PRO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         rd2::SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int grid = (int)(N < num_sms() ? N : num_sms());
+  k_readout2_tc<PRO><<<grid, rd2::threads(PRO), rd2::SMEM, st>>>(m[0], m[1], m[2], m[3], m[4], (int)N, S,
+                                                                  pa);
+  count_launch();
+  return cudaGetLastError();
+}
+
+bool tc_readout2_supported(int D) { return D == 128; }
+
+cudaError_t tc_readout2(const void* q, const void* sfr_f, const void* sfr_r, void* out_f,
+                        void* out_r, long long N, int S, int D, const ProArgs* pro,
+                        cudaStream_t st) {
+  if (D != 128) return cudaErrorNotSupported;
+  CUtensorMap m[5];
+  cudaError_t e = make_map_bf16_3d(&m[0], q, D, S, N, 64, rd2::TOK);
+  if (e == cudaSuccess) e = make_map_bf16_3d(&m[1], sfr_f, D, D, 2 * N, 64, 128);
+  if (e == cudaSuccess) e = make_map_bf16_3d(&m[2], sfr_r, D, D, 2 * N, 64, 128);
+  if (e == cudaSuccess) e = make_map_bf16_3d(&m[3], out_f, D, S, N, 64, rd2::TOK);
+  if (e == cudaSuccess) e = make_map_bf16_3d(&m[4], out_r, D, S, N, 64, rd2::TOK);
+  if (e != cudaSuccess) return e;
+  ProArgs pa = {};
+  if (pro) {
+    pa = *pro;
+    return launch_readout2<true>(m, N, S, pa, st);
+  }
+  return launch_readout2<false>(m, N, S, pa, st);
+}
+
 // ---- public entry points of the tensor-core kernels (dispatch on D) ----
 cudaError_t tc_contract(const void* k, const void* v, const float* beta, float* A, float* U,
                         long long N, int S, int D, float cA, float cU, int a_image,
