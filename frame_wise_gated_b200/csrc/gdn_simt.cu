@@ -194,28 +194,32 @@ cudaError_t simt_contract(bool bf16, const void* k, const void* v, const float* 
 // ----------------------------------------------------------------------------
 constexpr int kChainRows = 16;
 
+template <int D>
 __device__ __forceinline__ void chain_step(float* X, float* Yc, const float* __restrict__ Y,
-                                           const float* __restrict__ Z, float alpha, int D,
-                                           int row0, float* acc) {
+                                           const float* __restrict__ Z, float alpha, int row0,
+                                           bool reset) {
+  constexpr int NM = D / 16;
   const int r = threadIdx.x >> 4, l = threadIdx.x & 15;
-  const int nm = D >> 4;
-  for (int m = 0; m < nm; ++m) acc[m] = 0.f;
+  float acc[NM];
+#pragma unroll
+  for (int m = 0; m < NM; ++m) acc[m] = 0.f;
   for (int k0 = 0; k0 < D; k0 += 16) {
     for (int e = threadIdx.x; e < 16 * D; e += 256) Yc[e] = Y[(size_t)k0 * D + e];
     __syncthreads();
 #pragma unroll 4
     for (int kk = 0; kk < 16; ++kk) {
       const float x = X[r * D + k0 + kk];
-      for (int m = 0; m < nm; ++m) acc[m] = fmaf(x, Yc[kk * D + l + 16 * m], acc[m]);
+#pragma unroll
+      for (int m = 0; m < NM; ++m) acc[m] = fmaf(x, Yc[kk * D + l + 16 * m], acc[m]);
     }
     __syncthreads();
   }
   const int row = row0 + r;
-  if (row < D) {
-    for (int m = 0; m < nm; ++m) {
-      const int c = l + 16 * m;
-      X[r * D + c] = alpha * (X[r * D + c] - acc[m]) + Z[(size_t)row * D + c];
-    }
+#pragma unroll
+  for (int m = 0; m < NM; ++m) {
+    const int c = l + 16 * m;
+    const float z = Z[(size_t)row * D + c];
+    X[r * D + c] = reset ? z : alpha * (X[r * D + c] - acc[m]) + z;
   }
   __syncthreads();
 }
@@ -247,12 +251,12 @@ __device__ __forceinline__ void rows_load(float* X, const float* src, int D, int
   __syncthreads();
 }
 
+template <int D>
 __global__ void __launch_bounds__(256) k_chain_simt(ChainArgs a) {
   extern __shared__ float smem[];
-  const int D = a.D, T = a.T;
+  const int T = a.T;
   float* X = smem;                    // [16][D]
   float* Yc = smem + kChainRows * D;  // [16][D]
-  float acc[16];
   const int row0 = blockIdx.y * kChainRows;
   const int c = blockIdx.x;
 
@@ -270,11 +274,11 @@ __global__ void __launch_bounds__(256) k_chain_simt(ChainArgs a) {
     int tprev = -1;
     for (int j = j0; j < j1; ++j) {
       const int t = frame_at(j, T, a.reverse);
-      if (a.seg == SEG_SEQUENTIAL && a.seq_reset && j > 0 && (t / a.block) != (tprev / a.block))
-        rows_load(X, nullptr, D, row0);
+      const bool rst = a.seg == SEG_SEQUENTIAL && a.seq_reset && j > 0 &&
+                       (t / a.block) != (tprev / a.block);
       tprev = t;
       const size_t fi = (size_t)bh * T + t;
-      chain_step(X, Yc, a.A + fi * D * D, a.U + fi * D * D, a.gamma[fi], D, row0, acc);
+      chain_step<D>(X, Yc, a.A + fi * D * D, a.U + fi * D * D, a.gamma[fi], row0, rst);
       if (a.sfr_hilo)
         rows_store_hilo(X, (__nv_bfloat16*)a.Sfr + fi * 2 * D * D, D, row0);
       else
@@ -295,9 +299,9 @@ __global__ void __launch_bounds__(256) k_chain_simt(ChainArgs a) {
       const size_t fi = (size_t)bh * T + t;
       const float* Af = a.A + fi * D * D;
       if (which)
-        chain_step(X, Yc, Af, a.U + fi * D * D, a.gamma[fi], D, row0, acc);
+        chain_step<D>(X, Yc, Af, a.U + fi * D * D, a.gamma[fi], row0, false);
       else
-        chain_step(X, Yc, Af, Af, 1.0f, D, row0, acc);
+        chain_step<D>(X, Yc, Af, Af, 1.0f, row0, false);
       gp *= a.gamma[fi];
     }
     const size_t si = (size_t)bh * a.nseg + p;
@@ -309,22 +313,30 @@ __global__ void __launch_bounds__(256) k_chain_simt(ChainArgs a) {
     for (int p = 0; p < a.nseg; ++p) {
       const size_t si = (size_t)bh * a.nseg + p;
       rows_store(X, a.Sst + si * D * D, D, row0);
-      if (p + 1 < a.nseg) chain_step(X, Yc, a.E + si * D * D, a.Hc + si * D * D, a.g[si], D, row0, acc);
+      if (p + 1 < a.nseg)
+        chain_step<D>(X, Yc, a.E + si * D * D, a.Hc + si * D * D, a.g[si], row0, false);
     }
   }
 }
 
-cudaError_t simt_chain(const ChainArgs& a, int nchains, cudaStream_t st) {
-  const size_t smem = 2 * kChainRows * a.D * sizeof(float);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(k_chain_simt, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  dim3 grid((unsigned)nchains, (a.D + kChainRows - 1) / kChainRows);
-  k_chain_simt<<<grid, 256, smem, st>>>(a);
+template <int D>
+static cudaError_t chain_t(const ChainArgs& a, int nchains, cudaStream_t st) {
+  const size_t smem = 2 * kChainRows * D * sizeof(float);
+  dim3 grid((unsigned)nchains, (D + kChainRows - 1) / kChainRows);
+  k_chain_simt<D><<<grid, 256, smem, st>>>(a);
   count_launch();
   return cudaGetLastError();
+}
+
+cudaError_t simt_chain(const ChainArgs& a, int nchains, cudaStream_t st) {
+  switch (a.D) {
+    case 16: return chain_t<16>(a, nchains, st);
+    case 32: return chain_t<32>(a, nchains, st);
+    case 64: return chain_t<64>(a, nchains, st);
+    case 128: return chain_t<128>(a, nchains, st);
+    case 256: return chain_t<256>(a, nchains, st);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 // ----------------------------------------------------------------------------

@@ -424,7 +424,7 @@ __global__ void __launch_bounds__(ctr::THREADS, 1)
   }
 }
 
-bool tc_contract_supported(int D) { return D == 128 || D == 64; }
+bool tc_contract_supported(int D) { return D == 128 || D == 64 || D == 256; }
 int tc_prologue_max_positions() { return ctr::TAB_MAX / 32; }
 
 static cudaError_t tc_contract128(const void* k, const void* v, const float* beta, float* A,
@@ -479,7 +479,7 @@ constexpr uint32_t TMEM_COLS = 256;
 template <bool PRO>
 __global__ void __launch_bounds__(rdo::threads(PRO), 1)
     k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
-                 const __grid_constant__ CUtensorMap tmO, int N, int S, ProArgs pro) {
+                 const __grid_constant__ CUtensorMap tmO, int N, int S, ProArgs pro, int parts) {
   using namespace rdo;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -525,15 +525,22 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const int ntile = (S + TOK - 1) / TOK;
-  const int my_count = (int)blockIdx.x < N ? (N - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  // Work units: each frame-head's tiles in kParts contiguous parts (outputs are
+  // per token, so parts need no reduction); finer units even out the rounds.
+  const int kParts = parts;
+  const int NU = N * kParts;
+  const int my_count = (int)blockIdx.x < NU ? (NU - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
   if (warp == 0) {
     if (lane == 0) {
       int g = 0;
       bool ok = true;
       for (int i = 0; i < my_count && ok; ++i) {
-        const int n = blockIdx.x + i * gridDim.x;
-        ok = mbar_wait(bar_se, ((uint32_t)i & 1) ^ 1, abort_flag, &g_tc_status, 11);
+        const int unit = blockIdx.x + i * gridDim.x;
+        const int n = unit / kParts, part = unit % kParts;
+        const int tl0 = part * ntile / kParts, tl1 = (part + 1) * ntile / kParts;
+        (void)n;
+                ok = mbar_wait(bar_se, ((uint32_t)i & 1) ^ 1, abort_flag, &g_tc_status, 11);
         if (!ok) break;
         mbar_arrive_expect_tx(bar_sf, 4 * BOX);
         const uint32_t sd = sb + OFF_S;
@@ -541,7 +548,7 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
         tma_load_3d(sd + BOX, &tmS, bar_sf, 64, 0, 2 * n);
         tma_load_3d(sd + 2 * BOX, &tmS, bar_sf, 0, 0, 2 * n + 1);
         tma_load_3d(sd + 3 * BOX, &tmS, bar_sf, 64, 0, 2 * n + 1);
-        for (int tl = 0; tl < ntile; ++tl, ++g) {
+        for (int tl = tl0; tl < tl1; ++tl, ++g) {
           const int s = g % NQ;
           const uint32_t u = (uint32_t)(g / NQ);
           ok = mbar_wait(bar_qe + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 12);
@@ -563,10 +570,14 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
       int g = 0;
       bool ok = true;
       for (int i = 0; i < my_count && ok; ++i) {
+        const int unit = blockIdx.x + i * gridDim.x;
+        const int n = unit / kParts, part = unit % kParts;
+        const int tl0 = part * ntile / kParts, tl1 = (part + 1) * ntile / kParts;
+        (void)n;
         ok = mbar_wait(bar_sf, (uint32_t)i & 1, abort_flag, &g_tc_status, 15);
         if (!ok) break;
         tc_fence_after();
-        for (int tl = 0; tl < ntile; ++tl, ++g) {
+        for (int tl = tl0; tl < tl1; ++tl, ++g) {
           const int s = g % NQ;
           const uint32_t u = (uint32_t)(g / NQ);
           const int b = g & 1;
@@ -608,8 +619,11 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
     int g = 0;
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
-      const int n = blockIdx.x + i * gridDim.x;
-      for (int tl = 0; tl < ntile; ++tl, ++g) {
+      const int unit = blockIdx.x + i * gridDim.x;
+      const int n = unit / kParts, part = unit % kParts;
+      const int tl0 = part * ntile / kParts, tl1 = (part + 1) * ntile / kParts;
+      (void)n;
+            for (int tl = tl0; tl < tl1; ++tl, ++g) {
         const int b = g & 1;
         const uint32_t ub = (uint32_t)(g >> 1);
         mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 19);
@@ -659,7 +673,11 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
     int g = 0;
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
-      for (int tl = 0; tl < ntile; ++tl, ++g) {
+      const int unit = blockIdx.x + i * gridDim.x;
+      const int n = unit / kParts, part = unit % kParts;
+      const int tl0 = part * ntile / kParts, tl1 = (part + 1) * ntile / kParts;
+      (void)n;
+      for (int tl = tl0; tl < tl1; ++tl, ++g) {
         const int s = g % NQ;
         const uint32_t u = (uint32_t)(g / NQ);
         ok = mbar_wait(bar_qf + 8 * s, u & 1, abort_flag, &g_tc_status, 20);
@@ -682,7 +700,14 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
   }
 }
 
-bool tc_readout_supported(int D) { return D == 128 || D == 64; }
+bool tc_readout_supported(int D) { return D == 128 || D == 64 || D == 256; }
+
+// Readout work units: split each frame-head's tiles in two when there are
+// fewer than four rounds of frame-heads for the persistent grid (evens out
+// the last round); with more rounds the per-unit state loads cost more.
+static int readout_parts(long long N, int ntile) {
+  return (ntile >= 8 && N < 4LL * num_sms()) ? 2 : 1;
+}
 
 template <bool PRO>
 static cudaError_t launch_readout(const CUtensorMap& mq, const CUtensorMap& ms, const CUtensorMap& mo,
@@ -694,8 +719,10 @@ static cudaError_t launch_readout(const CUtensorMap& mq, const CUtensorMap& ms, 
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  const int grid = (int)(N < num_sms() ? N : num_sms());
-  k_readout_tc<PRO><<<grid, rdo::threads(PRO), rdo::SMEM, st>>>(mq, ms, mo, (int)N, S, pa);
+  const int parts = readout_parts(N, (S + rdo::TOK - 1) / rdo::TOK);
+  const long long units = N * parts;
+  const int grid = (int)(units < num_sms() ? units : num_sms());
+  k_readout_tc<PRO><<<grid, rdo::threads(PRO), rdo::SMEM, st>>>(mq, ms, mo, (int)N, S, pa, parts);
   count_launch();
   return cudaGetLastError();
 }
@@ -1744,7 +1771,7 @@ constexpr uint32_t TMEM_COLS = 128;
 
 __global__ void __launch_bounds__(r64::THREADS, 1)
     k_readout64_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
-                   const __grid_constant__ CUtensorMap tmO, int N, int S) {
+                   const __grid_constant__ CUtensorMap tmO, int N, int S, int parts) {
   using namespace r64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -1783,20 +1810,27 @@ __global__ void __launch_bounds__(r64::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const int ntile = (S + TOK - 1) / TOK;
-  const int my_count = (int)blockIdx.x < N ? (N - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  // Work units: each frame-head's tiles in kParts contiguous parts (outputs are
+  // per token, so parts need no reduction); finer units even out the rounds.
+  const int kParts = parts;
+  const int NU = N * kParts;
+  const int my_count = (int)blockIdx.x < NU ? (NU - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
   if (warp == 0) {
     if (lane == 0) {
       int g = 0;
       bool ok = true;
       for (int i = 0; i < my_count && ok; ++i) {
-        const int n = blockIdx.x + i * gridDim.x;
-        ok = mbar_wait(bar_se, ((uint32_t)i & 1) ^ 1, abort_flag, &g_tc_status, 61);
+        const int unit = blockIdx.x + i * gridDim.x;
+        const int n = unit / kParts, part = unit % kParts;
+        const int tl0 = part * ntile / kParts, tl1 = (part + 1) * ntile / kParts;
+        (void)n;
+                ok = mbar_wait(bar_se, ((uint32_t)i & 1) ^ 1, abort_flag, &g_tc_status, 61);
         if (!ok) break;
         mbar_arrive_expect_tx(bar_sf, 2 * SBOX);
         tma_load_3d(sb + OFF_S, &tmS, bar_sf, 0, 0, 2 * n);
         tma_load_3d(sb + OFF_S + SBOX, &tmS, bar_sf, 0, 0, 2 * n + 1);
-        for (int tl = 0; tl < ntile; ++tl, ++g) {
+        for (int tl = tl0; tl < tl1; ++tl, ++g) {
           const int s = g % NQ;
           const uint32_t u = (uint32_t)(g / NQ);
           ok = mbar_wait(bar_qe + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 62);
@@ -1816,10 +1850,14 @@ __global__ void __launch_bounds__(r64::THREADS, 1)
       int g = 0;
       bool ok = true;
       for (int i = 0; i < my_count && ok; ++i) {
+        const int unit = blockIdx.x + i * gridDim.x;
+        const int n = unit / kParts, part = unit % kParts;
+        const int tl0 = part * ntile / kParts, tl1 = (part + 1) * ntile / kParts;
+        (void)n;
         ok = mbar_wait(bar_sf, (uint32_t)i & 1, abort_flag, &g_tc_status, 65);
         if (!ok) break;
         tc_fence_after();
-        for (int tl = 0; tl < ntile; ++tl, ++g) {
+        for (int tl = tl0; tl < tl1; ++tl, ++g) {
           const int s = g % NQ;
           const uint32_t u = (uint32_t)(g / NQ);
           const int b = g & 1;
@@ -1857,8 +1895,11 @@ __global__ void __launch_bounds__(r64::THREADS, 1)
     int g = 0;
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
-      const int n = blockIdx.x + i * gridDim.x;
-      for (int tl = 0; tl < ntile; ++tl, ++g) {
+      const int unit = blockIdx.x + i * gridDim.x;
+      const int n = unit / kParts, part = unit % kParts;
+      const int tl0 = part * ntile / kParts, tl1 = (part + 1) * ntile / kParts;
+      (void)n;
+            for (int tl = tl0; tl < tl1; ++tl, ++g) {
         const int b = g & 1;
         const uint32_t ub = (uint32_t)(g >> 1);
         mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 69);
@@ -2218,7 +2259,8 @@ template <bool PRO>
 __global__ void __launch_bounds__(rd2::threads(PRO), 1)
     k_readout2_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmSF,
                   const __grid_constant__ CUtensorMap tmSR, const __grid_constant__ CUtensorMap tmOF,
-                  const __grid_constant__ CUtensorMap tmOR, int N, int S, ProArgs pro) {
+                  const __grid_constant__ CUtensorMap tmOR, int N, int S, ProArgs pro,
+                  int parts) {
   using namespace rd2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -2260,15 +2302,22 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const int ntile = (S + TOK - 1) / TOK;
-  const int my_count = (int)blockIdx.x < N ? (N - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  // Work units: each frame-head's tiles in kParts contiguous parts (outputs are
+  // per token, so parts need no reduction); finer units even out the rounds.
+  const int kParts = parts;
+  const int NU = N * kParts;
+  const int my_count = (int)blockIdx.x < NU ? (NU - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
   if (warp == 0) {
     if (lane == 0) {
       int g = 0;
       bool ok = true;
       for (int i = 0; i < my_count && ok; ++i) {
-        const int n = blockIdx.x + i * gridDim.x;
-        ok = mbar_wait(bar_se, ((uint32_t)i & 1) ^ 1, abort_flag, &g_tc_status, 81);
+        const int unit = blockIdx.x + i * gridDim.x;
+        const int n = unit / kParts, part = unit % kParts;
+        const int tl0 = part * ntile / kParts, tl1 = (part + 1) * ntile / kParts;
+        (void)n;
+                ok = mbar_wait(bar_se, ((uint32_t)i & 1) ^ 1, abort_flag, &g_tc_status, 81);
         if (!ok) break;
         mbar_arrive_expect_tx(bar_sf, 8 * BOX);
 #pragma unroll
@@ -2278,7 +2327,7 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
             tma_load_3d(sb + OFF_SF + (2 * hl + x) * BOX, &tmSF, bar_sf, 64 * x, 0, 2 * n + hl);
             tma_load_3d(sb + OFF_SR + (2 * hl + x) * BOX, &tmSR, bar_sf, 64 * x, 0, 2 * n + hl);
           }
-        for (int tl = 0; tl < ntile; ++tl, ++g) {
+        for (int tl = tl0; tl < tl1; ++tl, ++g) {
           const int s = g % NQ;
           const uint32_t u = (uint32_t)(g / NQ);
           ok = mbar_wait(bar_qe + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 82);
@@ -2300,10 +2349,14 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
       int g = 0;
       bool ok = true;
       for (int i = 0; i < my_count && ok; ++i) {
+        const int unit = blockIdx.x + i * gridDim.x;
+        const int n = unit / kParts, part = unit % kParts;
+        const int tl0 = part * ntile / kParts, tl1 = (part + 1) * ntile / kParts;
+        (void)n;
         ok = mbar_wait(bar_sf, (uint32_t)i & 1, abort_flag, &g_tc_status, 85);
         if (!ok) break;
         tc_fence_after();
-        for (int tl = 0; tl < ntile; ++tl, ++g) {
+        for (int tl = tl0; tl < tl1; ++tl, ++g) {
           const int s = g % NQ;
           const uint32_t u = (uint32_t)(g / NQ);
           const int b = g & 1;
@@ -2344,8 +2397,11 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
     int g = 0, nstores = 0;
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
-      const int n = blockIdx.x + i * gridDim.x;
-      for (int tl = 0; tl < ntile; ++tl, ++g) {
+      const int unit = blockIdx.x + i * gridDim.x;
+      const int n = unit / kParts, part = unit % kParts;
+      const int tl0 = part * ntile / kParts, tl1 = (part + 1) * ntile / kParts;
+      (void)n;
+            for (int tl = tl0; tl < tl1; ++tl, ++g) {
         const int b = g & 1;
         const uint32_t ub = (uint32_t)(g >> 1);
         mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 89);
@@ -2394,7 +2450,11 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
     int g = 0;
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
-      for (int tl = 0; tl < ntile; ++tl, ++g) {
+      const int unit = blockIdx.x + i * gridDim.x;
+      const int n = unit / kParts, part = unit % kParts;
+      const int tl0 = part * ntile / kParts, tl1 = (part + 1) * ntile / kParts;
+      (void)n;
+      for (int tl = tl0; tl < tl1; ++tl, ++g) {
         const int s = g % NQ;
         const uint32_t u = (uint32_t)(g / NQ);
         ok = mbar_wait(bar_qf + 8 * s, u & 1, abort_flag, &g_tc_status, 90);
@@ -2426,9 +2486,11 @@ static cudaError_t launch_readout2(const CUtensorMap* m, long long N, int S, con
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  const int grid = (int)(N < num_sms() ? N : num_sms());
+  const int parts = readout_parts(N, (S + rd2::TOK - 1) / rd2::TOK);
+  const long long units = N * parts;
+  const int grid = (int)(units < num_sms() ? units : num_sms());
   k_readout2_tc<PRO><<<grid, rd2::threads(PRO), rd2::SMEM, st>>>(m[0], m[1], m[2], m[3], m[4], (int)N, S,
-                                                                  pa);
+                                                                  pa, parts);
   count_launch();
   return cudaGetLastError();
 }
@@ -2454,10 +2516,451 @@ cudaError_t tc_readout2(const void* q, const void* sfr_f, const void* sfr_r, voi
   return launch_readout2<false>(m, N, S, pa, st);
 }
 
+// ============================================================================
+// D = 256 tensor-core contraction and readout.
+// Contraction: two CTAs per frame-head, one per 128-row half i of A and U:
+//   A[128i.., :] += K_i^T (beta K),  U[128i.., :] += V_i^T (beta K)
+// as M = 128, N = 256 MMAs (all 512 TMEM columns, no double buffer); the two
+// halves of a frame-head run on neighbouring CTAs, so K is read once from
+// HBM and once from L2. Readout: two CTAs per frame-head, one per 128-column
+// half j of O = Q S^T, holding rows 128j.. of S (hi, lo: 128 KiB) while Q
+// streams as [128 tokens][128 channels] half tiles (K split in two).
+// ============================================================================
+namespace c256 {
+constexpr int D = 256;
+constexpr int TOK = 64;
+constexpr int NST = 2;
+constexpr int BOX = TOK * 128;          // [64 tokens][64 channels]: 8 KiB
+constexpr int KT = 4 * BOX;             // K stage tile, all channels: 32 KiB
+constexpr int VT = 2 * BOX;             // V stage tile, one channel half: 16 KiB
+constexpr int OFF_K = 0;
+constexpr int OFF_V = OFF_K + NST * KT;
+constexpr int OFF_BK = OFF_V + NST * VT;
+constexpr int OFF_BETA = OFF_BK + NST * KT;
+constexpr int OFF_BAR = OFF_BETA + NST * TOK * 4;
+constexpr int NBAR = 3 * NST + 3;
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+constexpr int NSC = 256;
+constexpr int THREADS = 64 + NSC + 128;
+constexpr uint32_t TMEM_COLS = 512;
+}  // namespace c256
+
+__global__ void __launch_bounds__(c256::THREADS, 1)
+    k_contract256_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const float* __restrict__ beta, float* __restrict__ A, float* __restrict__ U,
+                     int N, int S, float cA, float cU) {
+  using namespace c256;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar_full = sb + OFF_BAR;
+  const uint32_t bar_bk = bar_full + 8 * NST;
+  const uint32_t bar_empty = bar_bk + 8 * NST;
+  const uint32_t bar_accf = bar_empty + 8 * NST;
+  const uint32_t bar_acce = bar_accf + 8;
+  const uint32_t bar_fin = bar_acce + 8;
+  uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bar_full + 8 * s, 33);
+      mbar_init(bar_bk + 8 * s, NSC);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    mbar_init(bar_accf, 1);
+    mbar_init(bar_acce, 128);
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int nst_frame = (S + TOK - 1) / TOK;
+  const int NU = 2 * N;
+  const int my_count = (int)blockIdx.x < NU ? (NU - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+  if (warp == 0) {
+    int g = 0;
+    bool ok = true;
+    for (int i = 0; i < my_count && ok; ++i) {
+      const int unit = blockIdx.x + i * gridDim.x, n = unit >> 1, half = unit & 1;
+      for (int st = 0; st < nst_frame; ++st, ++g) {
+        const int s = g % NST;
+        const uint32_t u = (uint32_t)(g / NST);
+        if (lane == 0) ok = mbar_wait(bar_empty + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 101);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar_full + 8 * s, KT + VT);
+#pragma unroll
+          for (int x = 0; x < 4; ++x)
+            tma_load_3d(sb + OFF_K + s * KT + x * BOX, &tmK, bar_full + 8 * s, 64 * x, st * TOK, n);
+#pragma unroll
+          for (int x = 0; x < 2; ++x)
+            tma_load_3d(sb + OFF_V + s * VT + x * BOX, &tmV, bar_full + 8 * s, 128 * half + 64 * x,
+                        st * TOK, n);
+        }
+        const uint32_t bsa = sb + OFF_BETA + s * TOK * 4;
+#pragma unroll
+        for (int r = lane; r < TOK; r += 32) {
+          const int tok = st * TOK + r;
+          const bool in = tok < S;
+          cp_async_4(bsa + r * 4, beta + (size_t)n * S + (in ? tok : 0), in ? 4u : 0u);
+        }
+        cp_async_arrive_noinc(bar_full + 8 * s);
+      }
+    }
+    if (lane == 0)
+      for (int gg = (g > NST ? g - NST : 0); gg < g; ++gg)
+        mbar_wait(bar_full + 8 * (gg % NST), (uint32_t)(gg / NST) & 1, abort_flag, &g_tc_status, 102);
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 256, true, true);
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; i < my_count && ok; ++i) {
+        const int half = (blockIdx.x + i * gridDim.x) & 1;
+        ok = mbar_wait(bar_acce, ((uint32_t)i & 1) ^ 1, abort_flag, &g_tc_status, 103);
+        if (!ok) break;
+        tc_fence_after();
+        for (int st = 0; st < nst_frame; ++st, ++g) {
+          const int s = g % NST;
+          const uint32_t u = (uint32_t)(g / NST);
+          ok = mbar_wait(bar_bk + 8 * s, u & 1, abort_flag, &g_tc_status, 104);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t ka = sb + OFF_K + s * KT + 2 * half * BOX, va = sb + OFF_V + s * VT,
+                         ba = sb + OFF_BK + s * KT;
+#pragma unroll
+          for (int kk = 0; kk < TOK / 16; ++kk) {
+            const uint64_t db = smem_desc_sw128(ba + kk * 2048, BOX, 1024);
+            const uint32_t acc = (st > 0 || kk > 0) ? 1u : 0u;
+            mma_bf16(tmem, smem_desc_sw128(ka + kk * 2048, BOX, 1024), db, idesc, acc);
+            mma_bf16(tmem + 256, smem_desc_sw128(va + kk * 2048, BOX, 1024), db, idesc, acc);
+          }
+          mma_commit(bar_empty + 8 * s);
+        }
+        if (!ok) break;
+        mma_commit(bar_accf);
+      }
+      mma_commit(bar_fin);
+      mbar_wait(bar_fin, 0, abort_flag, &g_tc_status, 105);
+    }
+    __syncwarp();
+  } else if (warp < 2 + NSC / 32) {
+    const int t = threadIdx.x - 64;
+    int g = 0;
+    bool ok = true;
+    for (int i = 0; i < my_count && ok; ++i) {
+      for (int st = 0; st < nst_frame; ++st, ++g) {
+        const int s = g % NST;
+        const uint32_t u = (uint32_t)(g / NST);
+        ok = mbar_wait(bar_full + 8 * s, u & 1, abort_flag, &g_tc_status, 106);
+        if (!ok) break;
+        const uint8_t* kt = smem + OFF_K + s * KT;
+        uint8_t* bt = smem + OFF_BK + s * KT;
+        const float* bs = (const float*)(smem + OFF_BETA) + s * TOK;
+#pragma unroll
+        for (int m = 0; m < (KT / 16) / NSC; ++m) {
+          const int c = t + NSC * m;
+          const float bv = bs[(c >> 3) & (TOK - 1)];
+          uint4 x = *(const uint4*)(kt + c * 16);
+          uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
+            w[e] = pack_bf16x2(f.x * bv, f.y * bv);
+          }
+          *(uint4*)(bt + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async();
+        mbar_arrive(bar_bk + 8 * s);
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    for (int i = 0; i < my_count; ++i) {
+      const int unit = blockIdx.x + i * gridDim.x, n = unit >> 1, half = unit & 1;
+      if (!mbar_wait(bar_accf, (uint32_t)i & 1, abort_flag, &g_tc_status, 107)) break;
+      tc_fence_after();
+#pragma unroll
+      for (int mat = 0; mat < 2; ++mat) {
+        float* dst = (mat ? U : A) + ((size_t)n * D + 128 * half + row) * D;
+        const float sc = mat ? cU : cA;
+        for (int c0 = 0; c0 < 256; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + mat * 256 + c0, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *(float4*)(dst + c0 + 4 * j) =
+                make_float4(__uint_as_float(r[4 * j]) * sc, __uint_as_float(r[4 * j + 1]) * sc,
+                            __uint_as_float(r[4 * j + 2]) * sc, __uint_as_float(r[4 * j + 3]) * sc);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_acce);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+namespace r256 {
+constexpr int D = 256;
+constexpr int TOK = 128;
+constexpr int NQ = 2;
+constexpr int BOX = TOK * 128;           // [128 rows][64 channels]: 16 KiB
+constexpr int QH = 2 * BOX;              // Q half tile (128 channels): 32 KiB
+constexpr int OFF_Q = 0;
+constexpr int OFF_S = OFF_Q + NQ * QH;   // S rows half: hi 4 atoms, lo 4 atoms (128 KiB)
+constexpr int OFF_O = OFF_S + 8 * BOX;   // output staging: 2 boxes
+constexpr int OFF_BAR = OFF_O + 2 * BOX;
+constexpr int NBAR = 2 * NQ + 2 + 4 + 1;
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 256;
+}  // namespace r256
+
+__global__ void __launch_bounds__(r256::THREADS, 1)
+    k_readout256_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
+                    const __grid_constant__ CUtensorMap tmO, int N, int S) {
+  using namespace r256;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar_qf = sb + OFF_BAR;
+  const uint32_t bar_qe = bar_qf + 8 * NQ;
+  const uint32_t bar_sf = bar_qe + 8 * NQ;
+  const uint32_t bar_se = bar_sf + 8;
+  const uint32_t bar_accf = bar_se + 8;
+  const uint32_t bar_acce = bar_accf + 16;
+  const uint32_t bar_fin = bar_acce + 16;
+  uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NQ; ++s) {
+      mbar_init(bar_qf + 8 * s, 1);
+      mbar_init(bar_qe + 8 * s, 1);
+    }
+    mbar_init(bar_sf, 1);
+    mbar_init(bar_se, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_accf + 8 * b, 1);
+      mbar_init(bar_acce + 8 * b, 128);
+    }
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int ntile = (S + TOK - 1) / TOK;
+  const int NU = 2 * N;
+  const int my_count = (int)blockIdx.x < NU ? (NU - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; i < my_count && ok; ++i) {
+        const int unit = blockIdx.x + i * gridDim.x, n = unit >> 1, half = unit & 1;
+        ok = mbar_wait(bar_se, ((uint32_t)i & 1) ^ 1, abort_flag, &g_tc_status, 111);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar_sf, 8 * BOX);
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+          for (int x = 0; x < 4; ++x)
+            tma_load_3d(sb + OFF_S + (4 * hl + x) * BOX, &tmS, bar_sf, 64 * x, 128 * half, 2 * n + hl);
+        for (int tl = 0; tl < ntile && ok; ++tl)
+          for (int kh = 0; kh < 2; ++kh, ++g) {
+            const int s = g % NQ;
+            const uint32_t u = (uint32_t)(g / NQ);
+            ok = mbar_wait(bar_qe + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 112);
+            if (!ok) break;
+            const uint32_t qd = sb + OFF_Q + s * QH;
+            mbar_arrive_expect_tx(bar_qf + 8 * s, QH);
+            tma_load_3d(qd, &tmQ, bar_qf + 8 * s, 128 * kh, tl * TOK, n);
+            tma_load_3d(qd + BOX, &tmQ, bar_qf + 8 * s, 128 * kh + 64, tl * TOK, n);
+          }
+      }
+      for (int gg = (g > NQ ? g - NQ : 0); gg < g; ++gg)
+        mbar_wait(bar_qf + 8 * (gg % NQ), (uint32_t)(gg / NQ) & 1, abort_flag, &g_tc_status, 113);
+      if (my_count > 0) mbar_wait(bar_sf, (uint32_t)(my_count - 1) & 1, abort_flag, &g_tc_status, 114);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+      int g = 0, gt = 0;
+      bool ok = true;
+      for (int i = 0; i < my_count && ok; ++i) {
+        ok = mbar_wait(bar_sf, (uint32_t)i & 1, abort_flag, &g_tc_status, 115);
+        if (!ok) break;
+        tc_fence_after();
+        for (int tl = 0; tl < ntile && ok; ++tl, ++gt) {
+          const int b = gt & 1;
+          const uint32_t ub = (uint32_t)(gt >> 1);
+          ok = mbar_wait(bar_acce + 8 * b, (ub & 1) ^ 1, abort_flag, &g_tc_status, 116);
+          if (!ok) break;
+          const uint32_t d = tmem + b * 128;
+          for (int kh = 0; kh < 2 && ok; ++kh, ++g) {
+            const int s = g % NQ;
+            const uint32_t u = (uint32_t)(g / NQ);
+            ok = mbar_wait(bar_qf + 8 * s, u & 1, abort_flag, &g_tc_status, 117);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t qa = sb + OFF_Q + s * QH;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t qoff = (kk >> 2) * BOX + (kk & 3) * 32;
+              const uint32_t soff = (2 * kh + (kk >> 2)) * BOX + (kk & 3) * 32;
+              const uint64_t dq = smem_desc_sw128(qa + qoff, 16, 1024);
+              mma_bf16(d, dq, smem_desc_sw128(sb + OFF_S + soff, 16, 1024), idesc,
+                       (kh > 0 || kk > 0) ? 1u : 0u);
+              mma_bf16(d, dq, smem_desc_sw128(sb + OFF_S + 4 * BOX + soff, 16, 1024), idesc, 1u);
+            }
+            mma_commit(bar_qe + 8 * s);
+          }
+          if (!ok) break;
+          mma_commit(bar_accf + 8 * b);
+        }
+        if (!ok) break;
+        mma_commit(bar_se);
+      }
+      mma_commit(bar_fin);
+      mbar_wait(bar_fin, 0, abort_flag, &g_tc_status, 118);
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int et = threadIdx.x - 64;
+    uint8_t* ost = smem + OFF_O;
+    int gt = 0;
+    bool ok = true;
+    for (int i = 0; i < my_count && ok; ++i) {
+      const int unit = blockIdx.x + i * gridDim.x, n = unit >> 1, half = unit & 1;
+      for (int tl = 0; tl < ntile; ++tl, ++gt) {
+        const int b = gt & 1;
+        const uint32_t ub = (uint32_t)(gt >> 1);
+        mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 119);
+        tc_fence_after();
+        if (et == 0) bulk_wait_read0();
+        named_bar_sync(1, 128);
+        if (*abort_flag) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+#pragma unroll
+          for (int c0 = 0; c0 < 64; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 128 + hb * 64 + c0, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              *(uint4*)(ost + hb * BOX + row * 128 + ((((c0 >> 3) + j) ^ (row & 7)) << 4)) = make_uint4(
+                  pack_bf16x2(__uint_as_float(r[8 * j]), __uint_as_float(r[8 * j + 1])),
+                  pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3])),
+                  pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5])),
+                  pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7])));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar_acce + 8 * b);
+        fence_proxy_async();
+        named_bar_sync(1, 128);
+        if (et == 0) {
+          tma_store_3d(&tmO, sb + OFF_O, 128 * half, tl * TOK, n);
+          tma_store_3d(&tmO, sb + OFF_O + BOX, 128 * half + 64, tl * TOK, n);
+          bulk_commit();
+        }
+      }
+    }
+    if (et == 0) bulk_wait0();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+static cudaError_t tc_contract256(const void* k, const void* v, const float* beta, float* A,
+                                  float* U, long long N, int S, float cA, float cU,
+                                  cudaStream_t st) {
+  CUtensorMap mk, mv;
+  cudaError_t e = make_map_bf16_3d(&mk, k, 256, S, N, 64, c256::TOK);
+  if (e != cudaSuccess) return e;
+  e = make_map_bf16_3d(&mv, v, 256, S, N, 64, c256::TOK);
+  if (e != cudaSuccess) return e;
+  static bool attr = false;
+  if (!attr) {
+    e = cudaFuncSetAttribute(k_contract256_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, c256::SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const long long units = 2 * N;
+  const int grid = (int)(units < num_sms() ? units : num_sms());
+  k_contract256_tc<<<grid, c256::THREADS, c256::SMEM, st>>>(mk, mv, beta, A, U, (int)N, S, cA, cU);
+  count_launch();
+  return cudaGetLastError();
+}
+
+static cudaError_t tc_readout256(const void* q, const void* Sfr_hilo, void* out, long long N, int S,
+                                 cudaStream_t st) {
+  CUtensorMap mq, ms, mo;
+  cudaError_t e = make_map_bf16_3d(&mq, q, 256, S, N, 64, r256::TOK);
+  if (e == cudaSuccess) e = make_map_bf16_3d(&ms, Sfr_hilo, 256, 256, 2 * N, 64, 128);
+  if (e == cudaSuccess) e = make_map_bf16_3d(&mo, out, 256, S, N, 64, r256::TOK);
+  if (e != cudaSuccess) return e;
+  static bool attr = false;
+  if (!attr) {
+    e = cudaFuncSetAttribute(k_readout256_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, r256::SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const long long units = 2 * N;
+  const int grid = (int)(units < num_sms() ? units : num_sms());
+  k_readout256_tc<<<grid, r256::THREADS, r256::SMEM, st>>>(mq, ms, mo, (int)N, S);
+  count_launch();
+  return cudaGetLastError();
+}
+
 // ---- public entry points of the tensor-core kernels (dispatch on D) ----
 cudaError_t tc_contract(const void* k, const void* v, const float* beta, float* A, float* U,
                         long long N, int S, int D, float cA, float cU, int a_image,
                         const ProArgs* pro, cudaStream_t st) {
+  if (D == 256) {
+    if (pro || a_image) return cudaErrorNotSupported;
+    return tc_contract256(k, v, beta, A, U, N, S, cA, cU, st);
+  }
   if (D == 64) {
     if (pro) return cudaErrorNotSupported;
     CUtensorMap mk, mv;
@@ -2482,6 +2985,10 @@ cudaError_t tc_contract(const void* k, const void* v, const float* beta, float* 
 
 cudaError_t tc_readout(const void* q, const void* Sfr_hilo, void* out, long long N, int S, int D,
                        const ProArgs* pro, cudaStream_t st) {
+  if (D == 256) {
+    if (pro) return cudaErrorNotSupported;
+    return tc_readout256(q, Sfr_hilo, out, N, S, st);
+  }
   if (D == 64) {
     if (pro) return cudaErrorNotSupported;
     CUtensorMap mq, ms, mo;
@@ -2497,8 +3004,10 @@ cudaError_t tc_readout(const void* q, const void* Sfr_hilo, void* out, long long
       if (e != cudaSuccess) return e;
       attr64 = true;
     }
-    const int grid = (int)(N < num_sms() ? N : num_sms());
-    k_readout64_tc<<<grid, r64::THREADS, r64::SMEM, st>>>(mq, ms, mo, (int)N, S);
+    const int parts = readout_parts(N, (S + r64::TOK - 1) / r64::TOK);
+    const long long units = N * parts;
+    const int grid = (int)(units < num_sms() ? units : num_sms());
+    k_readout64_tc<<<grid, r64::THREADS, r64::SMEM, st>>>(mq, ms, mo, (int)N, S, parts);
     count_launch();
     return cudaGetLastError();
   }
