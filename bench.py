@@ -1,13 +1,17 @@
 """Benchmark of the frame-wise GDN frame scan on B200.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                [--config NAME] [--e2e-steps K2] [--no-cpu-baseline]
+                [--config NAME] [--plan auto|chunked|sequential|separate]
+                [--e2e-steps K2] [--no-cpu-baseline]
 
-One step = one full pass of the scan (contraction, chunk composition, prefix,
-replay, readout) over one batch of the workload, inputs resident in HBM. The
-default workload is the 60 s 720p rollout, one GDN layer: B=1, H=16, D=128,
-S=80x45=3600 tokens per latent frame, T=121 latent frames, bf16 q/k/v, fp32
-state, chunk-parallel scan (8-frame spans).
+One step = one full pass of the scan (contraction, the chains of the
+recurrence, readout) over one batch of the workload, inputs resident in HBM.
+The default workload is the 60 s 720p rollout, one GDN layer: B=1, H=16,
+D=128, S=80x45=3600 tokens per latent frame, T=121 latent frames, bf16 q/k/v,
+fp32 state. The default plan is the library's own choice (for this workload:
+the sequential chains running alongside the contraction in one launch);
+--plan chunked times the span-composed scan (8-frame spans), --plan separate
+the sequential chains as their own launch.
 
 Metric: frame·head·tokens/s = B*H*T*S / step time, and the fraction of the
 HBM roofline. Under torchrun (N>1) every rank runs its own copy of the
@@ -69,6 +73,7 @@ def phase_bytes(cfg):
     nro = 2 if cfg.bidir_block else 1
     return {
         "contract": fh * cfg.S * (2 * cfg.D * e + 4),          # K, V, beta
+        "contract_scan": fh * cfg.S * (2 * cfg.D * e + 4),     # same, chains alongside
         "readout": fh * cfg.S * (2 + (1 if cfg.bidir_block else 0)) * cfg.D * e,  # Q in, O (and O_rev) out
         "scan_readout": fh * cfg.S * 2 * cfg.D * e,             # Q in, O out (replay fused)
         "prologue": fh * cfg.S * 4 * cfg.D * e,                 # raw q, k in; q^, k^ out
@@ -247,6 +252,32 @@ def whole_job_value(tokens_per_rank, world, ms_per_step):
     return tokens_per_rank * world / (ms_per_step * 1e-3)
 
 
+PLANS = {
+    "auto": {},
+    "chunked": {"chunked": True},
+    "sequential": {"sequential": True},
+    "separate": {"sequential": True, "overlap": False},
+}
+
+
+def plan_kw(plan):
+    return dict(PLANS[plan])
+
+
+def plan_desc(plan, phases):
+    """What ran: read from the phases the library recorded."""
+    ran = {p for p in phases if phases[p][1] > 0}
+    if "contract_scan" in ran:
+        how = "sequential chains alongside the contraction (one cooperative launch)"
+    elif "compose" in ran:
+        how = "chunked (8-frame spans, composed)"
+    elif "scan_readout" in ran:
+        how = "spans replayed inside the readout"
+    else:
+        how = "sequential chains (own launch)"
+    return f"{how}; plan {plan}"
+
+
 def run_ours(args, cfg):
     import torch
     from frame_wise_gated_b200 import api, build
@@ -286,15 +317,14 @@ def run_ours(args, cfg):
         pro = dict(w_q=torch.from_numpy(arr["w_q"]).to(dev), w_k=torch.from_numpy(arr["w_k"]).to(dev),
                    grid_h=cfg.grid_h, grid_w=cfg.grid_w)
     kw = dict(prologue=pro, bidir=bool(cfg.bidir_block), block_reset=bool(cfg.bidir_block),
-              block=cfg.bidir_block or 3, sequential=args.sequential,
-              fused_replay=args.fused_replay)
+              block=cfg.bidir_block or 3, fused_replay=args.fused_replay, **plan_kw(args.plan))
     out = torch.empty_like(q)
     out_rev = torch.empty_like(q) if cfg.bidir_block else None
     st_out = torch.empty((cfg.B, cfg.H, cfg.D, cfg.D), device=dev, dtype=torch.float32)
     st_rev = torch.empty_like(st_out) if cfg.bidir_block else None
     flags = api.scan_flags(bf16=cfg.bf16, prologue=pro is not None, bidir=bool(cfg.bidir_block),
                            block_reset=bool(cfg.bidir_block), block=cfg.bidir_block or 3,
-                           sequential=args.sequential, fused_replay=args.fused_replay)
+                           fused_replay=args.fused_replay, **plan_kw(args.plan))
     ws = torch.empty(api.workspace_bytes(cfg.B, cfg.H, cfg.T, cfg.S, cfg.D, flags),
                      device=dev, dtype=torch.uint8)
     stream = torch.cuda.current_stream(dev)
@@ -374,7 +404,7 @@ def run_ours(args, cfg):
             "dtype": "bf16" if cfg.bf16 else "f32", "data": "synthetic",
             "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "T": cfg.T, "S": cfg.S,
                        "D": cfg.D, "grid": f"{cfg.grid_w}x{cfg.grid_h}",
-                       "scan": "sequential" if args.sequential else "chunked (8-frame spans)",
+                       "scan": plan_desc(args.plan, phases),
                        "prologue": cfg.prologue, "bidir_block": cfg.bidir_block,
                        "l2": f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB algorithmic per step)",
                        "parallelism": f"replica x{world} (heads shard, no collective)"},
@@ -423,7 +453,7 @@ def run_e2e(args, cfg, arr, dev, api, barrier, dist, world):
         if ds0 is not None:
             ds0.copy_(hs0, non_blocking=True)
         api.frame_scan_fwd(dq, dk, dv, db, dg, ds0, out=dout, state_out=dst,
-                           sequential=args.sequential)
+                           **plan_kw(args.plan))
         hout.copy_(dout, non_blocking=True)
         hst.copy_(dst, non_blocking=True)
 
@@ -453,7 +483,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="rollout60s_720p", choices=sorted(synth.CONFIGS))
-    ap.add_argument("--sequential", action="store_true")
+    ap.add_argument("--plan", choices=sorted(PLANS), default="auto",
+                    help="scan plan: the library's choice, spans, or sequential chains "
+                         "(alongside the contraction, or as their own launch)")
     ap.add_argument("--fused-replay", action="store_true",
                     help="replay spans inside the readout kernel")
     ap.add_argument("--e2e-steps", type=int, default=5)

@@ -33,6 +33,8 @@ KEYS_SCALED = 0x20
 FORCE_SIMT = 0x40
 BIDIR = 0x80
 FUSED_REPLAY = 0x1000000
+CHUNKED = 0x2000000
+NO_OVERLAP = 0x4000000
 
 
 def make_block(n: int) -> int:
@@ -87,7 +89,8 @@ SIGNATURES = {
     "gdn_profile_read": (_I, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong), _I]),
 }
 
-PHASES = ("prologue", "contract", "compose", "prefix", "scan", "readout", "scan_readout")
+PHASES = ("prologue", "contract", "compose", "prefix", "scan", "readout", "scan_readout",
+          "contract_scan")
 
 _lib = None
 
@@ -137,8 +140,13 @@ def _want(t: torch.Tensor, name: str, dtype=None, shape=None):
 
 def scan_flags(*, bf16: bool, reverse=False, block_reset=False, block=3, chunk=8,
                sequential=False, keys_scaled=False, force_simt=False, prologue=False,
-               bidir=False, fused_replay=False) -> int:
+               bidir=False, fused_replay=False, chunked=False, overlap=True) -> int:
+    """Flag word of the C ABI. Plan: sequential=True forces one chain per head,
+    chunked=True the span-composed plan, neither lets the library choose;
+    overlap=False keeps the chains out of the contraction's launch."""
     f = (BF16 if bf16 else 0) | make_block(block) | make_chunk(chunk)
+    f |= CHUNKED if chunked else 0
+    f |= 0 if overlap else NO_OVERLAP
     f |= FUSED_REPLAY if fused_replay else 0
     f |= REVERSE if reverse else 0
     f |= BLOCK_RESET if block_reset else 0
@@ -156,8 +164,9 @@ def workspace_bytes(B, H, T, S, D, flags) -> int:
 
 def frame_scan_fwd_ex(q, k, v, beta, gamma, state_in=None, *, reverse=False, block_reset=False,
                       block=3, chunk=8, sequential=False, keys_scaled=False, force_simt=False,
-                      prologue=None, bidir=False, fused_replay=False, out=None, state_out=None,
-                      out_rev=None, state_out_rev=None, workspace=None, stream=None):
+                      prologue=None, bidir=False, fused_replay=False, chunked=False,
+                      overlap=True, out=None, state_out=None, out_rev=None, state_out_rev=None,
+                      workspace=None, stream=None):
     """The frame scan through gdn_frame_scan_fwd_ex.
 
     q, k, v [B,H,T,S,D] (bf16 or fp32); beta [B,H,T,S] fp32; gamma [B,H,T]
@@ -178,7 +187,7 @@ def frame_scan_fwd_ex(q, k, v, beta, gamma, state_in=None, *, reverse=False, blo
     flags = scan_flags(bf16=bf16, reverse=reverse, block_reset=block_reset, block=block,
                        chunk=chunk, sequential=sequential, keys_scaled=keys_scaled,
                        force_simt=force_simt, prologue=prologue is not None, bidir=bidir,
-                       fused_replay=fused_replay)
+                       fused_replay=fused_replay, chunked=chunked, overlap=overlap)
     out = torch.empty_like(q) if out is None else out
     state_out = torch.empty((B, H, D, D), device=q.device, dtype=torch.float32) \
         if state_out is None else state_out
@@ -212,7 +221,7 @@ def frame_scan_fwd_ex(q, k, v, beta, gamma, state_in=None, *, reverse=False, blo
 
 def frame_scan_fwd(q, k, v, beta, gamma, state_in=None, *, reverse=False, block_reset=False,
                    block=3, chunk=8, sequential=False, keys_scaled=False, force_simt=False,
-                   out=None, state_out=None, stream=None):
+                   chunked=False, overlap=True, out=None, state_out=None, stream=None):
     """The frame scan through gdn_frame_scan_fwd (scratch allocated by the
     library, stream-ordered). Returns (out, state_out)."""
     B, H, T, S, D = q.shape
@@ -222,7 +231,8 @@ def frame_scan_fwd(q, k, v, beta, gamma, state_in=None, *, reverse=False, block_
     _want(gamma, "gamma", torch.float32, (B, H, T))
     flags = scan_flags(bf16=q.dtype == torch.bfloat16, reverse=reverse, block_reset=block_reset,
                        block=block, chunk=chunk, sequential=sequential,
-                       keys_scaled=keys_scaled, force_simt=force_simt)
+                       keys_scaled=keys_scaled, force_simt=force_simt, chunked=chunked,
+                       overlap=overlap)
     out = torch.empty_like(q) if out is None else out
     state_out = torch.empty((B, H, D, D), device=q.device, dtype=torch.float32) \
         if state_out is None else state_out
@@ -237,8 +247,8 @@ STATIC_SCRATCH_BYTES = 32 << 20
 
 def frame_scan_fwd_static(q, k, v, beta, gamma, state_in=None, *, reverse=False,
                           block_reset=False, block=3, chunk=8, sequential=False,
-                          keys_scaled=False, force_simt=False, out=None, state_out=None,
-                          stream=None):
+                          keys_scaled=False, force_simt=False, chunked=False, overlap=True,
+                          out=None, state_out=None, stream=None):
     """The frame scan through gdn_frame_scan_fwd_static: for callers that must
     not allocate device memory per call (e.g. a streaming loop running one
     short block of frames at a time). Scratch is the library's fixed 32 MiB
@@ -251,7 +261,8 @@ def frame_scan_fwd_static(q, k, v, beta, gamma, state_in=None, *, reverse=False,
     _want(gamma, "gamma", torch.float32, (B, H, T))
     flags = scan_flags(bf16=q.dtype == torch.bfloat16, reverse=reverse, block_reset=block_reset,
                        block=block, chunk=chunk, sequential=sequential,
-                       keys_scaled=keys_scaled, force_simt=force_simt)
+                       keys_scaled=keys_scaled, force_simt=force_simt, chunked=chunked,
+                       overlap=overlap)
     out = torch.empty_like(q) if out is None else out
     state_out = torch.empty((B, H, D, D), device=q.device, dtype=torch.float32) \
         if state_out is None else state_out

@@ -31,7 +31,7 @@ void count_launch(int n) { t_launches += n; }
 // ---- phase timing with CUDA events (gdn_profile_enable / gdn_profile_read) ----
 enum Phase {
   PH_PROLOGUE = 0, PH_CONTRACT, PH_COMPOSE, PH_PREFIX, PH_SCAN, PH_READOUT, PH_SCAN_READOUT,
-  PH_COUNT
+  PH_CONTRACT_SCAN, PH_COUNT
 };
 struct ProfRec {
   int phase;
@@ -131,6 +131,8 @@ Layout make_layout(int B, int H, int T, int S, int D, unsigned flags) {
   off = align256(off + heads * L.nseg_max * mat);
   L.g = off;
   off = align256(off + heads * L.nseg_max * sizeof(float));
+  L.flags = off;  // per frame-head publication counters of the overlapped plan
+  off = align256(off + frames * sizeof(int));
   L.qh = L.kh = L.rope = off;
   if (flags & GDN_FUSED_PROLOGUE) {
     L.rope = off;  // (cos, sin) table: positions [0, S) x pairs [0, D/4)
@@ -282,6 +284,8 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
     return fail(GDN_ERR_INVALID, "GDN_BIDIR needs a separate, aligned out_rev%s");
   if ((f & GDN_BIDIR) && (f & GDN_REVERSE))
     return fail(GDN_ERR_INVALID, "GDN_BIDIR and GDN_REVERSE are exclusive%s");
+  if ((f & GDN_SEQUENTIAL) && (f & GDN_CHUNKED))
+    return fail(GDN_ERR_INVALID, "GDN_SEQUENTIAL and GDN_CHUNKED are exclusive%s");
   if (f & GDN_FUSED_PROLOGUE) {
     if (!p.w_q || !p.w_k) return fail(GDN_ERR_INVALID, "prologue needs w_q and w_k%s");
     if (p.grid_h < 1 || p.grid_w < 1 || (long long)p.grid_h * p.grid_w != p.S)
@@ -300,6 +304,7 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
   const bool simt = (f & GDN_FORCE_SIMT) || !bf16 || !sm100;
   const bool tc_contract_ok = !simt && tc_contract_supported(p.D);
   const bool tc_readout_ok = !simt && tc_readout_supported(p.D);
+  const bool seq_plan = (f & GDN_SEQUENTIAL) != 0;
   const bool tc_chain_ok = !simt && tc_chain_supported(p.D);
   char* ws = (char*)p.workspace;
   const long long frames = (long long)p.B * p.H * p.T;
@@ -346,6 +351,50 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
   const double c = keys_scaled ? 1.0 : 1.0 / std::sqrt((double)p.D * (double)p.S);
   float* A = (float*)(ws + L.A);
   float* U = (float*)(ws + L.U);
+  const bool block_reset = (f & GDN_BLOCK_RESET) != 0;
+
+  // Sequential chains alongside the contraction (one cooperative launch),
+  // then the readout: the plan unless chunks or separate launches are asked
+  // for, or the shape does not fit it.
+  const bool bidir = (f & GDN_BIDIR) != 0;
+  const int ndir = bidir ? 2 : 1;
+  const bool overlap = tc_contract_ok && tc_chain_ok && tc_readout_ok &&
+                       tc_overlap_supported(p.D) && !(f & (GDN_CHUNKED | GDN_NO_OVERLAP |
+                                                          GDN_FUSED_REPLAY)) &&
+                       (!bidir || (block_reset && tc_readout2_supported(p.D))) &&
+                       ndir * p.B * p.H <= tc_overlap_max_chains();
+  if (overlap) {
+    OvlArgs o;
+    memset(&o, 0, sizeof(o));
+    o.heads = p.B * p.H;
+    o.T = p.T;
+    o.block = block_len(f);
+    o.ndir = ndir;
+    o.gamma = p.gamma;
+    o.A = (const uint8_t*)A;
+    o.flags = (int*)(ws + L.flags);
+    if (bidir) {
+      // forward never reset; reverse reset per block, run block by block
+      o.dir[0] = OvlDir{0, 0, 0, p.state_in, p.state_out};
+      o.dir[1] = OvlDir{1, 1, 0, p.state_in, p.state_out_rev};
+    } else {
+      o.dir[0] = OvlDir{(f & GDN_REVERSE) ? 1 : 0, 0, block_reset ? 1 : 0, p.state_in,
+                        p.state_out};
+    }
+    {
+      PhaseScope ps(PH_CONTRACT_SCAN, st);
+      e = tc_contract_scan(k, p.v, p.beta, A, U, frames, p.S, (float)(c * c), (float)c, ppk, o,
+                           ws + L.Sfr, bidir ? ws + L.Sfr2 : nullptr, st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "contract + sequential scan");
+    PhaseScope ps(PH_READOUT, st);
+    if (bidir)
+      e = tc_readout2(q, ws + L.Sfr, ws + L.Sfr2, p.out, p.out_rev, frames, p.S, p.D, ppq, st);
+    else
+      e = tc_readout(q, ws + L.Sfr, p.out, frames, p.S, p.D, ppq, st);
+    if (e != cudaSuccess) return cuda_fail(e, "readout");
+    return GDN_OK;
+  }
   {
     PhaseScope ps(PH_CONTRACT, st);
     if (tc_contract_ok)
@@ -357,15 +406,16 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
   }
   if (e != cudaSuccess) return cuda_fail(e, "contract");
 
-  const bool block_reset = (f & GDN_BLOCK_RESET) != 0;
+  gdn_params pp = p;
+  if (seq_plan) pp.flags |= GDN_SEQUENTIAL;
   if (f & GDN_BIDIR) {
     // Both directions' states first, then (tensor-core path) one readout that
     // reads each Q tile once for both outputs.
     const bool both = tc_readout_ok && tc_chain_ok && tc_readout2_supported(p.D);
-    rc = run_direction(p, L, ws, false, false, q, p.out, p.state_out, tc_chain_ok,
+    rc = run_direction(pp, L, ws, false, false, q, p.out, p.state_out, tc_chain_ok,
                        tc_readout_ok, ppq, st, L.Sfr, !both);
     if (rc) return rc;
-    rc = run_direction(p, L, ws, true, block_reset, q, p.out_rev, p.state_out_rev, tc_chain_ok,
+    rc = run_direction(pp, L, ws, true, block_reset, q, p.out_rev, p.state_out_rev, tc_chain_ok,
                        tc_readout_ok, ppq, st, L.Sfr2, !both);
     if (rc || !both) return rc;
     PhaseScope ps(PH_READOUT, st);
@@ -373,7 +423,7 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
     if (e != cudaSuccess) return cuda_fail(e, "bidirectional readout");
     return GDN_OK;
   }
-  return run_direction(p, L, ws, (f & GDN_REVERSE) != 0, block_reset, q, p.out, p.state_out,
+  return run_direction(pp, L, ws, (f & GDN_REVERSE) != 0, block_reset, q, p.out, p.state_out,
                        tc_chain_ok, tc_readout_ok, ppq, st, L.Sfr, true);
 }
 

@@ -106,7 +106,7 @@ __host__ __device__ __forceinline__ void seg_range(const ChainArgs& a, int p, in
 
 // ---- workspace layout ---------------------------------------------------------
 struct Layout {
-  size_t A, U, Sfr, Sfr2, E, Hc, g, Sst, qh, kh, rope, total;
+  size_t A, U, Sfr, Sfr2, E, Hc, g, Sst, qh, kh, rope, flags, total;
   int nseg_max;
 };
 
@@ -161,6 +161,34 @@ bool tc_readout2_supported(int D);
 cudaError_t tc_readout2(const void* q, const void* sfr_f, const void* sfr_r, void* out_f,
                         void* out_r, long long N, int S, int D, const ProArgs* pro,
                         cudaStream_t st);
+// ---- contraction with the sequential scan alongside (one cooperative launch) ----
+// One direction of the overlapped scan.
+struct OvlDir {
+  int reverse;     // scan order T-1 .. 0
+  int blocks_asc;  // reverse scan reset per block, run block by block in
+                   // ascending time (frames descending inside each block)
+  int seq_reset;   // zero the state on entering a new block in scan order
+  const float* state_in;  // [heads, D, D] or null
+  float* state_out;       // [heads, D, D] or null
+};
+
+struct OvlArgs {
+  int heads, T, block, ndir;
+  const float* gamma;
+  const uint8_t* A;  // operand images of A_t, [heads*T][kImageBytes]
+  int* flags;        // [heads*T], zero before the launch
+  OvlDir dir[2];
+};
+
+bool tc_overlap_supported(int D);
+// Most chains one overlapped launch runs (the rest of the SMs contract).
+int tc_overlap_max_chains();
+// Contraction of all frame-heads (A_t as operand images, U_t fp32) while
+// o.ndir * o.heads CTAs run the sequential chains, storing each frame's state
+// as a bf16 (hi, lo) pair into sfr0 (direction 0) / sfr1 (direction 1).
+cudaError_t tc_contract_scan(const void* k, const void* v, const float* beta, float* A, float* U,
+                             long long N, int S, float cA, float cU, const ProArgs* pro,
+                             const OvlArgs& o, void* sfr0, void* sfr1, cudaStream_t st);
 bool tc_chain_supported(int D);
 cudaError_t tc_chain(const ChainArgs& a, int nchains, cudaStream_t st);
 cudaError_t tc_selftest_wait(int arrive, long long limit_ns, cudaStream_t st);

@@ -182,10 +182,18 @@ constexpr int THREADS = 64 + NSC + 128;  // producer, MMA, 8 scaler warps, 4 epi
 constexpr uint32_t TMEM_COLS = 512;
 }  // namespace ctr
 
-__global__ void __launch_bounds__(ctr::THREADS, 1)
-    k_contract_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                  const float* __restrict__ beta, float* __restrict__ A, float* __restrict__ U,
-                  int N, int S, float cA, float cU, int a_image, ProArgs pro) {
+// Body of the contraction for CTA `cta` of `ncta` contraction CTAs. Units are
+// frame-heads in order n, or, when `heads` > 0, in scan order across heads
+// (unit u -> head u % heads, scan position u / heads of T: frame u / heads, or
+// T - 1 - u / heads when `rev`). With `flags`, each of the 4 epilogue warps
+// publishes its rows of A_t, U_t by a release increment of flags[n], so a
+// concurrent scan may read frame-head n once flags[n] reaches 4. Warps beyond
+// the contraction's 14 (when the block is larger) only join the barriers.
+__device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                              const float* __restrict__ beta, float* __restrict__ A,
+                                              float* __restrict__ U, int N, int S, float cA,
+                                              float cU, int a_image, const ProArgs& pro, int cta,
+                                              int ncta, int heads, int T, int rev, int* flags) {
   using namespace ctr;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -216,7 +224,7 @@ __global__ void __launch_bounds__(ctr::THREADS, 1)
   }
   float2* tab = (float2*)(smem + OFF_TAB);
   if (pro.w)
-    for (int e = threadIdx.x; e < pro.npos * (D / 4); e += THREADS) tab[e] = pro.cs[e];
+    for (int e = threadIdx.x; e < pro.npos * (D / 4); e += (int)blockDim.x) tab[e] = pro.cs[e];
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
     tmem_relinquish();
@@ -226,14 +234,20 @@ __global__ void __launch_bounds__(ctr::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const int nst_frame = (S + TOK - 1) / TOK;
-  const int my_count = (int)blockIdx.x < N ? (N - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int my_count = cta < N ? (N - 1 - cta) / ncta + 1 : 0;
+  auto unit_n = [&](int i) -> int {
+    const int u = cta + i * ncta;
+    if (heads <= 0) return u;
+    const int j = u / heads;
+    return (u % heads) * T + (rev ? T - 1 - j : j);
+  };
 
   if (warp == 0) {
     // ---- TMA producer (lane 0 issues; the warp loads beta) ----
     int g = 0;
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
-      const int n = blockIdx.x + i * gridDim.x;
+      const int n = unit_n(i);
       for (int st = 0; st < nst_frame; ++st, ++g) {
         const int s = g % NST;
         const uint32_t u = (uint32_t)(g / NST);
@@ -362,16 +376,20 @@ __global__ void __launch_bounds__(ctr::THREADS, 1)
         mbar_arrive(bar_bk + 8 * s);
       }
     }
-  } else {
+  } else if (warp < 2 + NSC / 32 + 4) {
     // ---- epilogue: TMEM -> scale -> fp32 A_t, U_t rows ----
     const int q = warp & 3;
     const int row = q * 32 + lane;
     for (int i = 0; i < my_count; ++i) {
       const int b = i & 1;
       const uint32_t ub = (uint32_t)(i >> 1);
-      if (!mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 7)) break;
+      // lane 0 waits and the warp follows its decision (warp-uniform control flow)
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 7);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      __syncwarp();
       tc_fence_after();
-      const int n = blockIdx.x + i * gridDim.x;
+      const int n = unit_n(i);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         float* dst = (half ? U : A) + ((size_t)n * D + row) * D;
@@ -413,6 +431,15 @@ __global__ void __launch_bounds__(ctr::THREADS, 1)
       }
       tc_fence_before();
       mbar_arrive(bar_acce + 8 * b);
+      if (flags) {
+        // publish this warp's rows of A_t, U_t: its stores, made visible to
+        // other CTAs' bulk/TMA loads (async proxy), then a release increment
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __threadfence();
+        __syncwarp();
+        if (lane == 0)
+          asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(flags + n), "r"(1) : "memory");
+      }
     }
   }
 
@@ -422,6 +449,14 @@ __global__ void __launch_bounds__(ctr::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
+}
+
+__global__ void __launch_bounds__(ctr::THREADS, 1)
+    k_contract_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const float* __restrict__ beta, float* __restrict__ A, float* __restrict__ U,
+                  int N, int S, float cA, float cU, int a_image, ProArgs pro) {
+  contract_body(tmK, tmV, beta, A, U, N, S, cA, cU, a_image, pro, blockIdx.x, gridDim.x, 0, 0, 0,
+                nullptr);
 }
 
 bool tc_contract_supported(int D) { return D == 128 || D == 64 || D == 256; }
@@ -1536,6 +1571,327 @@ static cudaError_t tc_chain128(const ChainArgs& a, int nchains, cudaStream_t st)
 }
 
 // ============================================================================
+// Contraction and sequential scan in one launch (steps a2 and a5 side by
+// side), D = 128.
+//
+// The contraction is bound by HBM bandwidth and the sequential chain by the
+// latency of its steps, so on one GPU they run together: CTAs [0, nchain)
+// each run one chain of the recurrence over the frames of one head, while the
+// other CTAs run the contraction over frame-heads in scan order (all heads of
+// a frame before the next frame). Each contraction epilogue warp publishes its
+// rows of A_t, U_t with a release increment of flags[n]; a chain fetches
+// frame-head n's operands once flags[n] reaches 4. The launch is cooperative,
+// so every CTA is resident and a chain never waits on a CTA that cannot run;
+// every wait is bounded.
+//
+// Chain CTAs use 16 warps: warp w holds rows 32 (w % 4) .. +31 (its TMEM lane
+// quadrant) and columns 32 (w / 4) .. +31 of the fp32 state. Per step one
+// thread issues P = X_hi Y_hi + X_lo Y_hi + X_hi Y_lo (as the chain kernel
+// above), the warps apply X <- gamma (X - P) + U_t, write X back into the
+// operand tile as a bf16 (hi, lo) pair and one thread stores that tile (the
+// state after frame t) by TMA for the readout.
+// ============================================================================
+namespace ovl {
+constexpr int THREADS = 512;
+constexpr int SMEM = ctr::SMEM > chn::SMEM ? ctr::SMEM : chn::SMEM;
+constexpr int EPI_WARPS = 4;  // contraction epilogue warps: publishes per frame-head
+}  // namespace ovl
+
+// Scan step j of a direction: its frame, whether the state entering it is
+// replaced (by state_in when `seed`, else by zeros) and whether the state after
+// it is the direction's final state.
+struct OvlStep {
+  int t, reset, seed, last;
+};
+
+__device__ __forceinline__ OvlStep ovl_step(const OvlDir& d, int T, int block, int j) {
+  OvlStep s;
+  if (d.blocks_asc) {
+    const int b = j / block, o = j - b * block;
+    const int t1 = min(b * block + block, T);
+    s.t = t1 - 1 - o;
+    s.reset = o == 0;
+    s.seed = o == 0 && t1 == T;  // the block holding frame T-1 comes first in scan order
+    s.last = s.t == 0;
+  } else {
+    s.t = d.reverse ? T - 1 - j : j;
+    const int tp = d.reverse ? s.t + 1 : s.t - 1;
+    s.reset = j == 0 || (d.seq_reset && (s.t / block) != (tp / block));
+    s.seed = j == 0;
+    s.last = j == T - 1;
+  }
+  return s;
+}
+
+// Bounded wait until *f >= target (acquire); false on abort or timeout.
+__device__ __forceinline__ bool wait_flag_ge(const int* f, int target, volatile int* abort_flag,
+                                             int code) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+  if (v >= target) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    if (v >= target) return true;
+    if ((it & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > kWaitNs) {
+        atomicExch(&g_tc_status, code);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// 32 consecutive fp32 values of a row (16-byte aligned), or zeros.
+__device__ __forceinline__ void load_row32(const float* src, float* x) {
+  if (!src) {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) x[c] = 0.f;
+    return;
+  }
+#pragma unroll
+  for (int c = 0; c < 32; c += 4) {
+    const float4 f = __ldg((const float4*)(src + c));
+    x[c] = f.x; x[c + 1] = f.y; x[c + 2] = f.z; x[c + 3] = f.w;
+  }
+}
+
+// The thread's 32 state values (row `row`, columns 32 cg ..) into the X tile
+// as bf16 (hi, lo): atom cg / 2, 16-byte chunks 4 (cg % 2) .. +3.
+__device__ __forceinline__ void ovl_store_x(const float* x, uint8_t* xh, uint8_t* xl, int row,
+                                            int cg) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 hi, lo;
+    split_chunk(x + 8 * i, &hi, &lo);
+    const int off = tile_off(row, cg >> 1, 4 * (cg & 1) + i);
+    *(uint4*)(xh + off) = hi;
+    *(uint4*)(xl + off) = lo;
+  }
+}
+
+// Chain role of the overlapped launch: chain c = direction c / heads, head c % heads.
+__device__ __forceinline__ void ovl_chain_body(const OvlArgs& o, const CUtensorMap& tmZ,
+                                               const CUtensorMap& tmS0, const CUtensorMap& tmS1,
+                                               int c) {
+  using namespace chn;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q = warp & 3, cg = warp >> 2;
+  const int row = q * 32 + lane;
+  const bool leader = threadIdx.x == 0;
+  const uint32_t bar_mma = sb + OFF_BAR;
+  const uint32_t bar_y = bar_mma + 8;
+  const uint32_t bar_z = bar_mma + 16;
+  uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
+  const int di = c / o.heads, bh = c % o.heads;
+  const OvlDir d = di ? o.dir[1] : o.dir[0];
+  const CUtensorMap* tmS = di ? &tmS1 : &tmS0;
+  const int T = o.T;
+  const size_t DD = (size_t)D * D;
+
+  if (leader) {
+    mbar_init(bar_mma, 1);
+    mbar_init(bar_y, 1);
+    mbar_init(bar_z, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  // operands of the frame at scan step j: wait for its publication, then copy
+  int ny = 0, nz = 0, nstore = 0;  // copies issued (leader)
+  auto fetch_y = [&](int t) -> bool {
+    const int n = bh * T + t;
+    if (!wait_flag_ge(o.flags + n, ovl::EPI_WARPS, abort_flag, 31)) return false;
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    chain_fetch_y(sb + OFF_Y, o.A + (size_t)n * kImageBytes, bar_y);
+    ++ny;
+    return true;
+  };
+  auto fetch_z = [&](int t) {
+    const int n = bh * T + t;
+    mbar_arrive_expect_tx(bar_z, kImageBytes);
+#pragma unroll
+    for (int b = 0; b < 4; ++b) tma_load_3d(sb + OFF_Z + b * ATOM, &tmZ, bar_z, 32 * b, 0, n);
+    ++nz;
+  };
+  if (leader && T > 0) {
+    const int t0 = ovl_step(d, T, o.block, 0).t;
+    if (fetch_y(t0)) fetch_z(t0);
+  }
+
+  float x[32];
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, true);
+  for (int j = 0; j < T; ++j) {
+    const OvlStep st = ovl_step(d, T, o.block, j);
+    if (st.reset) {
+      // the state entering this step is replaced; the tile must be free first
+      if (leader && nstore > 0) bulk_wait_read0();
+      __syncthreads();
+      const float* init = st.seed && d.state_in ? d.state_in + (size_t)bh * DD : nullptr;
+      load_row32(init ? init + (size_t)row * D + 32 * cg : nullptr, x);
+      ovl_store_x(x, smem + OFF_XH, smem + OFF_XL, row, cg);
+      fence_proxy_async();
+    }
+    mbar_wait(bar_y, (uint32_t)j & 1, abort_flag, &g_tc_status, 32);
+    __syncthreads();
+    if (*abort_flag) break;  // uniform: read after the barrier
+    if (leader) {
+      tc_fence_after();
+      const uint32_t yh = sb + OFF_Y, yl = yh + 2 * ATOM;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t xo = (kk >> 2) * ATOM + (kk & 3) * 32;
+        const uint64_t dxh = smem_desc_sw128(sb + OFF_XH + xo, 16, 1024);
+        const uint64_t dxl = smem_desc_sw128(sb + OFF_XL + xo, 16, 1024);
+        const uint64_t dyh = smem_desc_sw128(yh + kk * 2048, ATOM, 1024);
+        const uint64_t dyl = smem_desc_sw128(yl + kk * 2048, ATOM, 1024);
+        mma_bf16(tmem, dxh, dyh, idesc, kk > 0 ? 1u : 0u);
+        mma_bf16(tmem, dxl, dyh, idesc, 1u);
+        mma_bf16(tmem, dxh, dyl, idesc, 1u);
+      }
+      mma_commit(bar_mma);
+    }
+    mbar_wait(bar_mma, (uint32_t)j & 1, abort_flag, &g_tc_status, 33);
+    tc_fence_after();
+    // the Y buffer is free: the next frame's A_t image, once published
+    int tn = -1;
+    if (j + 1 < T) tn = ovl_step(d, T, o.block, j + 1).t;
+    if (leader && tn >= 0) fetch_y(tn);
+    mbar_wait(bar_z, (uint32_t)j & 1, abort_flag, &g_tc_status, 34);
+    {
+      const float alpha = o.gamma[(size_t)bh * T + st.t];
+      uint32_t r[32];
+      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 32 * cg, r);
+      tmem_wait_ld();
+      const uint8_t* zb = smem + OFF_Z + cg * ATOM + row * 128;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        const float4 z = *(const float4*)(zb + ((ch ^ (row & 7)) << 4));
+        x[4 * ch] = alpha * (x[4 * ch] - __uint_as_float(r[4 * ch])) + z.x;
+        x[4 * ch + 1] = alpha * (x[4 * ch + 1] - __uint_as_float(r[4 * ch + 1])) + z.y;
+        x[4 * ch + 2] = alpha * (x[4 * ch + 2] - __uint_as_float(r[4 * ch + 2])) + z.z;
+        x[4 * ch + 3] = alpha * (x[4 * ch + 3] - __uint_as_float(r[4 * ch + 3])) + z.w;
+      }
+    }
+    tc_fence_before();
+    // every thread has read Z and P; the previous state store has read the tile
+    if (leader && nstore > 0) bulk_wait_read0();
+    __syncthreads();
+    if (leader && tn >= 0 && !*abort_flag) fetch_z(tn);
+    ovl_store_x(x, smem + OFF_XH, smem + OFF_XL, row, cg);
+    fence_proxy_async();
+    if (st.last && d.state_out) {
+      float* so = d.state_out + (size_t)bh * DD + (size_t)row * D + 32 * cg;
+#pragma unroll
+      for (int c4 = 0; c4 < 32; c4 += 4)
+        *(float4*)(so + c4) = make_float4(x[c4], x[c4 + 1], x[c4 + 2], x[c4 + 3]);
+    }
+    __syncthreads();
+    if (leader) {
+      // the state after frame t, as a bf16 (hi, lo) pair, for the readout
+      const int pair = bh * T + st.t;
+      tma_store_3d(tmS, sb + OFF_XH, 0, 0, 2 * pair);
+      tma_store_3d(tmS, sb + OFF_XH + ATOM, 64, 0, 2 * pair);
+      tma_store_3d(tmS, sb + OFF_XL, 0, 0, 2 * pair + 1);
+      tma_store_3d(tmS, sb + OFF_XL + ATOM, 64, 0, 2 * pair + 1);
+      bulk_commit();
+      ++nstore;
+    }
+  }
+  // Drain (bounded, and not cut short by an abort): copies in flight land
+  // before teardown.
+  if (leader) {
+    volatile int keep_waiting = 0;
+    if (nstore > 0) bulk_wait0();
+    if (ny > 0) mbar_wait(bar_y, (uint32_t)(ny - 1) & 1, &keep_waiting, &g_tc_status, 35);
+    if (nz > 0) mbar_wait(bar_z, (uint32_t)(nz - 1) & 1, &keep_waiting, &g_tc_status, 36);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+__global__ void __launch_bounds__(ovl::THREADS, 1)
+    k_contract_scan_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                       const float* __restrict__ beta, float* __restrict__ A, float* __restrict__ U,
+                       int N, int S, float cA, float cU, ProArgs pro, OvlArgs o, int nchain,
+                       const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmS0,
+                       const __grid_constant__ CUtensorMap tmS1) {
+  if ((int)blockIdx.x < nchain)
+    ovl_chain_body(o, tmZ, tmS0, tmS1, blockIdx.x);
+  else
+    contract_body(tmK, tmV, beta, A, U, N, S, cA, cU, 1, pro, (int)blockIdx.x - nchain,
+                  (int)gridDim.x - nchain, o.heads, o.T, o.dir[0].reverse && !o.dir[0].blocks_asc,
+                  o.flags);
+}
+
+bool tc_overlap_supported(int D) { return D == 128; }
+int tc_overlap_max_chains() { return num_sms() / 4; }
+
+cudaError_t tc_contract_scan(const void* k, const void* v, const float* beta, float* A, float* U,
+                             long long N, int S, float cA, float cU, const ProArgs* pro,
+                             const OvlArgs& o, void* sfr0, void* sfr1, cudaStream_t st) {
+  if (pro && pro->npos * (128 / 4) > ctr::TAB_MAX) return cudaErrorNotSupported;
+  const int nchain = o.ndir * o.heads;
+  if (o.ndir < 1 || o.ndir > 2 || nchain > tc_overlap_max_chains() ||
+      (long long)o.heads * o.T != N)
+    return cudaErrorNotSupported;
+  ProArgs pa = {};
+  if (pro) pa = *pro;
+  CUtensorMap mk, mv, mz, ms0, ms1;
+  cudaError_t e = make_map_bf16_3d(&mk, k, 128, S, N, 64, ctr::TOK);
+  if (e == cudaSuccess) e = make_map_bf16_3d(&mv, v, 128, S, N, 64, ctr::TOK);
+  if (e == cudaSuccess) e = make_map_f32_mats(&mz, U, (uint64_t)N);
+  if (e == cudaSuccess) e = make_map_bf16_3d(&ms0, sfr0, 128, 128, 2 * (uint64_t)N, 64, 128);
+  if (e == cudaSuccess)
+    e = make_map_bf16_3d(&ms1, sfr1 ? sfr1 : sfr0, 128, 128, 2 * (uint64_t)N, 64, 128);
+  if (e != cudaSuccess) return e;
+  static bool attr = false;
+  if (!attr) {
+    e = cudaFuncSetAttribute(k_contract_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ovl::SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  long long ncon = num_sms() - nchain;
+  if (ncon > N) ncon = N;
+  const int grid = nchain + (int)ncon;
+  e = cudaMemsetAsync(o.flags, 0, (size_t)N * sizeof(int), st);
+  if (e != cudaSuccess) return e;
+  const float* beta_a = beta;
+  float *A_a = A, *U_a = U;
+  int N_a = (int)N, S_a = S, nchain_a = nchain;
+  float cA_a = cA, cU_a = cU;
+  OvlArgs o_a = o;
+  void* args[] = {&mk, &mv, &beta_a, &A_a, &U_a, &N_a, &S_a, &cA_a, &cU_a,
+                  &pa, &o_a, &nchain_a, &mz, &ms0, &ms1};
+  // cooperative: every CTA is resident, so the chains' waits on the
+  // contraction CTAs always end
+  e = cudaLaunchCooperativeKernel((const void*)k_contract_scan_tc, dim3(grid), dim3(ovl::THREADS),
+                                  args, (size_t)ovl::SMEM, st);
+  count_launch();
+  return e;
+}
+
+// ============================================================================
 // D = 64 tensor-core kernels.
 //
 // Contraction: [K^T; V^T] is one M = 128 MN-major operand (the K and V boxes
@@ -2546,10 +2902,12 @@ constexpr int THREADS = 64 + NSC + 128;
 constexpr uint32_t TMEM_COLS = 512;
 }  // namespace c256
 
+__device__ __forceinline__ int img256_off(int k, int n8);
+
 __global__ void __launch_bounds__(c256::THREADS, 1)
     k_contract256_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const float* __restrict__ beta, float* __restrict__ A, float* __restrict__ U,
-                     int N, int S, float cA, float cU) {
+                     int N, int S, float cA, float cU, int a_image) {
   using namespace c256;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -2696,16 +3054,33 @@ __global__ void __launch_bounds__(c256::THREADS, 1)
 #pragma unroll
       for (int mat = 0; mat < 2; ++mat) {
         float* dst = (mat ? U : A) + ((size_t)n * D + 128 * half + row) * D;
+        uint8_t* img = (uint8_t*)A + (size_t)n * D * D * 4;
+        const int k = 128 * half + row;
         const float sc = mat ? cU : cA;
         for (int c0 = 0; c0 < 256; c0 += 32) {
           uint32_t r[32];
           tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + mat * 256 + c0, r);
           tmem_wait_ld();
+          if (mat == 0 && a_image) {
+            // row k of A_t into the operand image (hi, lo) of the D = 256 chains
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *(float4*)(dst + c0 + 4 * j) =
-                make_float4(__uint_as_float(r[4 * j]) * sc, __uint_as_float(r[4 * j + 1]) * sc,
-                            __uint_as_float(r[4 * j + 2]) * sc, __uint_as_float(r[4 * j + 3]) * sc);
+            for (int j = 0; j < 4; ++j) {
+              float v[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * j + e]) * sc;
+              uint4 hi, lo;
+              split_chunk(v, &hi, &lo);
+              const int off = img256_off(k, (c0 >> 3) + j);
+              *(uint4*)(img + off) = hi;
+              *(uint4*)(img + off + 8192) = lo;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *(float4*)(dst + c0 + 4 * j) =
+                  make_float4(__uint_as_float(r[4 * j]) * sc, __uint_as_float(r[4 * j + 1]) * sc,
+                              __uint_as_float(r[4 * j + 2]) * sc, __uint_as_float(r[4 * j + 3]) * sc);
+          }
         }
       }
       tc_fence_before();
@@ -2913,7 +3288,7 @@ __global__ void __launch_bounds__(r256::THREADS, 1)
 }
 
 static cudaError_t tc_contract256(const void* k, const void* v, const float* beta, float* A,
-                                  float* U, long long N, int S, float cA, float cU,
+                                  float* U, long long N, int S, float cA, float cU, int a_image,
                                   cudaStream_t st) {
   CUtensorMap mk, mv;
   cudaError_t e = make_map_bf16_3d(&mk, k, 256, S, N, 64, c256::TOK);
@@ -2928,7 +3303,8 @@ static cudaError_t tc_contract256(const void* k, const void* v, const float* bet
   }
   const long long units = 2 * N;
   const int grid = (int)(units < num_sms() ? units : num_sms());
-  k_contract256_tc<<<grid, c256::THREADS, c256::SMEM, st>>>(mk, mv, beta, A, U, (int)N, S, cA, cU);
+  k_contract256_tc<<<grid, c256::THREADS, c256::SMEM, st>>>(mk, mv, beta, A, U, (int)N, S, cA, cU,
+                                                            a_image);
   count_launch();
   return cudaGetLastError();
 }
@@ -2953,13 +3329,298 @@ static cudaError_t tc_readout256(const void* q, const void* Sfr_hilo, void* out,
   return cudaGetLastError();
 }
 
+// ============================================================================
+// Chains of the recurrence on tensor cores for D = 256 (steps a4/a5 as one
+// sequential chain per head, or one chain per reset block).
+//
+// Rows of the state are independent under X <- alpha (X - X Y) + Z, so each
+// chain runs as two CTAs, one per 128-row half h of the 256 x 256 state. Per
+// step one thread issues, over 16 slices of 16 k-rows,
+//     P = X_hi Y_hi + X_lo Y_hi + X_hi Y_lo     (M = 128, N = 256, fp32 in TMEM)
+// with X (this half's rows, K = 256) as a K-major bf16 (hi, lo) tile in shared
+// memory and Y = A_t streaming in slices of its operand image through a
+// 4-slot ring (one bulk copy per slice; the next frame's image and U_t rows
+// are prefetched into L2 a step ahead). The fp32 state itself stays in TMEM
+// next to P (columns 256..511). Eight epilogue warps read P and X, apply
+// X <- gamma (X - P) + U_t with U_t read from global memory (L2), write X
+// back to TMEM and, as a bf16 (hi, lo) pair, into the operand tile, which one
+// thread then stores by TMA as the frame's state for the readout.
+//
+// Operand image of a 256 x 256 matrix M (written by the contraction): 16
+// slices of 16 rows k; slice s holds bf16(M) then bf16(M - bf16(M)) for rows
+// 16s..16s+15, each as four 64-column blocks of [16 rows][128 B] in the
+// 128-byte swizzled layout (block stride 2 KiB): 16 KiB per slice, 256 KiB in
+// all (the size of the fp32 matrix).
+// ============================================================================
+namespace ch2 {
+constexpr int D = 256;
+constexpr int ATOM = 128 * 128;      // [128 rows][128 B]
+constexpr int XT = 4 * ATOM;         // X hi (or lo) tile, K = 256: 64 KiB
+constexpr int SLICE = 16 * 1024;     // 16 k-rows of the image: hi 8 KiB + lo 8 KiB
+constexpr int NSLICE = D / 16;
+constexpr int NSY = 4;               // Y ring slots
+constexpr int OFF_XH = 0;
+constexpr int OFF_XL = OFF_XH + XT;
+constexpr int OFF_Y = OFF_XL + XT;
+constexpr int OFF_BAR = OFF_Y + NSY * SLICE;
+constexpr int NBAR = 2 * NSY + 3;    // y_full, y_empty, p_full, x_ready, fin
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+constexpr int EPI = 256;             // 8 epilogue warps
+constexpr int THREADS = 64 + EPI;    // producer warp, MMA warp, epilogue
+constexpr uint32_t TMEM_COLS = 512;  // P: columns 0..255, fp32 state: 256..511
+constexpr size_t IMG = (size_t)D * D * 4;
+}  // namespace ch2
+
+// Byte offset of 16-byte chunk n8 (columns 8 n8 .. 8 n8 + 7) of row k in the
+// hi half of a D = 256 operand image (the lo half is 8 KiB further).
+__device__ __forceinline__ int img256_off(int k, int n8) {
+  const int s = k >> 4, rs = k & 15;
+  return s * ch2::SLICE + (n8 >> 3) * 2048 + rs * 128 + (((n8 & 7) ^ (rs & 7)) << 4);
+}
+
+__global__ void __launch_bounds__(ch2::THREADS, 1)
+    k_chain256_tc(ChainArgs a, const __grid_constant__ CUtensorMap tmSfr) {
+  using namespace ch2;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar_yf = sb + OFF_BAR;
+  const uint32_t bar_ye = bar_yf + 8 * NSY;
+  const uint32_t bar_p = bar_ye + 8 * NSY;
+  const uint32_t bar_x = bar_p + 8;
+  const uint32_t bar_fin = bar_x + 8;
+  uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
+  const int half = blockIdx.x & 1;
+  const ChainProg g = chain_prog(a, blockIdx.x >> 1);
+  const size_t DD = (size_t)D * D;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSY; ++s) {
+      mbar_init(bar_yf + 8 * s, 1);
+      mbar_init(bar_ye + 8 * s, 1);
+    }
+    mbar_init(bar_p, 1);
+    mbar_init(bar_x, EPI);
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ---- producer: Y slices through the ring; L2 prefetch a step ahead ----
+    if (lane == 0) {
+      int gi = 0;
+      bool ok = true;
+      for (int s = 0; s < g.n && ok; ++s) {
+        const ChainStep st = chain_step_at(a, g, s);
+        if (s + 1 < g.n) {
+          const ChainStep nx = chain_step_at(a, g, s + 1);
+          prefetch_l2(nx.Y, (uint32_t)IMG);
+          prefetch_l2(nx.Z + (size_t)half * 128 * D, (uint32_t)(IMG / 2));
+        }
+        for (int sl = 0; sl < NSLICE; ++sl, ++gi) {
+          const int slot = gi % NSY;
+          const uint32_t u = (uint32_t)(gi / NSY);
+          ok = mbar_wait(bar_ye + 8 * slot, (u & 1) ^ 1, abort_flag, &g_tc_status, 41);
+          if (!ok) break;
+          mbar_arrive_expect_tx(bar_yf + 8 * slot, SLICE);
+          bulk_load(sb + OFF_Y + slot * SLICE, (const uint8_t*)st.Y + (size_t)sl * SLICE, SLICE,
+                    bar_yf + 8 * slot);
+        }
+      }
+      // drain (bounded, not cut short by an abort): copies in flight land
+      volatile int keep_waiting = 0;
+      for (int gg = (gi > NSY ? gi - NSY : 0); gg < gi; ++gg)
+        mbar_wait(bar_yf + 8 * (gg % NSY), (uint32_t)(gg / NSY) & 1, &keep_waiting, &g_tc_status, 42);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---- MMA issuer ----
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 256, false, true);
+      int gi = 0;
+      bool ok = true;
+      for (int s = 0; s < g.n && ok; ++s) {
+        ok = mbar_wait(bar_x, (uint32_t)s & 1, abort_flag, &g_tc_status, 43);
+        if (!ok) break;
+        tc_fence_after();
+        for (int sl = 0; sl < NSLICE; ++sl, ++gi) {
+          const int slot = gi % NSY;
+          const uint32_t u = (uint32_t)(gi / NSY);
+          ok = mbar_wait(bar_yf + 8 * slot, u & 1, abort_flag, &g_tc_status, 44);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t xo = (sl >> 2) * ATOM + (sl & 3) * 32;
+          const uint64_t dxh = smem_desc_sw128(sb + OFF_XH + xo, 16, 1024);
+          const uint64_t dxl = smem_desc_sw128(sb + OFF_XL + xo, 16, 1024);
+          const uint32_t ya = sb + OFF_Y + slot * SLICE;
+          const uint64_t dyh = smem_desc_sw128(ya, 2048, 1024);
+          const uint64_t dyl = smem_desc_sw128(ya + SLICE / 2, 2048, 1024);
+          mma_bf16(tmem, dxh, dyh, idesc, sl > 0 ? 1u : 0u);
+          mma_bf16(tmem, dxl, dyh, idesc, 1u);
+          mma_bf16(tmem, dxh, dyl, idesc, 1u);
+          mma_commit(bar_ye + 8 * slot);
+        }
+        if (!ok) break;
+        mma_commit(bar_p);
+      }
+      mma_commit(bar_fin);
+      volatile int keep_waiting = 0;
+      mbar_wait(bar_fin, 0, &keep_waiting, &g_tc_status, 45);
+    }
+    __syncwarp();
+  } else {
+    // ---- epilogue: 8 warps; warp quadrant q = rows 32q.., column half ch ----
+    const int et = threadIdx.x - 64;
+    const int q = warp & 3, ch = et >> 7;
+    const int row = q * 32 + lane;            // row of this CTA's half
+    const size_t grow = (size_t)half * 128 + row;  // row of the state
+    const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+    const bool store_sfr = g.mode == CHAIN_SCAN;
+    int nstore = 0;
+    float zb[2][32];
+    auto load_z = [&](const float* Z, int c, float* z) {
+      const float* src = Z + grow * D + 128 * ch + 32 * c;
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        const float4 f = __ldg((const float4*)(src + i));
+        z[i] = f.x; z[i + 1] = f.y; z[i + 2] = f.z; z[i + 3] = f.w;
+      }
+    };
+    // the X tile (bf16 hi, lo) for columns 128 ch + 32 c .. +31 of this row
+    auto put_x = [&](const float* x, int c) {
+      const int col = 128 * ch + 32 * c;
+      const int at = col >> 6, c0 = (col & 63) >> 3;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint4 hi, lo;
+        split_chunk(x + 8 * i, &hi, &lo);
+        const int off = at * ATOM + row * 128 + (((c0 + i) ^ (row & 7)) << 4);
+        *(uint4*)(smem + OFF_XH + off) = hi;
+        *(uint4*)(smem + OFF_XL + off) = lo;
+      }
+    };
+    // initial state: fp32 rows of g.init (or zeros) into TMEM and the tile
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float x[32];
+      const float* src = g.init ? g.init + grow * D + 128 * ch + 32 * c : nullptr;
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        float4 f = src ? __ldg((const float4*)(src + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[i] = f.x; x[i + 1] = f.y; x[i + 2] = f.z; x[i + 3] = f.w;
+      }
+      tmem_st32(tl + 256 + 128 * ch + 32 * c, (const uint32_t*)x);
+      put_x(x, c);
+    }
+    tmem_wait_st();
+    fence_proxy_async();
+    tc_fence_before();
+    mbar_arrive(bar_x);
+    if (g.n > 0) {
+      const ChainStep st0 = chain_step_at(a, g, 0);
+      load_z(st0.Z, 0, zb[0]);
+      load_z(st0.Z, 1, zb[1]);
+    }
+    for (int s = 0; s < g.n; ++s) {
+      const ChainStep st = chain_step_at(a, g, s);
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(bar_p, (uint32_t)s & 1, abort_flag, &g_tc_status, 46);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      // the previous state store has read the tile; all agree on leaving
+      if (et == 0 && nstore > 0) bulk_wait_read0();
+      if (named_bar_or(1, EPI, !ok || *abort_flag)) break;
+      tc_fence_after();
+      const bool last = store_sfr && (g.j0 + s == a.T - 1) && a.state_out;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float* z = zb[c & 1];
+        uint32_t p[32], xr[32];
+        tmem_ld32(tl + 128 * ch + 32 * c, p);
+        tmem_ld32(tl + 256 + 128 * ch + 32 * c, xr);
+        tmem_wait_ld();
+        float x[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          x[i] = st.reset ? z[i] : st.alpha * (__uint_as_float(xr[i]) - __uint_as_float(p[i])) + z[i];
+        tmem_st32(tl + 256 + 128 * ch + 32 * c, (const uint32_t*)x);
+        put_x(x, c);
+        if (last) {
+          float* so = a.state_out + (size_t)g.bh * DD + grow * D + 128 * ch + 32 * c;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) *(float4*)(so + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+        }
+        if (c < 2) load_z(st.Z, c + 2, z);
+      }
+      tmem_wait_st();
+      fence_proxy_async();
+      tc_fence_before();
+      if (s + 1 < g.n) {
+        const ChainStep nx = chain_step_at(a, g, s + 1);
+        load_z(nx.Z, 0, zb[0]);
+        load_z(nx.Z, 1, zb[1]);
+      }
+      named_bar_sync(1, EPI);
+      if (et == 0 && store_sfr) {
+        // the state after frame t (this half's rows), as a bf16 (hi, lo) pair
+        const int pair = g.bh * a.T + st.t;
+#pragma unroll
+        for (int at = 0; at < 4; ++at) {
+          tma_store_3d(&tmSfr, sb + OFF_XH + at * ATOM, 64 * at, 128 * half, 2 * pair);
+          tma_store_3d(&tmSfr, sb + OFF_XL + at * ATOM, 64 * at, 128 * half, 2 * pair + 1);
+        }
+        bulk_commit();
+        ++nstore;
+      }
+      mbar_arrive(bar_x);
+    }
+    if (et == 0) bulk_wait0();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+static cudaError_t tc_chain256(const ChainArgs& a, int nchains, cudaStream_t st) {
+  if (a.D != 256 || !a.y_image || a.mode != CHAIN_SCAN || !a.sfr_hilo) return cudaErrorNotSupported;
+  if (a.seg == SEG_CHUNKS && a.nseg > 1) return cudaErrorNotSupported;  // span starts need the prefix
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e =
+        cudaFuncSetAttribute(k_chain256_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, ch2::SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const long long frames = (long long)a.heads * a.T;
+  CUtensorMap ms;
+  cudaError_t e = make_map_bf16_3d(&ms, a.Sfr, 256, 256, 2 * (uint64_t)frames, 64, 128);
+  if (e != cudaSuccess) return e;
+  k_chain256_tc<<<2 * nchains, ch2::THREADS, ch2::SMEM, st>>>(a, ms);
+  count_launch();
+  return cudaGetLastError();
+}
+
 // ---- public entry points of the tensor-core kernels (dispatch on D) ----
 cudaError_t tc_contract(const void* k, const void* v, const float* beta, float* A, float* U,
                         long long N, int S, int D, float cA, float cU, int a_image,
                         const ProArgs* pro, cudaStream_t st) {
   if (D == 256) {
-    if (pro || a_image) return cudaErrorNotSupported;
-    return tc_contract256(k, v, beta, A, U, N, S, cA, cU, st);
+    if (pro) return cudaErrorNotSupported;
+    return tc_contract256(k, v, beta, A, U, N, S, cA, cU, a_image, st);
   }
   if (D == 64) {
     if (pro) return cudaErrorNotSupported;
@@ -3016,6 +3677,7 @@ cudaError_t tc_readout(const void* q, const void* Sfr_hilo, void* out, long long
 
 cudaError_t tc_chain(const ChainArgs& a, int nchains, cudaStream_t st) {
   if (a.D == 64 && a.y_image) return tc_chain64(a, nchains, st);
+  if (a.D == 256) return tc_chain256(a, nchains, st);
   return tc_chain128(a, nchains, st);
 }
 

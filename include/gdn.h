@@ -82,6 +82,9 @@ enum {
 #define GDN_BIDIR 0x80u         /* _ex only: forward scan -> out, reverse scan -> out_rev */
 #define GDN_FUSED_REPLAY 0x1000000u /* tensor-core path: replay each span inside the readout
                                        kernel instead of storing S_t (spans/blocks, no prologue) */
+#define GDN_CHUNKED 0x2000000u  /* run the span-composed (chunk-parallel) plan */
+#define GDN_NO_OVERLAP 0x4000000u /* run the sequential chains as their own launch after
+                                     the contraction instead of alongside it */
 #define GDN_BLOCK(f) (((f) >> 8) & 0xffu)  /* reset block length; 0 means 3 */
 #define GDN_CHUNK(f) (((f) >> 16) & 0xffu) /* time-chunk length; 0 means 8 */
 #define GDN_MAKE_BLOCK(n) ((((unsigned)(n)) & 0xffu) << 8)
@@ -100,13 +103,25 @@ enum {
  *   state_out   [B,H,D,D]    fp32 state after the last frame in scan order
  *                            (frame T-1 forward, frame 0 reversed); NULL = not written
  *   flags       GDN_BF16 | GDN_REVERSE | GDN_BLOCK_RESET | GDN_SEQUENTIAL |
- *               GDN_KEYS_SCALED | GDN_FORCE_SIMT | GDN_FUSED_REPLAY |
- *               GDN_MAKE_BLOCK(n) | GDN_MAKE_CHUNK(n)
+ *               GDN_CHUNKED | GDN_NO_OVERLAP | GDN_KEYS_SCALED |
+ *               GDN_FORCE_SIMT | GDN_FUSED_REPLAY | GDN_MAKE_BLOCK(n) |
+ *               GDN_MAKE_CHUNK(n)
  *
  * Blocks for GDN_BLOCK_RESET are floor(t / block) counted from t = 0 in both
- * directions. Without GDN_SEQUENTIAL the scan runs as time chunks composed
- * through S_end = S_start C_p + H_p (equal to the sequential scan up to
- * rounding). Scratch comes from a stream-ordered allocation (cudaMallocAsync)
+ * directions.
+ *
+ * Plans (all equal up to rounding). GDN_SEQUENTIAL: one chain of the
+ * recurrence per head over all T frames. GDN_CHUNKED: time chunks composed
+ * through S_end = S_start C_p + H_p (SANA-WM blog, Context-Parallel section),
+ * run in parallel, then replayed. Neither flag: the sequential plan where it
+ * can run alongside the contraction, else the chunked plan. Alongside means
+ * one cooperative launch in which a few CTAs run the chains (one per head and
+ * direction) while the rest compute A_t, U_t frame by frame, so the
+ * latency-bound chains hide under the bandwidth-bound contraction. It needs
+ * the tensor-core path (bf16, sm_100a), D = 128, at most a quarter of the
+ * GPU's SMs in chains (B*H <= 37 on a 148-SM B200; 2*B*H for GDN_BIDIR, which
+ * also needs GDN_BLOCK_RESET), and no GDN_FUSED_REPLAY. GDN_NO_OVERLAP turns
+ * it off. Scratch comes from a stream-ordered allocation (cudaMallocAsync)
  * made and freed inside the call; use gdn_frame_scan_fwd_ex to pass your own.
  * Returns GDN_OK or a negative status.
  */
@@ -254,7 +269,8 @@ GDN_API int gdn_profile_enable(int enable);
 /* Sums the recorded kernel durations per phase, waiting on the events:
  * ms[i] and counts[i] for phase i < n, with phases 0 prologue, 1 contract,
  * 2 compose, 3 prefix, 4 scan/replay, 5 readout, 6 replay fused with the
- * readout. Returns the number of phases written, or a negative status. */
+ * readout, 7 contraction with the sequential scan alongside. Returns the
+ * number of phases written, or a negative status. */
 GDN_API int gdn_profile_read(double* ms, long long* counts, int n);
 
 /* ABI version: major * 10000 + minor * 100 + patch. */

@@ -93,14 +93,22 @@ def test_composites_stage(D, L, path):
 # the whole scan on small cases, every mode
 # ---------------------------------------------------------------------------
 
+# Plans: "auto" lets the library choose (the sequential chains alongside the
+# contraction on the tensor-core path at D = 128, else spans); the others force
+# one plan. overlap=False keeps the sequential chains in their own launch.
 MODES = {
-    "chunked": dict(),
-    "chunk3": dict(chunk=3),
+    "auto": dict(),
+    "chunked": dict(chunked=True),
+    "chunk3": dict(chunk=3, chunked=True),
     "sequential": dict(sequential=True),
+    "sequential_separate": dict(sequential=True, overlap=False),
     "reverse": dict(reverse=True),
+    "reverse_chunked": dict(reverse=True, chunked=True),
     "reverse_block": dict(reverse=True, block_reset=True),
+    "reverse_block_blocks": dict(reverse=True, block_reset=True, overlap=False),
     "forward_block": dict(block_reset=True, block=4),
-    "reverse_block_seq": dict(reverse=True, block_reset=True, sequential=True),
+    "forward_block_separate": dict(block_reset=True, block=4, sequential=True, overlap=False),
+    "reverse_block_seq": dict(reverse=True, block_reset=True, sequential=True, overlap=False),
     "fused_replay": dict(fused_replay=True),
     "fused_replay_rev_block": dict(fused_replay=True, reverse=True, block_reset=True),
 }
@@ -210,14 +218,16 @@ def test_prologue_stage(D, bf16):
     assert U.rel_frob_per_frame(U.host(kh), k_ref) < bound
 
 
+@pytest.mark.parametrize("overlap", [True, False])
 @pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("D", [64, 128])
-def test_fused_prologue_bidirectional(D, path):
+def test_fused_prologue_bidirectional(D, path, overlap):
     gh, gw, T = 6, 5, 8
-    arr = U.random_case(30 + D, 1, 2, T, gh * gw, D, bf16=True)
+    arr = U.random_case(30 + D, 1, 2, T, gh * gw, D, bf16=True, state=True)
     d = U.dev_inputs(arr, True)
     pro = dict(w_q=d["w_q"], w_k=d["w_k"], grid_h=gh, grid_w=gw)
-    out, st, out_r, st_r = run_scan(d, path, prologue=pro, bidir=True, block_reset=True, block=3)
+    out, st, out_r, st_r = run_scan(d, path, prologue=pro, bidir=True, block_reset=True, block=3,
+                                    overlap=overlap)
     torch.cuda.synchronize()
     for h in range(2):
         o_f, s_f = U.oracle_slab(arr, 0, h, True, prologue=(gw, 1e-6, 1e4))
@@ -234,10 +244,13 @@ def test_fused_prologue_bidirectional(D, path):
 
 FULL = [
     ("clip5s_720p", {}),
+    ("clip5s_720p", {"chunked": True}),
     ("clip5s_720p", {"fused_replay": True}),
     ("rollout60s_720p", {}),
-    ("rollout60s_720p", {"sequential": True}),
+    ("rollout60s_720p", {"chunked": True}),
+    ("rollout60s_720p", {"sequential": True, "overlap": False}),
     ("prologue_bidir_720p", {}),
+    ("prologue_bidir_720p", {"overlap": False}),
     ("sweep_d64", {}),
     ("sweep_d256", {}),
 ]
@@ -278,10 +291,44 @@ def test_chunked_matches_sequential_full_size():
     cfg = synth.CONFIGS["rollout60s_720p"]
     arr = synth.make_inputs(cfg)
     d = U.dev_inputs(arr, True)
-    o1, s1 = run_scan(d, "default")
-    o2, s2 = run_scan(d, "default", sequential=True)
+    o1, s1 = run_scan(d, "default", chunked=True)
+    for kw in (dict(sequential=True), dict(sequential=True, overlap=False)):
+        o2, s2 = run_scan(d, "default", **kw)
+        torch.cuda.synchronize()
+        num = (o1.float() - o2.float()).flatten(3).norm(dim=-1)
+        den = o2.float().flatten(3).norm(dim=-1)
+        assert float((num / den).max()) < 5e-3, kw
+        assert float(((s1 - s2).flatten(2).norm(dim=-1) / s2.flatten(2).norm(dim=-1)).max()) < 1e-3
+
+
+def _phase_launches(fn):
+    api.profile_enable(True)
+    fn()
     torch.cuda.synchronize()
-    num = (o1.float() - o2.float()).flatten(3).norm(dim=-1)
-    den = o2.float().flatten(3).norm(dim=-1)
-    assert float((num / den).max()) < 5e-3
-    assert float(((s1 - s2).flatten(2).norm(dim=-1) / s2.flatten(2).norm(dim=-1)).max()) < 1e-3
+    rec = api.profile_read()
+    api.profile_enable(False)
+    return {k: v[1] for k, v in rec.items()}
+
+
+def test_plan_selection():
+    """The library runs the chains alongside the contraction exactly where the
+    plan says so, and its result equals the separate-launch sequential scan."""
+    arr = U.random_case(77, 1, 3, 9, 150, 128, bf16=True, state=True)
+    d = U.dev_inputs(arr, True)
+    got = {}
+    for name, kw in (("auto", {}), ("chunked", dict(chunked=True)),
+                     ("separate", dict(sequential=True, overlap=False))):
+        def call(kw=kw, name=name):
+            got[name] = run_scan(d, "default", **kw)
+        n = _phase_launches(call)
+        assert n["contract_scan"] == (1 if name == "auto" else 0), (name, n)
+        assert n["contract"] == (0 if name == "auto" else 1), (name, n)
+    o_a, s_a = got["auto"]
+    o_s, s_s = got["separate"]
+    assert U.rel_frob_per_frame(U.host(o_a), U.host(o_s)) < 1e-3
+    assert U.rel_frob_per_frame(U.host(s_a)[None], U.host(s_s)[None]) < 1e-4
+    # more chains than a quarter of the SMs: the chunked plan
+    many = U.random_case(78, 1, 40, 10, 64, 128, bf16=True)
+    dm = U.dev_inputs(many, True)
+    n = _phase_launches(lambda: run_scan(dm, "default"))
+    assert n["contract_scan"] == 0 and n["compose"] == 1, n
