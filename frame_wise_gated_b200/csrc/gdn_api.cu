@@ -304,8 +304,11 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
   const bool simt = (f & GDN_FORCE_SIMT) || !bf16 || !sm100;
   const bool tc_contract_ok = !simt && tc_contract_supported(p.D);
   const bool tc_readout_ok = !simt && tc_readout_supported(p.D);
-  const bool seq_plan = (f & GDN_SEQUENTIAL) != 0;
-  const bool tc_chain_ok = !simt && tc_chain_supported(p.D);
+  // D = 256 has tensor-core chains for whole-scan chains only (sequential,
+  // or one per reset block): its plan is sequential unless spans are asked for.
+  const bool seq_plan = (f & GDN_SEQUENTIAL) ||
+                        (p.D == 256 && !simt && !(f & (GDN_CHUNKED | GDN_FUSED_REPLAY)));
+  const bool tc_chain_ok = !simt && (tc_chain_supported(p.D) || (p.D == 256 && seq_plan));
   char* ws = (char*)p.workspace;
   const long long frames = (long long)p.B * p.H * p.T;
   cudaError_t e;

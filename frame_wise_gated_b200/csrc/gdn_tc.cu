@@ -3521,7 +3521,10 @@ __global__ void __launch_bounds__(ch2::THREADS, 1)
         float4 f = src ? __ldg((const float4*)(src + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
         x[i] = f.x; x[i + 1] = f.y; x[i + 2] = f.z; x[i + 3] = f.w;
       }
-      tmem_st32(tl + 256 + 128 * ch + 32 * c, (const uint32_t*)x);
+      uint32_t xu[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) xu[i] = __float_as_uint(x[i]);
+      tmem_st32(tl + 256 + 128 * ch + 32 * c, xu);
       put_x(x, c);
     }
     tmem_wait_st();
@@ -3543,7 +3546,7 @@ __global__ void __launch_bounds__(ch2::THREADS, 1)
       if (named_bar_or(1, EPI, !ok || *abort_flag)) break;
       tc_fence_after();
       const bool last = store_sfr && (g.j0 + s == a.T - 1) && a.state_out;
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < 4; ++c) {
         float* z = zb[c & 1];
         uint32_t p[32], xr[32];
@@ -3552,9 +3555,11 @@ __global__ void __launch_bounds__(ch2::THREADS, 1)
         tmem_wait_ld();
         float x[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
+        for (int i = 0; i < 32; ++i) {
           x[i] = st.reset ? z[i] : st.alpha * (__uint_as_float(xr[i]) - __uint_as_float(p[i])) + z[i];
-        tmem_st32(tl + 256 + 128 * ch + 32 * c, (const uint32_t*)x);
+          xr[i] = __float_as_uint(x[i]);
+        }
+        tmem_st32(tl + 256 + 128 * ch + 32 * c, xr);
         put_x(x, c);
         if (last) {
           float* so = a.state_out + (size_t)g.bh * DD + grow * D + 128 * ch + 32 * c;

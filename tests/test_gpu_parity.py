@@ -253,6 +253,7 @@ FULL = [
     ("prologue_bidir_720p", {"overlap": False}),
     ("sweep_d64", {}),
     ("sweep_d256", {}),
+    ("sweep_d256", {"chunked": True}),
 ]
 
 
@@ -332,3 +333,19 @@ def test_plan_selection():
     dm = U.dev_inputs(many, True)
     n = _phase_launches(lambda: run_scan(dm, "default"))
     assert n["contract_scan"] == 0 and n["compose"] == 1, n
+
+
+def test_plan_selection_d256():
+    """D = 256: whole-scan tensor-core chains by default (one launch, no span
+    composition); spans when asked for; both equal the oracle."""
+    arr = U.random_case(79, 2, 1, 10, 90, 256, bf16=True, state=True)
+    d = U.dev_inputs(arr, True)
+    for kw, expect_compose in (({}, 0), (dict(chunked=True), 1)):
+        res = {}
+        n = _phase_launches(lambda: res.setdefault("r", run_scan(d, "default", **kw)))
+        assert n["compose"] == expect_compose and n["scan"] == 1, (kw, n)
+        out, st = res["r"]
+        for b in range(2):
+            o_ref, s_ref = U.oracle_slab(arr, b, 0, True)
+            assert U.rel_frob_per_frame(U.host(out[b, 0]), o_ref) < U.TOL_BF16, kw
+            assert U.rel_frob_per_frame(U.host(st[b, 0])[None], s_ref[None]) < U.TOL_BF16, kw
