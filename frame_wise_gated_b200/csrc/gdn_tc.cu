@@ -164,22 +164,34 @@ cudaError_t rope_table(float2* cs, int npos, int D, float base, cudaStream_t st)
 namespace ctr {
 constexpr int D = 128;
 constexpr int TOK = 64;                 // tokens per stage
-constexpr int NST = 4;                  // pipeline stages
 constexpr int BOX = TOK * 128;          // one [64 tokens][64 channels] bf16 box: 8 KiB
 constexpr int TILE = 2 * BOX;           // one tensor's stage tile: 16 KiB
-constexpr int OFF_K = 0;
-constexpr int OFF_V = OFF_K + NST * TILE;
-constexpr int OFF_BK = OFF_V + NST * TILE;
-constexpr int OFF_BETA = OFF_BK + NST * TILE;
-constexpr int OFF_BAR = OFF_BETA + NST * TOK * 4;
-constexpr int NBAR = 3 * NST + 5;       // full, bk_full, empty, acc_full[2], acc_empty[2], fin
-constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr int OFF_TAB = OFF_MISC + 16;  // prologue (cos, sin) table copy
-constexpr int TAB_MAX = 80 * 32;        // entries: positions x pairs (D/4 = 32)
-constexpr int SMEM = OFF_TAB + TAB_MAX * 8 + 1024;
+constexpr int NBK = 2;                  // beta * K slots (the MMA's B operand)
+constexpr int TAB_MAX = 80 * 32;        // prologue table entries: positions x pairs (D/4 = 32)
 constexpr int NSC = 256;                // scaler threads (8 warps)
 constexpr int THREADS = 64 + NSC + 128;  // producer, MMA, 8 scaler warps, 4 epilogue warps
 constexpr uint32_t TMEM_COLS = 512;
+// Shared-memory layout for an NST-stage K/V ring (deepest that fits: 6
+// stages without the prologue's (cos, sin) table, 5 with it).
+template <int NST>
+struct Lay {
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + NST * TILE;
+  static constexpr int OFF_BK = OFF_V + NST * TILE;
+  static constexpr int OFF_BETA = OFF_BK + NBK * TILE;
+  static constexpr int OFF_BAR = OFF_BETA + NST * TOK * 4;
+  // full, empty per stage; bk_full, bk_empty per slot; acc_full[2], acc_empty[2], fin
+  static constexpr int NBAR = 2 * NST + 2 * NBK + 5;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_TAB = OFF_MISC + 16;
+  static constexpr int SMEM_PLAIN = OFF_TAB + 1024;
+  static constexpr int SMEM_PRO = OFF_TAB + TAB_MAX * 8 + 1024;
+};
+constexpr int NST_PLAIN = 6;
+constexpr int NST_PRO = 5;
+constexpr int SMEM_PLAIN = Lay<NST_PLAIN>::SMEM_PLAIN;
+constexpr int SMEM_PRO = Lay<NST_PRO>::SMEM_PRO;
+static_assert(SMEM_PLAIN <= 232448 && SMEM_PRO <= 232448, "contraction shared memory");
 }  // namespace ctr
 
 // Body of the contraction for CTA `cta` of `ncta` contraction CTAs. Units are
@@ -189,20 +201,29 @@ constexpr uint32_t TMEM_COLS = 512;
 // publishes its rows of A_t, U_t by a release increment of flags[n], so a
 // concurrent scan may read frame-head n once flags[n] reaches 4. Warps beyond
 // the contraction's 14 (when the block is larger) only join the barriers.
+//
+// Rings: K and V tiles in NST stages (freed by the MMA commit of the stage),
+// beta * K in NBK slots of its own (written by the scalers once the MMAs of
+// the stage NBK earlier are done), so the ring that waits on HBM is deep.
+template <int NST>
 __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUtensorMap& tmV,
                                               const float* __restrict__ beta, float* __restrict__ A,
                                               float* __restrict__ U, int N, int S, float cA,
                                               float cU, int a_image, const ProArgs& pro, int cta,
                                               int ncta, int heads, int T, int rev, int* flags) {
   using namespace ctr;
+  using Ly = Lay<NST>;
+  constexpr int OFF_K = Ly::OFF_K, OFF_V = Ly::OFF_V, OFF_BK = Ly::OFF_BK, OFF_BETA = Ly::OFF_BETA;
+  constexpr int OFF_MISC = Ly::OFF_MISC, OFF_TAB = Ly::OFF_TAB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t bar_full = sb + OFF_BAR;
-  const uint32_t bar_bk = bar_full + 8 * NST;
-  const uint32_t bar_empty = bar_bk + 8 * NST;
-  const uint32_t bar_accf = bar_empty + 8 * NST;
+  const uint32_t bar_full = sb + Ly::OFF_BAR;
+  const uint32_t bar_empty = bar_full + 8 * NST;
+  const uint32_t bar_bkf = bar_empty + 8 * NST;
+  const uint32_t bar_bke = bar_bkf + 8 * NBK;
+  const uint32_t bar_accf = bar_bke + 8 * NBK;
   const uint32_t bar_acce = bar_accf + 16;
   const uint32_t bar_fin = bar_acce + 16;
   uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
@@ -211,8 +232,11 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(bar_full + 8 * s, 33);     // expect_tx arrival + 32 lanes' beta copies
-      mbar_init(bar_bk + 8 * s, NSC);      // every scaler thread
       mbar_init(bar_empty + 8 * s, 1);     // MMA commit
+    }
+    for (int s = 0; s < NBK; ++s) {
+      mbar_init(bar_bkf + 8 * s, NSC);     // every scaler thread
+      mbar_init(bar_bke + 8 * s, 1);       // MMA commit
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_accf + 8 * b, 1);
@@ -294,13 +318,12 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
         tc_fence_after();
         const uint32_t dA = tmem + b * 256, dU = dA + 128;
         for (int st = 0; st < nst_frame; ++st, ++g) {
-          const int s = g % NST;
-          const uint32_t u = (uint32_t)(g / NST);
-          ok = mbar_wait(bar_bk + 8 * s, u & 1, abort_flag, &g_tc_status, 4);
+          const int s = g % NST, kb = g % NBK;
+          ok = mbar_wait(bar_bkf + 8 * kb, (uint32_t)(g / NBK) & 1, abort_flag, &g_tc_status, 4);
           if (!ok) break;
           tc_fence_after();
           const uint32_t ka = sb + OFF_K + s * TILE, va = sb + OFF_V + s * TILE,
-                         ba = sb + OFF_BK + s * TILE;
+                         ba = sb + OFF_BK + kb * TILE;
 #pragma unroll
           for (int kk = 0; kk < TOK / 16; ++kk) {
             // 16 tokens = two 8-row groups of 1024 B
@@ -312,6 +335,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
             mma_bf16(dU, dv, db, idesc, acc);
           }
           mma_commit(bar_empty + 8 * s);
+          mma_commit(bar_bke + 8 * kb);
         }
         if (!ok) break;
         mma_commit(bar_accf + 8 * b);
@@ -334,12 +358,14 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
       for (int st = 0; st < nst_frame; ++st, ++g) {
-        const int s = g % NST;
+        const int s = g % NST, kb = g % NBK;
         const uint32_t u = (uint32_t)(g / NST);
         ok = mbar_wait(bar_full + 8 * s, u & 1, abort_flag, &g_tc_status, 6);
+        // the slot's previous beta * K has been consumed by its MMAs
+        if (ok) ok = mbar_wait(bar_bke + 8 * kb, ((uint32_t)(g / NBK) & 1) ^ 1, abort_flag, &g_tc_status, 8);
         if (!ok) break;
         uint8_t* kt = smem + OFF_K + s * TILE;
-        uint8_t* bt = smem + OFF_BK + s * TILE;
+        uint8_t* bt = smem + OFF_BK + kb * TILE;
         const float* bs = (const float*)(smem + OFF_BETA) + s * TOK;
         if (pro.w) {
           // raw k -> K^ in place (RMSNorm, ReLU, RoPE), then beta * K^
@@ -355,7 +381,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
                 pack_bf16x2(f[8 * c] * bv, f[8 * c + 1] * bv), pack_bf16x2(f[8 * c + 2] * bv, f[8 * c + 3] * bv),
                 pack_bf16x2(f[8 * c + 4] * bv, f[8 * c + 5] * bv), pack_bf16x2(f[8 * c + 6] * bv, f[8 * c + 7] * bv));
           fence_proxy_async();
-          mbar_arrive(bar_bk + 8 * s);
+          mbar_arrive(bar_bkf + 8 * kb);
           continue;
         }
 #pragma unroll
@@ -373,7 +399,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
           *(uint4*)(bt + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async();
-        mbar_arrive(bar_bk + 8 * s);
+        mbar_arrive(bar_bkf + 8 * kb);
       }
     }
   } else if (warp < 2 + NSC / 32 + 4) {
@@ -451,12 +477,13 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
   }
 }
 
+template <int NST>
 __global__ void __launch_bounds__(ctr::THREADS, 1)
     k_contract_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const float* __restrict__ beta, float* __restrict__ A, float* __restrict__ U,
                   int N, int S, float cA, float cU, int a_image, ProArgs pro) {
-  contract_body(tmK, tmV, beta, A, U, N, S, cA, cU, a_image, pro, blockIdx.x, gridDim.x, 0, 0, 0,
-                nullptr);
+  contract_body<NST>(tmK, tmV, beta, A, U, N, S, cA, cU, a_image, pro, blockIdx.x, gridDim.x, 0, 0,
+                     0, nullptr);
 }
 
 bool tc_contract_supported(int D) { return D == 128 || D == 64 || D == 256; }
@@ -476,13 +503,21 @@ static cudaError_t tc_contract128(const void* k, const void* v, const float* bet
   if (e != cudaSuccess) return e;
   static bool attr = false;
   if (!attr) {
-    e = cudaFuncSetAttribute(k_contract_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, ctr::SMEM);
+    e = cudaFuncSetAttribute(k_contract_tc<ctr::NST_PLAIN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             ctr::SMEM_PLAIN);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_contract_tc<ctr::NST_PRO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               ctr::SMEM_PRO);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   const int grid = (int)(N < num_sms() ? N : num_sms());
-  k_contract_tc<<<grid, ctr::THREADS, ctr::SMEM, st>>>(mk, mv, beta, A, U, (int)N, S, cA, cU,
-                                                        a_image, pa);
+  if (pro)
+    k_contract_tc<ctr::NST_PRO><<<grid, ctr::THREADS, ctr::SMEM_PRO, st>>>(mk, mv, beta, A, U, (int)N,
+                                                                           S, cA, cU, a_image, pa);
+  else
+    k_contract_tc<ctr::NST_PLAIN><<<grid, ctr::THREADS, ctr::SMEM_PLAIN, st>>>(
+        mk, mv, beta, A, U, (int)N, S, cA, cU, a_image, pa);
   count_launch();
   return cudaGetLastError();
 }
@@ -1593,7 +1628,7 @@ static cudaError_t tc_chain128(const ChainArgs& a, int nchains, cudaStream_t st)
 // ============================================================================
 namespace ovl {
 constexpr int THREADS = 512;
-constexpr int SMEM = ctr::SMEM > chn::SMEM ? ctr::SMEM : chn::SMEM;
+constexpr int smem(int contract_smem) { return contract_smem > chn::SMEM ? contract_smem : chn::SMEM; }
 constexpr int EPI_WARPS = 4;  // contraction epilogue warps: publishes per frame-head
 }  // namespace ovl
 
@@ -1829,6 +1864,7 @@ __device__ __forceinline__ void ovl_chain_body(const OvlArgs& o, const CUtensorM
   }
 }
 
+template <int NST>
 __global__ void __launch_bounds__(ovl::THREADS, 1)
     k_contract_scan_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const float* __restrict__ beta, float* __restrict__ A, float* __restrict__ U,
@@ -1838,7 +1874,7 @@ __global__ void __launch_bounds__(ovl::THREADS, 1)
   if ((int)blockIdx.x < nchain)
     ovl_chain_body(o, tmZ, tmS0, tmS1, blockIdx.x);
   else
-    contract_body(tmK, tmV, beta, A, U, N, S, cA, cU, 1, pro, (int)blockIdx.x - nchain,
+    contract_body<NST>(tmK, tmV, beta, A, U, N, S, cA, cU, 1, pro, (int)blockIdx.x - nchain,
                   (int)gridDim.x - nchain, o.heads, o.T, o.dir[0].reverse && !o.dir[0].blocks_asc,
                   o.flags);
 }
@@ -1864,10 +1900,14 @@ cudaError_t tc_contract_scan(const void* k, const void* v, const float* beta, fl
   if (e == cudaSuccess)
     e = make_map_bf16_3d(&ms1, sfr1 ? sfr1 : sfr0, 128, 128, 2 * (uint64_t)N, 64, 128);
   if (e != cudaSuccess) return e;
+  constexpr int smem_plain = ovl::smem(ctr::SMEM_PLAIN), smem_pro = ovl::smem(ctr::SMEM_PRO);
   static bool attr = false;
   if (!attr) {
-    e = cudaFuncSetAttribute(k_contract_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             ovl::SMEM);
+    e = cudaFuncSetAttribute(k_contract_scan_tc<ctr::NST_PLAIN>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem_plain);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_contract_scan_tc<ctr::NST_PRO>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, smem_pro);
     if (e != cudaSuccess) return e;
     attr = true;
   }
@@ -1885,8 +1925,12 @@ cudaError_t tc_contract_scan(const void* k, const void* v, const float* beta, fl
                   &pa, &o_a, &nchain_a, &mz, &ms0, &ms1};
   // cooperative: every CTA is resident, so the chains' waits on the
   // contraction CTAs always end
-  e = cudaLaunchCooperativeKernel((const void*)k_contract_scan_tc, dim3(grid), dim3(ovl::THREADS),
-                                  args, (size_t)ovl::SMEM, st);
+  if (pro)
+    e = cudaLaunchCooperativeKernel((const void*)k_contract_scan_tc<ctr::NST_PRO>, dim3(grid),
+                                    dim3(ovl::THREADS), args, (size_t)smem_pro, st);
+  else
+    e = cudaLaunchCooperativeKernel((const void*)k_contract_scan_tc<ctr::NST_PLAIN>, dim3(grid),
+                                    dim3(ovl::THREADS), args, (size_t)smem_plain, st);
   count_launch();
   return e;
 }
