@@ -6,14 +6,15 @@
 //
 // k_contract_tc (step a2), D = 128. One CTA per SM, persistent over
 // frame-heads. Per 64-token stage, TMA brings K and V tiles ([64 tokens][64 D]
-// boxes, 128-byte swizzle) into shared memory; four scaler warps write
-// beta * K next to them in the same layout; one thread issues, per 16 tokens,
-//   A_acc += K^T (beta K)   and   U_acc += V^T (beta K)
-// as two 128x128x16 bf16 MMAs sharing the B operand. K^T and V^T are read as
-// MN-major operands straight from the token-major tiles: no transposes. The
-// fp32 accumulators live in TMEM (2 x 256 columns, double-buffered so the
-// epilogue of one frame-head overlaps the MMAs of the next); four epilogue
-// warps scale them (1/(D S) and 1/sqrt(D S)) and store A_t, U_t in fp32.
+// boxes, 128-byte swizzle) side by side into shared memory; eight scaler warps
+// write beta * K in the same layout; one thread issues, per 16 tokens,
+//   [A_acc | U_acc^T] += (beta K)^T [K | V]
+// as one 128x256x16 bf16 MMA (A_t is symmetric, so (beta K)^T K = A_t).
+// (beta K)^T and [K | V] are read as MN-major operands straight from the
+// token-major tiles: no transposes. The fp32 accumulators live in TMEM
+// (2 x 256 columns, double-buffered so the epilogue of one frame-head overlaps
+// the MMAs of the next); four epilogue warps scale them (1/(D S) and
+// 1/sqrt(D S)) and store A_t (row by row) and U_t (column by column).
 //
 // k_readout_tc (step a6), D = 128. Per 128-token tile of a frame-head,
 //   O_tile = Q_tile S_t^T = Q_tile S_hi^T + Q_tile S_lo^T
@@ -175,9 +176,8 @@ constexpr uint32_t TMEM_COLS = 512;
 // stages without the prologue's (cos, sin) table, 5 with it).
 template <int NST>
 struct Lay {
-  static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = OFF_K + NST * TILE;
-  static constexpr int OFF_BK = OFF_V + NST * TILE;
+  static constexpr int OFF_K = 0;                     // stage s: K at s * 2 TILE, V after it
+  static constexpr int OFF_BK = OFF_K + NST * 2 * TILE;
   static constexpr int OFF_BETA = OFF_BK + NBK * TILE;
   static constexpr int OFF_BAR = OFF_BETA + NST * TOK * 4;
   // full, empty per stage; bk_full, bk_empty per slot; acc_full[2], acc_empty[2], fin
@@ -213,7 +213,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
                                               int ncta, int heads, int T, int rev, int* flags) {
   using namespace ctr;
   using Ly = Lay<NST>;
-  constexpr int OFF_K = Ly::OFF_K, OFF_V = Ly::OFF_V, OFF_BK = Ly::OFF_BK, OFF_BETA = Ly::OFF_BETA;
+  constexpr int OFF_K = Ly::OFF_K, OFF_BK = Ly::OFF_BK, OFF_BETA = Ly::OFF_BETA;
   constexpr int OFF_MISC = Ly::OFF_MISC, OFF_TAB = Ly::OFF_TAB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -279,7 +279,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         if (lane == 0) {
-          const uint32_t kd = sb + OFF_K + s * TILE, vd = sb + OFF_V + s * TILE;
+          const uint32_t kd = sb + OFF_K + s * 2 * TILE, vd = kd + TILE;
           mbar_arrive_expect_tx(bar_full + 8 * s, 2 * TILE);
           tma_load_3d(kd, &tmK, bar_full + 8 * s, 0, st * TOK, n);
           tma_load_3d(kd + BOX, &tmK, bar_full + 8 * s, 64, st * TOK, n);
@@ -307,7 +307,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
   } else if (warp == 1) {
     // ---- MMA issuer ----
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, true, true);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 256, true, true);
       int g = 0;
       bool ok = true;
       for (int i = 0; i < my_count && ok; ++i) {
@@ -316,23 +316,21 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
         ok = mbar_wait(bar_acce + 8 * b, (ub & 1) ^ 1, abort_flag, &g_tc_status, 3);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t dA = tmem + b * 256, dU = dA + 128;
+        const uint32_t dAU = tmem + b * 256;
         for (int st = 0; st < nst_frame; ++st, ++g) {
           const int s = g % NST, kb = g % NBK;
           ok = mbar_wait(bar_bkf + 8 * kb, (uint32_t)(g / NBK) & 1, abort_flag, &g_tc_status, 4);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t ka = sb + OFF_K + s * TILE, va = sb + OFF_V + s * TILE,
-                         ba = sb + OFF_BK + kb * TILE;
+          const uint32_t kva = sb + OFF_K + s * 2 * TILE, ba = sb + OFF_BK + kb * TILE;
 #pragma unroll
           for (int kk = 0; kk < TOK / 16; ++kk) {
-            // 16 tokens = two 8-row groups of 1024 B
-            const uint64_t dk = smem_desc_sw128(ka + kk * 2048, BOX, 1024);
-            const uint64_t dv = smem_desc_sw128(va + kk * 2048, BOX, 1024);
+            // 16 tokens = two 8-row groups of 1024 B; [K | V] is one N = 256
+            // operand of four 64-channel blocks
+            const uint64_t dkv = smem_desc_sw128(kva + kk * 2048, BOX, 1024);
             const uint64_t db = smem_desc_sw128(ba + kk * 2048, BOX, 1024);
             const uint32_t acc = (st > 0 || kk > 0) ? 1u : 0u;
-            mma_bf16(dA, dk, db, idesc, acc);
-            mma_bf16(dU, dv, db, idesc, acc);
+            mma_bf16(dAU, db, dkv, idesc, acc);
           }
           mma_commit(bar_empty + 8 * s);
           mma_commit(bar_bke + 8 * kb);
@@ -364,7 +362,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
         // the slot's previous beta * K has been consumed by its MMAs
         if (ok) ok = mbar_wait(bar_bke + 8 * kb, ((uint32_t)(g / NBK) & 1) ^ 1, abort_flag, &g_tc_status, 8);
         if (!ok) break;
-        uint8_t* kt = smem + OFF_K + s * TILE;
+        uint8_t* kt = smem + OFF_K + s * 2 * TILE;
         uint8_t* bt = smem + OFF_BK + kb * TILE;
         const float* bs = (const float*)(smem + OFF_BETA) + s * TOK;
         if (pro.w) {
@@ -444,7 +442,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
               *(uint4*)(img + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
               *(uint4*)(img + 32768 + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
             }
-          } else {
+          } else if (half == 0) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
               float4 v = make_float4(__uint_as_float(r[4 * j]) * sc, __uint_as_float(r[4 * j + 1]) * sc,
@@ -452,6 +450,13 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
                                      __uint_as_float(r[4 * j + 3]) * sc);
               *(float4*)(dst + c0 + 4 * j) = v;
             }
+          } else {
+            // TMEM holds U_t^T (lane = key channel `row`, column = value
+            // channel): column `row` of U_t, rows c0..c0+31; the warp's 32
+            // lanes store 32 consecutive floats of each row
+            float* ucol = U + (size_t)n * D * D + row;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ucol[(size_t)(c0 + j) * D] = __uint_as_float(r[j]) * sc;
           }
         }
       }
