@@ -2933,19 +2933,21 @@ cudaError_t tc_readout2(const void* q, const void* sfr_f, const void* sfr_r, voi
 // ============================================================================
 namespace c256 {
 constexpr int D = 256;
-constexpr int TOK = 64;
-constexpr int NST = 2;
-constexpr int BOX = TOK * 128;          // [64 tokens][64 channels]: 8 KiB
-constexpr int KT = 4 * BOX;             // K stage tile, all channels: 32 KiB
-constexpr int VT = 2 * BOX;             // V stage tile, one channel half: 16 KiB
+constexpr int TOK = 32;                 // tokens per stage
+constexpr int NST = 8;                  // K/V stages
+constexpr int NBK = 2;                  // beta * K slots
+constexpr int BOX = TOK * 128;          // [32 tokens][64 channels]: 4 KiB
+constexpr int KT = 4 * BOX;             // K stage tile, all channels: 16 KiB
+constexpr int VT = 2 * BOX;             // V stage tile, one channel half: 8 KiB
 constexpr int OFF_K = 0;
 constexpr int OFF_V = OFF_K + NST * KT;
 constexpr int OFF_BK = OFF_V + NST * VT;
-constexpr int OFF_BETA = OFF_BK + NST * KT;
+constexpr int OFF_BETA = OFF_BK + NBK * KT;
 constexpr int OFF_BAR = OFF_BETA + NST * TOK * 4;
-constexpr int NBAR = 3 * NST + 3;
+constexpr int NBAR = 2 * NST + 2 * NBK + 3;  // full, empty; bk_full, bk_empty; acc_full, acc_empty, fin
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM = OFF_MISC + 16 + 1024;
+static_assert(SMEM <= 232448, "D = 256 contraction shared memory");
 constexpr int NSC = 256;
 constexpr int THREADS = 64 + NSC + 128;
 constexpr uint32_t TMEM_COLS = 512;
@@ -2963,9 +2965,10 @@ __global__ void __launch_bounds__(c256::THREADS, 1)
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t bar_full = sb + OFF_BAR;
-  const uint32_t bar_bk = bar_full + 8 * NST;
-  const uint32_t bar_empty = bar_bk + 8 * NST;
-  const uint32_t bar_accf = bar_empty + 8 * NST;
+  const uint32_t bar_empty = bar_full + 8 * NST;
+  const uint32_t bar_bkf = bar_empty + 8 * NST;
+  const uint32_t bar_bke = bar_bkf + 8 * NBK;
+  const uint32_t bar_accf = bar_bke + 8 * NBK;
   const uint32_t bar_acce = bar_accf + 8;
   const uint32_t bar_fin = bar_acce + 8;
   uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
@@ -2973,8 +2976,11 @@ __global__ void __launch_bounds__(c256::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(bar_full + 8 * s, 33);
-      mbar_init(bar_bk + 8 * s, NSC);
       mbar_init(bar_empty + 8 * s, 1);
+    }
+    for (int s = 0; s < NBK; ++s) {
+      mbar_init(bar_bkf + 8 * s, NSC);
+      mbar_init(bar_bke + 8 * s, 1);
     }
     mbar_init(bar_accf, 1);
     mbar_init(bar_acce, 128);
@@ -3040,13 +3046,12 @@ __global__ void __launch_bounds__(c256::THREADS, 1)
         if (!ok) break;
         tc_fence_after();
         for (int st = 0; st < nst_frame; ++st, ++g) {
-          const int s = g % NST;
-          const uint32_t u = (uint32_t)(g / NST);
-          ok = mbar_wait(bar_bk + 8 * s, u & 1, abort_flag, &g_tc_status, 104);
+          const int s = g % NST, kb = g % NBK;
+          ok = mbar_wait(bar_bkf + 8 * kb, (uint32_t)(g / NBK) & 1, abort_flag, &g_tc_status, 104);
           if (!ok) break;
           tc_fence_after();
           const uint32_t ka = sb + OFF_K + s * KT + 2 * half * BOX, va = sb + OFF_V + s * VT,
-                         ba = sb + OFF_BK + s * KT;
+                         ba = sb + OFF_BK + kb * KT;
 #pragma unroll
           for (int kk = 0; kk < TOK / 16; ++kk) {
             const uint64_t db = smem_desc_sw128(ba + kk * 2048, BOX, 1024);
@@ -3055,6 +3060,7 @@ __global__ void __launch_bounds__(c256::THREADS, 1)
             mma_bf16(tmem + 256, smem_desc_sw128(va + kk * 2048, BOX, 1024), db, idesc, acc);
           }
           mma_commit(bar_empty + 8 * s);
+          mma_commit(bar_bke + 8 * kb);
         }
         if (!ok) break;
         mma_commit(bar_accf);
@@ -3069,12 +3075,14 @@ __global__ void __launch_bounds__(c256::THREADS, 1)
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
       for (int st = 0; st < nst_frame; ++st, ++g) {
-        const int s = g % NST;
+        const int s = g % NST, kb = g % NBK;
         const uint32_t u = (uint32_t)(g / NST);
         ok = mbar_wait(bar_full + 8 * s, u & 1, abort_flag, &g_tc_status, 106);
+        // the slot's previous beta * K has been consumed by its MMAs
+        if (ok) ok = mbar_wait(bar_bke + 8 * kb, ((uint32_t)(g / NBK) & 1) ^ 1, abort_flag, &g_tc_status, 108);
         if (!ok) break;
         const uint8_t* kt = smem + OFF_K + s * KT;
-        uint8_t* bt = smem + OFF_BK + s * KT;
+        uint8_t* bt = smem + OFF_BK + kb * KT;
         const float* bs = (const float*)(smem + OFF_BETA) + s * TOK;
 #pragma unroll
         for (int m = 0; m < (KT / 16) / NSC; ++m) {
@@ -3090,7 +3098,7 @@ __global__ void __launch_bounds__(c256::THREADS, 1)
           *(uint4*)(bt + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async();
-        mbar_arrive(bar_bk + 8 * s);
+        mbar_arrive(bar_bkf + 8 * kb);
       }
     }
   } else {
@@ -3388,7 +3396,7 @@ static cudaError_t tc_readout256(const void* q, const void* Sfr_hilo, void* out,
 //     P = X_hi Y_hi + X_lo Y_hi + X_hi Y_lo     (M = 128, N = 256, fp32 in TMEM)
 // with X (this half's rows, K = 256) as a K-major bf16 (hi, lo) tile in shared
 // memory and Y = A_t streaming in slices of its operand image through a
-// 4-slot ring (one bulk copy per slice; the next frame's image and U_t rows
+// 6-slot ring (one bulk copy per slice; the next frame's image and U_t rows
 // are prefetched into L2 a step ahead). The fp32 state itself stays in TMEM
 // next to P (columns 256..511). Eight epilogue warps read P and X, apply
 // X <- gamma (X - P) + U_t with U_t read from global memory (L2), write X
@@ -3407,7 +3415,7 @@ constexpr int ATOM = 128 * 128;      // [128 rows][128 B]
 constexpr int XT = 4 * ATOM;         // X hi (or lo) tile, K = 256: 64 KiB
 constexpr int SLICE = 16 * 1024;     // 16 k-rows of the image: hi 8 KiB + lo 8 KiB
 constexpr int NSLICE = D / 16;
-constexpr int NSY = 4;               // Y ring slots
+constexpr int NSY = 6;               // Y ring slots
 constexpr int OFF_XH = 0;
 constexpr int OFF_XL = OFF_XH + XT;
 constexpr int OFF_Y = OFF_XL + XT;
@@ -3415,6 +3423,7 @@ constexpr int OFF_BAR = OFF_Y + NSY * SLICE;
 constexpr int NBAR = 2 * NSY + 3;    // y_full, y_empty, p_full, x_ready, fin
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM = OFF_MISC + 16 + 1024;
+static_assert(SMEM <= 232448, "D = 256 chain shared memory");
 constexpr int EPI = 256;             // 8 epilogue warps
 constexpr int THREADS = 64 + EPI;    // producer warp, MMA warp, epilogue
 constexpr uint32_t TMEM_COLS = 512;  // P: columns 0..255, fp32 state: 256..511

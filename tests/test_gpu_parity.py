@@ -160,6 +160,27 @@ def test_plain_entry_allocates_its_own_scratch():
     assert torch.equal(out, out2) and torch.equal(st, st2)
 
 
+def test_host_streaming_call():
+    """frame_scan_fwd_host (host tensors, heads in chunks through ping-pong
+    device buffers on three streams) equals the device call head by head, and
+    the oracle."""
+    arr = U.random_case(11, 2, 3, 5, 100, 128, bf16=True, state=True)
+    d = U.dev_inputs(arr, True)
+    ref_o, ref_s = run_scan(d, "default")
+    torch.cuda.synchronize()
+    h = {n: (t.cpu().pin_memory() if t is not None else None) for n, t in d.items()
+         if n in ("q", "k", "v", "beta", "gamma", "state")}
+    for hpc in (1, 2, 4):
+        o, s = api.frame_scan_fwd_host(h["q"], h["k"], h["v"], h["beta"], h["gamma"], h["state"],
+                                       heads_per_chunk=hpc)
+        assert not o.is_cuda and not s.is_cuda
+        assert torch.equal(o, ref_o.cpu()) and torch.equal(s, ref_s.cpu()), hpc
+    for b in range(2):
+        for hh in range(3):
+            o_ref, s_ref = U.oracle_slab(arr, b, hh, True)
+            assert U.rel_frob_per_frame(U.host(o[b, hh]), o_ref) < U.TOL_BF16
+
+
 def test_streaming_split_equals_one_call():
     """A rollout split into two calls, carrying the state, equals one call."""
     arr = U.random_case(6, 1, 2, 12, 100, 64, bf16=True, state=True)
