@@ -55,6 +55,11 @@ Pins (tests/test_oracle_pins.py) and their status per function:
                                 orthogonality, identity, relative phase); its
                                 constants (eps, pair layout, axis split) are
                                 readings R8-R10, unpinned by the pages.
+  frame_scan_bwd                the pages print no backward; this is the
+                                adjoint of frame_scan derived by reverse-mode
+                                differentiation, pinned by central finite
+                                differences of frame_scan for every input
+                                (tests/test_oracle_backward.py).
 """
 
 from __future__ import annotations
@@ -76,6 +81,7 @@ __all__ = [
     "relu",
     "rope2d",
     "qk_prologue",
+    "frame_scan_bwd",
 ]
 
 
@@ -304,3 +310,90 @@ def qk_prologue(q_raw, k_raw, w_q, w_k, grid_w, *, eps=1e-6, base=10000.0):
     qh = rope2d(relu(rmsnorm(q_raw, w_q, eps)), grid_w, base)
     kh = rope2d(key_scale(D, S) * relu(rmsnorm(k_raw, w_k, eps)), grid_w, base)
     return qh, kh
+
+
+# ---------------------------------------------------------------------------
+# Backward of the frame scan (adjoint; the pages give no formula)
+# ---------------------------------------------------------------------------
+
+def frame_scan_bwd(q, k, v, beta, gamma, state_in, d_out, d_state_out=None, *,
+                   reverse=False, block=0, keys_scaled=False):
+    """Gradients of a scalar loss through frame_scan for one (b, h), float64.
+
+    Given d_out = dL/dO [T, S, D] and d_state_out = dL/d(state after the last
+    processed frame) [D, D] (or None), returns
+    (dq, dk, dv, dbeta, dgamma, d_state_in) with the shapes of the inputs
+    (d_state_in is zeros when state_in is None).
+
+    Derivation (reverse mode over the scan order j = 0..T-1, frame t_j):
+        X_j = g_j (X'_{j-1} - X'_{j-1} A_j) + U_j,  X'_{j-1} = X_{j-1}, or 0
+              after a reset, or state_in at j = 0;   O_{t_j} = Q_{t_j} X_j^T
+    The total gradient reaching X_j is
+        G_j = dO_{t_j}^T Q_{t_j} + [G_{j+1} M_{j+1}^T unless j+1 resets]
+              (+ d_state_out at the last j),   M = g (I - A),
+    and for frame j:  dU = G_j,  dM = X'_{j-1}^T G_j,
+        dA = -g_j dM,  dg_j = <dM, I - A_j>,  dQ_t = dO_t X_j.
+    Through A = K^^T diag(beta) K^ and U = V^T diag(beta) K^ (rows k^_s, v_s):
+        dk^_s = beta_s ((dA + dA^T) k^_s + dU^T v_s)
+        dv_s  = beta_s dU k^_s
+        dbeta_s = k^_s . dA k^_s + v_s . dU k^_s
+    and dk = c dk^ (c = 1/sqrt(D S) unless keys_scaled). d_state_in is the
+    carry G_0 M_0^T into the state entering the first frame.
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    beta = np.asarray(beta, np.float64)
+    gamma = np.asarray(gamma, np.float64)
+    d_out = np.asarray(d_out, np.float64)
+    T, S, D = q.shape
+    c = 1.0 if keys_scaled else key_scale(D, S)
+    order = scan_order(T, reverse)
+    resets = reset_before(order, block)
+    s0 = np.zeros((D, D)) if state_in is None else np.array(state_in, np.float64)
+    # forward, keeping the state entering each frame (after any reset) and A, U
+    prev, As, states = [], [], []
+    X = s0
+    for t, rst in zip(order, resets):
+        if rst:
+            X = np.zeros((D, D))
+        A, U = frame_terms(c * k[t], v[t], beta[t])
+        prev.append(X)  # state entering frame j (after any reset)
+        As.append(A)
+        X = gamma[t] * (X - X @ A) + U
+        states.append(X)  # state after frame j
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    dbeta = np.zeros_like(beta)
+    dgamma = np.zeros_like(gamma)
+    G_next = None
+    d_s0 = np.zeros((D, D))
+    I = np.eye(D)
+    for j in range(T - 1, -1, -1):
+        t = order[j]
+        G = d_out[t].T @ q[t]
+        if j == T - 1 and d_state_out is not None:
+            G = G + np.asarray(d_state_out, np.float64)
+        if G_next is not None:
+            G = G + G_next
+        dq[t] = d_out[t] @ states[j]
+        A = As[j]
+        dM = prev[j].T @ G
+        dA = -gamma[t] * dM
+        dgamma[t] = np.sum(dM * (I - A))
+        dU = G
+        kh = c * k[t]
+        sym = dA + dA.T
+        dkh = beta[t][:, None] * (kh @ sym.T + v[t] @ dU)
+        dv[t] = beta[t][:, None] * (kh @ dU.T)
+        dbeta[t] = np.einsum("sd,sd->s", kh, kh @ dA.T) + np.einsum("sd,sd->s", v[t] @ dU, kh)
+        dk[t] = c * dkh
+        carry = G @ (gamma[t] * (I - A)).T  # gradient reaching the state entering frame j
+        if resets[j]:
+            G_next = None
+        elif j == 0:
+            d_s0 = carry
+        else:
+            G_next = carry
+    return dq, dk, dv, dbeta, dgamma, d_s0
