@@ -65,6 +65,19 @@ class GdnParams(ctypes.Structure):
     ]
 
 
+class GdnBwdParams(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("beta", ctypes.c_void_p), ("gamma", ctypes.c_void_p), ("state_in", ctypes.c_void_p),
+        ("d_out", ctypes.c_void_p), ("d_state_out", ctypes.c_void_p),
+        ("dq", ctypes.c_void_p), ("dk", ctypes.c_void_p), ("dv", ctypes.c_void_p),
+        ("dbeta", ctypes.c_void_p), ("dgamma", ctypes.c_void_p), ("d_state_in", ctypes.c_void_p),
+        ("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int), ("S", ctypes.c_int),
+        ("D", ctypes.c_int), ("flags", ctypes.c_uint),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _U = ctypes.c_uint
@@ -77,6 +90,8 @@ SIGNATURES = {
     "gdn_frame_scan_fwd_ex": (_I, [ctypes.POINTER(GdnParams), _P]),
     "gdn_frame_scan_fwd_static": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _U, _P]),
     "gdn_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _U]),
+    "gdn_frame_scan_bwd": (_I, [ctypes.POINTER(GdnBwdParams), _P]),
+    "gdn_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _U]),
     "gdn_frame_contract": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _U, _P]),
     "gdn_chunk_composites": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _U, _P]),
     "gdn_check_device_status": (_I, [_P]),
@@ -319,6 +334,47 @@ def frame_scan_fwd_host(q, k, v, beta, gamma, state_in=None, *, out=None, state_
     # the copies out land in host memory: wait for them before returning
     torch.cuda.current_stream(dev).synchronize()
     return out, state_out
+
+
+def frame_scan_bwd(q, k, v, beta, gamma, state_in, d_out, d_state_out=None, *, reverse=False,
+                   block_reset=False, block=3, keys_scaled=False, want_state_in_grad=True,
+                   workspace=None, stream=None):
+    """Gradients through the frame scan (gdn_frame_scan_bwd): given
+    d_out = dL/dO [B,H,T,S,D] and d_state_out = dL/d(state_out) [B,H,D,D]
+    (or None), returns (dq, dk, dv, dbeta, dgamma, d_state_in) for the scan
+    with the same flags (d_state_in None unless want_state_in_grad)."""
+    B, H, T, S, D = q.shape
+    bf16 = q.dtype == torch.bfloat16
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (d_out, "d_out")):
+        _want(t, n, q.dtype, (B, H, T, S, D))
+    _want(beta, "beta", torch.float32, (B, H, T, S))
+    _want(gamma, "gamma", torch.float32, (B, H, T))
+    if state_in is not None:
+        _want(state_in, "state_in", torch.float32, (B, H, D, D))
+    if d_state_out is not None:
+        _want(d_state_out, "d_state_out", torch.float32, (B, H, D, D))
+    flags = scan_flags(bf16=bf16, reverse=reverse, block_reset=block_reset, block=block,
+                       keys_scaled=keys_scaled)
+    flags &= ~(CHUNKED | NO_OVERLAP | 0xFF0000)  # plan bits do not apply to the backward
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dbeta, dgamma = torch.empty_like(beta), torch.empty_like(gamma)
+    ds0 = torch.empty((B, H, D, D), device=q.device, dtype=torch.float32) \
+        if want_state_in_grad else None
+    need = int(lib().gdn_bwd_workspace_bytes(B, H, T, S, D, flags))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=q.device, dtype=torch.uint8)
+    p = GdnBwdParams()
+    p.q, p.k, p.v = _ptr(q), _ptr(k), _ptr(v)
+    p.beta, p.gamma, p.state_in = _ptr(beta), _ptr(gamma), _ptr(state_in)
+    p.d_out, p.d_state_out = _ptr(d_out), _ptr(d_state_out)
+    p.dq, p.dk, p.dv = _ptr(dq), _ptr(dk), _ptr(dv)
+    p.dbeta, p.dgamma, p.d_state_in = _ptr(dbeta), _ptr(dgamma), _ptr(ds0)
+    p.B, p.H, p.T, p.S, p.D = B, H, T, S, D
+    p.flags = flags
+    p.workspace = workspace.data_ptr()
+    p.workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().gdn_frame_scan_bwd(ctypes.byref(p), _stream(stream)), "gdn_frame_scan_bwd")
+    return dq, dk, dv, dbeta, dgamma, ds0
 
 
 STATIC_SCRATCH_BYTES = 32 << 20

@@ -430,6 +430,121 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
                        tc_chain_ok, tc_readout_ok, ppq, st, L.Sfr, true);
 }
 
+// ---- backward --------------------------------------------------------------
+struct BwdLayout {
+  size_t A, U, Sfr, W, G, dM, P2, P3, P5, total;
+};
+
+static BwdLayout make_bwd_layout(int B, int H, int T, int S, int D) {
+  BwdLayout L;
+  const size_t frames = (size_t)B * H * T;
+  const size_t mat = frames * D * D * sizeof(float);
+  const size_t tok = frames * S * D * sizeof(float);
+  size_t off = 0;
+  size_t* mats[] = {&L.A, &L.U, &L.Sfr, &L.W, &L.G, &L.dM};
+  for (size_t* m : mats) {
+    *m = off;
+    off = align256(off + mat);
+  }
+  size_t* toks[] = {&L.P2, &L.P3, &L.P5};
+  for (size_t* m : toks) {
+    *m = off;
+    off = align256(off + tok);
+  }
+  L.total = off;
+  return L;
+}
+
+static int scan_bwd(const gdn_bwd_params& p, cudaStream_t st) {
+  int rc = check_sizes(p.B, p.H, p.T, p.S, p.D);
+  if (rc) return rc;
+  const unsigned f = p.flags;
+  const unsigned allowed = GDN_BF16 | GDN_REVERSE | GDN_BLOCK_RESET | GDN_KEYS_SCALED |
+                           GDN_FORCE_SIMT | (0xffu << 8) | (0xffu << 16);
+  if (f & ~allowed) return fail(GDN_ERR_INVALID, "gdn_frame_scan_bwd: unsupported flag%s");
+  if (!p.q || !p.k || !p.v || !p.beta || !p.gamma || !p.d_out || !p.dq || !p.dk || !p.dv ||
+      !p.dbeta || !p.dgamma)
+    return fail(GDN_ERR_INVALID, "null input or gradient pointer%s");
+  const void* ptrs[] = {p.q, p.k, p.v, p.beta, p.gamma, p.d_out, p.dq, p.dk, p.dv, p.dbeta,
+                        p.dgamma};
+  for (const void* x : ptrs)
+    if (!aligned16(x)) return fail(GDN_ERR_INVALID, "pointers must be 16-byte aligned%s");
+  const void* outs[] = {p.dq, p.dk, p.dv};
+  const void* ins[] = {p.q, p.k, p.v, p.d_out};
+  for (const void* o : outs)
+    for (const void* i : ins)
+      if (o == i) return fail(GDN_ERR_INVALID, "gradients must not alias inputs%s");
+  const BwdLayout L = make_bwd_layout(p.B, p.H, p.T, p.S, p.D);
+  if (!p.workspace || p.workspace_bytes < L.total)
+    return fail(GDN_ERR_WORKSPACE, "workspace missing or smaller than gdn_bwd_workspace_bytes%s");
+  if (((uintptr_t)p.workspace & 255u) != 0)
+    return fail(GDN_ERR_INVALID, "workspace must be 256-byte aligned%s");
+
+  const bool bf16 = (f & GDN_BF16) != 0;
+  const bool reverse = (f & GDN_REVERSE) != 0;
+  const bool block_reset = (f & GDN_BLOCK_RESET) != 0;
+  const int block = block_len(f);
+  const long long frames = (long long)p.B * p.H * p.T;
+  const double c = (f & GDN_KEYS_SCALED) ? 1.0 : 1.0 / std::sqrt((double)p.D * (double)p.S);
+  char* ws = (char*)p.workspace;
+  float* A = (float*)(ws + L.A);
+  float* U = (float*)(ws + L.U);
+  float* Sfr = (float*)(ws + L.Sfr);
+  float* W = (float*)(ws + L.W);
+  float* G = (float*)(ws + L.G);
+  float* dM = (float*)(ws + L.dM);
+  float* P2 = (float*)(ws + L.P2);
+  float* P3 = (float*)(ws + L.P3);
+  float* P5 = (float*)(ws + L.P5);
+  cudaError_t e;
+  // 1. forward recompute: A_t, U_t, then the states S_t (one chain per head)
+  e = simt_contract(bf16, p.k, p.v, p.beta, A, U, frames, p.S, p.D, (float)(c * c), (float)c, st);
+  if (e != cudaSuccess) return cuda_fail(e, "backward: contract");
+  ChainArgs a;
+  memset(&a, 0, sizeof(a));
+  a.mode = CHAIN_SCAN;
+  a.seg = SEG_SEQUENTIAL;
+  a.D = p.D;
+  a.T = p.T;
+  a.L = 1;
+  a.block = block;
+  a.seq_reset = block_reset ? 1 : 0;
+  a.reverse = reverse ? 1 : 0;
+  a.nseg = 1;
+  a.heads = p.B * p.H;
+  a.A = A;
+  a.U = U;
+  a.gamma = p.gamma;
+  a.state_in = p.state_in;
+  a.Sfr = Sfr;
+  if ((e = simt_chain(a, a.heads, st)) != cudaSuccess) return cuda_fail(e, "backward: states");
+  // 2. W_t = dO_t^T Q_t (the contraction's U with keys := q, values := dO, beta = 1)
+  e = simt_contract(bf16, p.q, p.d_out, nullptr, nullptr, W, frames, p.S, p.D, 1.f, 1.f, st);
+  if (e != cudaSuccess) return cuda_fail(e, "backward: dO^T Q");
+  // 3. adjoint chain: G_t per frame, and the state_in gradient
+  ChainArgs b = a;
+  b.mode = CHAIN_ADJOINT;
+  b.Zw = W;
+  b.Gout = G;
+  b.dS_out = p.d_state_out;
+  b.dS_in = p.d_state_in;
+  if ((e = simt_chain(b, b.heads, st)) != cudaSuccess) return cuda_fail(e, "backward: adjoint chain");
+  // 4. per frame: dM = S'^T G -> dA + dA^T, dgamma
+  e = simt_bwd_dm(Sfr, p.state_in, G, dM, frames, p.T, p.D, a.reverse, a.seq_reset, block, st);
+  if (e == cudaSuccess) e = simt_bwd_dterm(dM, A, p.gamma, p.dgamma, frames, p.D, st);
+  if (e != cudaSuccess) return cuda_fail(e, "backward: per-frame terms");
+  // 5. per token: K^ (dA + dA^T), V G, K^ G^T, dQ = dO S_t; then dk, dv, dbeta
+  e = simt_rowmat(bf16, true, 0, p.k, dM, P2, frames, p.S, p.D, (float)c, st);
+  if (e == cudaSuccess) e = simt_rowmat(bf16, true, 1, p.v, G, P3, frames, p.S, p.D, 1.f, st);
+  if (e == cudaSuccess) e = simt_rowmat(bf16, true, 0, p.k, G, P5, frames, p.S, p.D, (float)c, st);
+  if (e == cudaSuccess) e = simt_rowmat(bf16, !bf16, 1, p.d_out, Sfr, p.dq, frames, p.S, p.D, 1.f, st);
+  if (e == cudaSuccess)
+    e = simt_bwd_combine(bf16, p.k, p.beta, P2, P3, P5, p.dk, p.dv, p.dbeta, frames * p.S, p.D,
+                         (float)c, st);
+  if (e != cudaSuccess) return cuda_fail(e, "backward: token gradients");
+  return GDN_OK;
+}
+
 int scan_ex_entry(const gdn_params& p, cudaStream_t st) {
   t_last_error.clear();
   return scan_ex(p, st);
@@ -466,6 +581,18 @@ long long gdn_launch_count(int reset) {
   long long n = t_launches;
   if (reset) t_launches = 0;
   return n;
+}
+
+int gdn_frame_scan_bwd(const gdn_bwd_params* p, gdn_stream_t stream) {
+  t_last_error.clear();
+  if (!p) return fail(GDN_ERR_INVALID, "null params%s");
+  return scan_bwd(*p, (cudaStream_t)stream);
+}
+
+size_t gdn_bwd_workspace_bytes(int B, int H, int T, int S, int D, unsigned flags) {
+  (void)flags;
+  if (B < 1 || H < 1 || T < 1 || S < 1 || D < 1) return 0;
+  return make_bwd_layout(B, H, T, S, D).total;
 }
 
 size_t gdn_workspace_bytes(int B, int H, int T, int S, int D, unsigned flags) {

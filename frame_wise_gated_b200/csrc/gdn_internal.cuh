@@ -40,6 +40,7 @@ enum ChainMode : int {
   CHAIN_SCAN = 0,     // S <- gamma (S - S A) + U per frame, store S_t
   CHAIN_COMPOSE = 1,  // per span: E <- E + A - E A and H <- gamma (H - H A) + U
   CHAIN_PREFIX = 2,   // per head: S_start(p+1) = g_p (S_start(p) - S_start(p) E_p) + H_p
+  CHAIN_ADJOINT = 3,  // backward: per head, G_j = W_j + g_{j+1} (G_{j+1} - G_{j+1} A_{j+1})
 };
 
 // Everything the chain kernels need; pointers are device pointers.
@@ -67,6 +68,11 @@ struct ChainArgs {
   int y_image;            // A (and E for the prefix) are stored as bf16 operand images
   int e_image;            // the compose chain writes E as an operand image
   int sst_hilo;           // Sst holds [heads*nseg][2][D][D] bf16 (hi, lo) pairs
+  // backward (CHAIN_ADJOINT)
+  const float* Zw;        // [heads*T, D, D] W_t = dO_t^T Q_t
+  float* Gout;            // [heads*T, D, D] total state gradients G_t
+  const float* dS_out;    // [heads, D, D] gradient of state_out, or null
+  float* dS_in;           // [heads, D, D] gradient of state_in, or null
 };
 
 // An "operand image" of a D x D fp32 matrix M (D = 128) is the exact
@@ -126,6 +132,22 @@ cudaError_t simt_contract(bool bf16, const void* k, const void* v, const float* 
 cudaError_t simt_chain(const ChainArgs& a, int nchains, cudaStream_t st);
 cudaError_t simt_readout(bool bf16, const void* q, const float* Sfr, void* out, long long N,
                          int S, int D, cudaStream_t st);
+
+// ---- backward (CUDA cores) ------------------------------------------------------
+// dM_j = S'_j^T G_j per frame (S'_j: state entering frame j of the scan order).
+cudaError_t simt_bwd_dm(const float* Sfr, const float* state_in, const float* G, float* dM,
+                        long long N, int T, int D, int reverse, int seq_reset, int block,
+                        cudaStream_t st);
+// In place dM -> dA + dA^T = -gamma (dM + dM^T); dgamma = <dM, I - A>.
+cudaError_t simt_bwd_dterm(float* dM, const float* A, const float* gamma, float* dgamma,
+                           long long N, int D, cudaStream_t st);
+// Per frame n: out[s, :] = scale * x[s, :] M_n^T (trans = 0) or x[s, :] M_n (trans = 1).
+cudaError_t simt_rowmat(bool bf16_in, bool f32_out, int trans, const void* x, const float* M,
+                        void* out, long long N, int S, int D, float scale, cudaStream_t st);
+// dk, dv, dbeta per token from the products P2, P3, P5.
+cudaError_t simt_bwd_combine(bool bf16, const void* k, const float* beta, const float* P2,
+                             const float* P3, const float* P5, void* dk, void* dv, float* dbeta,
+                             long long ntok, int D, float c, cudaStream_t st);
 
 // ---- tensor-core (tcgen05) kernels, bf16, sm_100a -------------------------------
 // Prologue applied inside the tensor-core loaders (RMSNorm -> ReLU -> 2-D RoPE;

@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(256)
   const int ti = blockIdx.y / nt, tj = blockIdx.y % nt;
   const T* kf = k + (size_t)n * S * D;
   const T* vf = v + (size_t)n * S * D;
-  const float* bf = beta + (size_t)n * S;
+  const float* bf = beta ? beta + (size_t)n * S : nullptr;  // null: beta = 1
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   float accA[R][R], accU[R][R];
 #pragma unroll
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(256)
       float ki = 0.f, kj = 0.f, vi = 0.f;
       if (s < S) {
         ki = ldf(kf + (size_t)s * D + ti * TILE + c);
-        kj = ldf(kf + (size_t)s * D + tj * TILE + c) * bf[s];
+        kj = ldf(kf + (size_t)s * D + tj * TILE + c) * (bf ? bf[s] : 1.0f);
         vi = ldf(vf + (size_t)s * D + ti * TILE + c);
       }
       Ki[r][c] = ki;
@@ -144,14 +144,14 @@ __global__ void __launch_bounds__(256)
     }
     __syncthreads();
   }
-  float* An = A + (size_t)n * D * D;
+  float* An = A ? A + (size_t)n * D * D : nullptr;
   float* Un = U + (size_t)n * D * D;
 #pragma unroll
   for (int i = 0; i < R; ++i)
 #pragma unroll
     for (int j = 0; j < R; ++j) {
       const size_t idx = (size_t)(ti * TILE + ty * R + i) * D + tj * TILE + tx * R + j;
-      An[idx] = accA[i][j] * cA;
+      if (A) An[idx] = accA[i][j] * cA;  // null A: only U is wanted
       Un[idx] = accU[i][j] * cU;
     }
 }
@@ -203,7 +203,7 @@ __device__ __forceinline__ void chain_step(float* X, float* Yc, const float* __r
   float acc[NM];
 #pragma unroll
   for (int m = 0; m < NM; ++m) acc[m] = 0.f;
-  for (int k0 = 0; k0 < D; k0 += 16) {
+  for (int k0 = 0; Y && k0 < D; k0 += 16) {  // null Y: X Y = 0
     for (int e = threadIdx.x; e < 16 * D; e += 256) Yc[e] = Y[(size_t)k0 * D + e];
     __syncthreads();
 #pragma unroll 4
@@ -218,7 +218,7 @@ __device__ __forceinline__ void chain_step(float* X, float* Yc, const float* __r
 #pragma unroll
   for (int m = 0; m < NM; ++m) {
     const int c = l + 16 * m;
-    const float z = Z[(size_t)row * D + c];
+    const float z = Z ? Z[(size_t)row * D + c] : 0.f;
     X[r * D + c] = reset ? z : alpha * (X[r * D + c] - acc[m]) + z;
   }
   __syncthreads();
@@ -307,6 +307,32 @@ __global__ void __launch_bounds__(256) k_chain_simt(ChainArgs a) {
     const size_t si = (size_t)bh * a.nseg + p;
     rows_store(X, (which ? a.Hc : a.E) + si * D * D, D, row0);
     if (!which && blockIdx.y == 0 && threadIdx.x == 0) a.g[si] = gp;
+  } else if (a.mode == CHAIN_ADJOINT) {
+    // Adjoint of a sequential scan (backward pass): per head, scan positions
+    // j = T-1 .. 0; G_j = W_j + g_{j+1} (G_{j+1} - G_{j+1} A_{j+1}) with the
+    // carry cut where the forward scan reset the state before position j+1,
+    // and G_{T-1} = W_{T-1} + dL/d(state_out). Each G_j is stored; finally the
+    // gradient of state_in, g_0 (G_0 - G_0 A_0).
+    const int bh = c;
+    rows_load(X, a.dS_out ? a.dS_out + (size_t)bh * D * D : nullptr, D, row0);
+    for (int j = T - 1; j >= 0; --j) {
+      const int t = frame_at(j, T, a.reverse);
+      const size_t fi = (size_t)bh * T + t;
+      if (j == T - 1) {
+        chain_step<D>(X, Yc, nullptr, a.Zw + fi * D * D, 1.0f, row0, false);
+      } else {
+        const int tn = frame_at(j + 1, T, a.reverse);
+        const bool cut = a.seq_reset && (t / a.block) != (tn / a.block);
+        const size_t fn = (size_t)bh * T + tn;
+        chain_step<D>(X, Yc, a.A + fn * D * D, a.Zw + fi * D * D, a.gamma[fn], row0, cut);
+      }
+      rows_store(X, a.Gout + fi * D * D, D, row0);
+    }
+    if (a.dS_in) {
+      const size_t f0 = (size_t)bh * T + frame_at(0, T, a.reverse);
+      chain_step<D>(X, Yc, a.A + f0 * D * D, nullptr, a.gamma[f0], row0, false);
+      rows_store(X, a.dS_in + (size_t)bh * D * D, D, row0);
+    }
   } else {  // CHAIN_PREFIX
     const int bh = c;
     rows_load(X, a.state_in ? a.state_in + (size_t)bh * D * D : nullptr, D, row0);

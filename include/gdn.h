@@ -210,6 +210,51 @@ GDN_API int gdn_frame_scan_fwd_static(const void* q, const void* k, const void* 
                                       int H, int T, int S, int D, unsigned flags,
                                       gdn_stream_t stream);
 
+/*
+ * gdn_frame_scan_bwd — gradients of a loss through gdn_frame_scan_fwd.
+ * (The pages print no backward; this is the adjoint of the same recurrence,
+ * derived by reverse-mode differentiation.) Given dL/dO and optionally
+ * dL/d(state_out), it returns dL/dq, dL/dk, dL/dv, dL/dbeta, dL/dgamma and
+ * optionally dL/d(state_in) for the scan the same flags describe:
+ *   G_j  = dO^T Q + gamma' (G' - G' A')       (G' of the next frame in scan
+ *          order, cut where the forward scan reset the state; the last frame
+ *          adds dL/d(state_out))
+ *   dq   = dO S_t,  dM = S'^T G (S': the state entering the frame),
+ *   dA   = -gamma dM,  dgamma = <dM, I - A>,  dU = G,
+ *   dk   = beta (K^ (dA + dA^T) + V G) / sqrt(D S),  dv = beta K^ G^T,
+ *   dbeta_s = k^_s . (K^ (dA + dA^T) / 2 + V G)_s.
+ * Forward quantities (A_t, U_t, the states) are recomputed inside the call.
+ * Layouts and dtypes as gdn_frame_scan_fwd: d_out, dq, dk, dv like q;
+ * dbeta like beta; dgamma like gamma; d_state_out, d_state_in [B,H,D,D] fp32
+ * (either may be NULL). Flags: GDN_BF16, GDN_REVERSE, GDN_BLOCK_RESET,
+ * GDN_MAKE_BLOCK(n), GDN_KEYS_SCALED; others return GDN_ERR_INVALID.
+ * Scratch: the caller's workspace of gdn_bwd_workspace_bytes (256-byte
+ * aligned). Returns GDN_OK or a negative status.
+ */
+typedef struct gdn_bwd_params {
+  const void* q;            /* [B,H,T,S,D] */
+  const void* k;            /* [B,H,T,S,D] */
+  const void* v;            /* [B,H,T,S,D] */
+  const float* beta;        /* [B,H,T,S] */
+  const float* gamma;       /* [B,H,T] */
+  const float* state_in;    /* [B,H,D,D] or NULL (zeros) */
+  const void* d_out;        /* [B,H,T,S,D] dL/dO */
+  const float* d_state_out; /* [B,H,D,D] dL/d(state_out) or NULL (zero) */
+  void* dq;                 /* [B,H,T,S,D] */
+  void* dk;                 /* [B,H,T,S,D] */
+  void* dv;                 /* [B,H,T,S,D] */
+  float* dbeta;             /* [B,H,T,S] */
+  float* dgamma;            /* [B,H,T] */
+  float* d_state_in;        /* [B,H,D,D] or NULL (not written) */
+  int B, H, T, S, D;
+  unsigned flags;
+  void* workspace;          /* device scratch, 256-byte aligned */
+  size_t workspace_bytes;   /* >= gdn_bwd_workspace_bytes(B,H,T,S,D,flags) */
+} gdn_bwd_params;
+
+GDN_API int gdn_frame_scan_bwd(const gdn_bwd_params* p, gdn_stream_t stream);
+GDN_API size_t gdn_bwd_workspace_bytes(int B, int H, int T, int S, int D, unsigned flags);
+
 /* Bytes of scratch gdn_frame_scan_fwd_ex needs for these sizes and flags
  * (0 on invalid sizes). */
 GDN_API size_t gdn_workspace_bytes(int B, int H, int T, int S, int D, unsigned flags);

@@ -1,0 +1,105 @@
+"""GPU parity of the backward pass (gdn_frame_scan_bwd) against the oracle's
+adjoint (pinned by finite differences), through the C ABI.
+
+Metric: per (b, h) slab and per gradient tensor, ||g_gpu - g_ref||_F /
+||g_ref||_F; bounds as the forward: 1e-4 for fp32 inputs, 1e-2 for bf16
+inputs (the same bf16-rounded inputs and upstream gradients go to the oracle).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from frame_wise_gated_b200 import api, synth
+from oracle import gdn_oracle as O
+from tests import gdn_testutil as U
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ("dq", "dk", "dv", "dbeta", "dgamma", "d_state_in")
+
+
+def rel(got, ref):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    return float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+
+
+def upstream(seed, B, H, T, S, D, bf16):
+    rng = np.random.default_rng(seed)
+    dO = rng.standard_normal((B, H, T, S, D), dtype=np.float32)
+    dO = synth.bf16_round_bits(dO) if bf16 else dO
+    dS = rng.standard_normal((B, H, D, D)).astype(np.float32)
+    return dO, dS
+
+
+def check_case(arr, dO, dS, bf16, tol, reverse=False, block=0, b_slabs=None):
+    d = U.dev_inputs(arr, bf16)
+    d_out = U.to_dev(dO, bf16)
+    d_s = torch.from_numpy(dS).cuda() if dS is not None else None
+    got = api.frame_scan_bwd(d["q"], d["k"], d["v"], d["beta"], d["gamma"], d["state"], d_out,
+                             d_s, reverse=reverse, block_reset=bool(block), block=block or 3)
+    torch.cuda.synchronize()
+    api.check_device_status()
+    B, H = arr["beta"].shape[:2]
+    slabs = b_slabs or [(b, h) for b in range(B) for h in range(H)]
+    worst = {}
+    for (b, h) in slabs:
+        ref = O.frame_scan_bwd(U.widen(arr["q"][b, h], bf16), U.widen(arr["k"][b, h], bf16),
+                               U.widen(arr["v"][b, h], bf16), arr["beta"][b, h].astype(np.float64),
+                               arr["gamma"][b, h].astype(np.float64),
+                               None if arr["state"] is None else arr["state"][b, h],
+                               U.widen(dO[b, h], bf16), None if dS is None else dS[b, h],
+                               reverse=reverse, block=block)
+        for name, g, r in zip(NAMES, got, ref):
+            if g is None:
+                continue
+            e = rel(U.host(g[b, h]), r)
+            worst[name] = max(worst.get(name, 0.0), e)
+    for name, e in worst.items():
+        assert e < tol, (name, e, worst)
+    return worst
+
+
+MODES = {"forward": dict(), "reverse": dict(reverse=True), "forward_block": dict(block=3),
+         "reverse_block": dict(reverse=True, block=3)}
+
+
+@pytest.mark.parametrize("mode", list(MODES))
+@pytest.mark.parametrize("D,bf16", [(16, False), (64, False), (128, False), (64, True),
+                                    (128, True), (256, True)])
+def test_backward_small(D, bf16, mode):
+    B, H, T, S = 2, 1, 7, 50
+    arr = U.random_case(3000 + D, B, H, T, S, D, bf16=bf16, state=True)
+    dO, dS = upstream(17 + D, B, H, T, S, D, bf16)
+    check_case(arr, dO, dS, bf16, U.TOL_BF16 if bf16 else U.TOL_FP32, **MODES[mode])
+
+
+def test_backward_without_state_terms():
+    """No state_in, no gradient of state_out: the pure output loss."""
+    arr = U.random_case(41, 1, 2, 5, 33, 32, bf16=False, state=False)
+    dO, _ = upstream(42, 1, 2, 5, 33, 32, False)
+    check_case(arr, dO, None, False, U.TOL_FP32)
+
+
+def test_backward_edge_sizes():
+    for (T, S, D) in [(1, 1, 16), (1, 5, 64), (2, 129, 128), (9, 1, 128)]:
+        arr = U.random_case(T * S + D + 7, 1, 1, T, S, D, bf16=True, state=True)
+        dO, dS = upstream(T + S + D, 1, 1, T, S, D, True)
+        check_case(arr, dO, dS, True, U.TOL_BF16)
+
+
+def test_backward_full_size_clip():
+    """The 5 s 720p clip (B=1, H=16, T=21, S=3600, D=128, bf16), sampled slabs."""
+    cfg = synth.CONFIGS["clip5s_720p"]
+    arr = synth.make_inputs(cfg)
+    dO, dS = upstream(2024, cfg.B, cfg.H, cfg.T, cfg.S, cfg.D, True)
+    check_case(arr, dO, dS, True, U.TOL_BF16, b_slabs=[(0, 0), (0, cfg.H - 1)])
+
+
+def test_backward_bad_arguments_fail_loudly():
+    arr = U.random_case(9, 1, 1, 2, 8, 16, bf16=False)
+    d = U.dev_inputs(arr, False)
+    with pytest.raises(api.GdnError):
+        api.frame_scan_bwd(d["q"], d["k"], d["v"], d["beta"], d["gamma"], None, d["q"],
+                           workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
