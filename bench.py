@@ -43,6 +43,7 @@ from frame_wise_gated_b200 import synth  # noqa: E402
 
 METRIC = "GDN frame-scan frame·head·tokens/s (% of HBM roofline), 1xB200"
 UNIT = "frame·head·tokens/s"
+METRIC_BWD = "GDN frame-scan BACKWARD frame·head·tokens/s (% of HBM roofline), 1xB200"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -63,6 +64,15 @@ def algorithmic_bytes(cfg, step=True):
     per_fh = cfg.S * (n_t * cfg.D * e + 4) + 4
     state = 2 * cfg.D * cfg.D * 4
     return cfg.frame_heads * per_fh + cfg.B * cfg.H * state
+
+
+def backward_bytes(cfg):
+    """Bytes the backward must move per step: q, k, v and dL/dO in, dq, dk, dv
+    out, beta in and dbeta out, gamma in and dgamma out, the state and its
+    gradients (state_in, dL/d(state_out) in; dL/d(state_in) out)."""
+    e = 2 if cfg.bf16 else 4
+    per_fh = cfg.S * (7 * cfg.D * e + 8) + 8
+    return cfg.frame_heads * per_fh + cfg.B * cfg.H * 3 * cfg.D * cfg.D * 4
 
 
 def phase_bytes(cfg):
@@ -333,6 +343,21 @@ def run_ours(args, cfg):
         api.frame_scan_fwd_ex(q, k, v, beta, gamma, s0, out=out, state_out=st_out,
                               out_rev=out_rev, state_out_rev=st_rev, workspace=ws, **kw)
 
+    if args.bwd:
+        # the backward pass: upstream gradients dL/dO and dL/d(state_out), seeded
+        if cfg.prologue:
+            raise SystemExit("--bwd: the backward covers the scan without the prologue")
+        g = torch.Generator(device="cpu").manual_seed(7)
+        d_out = torch.randn(q.shape, generator=g).to(dtype=q.dtype, device=dev)
+        d_st = torch.randn((cfg.B, cfg.H, cfg.D, cfg.D), generator=g).to(dev)
+        flags_b = api.scan_flags(bf16=cfg.bf16)
+        ws_b = torch.empty(int(api.lib().gdn_bwd_workspace_bytes(cfg.B, cfg.H, cfg.T, cfg.S, cfg.D,
+                                                                 flags_b)),
+                           device=dev, dtype=torch.uint8)
+
+        def step():  # noqa: F811
+            api.frame_scan_bwd(q, k, v, beta, gamma, s0, d_out, d_st, workspace=ws_b)
+
     def barrier():
         if dist is not None:
             dist.barrier()
@@ -369,42 +394,54 @@ def run_ours(args, cfg):
     # ---- dominant kernel roofline (live per-kernel events over the timed region) ----
     hbm, bf16_tf, peak_kind = peaks()
     pb = phase_bytes(cfg)
-    dom_all = max((p for p in phases if phases[p][1] > 0), key=lambda p: phases[p][0])
-    dom = max((p for p in phases if phases[p][1] > 0 and p in pb), key=lambda p: phases[p][0])
-    dom_ms = phases[dom][0] / phases[dom][1]
-    alg = pb.get(dom)
     roof = None
-    if alg is not None:
+    timed = [p for p in phases if phases[p][1] > 0]
+    dom_all = max(timed, key=lambda p: phases[p][0]) if timed else None
+    cand = [p for p in timed if p in pb]
+    alg = None
+    if cand:
+        dom = max(cand, key=lambda p: phases[p][0])
+        dom_ms = phases[dom][0] / phases[dom][1]
+        alg = pb.get(dom)
+    if alg is not None and not args.bwd:
         ach = alg / (dom_ms * 1e-3) / 1e9
         traffic = ncu_traffic(dom, cfg.name)
         roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
                 "frac": ach / hbm, "traffic": traffic, "peak_source": peak_kind,
                 "alg_bytes_per_launch": alg, "ms_per_launch": dom_ms,
                 "dominant_kernel_overall": dom_all}
-    step_bytes = algorithmic_bytes(cfg)
+    step_bytes = algorithmic_bytes(cfg) if not args.bwd else backward_bytes(cfg)
+    if args.bwd:
+        ach = step_bytes / (ms_step * 1e-3) / 1e9
+        roof = {"kernel": "backward step (all kernels)", "bound": "hbm", "achieved": ach,
+                "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "traffic": None,
+                "peak_source": peak_kind, "alg_bytes_per_launch": step_bytes,
+                "ms_per_launch": ms_step}
     step_roof = {"alg_bytes_per_step": step_bytes, "achieved_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
                  "frac": step_bytes / (ms_step * 1e-3) / 1e9 / hbm}
 
     # ---- end to end through the C ABI with host buffers ----
     e2e = None
-    if args.e2e_steps > 0:
+    if args.e2e_steps > 0 and not args.bwd:
         e2e = run_e2e(args, cfg, arr, dev, api, barrier, dist, world)
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.bwd:
         val, dt, desc = cpu_oracle_budget(cfg, seconds=args.cpu_seconds)
         cpu = {"value": val, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
                "sample": f"{desc}; {dt:.1f} s of float64 NumPy oracle (BLAS threads = all cores)"}
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "metric": METRIC if not args.bwd else METRIC_BWD, "value": value, "unit": UNIT,
+            "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if cfg.bf16 else "f32", "data": "synthetic",
             "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "T": cfg.T, "S": cfg.S,
                        "D": cfg.D, "grid": f"{cfg.grid_w}x{cfg.grid_h}",
-                       "scan": plan_desc(args.plan, phases),
+                       "scan": plan_desc(args.plan, phases) if not args.bwd else
+                       "backward: recompute, adjoint chain, per-frame and per-token gradients",
                        "prologue": cfg.prologue, "bidir_block": cfg.bidir_block,
                        "l2": f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB algorithmic per step)",
                        "parallelism": f"replica x{world} (heads shard, no collective)"},
@@ -480,6 +517,8 @@ def main():
                          "(alongside the contraction, or as their own launch)")
     ap.add_argument("--fused-replay", action="store_true",
                     help="replay spans inside the readout kernel")
+    ap.add_argument("--bwd", action="store_true",
+                    help="time the backward pass (gdn_frame_scan_bwd) instead of the forward")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-frames", type=int, default=6,

@@ -105,7 +105,7 @@ SIGNATURES = {
 }
 
 PHASES = ("prologue", "contract", "compose", "prefix", "scan", "readout", "scan_readout",
-          "contract_scan")
+          "contract_scan", "bwd_recompute", "bwd_w", "bwd_adjoint", "bwd_frame", "bwd_tokens")
 
 _lib = None
 
@@ -338,7 +338,7 @@ def frame_scan_fwd_host(q, k, v, beta, gamma, state_in=None, *, out=None, state_
 
 def frame_scan_bwd(q, k, v, beta, gamma, state_in, d_out, d_state_out=None, *, reverse=False,
                    block_reset=False, block=3, keys_scaled=False, want_state_in_grad=True,
-                   workspace=None, stream=None):
+                   force_simt=False, workspace=None, stream=None):
     """Gradients through the frame scan (gdn_frame_scan_bwd): given
     d_out = dL/dO [B,H,T,S,D] and d_state_out = dL/d(state_out) [B,H,D,D]
     (or None), returns (dq, dk, dv, dbeta, dgamma, d_state_in) for the scan
@@ -354,7 +354,7 @@ def frame_scan_bwd(q, k, v, beta, gamma, state_in, d_out, d_state_out=None, *, r
     if d_state_out is not None:
         _want(d_state_out, "d_state_out", torch.float32, (B, H, D, D))
     flags = scan_flags(bf16=bf16, reverse=reverse, block_reset=block_reset, block=block,
-                       keys_scaled=keys_scaled)
+                       keys_scaled=keys_scaled, force_simt=force_simt)
     flags &= ~(CHUNKED | NO_OVERLAP | 0xFF0000)  # plan bits do not apply to the backward
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     dbeta, dgamma = torch.empty_like(beta), torch.empty_like(gamma)

@@ -31,7 +31,8 @@ void count_launch(int n) { t_launches += n; }
 // ---- phase timing with CUDA events (gdn_profile_enable / gdn_profile_read) ----
 enum Phase {
   PH_PROLOGUE = 0, PH_CONTRACT, PH_COMPOSE, PH_PREFIX, PH_SCAN, PH_READOUT, PH_SCAN_READOUT,
-  PH_CONTRACT_SCAN, PH_COUNT
+  PH_CONTRACT_SCAN, PH_BWD_RECOMPUTE, PH_BWD_W, PH_BWD_ADJOINT, PH_BWD_FRAME, PH_BWD_TOKENS,
+  PH_COUNT
 };
 struct ProfRec {
   int phase;
@@ -431,28 +432,147 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
 }
 
 // ---- backward --------------------------------------------------------------
+// The tensor-core backward (D = 128, bf16) keeps per-frame matrices only; the
+// CUDA-core one also stages three fp32 token products.
+static bool bwd_tc_by_flags(int D, unsigned flags) {
+  return D == 128 && (flags & GDN_BF16) && !(flags & GDN_FORCE_SIMT);
+}
+
 struct BwdLayout {
-  size_t A, U, Sfr, W, G, dM, P2, P3, P5, total;
+  size_t A, U, Sfr, W, G, dM, Bimg, zero, flags, P2, P3, P5, total;
 };
 
-static BwdLayout make_bwd_layout(int B, int H, int T, int S, int D) {
+static BwdLayout make_bwd_layout(int B, int H, int T, int S, int D, unsigned f) {
   BwdLayout L;
   const size_t frames = (size_t)B * H * T;
   const size_t mat = frames * D * D * sizeof(float);
   const size_t tok = frames * S * D * sizeof(float);
+  const bool tc = bwd_tc_by_flags(D, f);
   size_t off = 0;
   size_t* mats[] = {&L.A, &L.U, &L.Sfr, &L.W, &L.G, &L.dM};
   for (size_t* m : mats) {
     *m = off;
     off = align256(off + mat);
   }
-  size_t* toks[] = {&L.P2, &L.P3, &L.P5};
-  for (size_t* m : toks) {
-    *m = off;
-    off = align256(off + tok);
+  L.Bimg = L.zero = L.flags = L.P2 = L.P3 = L.P5 = off;
+  if (tc) {
+    L.Bimg = off;  // per frame [dA + dA^T ; G] bf16, 64 KiB
+    off = align256(off + frames * 65536);
+    L.zero = off;  // an all-zero operand image
+    off = align256(off + (size_t)kImageBytes);
+    L.flags = off;  // publication counters of the overlapped recompute
+    off = align256(off + frames * sizeof(int));
+  } else {
+    size_t* toks[] = {&L.P2, &L.P3, &L.P5};
+    for (size_t* m : toks) {
+      *m = off;
+      off = align256(off + tok);
+    }
   }
   L.total = off;
   return L;
+}
+
+// Tensor-core backward, D = 128, bf16: recompute with the forward kernels
+// (states as bf16 hi/lo pairs), W = dO^T Q by the contraction, G by the
+// adjoint chain, per-frame terms on CUDA cores, token gradients and dq on
+// tensor cores.
+static int scan_bwd_tc(const gdn_bwd_params& p, char* ws, size_t oA, size_t oU, size_t oSfr,
+                       size_t oW, size_t oG, size_t odM, size_t oB, size_t oZero, size_t oFlags,
+                       cudaStream_t st) {
+  const unsigned f = p.flags;
+  const bool reverse = (f & GDN_REVERSE) != 0;
+  const bool block_reset = (f & GDN_BLOCK_RESET) != 0;
+  const int block = block_len(f);
+  const long long frames = (long long)p.B * p.H * p.T;
+  const int heads = p.B * p.H;
+  const double c = (f & GDN_KEYS_SCALED) ? 1.0 : 1.0 / std::sqrt((double)p.D * (double)p.S);
+  float* A = (float*)(ws + oA);
+  float* U = (float*)(ws + oU);
+  float* W = (float*)(ws + oW);
+  float* dM = (float*)(ws + odM);
+  cudaError_t e;
+  // 1. recompute A_t (operand images), U_t and the states S_t (hi/lo pairs)
+  ChainArgs a;
+  memset(&a, 0, sizeof(a));
+  a.mode = CHAIN_SCAN;
+  a.seg = SEG_SEQUENTIAL;
+  a.D = 128;
+  a.T = p.T;
+  a.L = 1;
+  a.block = block;
+  a.seq_reset = block_reset ? 1 : 0;
+  a.reverse = reverse ? 1 : 0;
+  a.nseg = 1;
+  a.heads = heads;
+  a.A = A;
+  a.U = U;
+  a.gamma = p.gamma;
+  a.state_in = p.state_in;
+  a.Sfr = (float*)(ws + oSfr);
+  a.sfr_hilo = 1;
+  a.y_image = 1;
+  {
+    PhaseScope ps(PH_BWD_RECOMPUTE, st);
+    if (heads <= tc_overlap_max_chains()) {
+      OvlArgs o;
+      memset(&o, 0, sizeof(o));
+      o.heads = heads;
+      o.T = p.T;
+      o.block = block;
+      o.ndir = 1;
+      o.gamma = p.gamma;
+      o.A = (const uint8_t*)A;
+      o.flags = (int*)(ws + oFlags);
+      o.dir[0] = OvlDir{a.reverse, 0, a.seq_reset, p.state_in, nullptr};
+      e = tc_contract_scan(p.k, p.v, p.beta, A, U, frames, p.S, (float)(c * c), (float)c, nullptr,
+                           o, a.Sfr, nullptr, st);
+    } else {
+      e = tc_contract(p.k, p.v, p.beta, A, U, frames, p.S, 128, (float)(c * c), (float)c, 1,
+                      nullptr, st);
+      if (e == cudaSuccess) e = tc_chain(a, heads, st);
+    }
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "backward: recompute");
+  // 2. W_t = dO_t^T Q_t: the contraction's U with keys := q, values := dO, beta = 1
+  {
+    PhaseScope ps(PH_BWD_W, st);
+    e = tc_contract(p.q, p.d_out, nullptr, A, W, frames, p.S, 128, 1.f, 1.f, 2, nullptr, st);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "backward: dO^T Q");
+  // 3. adjoint chain: G_t as hi/lo pairs
+  ChainArgs b = a;
+  b.mode = CHAIN_ADJOINT;
+  b.Zw = W;
+  b.Gout = (float*)(ws + oG);
+  b.dS_out = p.d_state_out;
+  b.zero_img = ws + oZero;
+  {
+    PhaseScope ps(PH_BWD_ADJOINT, st);
+    e = cudaMemsetAsync(ws + oZero, 0, kImageBytes, st);
+    if (e == cudaSuccess) e = tc_chain(b, heads, st);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "backward: adjoint chain");
+  // 4. per frame: dM = S'^T G, dA + dA^T and dgamma, the token kernel's operand
+  {
+    PhaseScope ps(PH_BWD_FRAME, st);
+    e = simt_bwd_dm(a.Sfr, p.state_in, b.Gout, dM, frames, p.T, 128, a.reverse, a.seq_reset,
+                    block, true, st);
+    if (e == cudaSuccess)
+      e = simt_bwd_dterm(dM, A, true, p.gamma, p.dgamma, frames, 128, b.Gout, ws + oB, st);
+    if (e == cudaSuccess && p.d_state_in)
+      e = simt_bwd_ds0(b.Gout, A, p.gamma, p.d_state_in, heads, p.T, frame_at(0, p.T, a.reverse),
+                       st);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "backward: per-frame terms");
+  // 5. token gradients and dq
+  {
+    PhaseScope ps(PH_BWD_TOKENS, st);
+    e = tc_bwd_tokens(p.k, p.v, p.beta, ws + oB, p.dk, p.dv, p.dbeta, frames, p.S, (float)c, st);
+    if (e == cudaSuccess) e = tc_readout_trans(p.d_out, a.Sfr, p.dq, frames, p.S, st);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "backward: token gradients");
+  return GDN_OK;
 }
 
 static int scan_bwd(const gdn_bwd_params& p, cudaStream_t st) {
@@ -474,7 +594,7 @@ static int scan_bwd(const gdn_bwd_params& p, cudaStream_t st) {
   for (const void* o : outs)
     for (const void* i : ins)
       if (o == i) return fail(GDN_ERR_INVALID, "gradients must not alias inputs%s");
-  const BwdLayout L = make_bwd_layout(p.B, p.H, p.T, p.S, p.D);
+  const BwdLayout L = make_bwd_layout(p.B, p.H, p.T, p.S, p.D, f);
   if (!p.workspace || p.workspace_bytes < L.total)
     return fail(GDN_ERR_WORKSPACE, "workspace missing or smaller than gdn_bwd_workspace_bytes%s");
   if (((uintptr_t)p.workspace & 255u) != 0)
@@ -497,6 +617,11 @@ static int scan_bwd(const gdn_bwd_params& p, cudaStream_t st) {
   float* P3 = (float*)(ws + L.P3);
   float* P5 = (float*)(ws + L.P5);
   cudaError_t e;
+  if (bwd_tc_by_flags(p.D, f)) {
+    if (device_cc_major() != 10)
+      return fail(GDN_ERR_UNSUPPORTED, "bf16 D = 128 backward runs on sm_100 (else pass GDN_FORCE_SIMT)%s");
+    return scan_bwd_tc(p, ws, L.A, L.U, L.Sfr, L.W, L.G, L.dM, L.Bimg, L.zero, L.flags, st);
+  }
   // 1. forward recompute: A_t, U_t, then the states S_t (one chain per head)
   e = simt_contract(bf16, p.k, p.v, p.beta, A, U, frames, p.S, p.D, (float)(c * c), (float)c, st);
   if (e != cudaSuccess) return cuda_fail(e, "backward: contract");
@@ -530,8 +655,10 @@ static int scan_bwd(const gdn_bwd_params& p, cudaStream_t st) {
   b.dS_in = p.d_state_in;
   if ((e = simt_chain(b, b.heads, st)) != cudaSuccess) return cuda_fail(e, "backward: adjoint chain");
   // 4. per frame: dM = S'^T G -> dA + dA^T, dgamma
-  e = simt_bwd_dm(Sfr, p.state_in, G, dM, frames, p.T, p.D, a.reverse, a.seq_reset, block, st);
-  if (e == cudaSuccess) e = simt_bwd_dterm(dM, A, p.gamma, p.dgamma, frames, p.D, st);
+  e = simt_bwd_dm(Sfr, p.state_in, G, dM, frames, p.T, p.D, a.reverse, a.seq_reset, block, false,
+                  st);
+  if (e == cudaSuccess)
+    e = simt_bwd_dterm(dM, A, false, p.gamma, p.dgamma, frames, p.D, nullptr, nullptr, st);
   if (e != cudaSuccess) return cuda_fail(e, "backward: per-frame terms");
   // 5. per token: K^ (dA + dA^T), V G, K^ G^T, dQ = dO S_t; then dk, dv, dbeta
   e = simt_rowmat(bf16, true, 0, p.k, dM, P2, frames, p.S, p.D, (float)c, st);
@@ -592,7 +719,7 @@ int gdn_frame_scan_bwd(const gdn_bwd_params* p, gdn_stream_t stream) {
 size_t gdn_bwd_workspace_bytes(int B, int H, int T, int S, int D, unsigned flags) {
   (void)flags;
   if (B < 1 || H < 1 || T < 1 || S < 1 || D < 1) return 0;
-  return make_bwd_layout(B, H, T, S, D).total;
+  return make_bwd_layout(B, H, T, S, D, flags).total;
 }
 
 size_t gdn_workspace_bytes(int B, int H, int T, int S, int D, unsigned flags) {

@@ -21,10 +21,29 @@ namespace gdn {
 // j), else the stored state after the previous frame in scan order.
 // One CTA per (frame, TILE x TILE tile of dM), rows r of S' and G streamed.
 // ----------------------------------------------------------------------------
-template <int TILE>
+// Element (r, c) of frame f of a matrix array stored as fp32 [F][D][D] or, with
+// HILO, as bf16 (hi, lo) pairs [F][2][D][D] (value = hi + lo).
+template <bool HILO>
+__device__ __forceinline__ float mat_at(const void* base, size_t f, int D, int r, int c) {
+  if (HILO) {
+    const __nv_bfloat16* b = (const __nv_bfloat16*)base + f * 2 * D * D + (size_t)r * D + c;
+    return __bfloat162float(b[0]) + __bfloat162float(b[(size_t)D * D]);
+  }
+  return ((const float*)base)[f * D * D + (size_t)r * D + c];
+}
+
+// Element (k, n) of the D = 128 operand image of A_t (bf16 hi, lo; 128-byte
+// swizzled MN-major blocks of 64 columns, hi in bytes [0, 32K), lo after).
+__device__ __forceinline__ float img128_at(const uint8_t* img, int k, int n) {
+  const int off = (n >> 6) * 16384 + k * 128 + ((((n & 63) >> 3) ^ (k & 7)) << 4) + (n & 7) * 2;
+  return __bfloat162float(*(const __nv_bfloat16*)(img + off)) +
+         __bfloat162float(*(const __nv_bfloat16*)(img + 32768 + off));
+}
+
+template <int TILE, bool HILO>
 __global__ void __launch_bounds__(256)
-    k_bwd_dm(const float* __restrict__ Sfr, const float* __restrict__ state_in,
-             const float* __restrict__ G, float* __restrict__ dM, int T, int D, int reverse,
+    k_bwd_dm(const void* __restrict__ Sfr, const float* __restrict__ state_in,
+             const void* __restrict__ G, float* __restrict__ dM, int T, int D, int reverse,
              int seq_reset, int block) {
   constexpr int R = TILE / 16;
   constexpr int KC = 32;
@@ -33,15 +52,17 @@ __global__ void __launch_bounds__(256)
   const long long n = blockIdx.x;
   const int bh = (int)(n / T), t = (int)(n % T);
   const int j = reverse ? T - 1 - t : t;
-  const float* Xp = nullptr;
+  // the state entering frame j: state_in (fp32), zeros, or the previous frame's
+  const float* X0 = nullptr;
+  long long fprev = -1;
   if (j == 0) {
-    Xp = state_in ? state_in + (size_t)bh * D * D : nullptr;
+    X0 = state_in ? state_in + (size_t)bh * D * D : nullptr;
   } else {
     const int tp = frame_at(j - 1, T, reverse);
     const bool rst = seq_reset && (t / block) != (tp / block);
-    if (!rst) Xp = Sfr + ((size_t)bh * T + tp) * D * D;
+    if (!rst) fprev = (long long)bh * T + tp;
   }
-  const float* Gn = G + (size_t)n * D * D;
+  const bool have_x = X0 || fprev >= 0;
   const int nt = D / TILE;
   const int ti = blockIdx.y / nt, tj = blockIdx.y % nt;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
@@ -50,11 +71,16 @@ __global__ void __launch_bounds__(256)
   for (int a = 0; a < R; ++a)
 #pragma unroll
     for (int b = 0; b < R; ++b) acc[a][b] = 0.f;
-  for (int r0 = 0; Xp && r0 < D; r0 += KC) {
+  for (int r0 = 0; have_x && r0 < D; r0 += KC) {
     for (int e = threadIdx.x; e < KC * TILE; e += 256) {
       const int r = e / TILE, c = e % TILE, rr = r0 + r;
-      Xs[r][c] = rr < D ? Xp[(size_t)rr * D + ti * TILE + c] : 0.f;
-      Gs[r][c] = rr < D ? Gn[(size_t)rr * D + tj * TILE + c] : 0.f;
+      float xv = 0.f, gv = 0.f;
+      if (rr < D) {
+        xv = X0 ? X0[(size_t)rr * D + ti * TILE + c] : mat_at<HILO>(Sfr, fprev, D, rr, ti * TILE + c);
+        gv = mat_at<HILO>(G, n, D, rr, tj * TILE + c);
+      }
+      Xs[r][c] = xv;
+      Gs[r][c] = gv;
     }
     __syncthreads();
 #pragma unroll 4
@@ -81,12 +107,28 @@ __global__ void __launch_bounds__(256)
 }
 
 // Per frame, in place: dM -> dA + dA^T = -g (dM + dM^T); dgamma = <dM, I - A>.
+// A_t is fp32, or (AIMG, D = 128) its operand image. With `bimg` (D = 128),
+// also writes the per-frame B operand of the tensor-core token kernel: bf16
+// rows n of [dA + dA^T ; G] (n < 128: dA + dA^T, n >= 128: G row n - 128) by
+// 128 columns, K-major, in two 64-column 128-byte-swizzled blocks of 256 rows
+// (32 KiB each); G is read from its (hi, lo) pairs and rounded once.
+__device__ __forceinline__ int bimg_off(int r, int c) {
+  return (c >> 6) * 32768 + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + (c & 7) * 2;
+}
+
+template <bool AIMG>
 __global__ void __launch_bounds__(256)
-    k_bwd_dterm(float* __restrict__ dM, const float* __restrict__ A,
-                const float* __restrict__ gamma, float* __restrict__ dgamma, int D) {
+    k_bwd_dterm(float* __restrict__ dM, const void* __restrict__ A,
+                const float* __restrict__ gamma, float* __restrict__ dgamma, int D,
+                const __nv_bfloat16* __restrict__ Ghilo, uint8_t* __restrict__ bimg) {
   const long long n = blockIdx.x;
   float* m = dM + (size_t)n * D * D;
-  const float* a = A + (size_t)n * D * D;
+  const float* a = AIMG ? nullptr : (const float*)A + (size_t)n * D * D;
+  const uint8_t* aimg = AIMG ? (const uint8_t*)A + (size_t)n * D * D * 4 : nullptr;
+  uint8_t* bo = bimg ? bimg + (size_t)n * 65536 : nullptr;
+  auto a_at = [&](int i, int j) -> float {
+    return AIMG ? img128_at(aimg, i, j) : a[(size_t)i * D + j];
+  };
   const float g = gamma[n];
   float part = 0.f;
   const int npair = D * (D + 1) / 2;
@@ -100,13 +142,27 @@ __global__ void __launch_bounds__(256)
     const int j = i + rem;
     const float mij = m[(size_t)i * D + j], mji = m[(size_t)j * D + i];
     if (i == j) {
-      part += mij * (1.f - a[(size_t)i * D + i]);
-      m[(size_t)i * D + i] = -2.f * g * mij;
+      part += mij * (1.f - a_at(i, i));
+      const float s = -2.f * g * mij;
+      m[(size_t)i * D + i] = s;
+      if (bo) *(__nv_bfloat16*)(bo + bimg_off(i, i)) = __float2bfloat16_rn(s);
     } else {
-      part -= (mij + mji) * a[(size_t)i * D + j];  // A symmetric
+      part -= (mij + mji) * a_at(i, j);  // A symmetric
       const float s = -g * (mij + mji);
       m[(size_t)i * D + j] = s;
       m[(size_t)j * D + i] = s;
+      if (bo) {
+        *(__nv_bfloat16*)(bo + bimg_off(i, j)) = __float2bfloat16_rn(s);
+        *(__nv_bfloat16*)(bo + bimg_off(j, i)) = __float2bfloat16_rn(s);
+      }
+    }
+  }
+  if (bo) {
+    const __nv_bfloat16* gh = Ghilo + (size_t)n * 2 * D * D;
+    for (int e = threadIdx.x; e < D * D; e += blockDim.x) {
+      const int r = e / D, c = e % D;
+      const float gv = __bfloat162float(gh[e]) + __bfloat162float(gh[(size_t)D * D + e]);
+      *(__nv_bfloat16*)(bo + bimg_off(128 + r, c)) = __float2bfloat16_rn(gv);
     }
   }
   __shared__ float red[32];
@@ -226,28 +282,86 @@ __global__ void __launch_bounds__(256)
   if (lane == 0) dbeta[tok] = part;
 }
 
-cudaError_t simt_bwd_dm(const float* Sfr, const float* state_in, const float* G, float* dM,
-                        long long N, int T, int D, int reverse, int seq_reset, int block,
-                        cudaStream_t st) {
+template <bool HILO>
+static cudaError_t bwd_dm_t(const void* Sfr, const float* state_in, const void* G, float* dM,
+                            long long N, int T, int D, int reverse, int seq_reset, int block,
+                            cudaStream_t st) {
   const int tile = D < 64 ? D : 64;
   dim3 grid((unsigned)N, (D / tile) * (D / tile));
   switch (tile) {
     case 16:
-      k_bwd_dm<16><<<grid, 256, 0, st>>>(Sfr, state_in, G, dM, T, D, reverse, seq_reset, block);
+      k_bwd_dm<16, HILO><<<grid, 256, 0, st>>>(Sfr, state_in, G, dM, T, D, reverse, seq_reset, block);
       break;
     case 32:
-      k_bwd_dm<32><<<grid, 256, 0, st>>>(Sfr, state_in, G, dM, T, D, reverse, seq_reset, block);
+      k_bwd_dm<32, HILO><<<grid, 256, 0, st>>>(Sfr, state_in, G, dM, T, D, reverse, seq_reset, block);
       break;
     default:
-      k_bwd_dm<64><<<grid, 256, 0, st>>>(Sfr, state_in, G, dM, T, D, reverse, seq_reset, block);
+      k_bwd_dm<64, HILO><<<grid, 256, 0, st>>>(Sfr, state_in, G, dM, T, D, reverse, seq_reset, block);
   }
   count_launch();
   return cudaGetLastError();
 }
 
-cudaError_t simt_bwd_dterm(float* dM, const float* A, const float* gamma, float* dgamma,
-                           long long N, int D, cudaStream_t st) {
-  k_bwd_dterm<<<(unsigned)N, 256, 0, st>>>(dM, A, gamma, dgamma, D);
+cudaError_t simt_bwd_dm(const void* Sfr, const float* state_in, const void* G, float* dM,
+                        long long N, int T, int D, int reverse, int seq_reset, int block,
+                        bool hilo, cudaStream_t st) {
+  return hilo ? bwd_dm_t<true>(Sfr, state_in, G, dM, N, T, D, reverse, seq_reset, block, st)
+              : bwd_dm_t<false>(Sfr, state_in, G, dM, N, T, D, reverse, seq_reset, block, st);
+}
+
+cudaError_t simt_bwd_dterm(float* dM, const void* A, bool a_image, const float* gamma,
+                           float* dgamma, long long N, int D, const void* G_hilo, void* bimg,
+                           cudaStream_t st) {
+  if (a_image)
+    k_bwd_dterm<true><<<(unsigned)N, 256, 0, st>>>(dM, A, gamma, dgamma, D,
+                                                   (const __nv_bfloat16*)G_hilo, (uint8_t*)bimg);
+  else
+    k_bwd_dterm<false><<<(unsigned)N, 256, 0, st>>>(dM, A, gamma, dgamma, D,
+                                                    (const __nv_bfloat16*)G_hilo, (uint8_t*)bimg);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// dL/d(state_in) = g_0 (G_0 - G_0 A_0) for the first frame t0 of the scan of
+// each head, from G_0 as (hi, lo) pairs and A_0 as its D = 128 operand image.
+// CTA = (head, 16 rows); thread (r, l): row r, columns l + 16 m.
+__global__ void __launch_bounds__(256)
+    k_bwd_ds0(const __nv_bfloat16* __restrict__ Ghilo, const uint8_t* __restrict__ Aimg,
+              const float* __restrict__ gamma, float* __restrict__ ds0, int T, int t0) {
+  constexpr int D = 128;
+  __shared__ float Xs[16][D];
+  __shared__ float Ys[16][D];
+  const int bh = blockIdx.x, row0 = blockIdx.y * 16;
+  const size_t f = (size_t)bh * T + t0;
+  const int r = threadIdx.x >> 4, l = threadIdx.x & 15;
+  for (int c = l; c < D; c += 16) Xs[r][c] = mat_at<true>(Ghilo, f, D, row0 + r, c);
+  float acc[D / 16];
+#pragma unroll
+  for (int m = 0; m < D / 16; ++m) acc[m] = 0.f;
+  const uint8_t* img = Aimg + f * D * D * 4;
+  for (int k0 = 0; k0 < D; k0 += 16) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < 16 * D; e += 256) Ys[e / D][e % D] = img128_at(img, k0 + e / D, e % D);
+    __syncthreads();
+#pragma unroll 4
+    for (int kk = 0; kk < 16; ++kk) {
+      const float x = Xs[r][k0 + kk];
+#pragma unroll
+      for (int m = 0; m < D / 16; ++m) acc[m] = fmaf(x, Ys[kk][l + 16 * m], acc[m]);
+    }
+  }
+  const float g = gamma[f];
+#pragma unroll
+  for (int m = 0; m < D / 16; ++m) {
+    const int c = l + 16 * m;
+    ds0[(size_t)bh * D * D + (size_t)(row0 + r) * D + c] = g * (Xs[r][c] - acc[m]);
+  }
+}
+
+cudaError_t simt_bwd_ds0(const void* G_hilo, const void* A_img, const float* gamma, float* ds0,
+                         int heads, int T, int t0, cudaStream_t st) {
+  k_bwd_ds0<<<dim3((unsigned)heads, 128 / 16), 256, 0, st>>>((const __nv_bfloat16*)G_hilo,
+                                                            (const uint8_t*)A_img, gamma, ds0, T, t0);
   count_launch();
   return cudaGetLastError();
 }

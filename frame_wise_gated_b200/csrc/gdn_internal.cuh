@@ -73,6 +73,7 @@ struct ChainArgs {
   float* Gout;            // [heads*T, D, D] total state gradients G_t
   const float* dS_out;    // [heads, D, D] gradient of state_out, or null
   float* dS_in;           // [heads, D, D] gradient of state_in, or null
+  const void* zero_img;   // an all-zero operand image (tensor-core adjoint chain)
 };
 
 // An "operand image" of a D x D fp32 matrix M (D = 128) is the exact
@@ -135,12 +136,20 @@ cudaError_t simt_readout(bool bf16, const void* q, const float* Sfr, void* out, 
 
 // ---- backward (CUDA cores) ------------------------------------------------------
 // dM_j = S'_j^T G_j per frame (S'_j: state entering frame j of the scan order).
-cudaError_t simt_bwd_dm(const float* Sfr, const float* state_in, const float* G, float* dM,
+// hilo: Sfr and G hold bf16 (hi, lo) pairs [F][2][D][D] instead of fp32.
+cudaError_t simt_bwd_dm(const void* Sfr, const float* state_in, const void* G, float* dM,
                         long long N, int T, int D, int reverse, int seq_reset, int block,
-                        cudaStream_t st);
-// In place dM -> dA + dA^T = -gamma (dM + dM^T); dgamma = <dM, I - A>.
-cudaError_t simt_bwd_dterm(float* dM, const float* A, const float* gamma, float* dgamma,
-                           long long N, int D, cudaStream_t st);
+                        bool hilo, cudaStream_t st);
+// In place dM -> dA + dA^T = -gamma (dM + dM^T); dgamma = <dM, I - A>. A is
+// fp32 or (a_image, D = 128) operand images; with bimg (D = 128, G_hilo set)
+// also writes the tensor-core token kernel's per-frame B operand (64 KiB).
+cudaError_t simt_bwd_dterm(float* dM, const void* A, bool a_image, const float* gamma,
+                           float* dgamma, long long N, int D, const void* G_hilo, void* bimg,
+                           cudaStream_t st);
+// dL/d(state_in) = g (G - G A) at the first frame t0 of each head (D = 128,
+// G as (hi, lo) pairs, A as operand images).
+cudaError_t simt_bwd_ds0(const void* G_hilo, const void* A_img, const float* gamma, float* ds0,
+                         int heads, int T, int t0, cudaStream_t st);
 // Per frame n: out[s, :] = scale * x[s, :] M_n^T (trans = 0) or x[s, :] M_n (trans = 1).
 cudaError_t simt_rowmat(bool bf16_in, bool f32_out, int trans, const void* x, const float* M,
                         void* out, long long N, int S, int D, float scale, cudaStream_t st);
@@ -211,6 +220,13 @@ int tc_overlap_max_chains();
 cudaError_t tc_contract_scan(const void* k, const void* v, const float* beta, float* A, float* U,
                              long long N, int S, float cA, float cU, const ProArgs* pro,
                              const OvlArgs& o, void* sfr0, void* sfr1, cudaStream_t st);
+// Backward, D = 128: dq = dO S_t (S_t as hi/lo pairs) and the token gradients
+// dk, dv, dbeta from the per-frame B operand [dA + dA^T ; G] (64 KiB bf16).
+cudaError_t tc_readout_trans(const void* x, const void* Sfr_hilo, void* out, long long N, int S,
+                             cudaStream_t st);
+cudaError_t tc_bwd_tokens(const void* k, const void* v, const float* beta, const void* bimg,
+                          void* dk, void* dv, float* dbeta, long long N, int S, float c,
+                          cudaStream_t st);
 bool tc_chain_supported(int D);
 cudaError_t tc_chain(const ChainArgs& a, int nchains, cudaStream_t st);
 cudaError_t tc_selftest_wait(int arrive, long long limit_ns, cudaStream_t st);

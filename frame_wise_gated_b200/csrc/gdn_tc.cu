@@ -289,13 +289,17 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
         // beta of the stage's tokens: asynchronous 4-byte copies (zeros past S)
         // that arrive on the same barrier, so the loop never waits on them.
         const uint32_t bsa = sb + OFF_BETA + s * TOK * 4;
+        if (beta) {
 #pragma unroll
-        for (int r = lane; r < TOK; r += 32) {
-          const int tok = st * TOK + r;
-          const bool in = tok < S;
-          cp_async_4(bsa + r * 4, beta + (size_t)n * S + (in ? tok : 0), in ? 4u : 0u);
+          for (int r = lane; r < TOK; r += 32) {
+            const int tok = st * TOK + r;
+            const bool in = tok < S;
+            cp_async_4(bsa + r * 4, beta + (size_t)n * S + (in ? tok : 0), in ? 4u : 0u);
+          }
+          cp_async_arrive_noinc(bar_full + 8 * s);
+        } else {
+          mbar_arrive(bar_full + 8 * s);  // beta = 1: nothing to copy
         }
-        cp_async_arrive_noinc(bar_full + 8 * s);
       }
     }
     // Drain: every TMA this CTA issued has landed before teardown.
@@ -370,7 +374,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
           const int tok = st * TOK + pr;
           float f[32];
           pro_row_part<4>(kt, BOX, pr, pc0, D, tok, tok < S, pro, wreg, tab, f);
-          const float bv = bs[pr];
+          const float bv = beta ? bs[pr] : 1.f;
           uint8_t* rowp = bt + (pc0 >> 6) * BOX + pr * 128;
           const int ch0 = (pc0 & 63) >> 3;
 #pragma unroll
@@ -385,7 +389,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
 #pragma unroll
         for (int m = 0; m < 1024 / NSC; ++m) {
           const int c = t + NSC * m;          // 16-byte chunk of the 16 KiB tile
-          const float bv = bs[(c >> 3) & (TOK - 1)];  // 8 chunks per 128-byte token row
+          const float bv = beta ? bs[(c >> 3) & (TOK - 1)] : 1.f;  // 8 chunks per 128-byte token row
           uint4 x = *(const uint4*)(kt + c * 16);
           uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
@@ -415,7 +419,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
       tc_fence_after();
       const int n = unit_n(i);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      for (int half = a_image == 2 ? 1 : 0; half < 2; ++half) {  // 2: only U is wanted
         float* dst = (half ? U : A) + ((size_t)n * D + row) * D;
         uint8_t* img = (uint8_t*)A + (size_t)n * kImageBytes;
         const float sc = half ? cU : cA;
@@ -551,7 +555,9 @@ constexpr int threads(bool pro) { return pro ? 448 : 192; }
 constexpr uint32_t TMEM_COLS = 256;
 }  // namespace rdo
 
-template <bool PRO>
+// TRANS: O = Q S_t (S_t as an MN-major operand) instead of Q S_t^T; the
+// backward's dQ = dO S_t.
+template <bool PRO, bool TRANS = false>
 __global__ void __launch_bounds__(rdo::threads(PRO), 1)
     k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
                  const __grid_constant__ CUtensorMap tmO, int N, int S, ProArgs pro, int parts) {
@@ -641,7 +647,7 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, TRANS);
       int g = 0;
       bool ok = true;
       for (int i = 0; i < my_count && ok; ++i) {
@@ -669,8 +675,11 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
             // K-major: 16 channels = 32 bytes inside a 128-byte swizzled row
             const uint32_t off = (kk >> 2) * BOX + (kk & 3) * 32;
             const uint64_t dq = smem_desc_sw128(qa + off, 16, 1024);
-            const uint64_t dh = smem_desc_sw128(sh + off, 16, 1024);
-            const uint64_t dl = smem_desc_sw128(sl + off, 16, 1024);
+            // S_t^T: K-major rows of S_t; S_t: 16 rows of k, two 64-column blocks
+            const uint64_t dh = TRANS ? smem_desc_sw128(sh + kk * 2048, BOX, 1024)
+                                      : smem_desc_sw128(sh + off, 16, 1024);
+            const uint64_t dl = TRANS ? smem_desc_sw128(sl + kk * 2048, BOX, 1024)
+                                      : smem_desc_sw128(sl + off, 16, 1024);
             mma_bf16(d, dq, dh, idesc, kk > 0 ? 1u : 0u);
             mma_bf16(d, dq, dl, idesc, 1u);
           }
@@ -784,12 +793,12 @@ static int readout_parts(long long N, int ntile) {
   return (ntile >= 8 && N < 4LL * num_sms()) ? 2 : 1;
 }
 
-template <bool PRO>
+template <bool PRO, bool TRANS = false>
 static cudaError_t launch_readout(const CUtensorMap& mq, const CUtensorMap& ms, const CUtensorMap& mo,
                                   long long N, int S, const ProArgs& pa, cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_readout_tc<PRO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(k_readout_tc<PRO, TRANS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          rdo::SMEM);
     if (e != cudaSuccess) return e;
     attr = true;
@@ -797,7 +806,8 @@ static cudaError_t launch_readout(const CUtensorMap& mq, const CUtensorMap& ms, 
   const int parts = readout_parts(N, (S + rdo::TOK - 1) / rdo::TOK);
   const long long units = N * parts;
   const int grid = (int)(units < num_sms() ? units : num_sms());
-  k_readout_tc<PRO><<<grid, rdo::threads(PRO), rdo::SMEM, st>>>(mq, ms, mo, (int)N, S, pa, parts);
+  k_readout_tc<PRO, TRANS><<<grid, rdo::threads(PRO), rdo::SMEM, st>>>(mq, ms, mo, (int)N, S, pa,
+                                                                      parts);
   count_launch();
   return cudaGetLastError();
 }
@@ -819,6 +829,18 @@ static cudaError_t tc_readout128(const void* q, const void* Sfr_hilo, void* out,
     return launch_readout<true>(mq, ms, mo, N, S, pa, st);
   }
   return launch_readout<false>(mq, ms, mo, N, S, pa, st);
+}
+
+// dQ_t = dO_t S_t for every frame-head (D = 128, bf16; S_t as bf16 hi/lo pairs).
+cudaError_t tc_readout_trans(const void* x, const void* Sfr_hilo, void* out, long long N, int S,
+                             cudaStream_t st) {
+  CUtensorMap mq, ms, mo;
+  cudaError_t e = make_map_bf16_3d(&mq, x, 128, S, N, 64, rdo::TOK);
+  if (e == cudaSuccess) e = make_map_bf16_3d(&ms, Sfr_hilo, 128, 128, 2 * N, 64, 128);
+  if (e == cudaSuccess) e = make_map_bf16_3d(&mo, out, 128, S, N, 64, rdo::TOK);
+  if (e != cudaSuccess) return e;
+  ProArgs pa = {};
+  return launch_readout<false, true>(mq, ms, mo, N, S, pa, st);
 }
 
 // ============================================================================
@@ -894,6 +916,14 @@ __device__ __forceinline__ ChainProg chain_prog(const ChainArgs& a, int c) {
     seg_range(a, g.p, &j0, &j1);
     g.j0 = j0;
     g.n = j1 - j0;
+  } else if (a.mode == CHAIN_ADJOINT) {
+    // backward: one chain per head over the scan positions T-1 .. 0, starting
+    // from the gradient of state_out
+    g.bh = c;
+    g.p = 0;
+    g.j0 = 0;
+    g.n = a.T;
+    g.init = a.dS_out ? a.dS_out + (size_t)g.bh * a.D * a.D : nullptr;
   } else {
     g.bh = c;
     g.p = 0;
@@ -914,6 +944,26 @@ __device__ __forceinline__ ChainStep chain_step_at(const ChainArgs& a, const Cha
     st.alpha = a.g[si];
     st.reset = 0;
     st.t = s;
+    return st;
+  }
+  if (g.mode == CHAIN_ADJOINT) {
+    // G_j = W_j + g_{j+1} (G_{j+1} - G_{j+1} A_{j+1}), cut where the forward
+    // scan reset before j+1; the first step (j = T-1) only adds W.
+    const int j = a.T - 1 - s;
+    const int t = frame_at(j, a.T, a.reverse);
+    st.t = t;
+    st.Z = a.Zw + ((size_t)g.bh * a.T + t) * DD;
+    st.reset = 0;
+    if (s == 0) {
+      st.Y = a.zero_img;
+      st.alpha = 1.0f;
+    } else {
+      const int tn = frame_at(j + 1, a.T, a.reverse);
+      const size_t fn = (size_t)g.bh * a.T + tn;
+      st.Y = a.A + fn * DD;
+      st.alpha = a.gamma[fn];
+      st.reset = a.seq_reset && (t / a.block) != (tn / a.block);
+    }
     return st;
   }
   const int j = g.j0 + s;
@@ -1050,7 +1100,7 @@ __global__ void __launch_bounds__(chn::THREADS, 1)
   // Z comes from global memory (TMA) except for the span composite E, whose
   // Z is its own Y (read back from the Y image).
   const bool z_global = !(g.mode == CHAIN_COMPOSE && g.which == 0);
-  const bool store_sfr = g.mode == CHAIN_SCAN;
+  const bool store_sfr = g.mode == CHAIN_SCAN || g.mode == CHAIN_ADJOINT;  // S_t, or G_t
 
   if (leader) {
     mbar_init(bar_mma, 1);
@@ -1192,6 +1242,7 @@ __global__ void __launch_bounds__(chn::THREADS, 1)
       }
     }
     if (g.mode == CHAIN_COMPOSE) gprod *= a.gamma[(size_t)g.bh * a.T + st.t];
+    if (g.mode == CHAIN_ADJOINT) tprev = st.t;
     if (g.mode == CHAIN_SCAN) {
       tprev = st.t;
       if (g.j0 + s == a.T - 1 && a.state_out)
@@ -1595,6 +1646,8 @@ static cudaError_t tc_chain128(const ChainArgs& a, int nchains, cudaStream_t st)
   cudaError_t e;
   if (a.mode == CHAIN_PREFIX)
     e = make_map_f32_mats(&mz, a.Hc, (uint64_t)a.heads * a.nseg);
+  else if (a.mode == CHAIN_ADJOINT)
+    e = make_map_f32_mats(&mz, a.Zw, (uint64_t)frames);
   else
     e = make_map_f32_mats(&mz, a.U, (uint64_t)frames);
   if (e != cudaSuccess) return e;
@@ -1602,8 +1655,11 @@ static cudaError_t tc_chain128(const ChainArgs& a, int nchains, cudaStream_t st)
   if (a.mode == CHAIN_PREFIX && a.sst_hilo)
     e = make_map_bf16_3d(&ms, a.Sst, 128, 128, 2 * (uint64_t)a.heads * a.nseg, 64, 128);
   else
-    e = make_map_bf16_3d(&ms, a.mode == CHAIN_SCAN ? (const void*)a.Sfr : (const void*)a.U, 128,
-                         128, 2 * frames, 64, 128);
+    e = make_map_bf16_3d(&ms,
+                         a.mode == CHAIN_SCAN      ? (const void*)a.Sfr
+                         : a.mode == CHAIN_ADJOINT ? (const void*)a.Gout
+                                                   : (const void*)a.U,
+                         128, 128, 2 * frames, 64, 128);
   if (e != cudaSuccess) return e;
   k_chain_tc<<<nchains, chn::THREADS, chn::SMEM, st>>>(a, mz, ms);
   count_launch();
@@ -3673,6 +3729,293 @@ static cudaError_t tc_chain256(const ChainArgs& a, int nchains, cudaStream_t st)
   cudaError_t e = make_map_bf16_3d(&ms, a.Sfr, 256, 256, 2 * (uint64_t)frames, 64, 128);
   if (e != cudaSuccess) return e;
   k_chain256_tc<<<2 * nchains, ch2::THREADS, ch2::SMEM, st>>>(a, ms);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ============================================================================
+// Backward token gradients on tensor cores (D = 128, bf16).
+//
+// Per frame-head, per 128-token tile of K and V (TMA, 128-byte swizzle):
+//   [P2 | P5] = K [dAs | G^T]   (M = 128 tokens, N = 256, K = 128 channels)
+//   P3        = V G             (N = 128; G read as an MN-major operand)
+// with dAs = dA + dA^T and G = dL/dS_t in one per-frame bf16 operand (64 KiB,
+// written by the per-frame kernel) kept in shared memory for the frame. With
+// k^ = c k (c = 1/sqrt(D S)), per token s:
+//   dk_s = c beta_s (c P2_s + P3_s),  dv_s = c beta_s P5_s,
+//   dbeta_s = k^_s . (c P2_s / 2 + P3_s).
+// Eight epilogue warps (two per TMEM lane quadrant, one per 64-channel half)
+// stage dk and dv as bf16 in the tile's own V and K buffers and one thread
+// stores them by TMA; dbeta halves meet in shared memory.
+// ============================================================================
+namespace btk {
+constexpr int D = 128;
+constexpr int TOK = 128;
+constexpr int BOX = TOK * 128;                   // [128 tokens][64 channels] bf16: 16 KiB
+constexpr int KT = 2 * BOX;                      // one tensor's tile: 32 KiB
+constexpr int NST = 2;                           // K/V stages (also the dk/dv staging)
+constexpr int BIMG = 65536;                      // per-frame B operand
+constexpr int OFF_B = 0;
+constexpr int OFF_KV = OFF_B + BIMG;             // stage s: K at OFF_KV + 2 s KT, V at + KT
+constexpr int OFF_BETA = OFF_KV + NST * 2 * KT;  // [NST][TOK] fp32
+constexpr int OFF_RED = OFF_BETA + NST * TOK * 4;  // [2][TOK][2] fp32 dbeta halves
+constexpr int OFF_BAR = OFF_RED + 2 * TOK * 2 * 4;
+constexpr int NBAR = 2 * NST + 5;  // full, empty per stage; b_full, b_empty, acc_full, acc_empty, fin
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+static_assert(SMEM <= 232448, "backward token kernel shared memory");
+constexpr int EPI = 256;
+constexpr int THREADS = 64 + EPI;
+constexpr uint32_t TMEM_COLS = 512;  // [P2 | P5]: columns 0..255, P3: 256..383
+}  // namespace btk
+
+__global__ void __launch_bounds__(btk::THREADS, 1)
+    k_bwd_tok_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
+                 const float* __restrict__ beta, const uint8_t* __restrict__ bimg,
+                 float* __restrict__ dbeta, int N, int S, float c) {
+  using namespace btk;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar_full = sb + OFF_BAR;
+  const uint32_t bar_empty = bar_full + 8 * NST;
+  const uint32_t bar_bf = bar_empty + 8 * NST;
+  const uint32_t bar_be = bar_bf + 8;
+  const uint32_t bar_accf = bar_be + 8;
+  const uint32_t bar_acce = bar_accf + 8;
+  const uint32_t bar_fin = bar_acce + 8;
+  uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bar_full + 8 * s, 33);  // expect_tx arrival + 32 lanes' beta copies
+      mbar_init(bar_empty + 8 * s, 1);  // the tile's dk/dv store has read its staging
+    }
+    mbar_init(bar_bf, 1);
+    mbar_init(bar_be, 1);
+    mbar_init(bar_accf, 1);
+    mbar_init(bar_acce, EPI);
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int ntile = (S + TOK - 1) / TOK;
+  const int my_count = (int)blockIdx.x < N ? (N - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+  if (warp == 0) {
+    // ---- producer: the frame's B operand, K and V tiles (TMA), beta ----
+    int g = 0, nb = 0;
+    bool ok = true;
+    for (int i = 0; i < my_count && ok; ++i) {
+      const int n = blockIdx.x + i * gridDim.x;
+      if (lane == 0) {
+        ok = mbar_wait(bar_be, ((uint32_t)i & 1) ^ 1, abort_flag, &g_tc_status, 61);
+        if (ok) {
+          mbar_arrive_expect_tx(bar_bf, BIMG);
+          bulk_load(sb + OFF_B, bimg + (size_t)n * BIMG, BIMG, bar_bf);
+          ++nb;
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      for (int tl = 0; tl < ntile && ok; ++tl, ++g) {
+        const int s = g % NST;
+        const uint32_t u = (uint32_t)(g / NST);
+        if (lane == 0) ok = mbar_wait(bar_empty + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 62);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        const uint32_t kd = sb + OFF_KV + s * 2 * KT, vd = kd + KT;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar_full + 8 * s, 2 * KT);
+          tma_load_3d(kd, &tmK, bar_full + 8 * s, 0, tl * TOK, n);
+          tma_load_3d(kd + BOX, &tmK, bar_full + 8 * s, 64, tl * TOK, n);
+          tma_load_3d(vd, &tmV, bar_full + 8 * s, 0, tl * TOK, n);
+          tma_load_3d(vd + BOX, &tmV, bar_full + 8 * s, 64, tl * TOK, n);
+        }
+        const uint32_t bsa = sb + OFF_BETA + s * TOK * 4;
+#pragma unroll
+        for (int r = lane; r < TOK; r += 32) {
+          const int tok = tl * TOK + r;
+          const bool in = tok < S;
+          cp_async_4(bsa + r * 4, beta + (size_t)n * S + (in ? tok : 0), in ? 4u : 0u);
+        }
+        cp_async_arrive_noinc(bar_full + 8 * s);
+      }
+    }
+    // drain (bounded, not cut short by an abort): copies in flight land
+    if (lane == 0) {
+      volatile int keep_waiting = 0;
+      for (int gg = (g > NST ? g - NST : 0); gg < g; ++gg)
+        mbar_wait(bar_full + 8 * (gg % NST), (uint32_t)(gg / NST) & 1, &keep_waiting, &g_tc_status, 63);
+      if (nb > 0) mbar_wait(bar_bf, (uint32_t)(nb - 1) & 1, &keep_waiting, &g_tc_status, 64);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---- MMA issuer ----
+    if (lane == 0) {
+      constexpr uint32_t idesc_k = idesc_bf16_f32(128, 256, false, false);
+      constexpr uint32_t idesc_g = idesc_bf16_f32(128, 128, false, true);
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; i < my_count && ok; ++i) {
+        ok = mbar_wait(bar_bf, (uint32_t)i & 1, abort_flag, &g_tc_status, 65);
+        if (!ok) break;
+        tc_fence_after();
+        for (int tl = 0; tl < ntile; ++tl, ++g) {
+          const int s = g % NST;
+          ok = mbar_wait(bar_full + 8 * s, (uint32_t)(g / NST) & 1, abort_flag, &g_tc_status, 66);
+          if (ok) ok = mbar_wait(bar_acce, ((uint32_t)g & 1) ^ 1, abort_flag, &g_tc_status, 67);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t ka = sb + OFF_KV + s * 2 * KT, va = ka + KT;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * BOX + (kk & 3) * 32;
+            const uint64_t dk = smem_desc_sw128(ka + off, 16, 1024);
+            const uint64_t dv = smem_desc_sw128(va + off, 16, 1024);
+            // [dAs ; G] rows, K-major: 256 rows per 64-channel block of 32 KiB
+            const uint64_t db = smem_desc_sw128(sb + OFF_B + (kk >> 2) * 32768 + (kk & 3) * 32, 16, 1024);
+            // G as MN-major: 16 rows of k, column blocks 32 KiB apart
+            const uint64_t dg = smem_desc_sw128(sb + OFF_B + 16384 + kk * 2048, 32768, 1024);
+            mma_bf16(tmem, dk, db, idesc_k, kk > 0 ? 1u : 0u);
+            mma_bf16(tmem + 256, dv, dg, idesc_g, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar_accf);
+        }
+        if (!ok) break;
+        mma_commit(bar_be);  // the frame's B operand is free once these MMAs are done
+      }
+      mma_commit(bar_fin);
+      volatile int keep_waiting = 0;
+      mbar_wait(bar_fin, 0, &keep_waiting, &g_tc_status, 68);
+    }
+    __syncwarp();
+  } else {
+    // ---- epilogue: 8 warps; quadrant q = token rows 32q.., half h = channels 64h.. ----
+    const int et = threadIdx.x - 64;
+    const int q = warp & 3, h = et >> 7;
+    const int row = q * 32 + lane;
+    const uint32_t tl_addr = tmem + ((uint32_t)(q * 32) << 16);
+    int g = 0;
+    for (int i = 0; i < my_count; ++i) {
+      const int n = blockIdx.x + i * gridDim.x;
+      bool stop = false;
+      for (int tl = 0; tl < ntile; ++tl, ++g) {
+        const int s = g % NST;
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(bar_accf, (uint32_t)g & 1, abort_flag, &g_tc_status, 69);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (named_bar_or(1, EPI, !ok || *abort_flag)) {
+          stop = true;
+          break;
+        }
+        tc_fence_after();
+        uint8_t* kt = smem + OFF_KV + s * 2 * KT;
+        uint8_t* vt = kt + KT;
+        const float bv = ((const float*)(smem + OFF_BETA))[s * TOK + row];
+        // this thread's 64 key channels (bf16 pairs), read before the K buffer
+        // becomes the dv staging
+        uint32_t kw[32];
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 x = *(const uint4*)(kt + h * BOX + row * 128 + ((ch ^ (row & 7)) << 4));
+          kw[4 * ch] = x.x; kw[4 * ch + 1] = x.y; kw[4 * ch + 2] = x.z; kw[4 * ch + 3] = x.w;
+        }
+        named_bar_sync(1, EPI);
+        float dbp = 0.f;
+#pragma unroll
+        for (int c32 = 0; c32 < 2; ++c32) {
+          uint32_t p2[32], p5[32], p3[32];
+          const uint32_t col = 64 * h + 32 * c32;
+          tmem_ld32(tl_addr + col, p2);
+          tmem_ld32(tl_addr + 128 + col, p5);
+          tmem_ld32(tl_addr + 256 + col, p3);
+          tmem_wait_ld();
+          float dkv[32], dvv[32];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kw[(32 * c32 + j) >> 1]));
+            const float a2 = c * __uint_as_float(p2[j]), b2 = c * __uint_as_float(p2[j + 1]);
+            const float a3 = __uint_as_float(p3[j]), b3 = __uint_as_float(p3[j + 1]);
+            dkv[j] = c * bv * (a2 + a3);
+            dkv[j + 1] = c * bv * (b2 + b3);
+            dvv[j] = c * bv * __uint_as_float(p5[j]);
+            dvv[j + 1] = c * bv * __uint_as_float(p5[j + 1]);
+            dbp = fmaf(c * kf.x, 0.5f * a2 + a3, dbp);
+            dbp = fmaf(c * kf.y, 0.5f * b2 + b3, dbp);
+          }
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int ch = 4 * c32 + m;  // 16-byte chunk of the 128-byte row of box h
+            const int off = h * BOX + row * 128 + ((ch ^ (row & 7)) << 4);
+            *(uint4*)(vt + off) = make_uint4(pack_bf16x2(dkv[8 * m], dkv[8 * m + 1]),
+                                             pack_bf16x2(dkv[8 * m + 2], dkv[8 * m + 3]),
+                                             pack_bf16x2(dkv[8 * m + 4], dkv[8 * m + 5]),
+                                             pack_bf16x2(dkv[8 * m + 6], dkv[8 * m + 7]));
+            *(uint4*)(kt + off) = make_uint4(pack_bf16x2(dvv[8 * m], dvv[8 * m + 1]),
+                                             pack_bf16x2(dvv[8 * m + 2], dvv[8 * m + 3]),
+                                             pack_bf16x2(dvv[8 * m + 4], dvv[8 * m + 5]),
+                                             pack_bf16x2(dvv[8 * m + 6], dvv[8 * m + 7]));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar_acce);
+        float* red = (float*)(smem + OFF_RED) + (g & 1) * TOK * 2;
+        red[row * 2 + h] = dbp;
+        fence_proxy_async();
+        named_bar_sync(1, EPI);
+        const int tok = tl * TOK + row;
+        if (h == 0 && tok < S) dbeta[(size_t)n * S + tok] = red[row * 2] + red[row * 2 + 1];
+        if (et == 0) {
+          // dk from the V buffer, dv from the K buffer (rows past S are clipped)
+          tma_store_3d(&tmDK, smem_u32(vt), 0, tl * TOK, n);
+          tma_store_3d(&tmDK, smem_u32(vt + BOX), 64, tl * TOK, n);
+          tma_store_3d(&tmDV, smem_u32(kt), 0, tl * TOK, n);
+          tma_store_3d(&tmDV, smem_u32(kt + BOX), 64, tl * TOK, n);
+          bulk_commit();
+          bulk_wait_read0();
+          mbar_arrive(bar_empty + 8 * s);
+        }
+      }
+      if (stop) break;
+    }
+    if (et == 0) bulk_wait0();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+cudaError_t tc_bwd_tokens(const void* k, const void* v, const float* beta, const void* bimg,
+                          void* dk, void* dv, float* dbeta, long long N, int S, float c,
+                          cudaStream_t st) {
+  CUtensorMap mk, mv, mdk, mdv;
+  cudaError_t e = make_map_bf16_3d(&mk, k, 128, S, N, 64, btk::TOK);
+  if (e == cudaSuccess) e = make_map_bf16_3d(&mv, v, 128, S, N, 64, btk::TOK);
+  if (e == cudaSuccess) e = make_map_bf16_3d(&mdk, dk, 128, S, N, 64, btk::TOK);
+  if (e == cudaSuccess) e = make_map_bf16_3d(&mdv, dv, 128, S, N, 64, btk::TOK);
+  if (e != cudaSuccess) return e;
+  static bool attr = false;
+  if (!attr) {
+    e = cudaFuncSetAttribute(k_bwd_tok_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, btk::SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int grid = (int)(N < num_sms() ? N : num_sms());
+  k_bwd_tok_tc<<<grid, btk::THREADS, btk::SMEM, st>>>(mk, mv, mdk, mdv, beta,
+                                                      (const uint8_t*)bimg, dbeta, (int)N, S, c);
   count_launch();
   return cudaGetLastError();
 }

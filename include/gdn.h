@@ -314,8 +314,10 @@ GDN_API int gdn_profile_enable(int enable);
 /* Sums the recorded kernel durations per phase, waiting on the events:
  * ms[i] and counts[i] for phase i < n, with phases 0 prologue, 1 contract,
  * 2 compose, 3 prefix, 4 scan/replay, 5 readout, 6 replay fused with the
- * readout, 7 contraction with the sequential scan alongside. Returns the
- * number of phases written, or a negative status. */
+ * readout, 7 contraction with the sequential scan alongside; backward:
+ * 8 recompute, 9 dO^T Q, 10 adjoint chain, 11 per-frame terms, 12 token
+ * gradients and dq. Returns the number of phases written, or a negative
+ * status. */
 GDN_API int gdn_profile_read(double* ms, long long* counts, int n);
 
 /* ABI version: major * 10000 + minor * 100 + patch. */

@@ -33,12 +33,13 @@ def upstream(seed, B, H, T, S, D, bf16):
     return dO, dS
 
 
-def check_case(arr, dO, dS, bf16, tol, reverse=False, block=0, b_slabs=None):
+def check_case(arr, dO, dS, bf16, tol, reverse=False, block=0, b_slabs=None, force_simt=False):
     d = U.dev_inputs(arr, bf16)
     d_out = U.to_dev(dO, bf16)
     d_s = torch.from_numpy(dS).cuda() if dS is not None else None
     got = api.frame_scan_bwd(d["q"], d["k"], d["v"], d["beta"], d["gamma"], d["state"], d_out,
-                             d_s, reverse=reverse, block_reset=bool(block), block=block or 3)
+                             d_s, reverse=reverse, block_reset=bool(block), block=block or 3,
+                             force_simt=force_simt)
     torch.cuda.synchronize()
     api.check_device_status()
     B, H = arr["beta"].shape[:2]
@@ -66,13 +67,24 @@ MODES = {"forward": dict(), "reverse": dict(reverse=True), "forward_block": dict
 
 
 @pytest.mark.parametrize("mode", list(MODES))
-@pytest.mark.parametrize("D,bf16", [(16, False), (64, False), (128, False), (64, True),
-                                    (128, True), (256, True)])
-def test_backward_small(D, bf16, mode):
-    B, H, T, S = 2, 1, 7, 50
+@pytest.mark.parametrize("D,bf16,simt", [(16, False, True), (64, False, True), (128, False, True),
+                                         (64, True, True), (128, True, False), (128, True, True),
+                                         (256, True, True)])
+def test_backward_small(D, bf16, simt, mode):
+    """Every mode; D = 128 bf16 on both the tensor-core and the CUDA-core path."""
+    B, H, T, S = 2, 1, 7, 150
     arr = U.random_case(3000 + D, B, H, T, S, D, bf16=bf16, state=True)
     dO, dS = upstream(17 + D, B, H, T, S, D, bf16)
-    check_case(arr, dO, dS, bf16, U.TOL_BF16 if bf16 else U.TOL_FP32, **MODES[mode])
+    check_case(arr, dO, dS, bf16, U.TOL_BF16 if bf16 else U.TOL_FP32, force_simt=simt,
+               **MODES[mode])
+
+
+def test_backward_many_heads_tc():
+    """More heads than chains fit beside the contraction: the recompute runs
+    as its own launches (tensor-core path)."""
+    arr = U.random_case(51, 1, 40, 4, 70, 128, bf16=True, state=True)
+    dO, dS = upstream(52, 1, 40, 4, 70, 128, True)
+    check_case(arr, dO, dS, True, U.TOL_BF16, b_slabs=[(0, 0), (0, 17), (0, 39)])
 
 
 def test_backward_without_state_terms():
@@ -89,9 +101,12 @@ def test_backward_edge_sizes():
         check_case(arr, dO, dS, True, U.TOL_BF16)
 
 
-def test_backward_full_size_clip():
-    """The 5 s 720p clip (B=1, H=16, T=21, S=3600, D=128, bf16), sampled slabs."""
-    cfg = synth.CONFIGS["clip5s_720p"]
+@pytest.mark.parametrize("name", ["clip5s_720p", "rollout60s_720p"])
+def test_backward_full_size(name):
+    """The 720p workloads (B=1, H=16, S=3600, D=128, bf16; T = 21 or 121) on the
+    tensor-core path, in the launch configuration bench.py --bwd times, sampled
+    slabs."""
+    cfg = synth.CONFIGS[name]
     arr = synth.make_inputs(cfg)
     dO, dS = upstream(2024, cfg.B, cfg.H, cfg.T, cfg.S, cfg.D, True)
     check_case(arr, dO, dS, True, U.TOL_BF16, b_slabs=[(0, 0), (0, cfg.H - 1)])
