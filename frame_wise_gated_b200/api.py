@@ -105,7 +105,8 @@ SIGNATURES = {
 }
 
 PHASES = ("prologue", "contract", "compose", "prefix", "scan", "readout", "scan_readout",
-          "contract_scan", "bwd_recompute", "bwd_w", "bwd_adjoint", "bwd_frame", "bwd_tokens")
+          "contract_scan", "bwd_recompute", "bwd_w", "bwd_adjoint", "bwd_frame", "bwd_tokens",
+          "bwd_dq")
 
 _lib = None
 

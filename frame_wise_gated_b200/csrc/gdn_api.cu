@@ -32,7 +32,7 @@ void count_launch(int n) { t_launches += n; }
 enum Phase {
   PH_PROLOGUE = 0, PH_CONTRACT, PH_COMPOSE, PH_PREFIX, PH_SCAN, PH_READOUT, PH_SCAN_READOUT,
   PH_CONTRACT_SCAN, PH_BWD_RECOMPUTE, PH_BWD_W, PH_BWD_ADJOINT, PH_BWD_FRAME, PH_BWD_TOKENS,
-  PH_COUNT
+  PH_BWD_DQ, PH_COUNT
 };
 struct ProfRec {
   int phase;
@@ -439,7 +439,7 @@ static bool bwd_tc_by_flags(int D, unsigned flags) {
 }
 
 struct BwdLayout {
-  size_t A, U, Sfr, W, G, dM, Bimg, zero, flags, P2, P3, P5, total;
+  size_t A, U, Sfr, W, G, dM, Bimg, zero, flags, s0, P2, P3, P5, total;
 };
 
 static BwdLayout make_bwd_layout(int B, int H, int T, int S, int D, unsigned f) {
@@ -454,8 +454,10 @@ static BwdLayout make_bwd_layout(int B, int H, int T, int S, int D, unsigned f) 
     *m = off;
     off = align256(off + mat);
   }
-  L.Bimg = L.zero = L.flags = L.P2 = L.P3 = L.P5 = off;
+  L.Bimg = L.zero = L.flags = L.s0 = L.P2 = L.P3 = L.P5 = off;
   if (tc) {
+    L.s0 = off;  // state_in as bf16 hi/lo pairs
+    off = align256(off + (size_t)B * H * 2 * D * D * 2);
     L.Bimg = off;  // per frame [dA + dA^T ; G] bf16, 64 KiB
     off = align256(off + frames * 65536);
     L.zero = off;  // an all-zero operand image
@@ -475,10 +477,9 @@ static BwdLayout make_bwd_layout(int B, int H, int T, int S, int D, unsigned f) 
 
 // Tensor-core backward, D = 128, bf16: recompute with the forward kernels
 // (states as bf16 hi/lo pairs), W = dO^T Q by the contraction, G by the
-// adjoint chain, per-frame terms on CUDA cores, token gradients and dq on
-// tensor cores.
+// adjoint chain, per-frame terms, token gradients and dq on tensor cores.
 static int scan_bwd_tc(const gdn_bwd_params& p, char* ws, size_t oA, size_t oU, size_t oSfr,
-                       size_t oW, size_t oG, size_t odM, size_t oB, size_t oZero, size_t oFlags,
+                       size_t oW, size_t oG, size_t oS0, size_t oB, size_t oZero, size_t oFlags,
                        cudaStream_t st) {
   const unsigned f = p.flags;
   const bool reverse = (f & GDN_REVERSE) != 0;
@@ -490,7 +491,6 @@ static int scan_bwd_tc(const gdn_bwd_params& p, char* ws, size_t oA, size_t oU, 
   float* A = (float*)(ws + oA);
   float* U = (float*)(ws + oU);
   float* W = (float*)(ws + oW);
-  float* dM = (float*)(ws + odM);
   cudaError_t e;
   // 1. recompute A_t (operand images), U_t and the states S_t (hi/lo pairs)
   ChainArgs a;
@@ -556,10 +556,8 @@ static int scan_bwd_tc(const gdn_bwd_params& p, char* ws, size_t oA, size_t oU, 
   // 4. per frame: dM = S'^T G, dA + dA^T and dgamma, the token kernel's operand
   {
     PhaseScope ps(PH_BWD_FRAME, st);
-    e = simt_bwd_dm(a.Sfr, p.state_in, b.Gout, dM, frames, p.T, 128, a.reverse, a.seq_reset,
-                    block, true, st);
-    if (e == cudaSuccess)
-      e = simt_bwd_dterm(dM, A, true, p.gamma, p.dgamma, frames, 128, b.Gout, ws + oB, st);
+    e = tc_bwd_frames(a.Sfr, p.state_in, ws + oS0, ws + oZero, b.Gout, A, p.gamma, p.dgamma,
+                      ws + oB, frames, heads, p.T, a.reverse, a.seq_reset, block, st);
     if (e == cudaSuccess && p.d_state_in)
       e = simt_bwd_ds0(b.Gout, A, p.gamma, p.d_state_in, heads, p.T, frame_at(0, p.T, a.reverse),
                        st);
@@ -569,7 +567,10 @@ static int scan_bwd_tc(const gdn_bwd_params& p, char* ws, size_t oA, size_t oU, 
   {
     PhaseScope ps(PH_BWD_TOKENS, st);
     e = tc_bwd_tokens(p.k, p.v, p.beta, ws + oB, p.dk, p.dv, p.dbeta, frames, p.S, (float)c, st);
-    if (e == cudaSuccess) e = tc_readout_trans(p.d_out, a.Sfr, p.dq, frames, p.S, st);
+  }
+  if (e == cudaSuccess) {
+    PhaseScope ps(PH_BWD_DQ, st);
+    e = tc_readout_trans(p.d_out, a.Sfr, p.dq, frames, p.S, st);
   }
   if (e != cudaSuccess) return cuda_fail(e, "backward: token gradients");
   return GDN_OK;
@@ -620,7 +621,7 @@ static int scan_bwd(const gdn_bwd_params& p, cudaStream_t st) {
   if (bwd_tc_by_flags(p.D, f)) {
     if (device_cc_major() != 10)
       return fail(GDN_ERR_UNSUPPORTED, "bf16 D = 128 backward runs on sm_100 (else pass GDN_FORCE_SIMT)%s");
-    return scan_bwd_tc(p, ws, L.A, L.U, L.Sfr, L.W, L.G, L.dM, L.Bimg, L.zero, L.flags, st);
+    return scan_bwd_tc(p, ws, L.A, L.U, L.Sfr, L.W, L.G, L.s0, L.Bimg, L.zero, L.flags, st);
   }
   // 1. forward recompute: A_t, U_t, then the states S_t (one chain per head)
   e = simt_contract(bf16, p.k, p.v, p.beta, A, U, frames, p.S, p.D, (float)(c * c), (float)c, st);

@@ -224,6 +224,13 @@ cudaError_t tc_contract_scan(const void* k, const void* v, const float* beta, fl
 // dk, dv, dbeta from the per-frame B operand [dA + dA^T ; G] (64 KiB bf16).
 cudaError_t tc_readout_trans(const void* x, const void* Sfr_hilo, void* out, long long N, int S,
                              cudaStream_t st);
+// Per-frame backward terms on tensor cores: dA + dA^T and G into the token
+// kernel's operand, dgamma. s0_hilo: scratch for state_in as hi/lo pairs
+// (heads x 64 KiB); zero_hilo: 64 KiB of zeros.
+cudaError_t tc_bwd_frames(const void* Sfr_hilo, const float* state_in, void* s0_hilo,
+                          const void* zero_hilo, const void* G_hilo, const void* A_img,
+                          const float* gamma, float* dgamma, void* bimg, long long N, int heads,
+                          int T, int reverse, int seq_reset, int block, cudaStream_t st);
 cudaError_t tc_bwd_tokens(const void* k, const void* v, const float* beta, const void* bimg,
                           void* dk, void* dv, float* dbeta, long long N, int S, float c,
                           cudaStream_t st);

@@ -4020,6 +4020,273 @@ cudaError_t tc_bwd_tokens(const void* k, const void* v, const float* beta, const
   return cudaGetLastError();
 }
 
+// ============================================================================
+// Backward per-frame terms on tensor cores (D = 128).
+//
+// Per frame (scan position j): dM = S'^T G and dM^T = G^T S' as split
+// products (hi/lo pairs of both, three MMAs per 16 rows: ~16-bit operands),
+// with S' = the state entering frame j (the previous frame's stored state,
+// state_in for the first frame, zeros after a reset) and G = dL/dS after
+// frame j, both bf16 (hi, lo) tiles brought in by TMA. Four epilogue warps
+// (row i of dM each) then write
+//   dA + dA^T = -gamma (dM + dM^T)        (rows 0..127 of the token kernel's
+//   G rounded to bf16                      operand; rows 128..255)
+//   dgamma = <dM, I - A>                   (A_t from its operand image)
+// The accumulators (dM | dM^T, 256 columns) are double-buffered in TMEM, so
+// one frame's epilogue runs under the next frame's loads and MMAs.
+// ============================================================================
+namespace bfr {
+constexpr int D = 128;
+constexpr int BOX = 128 * 128;          // [128 rows][64 columns] bf16: 16 KiB
+constexpr int MAT = 4 * BOX;            // hi (2 boxes) + lo (2 boxes): 64 KiB
+constexpr int OFF_S = 0;                // S' (hi, lo)
+constexpr int OFF_G = OFF_S + MAT;      // G (hi, lo)
+constexpr int OFF_BAR = OFF_G + MAT;
+constexpr int NBAR = 2 + 2 + 2 + 1;     // in_full, in_empty, acc_full[2], acc_empty[2], fin
+constexpr int OFF_RED = OFF_BAR + 64;
+constexpr int OFF_MISC = OFF_RED + 4 * 4;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+constexpr int THREADS = 64 + 128;
+constexpr uint32_t TMEM_COLS = 512;
+}  // namespace bfr
+
+// Which hi/lo source holds S' of frame-head n: 0 = stored states (index
+// prev), 1 = converted state_in (index bh), 2 = zeros.
+struct FrameSrc {
+  int kind, idx;
+};
+__device__ __forceinline__ FrameSrc frame_prev_src(int n, int T, int reverse, int seq_reset,
+                                                   int block, int has_s0) {
+  const int bh = n / T, t = n % T;
+  const int j = reverse ? T - 1 - t : t;
+  if (j == 0) return FrameSrc{has_s0 ? 1 : 2, has_s0 ? bh : 0};
+  const int tp = frame_at(j - 1, T, reverse);
+  if (seq_reset && (t / block) != (tp / block)) return FrameSrc{2, 0};
+  return FrameSrc{0, bh * T + tp};
+}
+
+__global__ void __launch_bounds__(bfr::THREADS, 1)
+    k_bwd_frame_tc(const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmS0,
+                   const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmG,
+                   const uint8_t* __restrict__ Aimg, const __nv_bfloat16* __restrict__ Ghilo,
+                   const float* __restrict__ gamma, float* __restrict__ dgamma,
+                   uint8_t* __restrict__ bimg, int N, int T, int reverse, int seq_reset, int block,
+                   int has_s0) {
+  using namespace bfr;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar_inf = sb + OFF_BAR;
+  const uint32_t bar_ine = bar_inf + 8;
+  const uint32_t bar_accf = bar_ine + 8;
+  const uint32_t bar_acce = bar_accf + 16;
+  const uint32_t bar_fin = bar_acce + 16;
+  uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
+  if (threadIdx.x == 0) {
+    mbar_init(bar_inf, 1);
+    mbar_init(bar_ine, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_accf + 8 * b, 1);
+      mbar_init(bar_acce + 8 * b, 128);
+    }
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int my_count = (int)blockIdx.x < N ? (N - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int nin = 0;
+      for (int i = 0; i < my_count; ++i) {
+        const int n = blockIdx.x + i * gridDim.x;
+        if (!mbar_wait(bar_ine, ((uint32_t)i & 1) ^ 1, abort_flag, &g_tc_status, 71)) break;
+        const FrameSrc src = frame_prev_src(n, T, reverse, seq_reset, block, has_s0);
+        const CUtensorMap* ms = src.kind == 0 ? &tmS : src.kind == 1 ? &tmS0 : &tmZ;
+        mbar_arrive_expect_tx(bar_inf, 2 * MAT);
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            tma_load_3d(sb + OFF_S + (2 * hl + x) * BOX, ms, bar_inf, 64 * x, 0, 2 * src.idx + hl);
+            tma_load_3d(sb + OFF_G + (2 * hl + x) * BOX, &tmG, bar_inf, 64 * x, 0, 2 * n + hl);
+          }
+        ++nin;
+      }
+      volatile int keep_waiting = 0;
+      if (nin > 0) mbar_wait(bar_inf, (uint32_t)(nin - 1) & 1, &keep_waiting, &g_tc_status, 72);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, true, true);
+      for (int i = 0; i < my_count; ++i) {
+        const int b = i & 1;
+        if (!mbar_wait(bar_acce + 8 * b, ((uint32_t)(i >> 1) & 1) ^ 1, abort_flag, &g_tc_status, 73))
+          break;
+        if (!mbar_wait(bar_inf, (uint32_t)i & 1, abort_flag, &g_tc_status, 74)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + b * 256;
+        const uint32_t sh = sb + OFF_S, sl = sh + 2 * BOX, gh = sb + OFF_G, gl = gh + 2 * BOX;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          // rows r = 16 kk ..: S'^T and G^T as MN-major A, G and S' as MN-major B
+          const uint32_t o = kk * 2048;
+          const uint64_t dsh = smem_desc_sw128(sh + o, BOX, 1024), dsl = smem_desc_sw128(sl + o, BOX, 1024);
+          const uint64_t dgh = smem_desc_sw128(gh + o, BOX, 1024), dgl = smem_desc_sw128(gl + o, BOX, 1024);
+          const uint32_t acc = kk > 0 ? 1u : 0u;
+          mma_bf16(d, dsh, dgh, idesc, acc);          // dM = S'^T G
+          mma_bf16(d, dsl, dgh, idesc, 1u);
+          mma_bf16(d, dsh, dgl, idesc, 1u);
+          mma_bf16(d + 128, dgh, dsh, idesc, acc);    // dM^T = G^T S'
+          mma_bf16(d + 128, dgl, dsh, idesc, 1u);
+          mma_bf16(d + 128, dgh, dsl, idesc, 1u);
+        }
+        mma_commit(bar_ine);
+        mma_commit(bar_accf + 8 * b);
+      }
+      mma_commit(bar_fin);
+      volatile int keep_waiting = 0;
+      mbar_wait(bar_fin, 0, &keep_waiting, &g_tc_status, 75);
+    }
+    __syncwarp();
+  } else {
+    // ---- epilogue: row i of dM per thread ----
+    const int q = warp & 3;
+    const int i_row = q * 32 + lane;
+    float* red = (float*)(smem + OFF_RED);
+    for (int i = 0; i < my_count; ++i) {
+      const int n = blockIdx.x + i * gridDim.x;
+      const int b = i & 1;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(bar_accf + 8 * b, (uint32_t)(i >> 1) & 1, abort_flag, &g_tc_status, 76);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (named_bar_or(1, 128, !ok || *abort_flag)) break;
+      tc_fence_after();
+      const float g = gamma[n];
+      const uint8_t* aimg = Aimg + (size_t)n * kImageBytes;
+      uint8_t* bo = bimg + (size_t)n * 65536;
+      float part = 0.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t m[32], mt[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 256 + c0, m);
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 256 + 128 + c0, mt);
+        tmem_wait_ld();
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          // 8 columns j = c0 + 8 ch ..: A_t row i_row from the image (hi + lo)
+          const int col = c0 + 8 * ch;
+          const int ao = (col >> 6) * 16384 + i_row * 128 + ((((col & 63) >> 3) ^ (i_row & 7)) << 4);
+          const uint4 ah = *(const uint4*)(aimg + ao), al = *(const uint4*)(aimg + 32768 + ao);
+          const uint32_t ahw[4] = {ah.x, ah.y, ah.z, ah.w}, alw[4] = {al.x, al.y, al.z, al.w};
+          float o[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 fh = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ahw[e]));
+            const float2 fl = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&alw[e]));
+            const float a0 = fh.x + fl.x, a1 = fh.y + fl.y;
+            const int j0 = col + 2 * e;
+            const float m0 = __uint_as_float(m[8 * ch + 2 * e]), m1 = __uint_as_float(m[8 * ch + 2 * e + 1]);
+            part += m0 * ((j0 == i_row ? 1.f : 0.f) - a0) + m1 * ((j0 + 1 == i_row ? 1.f : 0.f) - a1);
+            o[2 * e] = -g * (m0 + __uint_as_float(mt[8 * ch + 2 * e]));
+            o[2 * e + 1] = -g * (m1 + __uint_as_float(mt[8 * ch + 2 * e + 1]));
+          }
+          const int bo_off = (col >> 6) * 32768 + i_row * 128 + ((((col & 63) >> 3) ^ (i_row & 7)) << 4);
+          *(uint4*)(bo + bo_off) = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                                             pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_acce + 8 * b);
+      // G row i_row (hi + lo, rounded) -> operand row 128 + i_row
+      const __nv_bfloat16* gh = Ghilo + (size_t)n * 2 * D * D + (size_t)i_row * D;
+      const int r = 128 + i_row;
+#pragma unroll 2
+      for (int col = 0; col < 128; col += 8) {
+        const uint4 hv = *(const uint4*)(gh + col), lv = *(const uint4*)(gh + (size_t)D * D + col);
+        const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w}, lw[4] = {lv.x, lv.y, lv.z, lv.w};
+        uint32_t ow[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 fh = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hw[e]));
+          const float2 fl = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lw[e]));
+          ow[e] = pack_bf16x2(fh.x + fl.x, fh.y + fl.y);
+        }
+        const int off = (col >> 6) * 32768 + r * 128 + ((((col & 63) >> 3) ^ (r & 7)) << 4);
+        *(uint4*)(bo + off) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+      }
+      // dgamma: sum over the 128 rows
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+      if (lane == 0) red[q] = part;
+      named_bar_sync(1, 128);
+      if (threadIdx.x == 64) dgamma[n] = red[0] + red[1] + red[2] + red[3];
+      named_bar_sync(1, 128);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// fp32 states [heads][D][D] -> bf16 (hi, lo) pairs [heads][2][D][D].
+__global__ void k_to_hilo(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst, int D) {
+  const size_t mat = (size_t)D * D;
+  const float* m = src + (size_t)blockIdx.x * mat;
+  __nv_bfloat16* o = dst + (size_t)blockIdx.x * 2 * mat;
+  for (size_t e = threadIdx.x; e < mat; e += blockDim.x) {
+    const float x = m[e];
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    o[e] = h;
+    o[mat + e] = __float2bfloat16_rn(x - __bfloat162float(h));
+  }
+}
+
+cudaError_t tc_bwd_frames(const void* Sfr_hilo, const float* state_in, void* s0_hilo,
+                          const void* zero_hilo, const void* G_hilo, const void* A_img,
+                          const float* gamma, float* dgamma, void* bimg, long long N, int heads,
+                          int T, int reverse, int seq_reset, int block, cudaStream_t st) {
+  CUtensorMap ms, ms0, mz, mg;
+  cudaError_t e = make_map_bf16_3d(&ms, Sfr_hilo, 128, 128, 2 * (uint64_t)N, 64, 128);
+  if (e == cudaSuccess && state_in) {
+    k_to_hilo<<<heads, 256, 0, st>>>(state_in, (__nv_bfloat16*)s0_hilo, 128);
+    count_launch();
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess)
+    e = make_map_bf16_3d(&ms0, state_in ? s0_hilo : zero_hilo, 128, 128,
+                         state_in ? 2 * (uint64_t)heads : 2, 64, 128);
+  if (e == cudaSuccess) e = make_map_bf16_3d(&mz, zero_hilo, 128, 128, 2, 64, 128);
+  if (e == cudaSuccess) e = make_map_bf16_3d(&mg, G_hilo, 128, 128, 2 * (uint64_t)N, 64, 128);
+  if (e != cudaSuccess) return e;
+  static bool attr = false;
+  if (!attr) {
+    e = cudaFuncSetAttribute(k_bwd_frame_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, bfr::SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int grid = (int)(N < num_sms() ? N : num_sms());
+  k_bwd_frame_tc<<<grid, bfr::THREADS, bfr::SMEM, st>>>(
+      ms, ms0, mz, mg, (const uint8_t*)A_img, (const __nv_bfloat16*)G_hilo, gamma, dgamma,
+      (uint8_t*)bimg, (int)N, T, reverse, seq_reset, block, state_in ? 1 : 0);
+  count_launch();
+  return cudaGetLastError();
+}
+
 // ---- public entry points of the tensor-core kernels (dispatch on D) ----
 cudaError_t tc_contract(const void* k, const void* v, const float* beta, float* A, float* U,
                         long long N, int S, int D, float cA, float cU, int a_image,

@@ -316,7 +316,7 @@ GDN_API int gdn_profile_enable(int enable);
  * 2 compose, 3 prefix, 4 scan/replay, 5 readout, 6 replay fused with the
  * readout, 7 contraction with the sequential scan alongside; backward:
  * 8 recompute, 9 dO^T Q, 10 adjoint chain, 11 per-frame terms, 12 token
- * gradients and dq. Returns the number of phases written, or a negative
+ * gradients, 13 dq. Returns the number of phases written, or a negative
  * status. */
 GDN_API int gdn_profile_read(double* ms, long long* counts, int n);
 
