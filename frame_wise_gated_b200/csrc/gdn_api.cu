@@ -379,12 +379,14 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
     o.flags = (int*)(ws + L.flags);
     if (bidir) {
       // forward never reset; reverse reset per block, run block by block
-      o.dir[0] = OvlDir{0, 0, 0, p.state_in, p.state_out};
-      o.dir[1] = OvlDir{1, 1, 0, p.state_in, p.state_out_rev};
+      o.dir[0] = OvlDir{0, 0, 0, p.state_in, p.state_out, 0};
+      o.dir[1] = OvlDir{1, 1, 0, p.state_in, p.state_out_rev, 0};
     } else {
       o.dir[0] = OvlDir{(f & GDN_REVERSE) ? 1 : 0, 0, block_reset ? 1 : 0, p.state_in,
-                        p.state_out};
+                        p.state_out, 0};
     }
+    o.a_image = 1;
+    o.contract_rev = o.dir[0].reverse && !o.dir[0].blocks_asc;
     {
       PhaseScope ps(PH_CONTRACT_SCAN, st);
       e = tc_contract_scan(k, p.v, p.beta, A, U, frames, p.S, (float)(c * c), (float)c, ppk, o,
@@ -524,7 +526,9 @@ static int scan_bwd_tc(const gdn_bwd_params& p, char* ws, size_t oA, size_t oU, 
       o.gamma = p.gamma;
       o.A = (const uint8_t*)A;
       o.flags = (int*)(ws + oFlags);
-      o.dir[0] = OvlDir{a.reverse, 0, a.seq_reset, p.state_in, nullptr};
+      o.dir[0] = OvlDir{a.reverse, 0, a.seq_reset, p.state_in, nullptr, 0};
+      o.a_image = 1;
+      o.contract_rev = a.reverse;
       e = tc_contract_scan(p.k, p.v, p.beta, A, U, frames, p.S, (float)(c * c), (float)c, nullptr,
                            o, a.Sfr, nullptr, st);
     } else {
@@ -534,25 +538,46 @@ static int scan_bwd_tc(const gdn_bwd_params& p, char* ws, size_t oA, size_t oU, 
     }
   }
   if (e != cudaSuccess) return cuda_fail(e, "backward: recompute");
-  // 2. W_t = dO_t^T Q_t: the contraction's U with keys := q, values := dO, beta = 1
-  {
-    PhaseScope ps(PH_BWD_W, st);
-    e = tc_contract(p.q, p.d_out, nullptr, A, W, frames, p.S, 128, 1.f, 1.f, 2, nullptr, st);
-  }
-  if (e != cudaSuccess) return cuda_fail(e, "backward: dO^T Q");
-  // 3. adjoint chain: G_t as hi/lo pairs
+  // 2./3. W_t = dO_t^T Q_t (the contraction's U with keys := q, values := dO,
+  // beta = 1) and the adjoint chain for G_t (hi/lo pairs): side by side in one
+  // launch when the chains fit, the contraction visiting frames in the
+  // adjoint's order; else one after the other
   ChainArgs b = a;
   b.mode = CHAIN_ADJOINT;
   b.Zw = W;
   b.Gout = (float*)(ws + oG);
   b.dS_out = p.d_state_out;
   b.zero_img = ws + oZero;
-  {
+  e = cudaMemsetAsync(ws + oZero, 0, kImageBytes, st);
+  if (e != cudaSuccess) return cuda_fail(e, "backward: zero image");
+  if (heads <= tc_overlap_max_chains()) {
     PhaseScope ps(PH_BWD_ADJOINT, st);
-    e = cudaMemsetAsync(ws + oZero, 0, kImageBytes, st);
-    if (e == cudaSuccess) e = tc_chain(b, heads, st);
+    OvlArgs w;
+    memset(&w, 0, sizeof(w));
+    w.heads = heads;
+    w.T = p.T;
+    w.block = block;
+    w.ndir = 1;
+    w.gamma = p.gamma;
+    w.A = (const uint8_t*)A;
+    w.flags = (int*)(ws + oFlags);
+    w.zero_img = (const uint8_t*)(ws + oZero);
+    w.a_image = 2;  // keep the recomputed A_t images
+    w.contract_rev = !a.reverse;
+    w.dir[0] = OvlDir{a.reverse, 0, a.seq_reset, p.d_state_out, nullptr, 1};
+    e = tc_contract_scan(p.q, p.d_out, nullptr, A, W, frames, p.S, 1.f, 1.f, nullptr, w, b.Gout,
+                         nullptr, st);
+    if (e != cudaSuccess) return cuda_fail(e, "backward: dO^T Q + adjoint chain");
+  } else {
+    {
+      PhaseScope ps(PH_BWD_W, st);
+      e = tc_contract(p.q, p.d_out, nullptr, A, W, frames, p.S, 128, 1.f, 1.f, 2, nullptr, st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "backward: dO^T Q");
+    PhaseScope ps(PH_BWD_ADJOINT, st);
+    e = tc_chain(b, heads, st);
+    if (e != cudaSuccess) return cuda_fail(e, "backward: adjoint chain");
   }
-  if (e != cudaSuccess) return cuda_fail(e, "backward: adjoint chain");
   // 4. per frame: dM = S'^T G, dA + dA^T and dgamma, the token kernel's operand
   {
     PhaseScope ps(PH_BWD_FRAME, st);

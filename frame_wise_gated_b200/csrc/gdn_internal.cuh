@@ -199,8 +199,12 @@ struct OvlDir {
   int blocks_asc;  // reverse scan reset per block, run block by block in
                    // ascending time (frames descending inside each block)
   int seq_reset;   // zero the state on entering a new block in scan order
-  const float* state_in;  // [heads, D, D] or null
+  const float* state_in;  // [heads, D, D] or null (adjoint: dL/d(state_out))
   float* state_out;       // [heads, D, D] or null
+  int adjoint;     // backward: G over the forward scan (direction `reverse`)
+                   // backwards, G <- W_t + g' (G - G A') with A' = A of the
+                   // next forward frame (from `A`); the launch's contraction
+                   // computes W_t into its U output
 };
 
 struct OvlArgs {
@@ -209,6 +213,9 @@ struct OvlArgs {
   const uint8_t* A;  // operand images of A_t, [heads*T][kImageBytes]
   int* flags;        // [heads*T], zero before the launch
   OvlDir dir[2];
+  const uint8_t* zero_img;  // adjoint: an all-zero operand image
+  int a_image;       // the contraction's A output: 1 operand images, 2 not written
+  int contract_rev;  // the contraction visits frames in reverse time
 };
 
 bool tc_overlap_supported(int D);

@@ -1694,14 +1694,30 @@ constexpr int EPI_WARPS = 4;  // contraction epilogue warps: publishes per frame
 }  // namespace ovl
 
 // Scan step j of a direction: its frame, whether the state entering it is
-// replaced (by state_in when `seed`, else by zeros) and whether the state after
-// it is the direction's final state.
+// replaced (by state_in when `seed`, else by zeros), whether the state after
+// it is the direction's final state, the frame whose A image is Y (-1: zeros)
+// and the frame whose gamma is alpha (-1: 1).
 struct OvlStep {
-  int t, reset, seed, last;
+  int t, reset, seed, last, yt, at;
 };
 
 __device__ __forceinline__ OvlStep ovl_step(const OvlDir& d, int T, int block, int j) {
   OvlStep s;
+  if (d.adjoint) {
+    const int jf = T - 1 - j;  // forward scan position
+    s.t = d.reverse ? T - 1 - jf : jf;
+    s.last = 0;
+    if (j == 0) {
+      s.reset = s.seed = 1;  // G starts from dL/d(state_out)
+      s.yt = s.at = -1;
+    } else {
+      const int tn = d.reverse ? T - 2 - jf : jf + 1;  // next frame in forward order
+      s.reset = d.seq_reset && (s.t / block) != (tn / block);
+      s.seed = 0;
+      s.yt = s.at = tn;
+    }
+    return s;
+  }
   if (d.blocks_asc) {
     const int b = j / block, o = j - b * block;
     const int t1 = min(b * block + block, T);
@@ -1716,6 +1732,7 @@ __device__ __forceinline__ OvlStep ovl_step(const OvlDir& d, int T, int block, i
     s.seed = j == 0;
     s.last = j == T - 1;
   }
+  s.yt = s.at = s.t;
   return s;
 }
 
@@ -1810,11 +1827,14 @@ __device__ __forceinline__ void ovl_chain_body(const OvlArgs& o, const CUtensorM
 
   // operands of the frame at scan step j: wait for its publication, then copy
   int ny = 0, nz = 0, nstore = 0;  // copies issued (leader)
-  auto fetch_y = [&](int t) -> bool {
-    const int n = bh * T + t;
+  // Y of a step: the A image of st.yt (zeros when -1), once frame st.t's
+  // contraction output is published
+  auto fetch_y = [&](const OvlStep& st) -> bool {
+    const int n = bh * T + st.t;
     if (!wait_flag_ge(o.flags + n, ovl::EPI_WARPS, abort_flag, 31)) return false;
     asm volatile("fence.proxy.async.global;" ::: "memory");
-    chain_fetch_y(sb + OFF_Y, o.A + (size_t)n * kImageBytes, bar_y);
+    chain_fetch_y(sb + OFF_Y,
+                  st.yt >= 0 ? o.A + ((size_t)bh * T + st.yt) * kImageBytes : o.zero_img, bar_y);
     ++ny;
     return true;
   };
@@ -1826,8 +1846,8 @@ __device__ __forceinline__ void ovl_chain_body(const OvlArgs& o, const CUtensorM
     ++nz;
   };
   if (leader && T > 0) {
-    const int t0 = ovl_step(d, T, o.block, 0).t;
-    if (fetch_y(t0)) fetch_z(t0);
+    const OvlStep s0 = ovl_step(d, T, o.block, 0);
+    if (fetch_y(s0)) fetch_z(s0.t);
   }
 
   float x[32];
@@ -1864,13 +1884,16 @@ __device__ __forceinline__ void ovl_chain_body(const OvlArgs& o, const CUtensorM
     }
     mbar_wait(bar_mma, (uint32_t)j & 1, abort_flag, &g_tc_status, 33);
     tc_fence_after();
-    // the Y buffer is free: the next frame's A_t image, once published
+    // the Y buffer is free: the next step's image, once its frame is published
     int tn = -1;
-    if (j + 1 < T) tn = ovl_step(d, T, o.block, j + 1).t;
-    if (leader && tn >= 0) fetch_y(tn);
+    if (j + 1 < T) {
+      const OvlStep sn = ovl_step(d, T, o.block, j + 1);
+      tn = sn.t;
+      if (leader) fetch_y(sn);
+    }
     mbar_wait(bar_z, (uint32_t)j & 1, abort_flag, &g_tc_status, 34);
     {
-      const float alpha = o.gamma[(size_t)bh * T + st.t];
+      const float alpha = st.at >= 0 ? o.gamma[(size_t)bh * T + st.at] : 1.f;
       uint32_t r[32];
       tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + 32 * cg, r);
       tmem_wait_ld();
@@ -1935,9 +1958,9 @@ __global__ void __launch_bounds__(ovl::THREADS, 1)
   if ((int)blockIdx.x < nchain)
     ovl_chain_body(o, tmZ, tmS0, tmS1, blockIdx.x);
   else
-    contract_body<NST>(tmK, tmV, beta, A, U, N, S, cA, cU, 1, pro, (int)blockIdx.x - nchain,
-                  (int)gridDim.x - nchain, o.heads, o.T, o.dir[0].reverse && !o.dir[0].blocks_asc,
-                  o.flags);
+    contract_body<NST>(tmK, tmV, beta, A, U, N, S, cA, cU, o.a_image, pro,
+                       (int)blockIdx.x - nchain, (int)gridDim.x - nchain, o.heads, o.T,
+                       o.contract_rev, o.flags);
 }
 
 bool tc_overlap_supported(int D) { return D == 128; }
