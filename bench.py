@@ -44,6 +44,8 @@ from frame_wise_gated_b200 import synth  # noqa: E402
 METRIC = "GDN frame-scan frame·head·tokens/s (% of HBM roofline), 1xB200"
 UNIT = "frame·head·tokens/s"
 METRIC_BWD = "GDN frame-scan BACKWARD frame·head·tokens/s (% of HBM roofline), 1xB200"
+METRIC_TRAIN = ("GDN frame-scan TRAINING STEP (forward + backward from saved forward) "
+                "frame·head·tokens/s (% of HBM roofline), 1xB200")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -355,8 +357,16 @@ def run_ours(args, cfg):
                                                                  flags_b)),
                            device=dev, dtype=torch.uint8)
 
-        def step():  # noqa: F811
-            api.frame_scan_bwd(q, k, v, beta, gamma, s0, d_out, d_st, workspace=ws_b)
+        if args.train:
+            def step():  # noqa: F811
+                # forward, then the backward from the forward's saved workspace
+                api.frame_scan_fwd_ex(q, k, v, beta, gamma, s0, out=out, state_out=st_out,
+                                      workspace=ws, **kw)
+                api.frame_scan_bwd(q, k, v, beta, gamma, s0, d_out, d_st, workspace=ws_b,
+                                   saved_workspace=ws)
+        else:
+            def step():  # noqa: F811
+                api.frame_scan_bwd(q, k, v, beta, gamma, s0, d_out, d_st, workspace=ws_b)
 
     def barrier():
         if dist is not None:
@@ -411,6 +421,8 @@ def run_ours(args, cfg):
                 "alg_bytes_per_launch": alg, "ms_per_launch": dom_ms,
                 "dominant_kernel_overall": dom_all}
     step_bytes = algorithmic_bytes(cfg) if not args.bwd else backward_bytes(cfg)
+    if args.bwd and args.train:
+        step_bytes += algorithmic_bytes(cfg)
     if args.bwd:
         ach = step_bytes / (ms_step * 1e-3) / 1e9
         roof = {"kernel": "backward step (all kernels)", "bound": "hbm", "achieved": ach,
@@ -433,7 +445,8 @@ def run_ours(args, cfg):
 
     if rank == 0:
         line = {
-            "metric": METRIC if not args.bwd else METRIC_BWD, "value": value, "unit": UNIT,
+            "metric": METRIC if not args.bwd else (METRIC_TRAIN if args.train else METRIC_BWD),
+            "value": value, "unit": UNIT,
             "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -441,7 +454,8 @@ def run_ours(args, cfg):
             "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "T": cfg.T, "S": cfg.S,
                        "D": cfg.D, "grid": f"{cfg.grid_w}x{cfg.grid_h}",
                        "scan": plan_desc(args.plan, phases) if not args.bwd else
-                       "backward: recompute, adjoint chain, per-frame and per-token gradients",
+                       ("forward, then backward from its saved workspace" if args.train else
+                        "backward: recompute, adjoint chain, per-frame and per-token gradients"),
                        "prologue": cfg.prologue, "bidir_block": cfg.bidir_block,
                        "l2": f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB algorithmic per step)",
                        "parallelism": f"replica x{world} (heads shard, no collective)"},
@@ -519,6 +533,8 @@ def main():
                     help="replay spans inside the readout kernel")
     ap.add_argument("--bwd", action="store_true",
                     help="time the backward pass (gdn_frame_scan_bwd) instead of the forward")
+    ap.add_argument("--train", action="store_true",
+                    help="with --bwd: time forward + backward from the forward's saved workspace")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-frames", type=int, default=6,

@@ -75,6 +75,7 @@ class GdnBwdParams(ctypes.Structure):
         ("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int), ("S", ctypes.c_int),
         ("D", ctypes.c_int), ("flags", ctypes.c_uint),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("saved_workspace", ctypes.c_void_p),
     ]
 
 
@@ -339,11 +340,13 @@ def frame_scan_fwd_host(q, k, v, beta, gamma, state_in=None, *, out=None, state_
 
 def frame_scan_bwd(q, k, v, beta, gamma, state_in, d_out, d_state_out=None, *, reverse=False,
                    block_reset=False, block=3, keys_scaled=False, want_state_in_grad=True,
-                   force_simt=False, workspace=None, stream=None):
+                   force_simt=False, saved_workspace=None, workspace=None, stream=None):
     """Gradients through the frame scan (gdn_frame_scan_bwd): given
     d_out = dL/dO [B,H,T,S,D] and d_state_out = dL/d(state_out) [B,H,D,D]
     (or None), returns (dq, dk, dv, dbeta, dgamma, d_state_in) for the scan
-    with the same flags (d_state_in None unless want_state_in_grad)."""
+    with the same flags (d_state_in None unless want_state_in_grad).
+    saved_workspace: the workspace tensor of a frame_scan_fwd_ex call on the
+    same inputs and flags (bf16, D = 128), reused instead of recomputing."""
     B, H, T, S, D = q.shape
     bf16 = q.dtype == torch.bfloat16
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (d_out, "d_out")):
@@ -374,6 +377,7 @@ def frame_scan_bwd(q, k, v, beta, gamma, state_in, d_out, d_state_out=None, *, r
     p.flags = flags
     p.workspace = workspace.data_ptr()
     p.workspace_bytes = workspace.numel() * workspace.element_size()
+    p.saved_workspace = _ptr(saved_workspace)
     _check(lib().gdn_frame_scan_bwd(ctypes.byref(p), _stream(stream)), "gdn_frame_scan_bwd")
     return dq, dk, dv, dbeta, dgamma, ds0
 

@@ -494,6 +494,12 @@ static int scan_bwd_tc(const gdn_bwd_params& p, char* ws, size_t oA, size_t oU, 
   float* U = (float*)(ws + oU);
   float* W = (float*)(ws + oW);
   cudaError_t e;
+  const bool saved = p.saved_workspace != nullptr;
+  if (saved) {
+    // the forward call's A_t images and states (their offsets do not depend on flags)
+    const Layout Lf = make_layout(p.B, p.H, p.T, p.S, p.D, GDN_BF16);
+    A = (float*)((char*)p.saved_workspace + Lf.A);
+  }
   // 1. recompute A_t (operand images), U_t and the states S_t (hi/lo pairs)
   ChainArgs a;
   memset(&a, 0, sizeof(a));
@@ -511,10 +517,11 @@ static int scan_bwd_tc(const gdn_bwd_params& p, char* ws, size_t oA, size_t oU, 
   a.U = U;
   a.gamma = p.gamma;
   a.state_in = p.state_in;
-  a.Sfr = (float*)(ws + oSfr);
+  a.Sfr = saved ? (float*)((char*)p.saved_workspace + make_layout(p.B, p.H, p.T, p.S, p.D, GDN_BF16).Sfr)
+                : (float*)(ws + oSfr);
   a.sfr_hilo = 1;
   a.y_image = 1;
-  {
+  if (!saved) {
     PhaseScope ps(PH_BWD_RECOMPUTE, st);
     if (heads <= tc_overlap_max_chains()) {
       OvlArgs o;
@@ -536,8 +543,8 @@ static int scan_bwd_tc(const gdn_bwd_params& p, char* ws, size_t oA, size_t oU, 
                       nullptr, st);
       if (e == cudaSuccess) e = tc_chain(a, heads, st);
     }
+    if (e != cudaSuccess) return cuda_fail(e, "backward: recompute");
   }
-  if (e != cudaSuccess) return cuda_fail(e, "backward: recompute");
   // 2./3. W_t = dO_t^T Q_t (the contraction's U with keys := q, values := dO,
   // beta = 1) and the adjoint chain for G_t (hi/lo pairs): side by side in one
   // launch when the chains fit, the contraction visiting frames in the
@@ -643,6 +650,8 @@ static int scan_bwd(const gdn_bwd_params& p, cudaStream_t st) {
   float* P3 = (float*)(ws + L.P3);
   float* P5 = (float*)(ws + L.P5);
   cudaError_t e;
+  if (p.saved_workspace && !bwd_tc_by_flags(p.D, f))
+    return fail(GDN_ERR_INVALID, "saved_workspace needs the tensor-core backward (bf16, D = 128)%s");
   if (bwd_tc_by_flags(p.D, f)) {
     if (device_cc_major() != 10)
       return fail(GDN_ERR_UNSUPPORTED, "bf16 D = 128 backward runs on sm_100 (else pass GDN_FORCE_SIMT)%s");

@@ -223,7 +223,14 @@ GDN_API int gdn_frame_scan_fwd_static(const void* q, const void* k, const void* 
  *   dA   = -gamma dM,  dgamma = <dM, I - A>,  dU = G,
  *   dk   = beta (K^ (dA + dA^T) + V G) / sqrt(D S),  dv = beta K^ G^T,
  *   dbeta_s = k^_s . (K^ (dA + dA^T) / 2 + V G)_s.
- * Forward quantities (A_t, U_t, the states) are recomputed inside the call.
+ * Forward quantities (A_t, U_t, the states) are recomputed inside the call,
+ * unless saved_workspace is set (tensor-core path: bf16, D = 128): then it
+ * must be the workspace of a gdn_frame_scan_fwd_ex call on the same q, k, v,
+ * beta, gamma, state_in, sizes, GDN_REVERSE / GDN_BLOCK_RESET / block length,
+ * without GDN_BIDIR, GDN_FUSED_PROLOGUE or GDN_FUSED_REPLAY, left untouched
+ * since; the backward reads that call's A_t images and states from it and
+ * skips the recompute (the saved-for-backward pattern of training). Nothing
+ * can check this contract: a stale or foreign workspace gives wrong gradients.
  * Layouts and dtypes as gdn_frame_scan_fwd: d_out, dq, dk, dv like q;
  * dbeta like beta; dgamma like gamma; d_state_out, d_state_in [B,H,D,D] fp32
  * (either may be NULL). Flags: GDN_BF16, GDN_REVERSE, GDN_BLOCK_RESET,
@@ -250,6 +257,7 @@ typedef struct gdn_bwd_params {
   unsigned flags;
   void* workspace;          /* device scratch, 256-byte aligned */
   size_t workspace_bytes;   /* >= gdn_bwd_workspace_bytes(B,H,T,S,D,flags) */
+  const void* saved_workspace; /* NULL, or the forward call's workspace (see above) */
 } gdn_bwd_params;
 
 GDN_API int gdn_frame_scan_bwd(const gdn_bwd_params* p, gdn_stream_t stream);

@@ -118,3 +118,36 @@ def test_backward_bad_arguments_fail_loudly():
     with pytest.raises(api.GdnError):
         api.frame_scan_bwd(d["q"], d["k"], d["v"], d["beta"], d["gamma"], None, d["q"],
                            workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+
+
+@pytest.mark.parametrize("fwd_kw", [dict(), dict(chunked=True), dict(sequential=True, overlap=False),
+                                    dict(reverse=True, block_reset=True)])
+def test_backward_from_saved_forward(fwd_kw):
+    """The backward fed the forward call's workspace (no recompute) equals the
+    recomputing backward and the oracle."""
+    B, H, T, S, D = 1, 3, 9, 200, 128
+    arr = U.random_case(61, B, H, T, S, D, bf16=True, state=True)
+    dO, dS = upstream(62, B, H, T, S, D, True)
+    d = U.dev_inputs(arr, True)
+    d_out, d_s = U.to_dev(dO, True), torch.from_numpy(dS).cuda()
+    ws = torch.empty(api.workspace_bytes(B, H, T, S, D, api.scan_flags(bf16=True, bidir=False)) +
+                     (1 << 20), dtype=torch.uint8, device="cuda")
+    api.frame_scan_fwd_ex(d["q"], d["k"], d["v"], d["beta"], d["gamma"], d["state"],
+                          workspace=ws, **fwd_kw)
+    rkw = dict(reverse=fwd_kw.get("reverse", False), block_reset=fwd_kw.get("block_reset", False))
+    got = api.frame_scan_bwd(d["q"], d["k"], d["v"], d["beta"], d["gamma"], d["state"], d_out,
+                             d_s, saved_workspace=ws, **rkw)
+    ref = api.frame_scan_bwd(d["q"], d["k"], d["v"], d["beta"], d["gamma"], d["state"], d_out,
+                             d_s, **rkw)
+    torch.cuda.synchronize()
+    for name, g, r in zip(NAMES, got, ref):
+        assert rel(U.host(g), U.host(r)) < 2e-3, name
+    block = 3 if rkw["block_reset"] else 0
+    for h in range(H):
+        oref = O.frame_scan_bwd(U.widen(arr["q"][0, h], True), U.widen(arr["k"][0, h], True),
+                                U.widen(arr["v"][0, h], True), arr["beta"][0, h].astype(np.float64),
+                                arr["gamma"][0, h].astype(np.float64), arr["state"][0, h],
+                                U.widen(dO[0, h], True), dS[0, h], reverse=rkw["reverse"],
+                                block=block)
+        for name, g, r in zip(NAMES, got, oref):
+            assert rel(U.host(g[0, h]), r) < U.TOL_BF16, name
