@@ -35,6 +35,7 @@ BIDIR = 0x80
 FUSED_REPLAY = 0x1000000
 CHUNKED = 0x2000000
 NO_OVERLAP = 0x4000000
+REV_STATE_IN = 0x8000000
 
 
 def make_block(n: int) -> int:
@@ -62,6 +63,7 @@ class GdnParams(ctypes.Structure):
         ("D", ctypes.c_int), ("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int),
         ("eps", ctypes.c_float), ("rope_base", ctypes.c_float), ("flags", ctypes.c_uint),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("state_in_rev", ctypes.c_void_p),
     ]
 
 
@@ -183,14 +185,16 @@ def frame_scan_fwd_ex(q, k, v, beta, gamma, state_in=None, *, reverse=False, blo
                       block=3, chunk=8, sequential=False, keys_scaled=False, force_simt=False,
                       prologue=None, bidir=False, fused_replay=False, chunked=False,
                       overlap=True, out=None, state_out=None, out_rev=None, state_out_rev=None,
-                      workspace=None, stream=None):
+                      workspace=None, stream=None, state_in_rev=...):
     """The frame scan through gdn_frame_scan_fwd_ex.
 
     q, k, v [B,H,T,S,D] (bf16 or fp32); beta [B,H,T,S] fp32; gamma [B,H,T]
     fp32; state_in [B,H,D,D] fp32 or None. prologue = dict(w_q, w_k, grid_h,
     grid_w[, eps, rope_base]) applies the fused RMSNorm/ReLU/key-scale/RoPE to
     raw q, k. Returns (out, state_out) or, with bidir, (out, state_out,
-    out_rev, state_out_rev)."""
+    out_rev, state_out_rev). With bidir, state_in_rev (a tensor or None)
+    gives the reverse scan its own start state (GDN_REV_STATE_IN); left out,
+    state_in seeds both directions."""
     B, H, T, S, D = q.shape
     bf16 = q.dtype == torch.bfloat16
     if q.dtype not in (torch.bfloat16, torch.float32):
@@ -219,6 +223,11 @@ def frame_scan_fwd_ex(q, k, v, beta, gamma, state_in=None, *, reverse=False, blo
     p.beta, p.gamma, p.state_in = _ptr(beta), _ptr(gamma), _ptr(state_in)
     p.out, p.state_out = _ptr(out), _ptr(state_out)
     p.out_rev, p.state_out_rev = _ptr(out_rev), _ptr(state_out_rev)
+    if bidir and state_in_rev is not ...:
+        if state_in_rev is not None:
+            _want(state_in_rev, "state_in_rev", torch.float32, (B, H, D, D))
+        p.state_in_rev = _ptr(state_in_rev)
+        flags |= REV_STATE_IN
     if prologue is not None:
         _want(prologue["w_q"], "w_q", torch.float32, (D,))
         _want(prologue["w_k"], "w_k", torch.float32, (D,))

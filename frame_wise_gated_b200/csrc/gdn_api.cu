@@ -187,7 +187,8 @@ static int run_direction(const gdn_params& p, const Layout& L, char* ws, bool re
   a.A = (const float*)(ws + L.A);
   a.U = (const float*)(ws + L.U);
   a.gamma = p.gamma;
-  a.state_in = p.state_in;
+  a.state_in = reverse && (p.flags & GDN_BIDIR) && (p.flags & GDN_REV_STATE_IN) ? p.state_in_rev
+                                                                              : p.state_in;
   a.state_out = state_out;
   a.Sfr = (float*)(ws + sfr_off);
   a.sfr_hilo = use_tc_readout ? 1 : 0;
@@ -380,7 +381,8 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
     if (bidir) {
       // forward never reset; reverse reset per block, run block by block
       o.dir[0] = OvlDir{0, 0, 0, p.state_in, p.state_out, 0};
-      o.dir[1] = OvlDir{1, 1, 0, p.state_in, p.state_out_rev, 0};
+      o.dir[1] = OvlDir{1, 1, 0, (f & GDN_REV_STATE_IN) ? p.state_in_rev : p.state_in,
+                        p.state_out_rev, 0};
     } else {
       o.dir[0] = OvlDir{(f & GDN_REVERSE) ? 1 : 0, 0, block_reset ? 1 : 0, p.state_in,
                         p.state_out, 0};

@@ -60,6 +60,10 @@ CONFIGS = {
                                   prologue=True, bidir_block=3),
     "prologue_bidir_clip5s_720p": Config("prologue_bidir_clip5s_720p", 1, 16, 21, 3600, 128, 45,
                                          80, True, 7, prologue=True, bidir_block=3),
+    # one call of the chunk-causal streaming step: one 3-frame block, forward
+    # state carried in, reverse scan inside the block
+    "stream_block3_720p": Config("stream_block3_720p", 1, 16, 3, 3600, 128, 45, 80, True, 8,
+                                 prologue=True, bidir_block=3, state_sigma=0.1),
     "sweep_d64": Config("sweep_d64", 4, 32, 61, 3600, 64, 45, 80, True, 5,
                         beta_dist="beta22", gamma_lo=0.8, state_sigma=0.1),
     "sweep_d256": Config("sweep_d256", 4, 8, 61, 3600, 256, 45, 80, True, 6,

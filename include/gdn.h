@@ -83,6 +83,8 @@ enum {
 #define GDN_FUSED_REPLAY 0x1000000u /* tensor-core path: replay each span inside the readout
                                        kernel instead of storing S_t (spans/blocks, no prologue) */
 #define GDN_CHUNKED 0x2000000u  /* run the span-composed (chunk-parallel) plan */
+#define GDN_REV_STATE_IN 0x8000000u /* _ex with GDN_BIDIR: the reverse scan starts from
+                                       state_in_rev (NULL = zeros) instead of state_in */
 #define GDN_NO_OVERLAP 0x4000000u /* run the sequential chains as their own launch after
                                      the contraction instead of alongside it */
 #define GDN_BLOCK(f) (((f) >> 8) & 0xffu)  /* reset block length; 0 means 3 */
@@ -171,6 +173,9 @@ typedef struct gdn_params {
   unsigned flags;
   void* workspace;        /* device scratch, 256-byte aligned */
   size_t workspace_bytes; /* >= gdn_workspace_bytes(B,H,T,S,D,flags) */
+  const float* state_in_rev; /* GDN_BIDIR | GDN_REV_STATE_IN: [B,H,D,D] or NULL (zeros);
+                                the chunk-causal streaming step passes the carried
+                                forward state in state_in and no reverse state */
 } gdn_params;
 
 /*
@@ -179,6 +184,10 @@ typedef struct gdn_params {
  * reverse-time scan writes out_rev/state_out_rev; GDN_BLOCK_RESET then applies
  * to the reverse scan only (the chunk-causal variant of the hyper.ai summary,
  * "方法"); A_t and U_t are computed once and shared by both directions.
+ * state_in seeds both directions unless GDN_REV_STATE_IN gives the reverse its
+ * own (state_in_rev). Chunk-causal streaming runs one block of frames per call
+ * (T = block): state_in = the previous call's state_out, GDN_REV_STATE_IN with
+ * state_in_rev = NULL, so each call's reverse scan stays inside its block.
  * Returns GDN_OK or a negative status (GDN_ERR_WORKSPACE if scratch is short).
  */
 GDN_API int gdn_frame_scan_fwd_ex(const gdn_params* p, gdn_stream_t stream);

@@ -160,6 +160,41 @@ def test_plain_entry_allocates_its_own_scratch():
     assert torch.equal(out, out2) and torch.equal(st, st2)
 
 
+def test_chunk_causal_streaming_blocks():
+    """The chunk-causal inference step: one 3-frame block per call, the forward
+    state carried from call to call (state_in = previous state_out), the
+    reverse scan starting from zeros in every call (GDN_REV_STATE_IN with no
+    reverse state). Three calls equal one bidirectional call over 9 frames
+    (reset every 3 in reverse), and the oracle."""
+    gh, gw, T = 6, 5, 9
+    arr = U.random_case(71, 1, 2, T, gh * gw, 128, bf16=True, state=True)
+    d = U.dev_inputs(arr, True)
+    pro = dict(w_q=d["w_q"], w_k=d["w_k"], grid_h=gh, grid_w=gw)
+    o_f, s_f, o_r, _ = run_scan(d, "default", prologue=pro, bidir=True, block_reset=True, block=3,
+                                state_in_rev=None)
+    st = d["state"]
+    parts_f, parts_r = [], []
+    for b0 in range(0, T, 3):
+        sl = {n: d[n][:, :, b0:b0 + 3].contiguous() for n in ("q", "k", "v", "beta", "gamma")}
+        of, st, orr, _ = api.frame_scan_fwd_ex(sl["q"], sl["k"], sl["v"], sl["beta"], sl["gamma"],
+                                               st, prologue=pro, bidir=True, block_reset=True,
+                                               block=3, state_in_rev=None)
+        parts_f.append(of)
+        parts_r.append(orr)
+    torch.cuda.synchronize()
+    gf, gr = torch.cat(parts_f, dim=2), torch.cat(parts_r, dim=2)
+    assert U.rel_frob_per_frame(U.host(gf), U.host(o_f)) < 1e-3
+    assert U.rel_frob_per_frame(U.host(gr), U.host(o_r)) < 1e-3
+    assert U.rel_frob_per_frame(U.host(st)[None], U.host(s_f)[None]) < 1e-4
+    for h in range(2):
+        ref_f, ref_s = U.oracle_slab(arr, 0, h, True, prologue=(gw, 1e-6, 1e4))
+        a0 = dict(arr, state=None)
+        ref_r, _ = U.oracle_slab(a0, 0, h, True, prologue=(gw, 1e-6, 1e4), reverse=True, block=3)
+        assert U.rel_frob_per_frame(U.host(gf[0, h]), ref_f) < U.TOL_BF16
+        assert U.rel_frob_per_frame(U.host(gr[0, h]), ref_r) < U.TOL_BF16
+        assert U.rel_frob_per_frame(U.host(st[0, h])[None], ref_s[None]) < U.TOL_BF16
+
+
 def test_host_streaming_call():
     """frame_scan_fwd_host (host tensors, heads in chunks through ping-pong
     device buffers on three streams) equals the device call head by head, and
