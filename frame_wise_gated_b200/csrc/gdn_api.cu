@@ -363,7 +363,19 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
   // for, or the shape does not fit it.
   const bool bidir = (f & GDN_BIDIR) != 0;
   const int ndir = bidir ? 2 : 1;
-  const bool overlap = tc_contract_ok && tc_chain_ok && tc_readout_ok &&
+  // Few frame-heads (e.g. one 3-frame block per call): cut each frame-head's
+  // tokens over several CTAs (partial sums), then the chains in their own launch.
+  const int nsms = (tc_contract_ok && p.D == 128) ? tc_num_sms() : 0;
+  const int nst = (p.S + 63) / 64;
+  const bool split = tc_contract_ok && tc_chain_ok && tc_readout_ok && p.D == 128 &&
+                     !(f & GDN_FUSED_REPLAY) && frames * 2 <= nsms && nst >= 4;
+  int parts = 1;
+  if (split) {
+    parts = (int)(nsms / frames);
+    if (parts > nst / 2) parts = nst / 2;
+    if (parts > 8) parts = 8;
+  }
+  const bool overlap = !split && tc_contract_ok && tc_chain_ok && tc_readout_ok &&
                        tc_overlap_supported(p.D) && !(f & (GDN_CHUNKED | GDN_NO_OVERLAP |
                                                           GDN_FUSED_REPLAY)) &&
                        (!bidir || (block_reset && tc_readout2_supported(p.D))) &&
@@ -405,7 +417,12 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
   }
   {
     PhaseScope ps(PH_CONTRACT, st);
-    if (tc_contract_ok)
+    if (split) {
+      float* Aacc = (float*)(ws + L.Sfr);  // free until the chains store the states
+      e = tc_contract_split(k, p.v, p.beta, Aacc, U, frames, p.S, (float)(c * c), (float)c, parts,
+                            ppk, st);
+      if (e == cudaSuccess) e = tc_to_image(Aacc, A, frames, p.D, st);
+    } else if (tc_contract_ok)
       e = tc_contract(k, p.v, p.beta, A, U, frames, p.S, p.D, (float)(c * c), (float)c,
                       tc_chain_ok ? 1 : 0, ppk, st);
     else

@@ -178,6 +178,11 @@ bool tc_contract_supported(int D);
 cudaError_t tc_contract(const void* k, const void* v, const float* beta, float* A, float* U,
                         long long N, int S, int D, float cA, float cU, int a_image,
                         const ProArgs* pro, cudaStream_t st);
+// Token-split contraction (D = 128): `parts` CTAs per frame-head add partial
+// A_t, U_t into fp32 Aacc, U (both zeroed here); Aacc still needs tc_to_image.
+cudaError_t tc_contract_split(const void* k, const void* v, const float* beta, float* Aacc,
+                              float* U, long long N, int S, float cA, float cU, int parts,
+                              const ProArgs* pro, cudaStream_t st);
 // fp32 D x D matrices -> operand images (D = 64 or 128).
 cudaError_t tc_to_image(const float* src, void* dst, long long n, int D, cudaStream_t st);
 bool tc_readout_supported(int D);
@@ -219,6 +224,7 @@ struct OvlArgs {
 };
 
 bool tc_overlap_supported(int D);
+int tc_num_sms();
 // Most chains one overlapped launch runs (the rest of the SMs contract).
 int tc_overlap_max_chains();
 // Contraction of all frame-heads (A_t as operand images, U_t fp32) while

@@ -210,7 +210,8 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
                                               const float* __restrict__ beta, float* __restrict__ A,
                                               float* __restrict__ U, int N, int S, float cA,
                                               float cU, int a_image, const ProArgs& pro, int cta,
-                                              int ncta, int heads, int T, int rev, int* flags) {
+                                              int ncta, int heads, int T, int rev, int* flags,
+                                              int parts = 1) {
   using namespace ctr;
   using Ly = Lay<NST>;
   constexpr int OFF_K = Ly::OFF_K, OFF_BK = Ly::OFF_BK, OFF_BETA = Ly::OFF_BETA;
@@ -258,13 +259,19 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const int nst_frame = (S + TOK - 1) / TOK;
-  const int my_count = cta < N ? (N - 1 - cta) / ncta + 1 : 0;
+  // parts > 1: each frame-head's tokens are cut into `parts` stage ranges, one
+  // unit each, whose partial A_t, U_t are added (fp32 atomics) into A, U
+  const int NU = N * parts;
+  const int my_count = cta < NU ? (NU - 1 - cta) / ncta + 1 : 0;
+  const int per_part = (nst_frame + parts - 1) / parts;
   auto unit_n = [&](int i) -> int {
-    const int u = cta + i * ncta;
+    const int u = (cta + i * ncta) / parts;
     if (heads <= 0) return u;
     const int j = u / heads;
     return (u % heads) * T + (rev ? T - 1 - j : j);
   };
+  auto st_begin = [&](int i) -> int { return ((cta + i * ncta) % parts) * per_part; };
+  auto st_end = [&](int i) -> int { return min(st_begin(i) + per_part, nst_frame); };
 
   if (warp == 0) {
     // ---- TMA producer (lane 0 issues; the warp loads beta) ----
@@ -272,7 +279,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
       const int n = unit_n(i);
-      for (int st = 0; st < nst_frame; ++st, ++g) {
+      for (int st = st_begin(i); st < st_end(i); ++st, ++g) {
         const int s = g % NST;
         const uint32_t u = (uint32_t)(g / NST);
         if (lane == 0) ok = mbar_wait(bar_empty + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 1);
@@ -321,7 +328,8 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
         if (!ok) break;
         tc_fence_after();
         const uint32_t dAU = tmem + b * 256;
-        for (int st = 0; st < nst_frame; ++st, ++g) {
+        const int st0 = st_begin(i);
+        for (int st = st0; st < st_end(i); ++st, ++g) {
           const int s = g % NST, kb = g % NBK;
           ok = mbar_wait(bar_bkf + 8 * kb, (uint32_t)(g / NBK) & 1, abort_flag, &g_tc_status, 4);
           if (!ok) break;
@@ -333,7 +341,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
             // operand of four 64-channel blocks
             const uint64_t dkv = smem_desc_sw128(kva + kk * 2048, BOX, 1024);
             const uint64_t db = smem_desc_sw128(ba + kk * 2048, BOX, 1024);
-            const uint32_t acc = (st > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t acc = (st > st0 || kk > 0) ? 1u : 0u;
             mma_bf16(dAU, db, dkv, idesc, acc);
           }
           mma_commit(bar_empty + 8 * s);
@@ -359,7 +367,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
     int g = 0;
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
-      for (int st = 0; st < nst_frame; ++st, ++g) {
+      for (int st = st_begin(i); st < st_end(i); ++st, ++g) {
         const int s = g % NST, kb = g % NBK;
         const uint32_t u = (uint32_t)(g / NST);
         ok = mbar_wait(bar_full + 8 * s, u & 1, abort_flag, &g_tc_status, 6);
@@ -428,7 +436,21 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
           uint32_t r[32];
           tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 256 + half * 128 + c0, r);
           tmem_wait_ld();
-          if (half == 0 && a_image) {
+          if (parts > 1) {
+            // partial sums: row `row` of A_t (fp32, 16-byte atomics); column
+            // `row` of U_t (each warp adds 32 consecutive floats per row)
+            if (half == 0) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                atomicAdd((float4*)(dst + c0 + 4 * j),
+                          make_float4(__uint_as_float(r[4 * j]) * sc, __uint_as_float(r[4 * j + 1]) * sc,
+                                      __uint_as_float(r[4 * j + 2]) * sc, __uint_as_float(r[4 * j + 3]) * sc));
+            } else {
+              float* ucol = U + (size_t)n * D * D + row;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) atomicAdd(ucol + (size_t)(c0 + j) * D, __uint_as_float(r[j]) * sc);
+            }
+          } else if (half == 0 && a_image) {
             // A_t row `row` as the B-operand image (row k = row, columns c0..c0+31)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -490,17 +512,33 @@ template <int NST>
 __global__ void __launch_bounds__(ctr::THREADS, 1)
     k_contract_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const float* __restrict__ beta, float* __restrict__ A, float* __restrict__ U,
-                  int N, int S, float cA, float cU, int a_image, ProArgs pro) {
+                  int N, int S, float cA, float cU, int a_image, ProArgs pro, int parts) {
   contract_body<NST>(tmK, tmV, beta, A, U, N, S, cA, cU, a_image, pro, blockIdx.x, gridDim.x, 0, 0,
-                     0, nullptr);
+                     0, nullptr, parts);
 }
 
 bool tc_contract_supported(int D) { return D == 128 || D == 64 || D == 256; }
+
+// Token-split contraction (D = 128) for problems with few frame-heads: each
+// frame-head's tokens are cut into `parts` ranges on separate CTAs whose
+// partial A_t, U_t are added into the zeroed fp32 Aacc, U (the caller turns
+// Aacc into operand images afterwards).
+static cudaError_t tc_contract128(const void* k, const void* v, const float* beta, float* A,
+                                  float* U, long long N, int S, int D, float cA, float cU,
+                                  int a_image, const ProArgs* pro, cudaStream_t st, int parts);
+cudaError_t tc_contract_split(const void* k, const void* v, const float* beta, float* Aacc,
+                              float* U, long long N, int S, float cA, float cU, int parts,
+                              const ProArgs* pro, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(Aacc, 0, (size_t)N * 128 * 128 * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(U, 0, (size_t)N * 128 * 128 * 4, st);
+  if (e != cudaSuccess) return e;
+  return tc_contract128(k, v, beta, Aacc, U, N, S, 128, cA, cU, 0, pro, st, parts);
+}
 int tc_prologue_max_positions() { return ctr::TAB_MAX / 32; }
 
 static cudaError_t tc_contract128(const void* k, const void* v, const float* beta, float* A,
                                   float* U, long long N, int S, int D, float cA, float cU,
-                                  int a_image, const ProArgs* pro, cudaStream_t st) {
+                                  int a_image, const ProArgs* pro, cudaStream_t st, int parts = 1) {
   if (D != 128) return cudaErrorNotSupported;
   if (pro && pro->npos * (D / 4) > ctr::TAB_MAX) return cudaErrorNotSupported;
   ProArgs pa = {};
@@ -520,13 +558,14 @@ static cudaError_t tc_contract128(const void* k, const void* v, const float* bet
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  const int grid = (int)(N < num_sms() ? N : num_sms());
+  const long long units = N * parts;
+  const int grid = (int)(units < num_sms() ? units : num_sms());
   if (pro)
-    k_contract_tc<ctr::NST_PRO><<<grid, ctr::THREADS, ctr::SMEM_PRO, st>>>(mk, mv, beta, A, U, (int)N,
-                                                                           S, cA, cU, a_image, pa);
+    k_contract_tc<ctr::NST_PRO><<<grid, ctr::THREADS, ctr::SMEM_PRO, st>>>(
+        mk, mv, beta, A, U, (int)N, S, cA, cU, a_image, pa, parts);
   else
     k_contract_tc<ctr::NST_PLAIN><<<grid, ctr::THREADS, ctr::SMEM_PLAIN, st>>>(
-        mk, mv, beta, A, U, (int)N, S, cA, cU, a_image, pa);
+        mk, mv, beta, A, U, (int)N, S, cA, cU, a_image, pa, parts);
   count_launch();
   return cudaGetLastError();
 }
@@ -1964,6 +2003,7 @@ __global__ void __launch_bounds__(ovl::THREADS, 1)
 }
 
 bool tc_overlap_supported(int D) { return D == 128; }
+int tc_num_sms() { return num_sms(); }
 int tc_overlap_max_chains() { return num_sms() / 4; }
 
 cudaError_t tc_contract_scan(const void* k, const void* v, const float* beta, float* A, float* U,
