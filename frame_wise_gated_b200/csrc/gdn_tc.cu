@@ -236,8 +236,8 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
       mbar_init(bar_empty + 8 * s, 1);     // MMA commit
     }
     for (int s = 0; s < NBK; ++s) {
-      mbar_init(bar_bkf + 8 * s, NSC);     // every scaler thread
-      mbar_init(bar_bke + 8 * s, 1);       // MMA commit
+      mbar_init(bar_bkf + 8 * s, NSC / 2);  // every thread of the slot's scaler group
+      mbar_init(bar_bke + 8 * s, 1);        // MMA commit
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_accf + 8 * b, 1);
@@ -357,8 +357,11 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
   } else if (warp < 2 + NSC / 32) {
     // ---- beta * K into the B operand tile (same swizzled layout as K) ----
     const int t = threadIdx.x - 64;
-    // prologue: four threads per token (r = t / 4), 32 channels each
-    const int pr = t >> 2, pc0 = (t & 3) * 32;
+    // The scalers work as two groups of 4 warps on alternate stages (group
+    // g % 2 takes stage g and its beta * K slot), so two stages are in flight.
+    // Prologue: four threads per token, 32 channels each, tokens pr and pr + 32.
+    const int grp = t >> 7, tt = t & 127;
+    const int pr = tt >> 2, pc0 = (tt & 3) * 32;
     float wreg[32];
     if (pro.w) {
 #pragma unroll
@@ -368,6 +371,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
       for (int st = st_begin(i); st < st_end(i); ++st, ++g) {
+        if ((g & 1) != grp) continue;
         const int s = g % NST, kb = g % NBK;
         const uint32_t u = (uint32_t)(g / NST);
         ok = mbar_wait(bar_full + 8 * s, u & 1, abort_flag, &g_tc_status, 6);
@@ -379,24 +383,28 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
         const float* bs = (const float*)(smem + OFF_BETA) + s * TOK;
         if (pro.w) {
           // raw k -> K^ in place (RMSNorm, ReLU, RoPE), then beta * K^
-          const int tok = st * TOK + pr;
-          float f[32];
-          pro_row_part<4>(kt, BOX, pr, pc0, D, tok, tok < S, pro, wreg, tab, f);
-          const float bv = beta ? bs[pr] : 1.f;
-          uint8_t* rowp = bt + (pc0 >> 6) * BOX + pr * 128;
-          const int ch0 = (pc0 & 63) >> 3;
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            *(uint4*)(rowp + (((ch0 + c) ^ (pr & 7)) << 4)) = make_uint4(
-                pack_bf16x2(f[8 * c] * bv, f[8 * c + 1] * bv), pack_bf16x2(f[8 * c + 2] * bv, f[8 * c + 3] * bv),
-                pack_bf16x2(f[8 * c + 4] * bv, f[8 * c + 5] * bv), pack_bf16x2(f[8 * c + 6] * bv, f[8 * c + 7] * bv));
+          for (int half_tok = 0; half_tok < 2; ++half_tok) {
+            const int r = pr + 32 * half_tok;
+            const int tok = st * TOK + r;
+            float f[32];
+            pro_row_part<4>(kt, BOX, r, pc0, D, tok, tok < S, pro, wreg, tab, f);
+            const float bv = beta ? bs[r] : 1.f;
+            uint8_t* rowp = bt + (pc0 >> 6) * BOX + r * 128;
+            const int ch0 = (pc0 & 63) >> 3;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              *(uint4*)(rowp + (((ch0 + c) ^ (r & 7)) << 4)) = make_uint4(
+                  pack_bf16x2(f[8 * c] * bv, f[8 * c + 1] * bv), pack_bf16x2(f[8 * c + 2] * bv, f[8 * c + 3] * bv),
+                  pack_bf16x2(f[8 * c + 4] * bv, f[8 * c + 5] * bv), pack_bf16x2(f[8 * c + 6] * bv, f[8 * c + 7] * bv));
+          }
           fence_proxy_async();
           mbar_arrive(bar_bkf + 8 * kb);
           continue;
         }
 #pragma unroll
-        for (int m = 0; m < 1024 / NSC; ++m) {
-          const int c = t + NSC * m;          // 16-byte chunk of the 16 KiB tile
+        for (int m = 0; m < 1024 / (NSC / 2); ++m) {
+          const int c = tt + (NSC / 2) * m;   // 16-byte chunk of the 16 KiB tile
           const float bv = beta ? bs[(c >> 3) & (TOK - 1)] : 1.f;  // 8 chunks per 128-byte token row
           uint4 x = *(const uint4*)(kt + c * 16);
           uint32_t w[4] = {x.x, x.y, x.z, x.w};
@@ -2803,7 +2811,7 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NQ; ++s) {
       mbar_init(bar_qf + 8 * s, 1);
-      mbar_init(bar_qr + 8 * s, 256);
+      mbar_init(bar_qr + 8 * s, 128);  // the stage's prologue group
       mbar_init(bar_qe + 8 * s, 1);
     }
     mbar_init(bar_sf, 1);
@@ -2844,12 +2852,15 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
                 ok = mbar_wait(bar_se, ((uint32_t)i & 1) ^ 1, abort_flag, &g_tc_status, 81);
         if (!ok) break;
         mbar_arrive_expect_tx(bar_sf, 8 * BOX);
+        // [S_f ; S_r] as one K-major N = 256 operand: per hi / lo half, per
+        // 64-channel block x, the 128 rows of S_f then the 128 rows of S_r
 #pragma unroll
         for (int hl = 0; hl < 2; ++hl)
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
-            tma_load_3d(sb + OFF_SF + (2 * hl + x) * BOX, &tmSF, bar_sf, 64 * x, 0, 2 * n + hl);
-            tma_load_3d(sb + OFF_SR + (2 * hl + x) * BOX, &tmSR, bar_sf, 64 * x, 0, 2 * n + hl);
+            const uint32_t dst = sb + OFF_SF + hl * 4 * BOX + x * 2 * BOX;
+            tma_load_3d(dst, &tmSF, bar_sf, 64 * x, 0, 2 * n + hl);
+            tma_load_3d(dst + BOX, &tmSR, bar_sf, 64 * x, 0, 2 * n + hl);
           }
         for (int tl = tl0; tl < tl1; ++tl, ++g) {
           const int s = g % NQ;
@@ -2869,7 +2880,7 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 256, false, false);
       int g = 0;
       bool ok = true;
       for (int i = 0; i < my_count && ok; ++i) {
@@ -2891,17 +2902,16 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
           if (!ok) break;
           tc_fence_after();
           const uint32_t qa = sb + OFF_Q + s * QT;
+          // [O_f | O_r] = Q [S_f ; S_r]^T: one N = 256 MMA per 16 channels and half
+          const uint32_t d = tmem + b * 256;
+          const uint32_t sh = sb + OFF_SF, sl = sh + 4 * BOX;
 #pragma unroll
-          for (int dir = 0; dir < 2; ++dir) {
-            const uint32_t sh = sb + (dir ? OFF_SR : OFF_SF), sl = sh + 2 * BOX;
-            const uint32_t d = tmem + b * 256 + dir * 128;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * BOX + (kk & 3) * 32;
-              const uint64_t dq = smem_desc_sw128(qa + off, 16, 1024);
-              mma_bf16(d, dq, smem_desc_sw128(sh + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
-              mma_bf16(d, dq, smem_desc_sw128(sl + off, 16, 1024), idesc, 1u);
-            }
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * BOX + (kk & 3) * 32;
+            const uint32_t soff = (kk >> 2) * 2 * BOX + (kk & 3) * 32;
+            const uint64_t dq = smem_desc_sw128(qa + off, 16, 1024);
+            mma_bf16(d, dq, smem_desc_sw128(sh + soff, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+            mma_bf16(d, dq, smem_desc_sw128(sl + soff, 16, 1024), idesc, 1u);
           }
           mma_commit(bar_qe + 8 * s);
           mma_commit(bar_accf + 8 * b);
@@ -2969,8 +2979,11 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
     }
     if (et == 0) bulk_wait0();
   } else if (PRO) {
+    // two groups of 4 warps on alternate Q tiles (group g % 2 owns stage g % 2);
+    // two threads per token, 64 channels each, tokens r and r + 64
     const int t = threadIdx.x - 192;
-    const int r = t >> 1, h = t & 1;
+    const int grp = t >> 7, tt = t & 127;
+    const int r = tt >> 1, h = tt & 1;
     int g = 0;
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
@@ -2979,14 +2992,19 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
       const int tl0 = part * ntile / kParts, tl1 = (part + 1) * ntile / kParts;
       (void)n;
       for (int tl = tl0; tl < tl1; ++tl, ++g) {
+        if ((g & 1) != grp) continue;
         const int s = g % NQ;
         const uint32_t u = (uint32_t)(g / NQ);
         ok = mbar_wait(bar_qf + 8 * s, u & 1, abort_flag, &g_tc_status, 90);
         if (!ok) break;
-        const int tok = tl * TOK + r;
-        float f[64];
-        pro_row_part<8>(smem + OFF_Q + s * QT, BOX, r, 64 * h, D, tok, tok < S, pro,
-                        (const float*)(smem + OFF_W) + 64 * h, pro.cs, f);
+#pragma unroll 1
+        for (int half_tok = 0; half_tok < 2; ++half_tok) {
+          const int row = r + 64 * half_tok;
+          const int tok = tl * TOK + row;
+          float f[64];
+          pro_row_part<8>(smem + OFF_Q + s * QT, BOX, row, 64 * h, D, tok, tok < S, pro,
+                          (const float*)(smem + OFF_W) + 64 * h, pro.cs, f);
+        }
         fence_proxy_async();
         mbar_arrive(bar_qr + 8 * s);
       }
