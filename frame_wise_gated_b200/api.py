@@ -94,6 +94,9 @@ SIGNATURES = {
     "gdn_frame_scan_fwd_static": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _U, _P]),
     "gdn_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _U]),
     "gdn_frame_scan_bwd": (_I, [ctypes.POINTER(GdnBwdParams), _P]),
+    "gdn_cp_shard_composite": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _U, _P,
+                                    ctypes.c_size_t, _P]),
+    "gdn_cp_prefix": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "gdn_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _U]),
     "gdn_frame_contract": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _U, _P]),
     "gdn_chunk_composites": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _U, _P]),
@@ -389,6 +392,45 @@ def frame_scan_bwd(q, k, v, beta, gamma, state_in, d_out, d_state_out=None, *, r
     p.saved_workspace = _ptr(saved_workspace)
     _check(lib().gdn_frame_scan_bwd(ctypes.byref(p), _stream(stream)), "gdn_frame_scan_bwd")
     return dq, dk, dv, dbeta, dgamma, ds0
+
+
+def cp_shard_composite(k, v, beta, gamma, *, keys_scaled=False, force_simt=False,
+                       workspace=None, stream=None):
+    """This rank's frames as one affine map per head (gdn_cp_shard_composite):
+    returns E, H [B,H,D,D] and g [B,H] with S_end = g (S_start - S_start E) + H."""
+    B, H, T, S, D = k.shape
+    _want(v, "v", k.dtype, (B, H, T, S, D))
+    _want(beta, "beta", torch.float32, (B, H, T, S))
+    _want(gamma, "gamma", torch.float32, (B, H, T))
+    flags = scan_flags(bf16=k.dtype == torch.bfloat16, keys_scaled=keys_scaled,
+                       force_simt=force_simt)
+    E = torch.empty((B, H, D, D), device=k.device, dtype=torch.float32)
+    Hm = torch.empty_like(E)
+    g = torch.empty((B, H), device=k.device, dtype=torch.float32)
+    need = workspace_bytes(B, H, T, S, D, flags)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=k.device, dtype=torch.uint8)
+    _check(lib().gdn_cp_shard_composite(_ptr(k), _ptr(v), _ptr(beta), _ptr(gamma), _ptr(E),
+                                        _ptr(Hm), _ptr(g), B, H, T, S, D, flags,
+                                        workspace.data_ptr(),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream(stream)), "gdn_cp_shard_composite")
+    return E, Hm, g
+
+
+def cp_prefix(E_all, H_all, g_all, state_in, r, *, stream=None):
+    """Start state of rank r (gdn_cp_prefix) from the gathered maps
+    E_all, H_all [R,B,H,D,D], g_all [R,B,H]; state_in [B,H,D,D] or None."""
+    R, B, H, D = E_all.shape[0], E_all.shape[1], E_all.shape[2], E_all.shape[3]
+    _want(E_all, "E_all", torch.float32, (R, B, H, D, D))
+    _want(H_all, "H_all", torch.float32, (R, B, H, D, D))
+    _want(g_all, "g_all", torch.float32, (R, B, H))
+    if state_in is not None:
+        _want(state_in, "state_in", torch.float32, (B, H, D, D))
+    out = torch.empty((B, H, D, D), device=E_all.device, dtype=torch.float32)
+    _check(lib().gdn_cp_prefix(_ptr(E_all), _ptr(H_all), _ptr(g_all), _ptr(state_in), _ptr(out),
+                               R, int(r), B * H, D, _stream(stream)), "gdn_cp_prefix")
+    return out
 
 
 STATIC_SCRATCH_BYTES = 32 << 20

@@ -862,6 +862,74 @@ int gdn_frame_contract(const void* k, const void* v, const float* beta, float* A
   return GDN_OK;
 }
 
+int gdn_cp_shard_composite(const void* k, const void* v, const float* beta, const float* gamma,
+                           float* E, float* H, float* g, int B, int Hh, int T, int S, int D,
+                           unsigned flags, void* workspace, size_t workspace_bytes,
+                           gdn_stream_t stream) {
+  t_last_error.clear();
+  int rc = check_sizes(B, Hh, T, S, D);
+  if (rc) return rc;
+  if (!k || !v || !beta || !gamma || !E || !H || !g)
+    return fail(GDN_ERR_INVALID, "null pointer%s");
+  if (flags & ~(GDN_BF16 | GDN_KEYS_SCALED | GDN_FORCE_SIMT | (0xffu << 8) | (0xffu << 16)))
+    return fail(GDN_ERR_INVALID, "gdn_cp_shard_composite: unsupported flag%s");
+  const Layout L = make_layout(B, Hh, T, S, D, flags);
+  if (!workspace || workspace_bytes < L.total)
+    return fail(GDN_ERR_WORKSPACE, "workspace missing or smaller than gdn_workspace_bytes%s");
+  if (((uintptr_t)workspace & 255u) != 0)
+    return fail(GDN_ERR_INVALID, "workspace must be 256-byte aligned%s");
+  cudaStream_t st = (cudaStream_t)stream;
+  const bool bf16 = (flags & GDN_BF16) != 0;
+  const bool simt = (flags & GDN_FORCE_SIMT) || !bf16 || device_cc_major() != 10;
+  const bool tc_chain_ok = !simt && tc_chain_supported(D);  // composes on tensor cores
+  const bool tc_contract_ok = !simt && tc_contract_supported(D);
+  const long long frames = (long long)B * Hh * T;
+  const double c = (flags & GDN_KEYS_SCALED) ? 1.0 : 1.0 / std::sqrt((double)D * (double)S);
+  char* ws = (char*)workspace;
+  float* A = (float*)(ws + L.A);
+  float* U = (float*)(ws + L.U);
+  cudaError_t e;
+  if (tc_contract_ok)
+    e = tc_contract(k, v, beta, A, U, frames, S, D, (float)(c * c), (float)c, tc_chain_ok ? 1 : 0,
+                    nullptr, st);
+  else
+    e = simt_contract(bf16, k, v, beta, A, U, frames, S, D, (float)(c * c), (float)c, st);
+  if (e != cudaSuccess) return cuda_fail(e, "shard composite: contract");
+  ChainArgs a;
+  memset(&a, 0, sizeof(a));
+  a.mode = CHAIN_COMPOSE;
+  a.seg = SEG_CHUNKS;
+  a.D = D;
+  a.T = T;
+  a.L = T;  // one span: the whole shard
+  a.block = 3;
+  a.nseg = 1;
+  a.heads = B * Hh;
+  a.A = A;
+  a.U = U;
+  a.gamma = gamma;
+  a.E = E;
+  a.Hc = H;
+  a.g = g;
+  a.y_image = tc_chain_ok ? 1 : 0;
+  a.e_image = 0;  // E in fp32 for the exchange
+  e = tc_chain_ok ? tc_chain(a, 2 * a.heads, st) : simt_chain(a, 2 * a.heads, st);
+  if (e != cudaSuccess) return cuda_fail(e, "shard composite: compose");
+  return GDN_OK;
+}
+
+int gdn_cp_prefix(const float* E_all, const float* H_all, const float* g_all,
+                  const float* state_in, float* S_start, int R, int r, int heads, int D,
+                  gdn_stream_t stream) {
+  t_last_error.clear();
+  if (R < 1 || r < 0 || r >= R || heads < 1) return fail(GDN_ERR_INVALID, "bad rank or sizes%s");
+  if (!valid_D(D)) return fail(GDN_ERR_UNSUPPORTED, "D must be 16, 32, 64, 128 or 256%s");
+  if (!E_all || !H_all || !g_all || !S_start) return fail(GDN_ERR_INVALID, "null pointer%s");
+  cudaError_t e = simt_cp_prefix(E_all, H_all, g_all, state_in, S_start, r, heads, D,
+                                 (cudaStream_t)stream);
+  return e == cudaSuccess ? GDN_OK : cuda_fail(e, "cp prefix");
+}
+
 int gdn_chunk_composites(const float* A, const float* U, const float* gamma, float* E, float* Hc,
                          float* g, int N, int L, int D, unsigned flags, gdn_stream_t stream) {
   t_last_error.clear();

@@ -131,6 +131,9 @@ cudaError_t simt_contract(bool bf16, const void* k, const void* v, const float* 
                           float* U, long long N, int S, int D, float cA, float cU,
                           cudaStream_t st);
 cudaError_t simt_chain(const ChainArgs& a, int nchains, cudaStream_t st);
+// Context parallelism: start state of shard r from shard-major maps (E, H, g).
+cudaError_t simt_cp_prefix(const float* E, const float* Hc, const float* g, const float* s0,
+                           float* out, int r, int heads, int D, cudaStream_t st);
 cudaError_t simt_readout(bool bf16, const void* q, const float* Sfr, void* out, long long N,
                          int S, int D, cudaStream_t st);
 

@@ -354,6 +354,48 @@ static cudaError_t chain_t(const ChainArgs& a, int nchains, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// Context-parallel prefix: S_start of shard r = state_in folded through the
+// affine maps of shards 0..r-1 (S <- g (S - S E) + H), maps shard-major
+// [R][heads][D][D]. CTA = (head, 16 rows).
+template <int D>
+__global__ void __launch_bounds__(256)
+    k_cp_prefix(const float* __restrict__ E, const float* __restrict__ Hc,
+                const float* __restrict__ g, const float* __restrict__ state_in,
+                float* __restrict__ out, int r, int heads) {
+  extern __shared__ float smem[];
+  float* X = smem;
+  float* Yc = smem + kChainRows * D;
+  const int bh = blockIdx.x, row0 = blockIdx.y * kChainRows;
+  rows_load(X, state_in ? state_in + (size_t)bh * D * D : nullptr, D, row0);
+  for (int p = 0; p < r; ++p) {
+    const size_t si = (size_t)p * heads + bh;
+    chain_step<D>(X, Yc, E + si * D * D, Hc + si * D * D, g[si], row0, false);
+  }
+  rows_store(X, out + (size_t)bh * D * D, D, row0);
+}
+
+template <int D>
+static cudaError_t cp_prefix_t(const float* E, const float* Hc, const float* g, const float* s0,
+                               float* out, int r, int heads, cudaStream_t st) {
+  const size_t smem = 2 * kChainRows * D * sizeof(float);
+  dim3 grid((unsigned)heads, (D + kChainRows - 1) / kChainRows);
+  k_cp_prefix<D><<<grid, 256, smem, st>>>(E, Hc, g, s0, out, r, heads);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t simt_cp_prefix(const float* E, const float* Hc, const float* g, const float* s0,
+                           float* out, int r, int heads, int D, cudaStream_t st) {
+  switch (D) {
+    case 16: return cp_prefix_t<16>(E, Hc, g, s0, out, r, heads, st);
+    case 32: return cp_prefix_t<32>(E, Hc, g, s0, out, r, heads, st);
+    case 64: return cp_prefix_t<64>(E, Hc, g, s0, out, r, heads, st);
+    case 128: return cp_prefix_t<128>(E, Hc, g, s0, out, r, heads, st);
+    case 256: return cp_prefix_t<256>(E, Hc, g, s0, out, r, heads, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 cudaError_t simt_chain(const ChainArgs& a, int nchains, cudaStream_t st) {
   switch (a.D) {
     case 16: return chain_t<16>(a, nchains, st);

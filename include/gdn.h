@@ -299,6 +299,39 @@ GDN_API int gdn_frame_contract(const void* k, const void* v, const float* beta, 
 GDN_API int gdn_chunk_composites(const float* A, const float* U, const float* gamma, float* E, float* Hc,
                          float* g, int N, int L, int D, unsigned flags, gdn_stream_t stream);
 
+/*
+ * Time-sharded context parallelism (SANA-WM blog, Context-Parallel section:
+ * each device holds a span of frames; the span's affine map
+ * S_end = S_start C_p + H_p is exact, so after exchanging the maps every
+ * device knows its exact start state). With R ranks holding consecutive
+ * frame ranges of the same heads (rank order = time order):
+ *   1. gdn_cp_shard_composite on each rank's frames -> E, H, g per head
+ *      (C = g (I - E));
+ *   2. all-gather E, H, g over the ranks (the caller's collective, e.g.
+ *      NCCL): shard-major [R][B*H][D][D], [R][B*H];
+ *   3. gdn_cp_prefix -> this rank's start state;
+ *   4. gdn_frame_scan_fwd(_ex) on the rank's frames with state_in = that
+ *      state; the last rank's state_out is the sequence's.
+ * Forward scan order without block resets.
+ *
+ * gdn_cp_shard_composite: k, v [B,H,T,S,D] (dtype per GDN_BF16), beta
+ * [B,H,T,S], gamma [B,H,T] of this rank's T frames; writes E, H [B,H,D,D]
+ * and g [B,H] (fp32). Scratch: workspace of gdn_workspace_bytes(B,H,T,S,D,
+ * flags). Flags: GDN_BF16, GDN_KEYS_SCALED, GDN_FORCE_SIMT. Returns a status.
+ */
+GDN_API int gdn_cp_shard_composite(const void* k, const void* v, const float* beta,
+                                   const float* gamma, float* E, float* H, float* g, int B,
+                                   int Hh, int T, int S, int D, unsigned flags, void* workspace,
+                                   size_t workspace_bytes, gdn_stream_t stream);
+
+/* gdn_cp_prefix: S_start of rank r = state_in (NULL = zeros) folded through
+ * the maps of ranks 0..r-1: S <- g (S - S E) + H. E_all, H_all
+ * [R][heads][D][D], g_all [R][heads] fp32 (shard-major, as gathered);
+ * state_in, S_start [heads][D][D] fp32. Returns a status. */
+GDN_API int gdn_cp_prefix(const float* E_all, const float* H_all, const float* g_all,
+                          const float* state_in, float* S_start, int R, int r, int heads, int D,
+                          gdn_stream_t stream);
+
 /* Synchronises `stream`, then reads and clears the library's device status
  * word: GDN_OK, GDN_ERR_TIMEOUT if a kernel's bounded wait expired since the
  * last check, or GDN_ERR_CUDA if the stream reports an error. */
