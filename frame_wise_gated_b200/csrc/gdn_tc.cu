@@ -3268,6 +3268,13 @@ __global__ void __launch_bounds__(c256::THREADS, 1)
               *(uint4*)(img + off) = hi;
               *(uint4*)(img + off + 8192) = lo;
             }
+          } else if (mat == 1 && a_image) {
+            // U_t transposed for the D = 256 chains (their epilogue reads a
+            // column of U^T per row, 32 rows per warp: coalesced); each warp
+            // here writes 32 consecutive floats of a row of U^T
+            float* ut = U + (size_t)n * D * D + k;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ut[(size_t)(c0 + j) * D] = __uint_as_float(r[j]) * sc;
           } else {
 #pragma unroll
             for (int j = 0; j < 8; ++j)
@@ -3538,7 +3545,8 @@ static cudaError_t tc_readout256(const void* q, const void* Sfr_hilo, void* out,
 // next to P (columns 256..511). Eight epilogue warps read P and X, apply
 // X <- gamma (X - P) + U_t with U_t read from global memory (L2), write X
 // back to TMEM and, as a bf16 (hi, lo) pair, into the operand tile, which one
-// thread then stores by TMA as the frame's state for the readout.
+// thread then stores by TMA as the frame's state for the readout. U_t comes
+// transposed from the contraction, so those reads coalesce.
 //
 // Operand image of a 256 x 256 matrix M (written by the contraction): 16
 // slices of 16 rows k; slice s holds bf16(M) then bf16(M - bf16(M)) for rows
@@ -3622,7 +3630,7 @@ __global__ void __launch_bounds__(ch2::THREADS, 1)
         if (s + 1 < g.n) {
           const ChainStep nx = chain_step_at(a, g, s + 1);
           prefetch_l2(nx.Y, (uint32_t)IMG);
-          prefetch_l2(nx.Z + (size_t)half * 128 * D, (uint32_t)(IMG / 2));
+          prefetch_l2(nx.Z, (uint32_t)IMG);
         }
         for (int sl = 0; sl < NSLICE; ++sl, ++gi) {
           const int slot = gi % NSY;
@@ -3685,13 +3693,12 @@ __global__ void __launch_bounds__(ch2::THREADS, 1)
     const bool store_sfr = g.mode == CHAIN_SCAN;
     int nstore = 0;
     float zb[2][32];
+    // Z = U_t stored transposed: element (grow, col) at Z[col * D + grow], so
+    // the warp's 32 rows read 128 contiguous bytes per column
     auto load_z = [&](const float* Z, int c, float* z) {
-      const float* src = Z + grow * D + 128 * ch + 32 * c;
+      const float* src = Z + (size_t)(128 * ch + 32 * c) * D + grow;
 #pragma unroll
-      for (int i = 0; i < 32; i += 4) {
-        const float4 f = __ldg((const float4*)(src + i));
-        z[i] = f.x; z[i + 1] = f.y; z[i + 2] = f.z; z[i + 3] = f.w;
-      }
+      for (int i = 0; i < 32; ++i) z[i] = __ldg(src + (size_t)i * D);
     };
     // the X tile (bf16 hi, lo) for columns 128 ch + 32 c .. +31 of this row
     auto put_x = [&](const float* x, int c) {
