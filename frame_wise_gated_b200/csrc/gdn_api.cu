@@ -336,8 +336,8 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
         e = rope_table(cs, npos, p.D, base, st);
       }
       if (e != cudaSuccess) return cuda_fail(e, "rope table");
-      pro_k = ProArgs{p.w_k, cs, p.grid_w, eps, npos};
-      pro_q = ProArgs{p.w_q, cs, p.grid_w, eps, npos};
+      pro_k = ProArgs{p.w_k, cs, p.grid_w, eps, npos, base};
+      pro_q = ProArgs{p.w_q, cs, p.grid_w, eps, npos, base};
       ppk = &pro_k;
       ppq = &pro_q;
     } else {

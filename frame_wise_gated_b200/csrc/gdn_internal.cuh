@@ -170,6 +170,7 @@ struct ProArgs {
   int grid_w;
   float eps;
   int npos;
+  float base;        // RoPE base (pair i turns by pos * base^(-2i/(D/2)))
 };
 // (cos, sin) table, pair-major: cs[i * npos + pos], pos < npos, i < D/4
 // (consecutive tokens of a row read consecutive entries).

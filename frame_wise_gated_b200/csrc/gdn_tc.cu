@@ -100,10 +100,16 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // token; inside its half (y for channels < 64, x above) that is pair index
 // (c0 % 64)/2 + p of the (cos, sin) table row of the token's position.
 // ----------------------------------------------------------------------------
+// With `theta` (shared memory, the D/4 pair frequencies) the (cos, sin) of
+// each pair's angle pos * theta_i are computed here instead of read from the
+// table: the angle is reduced to [-pi, pi] (2 pi split in two parts) and
+// evaluated with the hardware sine/cosine, whose error on that range is near
+// 1e-6 -- below the bf16 rounding the result gets.
 template <int NCH>
 __device__ __forceinline__ void pro_row_part(uint8_t* tile, int box_bytes, int r, int c0, int D,
                                              int tok, bool valid, const ProArgs& pro,
-                                             const float* w, const float2* tab, float* f) {
+                                             const float* w, const float2* tab, float* f,
+                                             const float* theta = nullptr) {
   const int box = c0 >> 6, ch0 = (c0 & 63) >> 3;
   uint8_t* rowp = tile + box * box_bytes + r * 128;
   float ssp[4] = {0.f, 0.f, 0.f, 0.f};
@@ -125,11 +131,21 @@ __device__ __forceinline__ void pro_row_part(uint8_t* tile, int box_bytes, int r
   const float inv = 1.0f / sqrtf(ss / (float)D + pro.eps);
   const int pos = valid ? (box ? tok % pro.grid_w : tok / pro.grid_w) : 0;
   const float2* cs = tab + ((c0 & 63) >> 1) * pro.npos + pos;
+  const float* th = theta ? theta + ((c0 & 63) >> 1) : nullptr;
 #pragma unroll
   for (int j = 0; j < 4 * NCH; ++j) {
     const float a = fmaxf(f[2 * j] * w[2 * j], 0.f);
     const float b = fmaxf(f[2 * j + 1] * w[2 * j + 1], 0.f);
-    const float2 t = cs[j * pro.npos];
+    float2 t;
+    if (th) {
+      float ang = (float)pos * th[j];
+      const float kq = rintf(ang * 0.159154943091895f);  // 1 / (2 pi)
+      ang = fmaf(-kq, 6.28318548202514648f, ang);        // 2 pi, high part
+      ang = fmaf(-kq, -1.7484555314695172e-7f, ang);     // 2 pi, low part
+      __sincosf(ang, &t.y, &t.x);
+    } else {
+      t = cs[j * pro.npos];
+    }
     f[2 * j] = inv * (a * t.x - b * t.y);
     f[2 * j + 1] = inv * (a * t.y + b * t.x);
   }
@@ -2779,10 +2795,12 @@ constexpr int OFF_SF = OFF_Q + NQ * QT;  // forward state: hi (2 boxes), lo (2 b
 constexpr int OFF_SR = OFF_SF + 4 * BOX; // reverse state
 constexpr int OFF_O = OFF_SR + 4 * BOX;  // two staging boxes
 constexpr int OFF_W = OFF_O + 2 * BOX;   // prologue weights
-constexpr int OFF_BAR = OFF_W + D * 4;
+constexpr int OFF_TH = OFF_W + D * 4;    // prologue pair frequencies [D/4]
+constexpr int OFF_BAR = OFF_TH + (D / 4) * 4;
 constexpr int NBAR = 3 * NQ + 2 + 4 + 1;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM = OFF_MISC + 16 + 1024;
+static_assert(SMEM <= 232448, "bidirectional readout shared memory");
 constexpr int threads(bool pro) { return pro ? 448 : 192; }
 constexpr uint32_t TMEM_COLS = 512;
 }  // namespace rd2
@@ -2825,6 +2843,8 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
     fence_mbar_init();
   }
   if (PRO && threadIdx.x < D) ((float*)(smem + OFF_W))[threadIdx.x] = pro.w[threadIdx.x];
+  if (PRO && threadIdx.x < D / 4)  // pair frequencies, as the (cos, sin) table has them
+    ((float*)(smem + OFF_TH))[threadIdx.x] = powf(pro.base, -2.0f * (float)threadIdx.x / (float)(D / 2));
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
     tmem_relinquish();
@@ -3003,7 +3023,8 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
           const int tok = tl * TOK + row;
           float f[64];
           pro_row_part<8>(smem + OFF_Q + s * QT, BOX, row, 64 * h, D, tok, tok < S, pro,
-                          (const float*)(smem + OFF_W) + 64 * h, pro.cs, f);
+                          (const float*)(smem + OFF_W) + 64 * h, pro.cs, f,
+                          (const float*)(smem + OFF_TH));
         }
         fence_proxy_async();
         mbar_arrive(bar_qr + 8 * s);
