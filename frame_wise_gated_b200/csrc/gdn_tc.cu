@@ -88,72 +88,147 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 
 // ----------------------------------------------------------------------------
 // Prologue inside the loaders (SANA-WM blog, Context-Parallel section: the
-// fused op runs RMSNorm -> ReLU -> key scale -> RoPE ahead of the scan). A
-// group of 16 / NCH threads (consecutive lanes) handles one token row of a
-// tile made of two [rows][64] bf16 boxes with the 128-byte swizzle; each
-// thread owns NCH 16-byte chunks (8 * NCH channels starting at channel c0) and
-// the group combines its sums of squares. Since the RMSNorm factor
-// inv = 1/sqrt(mean(x^2) + eps) is positive and RoPE is linear,
+// fused op runs RMSNorm -> ReLU -> key scale -> RoPE ahead of the scan), D = 128.
+// Each thread takes NR token rows rr[] of a tile made of two [rows][64] bf16
+// boxes with the 128-byte swizzle, and in each row the 32 channels of its
+// quarter q (channels 32q .. 32q + 31: four 16-byte chunks); the four threads
+// that share a row (consecutive lanes) combine their sums of squares. With
+// NR = 2 the rows run side by side so that the latency of one (shared-memory
+// loads, shuffles, rsqrt) overlaps the arithmetic of the other. Since the RMSNorm
+// factor inv = 1/sqrt(mean(x^2) + eps) is positive and RoPE is linear,
 //     RoPE(max(x * inv * w, 0)) = inv * RoPE(max(x * w, 0)),
-// which saves a multiply per element. The row is written back in place and
-// returned in f (fp32). Pair p of the thread is channel pair c0/2 + p of the
-// token; inside its half (y for channels < 64, x above) that is pair index
-// (c0 % 64)/2 + p of the (cos, sin) table row of the token's position.
+// so inv scales the rotated pair. The rows are written back in place; with
+// `btile`, bv[k] * row k also goes to `btile` (same layout).
+//
+// Weights come from shared memory laid out by pro_w_copy: w4[p * 4 + q] =
+// (w[32q + 2p], w[32q + 2p + 1]), so the four quarters' threads of a warp read
+// 32 adjacent bytes. RoPE: pair i of a half (i < 32) turns by pos * theta_i,
+// pos the token's row (channels below 64) or column (above). With `theta`
+// (shared memory, the 32 frequencies) the (cos, sin) is computed: the angle
+// is reduced to [-pi, pi] (2 pi split in two parts) and evaluated with the
+// hardware sine/cosine, whose error on that range is near 1e-6 -- below the
+// bf16 rounding the result gets. Otherwise it is read from `tab`, a shared
+// copy of the table laid out by pro_table_index.
 // ----------------------------------------------------------------------------
-// With `theta` (shared memory, the D/4 pair frequencies) the (cos, sin) of
-// each pair's angle pos * theta_i are computed here instead of read from the
-// table: the angle is reduced to [-pi, pi] (2 pi split in two parts) and
-// evaluated with the hardware sine/cosine, whose error on that range is near
-// 1e-6 -- below the bf16 rounding the result gets.
-template <int NCH>
-__device__ __forceinline__ void pro_row_part(uint8_t* tile, int box_bytes, int r, int c0, int D,
-                                             int tok, bool valid, const ProArgs& pro,
-                                             const float* w, const float2* tab, float* f,
-                                             const float* theta = nullptr) {
-  const int box = c0 >> 6, ch0 = (c0 & 63) >> 3;
-  uint8_t* rowp = tile + box * box_bytes + r * 128;
-  float ssp[4] = {0.f, 0.f, 0.f, 0.f};
+constexpr int PRO_POS_PITCH = 80;  // positions per pair in the shared table (the most supported)
+__device__ __forceinline__ int pro_table_index(int i, int pos) {
+  // pairs i and i + 16 of one position are neighbours, positions of one pair
+  // are consecutive: the threads of a warp (8 tokens x 4 quarters) read
+  // 16 consecutive entries in the column half and 2 in the row half. The
+  // fixed pitch makes the pair offsets compile-time constants.
+  return (((i & 15) * PRO_POS_PITCH + pos) << 1) + (i >> 4);
+}
+
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+template <int NR>
+__device__ __forceinline__ void pro_rows(uint8_t* tile, int box_bytes, const int (&rr)[NR], int q,
+                                         const int (&tk)[NR], int S, const ProArgs& pro,
+                                         const float2* w4, const float2* tab, const float* theta,
+                                         uint8_t* btile, const float (&bv)[NR]) {
+  constexpr int D = 128, NW = 16;  // channel pairs (packed words) per thread row
+  const int box = q >> 1, ch0 = (q & 1) * 4, pb = (q & 1) * 16;
+  uint32_t u[NR][NW];
 #pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    const uint4 v = *(const uint4*)(rowp + (((ch0 + c) ^ (r & 7)) << 4));
-    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+  for (int k = 0; k < NR; ++k)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 v = *(const uint4*)(tile + box * box_bytes + rr[k] * 128 +
+                                      (((ch0 + c) ^ (rr[k] & 7)) << 4));
+      u[k][4 * c] = v.x;
+      u[k][4 * c + 1] = v.y;
+      u[k][4 * c + 2] = v.z;
+      u[k][4 * c + 3] = v.w;
+    }
+  float inv[NR], scb[NR];
+  int pos[NR];
+  const float2* trow[NR];  // table entries of the rows' positions (pair pb + p at p * 2 * pitch)
+  {
+    float2 acc[NR][2];
+#pragma unroll
+    for (int k = 0; k < NR; ++k) acc[k][0] = acc[k][1] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int e = 0; e < NW; ++e)
+#pragma unroll
+      for (int k = 0; k < NR; ++k) {
+        const float2 x = unpack_bf16x2(u[k][e]);
+        acc[k][e & 1] = __ffma2_rn(x, x, acc[k][e & 1]);
+      }
+    float ss[NR];
+#pragma unroll
+    for (int k = 0; k < NR; ++k) ss[k] = (acc[k][0].x + acc[k][0].y) + (acc[k][1].x + acc[k][1].y);
+#pragma unroll
+    for (int o = 1; o < 4; o <<= 1) {
+      float sh[NR];
+#pragma unroll
+      for (int k = 0; k < NR; ++k) sh[k] = __shfl_xor_sync(0xffffffffu, ss[k], o);
+#pragma unroll
+      for (int k = 0; k < NR; ++k) ss[k] += sh[k];
+    }
+#pragma unroll
+    for (int k = 0; k < NR; ++k) {
+      inv[k] = rsqrtf(fmaf(ss[k], 1.0f / (float)D, pro.eps));
+      scb[k] = inv[k] * bv[k];
+      pos[k] = tk[k] < S ? (box ? tk[k] % pro.grid_w : tk[k] / pro.grid_w) : 0;
+      trow[k] = tab + pro_table_index(pb, pos[k]);
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t ob[NR][4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wd[e]));
-      f[8 * c + 2 * e] = x.x;
-      f[8 * c + 2 * e + 1] = x.y;
-      ssp[e] = fmaf(x.x, x.x, fmaf(x.y, x.y, ssp[e]));
+      const int p = 4 * c + e;  // pair p of the thread: pair pb + p of its half
+      const float2 w2 = w4[p * 4 + q];
+#pragma unroll
+      for (int k = 0; k < NR; ++k) {
+        const float2 m = __fmul2_rn(unpack_bf16x2(u[k][p]), w2);
+        const float a = fmaxf(m.x, 0.f), b = fmaxf(m.y, 0.f);
+        float2 t;
+        if (theta) {
+          float ang = (float)pos[k] * theta[pb + p];
+          const float kq = rintf(ang * 0.159154943091895f);  // 1 / (2 pi)
+          ang = fmaf(-kq, 6.28318548202514648f, ang);        // 2 pi, high part
+          ang = fmaf(-kq, -1.7484555314695172e-7f, ang);     // 2 pi, low part
+          __sincosf(ang, &t.y, &t.x);
+        } else {
+          t = trow[k][p * 2 * PRO_POS_PITCH];
+        }
+        const float2 o = make_float2(a * t.x - b * t.y, a * t.y + b * t.x);
+        const float2 kh = __fmul2_rn(o, make_float2(inv[k], inv[k]));
+        u[k][p] = pack_bf16x2(kh.x, kh.y);
+        if (btile) {
+          const float2 bk = __fmul2_rn(o, make_float2(scb[k], scb[k]));
+          ob[k][e] = pack_bf16x2(bk.x, bk.y);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < NR; ++k) {
+      const int off = box * box_bytes + rr[k] * 128 + (((ch0 + c) ^ (rr[k] & 7)) << 4);
+      *(uint4*)(tile + off) = make_uint4(u[k][4 * c], u[k][4 * c + 1], u[k][4 * c + 2], u[k][4 * c + 3]);
+      if (btile) *(uint4*)(btile + off) = make_uint4(ob[k][0], ob[k][1], ob[k][2], ob[k][3]);
     }
   }
-  float ss = (ssp[0] + ssp[1]) + (ssp[2] + ssp[3]);
-#pragma unroll
-  for (int o = 1; o < 16 / NCH; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  const float inv = 1.0f / sqrtf(ss / (float)D + pro.eps);
-  const int pos = valid ? (box ? tok % pro.grid_w : tok / pro.grid_w) : 0;
-  const float2* cs = tab + ((c0 & 63) >> 1) * pro.npos + pos;
-  const float* th = theta ? theta + ((c0 & 63) >> 1) : nullptr;
-#pragma unroll
-  for (int j = 0; j < 4 * NCH; ++j) {
-    const float a = fmaxf(f[2 * j] * w[2 * j], 0.f);
-    const float b = fmaxf(f[2 * j + 1] * w[2 * j + 1], 0.f);
-    float2 t;
-    if (th) {
-      float ang = (float)pos * th[j];
-      const float kq = rintf(ang * 0.159154943091895f);  // 1 / (2 pi)
-      ang = fmaf(-kq, 6.28318548202514648f, ang);        // 2 pi, high part
-      ang = fmaf(-kq, -1.7484555314695172e-7f, ang);     // 2 pi, low part
-      __sincosf(ang, &t.y, &t.x);
-    } else {
-      t = cs[j * pro.npos];
-    }
-    f[2 * j] = inv * (a * t.x - b * t.y);
-    f[2 * j + 1] = inv * (a * t.y + b * t.x);
+}
+
+// Copies the (cos, sin) table (pair-major, cs[i * npos + pos]) into shared
+// memory in pro_table_index order.
+__device__ __forceinline__ void pro_table_copy(float2* tab, const ProArgs& pro) {
+  for (int e = threadIdx.x; e < pro.npos * 32; e += (int)blockDim.x) {
+    const int i = e / pro.npos, pos = e - i * pro.npos;
+    tab[pro_table_index(i, pos)] = pro.cs[e];
   }
-#pragma unroll
-  for (int c = 0; c < NCH; ++c)
-    *(uint4*)(rowp + (((ch0 + c) ^ (r & 7)) << 4)) =
-        make_uint4(pack_bf16x2(f[8 * c], f[8 * c + 1]), pack_bf16x2(f[8 * c + 2], f[8 * c + 3]),
-                   pack_bf16x2(f[8 * c + 4], f[8 * c + 5]), pack_bf16x2(f[8 * c + 6], f[8 * c + 7]));
+}
+
+// Copies the RMSNorm weights w[128] into shared memory in pro_rows' order.
+__device__ __forceinline__ void pro_w_copy(float2* w4, const float* w) {
+  for (int e = threadIdx.x; e < 64; e += (int)blockDim.x) {
+    const int p = e & 15, q = e >> 4;
+    w4[p * 4 + q] = make_float2(w[32 * q + 2 * p], w[32 * q + 2 * p + 1]);
+  }
 }
 
 // (cos, sin) of pos * base^(-2i/(D/2)) for pos < npos, i < D/4, at cs[i * npos + pos].
@@ -183,15 +258,19 @@ constexpr int D = 128;
 constexpr int TOK = 64;                 // tokens per stage
 constexpr int BOX = TOK * 128;          // one [64 tokens][64 channels] bf16 box: 8 KiB
 constexpr int TILE = 2 * BOX;           // one tensor's stage tile: 16 KiB
-constexpr int NBK = 2;                  // beta * K slots (the MMA's B operand)
-constexpr int TAB_MAX = 80 * 32;        // prologue table entries: positions x pairs (D/4 = 32)
+constexpr int TAB_MAX = PRO_POS_PITCH * 32;  // prologue table entries: positions x pairs (D/4 = 32)
 constexpr int NSC = 256;                // scaler threads (8 warps)
 constexpr int THREADS = 64 + NSC + 128;  // producer, MMA, 8 scaler warps, 4 epilogue warps
 constexpr uint32_t TMEM_COLS = 512;
-// Shared-memory layout for an NST-stage K/V ring (deepest that fits: 6
-// stages without the prologue's (cos, sin) table, 5 with it).
+constexpr int NST_PLAIN = 6;
+constexpr int NST_PRO = 4;
+// Shared-memory layout for an NST-stage K/V ring: 6 stages and 2 beta * K
+// slots without the prologue; with it, 4 stages, 4 slots and the (cos, sin)
+// table. The two scaler groups take alternate stages, so with 4 slots a group
+// starts its next stage while the MMAs of its last one still read their slot.
 template <int NST>
 struct Lay {
+  static constexpr int NBK = NST == NST_PRO ? 4 : 2;  // beta * K slots (the MMA's B operand)
   static constexpr int OFF_K = 0;                     // stage s: K at s * 2 TILE, V after it
   static constexpr int OFF_BK = OFF_K + NST * 2 * TILE;
   static constexpr int OFF_BETA = OFF_BK + NBK * TILE;
@@ -201,10 +280,9 @@ struct Lay {
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_TAB = OFF_MISC + 16;
   static constexpr int SMEM_PLAIN = OFF_TAB + 1024;
-  static constexpr int SMEM_PRO = OFF_TAB + TAB_MAX * 8 + 1024;
+  static constexpr int OFF_W4 = OFF_TAB + TAB_MAX * 8;  // prologue weights (pro_w_copy order)
+  static constexpr int SMEM_PRO = OFF_W4 + 512 + 1024;
 };
-constexpr int NST_PLAIN = 6;
-constexpr int NST_PRO = 5;
 constexpr int SMEM_PLAIN = Lay<NST_PLAIN>::SMEM_PLAIN;
 constexpr int SMEM_PRO = Lay<NST_PRO>::SMEM_PRO;
 static_assert(SMEM_PLAIN <= 232448 && SMEM_PRO <= 232448, "contraction shared memory");
@@ -230,6 +308,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
                                               int parts = 1) {
   using namespace ctr;
   using Ly = Lay<NST>;
+  constexpr int NBK = Ly::NBK;
   constexpr int OFF_K = Ly::OFF_K, OFF_BK = Ly::OFF_BK, OFF_BETA = Ly::OFF_BETA;
   constexpr int OFF_MISC = Ly::OFF_MISC, OFF_TAB = Ly::OFF_TAB;
   extern __shared__ uint8_t smem_raw[];
@@ -264,8 +343,11 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
     fence_mbar_init();
   }
   float2* tab = (float2*)(smem + OFF_TAB);
-  if (pro.w)
-    for (int e = threadIdx.x; e < pro.npos * (D / 4); e += (int)blockDim.x) tab[e] = pro.cs[e];
+  float2* w4 = (float2*)(smem + Ly::OFF_W4);
+  if (pro.w) {
+    pro_table_copy(tab, pro);
+    pro_w_copy(w4, pro.w);
+  }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
     tmem_relinquish();
@@ -375,14 +457,9 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
     const int t = threadIdx.x - 64;
     // The scalers work as two groups of 4 warps on alternate stages (group
     // g % 2 takes stage g and its beta * K slot), so two stages are in flight.
-    // Prologue: four threads per token, 32 channels each, tokens pr and pr + 32.
+    // Prologue: four threads per token (32 channels each), tokens pr and pr + 32.
     const int grp = t >> 7, tt = t & 127;
-    const int pr = tt >> 2, pc0 = (tt & 3) * 32;
-    float wreg[32];
-    if (pro.w) {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) wreg[j] = __ldg(pro.w + pc0 + j);
-    }
+    const int pr = tt >> 2, pq = tt & 3;
     int g = 0;
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
@@ -398,22 +475,10 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
         uint8_t* bt = smem + OFF_BK + kb * TILE;
         const float* bs = (const float*)(smem + OFF_BETA) + s * TOK;
         if (pro.w) {
-          // raw k -> K^ in place (RMSNorm, ReLU, RoPE), then beta * K^
-#pragma unroll
-          for (int half_tok = 0; half_tok < 2; ++half_tok) {
-            const int r = pr + 32 * half_tok;
-            const int tok = st * TOK + r;
-            float f[32];
-            pro_row_part<4>(kt, BOX, r, pc0, D, tok, tok < S, pro, wreg, tab, f);
-            const float bv = beta ? bs[r] : 1.f;
-            uint8_t* rowp = bt + (pc0 >> 6) * BOX + r * 128;
-            const int ch0 = (pc0 & 63) >> 3;
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-              *(uint4*)(rowp + (((ch0 + c) ^ (r & 7)) << 4)) = make_uint4(
-                  pack_bf16x2(f[8 * c] * bv, f[8 * c + 1] * bv), pack_bf16x2(f[8 * c + 2] * bv, f[8 * c + 3] * bv),
-                  pack_bf16x2(f[8 * c + 4] * bv, f[8 * c + 5] * bv), pack_bf16x2(f[8 * c + 6] * bv, f[8 * c + 7] * bv));
-          }
+          // raw k -> K^ in place (RMSNorm, ReLU, RoPE) and beta * K^ into the slot
+          const int rr[2] = {pr, pr + 32}, tk[2] = {st * TOK + pr, st * TOK + pr + 32};
+          const float bv[2] = {beta ? bs[pr] : 1.f, beta ? bs[pr + 32] : 1.f};
+          pro_rows<2>(kt, BOX, rr, pq, tk, S, pro, w4, tab, nullptr, bt, bv);
           fence_proxy_async();
           mbar_arrive(bar_bkf + 8 * kb);
           continue;
@@ -609,10 +674,10 @@ constexpr int OFF_O = OFF_S + 4 * BOX;  // output staging, 2 boxes: 32 KiB
 constexpr int OFF_BAR = OFF_O + 2 * BOX;
 constexpr int NBAR = 3 * NQ + 2 + 4 + 1;  // q_full, q_ready, q_empty, s_full, s_empty, acc f/e x2, fin
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr int OFF_W = OFF_MISC + 16;    // prologue weights [D] fp32
-constexpr int OFF_TAB = OFF_W + D * 4;  // prologue (cos, sin) table copy
-constexpr int TAB_MAX = 80 * 32;
-constexpr int SMEM = OFF_TAB + TAB_MAX * 8 + 1024;
+constexpr int OFF_TAB = OFF_MISC + 16;  // prologue (cos, sin) table copy
+constexpr int TAB_MAX = PRO_POS_PITCH * 32;
+constexpr int OFF_W4 = OFF_TAB + TAB_MAX * 8;  // prologue weights (pro_w_copy order)
+constexpr int SMEM = OFF_W4 + 512 + 1024;
 // producer, MMA, 4 epilogue warps (+ 8 warps applying the prologue to Q tiles)
 constexpr int threads(bool pro) { return pro ? 448 : 192; }
 constexpr uint32_t TMEM_COLS = 256;
@@ -656,10 +721,10 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (PRO && threadIdx.x < D) ((float*)(smem + OFF_W))[threadIdx.x] = pro.w[threadIdx.x];
-  if (PRO)
-    for (int e = threadIdx.x; e < pro.npos * (D / 4); e += (int)blockDim.x)
-      ((float2*)(smem + OFF_TAB))[e] = pro.cs[e];
+  if (PRO) {
+    pro_table_copy((float2*)(smem + OFF_TAB), pro);
+    pro_w_copy((float2*)(smem + OFF_W4), pro.w);
+  }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
     tmem_relinquish();
@@ -814,9 +879,10 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
     }
     if (et == 0) bulk_wait0();
   } else if (PRO) {
-    // ---- prologue on each raw Q tile, in place (two threads per token) ----
+    // ---- prologue on each raw Q tile, in place: four threads per token
+    // (32 channels each), tokens pr and pr + 64 ----
     const int t = threadIdx.x - 192;
-    const int r = t >> 1, h = t & 1;
+    const int pr = t >> 2, pq = t & 3;
     int g = 0;
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
@@ -829,10 +895,10 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
         const uint32_t u = (uint32_t)(g / NQ);
         ok = mbar_wait(bar_qf + 8 * s, u & 1, abort_flag, &g_tc_status, 20);
         if (!ok) break;
-        const int tok = tl * TOK + r;
-        float f[64];
-        pro_row_part<8>(smem + OFF_Q + s * QT, BOX, r, 64 * h, D, tok, tok < S, pro,
-                        (const float*)(smem + OFF_W) + 64 * h, (const float2*)(smem + OFF_TAB), f);
+        const int rr[2] = {pr, pr + 64}, tk[2] = {tl * TOK + pr, tl * TOK + pr + 64};
+        const float bv[2] = {1.f, 1.f};
+        pro_rows<2>(smem + OFF_Q + s * QT, BOX, rr, pq, tk, S, pro, (const float2*)(smem + OFF_W4),
+                    (const float2*)(smem + OFF_TAB), nullptr, nullptr, bv);
         fence_proxy_async();
         mbar_arrive(bar_qr + 8 * s);
       }
@@ -2782,7 +2848,8 @@ static cudaError_t tc_chain64(const ChainArgs& a, int nchains, cudaStream_t st) 
 //   O_fwd = Q S_fwd_hi^T + Q S_fwd_lo^T,   O_rev = Q S_rev_hi^T + Q S_rev_lo^T
 // (four fp32 TMEM accumulators: two tiles in flight x two directions). Both
 // outputs leave through two 16 KiB swizzled staging buffers and TMA stores.
-// The prologue's (cos, sin) table is read through L1 (no room in smem).
+// With the prologue, the eight prologue warps transform every Q tile together
+// and compute the RoPE angles (no room in shared memory for the table).
 // ============================================================================
 namespace rd2 {
 constexpr int D = 128;
@@ -2829,7 +2896,7 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NQ; ++s) {
       mbar_init(bar_qf + 8 * s, 1);
-      mbar_init(bar_qr + 8 * s, 128);  // the stage's prologue group
+      mbar_init(bar_qr + 8 * s, 256);  // every prologue thread
       mbar_init(bar_qe + 8 * s, 1);
     }
     mbar_init(bar_sf, 1);
@@ -2842,7 +2909,7 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (PRO && threadIdx.x < D) ((float*)(smem + OFF_W))[threadIdx.x] = pro.w[threadIdx.x];
+  if (PRO) pro_w_copy((float2*)(smem + OFF_W), pro.w);
   if (PRO && threadIdx.x < D / 4)  // pair frequencies, as the (cos, sin) table has them
     ((float*)(smem + OFF_TH))[threadIdx.x] = powf(pro.base, -2.0f * (float)threadIdx.x / (float)(D / 2));
   if (warp == 1) {
@@ -2999,11 +3066,10 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
     }
     if (et == 0) bulk_wait0();
   } else if (PRO) {
-    // two groups of 4 warps on alternate Q tiles (group g % 2 owns stage g % 2);
-    // two threads per token, 64 channels each, tokens r and r + 64
+    // all eight warps on every Q tile: four threads per token (32 channels
+    // each), tokens pr and pr + 64
     const int t = threadIdx.x - 192;
-    const int grp = t >> 7, tt = t & 127;
-    const int r = tt >> 1, h = tt & 1;
+    const int pr = t >> 2, pq = t & 3;
     int g = 0;
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
@@ -3012,20 +3078,14 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
       const int tl0 = part * ntile / kParts, tl1 = (part + 1) * ntile / kParts;
       (void)n;
       for (int tl = tl0; tl < tl1; ++tl, ++g) {
-        if ((g & 1) != grp) continue;
         const int s = g % NQ;
         const uint32_t u = (uint32_t)(g / NQ);
         ok = mbar_wait(bar_qf + 8 * s, u & 1, abort_flag, &g_tc_status, 90);
         if (!ok) break;
-#pragma unroll 1
-        for (int half_tok = 0; half_tok < 2; ++half_tok) {
-          const int row = r + 64 * half_tok;
-          const int tok = tl * TOK + row;
-          float f[64];
-          pro_row_part<8>(smem + OFF_Q + s * QT, BOX, row, 64 * h, D, tok, tok < S, pro,
-                          (const float*)(smem + OFF_W) + 64 * h, pro.cs, f,
-                          (const float*)(smem + OFF_TH));
-        }
+        const int rr[2] = {pr, pr + 64}, tk[2] = {tl * TOK + pr, tl * TOK + pr + 64};
+        const float bv[2] = {1.f, 1.f};
+        pro_rows<2>(smem + OFF_Q + s * QT, BOX, rr, pq, tk, S, pro, (const float2*)(smem + OFF_W),
+                    nullptr, (const float*)(smem + OFF_TH), nullptr, bv);
         fence_proxy_async();
         mbar_arrive(bar_qr + 8 * s);
       }

@@ -294,6 +294,45 @@ def test_fused_prologue_bidirectional(D, path, overlap):
         assert U.rel_frob_per_frame(U.host(st_r[0, h])[None], s_r[None]) < U.TOL_BF16
 
 
+@pytest.mark.parametrize("reverse", [False, True])
+@pytest.mark.parametrize("path", PATHS)
+def test_fused_prologue_one_direction(path, reverse):
+    """Fused prologue with a single scan direction, on a 9 x 23 grid: 207
+    tokens span several contraction stages and readout tiles with a ragged
+    tail, and rows of the grid straddle tile boundaries."""
+    gh, gw, T = 9, 23, 5
+    arr = U.random_case(41, 1, 2, T, gh * gw, 128, bf16=True, state=True)
+    d = U.dev_inputs(arr, True)
+    pro = dict(w_q=d["w_q"], w_k=d["w_k"], grid_h=gh, grid_w=gw)
+    block = 2 if reverse else 3
+    out, st = run_scan(d, path, prologue=pro, reverse=reverse, block_reset=reverse, block=block)
+    torch.cuda.synchronize()
+    for h in range(2):
+        o_ref, s_ref = U.oracle_slab(arr, 0, h, True, prologue=(gw, 1e-6, 1e4), reverse=reverse,
+                                     block=block if reverse else 0)
+        assert U.rel_frob_per_frame(U.host(out[0, h]), o_ref) < U.TOL_BF16
+        assert U.rel_frob_per_frame(U.host(st[0, h])[None], s_ref[None]) < U.TOL_BF16
+
+
+@pytest.mark.parametrize("overlap", [True, False])
+def test_fused_prologue_bidirectional_multitile(overlap):
+    """Bidirectional form on a 9 x 23 grid (several tiles, ragged tail)."""
+    gh, gw, T = 9, 23, 7
+    arr = U.random_case(43, 1, 2, T, gh * gw, 128, bf16=True, state=True)
+    d = U.dev_inputs(arr, True)
+    pro = dict(w_q=d["w_q"], w_k=d["w_k"], grid_h=gh, grid_w=gw)
+    out, st, out_r, st_r = run_scan(d, "default", prologue=pro, bidir=True, block_reset=True,
+                                    block=3, overlap=overlap)
+    torch.cuda.synchronize()
+    for h in range(2):
+        o_f, s_f = U.oracle_slab(arr, 0, h, True, prologue=(gw, 1e-6, 1e4))
+        o_r, s_r = U.oracle_slab(arr, 0, h, True, prologue=(gw, 1e-6, 1e4), reverse=True, block=3)
+        assert U.rel_frob_per_frame(U.host(out[0, h]), o_f) < U.TOL_BF16
+        assert U.rel_frob_per_frame(U.host(out_r[0, h]), o_r) < U.TOL_BF16
+        assert U.rel_frob_per_frame(U.host(st[0, h])[None], s_f[None]) < U.TOL_BF16
+        assert U.rel_frob_per_frame(U.host(st_r[0, h])[None], s_r[None]) < U.TOL_BF16
+
+
 # ---------------------------------------------------------------------------
 # full-size workloads, as bench.py launches them; sampled slabs vs the oracle
 # ---------------------------------------------------------------------------
