@@ -82,8 +82,13 @@ static int num_sms() {
   return n;
 }
 
+// Rounds the dynamic shared-memory base up to 1024 bytes (the 128-byte
+// swizzle atom repeats every 1024). The offset is added to the pointer itself,
+// so the compiler still knows the result addresses shared memory and emits
+// shared-memory loads and stores for it rather than generic ones.
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-  return (uint8_t*)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
+  const uint32_t a = (uint32_t)__cvta_generic_to_shared(p);
+  return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
 // ----------------------------------------------------------------------------
