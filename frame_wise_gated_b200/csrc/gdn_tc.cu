@@ -97,7 +97,10 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // Each thread takes NR token rows rr[] of a tile made of two [rows][64] bf16
 // boxes with the 128-byte swizzle, and in each row the 32 channels of its
 // quarter q (channels 32q .. 32q + 31: four 16-byte chunks); the four threads
-// that share a row (consecutive lanes) combine their sums of squares. With
+// that share a row combine their sums of squares. Lane layout (pro_lane): a
+// warp holds 8 rows; lane 8q + j takes quarter q of row j. Each 8-lane phase
+// of a 16-byte access then covers 8 rows of one quarter, whose swizzled
+// chunks fall in 8 distinct bank groups: no bank conflicts. With
 // NR = 2 the rows run side by side so that the latency of one (shared-memory
 // loads, shuffles, rsqrt) overlaps the arithmetic of the other. Since the RMSNorm
 // factor inv = 1/sqrt(mean(x^2) + eps) is positive and RoPE is linear,
@@ -113,7 +116,8 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // is reduced to [-pi, pi] (2 pi split in two parts) and evaluated with the
 // hardware sine/cosine, whose error on that range is near 1e-6 -- below the
 // bf16 rounding the result gets. Otherwise it is read from `tab`, a shared
-// copy of the table laid out by pro_table_index.
+// copy of the table laid out by pro_table_index. THETA and BTILE are template
+// flags so that the unrolled pair loop holds no branches.
 // ----------------------------------------------------------------------------
 constexpr int PRO_POS_PITCH = 80;  // positions per pair in the shared table (the most supported)
 __device__ __forceinline__ int pro_table_index(int i, int pos) {
@@ -128,7 +132,11 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
   return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
-template <int NR>
+// Row (of the warp's 8, plus 8 per warp before it) and quarter of thread t.
+__device__ __forceinline__ int pro_lane_row(int t) { return ((t >> 5) << 3) + (t & 7); }
+__device__ __forceinline__ int pro_lane_quarter(int t) { return (t >> 3) & 3; }
+
+template <int NR, bool THETA, bool BTILE>
 __device__ __forceinline__ void pro_rows(uint8_t* tile, int box_bytes, const int (&rr)[NR], int q,
                                          const int (&tk)[NR], int S, const ProArgs& pro,
                                          const float2* w4, const float2* tab, const float* theta,
@@ -165,7 +173,7 @@ __device__ __forceinline__ void pro_rows(uint8_t* tile, int box_bytes, const int
 #pragma unroll
     for (int k = 0; k < NR; ++k) ss[k] = (acc[k][0].x + acc[k][0].y) + (acc[k][1].x + acc[k][1].y);
 #pragma unroll
-    for (int o = 1; o < 4; o <<= 1) {
+    for (int o = 8; o < 32; o <<= 1) {  // the row's four quarters: lanes j, j + 8, j + 16, j + 24
       float sh[NR];
 #pragma unroll
       for (int k = 0; k < NR; ++k) sh[k] = __shfl_xor_sync(0xffffffffu, ss[k], o);
@@ -192,7 +200,7 @@ __device__ __forceinline__ void pro_rows(uint8_t* tile, int box_bytes, const int
         const float2 m = __fmul2_rn(unpack_bf16x2(u[k][p]), w2);
         const float a = fmaxf(m.x, 0.f), b = fmaxf(m.y, 0.f);
         float2 t;
-        if (theta) {
+        if (THETA) {
           float ang = (float)pos[k] * theta[pb + p];
           const float kq = rintf(ang * 0.159154943091895f);  // 1 / (2 pi)
           ang = fmaf(-kq, 6.28318548202514648f, ang);        // 2 pi, high part
@@ -204,7 +212,7 @@ __device__ __forceinline__ void pro_rows(uint8_t* tile, int box_bytes, const int
         const float2 o = make_float2(a * t.x - b * t.y, a * t.y + b * t.x);
         const float2 kh = __fmul2_rn(o, make_float2(inv[k], inv[k]));
         u[k][p] = pack_bf16x2(kh.x, kh.y);
-        if (btile) {
+        if (BTILE) {
           const float2 bk = __fmul2_rn(o, make_float2(scb[k], scb[k]));
           ob[k][e] = pack_bf16x2(bk.x, bk.y);
         }
@@ -214,7 +222,7 @@ __device__ __forceinline__ void pro_rows(uint8_t* tile, int box_bytes, const int
     for (int k = 0; k < NR; ++k) {
       const int off = box * box_bytes + rr[k] * 128 + (((ch0 + c) ^ (rr[k] & 7)) << 4);
       *(uint4*)(tile + off) = make_uint4(u[k][4 * c], u[k][4 * c + 1], u[k][4 * c + 2], u[k][4 * c + 3]);
-      if (btile) *(uint4*)(btile + off) = make_uint4(ob[k][0], ob[k][1], ob[k][2], ob[k][3]);
+      if (BTILE) *(uint4*)(btile + off) = make_uint4(ob[k][0], ob[k][1], ob[k][2], ob[k][3]);
     }
   }
 }
@@ -464,7 +472,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
     // g % 2 takes stage g and its beta * K slot), so two stages are in flight.
     // Prologue: four threads per token (32 channels each), tokens pr and pr + 32.
     const int grp = t >> 7, tt = t & 127;
-    const int pr = tt >> 2, pq = tt & 3;
+    const int pr = pro_lane_row(tt), pq = pro_lane_quarter(tt);
     int g = 0;
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
@@ -483,7 +491,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
           // raw k -> K^ in place (RMSNorm, ReLU, RoPE) and beta * K^ into the slot
           const int rr[2] = {pr, pr + 32}, tk[2] = {st * TOK + pr, st * TOK + pr + 32};
           const float bv[2] = {beta ? bs[pr] : 1.f, beta ? bs[pr + 32] : 1.f};
-          pro_rows<2>(kt, BOX, rr, pq, tk, S, pro, w4, tab, nullptr, bt, bv);
+          pro_rows<2, false, true>(kt, BOX, rr, pq, tk, S, pro, w4, tab, nullptr, bt, bv);
           fence_proxy_async();
           mbar_arrive(bar_bkf + 8 * kb);
           continue;
@@ -887,7 +895,7 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
     // ---- prologue on each raw Q tile, in place: four threads per token
     // (32 channels each), tokens pr and pr + 64 ----
     const int t = threadIdx.x - 192;
-    const int pr = t >> 2, pq = t & 3;
+    const int pr = pro_lane_row(t), pq = pro_lane_quarter(t);
     int g = 0;
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
@@ -902,8 +910,9 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
         if (!ok) break;
         const int rr[2] = {pr, pr + 64}, tk[2] = {tl * TOK + pr, tl * TOK + pr + 64};
         const float bv[2] = {1.f, 1.f};
-        pro_rows<2>(smem + OFF_Q + s * QT, BOX, rr, pq, tk, S, pro, (const float2*)(smem + OFF_W4),
-                    (const float2*)(smem + OFF_TAB), nullptr, nullptr, bv);
+        pro_rows<2, false, false>(smem + OFF_Q + s * QT, BOX, rr, pq, tk, S, pro,
+                                  (const float2*)(smem + OFF_W4), (const float2*)(smem + OFF_TAB),
+                                  nullptr, nullptr, bv);
         fence_proxy_async();
         mbar_arrive(bar_qr + 8 * s);
       }
@@ -3074,7 +3083,7 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
     // all eight warps on every Q tile: four threads per token (32 channels
     // each), tokens pr and pr + 64
     const int t = threadIdx.x - 192;
-    const int pr = t >> 2, pq = t & 3;
+    const int pr = pro_lane_row(t), pq = pro_lane_quarter(t);
     int g = 0;
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
@@ -3089,8 +3098,9 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
         if (!ok) break;
         const int rr[2] = {pr, pr + 64}, tk[2] = {tl * TOK + pr, tl * TOK + pr + 64};
         const float bv[2] = {1.f, 1.f};
-        pro_rows<2>(smem + OFF_Q + s * QT, BOX, rr, pq, tk, S, pro, (const float2*)(smem + OFF_W),
-                    nullptr, (const float*)(smem + OFF_TH), nullptr, bv);
+        pro_rows<2, true, false>(smem + OFF_Q + s * QT, BOX, rr, pq, tk, S, pro,
+                                 (const float2*)(smem + OFF_W), nullptr, (const float*)(smem + OFF_TH),
+                                 nullptr, bv);
         fence_proxy_async();
         mbar_arrive(bar_qr + 8 * s);
       }
