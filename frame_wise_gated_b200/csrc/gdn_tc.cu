@@ -2862,7 +2862,7 @@ static cudaError_t tc_chain64(const ChainArgs& a, int nchains, cudaStream_t st) 
 //   O_fwd = Q S_fwd_hi^T + Q S_fwd_lo^T,   O_rev = Q S_rev_hi^T + Q S_rev_lo^T
 // (four fp32 TMEM accumulators: two tiles in flight x two directions). Both
 // outputs leave through two 16 KiB swizzled staging buffers and TMA stores.
-// With the prologue, the eight prologue warps transform every Q tile together
+// With the prologue, sixteen prologue warps transform every Q tile together
 // and compute the RoPE angles (no room in shared memory for the table).
 // ============================================================================
 namespace rd2 {
@@ -2882,7 +2882,7 @@ constexpr int NBAR = 3 * NQ + 2 + 4 + 1;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr int SMEM = OFF_MISC + 16 + 1024;
 static_assert(SMEM <= 232448, "bidirectional readout shared memory");
-constexpr int threads(bool pro) { return pro ? 448 : 192; }
+constexpr int threads(bool pro) { return pro ? 704 : 192; }  // + 16 prologue warps
 constexpr uint32_t TMEM_COLS = 512;
 }  // namespace rd2
 
@@ -2910,7 +2910,7 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NQ; ++s) {
       mbar_init(bar_qf + 8 * s, 1);
-      mbar_init(bar_qr + 8 * s, 256);  // every prologue thread
+      mbar_init(bar_qr + 8 * s, 512);  // every prologue thread
       mbar_init(bar_qe + 8 * s, 1);
     }
     mbar_init(bar_sf, 1);
@@ -3080,8 +3080,8 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
     }
     if (et == 0) bulk_wait0();
   } else if (PRO) {
-    // all eight warps on every Q tile: four threads per token (32 channels
-    // each), tokens pr and pr + 64
+    // all sixteen prologue warps on every Q tile: four threads per token
+    // (32 channels each), one token each
     const int t = threadIdx.x - 192;
     const int pr = pro_lane_row(t), pq = pro_lane_quarter(t);
     int g = 0;
@@ -3096,9 +3096,9 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
         const uint32_t u = (uint32_t)(g / NQ);
         ok = mbar_wait(bar_qf + 8 * s, u & 1, abort_flag, &g_tc_status, 90);
         if (!ok) break;
-        const int rr[2] = {pr, pr + 64}, tk[2] = {tl * TOK + pr, tl * TOK + pr + 64};
-        const float bv[2] = {1.f, 1.f};
-        pro_rows<2, true, false>(smem + OFF_Q + s * QT, BOX, rr, pq, tk, S, pro,
+        const int rr[1] = {pr}, tk[1] = {tl * TOK + pr};
+        const float bv[1] = {1.f};
+        pro_rows<1, true, false>(smem + OFF_Q + s * QT, BOX, rr, pq, tk, S, pro,
                                  (const float2*)(smem + OFF_W), nullptr, (const float*)(smem + OFF_TH),
                                  nullptr, bv);
         fence_proxy_async();
