@@ -929,10 +929,14 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
 
 bool tc_readout_supported(int D) { return D == 128 || D == 64 || D == 256; }
 
-// Readout work units: split each frame-head's tiles in two when there are
-// fewer than four rounds of frame-heads for the persistent grid (evens out
-// the last round); with more rounds the per-unit state loads cost more.
+// Readout work units: each frame-head's tiles in three contiguous parts when
+// a part still holds four tiles or more and there are fewer than 32 rounds
+// of frame-heads (finer units even out the last round of the persistent grid;
+// measured on 720p frames, 29 tiles: 3 parts beat 1, 2 and 4 for 48, 336 and
+// 1936 frame-heads; with 7808 the extra state loads cost more than they
+// save), else two when there are fewer than four rounds.
 static int readout_parts(long long N, int ntile) {
+  if (ntile >= 12 && N < 32LL * num_sms()) return 3;
   return (ntile >= 8 && N < 4LL * num_sms()) ? 2 : 1;
 }
 
