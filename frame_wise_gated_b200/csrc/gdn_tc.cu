@@ -91,6 +91,14 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
+// One arrival per warp on `bar` (initialised with a count of warps), after
+// every lane's own fences: 32 lanes arriving one by one serialise on the
+// barrier word.
+__device__ __forceinline__ void warp_arrive(uint32_t bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 // ----------------------------------------------------------------------------
 // Prologue inside the loaders (SANA-WM blog, Context-Parallel section: the
 // fused op runs RMSNorm -> ReLU -> key scale -> RoPE ahead of the scan), D = 128.
@@ -344,7 +352,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
       mbar_init(bar_empty + 8 * s, 1);     // MMA commit
     }
     for (int s = 0; s < NBK; ++s) {
-      mbar_init(bar_bkf + 8 * s, NSC / 2);  // every thread of the slot's scaler group
+      mbar_init(bar_bkf + 8 * s, NSC / 64);  // every warp of the slot's scaler group
       mbar_init(bar_bke + 8 * s, 1);        // MMA commit
     }
     for (int b = 0; b < 2; ++b) {
@@ -493,7 +501,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
           const float bv[2] = {beta ? bs[pr] : 1.f, beta ? bs[pr + 32] : 1.f};
           pro_rows<2, false, true>(kt, BOX, rr, pq, tk, S, pro, w4, tab, nullptr, bt, bv);
           fence_proxy_async();
-          mbar_arrive(bar_bkf + 8 * kb);
+          warp_arrive(bar_bkf + 8 * kb);
           continue;
         }
 #pragma unroll
@@ -511,7 +519,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
           *(uint4*)(bt + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async();
-        mbar_arrive(bar_bkf + 8 * kb);
+        warp_arrive(bar_bkf + 8 * kb);
       }
     }
   } else if (warp < 2 + NSC / 32 + 4) {
@@ -721,14 +729,14 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NQ; ++s) {
       mbar_init(bar_qf + 8 * s, 1);
-      mbar_init(bar_qr + 8 * s, 256);
+      mbar_init(bar_qr + 8 * s, 8);  // every prologue warp
       mbar_init(bar_qe + 8 * s, 1);
     }
     mbar_init(bar_sf, 1);
     mbar_init(bar_se, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_accf + 8 * b, 1);
-      mbar_init(bar_acce + 8 * b, 128);
+      mbar_init(bar_acce + 8 * b, 4);  // every epilogue warp
     }
     mbar_init(bar_fin, 1);
     *abort_flag = 0;
@@ -880,7 +888,7 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
           }
         }
         tc_fence_before();
-        mbar_arrive(bar_acce + 8 * b);
+        warp_arrive(bar_acce + 8 * b);
         fence_proxy_async();
         named_bar_sync(1, 128);
         if (et == 0) {
@@ -914,7 +922,7 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
                                   (const float2*)(smem + OFF_W4), (const float2*)(smem + OFF_TAB),
                                   nullptr, nullptr, bv);
         fence_proxy_async();
-        mbar_arrive(bar_qr + 8 * s);
+        warp_arrive(bar_qr + 8 * s);
       }
     }
   }
@@ -2914,14 +2922,14 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NQ; ++s) {
       mbar_init(bar_qf + 8 * s, 1);
-      mbar_init(bar_qr + 8 * s, 512);  // every prologue thread
+      mbar_init(bar_qr + 8 * s, 16);  // every prologue warp
       mbar_init(bar_qe + 8 * s, 1);
     }
     mbar_init(bar_sf, 1);
     mbar_init(bar_se, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_accf + 8 * b, 1);
-      mbar_init(bar_acce + 8 * b, 128);
+      mbar_init(bar_acce + 8 * b, 4);  // every epilogue warp
     }
     mbar_init(bar_fin, 1);
     *abort_flag = 0;
@@ -3079,7 +3087,7 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
         }
         if (!ok) break;
         tc_fence_before();
-        mbar_arrive(bar_acce + 8 * b);
+        warp_arrive(bar_acce + 8 * b);
       }
     }
     if (et == 0) bulk_wait0();
@@ -3106,7 +3114,7 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
                                  (const float2*)(smem + OFF_W), nullptr, (const float*)(smem + OFF_TH),
                                  nullptr, bv);
         fence_proxy_async();
-        mbar_arrive(bar_qr + 8 * s);
+        warp_arrive(bar_qr + 8 * s);
       }
     }
   }
