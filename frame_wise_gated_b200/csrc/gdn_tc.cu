@@ -357,7 +357,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_accf + 8 * b, 1);
-      mbar_init(bar_acce + 8 * b, 128);
+      mbar_init(bar_acce + 8 * b, 4);
     }
     mbar_init(bar_fin, 1);
     *abort_flag = 0;
@@ -597,7 +597,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
         }
       }
       tc_fence_before();
-      mbar_arrive(bar_acce + 8 * b);
+      warp_arrive(bar_acce + 8 * b);
       if (flags) {
         // publish this warp's rows of A_t, U_t: its stores, made visible to
         // other CTAs' bulk/TMA loads (async proxy), then a release increment
@@ -1532,12 +1532,12 @@ __global__ void __launch_bounds__(sro::THREADS, 1)
       mbar_init(bar_qe + 8 * s, 1);
     }
     mbar_init(bar_yf, 1);
-    mbar_init(bar_xf, 256);
+    mbar_init(bar_xf, 8);
     mbar_init(bar_pf, 1);
     mbar_init(bar_rd, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_accf + 8 * b, 1);
-      mbar_init(bar_acce + 8 * b, 256);
+      mbar_init(bar_acce + 8 * b, 8);
     }
     mbar_init(bar_fin, 1);
     *abort_flag = 0;
@@ -1668,7 +1668,7 @@ __global__ void __launch_bounds__(sro::THREADS, 1)
       chain_store_x(x, xtile, xtile + 2 * BOX, row, h);
       fence_proxy_async();
       tc_fence_before();
-      mbar_arrive(bar_xf);
+      warp_arrive(bar_xf);
     };
     for (int c = blockIdx.x; c < nchains; c += gridDim.x) {
       const ChainProg pg = chain_prog(a, c);
@@ -1730,7 +1730,7 @@ __global__ void __launch_bounds__(sro::THREADS, 1)
             }
           }
           tc_fence_before();
-          mbar_arrive(bar_acce + 8 * b);
+          warp_arrive(bar_acce + 8 * b);
         }
         ++ridx;
       }
@@ -2225,12 +2225,12 @@ __global__ void __launch_bounds__(c64::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(bar_full + 8 * s, 33);
-      mbar_init(bar_bk + 8 * s, NSC);
+      mbar_init(bar_bk + 8 * s, NSC / 32);
       mbar_init(bar_empty + 8 * s, 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_accf + 8 * b, 1);
-      mbar_init(bar_acce + 8 * b, 128);
+      mbar_init(bar_acce + 8 * b, 4);
     }
     mbar_init(bar_fin, 1);
     *abort_flag = 0;
@@ -2340,7 +2340,7 @@ __global__ void __launch_bounds__(c64::THREADS, 1)
           *(uint4*)(bt + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async();
-        mbar_arrive(bar_bk + 8 * s);
+        warp_arrive(bar_bk + 8 * s);
       }
     }
   } else {
@@ -2381,7 +2381,7 @@ __global__ void __launch_bounds__(c64::THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar_acce + 8 * b);
+      warp_arrive(bar_acce + 8 * b);
     }
   }
   tc_fence_before();
@@ -2435,7 +2435,7 @@ __global__ void __launch_bounds__(r64::THREADS, 1)
     mbar_init(bar_se, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_accf + 8 * b, 1);
-      mbar_init(bar_acce + 8 * b, 128);
+      mbar_init(bar_acce + 8 * b, 4);
     }
     mbar_init(bar_fin, 1);
     *abort_flag = 0;
@@ -2564,7 +2564,7 @@ __global__ void __launch_bounds__(r64::THREADS, 1)
                 pack_bf16x2(__uint_as_float(rr[8 * j + 6]), __uint_as_float(rr[8 * j + 7])));
         }
         tc_fence_before();
-        mbar_arrive(bar_acce + 8 * b);
+        warp_arrive(bar_acce + 8 * b);
         fence_proxy_async();
         named_bar_sync(1, 128);
         if (et == 0) {
@@ -3224,11 +3224,11 @@ __global__ void __launch_bounds__(c256::THREADS, 1)
       mbar_init(bar_empty + 8 * s, 1);
     }
     for (int s = 0; s < NBK; ++s) {
-      mbar_init(bar_bkf + 8 * s, NSC);
+      mbar_init(bar_bkf + 8 * s, NSC / 32);
       mbar_init(bar_bke + 8 * s, 1);
     }
     mbar_init(bar_accf, 1);
-    mbar_init(bar_acce, 128);
+    mbar_init(bar_acce, 4);
     mbar_init(bar_fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -3343,7 +3343,7 @@ __global__ void __launch_bounds__(c256::THREADS, 1)
           *(uint4*)(bt + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async();
-        mbar_arrive(bar_bkf + 8 * kb);
+        warp_arrive(bar_bkf + 8 * kb);
       }
     }
   } else {
@@ -3393,7 +3393,7 @@ __global__ void __launch_bounds__(c256::THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar_acce);
+      warp_arrive(bar_acce);
     }
   }
   tc_fence_before();
@@ -3447,7 +3447,7 @@ __global__ void __launch_bounds__(r256::THREADS, 1)
     mbar_init(bar_se, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_accf + 8 * b, 1);
-      mbar_init(bar_acce + 8 * b, 128);
+      mbar_init(bar_acce + 8 * b, 4);
     }
     mbar_init(bar_fin, 1);
     *abort_flag = 0;
@@ -3576,7 +3576,7 @@ __global__ void __launch_bounds__(r256::THREADS, 1)
           }
         }
         tc_fence_before();
-        mbar_arrive(bar_acce + 8 * b);
+        warp_arrive(bar_acce + 8 * b);
         fence_proxy_async();
         named_bar_sync(1, 128);
         if (et == 0) {
@@ -3714,7 +3714,7 @@ __global__ void __launch_bounds__(ch2::THREADS, 1)
       mbar_init(bar_ye + 8 * s, 1);
     }
     mbar_init(bar_p, 1);
-    mbar_init(bar_x, EPI);
+    mbar_init(bar_x, EPI / 32);
     mbar_init(bar_fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -3840,7 +3840,7 @@ __global__ void __launch_bounds__(ch2::THREADS, 1)
     tmem_wait_st();
     fence_proxy_async();
     tc_fence_before();
-    mbar_arrive(bar_x);
+    warp_arrive(bar_x);
     if (g.n > 0) {
       const ChainStep st0 = chain_step_at(a, g, 0);
       load_z(st0.Z, 0, zb[0]);
@@ -3898,7 +3898,7 @@ __global__ void __launch_bounds__(ch2::THREADS, 1)
         bulk_commit();
         ++nstore;
       }
-      mbar_arrive(bar_x);
+      warp_arrive(bar_x);
     }
     if (et == 0) bulk_wait0();
   }
@@ -3992,7 +3992,7 @@ __global__ void __launch_bounds__(btk::THREADS, 1)
     mbar_init(bar_bf, 1);
     mbar_init(bar_be, 1);
     mbar_init(bar_accf, 1);
-    mbar_init(bar_acce, EPI);
+    mbar_init(bar_acce, EPI / 32);
     mbar_init(bar_fin, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -4164,7 +4164,7 @@ __global__ void __launch_bounds__(btk::THREADS, 1)
           }
         }
         tc_fence_before();
-        mbar_arrive(bar_acce);
+        warp_arrive(bar_acce);
         float* red = (float*)(smem + OFF_RED) + (g & 1) * TOK * 2;
         red[row * 2 + h] = dbp;
         fence_proxy_async();
@@ -4285,7 +4285,7 @@ __global__ void __launch_bounds__(bfr::THREADS, 1)
     mbar_init(bar_ine, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_accf + 8 * b, 1);
-      mbar_init(bar_acce + 8 * b, 128);
+      mbar_init(bar_acce + 8 * b, 4);
     }
     mbar_init(bar_fin, 1);
     *abort_flag = 0;
@@ -4404,7 +4404,7 @@ __global__ void __launch_bounds__(bfr::THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar_acce + 8 * b);
+      warp_arrive(bar_acce + 8 * b);
       // G row i_row (hi + lo, rounded) -> operand row 128 + i_row
       const __nv_bfloat16* gh = Ghilo + (size_t)n * 2 * D * D + (size_t)i_row * D;
       const int r = 128 + i_row;
