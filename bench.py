@@ -517,7 +517,7 @@ def run_e2e(args, cfg, arr, dev, api, barrier, dist, world):
     hst = torch.empty((cfg.B, cfg.H, cfg.D, cfg.D), dtype=torch.float32).pin_memory()
     h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hb, hg) + ((hs0,) if hs0 is not None else ()))
     d2h = hout.numel() * hout.element_size() + hst.numel() * 4
-    hpc = max(1, (cfg.B * cfg.H) // 4)
+    hpc = max(1, (cfg.B * cfg.H) // max(1, args.e2e_chunks))
 
     def step():
         api.frame_scan_fwd_host(hq, hk, hv, hb, hg, hs0, out=hout, state_out=hst,
@@ -560,6 +560,9 @@ def main():
     ap.add_argument("--train", action="store_true",
                     help="with --bwd: time forward + backward from the forward's saved workspace")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-chunks", type=int, default=8,
+                    help="head chunks of the end-to-end host-streaming call (copies of one "
+                         "chunk overlap the scan of the next)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-frames", type=int, default=6,
                     help="frames of one slab per reference step")
