@@ -3410,6 +3410,7 @@ constexpr int TOK = 128;
 constexpr int NQ = 2;
 constexpr int BOX = TOK * 128;           // [128 rows][64 channels]: 16 KiB
 constexpr int QH = 2 * BOX;              // Q half tile (128 channels): 32 KiB
+static_assert(2 * QH == TOK * D * 2, "two half tiles hold a tile's D bf16 channels");
 constexpr int OFF_Q = 0;
 constexpr int OFF_S = OFF_Q + NQ * QH;   // S rows half: hi 4 atoms, lo 4 atoms (128 KiB)
 constexpr int OFF_O = OFF_S + 8 * BOX;   // output staging: 2 boxes
@@ -4239,7 +4240,7 @@ constexpr int OFF_S = 0;                // S' (hi, lo)
 constexpr int OFF_G = OFF_S + MAT;      // G (hi, lo)
 constexpr int OFF_BAR = OFF_G + MAT;
 constexpr int NBAR = 2 + 2 + 2 + 1;     // in_full, in_empty, acc_full[2], acc_empty[2], fin
-constexpr int OFF_RED = OFF_BAR + 64;
+constexpr int OFF_RED = OFF_BAR + 8 * (NBAR + 1);
 constexpr int OFF_MISC = OFF_RED + 4 * 4;
 constexpr int SMEM = OFF_MISC + 16 + 1024;
 constexpr int THREADS = 64 + 128;
