@@ -101,6 +101,14 @@ def test_backward_edge_sizes():
         check_case(arr, dO, dS, True, U.TOL_BF16)
 
 
+def test_backward_three_part_dq_units():
+    """Frames of 1496 tokens (12 tiles of 128, the last 88 tokens): the dq
+    readout splits each frame-head into three units of 4 tiles."""
+    arr = U.random_case(61, 1, 2, 3, 1496, 128, bf16=True, state=True)
+    dO, dS = upstream(62, 1, 2, 3, 1496, 128, True)
+    check_case(arr, dO, dS, True, U.TOL_BF16)
+
+
 @pytest.mark.parametrize("name", ["clip5s_720p", "rollout60s_720p"])
 def test_backward_full_size(name):
     """The 720p workloads (B=1, H=16, S=3600, D=128, bf16; T = 21 or 121) on the

@@ -333,6 +333,33 @@ def test_fused_prologue_bidirectional_multitile(overlap):
         assert U.rel_frob_per_frame(U.host(st_r[0, h])[None], s_r[None]) < U.TOL_BF16
 
 
+@pytest.mark.parametrize("bidir_prologue", [False, True])
+def test_readout_three_part_units(bidir_prologue):
+    """Frames of 1496 tokens (a 34 x 44 grid: 12 readout tiles, the last one
+    88 tokens): each frame-head's tiles go to three work units of 4 tiles, so
+    unit boundaries, ragged tails and several units per CTA all occur; forward
+    scan, or the fused-prologue bidirectional form."""
+    gh, gw, T = 34, 44, 4
+    arr = U.random_case(47, 1, 3, T, gh * gw, 128, bf16=True, state=True)
+    d = U.dev_inputs(arr, True)
+    if bidir_prologue:
+        pro = dict(w_q=d["w_q"], w_k=d["w_k"], grid_h=gh, grid_w=gw)
+        out, st, out_r, st_r = run_scan(d, "default", prologue=pro, bidir=True, block_reset=True,
+                                        block=3)
+    else:
+        out, st = run_scan(d, "default")
+    torch.cuda.synchronize()
+    for h in range(3):
+        if bidir_prologue:
+            o_ref, s_ref = U.oracle_slab(arr, 0, h, True, prologue=(gw, 1e-6, 1e4))
+            o_rr, _ = U.oracle_slab(arr, 0, h, True, prologue=(gw, 1e-6, 1e4), reverse=True, block=3)
+            assert U.rel_frob_per_frame(U.host(out_r[0, h]), o_rr) < U.TOL_BF16
+        else:
+            o_ref, s_ref = U.oracle_slab(arr, 0, h, True)
+        assert U.rel_frob_per_frame(U.host(out[0, h]), o_ref) < U.TOL_BF16
+        assert U.rel_frob_per_frame(U.host(st[0, h])[None], s_ref[None]) < U.TOL_BF16
+
+
 # ---------------------------------------------------------------------------
 # full-size workloads, as bench.py launches them; sampled slabs vs the oracle
 # ---------------------------------------------------------------------------
