@@ -363,12 +363,15 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
   // for, or the shape does not fit it.
   const bool bidir = (f & GDN_BIDIR) != 0;
   const int ndir = bidir ? 2 : 1;
-  // Few frame-heads (e.g. one 3-frame block per call): cut each frame-head's
-  // tokens over several CTAs (partial sums), then the chains in their own launch.
+  // Very few frame-heads (at most a quarter of the SMs): cut each frame-head's
+  // tokens over several CTAs (partial sums), then the chains in their own
+  // launch. From a quarter on, the chains alongside the contraction win (one
+  // 3-frame block of 16 heads, 48 frame-heads at 720p: 0.149 against 0.168 ms
+  // per call).
   const int nsms = (tc_contract_ok && p.D == 128) ? tc_num_sms() : 0;
   const int nst = (p.S + 63) / 64;
   const bool split = tc_contract_ok && tc_chain_ok && tc_readout_ok && p.D == 128 &&
-                     !(f & GDN_FUSED_REPLAY) && frames * 2 <= nsms && nst >= 4;
+                     !(f & GDN_FUSED_REPLAY) && frames * 4 <= nsms && nst >= 4;
   int parts = 1;
   if (split) {
     parts = (int)(nsms / frames);

@@ -376,6 +376,8 @@ FULL = [
     ("sweep_d64", {}),
     ("sweep_d256", {}),
     ("sweep_d256", {"chunked": True}),
+    ("stream_block3_720p", {}),
+    ("stream_block3_720p", {"overlap": False}),
 ]
 
 
