@@ -123,7 +123,10 @@ enum {
  * the tensor-core path (bf16, sm_100a), D = 128, at most a quarter of the
  * GPU's SMs in chains (B*H <= 37 on a 148-SM B200; 2*B*H for GDN_BIDIR, which
  * also needs GDN_BLOCK_RESET), and no GDN_FUSED_REPLAY. GDN_NO_OVERLAP turns
- * it off. Scratch comes from a stream-ordered allocation (cudaMallocAsync)
+ * it off. With very few frame-heads (B*H*T at most a quarter of the SMs, at
+ * least 193 tokens per frame) the contraction instead cuts each frame-head's
+ * tokens over several CTAs and the chains follow in their own launch.
+ * Scratch comes from a stream-ordered allocation (cudaMallocAsync)
  * made and freed inside the call; use gdn_frame_scan_fwd_ex to pass your own.
  * Returns GDN_OK or a negative status.
  */
