@@ -52,9 +52,13 @@ Pins (tests/test_oracle_pins.py) and their status per function:
   readout (inside frame_scan)   definition pinned by reading R1 only: parity
                                 with the pages' own readout is unpinned.
   qk_prologue                   pinned by invariants (mean square, sign,
-                                orthogonality, identity, relative phase); its
-                                constants (eps, pair layout, axis split) are
-                                readings R8-R10, unpinned by the pages.
+                                orthogonality, identity, relative phase) and
+                                by hand-worked fixtures of its constants
+                                (eps inside the root and the weight after the
+                                normalisation; every pair's frequency, the
+                                axis split, the pair layout and the turn
+                                direction). The constants themselves are
+                                readings R8-R10: the pages do not fix them.
   frame_scan_bwd                the pages print no backward; this is the
                                 adjoint of frame_scan derived by reverse-mode
                                 differentiation, pinned by central finite

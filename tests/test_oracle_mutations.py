@@ -84,3 +84,90 @@ def test_unmutated_copy_passes():
     "gamma_dropped", "readout_untransposed", "readout_pre_update", "scale_sqrt_S_only"])
 def test_pins_catch_mutation(mutation):
     assert not pins_pass(make_scan(mutation))
+
+
+# --- the prologue: planted mistakes in copies of rmsnorm / rope2d ----------
+
+def make_rmsnorm(mutation):
+    def rmsnorm(x, w, eps=1e-6):
+        x = np.asarray(x, np.float64)
+        w = np.asarray(w, np.float64)
+        ms = np.mean(x * x, axis=-1, keepdims=True)
+        if mutation == "eps_outside_root":
+            return x / (np.sqrt(ms) + eps) * w
+        if mutation == "eps_dropped":
+            return x / np.sqrt(ms) * w
+        if mutation == "weight_before_norm":
+            xw = x * w
+            return xw / np.sqrt(np.mean(xw * xw, axis=-1, keepdims=True) + eps)
+        return x / np.sqrt(ms + eps) * w
+    return rmsnorm
+
+
+def make_rope2d(mutation):
+    def rope2d(x, grid_w, base=10000.0):
+        x = np.array(x, np.float64)
+        S, D = x.shape[-2], x.shape[-1]
+        half = D // 2
+        s = np.arange(S)
+        pos_y, pos_x = s // grid_w, s % grid_w
+        if mutation == "axes_swapped":
+            pos_y, pos_x = pos_x, pos_y
+        out = x.copy()
+        for i in range(D // 4):
+            expo = 2.0 * i / (D if mutation == "full_D_exponent" else half)
+            theta = base ** (-expo)
+            for off, pos in ((0, pos_y), (half, pos_x)):
+                phi = pos * theta
+                cs, sn = np.cos(phi), np.sin(phi)
+                if mutation == "sign_flipped":
+                    sn = -sn
+                if mutation == "rotate_half_pairs":   # pairs (i, i + D/4) instead of (2i, 2i+1)
+                    ia, ib = off + i, off + i + D // 4
+                else:
+                    ia, ib = off + 2 * i, off + 2 * i + 1
+                a, b = x[..., ia], x[..., ib]
+                out[..., ia] = a * cs - b * sn
+                out[..., ib] = a * sn + b * cs
+        return out
+    return rope2d
+
+
+def prologue_pins_pass(rmsnorm, rope2d):
+    ok = True
+    g = json.load(open(os.path.join(GOLD, "rope2d_pair1.json")))
+    for c in g["cases"]:
+        x = np.zeros((c["S"], g["D"]))
+        x[g["token"]] = g["x_in"]
+        ok &= np.allclose(rope2d(x, c["grid_w"], g["base"])[g["token"]], c["expected"], atol=1e-12)
+    g = json.load(open(os.path.join(GOLD, "rmsnorm_eps.json")))
+    ok &= np.allclose(rmsnorm(np.array(g["x"]), np.array(g["w"]), eps=g["eps"]), g["expected"],
+                      atol=1e-14)
+    # the first pair of each half turns by exactly pos radians
+    x = np.zeros((8, 8))
+    x[:, 0] = 1.0
+    x[:, 4] = 1.0
+    y = rope2d(x, 4)
+    ok &= np.allclose(y[6, :2], [np.cos(1.0), np.sin(1.0)]) and np.allclose(
+        y[6, 4:6], [np.cos(2.0), np.sin(2.0)])
+    return bool(ok)
+
+
+def test_unmutated_prologue_copy_passes():
+    assert prologue_pins_pass(make_rmsnorm(None), make_rope2d(None))
+    # and the copies agree with the oracle itself
+    rng = np.random.default_rng(11)
+    x, w = rng.standard_normal((12, 16)), 0.5 + rng.random(16)
+    np.testing.assert_allclose(make_rmsnorm(None)(x, w, 0.3), O.rmsnorm(x, w, 0.3), rtol=1e-15)
+    np.testing.assert_allclose(make_rope2d(None)(x, 4), O.rope2d(x, 4), rtol=1e-15)
+
+
+@pytest.mark.parametrize("mutation", ["eps_outside_root", "eps_dropped", "weight_before_norm"])
+def test_pins_catch_rmsnorm_mutation(mutation):
+    assert not prologue_pins_pass(make_rmsnorm(mutation), make_rope2d(None))
+
+
+@pytest.mark.parametrize("mutation", ["full_D_exponent", "axes_swapped", "sign_flipped",
+                                      "rotate_half_pairs"])
+def test_pins_catch_rope_mutation(mutation):
+    assert not prologue_pins_pass(make_rmsnorm(None), make_rope2d(mutation))

@@ -348,6 +348,25 @@ def test_rope_frequency_of_first_pair():
     assert y[s, 4] == pytest.approx(np.cos(2.0)) and y[s, 5] == pytest.approx(np.sin(2.0))
 
 
+def test_rope_golden_pair_frequencies():
+    """Hand-worked: at D = 8 pair 1 of each half turns by 10000^(-1/2) per
+    position, so position 100 turns it by exactly 1 rad (derivation in the
+    fixture); pins the frequency of every pair past the first."""
+    g = json.load(open(os.path.join(GOLD, "rope2d_pair1.json")))
+    for c in g["cases"]:
+        x = np.zeros((c["S"], g["D"]))
+        x[g["token"]] = g["x_in"]
+        y = O.rope2d(x, c["grid_w"], g["base"])
+        np.testing.assert_allclose(y[g["token"]], c["expected"], rtol=0, atol=1e-12)
+
+
+def test_rmsnorm_golden_eps_inside_root():
+    """Hand-worked: x = (3, 4), w = (2, 1/2), eps = 1/2 gives (6, 2)/sqrt(13)."""
+    g = json.load(open(os.path.join(GOLD, "rmsnorm_eps.json")))
+    y = O.rmsnorm(np.array(g["x"]), np.array(g["w"]), eps=g["eps"])
+    np.testing.assert_allclose(y, g["expected"], rtol=0, atol=1e-14)
+
+
 def test_prologue_order_and_key_scale():
     rng = np.random.default_rng(30)
     W, Hh, D = 4, 4, 16
