@@ -107,6 +107,8 @@ SIGNATURES = {
     "gdn_launch_count": (ctypes.c_longlong, [_I]),
     "gdn_version": (_I, []),
     "gdn_profile_enable": (_I, [_I]),
+    "gdn_fault_inject": (_I, [_I]),
+    "gdn_rope_eval": (_I, [_I, _I, _F, _I, _P, _P]),
     "gdn_profile_read": (_I, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong), _I]),
 }
 
@@ -160,6 +162,18 @@ def _want(t: torch.Tensor, name: str, dtype=None, shape=None):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
+def _want_states_outputs(q, state_in, out, state_out):
+    """Checks caller-supplied state_in / out / state_out against q's sizes:
+    a wrong dtype or size would make the kernels read or write past them."""
+    B, H, T, S, D = q.shape
+    if state_in is not None:
+        _want(state_in, "state_in", torch.float32, (B, H, D, D))
+    if out is not None:
+        _want(out, "out", q.dtype, (B, H, T, S, D))
+    if state_out is not None:
+        _want(state_out, "state_out", torch.float32, (B, H, D, D))
+
+
 def scan_flags(*, bf16: bool, reverse=False, block_reset=False, block=3, chunk=8,
                sequential=False, keys_scaled=False, force_simt=False, prologue=False,
                bidir=False, fused_replay=False, chunked=False, overlap=True) -> int:
@@ -206,8 +220,11 @@ def frame_scan_fwd_ex(q, k, v, beta, gamma, state_in=None, *, reverse=False, blo
         _want(t, n, q.dtype, (B, H, T, S, D))
     _want(beta, "beta", torch.float32, (B, H, T, S))
     _want(gamma, "gamma", torch.float32, (B, H, T))
-    if state_in is not None:
-        _want(state_in, "state_in", torch.float32, (B, H, D, D))
+    _want_states_outputs(q, state_in, out, state_out)
+    if out_rev is not None:
+        _want(out_rev, "out_rev", q.dtype, (B, H, T, S, D))
+    if state_out_rev is not None:
+        _want(state_out_rev, "state_out_rev", torch.float32, (B, H, D, D))
     flags = scan_flags(bf16=bf16, reverse=reverse, block_reset=block_reset, block=block,
                        chunk=chunk, sequential=sequential, keys_scaled=keys_scaled,
                        force_simt=force_simt, prologue=prologue is not None, bidir=bidir,
@@ -258,6 +275,7 @@ def frame_scan_fwd(q, k, v, beta, gamma, state_in=None, *, reverse=False, block_
         _want(t, n, q.dtype, (B, H, T, S, D))
     _want(beta, "beta", torch.float32, (B, H, T, S))
     _want(gamma, "gamma", torch.float32, (B, H, T))
+    _want_states_outputs(q, state_in, out, state_out)
     flags = scan_flags(bf16=q.dtype == torch.bfloat16, reverse=reverse, block_reset=block_reset,
                        block=block, chunk=chunk, sequential=sequential,
                        keys_scaled=keys_scaled, force_simt=force_simt, chunked=chunked,
@@ -352,13 +370,16 @@ def frame_scan_fwd_host(q, k, v, beta, gamma, state_in=None, *, out=None, state_
 
 def frame_scan_bwd(q, k, v, beta, gamma, state_in, d_out, d_state_out=None, *, reverse=False,
                    block_reset=False, block=3, keys_scaled=False, want_state_in_grad=True,
-                   force_simt=False, saved_workspace=None, workspace=None, stream=None):
+                   force_simt=False, saved_workspace=None, workspace=None, grads=None,
+                   stream=None):
     """Gradients through the frame scan (gdn_frame_scan_bwd): given
     d_out = dL/dO [B,H,T,S,D] and d_state_out = dL/d(state_out) [B,H,D,D]
     (or None), returns (dq, dk, dv, dbeta, dgamma, d_state_in) for the scan
     with the same flags (d_state_in None unless want_state_in_grad).
     saved_workspace: the workspace tensor of a frame_scan_fwd_ex call on the
-    same inputs and flags (bf16, D = 128), reused instead of recomputing."""
+    same inputs and flags (bf16, D = 128), reused instead of recomputing.
+    grads: optional dict of caller-owned output tensors (dq, dk, dv, dbeta,
+    dgamma, d_state_in) to write into instead of allocating."""
     B, H, T, S, D = q.shape
     bf16 = q.dtype == torch.bfloat16
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (d_out, "d_out")):
@@ -372,10 +393,26 @@ def frame_scan_bwd(q, k, v, beta, gamma, state_in, d_out, d_state_out=None, *, r
     flags = scan_flags(bf16=bf16, reverse=reverse, block_reset=block_reset, block=block,
                        keys_scaled=keys_scaled, force_simt=force_simt)
     flags &= ~(CHUNKED | NO_OVERLAP | 0xFF0000)  # plan bits do not apply to the backward
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    dbeta, dgamma = torch.empty_like(beta), torch.empty_like(gamma)
-    ds0 = torch.empty((B, H, D, D), device=q.device, dtype=torch.float32) \
-        if want_state_in_grad else None
+    g = dict(grads or {})
+    dq = g.get("dq", None)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = g.get("dk", None)
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = g.get("dv", None)
+    dv = torch.empty_like(v) if dv is None else dv
+    dbeta = g.get("dbeta", None)
+    dbeta = torch.empty_like(beta) if dbeta is None else dbeta
+    dgamma = g.get("dgamma", None)
+    dgamma = torch.empty_like(gamma) if dgamma is None else dgamma
+    ds0 = g.get("d_state_in", None)
+    if ds0 is None and want_state_in_grad:
+        ds0 = torch.empty((B, H, D, D), device=q.device, dtype=torch.float32)
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _want(t, n, q.dtype, (B, H, T, S, D))
+    _want(dbeta, "dbeta", torch.float32, (B, H, T, S))
+    _want(dgamma, "dgamma", torch.float32, (B, H, T))
+    if ds0 is not None:
+        _want(ds0, "d_state_in", torch.float32, (B, H, D, D))
     need = int(lib().gdn_bwd_workspace_bytes(B, H, T, S, D, flags))
     if workspace is None:
         workspace = torch.empty(max(need, 1), device=q.device, dtype=torch.uint8)
@@ -450,6 +487,7 @@ def frame_scan_fwd_static(q, k, v, beta, gamma, state_in=None, *, reverse=False,
         _want(t, n, q.dtype, (B, H, T, S, D))
     _want(beta, "beta", torch.float32, (B, H, T, S))
     _want(gamma, "gamma", torch.float32, (B, H, T))
+    _want_states_outputs(q, state_in, out, state_out)
     flags = scan_flags(bf16=q.dtype == torch.bfloat16, reverse=reverse, block_reset=block_reset,
                        block=block, chunk=chunk, sequential=sequential,
                        keys_scaled=keys_scaled, force_simt=force_simt, chunked=chunked,
@@ -513,6 +551,12 @@ def chunk_composites(A, U, gamma, L, *, force_simt=False, stream=None):
 
 def check_device_status(stream=None) -> None:
     _check(lib().gdn_check_device_status(_stream(stream)), "gdn_check_device_status")
+
+
+def fault_inject(n: int) -> int:
+    """Arms host-side fault injection: the next n scan calls on this thread
+    fail with GDN_ERR_CUDA before launching. Returns the previous pending count."""
+    return int(lib().gdn_fault_inject(int(n)))
 
 
 def launch_count(reset: bool = False) -> int:

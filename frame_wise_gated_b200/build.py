@@ -1,6 +1,6 @@
 """Builds libgdnscan.so in-tree with nvcc for sm_100a.
 
-Usage: python -m frame_wise_gated_b200.build [--debug]
+Usage: python -m frame_wise_gated_b200.build [-v]
 """
 
 from __future__ import annotations
@@ -23,18 +23,16 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def build(debug: bool = False, verbose: bool = False) -> str:
+def build(verbose: bool = False) -> str:
     srcs = sorted(glob.glob(os.path.join(PKG, "csrc", "*.cu")))
     deps = srcs + glob.glob(os.path.join(PKG, "csrc", "*.cuh")) + [os.path.join(ROOT, "include", "gdn.h")]
-    if os.path.exists(LIB) and not debug:
+    if os.path.exists(LIB):
         t = os.path.getmtime(LIB)
         if all(os.path.getmtime(d) <= t for d in deps):
             return LIB
     cmd = [nvcc_path(), "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
            "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hidden", "-shared",
            "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp"] + srcs
-    if debug:
-        cmd += ["-DGDN_DEBUG=1"]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     subprocess.run(cmd, check=True)
@@ -43,4 +41,4 @@ def build(debug: bool = False, verbose: bool = False) -> str:
 
 
 if __name__ == "__main__":
-    print(build(debug="--debug" in sys.argv, verbose="-v" in sys.argv))
+    print(build(verbose="-v" in sys.argv))

@@ -84,6 +84,17 @@ static int fail(int status, const char* fmt, const char* detail = "") {
   return status;
 }
 
+// Host-side fault injection (gdn_fault_inject): the next t_inject scan calls
+// on this host thread report a launch failure once their arguments have been
+// checked, before they allocate or launch anything.
+static thread_local int t_inject = 0;
+
+static int injected_failure() {
+  if (t_inject <= 0) return GDN_OK;
+  --t_inject;
+  return fail(GDN_ERR_CUDA, "injected launch failure (gdn_fault_inject)%s");
+}
+
 static int cuda_fail(cudaError_t e, const char* where) {
   char buf[512];
   snprintf(buf, sizeof(buf), "%s: %s", where, cudaGetErrorString(e));
@@ -300,6 +311,7 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
     return fail(GDN_ERR_WORKSPACE, "workspace missing or smaller than gdn_workspace_bytes%s");
   if (((uintptr_t)p.workspace & 255u) != 0)
     return fail(GDN_ERR_INVALID, "workspace must be 256-byte aligned%s");
+  if ((rc = injected_failure()) != GDN_OK) return rc;
 
   const bool bf16 = (f & GDN_BF16) != 0;
   const bool sm100 = device_cc_major() == 10;
@@ -654,6 +666,7 @@ static int scan_bwd(const gdn_bwd_params& p, cudaStream_t st) {
     return fail(GDN_ERR_WORKSPACE, "workspace missing or smaller than gdn_bwd_workspace_bytes%s");
   if (((uintptr_t)p.workspace & 255u) != 0)
     return fail(GDN_ERR_INVALID, "workspace must be 256-byte aligned%s");
+  if ((rc = injected_failure()) != GDN_OK) return rc;
 
   const bool bf16 = (f & GDN_BF16) != 0;
   const bool reverse = (f & GDN_REVERSE) != 0;
@@ -760,6 +773,12 @@ const char* gdn_status_string(int s) {
 }
 
 const char* gdn_last_error(void) { return t_last_error.c_str(); }
+
+int gdn_fault_inject(int n) {
+  const int pending = t_inject;
+  t_inject = n > 0 ? n : 0;
+  return pending;
+}
 
 long long gdn_launch_count(int reset) {
   long long n = t_launches;
@@ -1012,6 +1031,18 @@ int gdn_selftest_wait(int arrive, long long limit_ns, gdn_stream_t stream) {
     return fail(GDN_ERR_INVALID, "limit_ns must be in [0, 1e9]%s");
   cudaError_t e = tc_selftest_wait(arrive, limit_ns, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+  return GDN_OK;
+}
+
+int gdn_rope_eval(int npos, int D, float rope_base, int reduced, float* cs, gdn_stream_t stream) {
+  t_last_error.clear();
+  if (!cs || !aligned16(cs)) return fail(GDN_ERR_INVALID, "cs must be a 16-byte aligned device pointer%s");
+  if (npos < 1 || npos > (1 << 20) || !valid_D(D) || !(rope_base > 1.0f))
+    return fail(GDN_ERR_INVALID, "need 1 <= npos <= 2^20, a supported D and rope_base > 1%s");
+  const float base = rope_base;
+  cudaError_t e = reduced ? rope_reduced((float2*)cs, npos, D, base, (cudaStream_t)stream)
+                          : rope_table((float2*)cs, npos, D, base, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "rope eval launch");
   return GDN_OK;
 }
 

@@ -175,6 +175,7 @@ struct ProArgs {
 // (cos, sin) table, pair-major: cs[i * npos + pos], pos < npos, i < D/4
 // (consecutive tokens of a row read consecutive entries).
 cudaError_t rope_table(float2* cs, int npos, int D, float base, cudaStream_t st);
+cudaError_t rope_reduced(float2* cs, int npos, int D, float base, cudaStream_t st);
 
 // Largest max(grid_h, grid_w) the fused prologue's shared-memory table holds (D = 128).
 int tc_prologue_max_positions();

@@ -82,6 +82,27 @@ static int num_sms() {
   return n;
 }
 
+// Kernel attributes such as the dynamic shared-memory limit belong to the
+// kernel as loaded on one device, so each launch site sets them once per
+// device: one bit per device, a mutex for concurrent host threads.
+struct DeviceOnce {
+  std::mutex mu;
+  unsigned long long done = 0;
+};
+
+template <class F>
+static cudaError_t once_per_device(DeviceOnce& o, F&& set) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(o.mu);
+  if ((o.done >> dev) & 1ull) return cudaSuccess;
+  e = set();
+  if (e == cudaSuccess) o.done |= 1ull << dev;
+  return e;
+}
+
 // Rounds the dynamic shared-memory base up to 1024 bytes (the 128-byte
 // swizzle atom repeats every 1024). The offset is added to the pointer itself,
 // so the compiler still knows the result addresses shared memory and emits
@@ -120,13 +141,35 @@ __device__ __forceinline__ void warp_arrive(uint32_t bar) {
 // (w[32q + 2p], w[32q + 2p + 1]), so the four quarters' threads of a warp read
 // 32 adjacent bytes. RoPE: pair i of a half (i < 32) turns by pos * theta_i,
 // pos the token's row (channels below 64) or column (above). With `theta`
-// (shared memory, the 32 frequencies) the (cos, sin) is computed: the angle
-// is reduced to [-pi, pi] (2 pi split in two parts) and evaluated with the
-// hardware sine/cosine, whose error on that range is near 1e-6 -- below the
-// bf16 rounding the result gets. Otherwise it is read from `tab`, a shared
-// copy of the table laid out by pro_table_index. THETA and BTILE are template
-// flags so that the unrolled pair loop holds no branches.
+// (shared memory, the 32 frequencies) the (cos, sin) is computed by
+// rope_cs_reduced. Otherwise it is read from `tab`, a shared copy of the
+// table laid out by pro_table_index. THETA and BTILE are template flags so
+// that the unrolled pair loop holds no branches.
 // ----------------------------------------------------------------------------
+// Frequency of pair i of an axis half of D/2 channels: base^(-2i/(D/2)).
+__device__ __forceinline__ float rope_theta(float base, int i, int D) {
+  return powf(base, -2.0f * (float)i / (float)(D / 2));
+}
+
+// (cos, sin) of ang = pos * theta for the hardware sine/cosine, which is
+// accurate only near zero. The angle is first brought to [-pi, pi] by
+// Cody-Waite reduction (W. J. Cody and W. Waite, "Software Manual for the
+// Elementary Functions", 1980): k = rint(ang / 2pi), then ang - k * C1 - k * C2
+// with 2pi = C1 + C2, C1 the fp32 nearest 2pi and C2 the remainder. Each step
+// is a fused multiply-add, rounded once on a result already near zero, so C1
+// needs no shortened mantissa. The error is then about 1e-6 plus the fp32
+// rounding of pos * theta (2^-24 of the angle), below the bf16 rounding the
+// prologue's result gets.
+__device__ __forceinline__ float2 rope_cs_reduced(int pos, float theta) {
+  float ang = (float)pos * theta;
+  const float k = rintf(ang * 0.159154943091895f);  // 1 / (2 pi)
+  ang = fmaf(-k, 6.28318548202514648f, ang);         // C1 = 2 pi rounded to fp32
+  ang = fmaf(-k, -1.7484555314695172e-7f, ang);      // C2 = 2 pi - C1
+  float2 cs;
+  __sincosf(ang, &cs.y, &cs.x);
+  return cs;
+}
+
 constexpr int PRO_POS_PITCH = 80;  // positions per pair in the shared table (the most supported)
 __device__ __forceinline__ int pro_table_index(int i, int pos) {
   // pairs i and i + 16 of one position are neighbours, positions of one pair
@@ -209,11 +252,7 @@ __device__ __forceinline__ void pro_rows(uint8_t* tile, int box_bytes, const int
         const float a = fmaxf(m.x, 0.f), b = fmaxf(m.y, 0.f);
         float2 t;
         if (THETA) {
-          float ang = (float)pos[k] * theta[pb + p];
-          const float kq = rintf(ang * 0.159154943091895f);  // 1 / (2 pi)
-          ang = fmaf(-kq, 6.28318548202514648f, ang);        // 2 pi, high part
-          ang = fmaf(-kq, -1.7484555314695172e-7f, ang);     // 2 pi, low part
-          __sincosf(ang, &t.y, &t.x);
+          t = rope_cs_reduced(pos[k], theta[pb + p]);
         } else {
           t = trow[k][p * 2 * PRO_POS_PITCH];
         }
@@ -257,16 +296,33 @@ __global__ void k_rope_table(float2* cs, int npos, int D, float base) {
   const int n = npos * (D / 4);
   for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += gridDim.x * blockDim.x) {
     const int i = e / npos, pos = e % npos;
-    const float theta = powf(base, -2.0f * (float)i / (float)(D / 2));
+    const float theta = rope_theta(base, i, D);
     float sn, c;
     sincosf((float)pos * theta, &sn, &c);
     cs[e] = make_float2(c, sn);
   }
 }
 
+// The same layout as k_rope_table, through rope_cs_reduced (the path the
+// bidirectional readout's prologue takes); for tests of its accuracy.
+__global__ void k_rope_reduced(float2* cs, int npos, int D, float base) {
+  const int n = npos * (D / 4);
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += gridDim.x * blockDim.x) {
+    const int i = e / npos, pos = e % npos;
+    cs[e] = rope_cs_reduced(pos, rope_theta(base, i, D));
+  }
+}
+
 cudaError_t rope_table(float2* cs, int npos, int D, float base, cudaStream_t st) {
   const int n = npos * (D / 4);
   k_rope_table<<<(n + 255) / 256, 256, 0, st>>>(cs, npos, D, base);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t rope_reduced(float2* cs, int npos, int D, float base, cudaStream_t st) {
+  const int n = npos * (D / 4);
+  k_rope_reduced<<<(n + 255) / 256, 256, 0, st>>>(cs, npos, D, base);
   count_launch();
   return cudaGetLastError();
 }
@@ -658,16 +714,16 @@ static cudaError_t tc_contract128(const void* k, const void* v, const float* bet
   if (e != cudaSuccess) return e;
   e = make_map_bf16_3d(&mv, v, D, S, N, 64, ctr::TOK);
   if (e != cudaSuccess) return e;
-  static bool attr = false;
-  if (!attr) {
-    e = cudaFuncSetAttribute(k_contract_tc<ctr::NST_PLAIN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  static DeviceOnce attr_once;
+  const cudaError_t attr_status = once_per_device(attr_once, [&]() -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(k_contract_tc<ctr::NST_PLAIN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              ctr::SMEM_PLAIN);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_contract_tc<ctr::NST_PRO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                ctr::SMEM_PRO);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (attr_status != cudaSuccess) return attr_status;
   const long long units = N * parts;
   const int grid = (int)(units < num_sms() ? units : num_sms());
   if (pro)
@@ -951,13 +1007,13 @@ static int readout_parts(long long N, int ntile) {
 template <bool PRO, bool TRANS = false>
 static cudaError_t launch_readout(const CUtensorMap& mq, const CUtensorMap& ms, const CUtensorMap& mo,
                                   long long N, int S, const ProArgs& pa, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
+  static DeviceOnce attr_once;
+  const cudaError_t attr_status = once_per_device(attr_once, [&]() -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(k_readout_tc<PRO, TRANS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          rdo::SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (attr_status != cudaSuccess) return attr_status;
   const int parts = readout_parts(N, (S + rdo::TOK - 1) / rdo::TOK);
   const long long units = N * parts;
   const int grid = (int)(units < num_sms() ? units : num_sms());
@@ -1757,13 +1813,13 @@ cudaError_t tc_scan_readout(const ChainArgs& a, int nchains, const void* q, void
   const long long N = (long long)a.heads * a.T;
   cudaError_t e = make_map_bf16_3d(&mq, q, 128, S, N, 64, sro::TOK);
   if (e != cudaSuccess) return e;
-  static bool attr = false;
-  if (!attr) {
-    e = cudaFuncSetAttribute(k_scan_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  static DeviceOnce attr_once;
+  const cudaError_t attr_status = once_per_device(attr_once, [&]() -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(k_scan_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              sro::SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (attr_status != cudaSuccess) return attr_status;
   const int grid = nchains < num_sms() ? nchains : num_sms();
   k_scan_readout_tc<<<grid, sro::THREADS, sro::SMEM, st>>>(a, mq, (__nv_bfloat16*)out, S, nchains);
   count_launch();
@@ -1789,13 +1845,13 @@ static cudaError_t make_map_f32_mats(CUtensorMap* m, const void* base, uint64_t 
 static cudaError_t tc_chain128(const ChainArgs& a, int nchains, cudaStream_t st) {
   if (a.D != 128 || !a.y_image) return cudaErrorNotSupported;
   if (a.mode == CHAIN_SCAN && !a.sfr_hilo) return cudaErrorNotSupported;
-  static bool attr = false;
-  if (!attr) {
+  static DeviceOnce attr_once;
+  const cudaError_t attr_status = once_per_device(attr_once, [&]() -> cudaError_t {
     cudaError_t e =
         cudaFuncSetAttribute(k_chain_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, chn::SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (attr_status != cudaSuccess) return attr_status;
   const long long frames = (long long)a.heads * a.T;
   CUtensorMap mz, ms;
   cudaError_t e;
@@ -2141,16 +2197,16 @@ cudaError_t tc_contract_scan(const void* k, const void* v, const float* beta, fl
     e = make_map_bf16_3d(&ms1, sfr1 ? sfr1 : sfr0, 128, 128, 2 * (uint64_t)N, 64, 128);
   if (e != cudaSuccess) return e;
   constexpr int smem_plain = ovl::smem(ctr::SMEM_PLAIN), smem_pro = ovl::smem(ctr::SMEM_PRO);
-  static bool attr = false;
-  if (!attr) {
-    e = cudaFuncSetAttribute(k_contract_scan_tc<ctr::NST_PLAIN>,
+  static DeviceOnce attr_once;
+  const cudaError_t attr_status = once_per_device(attr_once, [&]() -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(k_contract_scan_tc<ctr::NST_PLAIN>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem_plain);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_contract_scan_tc<ctr::NST_PRO>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, smem_pro);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (attr_status != cudaSuccess) return attr_status;
   long long ncon = num_sms() - nchain;
   if (ncon > N) ncon = N;
   const int grid = nchain + (int)ncon;
@@ -2842,13 +2898,13 @@ static cudaError_t make_map_f32_mats64(CUtensorMap* m, const void* base, uint64_
 
 static cudaError_t tc_chain64(const ChainArgs& a, int nchains, cudaStream_t st) {
   if (a.mode == CHAIN_SCAN && !a.sfr_hilo) return cudaErrorNotSupported;
-  static bool attr = false;
-  if (!attr) {
+  static DeviceOnce attr_once;
+  const cudaError_t attr_status = once_per_device(attr_once, [&]() -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(k_chain64_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          h64::SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (attr_status != cudaSuccess) return attr_status;
   const long long frames = (long long)a.heads * a.T;
   CUtensorMap mz, ms;
   cudaError_t e = a.mode == CHAIN_PREFIX ? make_map_f32_mats64(&mz, a.Hc, (uint64_t)a.heads * a.nseg)
@@ -2937,7 +2993,7 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
   }
   if (PRO) pro_w_copy((float2*)(smem + OFF_W), pro.w);
   if (PRO && threadIdx.x < D / 4)  // pair frequencies, as the (cos, sin) table has them
-    ((float*)(smem + OFF_TH))[threadIdx.x] = powf(pro.base, -2.0f * (float)threadIdx.x / (float)(D / 2));
+    ((float*)(smem + OFF_TH))[threadIdx.x] = rope_theta(pro.base, threadIdx.x, D);
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
     tmem_relinquish();
@@ -3129,13 +3185,13 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
 template <bool PRO>
 static cudaError_t launch_readout2(const CUtensorMap* m, long long N, int S, const ProArgs& pa,
                                    cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
+  static DeviceOnce attr_once;
+  const cudaError_t attr_status = once_per_device(attr_once, [&]() -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(k_readout2_tc<PRO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          rd2::SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (attr_status != cudaSuccess) return attr_status;
   const int parts = readout_parts(N, (S + rd2::TOK - 1) / rd2::TOK);
   const long long units = N * parts;
   const int grid = (int)(units < num_sms() ? units : num_sms());
@@ -3605,12 +3661,12 @@ static cudaError_t tc_contract256(const void* k, const void* v, const float* bet
   if (e != cudaSuccess) return e;
   e = make_map_bf16_3d(&mv, v, 256, S, N, 64, c256::TOK);
   if (e != cudaSuccess) return e;
-  static bool attr = false;
-  if (!attr) {
-    e = cudaFuncSetAttribute(k_contract256_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, c256::SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static DeviceOnce attr_once;
+  const cudaError_t attr_status = once_per_device(attr_once, [&]() -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(k_contract256_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, c256::SMEM);
+    return e;
+  });
+  if (attr_status != cudaSuccess) return attr_status;
   const long long units = 2 * N;
   const int grid = (int)(units < num_sms() ? units : num_sms());
   k_contract256_tc<<<grid, c256::THREADS, c256::SMEM, st>>>(mk, mv, beta, A, U, (int)N, S, cA, cU,
@@ -3626,12 +3682,12 @@ static cudaError_t tc_readout256(const void* q, const void* Sfr_hilo, void* out,
   if (e == cudaSuccess) e = make_map_bf16_3d(&ms, Sfr_hilo, 256, 256, 2 * N, 64, 128);
   if (e == cudaSuccess) e = make_map_bf16_3d(&mo, out, 256, S, N, 64, r256::TOK);
   if (e != cudaSuccess) return e;
-  static bool attr = false;
-  if (!attr) {
-    e = cudaFuncSetAttribute(k_readout256_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, r256::SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static DeviceOnce attr_once;
+  const cudaError_t attr_status = once_per_device(attr_once, [&]() -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(k_readout256_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, r256::SMEM);
+    return e;
+  });
+  if (attr_status != cudaSuccess) return attr_status;
   const long long units = 2 * N;
   const int grid = (int)(units < num_sms() ? units : num_sms());
   k_readout256_tc<<<grid, r256::THREADS, r256::SMEM, st>>>(mq, ms, mo, (int)N, S);
@@ -3914,13 +3970,13 @@ __global__ void __launch_bounds__(ch2::THREADS, 1)
 static cudaError_t tc_chain256(const ChainArgs& a, int nchains, cudaStream_t st) {
   if (a.D != 256 || !a.y_image || a.mode != CHAIN_SCAN || !a.sfr_hilo) return cudaErrorNotSupported;
   if (a.seg == SEG_CHUNKS && a.nseg > 1) return cudaErrorNotSupported;  // span starts need the prefix
-  static bool attr = false;
-  if (!attr) {
+  static DeviceOnce attr_once;
+  const cudaError_t attr_status = once_per_device(attr_once, [&]() -> cudaError_t {
     cudaError_t e =
         cudaFuncSetAttribute(k_chain256_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, ch2::SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (attr_status != cudaSuccess) return attr_status;
   const long long frames = (long long)a.heads * a.T;
   CUtensorMap ms;
   cudaError_t e = make_map_bf16_3d(&ms, a.Sfr, 256, 256, 2 * (uint64_t)frames, 64, 128);
@@ -4204,12 +4260,12 @@ cudaError_t tc_bwd_tokens(const void* k, const void* v, const float* beta, const
   if (e == cudaSuccess) e = make_map_bf16_3d(&mdk, dk, 128, S, N, 64, btk::TOK);
   if (e == cudaSuccess) e = make_map_bf16_3d(&mdv, dv, 128, S, N, 64, btk::TOK);
   if (e != cudaSuccess) return e;
-  static bool attr = false;
-  if (!attr) {
-    e = cudaFuncSetAttribute(k_bwd_tok_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, btk::SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static DeviceOnce attr_once;
+  const cudaError_t attr_status = once_per_device(attr_once, [&]() -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(k_bwd_tok_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, btk::SMEM);
+    return e;
+  });
+  if (attr_status != cudaSuccess) return attr_status;
   const int grid = (int)(N < num_sms() ? N : num_sms());
   k_bwd_tok_tc<<<grid, btk::THREADS, btk::SMEM, st>>>(mk, mv, mdk, mdv, beta,
                                                       (const uint8_t*)bimg, dbeta, (int)N, S, c);
@@ -4470,12 +4526,12 @@ cudaError_t tc_bwd_frames(const void* Sfr_hilo, const float* state_in, void* s0_
   if (e == cudaSuccess) e = make_map_bf16_3d(&mz, zero_hilo, 128, 128, 2, 64, 128);
   if (e == cudaSuccess) e = make_map_bf16_3d(&mg, G_hilo, 128, 128, 2 * (uint64_t)N, 64, 128);
   if (e != cudaSuccess) return e;
-  static bool attr = false;
-  if (!attr) {
-    e = cudaFuncSetAttribute(k_bwd_frame_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, bfr::SMEM);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static DeviceOnce attr_once;
+  const cudaError_t attr_status = once_per_device(attr_once, [&]() -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(k_bwd_frame_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, bfr::SMEM);
+    return e;
+  });
+  if (attr_status != cudaSuccess) return attr_status;
   const int grid = (int)(N < num_sms() ? N : num_sms());
   k_bwd_frame_tc<<<grid, bfr::THREADS, bfr::SMEM, st>>>(
       ms, ms0, mz, mg, (const uint8_t*)A_img, (const __nv_bfloat16*)G_hilo, gamma, dgamma,
@@ -4499,12 +4555,12 @@ cudaError_t tc_contract(const void* k, const void* v, const float* beta, float* 
     if (e != cudaSuccess) return e;
     e = make_map_bf16_3d(&mv, v, 64, S, N, 64, c64::TOK);
     if (e != cudaSuccess) return e;
-    static bool attr64 = false;
-    if (!attr64) {
-      e = cudaFuncSetAttribute(k_contract64_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, c64::SMEM);
-      if (e != cudaSuccess) return e;
-      attr64 = true;
-    }
+    static DeviceOnce attr64_once;
+    const cudaError_t attr_status = once_per_device(attr64_once, [&]() -> cudaError_t {
+      cudaError_t e = cudaFuncSetAttribute(k_contract64_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, c64::SMEM);
+      return e;
+    });
+    if (attr_status != cudaSuccess) return attr_status;
     const int grid = (int)(N < num_sms() ? N : num_sms());
     k_contract64_tc<<<grid, c64::THREADS, c64::SMEM, st>>>(mk, mv, beta, A, U, (int)N, S, cA, cU,
                                                             a_image);
@@ -4529,12 +4585,12 @@ cudaError_t tc_readout(const void* q, const void* Sfr_hilo, void* out, long long
     if (e != cudaSuccess) return e;
     e = make_map_bf16_3d(&mo, out, 64, S, N, 64, r64::TOK);
     if (e != cudaSuccess) return e;
-    static bool attr64 = false;
-    if (!attr64) {
-      e = cudaFuncSetAttribute(k_readout64_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, r64::SMEM);
-      if (e != cudaSuccess) return e;
-      attr64 = true;
-    }
+    static DeviceOnce attr64_once;
+    const cudaError_t attr_status = once_per_device(attr64_once, [&]() -> cudaError_t {
+      cudaError_t e = cudaFuncSetAttribute(k_readout64_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, r64::SMEM);
+      return e;
+    });
+    if (attr_status != cudaSuccess) return attr_status;
     const int parts = readout_parts(N, (S + r64::TOK - 1) / r64::TOK);
     const long long units = N * parts;
     const int grid = (int)(units < num_sms() ? units : num_sms());

@@ -212,6 +212,8 @@ GDN_API int gdn_frame_scan_fwd_ex(const gdn_params* p, gdn_stream_t stream);
  * 121-frame rollout does not fit) return GDN_ERR_WORKSPACE before any launch.
  * The first call on each device looks up the array's device address (a
  * one-time runtime query); make that first call before any stream capture.
+ * The address is kept for the life of the process: do not use this entry
+ * point across a cudaDeviceReset, after which the array may move.
  * All calls share the array: calls ordered on one stream are safe, calls that
  * overlap on the GPU (other streams, unordered host threads) race. No part of
  * the scratch has to start at zero: a call writes every byte it reads.
@@ -348,11 +350,34 @@ GDN_API int gdn_check_device_status(gdn_stream_t stream);
  * GDN_ERR_TIMEOUT and the context stays usable. Returns the launch status. */
 GDN_API int gdn_selftest_wait(int arrive, long long limit_ns, gdn_stream_t stream);
 
+/* gdn_rope_eval — the (cos, sin) pairs the fused prologue's 2-D RoPE uses,
+ * for tests of their accuracy: for pair i < D/4 of an axis half and position
+ * pos < npos, writes (cos, sin) of pos * rope_base^(-2i/(D/2)) to
+ * cs[2 * (i * npos + pos)], cs[2 * (i * npos + pos) + 1] (device, fp32,
+ * 16-byte aligned, 2 * npos * D/4 floats). reduced = 0: the table the
+ * contraction and the one-direction readout copy into shared memory (full
+ * precision sine/cosine of the fp32 angle); reduced = 1: the angle reduced to
+ * [-pi, pi] by Cody-Waite reduction and the hardware sine/cosine, as the
+ * bidirectional readout computes them per token. npos in [1, 2^20].
+ * Returns a status. */
+GDN_API int gdn_rope_eval(int npos, int D, float rope_base, int reduced, float* cs,
+                          gdn_stream_t stream);
+
 /* Static description of a status code. */
 GDN_API const char* gdn_status_string(int status);
 
 /* One-line description of the last failure on this host thread ("" if none). */
 GDN_API const char* gdn_last_error(void);
+
+/* gdn_fault_inject — host-side fault injection for tests of the callers'
+ * error paths, with no device fault: the next n calls of gdn_frame_scan_fwd,
+ * gdn_frame_scan_fwd_ex, gdn_frame_scan_fwd_static and gdn_frame_scan_bwd on
+ * this host thread return GDN_ERR_CUDA ("injected launch failure") once their
+ * arguments have passed the checks, before anything is launched (the plain
+ * entry has already taken its stream-ordered workspace, which it frees).
+ * Outputs are left untouched. n <= 0 disarms. Returns the number of injected
+ * failures still pending before this call. */
+GDN_API int gdn_fault_inject(int n);
 
 /* Kernel launches made by this host thread's gdn_* calls since the last reset;
  * reset = 1 clears the counter after reading it. */

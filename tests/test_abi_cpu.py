@@ -72,3 +72,27 @@ def test_product_path_does_not_import_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 txt = open(os.path.join(dirpath, f), encoding="utf-8").read()
                 assert "import oracle" not in txt and "from oracle" not in txt, f
+
+
+def test_fault_injection_fails_before_any_launch(lib):
+    """The armed injection turns the next scan call, once its arguments pass
+    the checks, into GDN_ERR_CUDA without a launch (no GPU needed: the
+    pointers are never dereferenced)."""
+    fake = lambda i: ctypes.c_void_p(0x10000000 + 0x100000 * i)
+    p = api.GdnParams()
+    p.q, p.k, p.v, p.beta, p.gamma, p.out = (fake(i) for i in range(6))
+    p.B, p.H, p.T, p.S, p.D = 1, 2, 3, 64, 128
+    p.flags = api.BF16
+    p.workspace = 0x40000000
+    p.workspace_bytes = api.workspace_bytes(1, 2, 3, 64, 128, api.BF16)
+    assert lib.gdn_fault_inject(1) == 0
+    before = lib.gdn_launch_count(0)
+    assert lib.gdn_frame_scan_fwd_ex(ctypes.byref(p), None) == api.GDN_ERR_CUDA
+    assert b"injected" in lib.gdn_last_error()
+    assert lib.gdn_launch_count(0) == before
+    assert lib.gdn_fault_inject(0) == 0  # consumed by that one call
+    # argument errors still come first: an invalid call does not consume it
+    assert lib.gdn_fault_inject(1) == 0
+    p.out = p.q
+    assert lib.gdn_frame_scan_fwd_ex(ctypes.byref(p), None) == api.GDN_ERR_INVALID
+    assert lib.gdn_fault_inject(0) == 1
