@@ -30,7 +30,10 @@ std::mutex g_mu;
 void* g_ptr[kMaxDevices] = {};
 
 // The device address of the array on the current device, looked up once per
-// device (host code only sees a host-side stand-in for the symbol).
+// device (host code only sees a host-side stand-in for the symbol). The address
+// stays valid for the life of the device's primary context; after a
+// cudaDeviceReset the module may load elsewhere, so this entry point must not
+// be used across a device reset.
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
