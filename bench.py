@@ -367,7 +367,7 @@ def run_ours(args, cfg):
             def step():  # noqa: F811
                 # forward, then the backward from the forward's saved workspace
                 api.frame_scan_fwd_ex(q, k, v, beta, gamma, s0, out=out, state_out=st_out,
-                                      workspace=ws, **kw)
+                                      workspace=ws, save_for_backward=True, **kw)
                 api.frame_scan_bwd(q, k, v, beta, gamma, s0, d_out, d_st, workspace=ws_b,
                                    saved_workspace=ws)
         else:

@@ -35,6 +35,7 @@ BIDIR = 0x80
 FUSED_REPLAY = 0x1000000
 CHUNKED = 0x2000000
 NO_OVERLAP = 0x4000000
+SAVE_FOR_BACKWARD = 0x10000000
 REV_STATE_IN = 0x8000000
 
 
@@ -176,7 +177,8 @@ def _want_states_outputs(q, state_in, out, state_out):
 
 def scan_flags(*, bf16: bool, reverse=False, block_reset=False, block=3, chunk=8,
                sequential=False, keys_scaled=False, force_simt=False, prologue=False,
-               bidir=False, fused_replay=False, chunked=False, overlap=True) -> int:
+               bidir=False, fused_replay=False, chunked=False, overlap=True,
+               save_for_backward=False) -> int:
     """Flag word of the C ABI. Plan: sequential=True forces one chain per head,
     chunked=True the span-composed plan, neither lets the library choose;
     overlap=False keeps the chains out of the contraction's launch."""
@@ -191,6 +193,7 @@ def scan_flags(*, bf16: bool, reverse=False, block_reset=False, block=3, chunk=8
     f |= FORCE_SIMT if force_simt else 0
     f |= FUSED_PROLOGUE if prologue else 0
     f |= BIDIR if bidir else 0
+    f |= SAVE_FOR_BACKWARD if save_for_backward else 0
     return f
 
 
@@ -202,7 +205,7 @@ def frame_scan_fwd_ex(q, k, v, beta, gamma, state_in=None, *, reverse=False, blo
                       block=3, chunk=8, sequential=False, keys_scaled=False, force_simt=False,
                       prologue=None, bidir=False, fused_replay=False, chunked=False,
                       overlap=True, out=None, state_out=None, out_rev=None, state_out_rev=None,
-                      workspace=None, stream=None, state_in_rev=...):
+                      workspace=None, stream=None, state_in_rev=..., save_for_backward=False):
     """The frame scan through gdn_frame_scan_fwd_ex.
 
     q, k, v [B,H,T,S,D] (bf16 or fp32); beta [B,H,T,S] fp32; gamma [B,H,T]
@@ -211,7 +214,8 @@ def frame_scan_fwd_ex(q, k, v, beta, gamma, state_in=None, *, reverse=False, blo
     raw q, k. Returns (out, state_out) or, with bidir, (out, state_out,
     out_rev, state_out_rev). With bidir, state_in_rev (a tensor or None)
     gives the reverse scan its own start state (GDN_REV_STATE_IN); left out,
-    state_in seeds both directions."""
+    state_in seeds both directions. save_for_backward keeps what a later
+    frame_scan_bwd(saved_workspace=workspace) reads (GDN_SAVE_FOR_BACKWARD)."""
     B, H, T, S, D = q.shape
     bf16 = q.dtype == torch.bfloat16
     if q.dtype not in (torch.bfloat16, torch.float32):
@@ -228,7 +232,8 @@ def frame_scan_fwd_ex(q, k, v, beta, gamma, state_in=None, *, reverse=False, blo
     flags = scan_flags(bf16=bf16, reverse=reverse, block_reset=block_reset, block=block,
                        chunk=chunk, sequential=sequential, keys_scaled=keys_scaled,
                        force_simt=force_simt, prologue=prologue is not None, bidir=bidir,
-                       fused_replay=fused_replay, chunked=chunked, overlap=overlap)
+                       fused_replay=fused_replay, chunked=chunked, overlap=overlap,
+                       save_for_backward=save_for_backward)
     out = torch.empty_like(q) if out is None else out
     state_out = torch.empty((B, H, D, D), device=q.device, dtype=torch.float32) \
         if state_out is None else state_out

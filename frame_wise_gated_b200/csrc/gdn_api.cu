@@ -416,6 +416,10 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
     }
     o.a_image = 1;
     o.contract_rev = o.dir[0].reverse && !o.dir[0].blocks_asc;
+    // one chain per head reads each frame's A_t image and U_t once: their L2
+    // lines are dropped after that read instead of being written back (the
+    // A_t images stay for a later gdn_frame_scan_bwd when asked to)
+    if (!bidir) o.discard = 1 | ((f & GDN_SAVE_FOR_BACKWARD) ? 0 : 2);
     {
       PhaseScope ps(PH_CONTRACT_SCAN, st);
       e = tc_contract_scan(k, p.v, p.beta, A, U, frames, p.S, (float)(c * c), (float)c, ppk, o,

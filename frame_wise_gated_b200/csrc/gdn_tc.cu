@@ -461,12 +461,15 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         if (lane == 0) {
+          // K and V are read once: evict-first keeps L2 for the A_t, U_t and
+          // state lines that the chains read back
+          const uint64_t pol = l2_policy_evict_first();
           const uint32_t kd = sb + OFF_K + s * 2 * TILE, vd = kd + TILE;
           mbar_arrive_expect_tx(bar_full + 8 * s, 2 * TILE);
-          tma_load_3d(kd, &tmK, bar_full + 8 * s, 0, st * TOK, n);
-          tma_load_3d(kd + BOX, &tmK, bar_full + 8 * s, 64, st * TOK, n);
-          tma_load_3d(vd, &tmV, bar_full + 8 * s, 0, st * TOK, n);
-          tma_load_3d(vd + BOX, &tmV, bar_full + 8 * s, 64, st * TOK, n);
+          tma_load_3d_hint(kd, &tmK, bar_full + 8 * s, 0, st * TOK, n, pol);
+          tma_load_3d_hint(kd + BOX, &tmK, bar_full + 8 * s, 64, st * TOK, n, pol);
+          tma_load_3d_hint(vd, &tmV, bar_full + 8 * s, 0, st * TOK, n, pol);
+          tma_load_3d_hint(vd + BOX, &tmV, bar_full + 8 * s, 64, st * TOK, n, pol);
         }
         // beta of the stage's tokens: asynchronous 4-byte copies (zeros past S)
         // that arrive on the same barrier, so the loop never waits on them.
@@ -2103,6 +2106,15 @@ __device__ __forceinline__ void ovl_chain_body(const OvlArgs& o, const CUtensorM
       if (leader) fetch_y(sn);
     }
     mbar_wait(bar_z, (uint32_t)j & 1, abort_flag, &g_tc_status, 34);
+    if (o.discard) {
+      // this frame's A_t image and U_t now sit in shared memory and nothing
+      // reads them from global memory again: drop their L2 lines (one 128-byte
+      // line of each per thread) before they are written back
+      const size_t n = (size_t)bh * T + st.t;
+      if ((o.discard & 2) && st.yt >= 0)
+        discard_l2_line(o.A + ((size_t)bh * T + st.yt) * kImageBytes + (size_t)threadIdx.x * 128);
+      if (o.discard & 1) discard_l2_line(o.U + n * (kImageBytes / 4) + (size_t)threadIdx.x * 32);
+    }
     {
       const float alpha = st.at >= 0 ? o.gamma[(size_t)bh * T + st.at] : 1.f;
       uint32_t r[32];
@@ -2217,6 +2229,7 @@ cudaError_t tc_contract_scan(const void* k, const void* v, const float* beta, fl
   int N_a = (int)N, S_a = S, nchain_a = nchain;
   float cA_a = cA, cU_a = cU;
   OvlArgs o_a = o;
+  o_a.U = U;
   void* args[] = {&mk, &mv, &beta_a, &A_a, &U_a, &N_a, &S_a, &cA_a, &cU_a,
                   &pa, &o_a, &nchain_a, &mz, &ms0, &ms1};
   // cooperative: every CTA is resident, so the chains' waits on the

@@ -87,6 +87,11 @@ enum {
                                        state_in_rev (NULL = zeros) instead of state_in */
 #define GDN_NO_OVERLAP 0x4000000u /* run the sequential chains as their own launch after
                                      the contraction instead of alongside it */
+#define GDN_SAVE_FOR_BACKWARD 0x10000000u /* _ex: leave the A_t operand images and the
+                                     states in the workspace for gdn_frame_scan_bwd's
+                                     saved_workspace (otherwise the plan with the chains
+                                     alongside the contraction lets the A_t images go
+                                     once read, so they never cost an HBM write) */
 #define GDN_BLOCK(f) (((f) >> 8) & 0xffu)  /* reset block length; 0 means 3 */
 #define GDN_CHUNK(f) (((f) >> 16) & 0xffu) /* time-chunk length; 0 means 8 */
 #define GDN_MAKE_BLOCK(n) ((((unsigned)(n)) & 0xffu) << 8)
@@ -239,9 +244,10 @@ GDN_API int gdn_frame_scan_fwd_static(const void* q, const void* k, const void* 
  *   dbeta_s = k^_s . (K^ (dA + dA^T) / 2 + V G)_s.
  * Forward quantities (A_t, U_t, the states) are recomputed inside the call,
  * unless saved_workspace is set (tensor-core path: bf16, D = 128): then it
- * must be the workspace of a gdn_frame_scan_fwd_ex call on the same q, k, v,
- * beta, gamma, state_in, sizes, GDN_REVERSE / GDN_BLOCK_RESET / block length,
- * without GDN_BIDIR, GDN_FUSED_PROLOGUE or GDN_FUSED_REPLAY, left untouched
+ * must be the workspace of a gdn_frame_scan_fwd_ex call with
+ * GDN_SAVE_FOR_BACKWARD on the same q, k, v, beta, gamma, state_in, sizes,
+ * GDN_REVERSE / GDN_BLOCK_RESET / block length, without GDN_BIDIR,
+ * GDN_FUSED_PROLOGUE or GDN_FUSED_REPLAY, left untouched
  * since; the backward reads that call's A_t images and states from it and
  * skips the recompute (the saved-for-backward pattern of training). Nothing
  * can check this contract: a stale or foreign workspace gives wrong gradients.

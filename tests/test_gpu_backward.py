@@ -141,7 +141,7 @@ def test_backward_from_saved_forward(fwd_kw):
     ws = torch.empty(api.workspace_bytes(B, H, T, S, D, api.scan_flags(bf16=True, bidir=False)) +
                      (1 << 20), dtype=torch.uint8, device="cuda")
     api.frame_scan_fwd_ex(d["q"], d["k"], d["v"], d["beta"], d["gamma"], d["state"],
-                          workspace=ws, **fwd_kw)
+                          workspace=ws, save_for_backward=True, **fwd_kw)
     rkw = dict(reverse=fwd_kw.get("reverse", False), block_reset=fwd_kw.get("block_reset", False))
     got = api.frame_scan_bwd(d["q"], d["k"], d["v"], d["beta"], d["gamma"], d["state"], d_out,
                              d_s, saved_workspace=ws, **rkw)
