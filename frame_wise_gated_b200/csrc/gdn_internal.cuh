@@ -226,9 +226,9 @@ struct OvlArgs {
   const uint8_t* zero_img;  // adjoint: an all-zero operand image
   int a_image;       // the contraction's A output: 1 operand images, 2 not written
   int contract_rev;  // the contraction visits frames in reverse time
-  const float* U;    // U_t [heads*T][D][D] (set by tc_contract_scan; used by `discard`)
+  const float* U;    // U_t [heads*T][D][D] (set by tc_contract_scan)
   int discard;       // one direction only: once a chain has copied a frame's operands
-                     // it drops their L2 lines unwritten: 1 = U_t, 2 = the A_t image
+                     // their L2 lines are dropped unwritten: 1 = U_t, 2 = the A_t image
 };
 
 bool tc_overlap_supported(int D);

@@ -365,6 +365,37 @@ constexpr int SMEM_PRO = Lay<NST_PRO>::SMEM_PRO;
 static_assert(SMEM_PLAIN <= 232448 && SMEM_PRO <= 232448, "contraction shared memory");
 }  // namespace ctr
 
+// Frame-head n's A_t image (discard & 2) and U_t (discard & 1) are read once, by
+// its chain, which then adds a fifth count to flags[n]. Once that count is
+// there, epilogue warp q drops its quarter of their L2 lines without a write
+// back. With `wait` the warp polls for the count for at most 100 us; otherwise
+// it looks once. A line that is not dropped is simply written back later.
+__device__ __forceinline__ void drop_consumed(float* A, float* U, const int* flags, int n, int q,
+                                             int lane, int discard, int wait) {
+  int ok = 0;
+  if (lane == 0) {
+    const unsigned long long t0 = wait ? globaltimer() : 0ull;
+    for (;;) {
+      int v;
+      asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(flags + n) : "memory");
+      if (v >= 5) {
+        ok = 1;
+        break;
+      }
+      if (!wait || globaltimer() - t0 > 100000ull) break;
+      __nanosleep(256);
+    }
+  }
+  if (!__shfl_sync(0xffffffffu, ok, 0)) return;
+  const size_t base = (size_t)n * kImageBytes + (size_t)q * (kImageBytes / 4);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {  // 4 lines of 128 bytes per lane: the warp's 16 KiB quarter
+    const size_t off = base + (size_t)(j * 32 + lane) * 128;
+    if (discard & 2) discard_l2_line((const uint8_t*)A + off);
+    if (discard & 1) discard_l2_line((const uint8_t*)U + off);
+  }
+}
+
 // Body of the contraction for CTA `cta` of `ncta` contraction CTAs. Units are
 // frame-heads in order n, or, when `heads` > 0, in scan order across heads
 // (unit u -> head u % heads, scan position u / heads of T: frame u / heads, or
@@ -382,7 +413,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
                                               float* __restrict__ U, int N, int S, float cA,
                                               float cU, int a_image, const ProArgs& pro, int cta,
                                               int ncta, int heads, int T, int rev, int* flags,
-                                              int parts = 1) {
+                                              int parts = 1, int discard = 0) {
   using namespace ctr;
   using Ly = Lay<NST>;
   constexpr int NBK = Ly::NBK;
@@ -665,8 +696,13 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
         __syncwarp();
         if (lane == 0)
           asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(flags + n), "r"(1) : "memory");
+        // the previous unit's A_t image and U_t, once its chain has copied them
+        // (count 5: 4 publications + 1 consumption), are never read again
+        if (discard && i > 0) drop_consumed(A, U, flags, unit_n(i - 1), q, lane, discard, 0);
       }
     }
+    // this CTA's last unit: its chain reads it shortly; wait for that a while
+    if (discard && my_count > 0) drop_consumed(A, U, flags, unit_n(my_count - 1), q, lane, discard, 1);
   }
 
   tc_fence_before();
@@ -2106,14 +2142,13 @@ __device__ __forceinline__ void ovl_chain_body(const OvlArgs& o, const CUtensorM
       if (leader) fetch_y(sn);
     }
     mbar_wait(bar_z, (uint32_t)j & 1, abort_flag, &g_tc_status, 34);
-    if (o.discard) {
-      // this frame's A_t image and U_t now sit in shared memory and nothing
-      // reads them from global memory again: drop their L2 lines (one 128-byte
-      // line of each per thread) before they are written back
-      const size_t n = (size_t)bh * T + st.t;
-      if ((o.discard & 2) && st.yt >= 0)
-        discard_l2_line(o.A + ((size_t)bh * T + st.yt) * kImageBytes + (size_t)threadIdx.x * 128);
-      if (o.discard & 1) discard_l2_line(o.U + n * (kImageBytes / 4) + (size_t)threadIdx.x * 32);
+    if (o.discard && leader) {
+      // this frame's A_t image and U_t now sit in shared memory: one more count
+      // on its flag tells the contraction CTA that wrote them that their L2
+      // lines can go unwritten (it drops them off this chain's critical path)
+      asm volatile("red.relaxed.gpu.global.add.s32 [%0], %1;" ::"l"(o.flags + (size_t)bh * T + st.t),
+                   "r"(1)
+                   : "memory");
     }
     {
       const float alpha = st.at >= 0 ? o.gamma[(size_t)bh * T + st.at] : 1.f;
@@ -2183,7 +2218,7 @@ __global__ void __launch_bounds__(ovl::THREADS, 1)
   else
     contract_body<NST>(tmK, tmV, beta, A, U, N, S, cA, cU, o.a_image, pro,
                        (int)blockIdx.x - nchain, (int)gridDim.x - nchain, o.heads, o.T,
-                       o.contract_rev, o.flags);
+                       o.contract_rev, o.flags, 1, o.discard);
 }
 
 bool tc_overlap_supported(int D) { return D == 128; }
