@@ -43,6 +43,12 @@ Readings where the pages are silent (each is listed in the design notes):
       only) the key scale, then a 2-D spatial RoPE: token s = y*W + x; channels
       [0, D/2) rotate with y, [D/2, D) with x; inside each half the pairs
       (2i, 2i+1), i < D/4, turn by pos * base^(-2i/(D/2)).
+  R20 camera encoding (UCPE): the caller gives each token's 4 x 4 matrices,
+      D_{t,s}^T for queries and D_{t,s}^-1 for keys (D_{t,s}: world -> the
+      token's ray-local frame), shared by all heads; a query-key product then
+      depends on D_i D_j^-1 only, not on the world frame.
+  R21 "combined orthogonally with RoPE": on separate channels; the camera
+      blocks of 4 take [0, D/2), the 2-D RoPE (R10 on D/2 channels) [D/2, D).
 
 Pins (tests/test_oracle_pins.py) and their status per function:
   frame_scan / gdn_frame_scan   pinned (token-wise reduction, delta-rule
@@ -59,6 +65,15 @@ Pins (tests/test_oracle_pins.py) and their status per function:
                                 axis split, the pair layout and the turn
                                 direction). The constants themselves are
                                 readings R8-R10: the pages do not fix them.
+  ucpe_rope                     pinned by a hand-worked fixture (a quarter
+                                turn of one block plus RoPE on the rest),
+                                the identity transform reducing to rope2d on
+                                the upper half, invariance of every
+                                query-key product under a change of world
+                                frame, and norm preservation for rotations.
+                                The transform's source (ray-local frames
+                                from poses) is the caller's, readings
+                                R20-R21.
   frame_scan_bwd                the pages print no backward; this is the
                                 adjoint of frame_scan derived by reverse-mode
                                 differentiation, pinned by central finite
@@ -82,6 +97,7 @@ __all__ = [
     "chunked_frame_scan",
     "token_wise_gdn",
     "rmsnorm",
+    "ucpe_rope",
     "relu",
     "rope2d",
     "qk_prologue",
@@ -306,14 +322,41 @@ def rope2d(x, grid_w, base=10000.0):
     return out
 
 
-def qk_prologue(q_raw, k_raw, w_q, w_k, grid_w, *, eps=1e-6, base=10000.0):
+def ucpe_rope(x, M, grid_w, base=10000.0):
+    """Camera encoding composed with the 2-D RoPE on separate channels
+    ([HD] section 双分支相机控制: a per-token homogeneous transform D_{t,s}
+    from world to the token's ray-local frame, combined orthogonally with
+    RoPE; [JY] 2.3; readings R20-R21).
+
+    x: [..., S, D]; M: [..., S, 4, 4], the matrix applied to this side's
+    tokens (queries take D_{t,s}^T, keys D_{t,s}^-1, so that a query-key
+    product sees D_i D_j^-1 only). Channels [0, D/2) form D/8 blocks of 4
+    (block b = channels 4b .. 4b+3); each block of token s becomes M[s] times
+    it. Channels [D/2, D) get rope2d as a vector of D/2 channels (its y half
+    first, then its x half)."""
+    x = np.array(x, np.float64)
+    M = np.asarray(M, np.float64)
+    D = x.shape[-1]
+    h = D // 2
+    out = x.copy()
+    for b in range(h // 4):
+        blk = x[..., 4 * b:4 * b + 4]
+        out[..., 4 * b:4 * b + 4] = np.einsum("...ij,...j->...i", M, blk)
+    out[..., h:] = rope2d(x[..., h:], grid_w, base)
+    return out
+
+
+def qk_prologue(q_raw, k_raw, w_q, w_k, grid_w, *, eps=1e-6, base=10000.0, ucpe=None):
     """Prologue in the pages' order ([HD] 显存分片 section; readings R8-R10):
-    RMSNorm -> ReLU -> key scale 1/sqrt(D*S) (keys only) -> 2-D RoPE.
+    RMSNorm -> ReLU -> key scale 1/sqrt(D*S) (keys only) -> 2-D RoPE, or,
+    with ucpe = (M_q, M_k) ([..., S, 4, 4] each), -> ucpe_rope.
     q_raw, k_raw: [..., S, D]. Returns (q^, k^); k^ carries the key scale."""
     S, D = np.shape(q_raw)[-2], np.shape(q_raw)[-1]
-    qh = rope2d(relu(rmsnorm(q_raw, w_q, eps)), grid_w, base)
-    kh = rope2d(key_scale(D, S) * relu(rmsnorm(k_raw, w_k, eps)), grid_w, base)
-    return qh, kh
+    qn = relu(rmsnorm(q_raw, w_q, eps))
+    kn = key_scale(D, S) * relu(rmsnorm(k_raw, w_k, eps))
+    if ucpe is None:
+        return rope2d(qn, grid_w, base), rope2d(kn, grid_w, base)
+    return ucpe_rope(qn, ucpe[0], grid_w, base), ucpe_rope(kn, ucpe[1], grid_w, base)
 
 
 # ---------------------------------------------------------------------------

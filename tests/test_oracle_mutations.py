@@ -171,3 +171,62 @@ def test_pins_catch_rmsnorm_mutation(mutation):
                                       "rotate_half_pairs"])
 def test_pins_catch_rope_mutation(mutation):
     assert not prologue_pins_pass(make_rmsnorm(None), make_rope2d(mutation))
+
+
+# --- the camera encoding: planted mistakes in copies of ucpe_rope ------------
+
+def make_ucpe(mutation):
+    def ucpe_rope(x, M, grid_w, base=10000.0):
+        x = np.array(x, np.float64)
+        M = np.asarray(M, np.float64)
+        if mutation == "transposed":
+            M = np.swapaxes(M, -1, -2)
+        D = x.shape[-1]
+        h = D // 2
+        lo, hi = (slice(h, D), slice(0, h)) if mutation == "halves_swapped" else (slice(0, h), slice(h, D))
+        out = x.copy()
+        xs = x[..., lo]
+        ys = out[..., lo]
+        for b in range(h // 4):
+            if mutation == "strided_blocks":   # block b = channels b, b + D/8, ... instead of 4b..4b+3
+                idx = [b + j * (h // 4) for j in range(4)]
+            else:
+                idx = list(range(4 * b, 4 * b + 4))
+            ys[..., idx] = np.einsum("...ij,...j->...i", M, xs[..., idx])
+        out[..., lo] = ys
+        out[..., hi] = O.rope2d(x[..., hi], grid_w, base)
+        return out
+    return ucpe_rope
+
+
+def ucpe_pins_pass(fn):
+    g = json.load(open(os.path.join(GOLD, "ucpe_rope_d8.json")))
+    x = np.zeros((g["S"], g["D"]))
+    x[g["token"]] = g["x_in"]
+    M = np.tile(np.eye(4), (g["S"], 1, 1))
+    M[g["token"]] = g["M"]
+    ok = np.allclose(fn(x, M, g["grid_w"], g["base"])[g["token"]], g["expected"], atol=1e-12)
+    rng = np.random.default_rng(43)
+    x = rng.standard_normal((6, 32))
+    y = fn(x, np.tile(np.eye(4), (6, 1, 1)), 3)
+    ok &= np.array_equal(y[:, :16], x[:, :16]) and np.allclose(y[:, 16:], O.rope2d(x[:, 16:], 3))
+    # index loops at D = 16: two camera blocks of 4 consecutive channels
+    x, M = rng.standard_normal((6, 16)), rng.standard_normal((6, 4, 4))
+    y = fn(x, M, 3)
+    for s_ in range(6):
+        for b in range(2):
+            for i in range(4):
+                ok &= abs(y[s_][4 * b + i] - sum(M[s_][i][j] * x[s_][4 * b + j] for j in range(4))) < 1e-12
+    return bool(ok)
+
+
+def test_unmutated_ucpe_copy_passes():
+    assert ucpe_pins_pass(make_ucpe(None))
+    rng = np.random.default_rng(44)
+    x, M = rng.standard_normal((6, 32)), rng.standard_normal((6, 4, 4))
+    np.testing.assert_allclose(make_ucpe(None)(x, M, 3), O.ucpe_rope(x, M, 3), rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("mutation", ["transposed", "halves_swapped", "strided_blocks"])
+def test_pins_catch_ucpe_mutation(mutation):
+    assert not ucpe_pins_pass(make_ucpe(mutation))

@@ -381,3 +381,95 @@ def test_prologue_order_and_key_scale():
     assert np.all(np.abs(np.linalg.norm(qh, axis=-1) -
                          np.linalg.norm(O.relu(O.rmsnorm(q, wq)), axis=-1)) < 1e-12)
     np.testing.assert_allclose(kh[0], k_pre[0], atol=1e-15)    # token 0: no rotation
+
+
+# --- camera encoding (UCPE) composed with the RoPE ----------------------------
+
+def _rigid(rng):
+    """A random rigid transform [[R, t], [0, 1]] (R a rotation)."""
+    R, _ = np.linalg.qr(rng.standard_normal((3, 3)))
+    if np.linalg.det(R) < 0:
+        R[:, 0] *= -1
+    T = np.eye(4)
+    T[:3, :3] = R
+    T[:3, 3] = 0.5 * rng.standard_normal(3)
+    return T
+
+
+def test_ucpe_golden():
+    """Hand-worked (derivation in the fixture): a quarter turn with a shift on
+    the camera block, RoPE on the other half."""
+    g = json.load(open(os.path.join(GOLD, "ucpe_rope_d8.json")))
+    x = np.zeros((g["S"], g["D"]))
+    x[g["token"]] = g["x_in"]
+    M = np.tile(np.eye(4), (g["S"], 1, 1))
+    M[g["token"]] = g["M"]
+    y = O.ucpe_rope(x, M, g["grid_w"], g["base"])
+    np.testing.assert_allclose(y[g["token"]], g["expected"], rtol=0, atol=1e-12)
+
+
+def test_ucpe_identity_is_rope_on_upper_half():
+    rng = np.random.default_rng(40)
+    W, Hh, D = 5, 3, 32
+    S = W * Hh
+    x = rng.standard_normal((S, D))
+    y = O.ucpe_rope(x, np.tile(np.eye(4), (S, 1, 1)), W)
+    np.testing.assert_array_equal(y[:, :D // 2], x[:, :D // 2])
+    np.testing.assert_allclose(y[:, D // 2:], O.rope2d(x[:, D // 2:], W), rtol=0, atol=0)
+
+
+def test_ucpe_scores_do_not_depend_on_the_world_frame():
+    """Queries take D^T and keys D^-1 per token: every query-key product then
+    depends on D_i D_j^-1 only, so moving the world frame (D -> D G^-1 for
+    all tokens) leaves all products unchanged; a different world motion per
+    token does not."""
+    rng = np.random.default_rng(41)
+    W, Hh, D = 4, 3, 16
+    S = W * Hh
+    q, k = rng.standard_normal((S, D)), rng.standard_normal((S, D))
+    Dm = np.stack([_rigid(rng) for _ in range(S)])
+    G = np.linalg.inv(_rigid(rng))
+
+    def scores(Dm):
+        qh = O.ucpe_rope(q, np.transpose(Dm, (0, 2, 1)), W)
+        kh = O.ucpe_rope(k, np.linalg.inv(Dm), W)
+        return qh @ kh.T
+
+    base = scores(Dm)
+    np.testing.assert_allclose(scores(Dm @ G), base, rtol=1e-10, atol=1e-10)
+    Dm2 = Dm.copy()
+    Dm2[3] = Dm2[3] @ G
+    assert not np.allclose(scores(Dm2), base, atol=1e-6)
+
+
+def test_ucpe_rotations_preserve_norms_and_prologue_uses_both_sides():
+    rng = np.random.default_rng(42)
+    W, Hh, D = 4, 2, 16
+    S = W * Hh
+    R = np.stack([_rigid(rng) for _ in range(S)])
+    R[:, :3, 3] = 0.0                       # pure rotations: M^T = M^-1
+    x = rng.standard_normal((S, D))
+    y = O.ucpe_rope(x, R, W)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-12)
+    q, k = rng.standard_normal((S, D)), rng.standard_normal((S, D))
+    w = 0.5 + rng.random(D)
+    Mq, Mk = np.transpose(R, (0, 2, 1)), np.linalg.inv(R)
+    qh, kh = O.qk_prologue(q, k, w, w, W, ucpe=(Mq, Mk))
+    np.testing.assert_allclose(qh, O.ucpe_rope(O.relu(O.rmsnorm(q, w)), Mq, W), rtol=1e-13)
+    np.testing.assert_allclose(kh, O.ucpe_rope(O.key_scale(D, S) * O.relu(O.rmsnorm(k, w)), Mk, W),
+                               rtol=1e-13)
+
+
+def test_ucpe_blocks_by_index_loops():
+    """Brute force at D = 16 (two camera blocks): out[4b + i] = sum_j M[i][j] x[4b + j]."""
+    rng = np.random.default_rng(45)
+    S, D = 6, 16
+    x, M = rng.standard_normal((S, D)), rng.standard_normal((S, 4, 4))
+    y = O.ucpe_rope(x, M, 3)
+    for s_ in range(S):
+        for b in range(D // 8):
+            for i in range(4):
+                acc = 0.0
+                for j in range(4):
+                    acc += M[s_][i][j] * x[s_][4 * b + j]
+                assert abs(y[s_][4 * b + i] - acc) < 1e-12
