@@ -466,18 +466,20 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
   const uint32_t tmem = *tmem_holder;
   const int nst_frame = (S + TOK - 1) / TOK;
   // parts > 1: each frame-head's tokens are cut into `parts` stage ranges, one
-  // unit each, whose partial A_t, U_t are added (fp32 atomics) into A, U
+  // unit each, whose partial A_t, U_t are added (fp32 atomics) into A, U. The
+  // ranges are balanced, part * nst / parts .. (part + 1) * nst / parts, so
+  // none is empty while parts <= nst (the host keeps parts <= nst / 2): an
+  // empty unit would add a stale TMEM accumulator into A_t, U_t.
   const int NU = N * parts;
   const int my_count = cta < NU ? (NU - 1 - cta) / ncta + 1 : 0;
-  const int per_part = (nst_frame + parts - 1) / parts;
   auto unit_n = [&](int i) -> int {
     const int u = (cta + i * ncta) / parts;
     if (heads <= 0) return u;
     const int j = u / heads;
     return (u % heads) * T + (rev ? T - 1 - j : j);
   };
-  auto st_begin = [&](int i) -> int { return ((cta + i * ncta) % parts) * per_part; };
-  auto st_end = [&](int i) -> int { return min(st_begin(i) + per_part, nst_frame); };
+  auto st_begin = [&](int i) -> int { return ((cta + i * ncta) % parts) * nst_frame / parts; };
+  auto st_end = [&](int i) -> int { return ((cta + i * ncta) % parts + 1) * nst_frame / parts; };
 
   if (warp == 0) {
     // ---- TMA producer (lane 0 issues; the warp loads beta) ----

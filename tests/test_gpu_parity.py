@@ -473,3 +473,20 @@ def test_plan_selection_d256():
             o_ref, s_ref = U.oracle_slab(arr, b, 0, True)
             assert U.rel_frob_per_frame(U.host(out[b, 0]), o_ref) < U.TOL_BF16, kw
             assert U.rel_frob_per_frame(U.host(st[b, 0])[None], s_ref[None]) < U.TOL_BF16, kw
+
+
+@pytest.mark.parametrize("H,T,S", [(3, 7, 1000), (1, 5, 300), (2, 3, 600), (4, 9, 2000)])
+def test_token_split_ranges_repeated_calls(H, T, S):
+    """Token-split plan (at most a quarter of the SMs in frame-heads): sizes
+    whose parts do not divide a frame's stages evenly, three calls in a row
+    (a stale accumulator would show up from the second call on)."""
+    arr = U.random_case(300 + H * T, 1, H, T, S, 128, bf16=True, state=True)
+    d = U.dev_inputs(arr, True)
+    refs = [U.oracle_slab(arr, 0, h, True) for h in range(H)]
+    for call in range(3):
+        out, st = api.frame_scan_fwd_ex(d["q"], d["k"], d["v"], d["beta"], d["gamma"], d["state"])
+        torch.cuda.synchronize()
+        api.check_device_status()
+        for h, (o_ref, s_ref) in enumerate(refs):
+            assert U.rel_frob_per_frame(U.host(out[0, h]), o_ref) < U.TOL_BF16, (call, h)
+            assert U.rel_frob_per_frame(U.host(st[0, h])[None], s_ref[None]) < U.TOL_BF16, (call, h)
