@@ -36,6 +36,7 @@ FUSED_REPLAY = 0x1000000
 CHUNKED = 0x2000000
 NO_OVERLAP = 0x4000000
 SAVE_FOR_BACKWARD = 0x10000000
+UCPE = 0x20000000
 REV_STATE_IN = 0x8000000
 
 
@@ -65,6 +66,8 @@ class GdnParams(ctypes.Structure):
         ("eps", ctypes.c_float), ("rope_base", ctypes.c_float), ("flags", ctypes.c_uint),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("state_in_rev", ctypes.c_void_p),
+        ("ucpe_q", ctypes.c_void_p),
+        ("ucpe_k", ctypes.c_void_p),
     ]
 
 
@@ -91,6 +94,8 @@ _F = ctypes.c_float
 SIGNATURES = {
     "gdn_frame_scan_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _U, _P]),
     "gdn_qk_prologue": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _F, _U, _P]),
+    "gdn_qk_prologue_ucpe": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _F,
+                                  _U, _P]),
     "gdn_frame_scan_fwd_ex": (_I, [ctypes.POINTER(GdnParams), _P]),
     "gdn_frame_scan_fwd_static": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _U, _P]),
     "gdn_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _U]),
@@ -210,8 +215,10 @@ def frame_scan_fwd_ex(q, k, v, beta, gamma, state_in=None, *, reverse=False, blo
 
     q, k, v [B,H,T,S,D] (bf16 or fp32); beta [B,H,T,S] fp32; gamma [B,H,T]
     fp32; state_in [B,H,D,D] fp32 or None. prologue = dict(w_q, w_k, grid_h,
-    grid_w[, eps, rope_base]) applies the fused RMSNorm/ReLU/key-scale/RoPE to
-    raw q, k. Returns (out, state_out) or, with bidir, (out, state_out,
+    grid_w[, eps, rope_base, ucpe_q, ucpe_k]) applies the fused
+    RMSNorm/ReLU/key-scale/RoPE to raw q, k; with ucpe_q and ucpe_k
+    ([B,T,S,4,4] fp32: D^T and D^-1 per token) the camera encoding takes
+    channels [0, D/2) and the RoPE the rest (GDN_UCPE). Returns (out, state_out) or, with bidir, (out, state_out,
     out_rev, state_out_rev). With bidir, state_in_rev (a tensor or None)
     gives the reverse scan its own start state (GDN_REV_STATE_IN); left out,
     state_in seeds both directions. save_for_backward keeps what a later
@@ -258,6 +265,11 @@ def frame_scan_fwd_ex(q, k, v, beta, gamma, state_in=None, *, reverse=False, blo
         _want(prologue["w_k"], "w_k", torch.float32, (D,))
         p.w_q, p.w_k = _ptr(prologue["w_q"]), _ptr(prologue["w_k"])
         p.grid_h, p.grid_w = int(prologue["grid_h"]), int(prologue["grid_w"])
+        if prologue.get("ucpe_q") is not None or prologue.get("ucpe_k") is not None:
+            for n in ("ucpe_q", "ucpe_k"):
+                _want(prologue[n], n, torch.float32, (B, T, S, 4, 4))
+            p.ucpe_q, p.ucpe_k = _ptr(prologue["ucpe_q"]), _ptr(prologue["ucpe_k"])
+            flags |= UCPE
         p.eps = float(prologue.get("eps", 1e-6))
         p.rope_base = float(prologue.get("rope_base", 10000.0))
     p.B, p.H, p.T, p.S, p.D = B, H, T, S, D
@@ -508,8 +520,10 @@ def frame_scan_fwd_static(q, k, v, beta, gamma, state_in=None, *, reverse=False,
 
 
 def qk_prologue(q_raw, k_raw, w_q, w_k, grid_h, grid_w, *, eps=1e-6, rope_base=10000.0,
-                stream=None):
-    """RMSNorm -> ReLU -> key scale -> 2-D RoPE on raw q, k [B,H,T,S,D]."""
+                ucpe=None, stream=None):
+    """RMSNorm -> ReLU -> key scale -> 2-D RoPE on raw q, k [B,H,T,S,D];
+    with ucpe = (ucpe_q, ucpe_k) ([B,T,S,4,4] fp32) the camera encoding takes
+    channels [0, D/2) and the RoPE the rest (gdn_qk_prologue_ucpe)."""
     B, H, T, S, D = q_raw.shape
     _want(q_raw, "q_raw", None, (B, H, T, S, D))
     _want(k_raw, "k_raw", q_raw.dtype, (B, H, T, S, D))
@@ -517,9 +531,17 @@ def qk_prologue(q_raw, k_raw, w_q, w_k, grid_h, grid_w, *, eps=1e-6, rope_base=1
     _want(w_k, "w_k", torch.float32, (D,))
     q_out, k_out = torch.empty_like(q_raw), torch.empty_like(k_raw)
     flags = BF16 if q_raw.dtype == torch.bfloat16 else 0
-    _check(lib().gdn_qk_prologue(_ptr(q_raw), _ptr(k_raw), _ptr(w_q), _ptr(w_k), _ptr(q_out),
-                                 _ptr(k_out), B, H, T, grid_h, grid_w, D, eps, rope_base, flags,
-                                 _stream(stream)), "gdn_qk_prologue")
+    if ucpe is None:
+        _check(lib().gdn_qk_prologue(_ptr(q_raw), _ptr(k_raw), _ptr(w_q), _ptr(w_k),
+                                     _ptr(q_out), _ptr(k_out), B, H, T, grid_h, grid_w, D, eps,
+                                     rope_base, flags, _stream(stream)), "gdn_qk_prologue")
+        return q_out, k_out
+    for t, n in zip(ucpe, ("ucpe_q", "ucpe_k")):
+        _want(t, n, torch.float32, (B, T, S, 4, 4))
+    _check(lib().gdn_qk_prologue_ucpe(_ptr(q_raw), _ptr(k_raw), _ptr(w_q), _ptr(w_k),
+                                      _ptr(ucpe[0]), _ptr(ucpe[1]), _ptr(q_out), _ptr(k_out),
+                                      B, H, T, grid_h, grid_w, D, eps, rope_base, flags,
+                                      _stream(stream)), "gdn_qk_prologue_ucpe")
     return q_out, k_out
 
 

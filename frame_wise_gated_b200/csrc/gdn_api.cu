@@ -299,6 +299,10 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
     return fail(GDN_ERR_INVALID, "GDN_BIDIR and GDN_REVERSE are exclusive%s");
   if ((f & GDN_SEQUENTIAL) && (f & GDN_CHUNKED))
     return fail(GDN_ERR_INVALID, "GDN_SEQUENTIAL and GDN_CHUNKED are exclusive%s");
+  if ((f & GDN_UCPE) && !(f & GDN_FUSED_PROLOGUE))
+    return fail(GDN_ERR_INVALID, "GDN_UCPE is part of GDN_FUSED_PROLOGUE%s");
+  if ((f & GDN_UCPE) && (!p.ucpe_q || !p.ucpe_k || !aligned16(p.ucpe_q) || !aligned16(p.ucpe_k)))
+    return fail(GDN_ERR_INVALID, "GDN_UCPE needs 16-byte aligned ucpe_q and ucpe_k%s");
   if (f & GDN_FUSED_PROLOGUE) {
     if (!p.w_q || !p.w_k) return fail(GDN_ERR_INVALID, "prologue needs w_q and w_k%s");
     if (p.grid_h < 1 || p.grid_w < 1 || (long long)p.grid_h * p.grid_w != p.S)
@@ -337,7 +341,8 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
     const float eps = p.eps > 0.f ? p.eps : 1e-6f;
     const float base = p.rope_base > 0.f ? p.rope_base : 10000.f;
     const int npos_max = p.grid_h > p.grid_w ? p.grid_h : p.grid_w;
-    if (tc_contract_ok && tc_readout_ok && p.D == 128 && npos_max <= tc_prologue_max_positions()) {
+    if (tc_contract_ok && tc_readout_ok && p.D == 128 && npos_max <= tc_prologue_max_positions() &&
+        !(f & GDN_UCPE)) {
       // Fused: the tensor-core loaders apply RMSNorm, ReLU and RoPE to the raw
       // tiles in shared memory; the key scale goes into the contraction's
       // epilogue constants (RoPE is linear, so the order does not matter).
@@ -357,7 +362,8 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
       {
         PhaseScope ps(PH_PROLOGUE, st);
         e = simt_prologue(bf16, p.q, p.k, p.w_q, p.w_k, ws + L.qh, ws + L.kh, frames, p.S,
-                          p.grid_w, p.D, eps, base, ks, st);
+                          p.grid_w, p.D, eps, base, ks, st, (f & GDN_UCPE) ? p.ucpe_q : nullptr,
+                          (f & GDN_UCPE) ? p.ucpe_k : nullptr, p.H, p.T);
       }
       if (e != cudaSuccess) return cuda_fail(e, "prologue");
       q = ws + L.qh;
@@ -385,7 +391,7 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
   const bool split = tc_contract_ok && tc_chain_ok && tc_readout_ok && p.D == 128 &&
                      !(f & GDN_FUSED_REPLAY) && frames * 4 <= nsms && nst >= 4;
   int parts = 1;
-  if (split) {
+  if (split) {  // 2 <= parts <= nst / 2: every part holds at least 2 stages
     parts = (int)(nsms / frames);
     if (parts > nst / 2) parts = nst / 2;
     if (parts > 8) parts = 8;
@@ -847,10 +853,10 @@ int gdn_frame_scan_fwd(const void* q, const void* k, const void* v, const float*
   return rc;
 }
 
-int gdn_qk_prologue(const void* q_raw, const void* k_raw, const float* w_q, const float* w_k,
-                    void* q_out, void* k_out, int B, int H, int T, int grid_h, int grid_w, int D,
-                    float eps, float rope_base, unsigned flags, gdn_stream_t stream) {
-  t_last_error.clear();
+static int qk_prologue(const void* q_raw, const void* k_raw, const float* w_q, const float* w_k,
+                       const float* ucpe_q, const float* ucpe_k, void* q_out, void* k_out, int B,
+                       int H, int T, int grid_h, int grid_w, int D, float eps, float rope_base,
+                       unsigned flags, cudaStream_t stream) {
   if (grid_h < 1 || grid_w < 1) return fail(GDN_ERR_INVALID, "grid must be >= 1%s");
   const long long S = (long long)grid_h * grid_w;
   if (S > 65535 * 64) return fail(GDN_ERR_UNSUPPORTED, "S above 4194240%s");
@@ -864,9 +870,28 @@ int gdn_qk_prologue(const void* q_raw, const void* k_raw, const float* w_q, cons
   cudaError_t e = simt_prologue((flags & GDN_BF16) != 0, q_raw, k_raw, w_q, w_k, q_out, k_out,
                                 (long long)B * H * T, (int)S, grid_w, D,
                                 eps > 0.f ? eps : 1e-6f, rope_base > 0.f ? rope_base : 10000.f,
-                                ks, (cudaStream_t)stream);
+                                ks, stream, ucpe_q, ucpe_k, H, T);
   if (e != cudaSuccess) return cuda_fail(e, "prologue");
   return GDN_OK;
+}
+
+int gdn_qk_prologue(const void* q_raw, const void* k_raw, const float* w_q, const float* w_k,
+                    void* q_out, void* k_out, int B, int H, int T, int grid_h, int grid_w, int D,
+                    float eps, float rope_base, unsigned flags, gdn_stream_t stream) {
+  t_last_error.clear();
+  return qk_prologue(q_raw, k_raw, w_q, w_k, nullptr, nullptr, q_out, k_out, B, H, T, grid_h,
+                     grid_w, D, eps, rope_base, flags, (cudaStream_t)stream);
+}
+
+int gdn_qk_prologue_ucpe(const void* q_raw, const void* k_raw, const float* w_q, const float* w_k,
+                         const float* ucpe_q, const float* ucpe_k, void* q_out, void* k_out,
+                         int B, int H, int T, int grid_h, int grid_w, int D, float eps,
+                         float rope_base, unsigned flags, gdn_stream_t stream) {
+  t_last_error.clear();
+  if (!ucpe_q || !ucpe_k || !aligned16(ucpe_q) || !aligned16(ucpe_k))
+    return fail(GDN_ERR_INVALID, "ucpe_q and ucpe_k must be 16-byte aligned device pointers%s");
+  return qk_prologue(q_raw, k_raw, w_q, w_k, ucpe_q, ucpe_k, q_out, k_out, B, H, T, grid_h,
+                     grid_w, D, eps, rope_base, flags, (cudaStream_t)stream);
 }
 
 int gdn_frame_contract(const void* k, const void* v, const float* beta, float* A, float* U,

@@ -123,10 +123,13 @@ Layout make_layout(int B, int H, int T, int S, int D, unsigned flags);
 void count_launch(int n = 1);
 
 // ---- SIMT (CUDA-core) kernels: any D in {16..256}, fp32 or bf16 -----------------
+// mq, mk: per-token camera matrices [B][T][S][4][4] (both null: no camera
+// encoding, RoPE on all D channels); H, T locate a frame-head's (b, t).
 cudaError_t simt_prologue(bool bf16, const void* q_raw, const void* k_raw, const float* w_q,
                           const float* w_k, void* q_out, void* k_out, long long frames, int S,
                           int grid_w, int D, float eps, float base, float kscale,
-                          cudaStream_t st);
+                          cudaStream_t st, const float* mq = nullptr, const float* mk = nullptr,
+                          int H = 1, int T = 1);
 cudaError_t simt_contract(bool bf16, const void* k, const void* v, const float* beta, float* A,
                           float* U, long long N, int S, int D, float cA, float cU,
                           cudaStream_t st);

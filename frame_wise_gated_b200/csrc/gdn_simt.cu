@@ -14,16 +14,21 @@ namespace gdn {
 
 // ----------------------------------------------------------------------------
 // Prologue: RMSNorm -> ReLU -> key scale -> 2-D spatial RoPE, one warp per token
-// (SANA-WM blog, Context-Parallel section, the fused-op order).
+// (SANA-WM blog, Context-Parallel section, the fused-op order). With UCPE the
+// camera encoding (same page, section 双分支相机控制) takes channels [0, D/2):
+// each block of 4 channels of token (b, t, s) is multiplied by that token's
+// 4 x 4 matrix (mq for queries, mk for keys: [B][T][S][4][4] fp32, shared by
+// the heads), and the RoPE acts on [D/2, D) as a vector of D/2 channels.
 // ----------------------------------------------------------------------------
-template <typename T>
+template <typename T, bool UCPE>
 __global__ void __launch_bounds__(256)
     k_prologue(const T* __restrict__ qin, const T* __restrict__ kin, const float* __restrict__ wq,
                const float* __restrict__ wk, T* __restrict__ qout, T* __restrict__ kout,
-               long long ntok, int S, int grid_w, int D, float eps, float base, float kscale) {
+               long long ntok, int S, int grid_w, int D, float eps, float base, float kscale,
+               const float* __restrict__ mq, const float* __restrict__ mk, int H, int Tn) {
   const long long tok = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (tok >= ntok) return;
+  if (tok >= ntok) return;  // warp-uniform: one token per warp
   const int which = blockIdx.y;  // 0: q, 1: k
   const T* in = which ? kin : qin;
   T* out = which ? kout : qout;
@@ -32,7 +37,10 @@ __global__ void __launch_bounds__(256)
   const size_t off = (size_t)tok * D;
   const int s = (int)(tok % S);
   const int py = s / grid_w, px = s % grid_w;
-  const int npairs = D >> 1, quarter = D >> 2, half = D >> 1;
+  const int npairs = D >> 1;
+  // RoPE channels: all D (pairs from 0), or the upper D/2 with UCPE
+  const int rope_p0 = UCPE ? D >> 2 : 0, rope_ch = UCPE ? D >> 1 : D;
+  const int quarter = rope_ch >> 2, half = rope_ch >> 1;
 
   float a[4], b[4];
   float ss = 0.f;
@@ -49,13 +57,40 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   const float inv = 1.0f / sqrtf(ss / (float)D + eps);
+  float M[16];
+  if (UCPE) {
+    const long long n = tok / S;  // frame-head (b * H + h) * T + t
+    const long long bt = (n / ((long long)H * Tn)) * Tn + n % Tn;
+    const float4* src = (const float4*)((which ? mk : mq) + ((size_t)bt * S + s) * 16);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float4 v = __ldg(src + r);
+      M[4 * r] = v.x; M[4 * r + 1] = v.y; M[4 * r + 2] = v.z; M[4 * r + 3] = v.w;
+    }
+  }
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
     const int p = lane + 32 * m;
+    // every lane of a warp takes the same m-iterations, so the shuffle below
+    // sees all 32 lanes (pairs past D/2 simply hold zeros)
+    const float x0 = p < npairs ? fmaxf(a[m] * inv * w[2 * p], 0.f) * scale : 0.f;
+    const float x1 = p < npairs ? fmaxf(b[m] * inv * w[2 * p + 1], 0.f) * scale : 0.f;
+    if (UCPE && 32 * m < rope_p0) {
+      // camera block p / 2: this lane's pair and its neighbour's (lane ^ 1)
+      const float y0 = __shfl_xor_sync(0xffffffffu, x0, 1);
+      const float y1 = __shfl_xor_sync(0xffffffffu, x1, 1);
+      if (p < rope_p0) {
+        const int hi = p & 1;  // rows 2, 3 of the block for the odd pair
+        const float v0 = hi ? y0 : x0, v1 = hi ? y1 : x1, v2 = hi ? x0 : y0, v3 = hi ? x1 : y1;
+        const float* r0 = M + 8 * hi;
+        stf(out + off + 2 * p, r0[0] * v0 + r0[1] * v1 + r0[2] * v2 + r0[3] * v3);
+        stf(out + off + 2 * p + 1, r0[4] * v0 + r0[5] * v1 + r0[6] * v2 + r0[7] * v3);
+        continue;
+      }
+    }
     if (p < npairs) {
-      const float x0 = fmaxf(a[m] * inv * w[2 * p], 0.f) * scale;
-      const float x1 = fmaxf(b[m] * inv * w[2 * p + 1], 0.f) * scale;
-      const int hsel = p / quarter, i = p % quarter;
+      const int pr = p - rope_p0;  // pair index inside the RoPE channels
+      const int hsel = pr / quarter, i = pr % quarter;
       const float pos = hsel ? (float)px : (float)py;
       const float theta = powf(base, -2.0f * (float)i / (float)half);
       float sn, cs;
@@ -69,17 +104,28 @@ __global__ void __launch_bounds__(256)
 cudaError_t simt_prologue(bool bf16, const void* q_raw, const void* k_raw, const float* w_q,
                           const float* w_k, void* q_out, void* k_out, long long frames, int S,
                           int grid_w, int D, float eps, float base, float kscale,
-                          cudaStream_t st) {
+                          cudaStream_t st, const float* mq, const float* mk, int H, int T) {
   const long long ntok = frames * S;
   dim3 grid((unsigned)((ntok + 7) / 8), 2);
-  if (bf16)
-    k_prologue<__nv_bfloat16><<<grid, 256, 0, st>>>(
+  const bool ucpe = mq && mk;
+  if (bf16 && ucpe)
+    k_prologue<__nv_bfloat16, true><<<grid, 256, 0, st>>>(
         (const __nv_bfloat16*)q_raw, (const __nv_bfloat16*)k_raw, w_q, w_k,
-        (__nv_bfloat16*)q_out, (__nv_bfloat16*)k_out, ntok, S, grid_w, D, eps, base, kscale);
+        (__nv_bfloat16*)q_out, (__nv_bfloat16*)k_out, ntok, S, grid_w, D, eps, base, kscale, mq,
+        mk, H, T);
+  else if (bf16)
+    k_prologue<__nv_bfloat16, false><<<grid, 256, 0, st>>>(
+        (const __nv_bfloat16*)q_raw, (const __nv_bfloat16*)k_raw, w_q, w_k,
+        (__nv_bfloat16*)q_out, (__nv_bfloat16*)k_out, ntok, S, grid_w, D, eps, base, kscale, mq,
+        mk, H, T);
+  else if (ucpe)
+    k_prologue<float, true><<<grid, 256, 0, st>>>((const float*)q_raw, (const float*)k_raw, w_q,
+                                                  w_k, (float*)q_out, (float*)k_out, ntok, S,
+                                                  grid_w, D, eps, base, kscale, mq, mk, H, T);
   else
-    k_prologue<float><<<grid, 256, 0, st>>>((const float*)q_raw, (const float*)k_raw, w_q, w_k,
-                                            (float*)q_out, (float*)k_out, ntok, S, grid_w, D,
-                                            eps, base, kscale);
+    k_prologue<float, false><<<grid, 256, 0, st>>>((const float*)q_raw, (const float*)k_raw, w_q,
+                                                   w_k, (float*)q_out, (float*)k_out, ntok, S,
+                                                   grid_w, D, eps, base, kscale, mq, mk, H, T);
   count_launch();
   return cudaGetLastError();
 }

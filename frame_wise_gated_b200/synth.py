@@ -22,7 +22,7 @@ import os
 import numpy as np
 
 __all__ = ["Config", "CONFIGS", "bf16_round_bits", "bf16_bits_to_f32",
-           "make_slab", "make_inputs", "make_state", "make_weights"]
+           "make_slab", "make_inputs", "make_state", "make_weights", "make_camera"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -139,3 +139,54 @@ def make_inputs(cfg: Config, threads: int | None = None):
     arr["state"] = make_state(cfg)
     arr["w_q"], arr["w_k"] = make_weights(cfg)
     return arr
+
+
+def _rot(axis: int, a: float) -> np.ndarray:
+    c, s_ = np.cos(a), np.sin(a)
+    i, j = [(1, 2), (0, 2), (0, 1)][axis]
+    R = np.eye(3)
+    R[i, i] = R[j, j] = c
+    R[i, j], R[j, i] = -s_, s_
+    return R
+
+
+def make_camera(B: int, T: int, grid_h: int, grid_w: int, seed: int):
+    """Synthetic camera geometry for the camera encoding: per batch b a smooth
+    trajectory over the T latent frames (yaw and pitch growing with t, the
+    centre on a small arc, |c| <= 0.5) seen through a pinhole camera with a
+    90-degree horizontal field of view on the grid_h x grid_w latent grid.
+    For token s = y * grid_w + x of frame t the ray through the pixel centre
+    defines a ray-local frame (z along the ray, x perpendicular to it and to
+    the camera's up axis); D_{t,s} maps world coordinates into that frame.
+    Returns (M_q, M_k) [B, T, S, 4, 4] float32: D^T for queries and D^-1 for
+    keys. Geometry only: the transforms are inputs of the prologue."""
+    rng = np.random.default_rng([seed, 1_000_005])
+    S = grid_h * grid_w
+    f = grid_w / 2.0
+    ys, xs = np.divmod(np.arange(S), grid_w)
+    d = np.stack([(xs + 0.5 - grid_w / 2.0) / f, (ys + 0.5 - grid_h / 2.0) / f, np.ones(S)], -1)
+    d /= np.linalg.norm(d, axis=-1, keepdims=True)
+    up = np.array([0.0, 1.0, 0.0])
+    xr = np.cross(up, d)
+    xr /= np.linalg.norm(xr, axis=-1, keepdims=True)
+    yr = np.cross(d, xr)
+    R_ray = np.stack([xr, yr, d], 1)                     # [S, 3, 3]: camera -> ray-local
+    Mq = np.empty((B, T, S, 4, 4), np.float32)
+    Mk = np.empty((B, T, S, 4, 4), np.float32)
+    for b in range(B):
+        yaw0, pitch0 = rng.uniform(-0.5, 0.5, 2)
+        for t in range(T):
+            R_t = _rot(1, yaw0 + 0.03 * t) @ _rot(0, pitch0 + 0.01 * t)   # camera -> world
+            c = 0.4 * np.array([np.sin(0.05 * t), 0.1 * np.sin(0.1 * t), 1.0 - np.cos(0.05 * t)])
+            Rw = R_ray @ R_t.T                                           # world -> ray-local
+            Dm = np.zeros((S, 4, 4))
+            Dm[:, :3, :3] = Rw
+            Dm[:, :3, 3] = -Rw @ c
+            Dm[:, 3, 3] = 1.0
+            Di = np.zeros((S, 4, 4))
+            Di[:, :3, :3] = np.transpose(Rw, (0, 2, 1))
+            Di[:, :3, 3] = c
+            Di[:, 3, 3] = 1.0
+            Mq[b, t] = np.transpose(Dm, (0, 2, 1))
+            Mk[b, t] = Di
+    return Mq, Mk

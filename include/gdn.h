@@ -87,6 +87,9 @@ enum {
                                        state_in_rev (NULL = zeros) instead of state_in */
 #define GDN_NO_OVERLAP 0x4000000u /* run the sequential chains as their own launch after
                                      the contraction instead of alongside it */
+#define GDN_UCPE 0x20000000u     /* _ex with GDN_FUSED_PROLOGUE: camera encoding on
+                                   channels [0, D/2) (ucpe_q, ucpe_k), RoPE on [D/2, D);
+                                   see gdn_qk_prologue_ucpe */
 #define GDN_SAVE_FOR_BACKWARD 0x10000000u /* _ex: leave the A_t operand images and the
                                      states in the workspace for gdn_frame_scan_bwd's
                                      saved_workspace (otherwise the plan with the chains
@@ -159,6 +162,31 @@ GDN_API int gdn_qk_prologue(const void* q_raw, const void* k_raw, const float* w
                     void* q_out, void* k_out, int B, int H, int T, int grid_h, int grid_w, int D,
                     float eps, float rope_base, unsigned flags, gdn_stream_t stream);
 
+/*
+ * gdn_qk_prologue_ucpe — the prologue with the camera encoding (SANA-WM blog,
+ * section 双分支相机控制：从粗到细的 6-DoF 轨迹: for every token a homogeneous
+ * transform D_{t,s} from world coordinates into the token's ray-local frame,
+ * combined orthogonally with the RoPE; "Jiayun's Blog", section 2.3). The
+ * pages do not say how the two are combined or how D enters the attention;
+ * readings: they act on separate channels, and queries take D^T, keys D^-1,
+ * so that a query-key product depends only on D_i D_j^-1 (not on the world
+ * frame). Per token, after RMSNorm, ReLU and (keys) the key scale:
+ *     channels [0, D/2): block b (channels 4b .. 4b+3) <- M block b, with M
+ *                        = ucpe_q[b,t,s] for q and ucpe_k[b,t,s] for k;
+ *     channels [D/2, D): the 2-D RoPE of gdn_qk_prologue applied to them as
+ *                        a vector of D/2 channels (its first half turns with
+ *                        y, its second half with x).
+ *   ucpe_q, ucpe_k  [B,T,S,4,4] fp32 row-major device arrays, 16-byte aligned,
+ *                   shared by all heads (for pure rotations D^T = D^-1: pass
+ *                   the same array twice). Computing D_{t,s} from camera
+ *                   poses and intrinsics is the caller's.
+ * Other arguments, outputs and errors as gdn_qk_prologue. */
+GDN_API int gdn_qk_prologue_ucpe(const void* q_raw, const void* k_raw, const float* w_q,
+                                 const float* w_k, const float* ucpe_q, const float* ucpe_k,
+                                 void* q_out, void* k_out, int B, int H, int T, int grid_h,
+                                 int grid_w, int D, float eps, float rope_base, unsigned flags,
+                                 gdn_stream_t stream);
+
 /* Everything gdn_frame_scan_fwd takes, plus the prologue, the second
  * direction and caller-owned scratch. Zero-initialise and fill. */
 typedef struct gdn_params {
@@ -184,6 +212,8 @@ typedef struct gdn_params {
   const float* state_in_rev; /* GDN_BIDIR | GDN_REV_STATE_IN: [B,H,D,D] or NULL (zeros);
                                 the chunk-causal streaming step passes the carried
                                 forward state in state_in and no reverse state */
+  const float* ucpe_q;    /* GDN_UCPE: [B,T,S,4,4] per-token camera matrix of q (D^T) */
+  const float* ucpe_k;    /* GDN_UCPE: [B,T,S,4,4] per-token camera matrix of k (D^-1) */
 } gdn_params;
 
 /*

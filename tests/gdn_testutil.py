@@ -72,14 +72,17 @@ def random_case(seed, B, H, T, S, D, *, bf16, state=False, beta_hi=1.0, gamma_lo
     return arr
 
 
-def oracle_slab(arr, b, h, bf16, *, reverse=False, block=0, keys_scaled=False, prologue=None):
-    """Oracle output and final state for slab (b, h). prologue = (grid_w, eps, base)."""
+def oracle_slab(arr, b, h, bf16, *, reverse=False, block=0, keys_scaled=False, prologue=None,
+                ucpe=None):
+    """Oracle output and final state for slab (b, h). prologue = (grid_w, eps, base);
+    ucpe = (M_q, M_k) [B, T, S, 4, 4] camera matrices (with the prologue)."""
     q = widen(arr["q"][b, h], bf16)
     k = widen(arr["k"][b, h], bf16)
     v = widen(arr["v"][b, h], bf16)
     if prologue is not None:
         grid_w, eps, base = prologue
-        q, k = O.qk_prologue(q, k, arr["w_q"], arr["w_k"], grid_w, eps=eps, base=base)
+        cam = None if ucpe is None else (ucpe[0][b], ucpe[1][b])
+        q, k = O.qk_prologue(q, k, arr["w_q"], arr["w_k"], grid_w, eps=eps, base=base, ucpe=cam)
         keys_scaled = True
     s0 = None if arr.get("state") is None else arr["state"][b, h]
     return O.frame_scan(q, k, v, arr["beta"][b, h].astype(np.float64),
