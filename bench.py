@@ -25,6 +25,7 @@ of this build) on a bounded sample of the same workload, on rank 0 only.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import glob
 import json
@@ -500,11 +501,11 @@ def run_ours(args, cfg):
 
 
 def run_e2e(args, cfg, arr, dev, api, barrier, dist, world):
-    """Same metric through the library's host-streaming call
-    (api.frame_scan_fwd_host: heads in chunks, copies in and out overlapping
-    the scans on three streams, each chunk one gdn_frame_scan_fwd_ex call) with
-    inputs and outputs in pinned host memory: every step copies all inputs to
-    the device and all outputs back, inside the timed region."""
+    """Same metric through the C-ABI host-buffer call gdn_frame_scan_fwd_host
+    (heads in chunks, copies in and out overlapping the scans on three
+    streams inside the library) with inputs and outputs in pinned host
+    memory: every step copies all inputs to the device and all outputs back,
+    inside the timed region."""
     import torch
     if cfg.prologue:
         return None  # the host-streaming call takes prepared q, k (no fused prologue)
@@ -544,8 +545,8 @@ def run_e2e(args, cfg, arr, dev, api, barrier, dist, world):
     return {"value": whole_job_value(cfg.tokens, world, ms_step), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_step,
             "steps": args.e2e_steps,
-            "entry": f"frame_scan_fwd_host (pinned host buffers, {hpc} heads per chunk, "
-                     "copies overlapping the scans; gdn_frame_scan_fwd_ex per chunk)"}
+            "entry": f"gdn_frame_scan_fwd_host (pinned host buffers, {hpc} heads per chunk, "
+                     "copies overlapping the scans inside the library)"}
 
 
 def main():
@@ -573,9 +574,14 @@ def main():
                     help="frames of one slab per reference step")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU work budget of the cpu_baseline sample")
+    ap.add_argument("--frames", type=int, default=0,
+                    help="override the workload's number of latent frames T (a smaller "
+                         "case of the same shape, e.g. for profiler captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     cfg = synth.CONFIGS[args.config]
+    if args.frames > 0:
+        cfg = dataclasses.replace(cfg, name=f"{cfg.name}_T{args.frames}", T=args.frames)
     if args.impl == "reference":
         return run_reference(args, cfg)
     return run_ours(args, cfg)

@@ -98,6 +98,8 @@ SIGNATURES = {
                                   _U, _P]),
     "gdn_frame_scan_fwd_ex": (_I, [ctypes.POINTER(GdnParams), _P]),
     "gdn_frame_scan_fwd_static": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _U, _P]),
+    "gdn_frame_scan_fwd_host": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _U, _I,
+                                     _P]),
     "gdn_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _U]),
     "gdn_frame_scan_bwd": (_I, [ctypes.POINTER(GdnBwdParams), _P]),
     "gdn_cp_shard_composite": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _U, _P,
@@ -307,83 +309,42 @@ def frame_scan_fwd(q, k, v, beta, gamma, state_in=None, *, reverse=False, block_
 
 
 def frame_scan_fwd_host(q, k, v, beta, gamma, state_in=None, *, out=None, state_out=None,
-                        heads_per_chunk=4, device=None, **plan):
-    """The scan over HOST tensors (pinned memory for full overlap), streamed
-    through the GPU in chunks of heads: while chunk c is scanned, chunk c+1 is
-    copied in and chunk c-1 copied out, on three CUDA streams, so PCIe carries
-    both directions at once. Heads are independent, so each chunk is one call
-    of gdn_frame_scan_fwd_ex on its own two device buffer sets (ping-pong).
+                        heads_per_chunk=2, device=None, **plan):
+    """The scan over HOST tensors through gdn_frame_scan_fwd_host: the library
+    streams the heads through the GPU in chunks (copies in, scans and copies
+    out overlapping on three streams; pinned memory for full overlap) and
+    returns once the results are in host memory.
 
     q, k, v [B,H,T,S,D] bf16 or fp32; beta [B,H,T,S], gamma [B,H,T],
-    state_in [B,H,D,D] (or None), all on the host. plan: the scan-plan keywords
-    of frame_scan_fwd_ex (reverse, block_reset, block, chunk, sequential,
-    chunked, overlap, keys_scaled). Returns host (out, state_out); the call
-    returns once they are complete."""
+    state_in [B,H,D,D] (or None), all contiguous host tensors. plan: the
+    scan-plan keywords of frame_scan_fwd (reverse, block_reset, block, chunk,
+    sequential, chunked, overlap, keys_scaled, force_simt). Returns host
+    (out, state_out)."""
     B, H, T, S, D = q.shape
-    BH = B * H
-    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         if t.is_cuda or t.shape != q.shape or t.dtype != q.dtype or not t.is_contiguous():
             raise ValueError(f"{n} must be a contiguous host tensor shaped and typed like q")
-    for t, n, shp in ((beta, "beta", (B, H, T, S)), (gamma, "gamma", (B, H, T))):
-        if t.is_cuda or tuple(t.shape) != shp or t.dtype != torch.float32 or not t.is_contiguous():
-            raise ValueError(f"{n} must be a contiguous fp32 host tensor of shape {shp}")
-    if state_in is not None and (state_in.is_cuda or tuple(state_in.shape) != (B, H, D, D)):
-        raise ValueError("state_in must be a host tensor [B,H,D,D]")
+    shapes = [(beta, "beta", (B, H, T, S)), (gamma, "gamma", (B, H, T))]
+    if state_in is not None:
+        shapes.append((state_in, "state_in", (B, H, D, D)))
     out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True) if out is None else out
     state_out = torch.empty((B, H, D, D), dtype=torch.float32, pin_memory=True) \
         if state_out is None else state_out
-    hc = max(1, min(int(heads_per_chunk), BH))
-    flat = lambda t: t.view(BH, *t.shape[2:])
-    src = [flat(q), flat(k), flat(v), flat(beta), flat(gamma)] + \
-          ([flat(state_in)] if state_in is not None else [])
-    dst = [flat(out), flat(state_out)]
-    # two slots of device buffers, each for hc heads
-    slots = []
-    for _ in range(2):
-        ins = [torch.empty((hc, *x.shape[1:]), dtype=x.dtype, device=dev) for x in src]
-        outs = [torch.empty((hc, *x.shape[1:]), dtype=x.dtype, device=dev) for x in dst]
-        slots.append((ins, outs))
-    s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
-    ev = {(kind, i): torch.cuda.Event() for kind in ("in", "cmp", "out") for i in range(2)}
-    used = [False, False]
-    cur = torch.cuda.current_stream(dev)
-    for st_ in (s_in, s_cmp, s_out):
-        st_.wait_stream(cur)
-    nchunk = (BH + hc - 1) // hc
-    for c in range(nchunk):
-        i0, i1 = c * hc, min(BH, (c + 1) * hc)
-        n = i1 - i0
-        slot = c & 1
-        ins, outs = slots[slot]
-        with torch.cuda.stream(s_in):
-            if used[slot]:
-                s_in.wait_event(ev[("cmp", slot)])  # the scan of chunk c-2 has read this slot
-            for d_, h_ in zip(ins, src):
-                d_[:n].copy_(h_[i0:i1], non_blocking=True)
-            ev[("in", slot)].record(s_in)
-        with torch.cuda.stream(s_cmp):
-            s_cmp.wait_event(ev[("in", slot)])
-            if used[slot]:
-                s_cmp.wait_event(ev[("out", slot)])  # chunk c-2's results have left this slot
-            view = lambda t: t[:n].view(1, n, *t.shape[1:])
-            frame_scan_fwd_ex(view(ins[0]), view(ins[1]), view(ins[2]), view(ins[3]),
-                              view(ins[4]), view(ins[5]) if len(ins) > 5 else None,
-                              out=view(outs[0]), state_out=view(outs[1]), stream=s_cmp, **plan)
-            ev[("cmp", slot)].record(s_cmp)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(ev[("cmp", slot)])
-            for h_, d_ in zip(dst, outs):
-                h_[i0:i1].copy_(d_[:n], non_blocking=True)
-            ev[("out", slot)].record(s_out)
-        used[slot] = True
-    cur.wait_stream(s_out)
-    cur.wait_stream(s_cmp)
-    cur.wait_stream(s_in)
-    # the copies out land in host memory: wait for them before returning
-    torch.cuda.current_stream(dev).synchronize()
+    shapes.append((state_out, "state_out", (B, H, D, D)))
+    for t, n, shp in shapes:
+        if t.is_cuda or tuple(t.shape) != shp or t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous fp32 host tensor of shape {shp}")
+    if out.is_cuda or out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous():
+        raise ValueError("out must be a contiguous host tensor shaped and typed like q")
+    flags = scan_flags(bf16=q.dtype == torch.bfloat16, **plan)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        _check(lib().gdn_frame_scan_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(gamma),
+                                             _ptr(state_in), _ptr(out), _ptr(state_out),
+                                             B, H, T, S, D, flags, int(heads_per_chunk),
+                                             _stream(torch.cuda.current_stream(dev))),
+               "gdn_frame_scan_fwd_host")
     return out, state_out
-
 
 def frame_scan_bwd(q, k, v, beta, gamma, state_in, d_out, d_state_out=None, *, reverse=False,
                    block_reset=False, block=3, keys_scaled=False, want_state_in_grad=True,

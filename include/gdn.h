@@ -260,6 +260,28 @@ GDN_API int gdn_frame_scan_fwd_static(const void* q, const void* k, const void* 
                                       gdn_stream_t stream);
 
 /*
+ * gdn_frame_scan_fwd_host — gdn_frame_scan_fwd over buffers in HOST memory
+ * (the end-to-end form: inputs start and results end in host memory). Same
+ * arguments, layouts, flags and results as gdn_frame_scan_fwd, except that
+ * q, k, v, beta, gamma, state_in, out and state_out are host pointers
+ * (page-locked memory lets the copies overlap; pageable memory works, with
+ * the copies serialised). Heads are independent: the call streams them
+ * through the GPU in chunks of heads_per_chunk whole heads (0: 2), with two
+ * device slots alternating, so that while one chunk is scanned the next is
+ * copied in and the previous copied out, on three internal streams (one
+ * cudaMemcpyAsync per tensor and chunk). Device memory (two slots of inputs,
+ * outputs and scan workspace for one chunk each) is taken stream-ordered from
+ * `stream`'s memory pool and given back before returning. The work starts
+ * after the work already enqueued on `stream`; the call returns once the
+ * results are in host memory (it synchronises). Returns GDN_OK or a status.
+ */
+GDN_API int gdn_frame_scan_fwd_host(const void* q, const void* k, const void* v,
+                                    const float* beta, const float* gamma,
+                                    const float* state_in, void* out, float* state_out, int B,
+                                    int H, int T, int S, int D, unsigned flags,
+                                    int heads_per_chunk, gdn_stream_t stream);
+
+/*
  * gdn_frame_scan_bwd — gradients of a loss through gdn_frame_scan_fwd.
  * (The pages print no backward; this is the adjoint of the same recurrence,
  * derived by reverse-mode differentiation.) Given dL/dO and optionally

@@ -205,11 +205,18 @@ def test_host_streaming_call():
     torch.cuda.synchronize()
     h = {n: (t.cpu().pin_memory() if t is not None else None) for n, t in d.items()
          if n in ("q", "k", "v", "beta", "gamma", "state")}
-    for hpc in (1, 2, 4):
+    for hpc in (0, 1, 2, 4):  # 0: the library's default chunk
         o, s = api.frame_scan_fwd_host(h["q"], h["k"], h["v"], h["beta"], h["gamma"], h["state"],
                                        heads_per_chunk=hpc)
         assert not o.is_cuda and not s.is_cuda
         assert torch.equal(o, ref_o.cpu()) and torch.equal(s, ref_s.cpu()), hpc
+    # pageable host memory (copies serialised) and no start state
+    pg = {n: t.clone() for n, t in h.items() if t is not None}
+    o2, s2 = api.frame_scan_fwd_host(pg["q"], pg["k"], pg["v"], pg["beta"], pg["gamma"], None,
+                                     heads_per_chunk=2)
+    ref2_o, ref2_s = api.frame_scan_fwd_ex(d["q"], d["k"], d["v"], d["beta"], d["gamma"], None)
+    torch.cuda.synchronize()
+    assert torch.equal(o2, ref2_o.cpu()) and torch.equal(s2, ref2_s.cpu())
     for b in range(2):
         for hh in range(3):
             o_ref, s_ref = U.oracle_slab(arr, b, hh, True)
