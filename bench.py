@@ -70,7 +70,8 @@ def algorithmic_bytes(cfg, step=True):
     n_t = 5 if cfg.prologue else 4
     per_fh = cfg.S * (n_t * cfg.D * e + 4) + 4
     state = 2 * cfg.D * cfg.D * 4
-    return cfg.frame_heads * per_fh + cfg.B * cfg.H * state
+    camera = 2 * cfg.B * cfg.T * cfg.S * 64 if cfg.ucpe else 0  # 4x4 fp32 for q and k per token
+    return cfg.frame_heads * per_fh + cfg.B * cfg.H * state + camera
 
 
 def backward_bytes(cfg):
@@ -205,10 +206,14 @@ def cpu_oracle_sample(cfg, frames=None, slab=(0, 0)):
     gamma = sl["gamma"][:T].astype(np.float64)
     st = synth.make_state(cfg)
     s0 = None if st is None else st[b, h]
+    cam = None
+    if cfg.ucpe:
+        mq, mk = synth.make_camera(cfg.B, cfg.T, cfg.grid_h, cfg.grid_w, cfg.seed)
+        cam = (mq[b, :T], mk[b, :T])
     t0 = time.perf_counter()
     if cfg.prologue:
         wq, wk = synth.make_weights(cfg)
-        qh, kh = O.qk_prologue(q, k, wq, wk, cfg.grid_w)
+        qh, kh = O.qk_prologue(q, k, wq, wk, cfg.grid_w, ucpe=cam)
         O.frame_scan(qh, kh, v, beta, gamma, s0, keys_scaled=True)
         O.frame_scan(qh, kh, v, beta, gamma, s0, reverse=True, block=cfg.bidir_block,
                      keys_scaled=True)
@@ -333,6 +338,9 @@ def run_ours(args, cfg):
     if cfg.prologue:
         pro = dict(w_q=torch.from_numpy(arr["w_q"]).to(dev), w_k=torch.from_numpy(arr["w_k"]).to(dev),
                    grid_h=cfg.grid_h, grid_w=cfg.grid_w)
+        if cfg.ucpe:
+            mq, mk = synth.make_camera(cfg.B, cfg.T, cfg.grid_h, cfg.grid_w, cfg.seed)
+            pro["ucpe_q"], pro["ucpe_k"] = torch.from_numpy(mq).to(dev), torch.from_numpy(mk).to(dev)
     kw = dict(prologue=pro, bidir=bool(cfg.bidir_block), block_reset=bool(cfg.bidir_block),
               block=cfg.bidir_block or 3, fused_replay=args.fused_replay, **plan_kw(args.plan))
     if cfg.bidir_block and cfg.T == cfg.bidir_block:
@@ -341,7 +349,8 @@ def run_ours(args, cfg):
     out_rev = torch.empty_like(q) if cfg.bidir_block else None
     st_out = torch.empty((cfg.B, cfg.H, cfg.D, cfg.D), device=dev, dtype=torch.float32)
     st_rev = torch.empty_like(st_out) if cfg.bidir_block else None
-    flags = api.scan_flags(bf16=cfg.bf16, prologue=pro is not None, bidir=bool(cfg.bidir_block),
+    flags = (api.UCPE if cfg.ucpe else 0) | api.scan_flags(
+        bf16=cfg.bf16, prologue=pro is not None, bidir=bool(cfg.bidir_block),
                            block_reset=bool(cfg.bidir_block), block=cfg.bidir_block or 3,
                            fused_replay=args.fused_replay, **plan_kw(args.plan))
     ws = torch.empty(api.workspace_bytes(cfg.B, cfg.H, cfg.T, cfg.S, cfg.D, flags),
@@ -484,6 +493,7 @@ def run_ours(args, cfg):
                        ("forward, then backward from its saved workspace" if args.train else
                         "backward: recompute, adjoint chain, per-frame and per-token gradients"),
                        "prologue": cfg.prologue, "bidir_block": cfg.bidir_block,
+                       "camera_encoding": cfg.ucpe,
                        "l2": (f"inputs larger than L2 ({step_bytes / 1e9:.2f} GB algorithmic per step)"
                               if flush is None else
                               f"L2 flushed before every step ({2 * L2_BYTES >> 20} MiB written); "

@@ -42,6 +42,7 @@ class Config:
     state_sigma: float = 0.0        # S_0 ~ N(0, sigma^2) per entry, 0 -> zeros
     prologue: bool = False          # raw q, k go through the fused prologue
     bidir_block: int = 0            # >0: forward scan + reverse scan reset every block
+    ucpe: bool = False              # the prologue includes the camera encoding
 
     @property
     def frame_heads(self) -> int:
@@ -58,6 +59,10 @@ CONFIGS = {
     "rollout60s_720p": Config("rollout60s_720p", 1, 16, 121, 3600, 128, 45, 80, True, 3),
     "prologue_bidir_720p": Config("prologue_bidir_720p", 1, 16, 121, 3600, 128, 45, 80, True, 4,
                                   prologue=True, bidir_block=3),
+    # config 4 plus the camera encoding (per-token ray-local transforms of a
+    # synthetic camera trajectory, see make_camera)
+    "prologue_ucpe_bidir_720p": Config("prologue_ucpe_bidir_720p", 1, 16, 121, 3600, 128, 45, 80,
+                                       True, 9, prologue=True, bidir_block=3, ucpe=True),
     "prologue_bidir_clip5s_720p": Config("prologue_bidir_clip5s_720p", 1, 16, 21, 3600, 128, 45,
                                          80, True, 7, prologue=True, bidir_block=3),
     # one call of the chunk-causal streaming step: one 3-frame block, forward
