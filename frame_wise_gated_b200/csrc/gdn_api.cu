@@ -341,8 +341,7 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
     const float eps = p.eps > 0.f ? p.eps : 1e-6f;
     const float base = p.rope_base > 0.f ? p.rope_base : 10000.f;
     const int npos_max = p.grid_h > p.grid_w ? p.grid_h : p.grid_w;
-    if (tc_contract_ok && tc_readout_ok && p.D == 128 && npos_max <= tc_prologue_max_positions() &&
-        !(f & GDN_UCPE)) {
+    if (tc_contract_ok && tc_readout_ok && p.D == 128 && npos_max <= tc_prologue_max_positions()) {
       // Fused: the tensor-core loaders apply RMSNorm, ReLU and RoPE to the raw
       // tiles in shared memory; the key scale goes into the contraction's
       // epilogue constants (RoPE is linear, so the order does not matter).
@@ -350,11 +349,13 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
       float2* cs = (float2*)(ws + L.rope);
       {
         PhaseScope ps(PH_PROLOGUE, st);
-        e = rope_table(cs, npos, p.D, base, st);
+        // with the camera encoding the RoPE acts on D/2 channels
+        e = rope_table(cs, npos, (f & GDN_UCPE) ? p.D / 2 : p.D, base, st);
       }
       if (e != cudaSuccess) return cuda_fail(e, "rope table");
-      pro_k = ProArgs{p.w_k, cs, p.grid_w, eps, npos, base};
-      pro_q = ProArgs{p.w_q, cs, p.grid_w, eps, npos, base};
+      const bool cam = (f & GDN_UCPE) != 0;
+      pro_k = ProArgs{p.w_k, cs, p.grid_w, eps, npos, base, cam ? p.ucpe_k : nullptr, p.H, p.T};
+      pro_q = ProArgs{p.w_q, cs, p.grid_w, eps, npos, base, cam ? p.ucpe_q : nullptr, p.H, p.T};
       ppk = &pro_k;
       ppq = &pro_q;
     } else {

@@ -169,11 +169,15 @@ cudaError_t simt_bwd_combine(bool bf16, const void* k, const float* beta, const 
 // the key scale is folded into the contraction's epilogue constants).
 struct ProArgs {
   const float* w;    // [D] RMSNorm weight
-  const float2* cs;  // [D/4][npos] (cos, sin) of pos * base^(-2i/(D/2)), pair-major
+  const float2* cs;  // [D/4][npos] (cos, sin) of pos * base^(-2i/(D/2)), pair-major; with
+                     // ucpe: [D/8][npos] of the RoPE on D/2 channels
   int grid_w;
   float eps;
   int npos;
   float base;        // RoPE base (pair i turns by pos * base^(-2i/(D/2)))
+  const float* ucpe; // null, or this side's camera matrices [B][T][S][4][4]: channels
+                     // [0, D/2) in blocks of 4 take them, the RoPE takes [D/2, D)
+  int H, T;          // heads and frames: frame-head n = (b * H + h) * T + t
 };
 // (cos, sin) table, pair-major: cs[i * npos + pos], pos < npos, i < D/4
 // (consecutive tokens of a row read consecutive entries).

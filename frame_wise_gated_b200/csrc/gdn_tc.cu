@@ -187,11 +187,153 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
 __device__ __forceinline__ int pro_lane_row(int t) { return ((t >> 5) << 3) + (t & 7); }
 __device__ __forceinline__ int pro_lane_quarter(int t) { return (t >> 3) & 3; }
 
+// The prologue with the camera encoding (SANA-WM blog, section 双分支相机控制:
+// each token's transform into its ray-local frame, combined with the RoPE on
+// separate channels): channels 0-63 (box 0) form 16 blocks of 4, each
+// multiplied by the token's 4 x 4 matrix (pro.ucpe at frame-head n); channels
+// 64-127 (box 1) carry the 2-D RoPE of a 64-channel vector, y on channels
+// 64-95 and x on 96-127, 16 pairs each (table / theta entries 0-15). RMSNorm,
+// ReLU and the beta * K^ copy as in pro_rows.
+// Threads keep pro_rows' layout for the sum of squares (lane 8 q + j: quarter
+// q of row j). For the transform every lane takes the same work, so a warp
+// never splits between the two kinds: 16-byte chunks 2q and 2q + 1 of box 0
+// (two camera blocks each) and of box 1 (eight RoPE pairs). The lanes of a row
+// read its raw chunks before __syncwarp, then write. The matrices come from
+// global memory (L2: the heads of a frame share them); rows past S clamp to
+// token S - 1 (their data are zeros).
 template <int NR, bool THETA, bool BTILE>
-__device__ __forceinline__ void pro_rows(uint8_t* tile, int box_bytes, const int (&rr)[NR], int q,
-                                         const int (&tk)[NR], int S, const ProArgs& pro,
-                                         const float2* w4, const float2* tab, const float* theta,
-                                         uint8_t* btile, const float (&bv)[NR]) {
+__device__ __forceinline__ void pro_rows_ucpe(uint8_t* tile, int box_bytes, const int (&rr)[NR],
+                                              int q, const int (&tk)[NR], int S,
+                                              const ProArgs& pro, const float2* w4,
+                                              const float2* tab, const float* theta,
+                                              uint8_t* btile, const float (&bv)[NR], int n) {
+  constexpr int D = 128;
+  auto chunk_off = [&](int box, int row, int ch) {
+    return box * box_bytes + row * 128 + ((ch ^ (row & 7)) << 4);
+  };
+  float inv[NR], scb[NR];
+  {
+    float ss[NR];
+#pragma unroll
+    for (int k = 0; k < NR; ++k) {
+      float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint4 v = *(const uint4*)(tile + chunk_off(q >> 1, rr[k], (q & 1) * 4 + c));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 x = unpack_bf16x2(w[e]);
+          acc = __ffma2_rn(x, x, acc);
+        }
+      }
+      ss[k] = acc.x + acc.y;
+    }
+#pragma unroll
+    for (int o = 8; o < 32; o <<= 1) {  // the row's four quarters: lanes j, j + 8, j + 16, j + 24
+#pragma unroll
+      for (int k = 0; k < NR; ++k) ss[k] += __shfl_xor_sync(0xffffffffu, ss[k], o);
+    }
+#pragma unroll
+    for (int k = 0; k < NR; ++k) {
+      inv[k] = rsqrtf(fmaf(ss[k], 1.0f / (float)D, pro.eps));
+      scb[k] = inv[k] * bv[k];
+    }
+  }
+  // this lane's raw chunks: camera chunks 2q, 2q + 1 of box 0, RoPE chunks of box 1
+  uint32_t cw[NR][8], rw[NR][8];
+#pragma unroll
+  for (int k = 0; k < NR; ++k)
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint4 a = *(const uint4*)(tile + chunk_off(0, rr[k], 2 * q + i));
+      const uint4 b = *(const uint4*)(tile + chunk_off(1, rr[k], 2 * q + i));
+      cw[k][4 * i] = a.x; cw[k][4 * i + 1] = a.y; cw[k][4 * i + 2] = a.z; cw[k][4 * i + 3] = a.w;
+      rw[k][4 * i] = b.x; rw[k][4 * i + 1] = b.y; rw[k][4 * i + 2] = b.z; rw[k][4 * i + 3] = b.w;
+    }
+  __syncwarp();  // the lanes of each row have read their raw chunks
+  // camera: chunk ch = 2q + i of box 0 holds channels 8 ch .. 8 ch + 7 (quarter
+  // ch / 4, words 4 (ch % 4) .. + 3 of it): blocks 2 ch and 2 ch + 1
+  const long long bt = (long long)(n / (pro.H * pro.T)) * pro.T + n % pro.T;
+#pragma unroll
+  for (int k = 0; k < NR; ++k) {
+    const int s = tk[k] < S ? tk[k] : S - 1;
+    const float4* mp = (const float4*)(pro.ucpe + ((size_t)bt * S + s) * 16);
+    const float4 m0 = __ldg(mp), m1 = __ldg(mp + 1), m2 = __ldg(mp + 2), m3 = __ldg(mp + 3);
+    // the matrix by column pairs, the RMSNorm factor folded in: output rows
+    // (0, 1) are sum_j c01[j] v_j and rows (2, 3) sum_j c23[j] v_j (packed fp32x2)
+    const float f = inv[k];
+    const float2 c01[4] = {make_float2(m0.x * f, m1.x * f), make_float2(m0.y * f, m1.y * f),
+                           make_float2(m0.z * f, m1.z * f), make_float2(m0.w * f, m1.w * f)};
+    const float2 c23[4] = {make_float2(m2.x * f, m3.x * f), make_float2(m2.y * f, m3.y * f),
+                           make_float2(m2.z * f, m3.z * f), make_float2(m2.w * f, m3.w * f)};
+    const float bq = BTILE ? bv[k] : 1.f;  // beta: scb / inv
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int ch = 2 * q + i, qc = ch >> 2, pw = 4 * (ch & 3);
+      uint32_t ow[4], obw[4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float2 x0 = __fmul2_rn(unpack_bf16x2(cw[k][4 * i + 2 * h]), w4[(pw + 2 * h) * 4 + qc]);
+        const float2 x1 =
+            __fmul2_rn(unpack_bf16x2(cw[k][4 * i + 2 * h + 1]), w4[(pw + 2 * h + 1) * 4 + qc]);
+        const float v0 = fmaxf(x0.x, 0.f), v1 = fmaxf(x0.y, 0.f), v2 = fmaxf(x1.x, 0.f),
+                    v3 = fmaxf(x1.y, 0.f);
+        float2 o01 = __fmul2_rn(c01[0], make_float2(v0, v0));
+        float2 o23 = __fmul2_rn(c23[0], make_float2(v0, v0));
+        o01 = __ffma2_rn(c01[1], make_float2(v1, v1), o01);
+        o23 = __ffma2_rn(c23[1], make_float2(v1, v1), o23);
+        o01 = __ffma2_rn(c01[2], make_float2(v2, v2), o01);
+        o23 = __ffma2_rn(c23[2], make_float2(v2, v2), o23);
+        o01 = __ffma2_rn(c01[3], make_float2(v3, v3), o01);
+        o23 = __ffma2_rn(c23[3], make_float2(v3, v3), o23);
+        ow[2 * h] = pack_bf16x2(o01.x, o01.y);
+        ow[2 * h + 1] = pack_bf16x2(o23.x, o23.y);
+        if (BTILE) {
+          const float2 b01 = __fmul2_rn(o01, make_float2(bq, bq));
+          const float2 b23 = __fmul2_rn(o23, make_float2(bq, bq));
+          obw[2 * h] = pack_bf16x2(b01.x, b01.y);
+          obw[2 * h + 1] = pack_bf16x2(b23.x, b23.y);
+        }
+      }
+      const int off = chunk_off(0, rr[k], ch);
+      *(uint4*)(tile + off) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+      if (BTILE) *(uint4*)(btile + off) = make_uint4(obw[0], obw[1], obw[2], obw[3]);
+    }
+  }
+  // RoPE: chunk ch = 2q + i of box 1 is quarter 2 + ch / 4 (y for ch < 4, x
+  // after), words 4 (ch % 4) .. + 3 = pairs of the same index
+#pragma unroll
+  for (int k = 0; k < NR; ++k) {
+    const int pos = tk[k] < S ? ((q >> 1) ? tk[k] % pro.grid_w : tk[k] / pro.grid_w) : 0;
+    const float2* trow = tab + pro_table_index(0, pos);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int ch = 2 * q + i, qr = 2 + (ch >> 2), pw = 4 * (ch & 3);
+      uint32_t ow[4], obw[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int p = pw + e;
+        const float2 m = __fmul2_rn(unpack_bf16x2(rw[k][4 * i + e]), w4[p * 4 + qr]);
+        const float a = fmaxf(m.x, 0.f), b = fmaxf(m.y, 0.f);
+        const float2 t = THETA ? rope_cs_reduced(pos, theta[p]) : trow[p * 2 * PRO_POS_PITCH];
+        const float2 o = make_float2(a * t.x - b * t.y, a * t.y + b * t.x);
+        ow[e] = pack_bf16x2(o.x * inv[k], o.y * inv[k]);
+        if (BTILE) obw[e] = pack_bf16x2(o.x * scb[k], o.y * scb[k]);
+      }
+      const int off = chunk_off(1, rr[k], ch);
+      *(uint4*)(tile + off) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+      if (BTILE) *(uint4*)(btile + off) = make_uint4(obw[0], obw[1], obw[2], obw[3]);
+    }
+  }
+}
+
+template <int NR, bool THETA, bool BTILE>
+__device__ __forceinline__ void pro_rows_rope(uint8_t* tile, int box_bytes, const int (&rr)[NR],
+                                              int q, const int (&tk)[NR], int S,
+                                              const ProArgs& pro, const float2* w4,
+                                              const float2* tab, const float* theta,
+                                              uint8_t* btile, const float (&bv)[NR]) {
   constexpr int D = 128, NW = 16;  // channel pairs (packed words) per thread row
   const int box = q >> 1, ch0 = (q & 1) * 4, pb = (q & 1) * 16;
   uint32_t u[NR][NW];
@@ -274,10 +416,25 @@ __device__ __forceinline__ void pro_rows(uint8_t* tile, int box_bytes, const int
   }
 }
 
+// The prologue of NR rows; UC (the camera encoding) is a compile-time choice so
+// that the kernels without it keep their register allocation.
+template <int NR, bool THETA, bool BTILE, bool UC>
+__device__ __forceinline__ void pro_rows(uint8_t* tile, int box_bytes, const int (&rr)[NR], int q,
+                                         const int (&tk)[NR], int S, const ProArgs& pro,
+                                         const float2* w4, const float2* tab, const float* theta,
+                                         uint8_t* btile, const float (&bv)[NR], int n) {
+  if constexpr (UC)
+    pro_rows_ucpe<NR, THETA, BTILE>(tile, box_bytes, rr, q, tk, S, pro, w4, tab, theta, btile, bv,
+                                    n);
+  else
+    pro_rows_rope<NR, THETA, BTILE>(tile, box_bytes, rr, q, tk, S, pro, w4, tab, theta, btile, bv);
+}
+
 // Copies the (cos, sin) table (pair-major, cs[i * npos + pos]) into shared
 // memory in pro_table_index order.
 __device__ __forceinline__ void pro_table_copy(float2* tab, const ProArgs& pro) {
-  for (int e = threadIdx.x; e < pro.npos * 32; e += (int)blockDim.x) {
+  const int npairs = pro.ucpe ? 16 : 32;  // the RoPE's channels: 64 with the camera encoding
+  for (int e = threadIdx.x; e < pro.npos * npairs; e += (int)blockDim.x) {
     const int i = e / pro.npos, pos = e - i * pro.npos;
     tab[pro_table_index(i, pos)] = pro.cs[e];
   }
@@ -407,7 +564,7 @@ __device__ __forceinline__ void drop_consumed(float* A, float* U, const int* fla
 // Rings: K and V tiles in NST stages (freed by the MMA commit of the stage),
 // beta * K in NBK slots of its own (written by the scalers once the MMAs of
 // the stage NBK earlier are done), so the ring that waits on HBM is deep.
-template <int NST>
+template <int NST, bool UC = false>
 __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUtensorMap& tmV,
                                               const float* __restrict__ beta, float* __restrict__ A,
                                               float* __restrict__ U, int N, int S, float cA,
@@ -591,7 +748,8 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
           // raw k -> K^ in place (RMSNorm, ReLU, RoPE) and beta * K^ into the slot
           const int rr[2] = {pr, pr + 32}, tk[2] = {st * TOK + pr, st * TOK + pr + 32};
           const float bv[2] = {beta ? bs[pr] : 1.f, beta ? bs[pr + 32] : 1.f};
-          pro_rows<2, false, true>(kt, BOX, rr, pq, tk, S, pro, w4, tab, nullptr, bt, bv);
+          pro_rows<2, false, true, UC>(kt, BOX, rr, pq, tk, S, pro, w4, tab, nullptr, bt, bv,
+                                       unit_n(i));
           fence_proxy_async();
           warp_arrive(bar_bkf + 8 * kb);
           continue;
@@ -715,12 +873,12 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
   }
 }
 
-template <int NST>
+template <int NST, bool UC = false>
 __global__ void __launch_bounds__(ctr::THREADS, 1)
     k_contract_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const float* __restrict__ beta, float* __restrict__ A, float* __restrict__ U,
                   int N, int S, float cA, float cU, int a_image, ProArgs pro, int parts) {
-  contract_body<NST>(tmK, tmV, beta, A, U, N, S, cA, cU, a_image, pro, blockIdx.x, gridDim.x, 0, 0,
+  contract_body<NST, UC>(tmK, tmV, beta, A, U, N, S, cA, cU, a_image, pro, blockIdx.x, gridDim.x, 0, 0,
                      0, nullptr, parts);
 }
 
@@ -762,12 +920,18 @@ static cudaError_t tc_contract128(const void* k, const void* v, const float* bet
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_contract_tc<ctr::NST_PRO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                ctr::SMEM_PRO);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_contract_tc<ctr::NST_PRO, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, ctr::SMEM_PRO);
     return e;
   });
   if (attr_status != cudaSuccess) return attr_status;
   const long long units = N * parts;
   const int grid = (int)(units < num_sms() ? units : num_sms());
-  if (pro)
+  if (pro && pro->ucpe)
+    k_contract_tc<ctr::NST_PRO, true><<<grid, ctr::THREADS, ctr::SMEM_PRO, st>>>(
+        mk, mv, beta, A, U, (int)N, S, cA, cU, a_image, pa, parts);
+  else if (pro)
     k_contract_tc<ctr::NST_PRO><<<grid, ctr::THREADS, ctr::SMEM_PRO, st>>>(
         mk, mv, beta, A, U, (int)N, S, cA, cU, a_image, pa, parts);
   else
@@ -803,7 +967,7 @@ constexpr uint32_t TMEM_COLS = 256;
 
 // TRANS: O = Q S_t (S_t as an MN-major operand) instead of Q S_t^T; the
 // backward's dQ = dO S_t.
-template <bool PRO, bool TRANS = false>
+template <bool PRO, bool TRANS = false, bool UC = false>
 __global__ void __launch_bounds__(rdo::threads(PRO), 1)
     k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
                  const __grid_constant__ CUtensorMap tmO, int N, int S, ProArgs pro, int parts) {
@@ -1015,9 +1179,9 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
         if (!ok) break;
         const int rr[2] = {pr, pr + 64}, tk[2] = {tl * TOK + pr, tl * TOK + pr + 64};
         const float bv[2] = {1.f, 1.f};
-        pro_rows<2, false, false>(smem + OFF_Q + s * QT, BOX, rr, pq, tk, S, pro,
+        pro_rows<2, false, false, UC>(smem + OFF_Q + s * QT, BOX, rr, pq, tk, S, pro,
                                   (const float2*)(smem + OFF_W4), (const float2*)(smem + OFF_TAB),
-                                  nullptr, nullptr, bv);
+                                  nullptr, nullptr, bv, n);
         fence_proxy_async();
         warp_arrive(bar_qr + 8 * s);
       }
@@ -1045,12 +1209,12 @@ static int readout_parts(long long N, int ntile) {
   return (ntile >= 8 && N < 4LL * num_sms()) ? 2 : 1;
 }
 
-template <bool PRO, bool TRANS = false>
+template <bool PRO, bool TRANS = false, bool UC = false>
 static cudaError_t launch_readout(const CUtensorMap& mq, const CUtensorMap& ms, const CUtensorMap& mo,
                                   long long N, int S, const ProArgs& pa, cudaStream_t st) {
   static DeviceOnce attr_once;
   const cudaError_t attr_status = once_per_device(attr_once, [&]() -> cudaError_t {
-    cudaError_t e = cudaFuncSetAttribute(k_readout_tc<PRO, TRANS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(k_readout_tc<PRO, TRANS, UC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          rdo::SMEM);
     return e;
   });
@@ -1058,8 +1222,8 @@ static cudaError_t launch_readout(const CUtensorMap& mq, const CUtensorMap& ms, 
   const int parts = readout_parts(N, (S + rdo::TOK - 1) / rdo::TOK);
   const long long units = N * parts;
   const int grid = (int)(units < num_sms() ? units : num_sms());
-  k_readout_tc<PRO, TRANS><<<grid, rdo::threads(PRO), rdo::SMEM, st>>>(mq, ms, mo, (int)N, S, pa,
-                                                                      parts);
+  k_readout_tc<PRO, TRANS, UC><<<grid, rdo::threads(PRO), rdo::SMEM, st>>>(mq, ms, mo, (int)N, S,
+                                                                          pa, parts);
   count_launch();
   return cudaGetLastError();
 }
@@ -1078,6 +1242,7 @@ static cudaError_t tc_readout128(const void* q, const void* Sfr_hilo, void* out,
   ProArgs pa = {};
   if (pro) {
     pa = *pro;
+    if (pa.ucpe) return launch_readout<true, false, true>(mq, ms, mo, N, S, pa, st);
     return launch_readout<true>(mq, ms, mo, N, S, pa, st);
   }
   return launch_readout<false>(mq, ms, mo, N, S, pa, st);
@@ -2208,7 +2373,7 @@ __device__ __forceinline__ void ovl_chain_body(const OvlArgs& o, const CUtensorM
   }
 }
 
-template <int NST>
+template <int NST, bool UC = false>
 __global__ void __launch_bounds__(ovl::THREADS, 1)
     k_contract_scan_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const float* __restrict__ beta, float* __restrict__ A, float* __restrict__ U,
@@ -2218,9 +2383,9 @@ __global__ void __launch_bounds__(ovl::THREADS, 1)
   if ((int)blockIdx.x < nchain)
     ovl_chain_body(o, tmZ, tmS0, tmS1, blockIdx.x);
   else
-    contract_body<NST>(tmK, tmV, beta, A, U, N, S, cA, cU, o.a_image, pro,
-                       (int)blockIdx.x - nchain, (int)gridDim.x - nchain, o.heads, o.T,
-                       o.contract_rev, o.flags, 1, o.discard);
+    contract_body<NST, UC>(tmK, tmV, beta, A, U, N, S, cA, cU, o.a_image, pro,
+                           (int)blockIdx.x - nchain, (int)gridDim.x - nchain, o.heads, o.T,
+                           o.contract_rev, o.flags, 1, o.discard);
 }
 
 bool tc_overlap_supported(int D) { return D == 128; }
@@ -2253,6 +2418,9 @@ cudaError_t tc_contract_scan(const void* k, const void* v, const float* beta, fl
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_contract_scan_tc<ctr::NST_PRO>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, smem_pro);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_contract_scan_tc<ctr::NST_PRO, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, smem_pro);
     return e;
   });
   if (attr_status != cudaSuccess) return attr_status;
@@ -2271,7 +2439,10 @@ cudaError_t tc_contract_scan(const void* k, const void* v, const float* beta, fl
                   &pa, &o_a, &nchain_a, &mz, &ms0, &ms1};
   // cooperative: every CTA is resident, so the chains' waits on the
   // contraction CTAs always end
-  if (pro)
+  if (pro && pro->ucpe)
+    e = cudaLaunchCooperativeKernel((const void*)k_contract_scan_tc<ctr::NST_PRO, true>, dim3(grid),
+                                    dim3(ovl::THREADS), args, (size_t)smem_pro, st);
+  else if (pro)
     e = cudaLaunchCooperativeKernel((const void*)k_contract_scan_tc<ctr::NST_PRO>, dim3(grid),
                                     dim3(ovl::THREADS), args, (size_t)smem_pro, st);
   else
@@ -3004,7 +3175,7 @@ constexpr int threads(bool pro) { return pro ? 704 : 192; }  // + 16 prologue wa
 constexpr uint32_t TMEM_COLS = 512;
 }  // namespace rd2
 
-template <bool PRO>
+template <bool PRO, bool UC = false>
 __global__ void __launch_bounds__(rd2::threads(PRO), 1)
     k_readout2_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmSF,
                   const __grid_constant__ CUtensorMap tmSR, const __grid_constant__ CUtensorMap tmOF,
@@ -3043,7 +3214,8 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
   }
   if (PRO) pro_w_copy((float2*)(smem + OFF_W), pro.w);
   if (PRO && threadIdx.x < D / 4)  // pair frequencies, as the (cos, sin) table has them
-    ((float*)(smem + OFF_TH))[threadIdx.x] = rope_theta(pro.base, threadIdx.x, D);
+    ((float*)(smem + OFF_TH))[threadIdx.x] =
+        rope_theta(pro.base, threadIdx.x, pro.ucpe ? D / 2 : D);  // entries 0-15 with the camera
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
     tmem_relinquish();
@@ -3216,9 +3388,9 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
         if (!ok) break;
         const int rr[1] = {pr}, tk[1] = {tl * TOK + pr};
         const float bv[1] = {1.f};
-        pro_rows<1, true, false>(smem + OFF_Q + s * QT, BOX, rr, pq, tk, S, pro,
+        pro_rows<1, true, false, UC>(smem + OFF_Q + s * QT, BOX, rr, pq, tk, S, pro,
                                  (const float2*)(smem + OFF_W), nullptr, (const float*)(smem + OFF_TH),
-                                 nullptr, bv);
+                                 nullptr, bv, n);
         fence_proxy_async();
         warp_arrive(bar_qr + 8 * s);
       }
@@ -3232,12 +3404,12 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
   }
 }
 
-template <bool PRO>
+template <bool PRO, bool UC = false>
 static cudaError_t launch_readout2(const CUtensorMap* m, long long N, int S, const ProArgs& pa,
                                    cudaStream_t st) {
   static DeviceOnce attr_once;
   const cudaError_t attr_status = once_per_device(attr_once, [&]() -> cudaError_t {
-    cudaError_t e = cudaFuncSetAttribute(k_readout2_tc<PRO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(k_readout2_tc<PRO, UC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          rd2::SMEM);
     return e;
   });
@@ -3245,8 +3417,8 @@ static cudaError_t launch_readout2(const CUtensorMap* m, long long N, int S, con
   const int parts = readout_parts(N, (S + rd2::TOK - 1) / rd2::TOK);
   const long long units = N * parts;
   const int grid = (int)(units < num_sms() ? units : num_sms());
-  k_readout2_tc<PRO><<<grid, rd2::threads(PRO), rd2::SMEM, st>>>(m[0], m[1], m[2], m[3], m[4], (int)N, S,
-                                                                  pa, parts);
+  k_readout2_tc<PRO, UC><<<grid, rd2::threads(PRO), rd2::SMEM, st>>>(m[0], m[1], m[2], m[3], m[4],
+                                                                      (int)N, S, pa, parts);
   count_launch();
   return cudaGetLastError();
 }
@@ -3267,6 +3439,7 @@ cudaError_t tc_readout2(const void* q, const void* sfr_f, const void* sfr_r, voi
   ProArgs pa = {};
   if (pro) {
     pa = *pro;
+    if (pa.ucpe) return launch_readout2<true, true>(m, N, S, pa, st);
     return launch_readout2<true>(m, N, S, pa, st);
   }
   return launch_readout2<false>(m, N, S, pa, st);

@@ -14,7 +14,7 @@ import math
 import pytest
 import torch
 
-from frame_wise_gated_b200 import api
+from frame_wise_gated_b200 import api, synth
 from tests import gdn_testutil as U
 
 pytestmark = pytest.mark.gpu
@@ -80,17 +80,21 @@ def test_forward_writes_stay_inside_buffers(case):
         assert torch.equal(out.view, ref_o) and torch.equal(st.view, ref_s), name
 
 
+@pytest.mark.parametrize("camera", [False, True])
 @pytest.mark.parametrize("bidir", [True, False])
-def test_fused_prologue_writes_stay_inside_buffers(bidir):
+def test_fused_prologue_writes_stay_inside_buffers(bidir, camera):
     B, H, T, gh, gw, D = 1, 3, 13, 20, 50, 128
     S = gh * gw
     arr = U.random_case(61, B, H, T, S, D, bf16=True, state=True)
     d = U.dev_inputs(arr, True)
     pro = dict(w_q=d["w_q"], w_k=d["w_k"], grid_h=gh, grid_w=gw)
+    if camera:
+        mq, mk = synth.make_camera(B, T, gh, gw, 61)
+        pro["ucpe_q"], pro["ucpe_k"] = torch.from_numpy(mq).cuda(), torch.from_numpy(mk).cuda()
     kw = dict(bidir=True, block_reset=True) if bidir else dict()
     out, out_r = Guarded((B, H, T, S, D), torch.bfloat16), Guarded((B, H, T, S, D), torch.bfloat16)
     st, st_r = Guarded((B, H, D, D), torch.float32), Guarded((B, H, D, D), torch.float32)
-    flags = api.scan_flags(bf16=True, prologue=True, **kw)
+    flags = api.scan_flags(bf16=True, prologue=True, **kw) | (api.UCPE if camera else 0)
     ws = guarded_ws(api.workspace_bytes(B, H, T, S, D, flags))
     extra = dict(out_rev=out_r.view, state_out_rev=st_r.view) if bidir else {}
     got = api.frame_scan_fwd_ex(d["q"], d["k"], d["v"], d["beta"], d["gamma"], d["state"],

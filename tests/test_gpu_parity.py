@@ -380,6 +380,7 @@ FULL = [
     ("rollout60s_720p", {"sequential": True, "overlap": False}),
     ("prologue_bidir_720p", {}),
     ("prologue_bidir_720p", {"overlap": False}),
+    ("prologue_ucpe_bidir_720p", {}),
     ("sweep_d64", {}),
     ("sweep_d256", {}),
     ("sweep_d256", {"chunked": True}),
@@ -393,8 +394,13 @@ def test_full_size_sampled(name, kw):
     cfg = synth.CONFIGS[name]
     arr = synth.make_inputs(cfg)
     d = U.dev_inputs(arr, cfg.bf16)
+    cam = None
+    if cfg.ucpe:  # camera matrices of the synthetic trajectory (queries D^T, keys D^-1)
+        cam = synth.make_camera(cfg.B, cfg.T, cfg.grid_h, cfg.grid_w, cfg.seed)
     if cfg.prologue:
         pro = dict(w_q=d["w_q"], w_k=d["w_k"], grid_h=cfg.grid_h, grid_w=cfg.grid_w)
+        if cam is not None:
+            pro["ucpe_q"], pro["ucpe_k"] = (torch.from_numpy(m).cuda() for m in cam)
         out, st, out_r, st_r = run_scan(d, "default", prologue=pro, bidir=True,
                                         block_reset=True, block=cfg.bidir_block, **kw)
     else:
@@ -408,9 +414,9 @@ def test_full_size_sampled(name, kw):
     for (b, h) in sorted(samples):
         if cfg.prologue:
             pro_o = (cfg.grid_w, 1e-6, 1e4)
-            o_ref, s_ref = U.oracle_slab(arr, b, h, True, prologue=pro_o)
+            o_ref, s_ref = U.oracle_slab(arr, b, h, True, prologue=pro_o, ucpe=cam)
             o_rr, s_rr = U.oracle_slab(arr, b, h, True, prologue=pro_o, reverse=True,
-                                       block=cfg.bidir_block)
+                                       block=cfg.bidir_block, ucpe=cam)
             assert U.rel_frob_per_frame(U.host(out_r[b, h]), o_rr) < U.TOL_BF16
             assert U.rel_frob_per_frame(U.host(st_r[b, h])[None], s_rr[None]) < U.TOL_BF16
         else:
