@@ -1083,8 +1083,11 @@ int gdn_check_device_status(gdn_stream_t stream) {
   int status = 0;
   e = tc_read_status(&status, st);
   if (e != cudaSuccess) return cuda_fail(e, "status read");
-  if (status) return fail(GDN_ERR_TIMEOUT, "a device-side wait ran out (code %s)",
-                          status == 1 ? "mbarrier" : "other");
+  if (status) {
+    char code[32];
+    snprintf(code, sizeof(code), "%d", status);
+    return fail(GDN_ERR_TIMEOUT, "a device-side wait ran out (wait code %s)", code);
+  }
   return GDN_OK;
 }
 

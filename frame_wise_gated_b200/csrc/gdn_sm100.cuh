@@ -63,7 +63,7 @@ __device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity,
     if ((it & 63u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer() - t0 > limit_ns) {
-        atomicExch(status, code);
+        atomicCAS(status, 0, code);  // the first wait to run out is the cause
         *abort_flag = 1;
         return false;
       }

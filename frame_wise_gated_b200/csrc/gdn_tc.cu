@@ -522,6 +522,25 @@ constexpr int SMEM_PRO = Lay<NST_PRO>::SMEM_PRO;
 static_assert(SMEM_PLAIN <= 232448 && SMEM_PRO <= 232448, "contraction shared memory");
 }  // namespace ctr
 
+// Bounded wait until the shared counter *c reaches `target`; false on abort or
+// when 2 s run out (the timeout is recorded with `code`).
+__device__ __forceinline__ bool wait_count_ge(volatile int* c, int target, volatile int* abort_flag,
+                                              int code) {
+  if (*c >= target) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (*c >= target) return true;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > kWaitNs) {
+        atomicCAS(&g_tc_status, 0, code);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // Frame-head n's A_t image (discard & 2) and U_t (discard & 1) are read once, by
 // its chain, which then adds a fifth count to flags[n]. Once that count is
 // there, epilogue warp q drops its quarter of their L2 lines without a write
@@ -589,6 +608,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
   const uint32_t bar_fin = bar_acce + 16;
   uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
   volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
+  volatile int* mma_issued = (volatile int*)(smem + OFF_MISC + 8);  // stages the MMA has issued
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
@@ -605,6 +625,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
     }
     mbar_init(bar_fin, 1);
     *abort_flag = 0;
+    *mma_issued = 0;
     fence_mbar_init();
   }
   float2* tab = (float2*)(smem + OFF_TAB);
@@ -637,6 +658,66 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
   };
   auto st_begin = [&](int i) -> int { return ((cta + i * ncta) % parts) * nst_frame / parts; };
   auto st_end = [&](int i) -> int { return ((cta + i * ncta) % parts + 1) * nst_frame / parts; };
+
+  // Stages of beta * K are taken by groups of 4 warps (128 threads each,
+  // four threads per token with the prologue: tokens pr and pr + 32 of the
+  // stage). Two scaler groups alternate stages. With the prologue, whose
+  // arithmetic sets the pace, the 4 epilogue warps (busy only once per unit)
+  // form a third group: a unit's first 8 stages alternate between groups 0
+  // and 1, later stages rotate over all three, so the epilogue's drain of
+  // the previous unit at the start of a unit holds up no early stage.
+  constexpr bool EPI3 = NST == NST_PRO;
+  auto stage_owner = [&](int i, int st, int g) -> int {
+    if (!EPI3) return g & 1;
+    const int r = st - st_begin(i);
+    return r < 8 ? (r & 1) : (r - 8) % 3;
+  };
+  // One stage by one group (tt = 0..127); false if a wait ran out.
+  auto scale_stage = [&](int i, int st, int g, int tt) -> bool {
+    const int pr = pro_lane_row(tt), pq = pro_lane_quarter(tt);
+    const int s = g % NST, kb = g % NBK;
+    const uint32_t u = (uint32_t)(g / NST);
+    // Stage s and slot kb pass between groups, and their barriers are waited
+    // on by parity, which tells only the last two phases apart: with three
+    // groups, first let the MMA issue the previous uses of both (stages
+    // g - NST and g - NBK). Then the wanted phase is the next one on each.
+    constexpr int PREV = NST < NBK ? NST : NBK;
+    if (EPI3 && !wait_count_ge(mma_issued, g - PREV + 1, abort_flag, 9)) return false;
+    bool ok = mbar_wait(bar_full + 8 * s, u & 1, abort_flag, &g_tc_status, 6);
+    // the slot's previous beta * K has been consumed by its MMAs
+    if (ok) ok = mbar_wait(bar_bke + 8 * kb, ((uint32_t)(g / NBK) & 1) ^ 1, abort_flag, &g_tc_status, 8);
+    if (!ok) return false;
+    uint8_t* kt = smem + OFF_K + s * 2 * TILE;
+    uint8_t* bt = smem + OFF_BK + kb * TILE;
+    const float* bs = (const float*)(smem + OFF_BETA) + s * TOK;
+    if (pro.w) {
+      // raw k -> K^ in place (RMSNorm, ReLU, RoPE) and beta * K^ into the slot
+      const int rr[2] = {pr, pr + 32}, tk[2] = {st * TOK + pr, st * TOK + pr + 32};
+      const float bv[2] = {beta ? bs[pr] : 1.f, beta ? bs[pr + 32] : 1.f};
+      pro_rows<2, false, true, UC>(kt, BOX, rr, pq, tk, S, pro, w4, tab, nullptr, bt, bv,
+                                   unit_n(i));
+      fence_proxy_async();
+      warp_arrive(bar_bkf + 8 * kb);
+      return true;
+    }
+#pragma unroll
+    for (int m = 0; m < 1024 / (NSC / 2); ++m) {
+      const int c = tt + (NSC / 2) * m;   // 16-byte chunk of the 16 KiB tile
+      const float bv = beta ? bs[(c >> 3) & (TOK - 1)] : 1.f;  // 8 chunks per 128-byte token row
+      uint4 x = *(const uint4*)(kt + c * 16);
+      uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&w[e]);
+        float2 f = __bfloat1622float2(h);
+        w[e] = pack_bf16x2(f.x * bv, f.y * bv);
+      }
+      *(uint4*)(bt + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    fence_proxy_async();
+    warp_arrive(bar_bkf + 8 * kb);
+    return true;
+  };
 
   if (warp == 0) {
     // ---- TMA producer (lane 0 issues; the warp loads beta) ----
@@ -714,6 +795,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
           }
           mma_commit(bar_empty + 8 * s);
           mma_commit(bar_bke + 8 * kb);
+          if (EPI3) *mma_issued = g + 1;
         }
         if (!ok) break;
         mma_commit(bar_accf + 8 * b);
@@ -725,64 +807,30 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
   } else if (warp < 2 + NSC / 32) {
     // ---- beta * K into the B operand tile (same swizzled layout as K) ----
     const int t = threadIdx.x - 64;
-    // The scalers work as two groups of 4 warps on alternate stages (group
-    // g % 2 takes stage g and its beta * K slot), so two stages are in flight.
-    // Prologue: four threads per token (32 channels each), tokens pr and pr + 32.
     const int grp = t >> 7, tt = t & 127;
-    const int pr = pro_lane_row(tt), pq = pro_lane_quarter(tt);
     int g = 0;
     bool ok = true;
     for (int i = 0; i < my_count && ok; ++i) {
       for (int st = st_begin(i); st < st_end(i); ++st, ++g) {
-        if ((g & 1) != grp) continue;
-        const int s = g % NST, kb = g % NBK;
-        const uint32_t u = (uint32_t)(g / NST);
-        ok = mbar_wait(bar_full + 8 * s, u & 1, abort_flag, &g_tc_status, 6);
-        // the slot's previous beta * K has been consumed by its MMAs
-        if (ok) ok = mbar_wait(bar_bke + 8 * kb, ((uint32_t)(g / NBK) & 1) ^ 1, abort_flag, &g_tc_status, 8);
-        if (!ok) break;
-        uint8_t* kt = smem + OFF_K + s * 2 * TILE;
-        uint8_t* bt = smem + OFF_BK + kb * TILE;
-        const float* bs = (const float*)(smem + OFF_BETA) + s * TOK;
-        if (pro.w) {
-          // raw k -> K^ in place (RMSNorm, ReLU, RoPE) and beta * K^ into the slot
-          const int rr[2] = {pr, pr + 32}, tk[2] = {st * TOK + pr, st * TOK + pr + 32};
-          const float bv[2] = {beta ? bs[pr] : 1.f, beta ? bs[pr + 32] : 1.f};
-          pro_rows<2, false, true, UC>(kt, BOX, rr, pq, tk, S, pro, w4, tab, nullptr, bt, bv,
-                                       unit_n(i));
-          fence_proxy_async();
-          warp_arrive(bar_bkf + 8 * kb);
-          continue;
+        if (stage_owner(i, st, g) != grp) continue;
+        if (!scale_stage(i, st, g, tt)) {
+          ok = false;
+          break;
         }
-#pragma unroll
-        for (int m = 0; m < 1024 / (NSC / 2); ++m) {
-          const int c = tt + (NSC / 2) * m;   // 16-byte chunk of the 16 KiB tile
-          const float bv = beta ? bs[(c >> 3) & (TOK - 1)] : 1.f;  // 8 chunks per 128-byte token row
-          uint4 x = *(const uint4*)(kt + c * 16);
-          uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&w[e]);
-            float2 f = __bfloat1622float2(h);
-            w[e] = pack_bf16x2(f.x * bv, f.y * bv);
-          }
-          *(uint4*)(bt + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        fence_proxy_async();
-        warp_arrive(bar_bkf + 8 * kb);
       }
     }
   } else if (warp < 2 + NSC / 32 + 4) {
     // ---- epilogue: TMEM -> scale -> fp32 A_t, U_t rows ----
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    for (int i = 0; i < my_count; ++i) {
+    // unit i's accumulator out of TMEM; false if a wait ran out
+    auto epi = [&](int i) -> bool {
       const int b = i & 1;
       const uint32_t ub = (uint32_t)(i >> 1);
       // lane 0 waits and the warp follows its decision (warp-uniform control flow)
       int ok = 1;
       if (lane == 0) ok = mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 7);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
       __syncwarp();
       tc_fence_after();
       const int n = unit_n(i);
@@ -860,11 +908,34 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
         // (count 5: 4 publications + 1 consumption), are never read again
         if (discard && i > 0) drop_consumed(A, U, flags, unit_n(i - 1), q, lane, discard, 0);
       }
+      return true;
+    };
+    if (EPI3) {
+      // third scaler group: drain the previous unit, then take this unit's stages
+      const int tt = threadIdx.x - (64 + NSC);
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; i < my_count && ok; ++i) {
+        if (i > 0 && !epi(i - 1)) {
+          ok = false;
+          break;
+        }
+        for (int st = st_begin(i); st < st_end(i); ++st, ++g) {
+          if (stage_owner(i, st, g) != 2) continue;
+          if (!scale_stage(i, st, g, tt)) {
+            ok = false;
+            break;
+          }
+        }
+      }
+      if (ok && my_count > 0) epi(my_count - 1);
+    } else {
+      for (int i = 0; i < my_count; ++i)
+        if (!epi(i)) break;
     }
     // this CTA's last unit: its chain reads it shortly; wait for that a while
     if (discard && my_count > 0) drop_consumed(A, U, flags, unit_n(my_count - 1), q, lane, discard, 1);
   }
-
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -2167,7 +2238,7 @@ __device__ __forceinline__ bool wait_flag_ge(const int* f, int target, volatile 
     if ((it & 15u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer() - t0 > kWaitNs) {
-        atomicExch(&g_tc_status, code);
+        atomicCAS(&g_tc_status, 0, code);  // the first wait to run out is the cause
         *abort_flag = 1;
         return false;
       }
