@@ -145,10 +145,8 @@ Layout make_layout(int B, int H, int T, int S, int D, unsigned flags) {
   off = align256(off + heads * L.nseg_max * sizeof(float));
   L.flags = off;  // per frame-head publication counters of the overlapped plan
   off = align256(off + frames * sizeof(int));
-  L.qh = L.kh = L.rope = off;
+  L.qh = L.kh = off;
   if (flags & GDN_FUSED_PROLOGUE) {
-    L.rope = off;  // (cos, sin) table: positions [0, S) x pairs [0, D/4)
-    off = align256(off + (size_t)S * (D / 4) * 8);
     const size_t elt = (flags & GDN_BF16) ? 2 : 4;
     const size_t tens = frames * (size_t)S * D * elt;
     L.qh = off;
@@ -345,17 +343,11 @@ static int scan_ex(const gdn_params& p, cudaStream_t st) {
       // Fused: the tensor-core loaders apply RMSNorm, ReLU and RoPE to the raw
       // tiles in shared memory; the key scale goes into the contraction's
       // epilogue constants (RoPE is linear, so the order does not matter).
+      // Each CTA computes its (cos, sin) table into shared memory at start-up.
       const int npos = p.grid_h > p.grid_w ? p.grid_h : p.grid_w;
-      float2* cs = (float2*)(ws + L.rope);
-      {
-        PhaseScope ps(PH_PROLOGUE, st);
-        // with the camera encoding the RoPE acts on D/2 channels
-        e = rope_table(cs, npos, (f & GDN_UCPE) ? p.D / 2 : p.D, base, st);
-      }
-      if (e != cudaSuccess) return cuda_fail(e, "rope table");
       const bool cam = (f & GDN_UCPE) != 0;
-      pro_k = ProArgs{p.w_k, cs, p.grid_w, eps, npos, base, cam ? p.ucpe_k : nullptr, p.H, p.T};
-      pro_q = ProArgs{p.w_q, cs, p.grid_w, eps, npos, base, cam ? p.ucpe_q : nullptr, p.H, p.T};
+      pro_k = ProArgs{p.w_k, p.grid_w, eps, npos, base, cam ? p.ucpe_k : nullptr, p.H, p.T};
+      pro_q = ProArgs{p.w_q, p.grid_w, eps, npos, base, cam ? p.ucpe_q : nullptr, p.H, p.T};
       ppk = &pro_k;
       ppq = &pro_q;
     } else {

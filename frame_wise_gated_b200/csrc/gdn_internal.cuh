@@ -113,7 +113,7 @@ __host__ __device__ __forceinline__ void seg_range(const ChainArgs& a, int p, in
 
 // ---- workspace layout ---------------------------------------------------------
 struct Layout {
-  size_t A, U, Sfr, Sfr2, E, Hc, g, Sst, qh, kh, rope, flags, total;
+  size_t A, U, Sfr, Sfr2, E, Hc, g, Sst, qh, kh, flags, total;
   int nseg_max;
 };
 
@@ -169,8 +169,6 @@ cudaError_t simt_bwd_combine(bool bf16, const void* k, const float* beta, const 
 // the key scale is folded into the contraction's epilogue constants).
 struct ProArgs {
   const float* w;    // [D] RMSNorm weight
-  const float2* cs;  // [D/4][npos] (cos, sin) of pos * base^(-2i/(D/2)), pair-major; with
-                     // ucpe: [D/8][npos] of the RoPE on D/2 channels
   int grid_w;
   float eps;
   int npos;

@@ -430,13 +430,18 @@ __device__ __forceinline__ void pro_rows(uint8_t* tile, int box_bytes, const int
     pro_rows_rope<NR, THETA, BTILE>(tile, box_bytes, rr, q, tk, S, pro, w4, tab, theta, btile, bv);
 }
 
-// Copies the (cos, sin) table (pair-major, cs[i * npos + pos]) into shared
-// memory in pro_table_index order.
-__device__ __forceinline__ void pro_table_copy(float2* tab, const ProArgs& pro) {
-  const int npairs = pro.ucpe ? 16 : 32;  // the RoPE's channels: 64 with the camera encoding
+// Fills the shared (cos, sin) table in pro_table_index order: entry (i, pos)
+// holds the turn of pair i at position pos, pos * base^(-2i/(Dr/2)) for the
+// RoPE's Dr channels (128, or 64 with the camera encoding), by
+// rope_cs_reduced (the bidirectional readout's function). Each CTA computes
+// its own copy at start-up (a few thousand entries over all its threads), so
+// no separate table launch precedes the kernel.
+__device__ __forceinline__ void pro_table_fill(float2* tab, const ProArgs& pro) {
+  const int dr = pro.ucpe ? 64 : 128;
+  const int npairs = dr / 4;
   for (int e = threadIdx.x; e < pro.npos * npairs; e += (int)blockDim.x) {
     const int i = e / pro.npos, pos = e - i * pro.npos;
-    tab[pro_table_index(i, pos)] = pro.cs[e];
+    tab[pro_table_index(i, pos)] = rope_cs_reduced(pos, rope_theta(pro.base, i, dr));
   }
 }
 
@@ -631,7 +636,7 @@ __device__ __forceinline__ void contract_body(const CUtensorMap& tmK, const CUte
   float2* tab = (float2*)(smem + OFF_TAB);
   float2* w4 = (float2*)(smem + Ly::OFF_W4);
   if (pro.w) {
-    pro_table_copy(tab, pro);
+    pro_table_fill(tab, pro);
     pro_w_copy(w4, pro.w);
   }
   if (warp == 1) {
@@ -1075,7 +1080,7 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
     fence_mbar_init();
   }
   if (PRO) {
-    pro_table_copy((float2*)(smem + OFF_TAB), pro);
+    pro_table_fill((float2*)(smem + OFF_TAB), pro);
     pro_w_copy((float2*)(smem + OFF_W4), pro.w);
   }
   if (warp == 1) {
@@ -1195,8 +1200,8 @@ __global__ void __launch_bounds__(rdo::threads(PRO), 1)
         tc_fence_after();
         // the previous tile's TMA store has finished reading the staging tile
         if (et == 0) bulk_wait_read0();
-        named_bar_sync(1, 128);
-        if (*abort_flag) {  // uniform across the four epilogue warps
+        // one decision for all four epilogue warps: the flag may be set while they read it
+        if (named_bar_or(1, 128, *abort_flag != 0)) {
           ok = false;
           break;
         }
@@ -1672,8 +1677,7 @@ __global__ void __launch_bounds__(chn::THREADS, 1)
         }
       }
     }
-    __syncthreads();
-    if (*abort_flag) break;  // uniform: read after the barrier
+    if (__syncthreads_or(*abort_flag != 0)) break;  // one decision for the CTA
     if (leader) {
       if (store_sfr && tprev >= 0) store_tile(g.bh * a.T + tprev);  // S after frame tprev
       if (store_sst) store_tile(g.bh * a.nseg + s);                  // S_start(s)
@@ -2352,8 +2356,7 @@ __device__ __forceinline__ void ovl_chain_body(const OvlArgs& o, const CUtensorM
       fence_proxy_async();
     }
     mbar_wait(bar_y, (uint32_t)j & 1, abort_flag, &g_tc_status, 32);
-    __syncthreads();
-    if (*abort_flag) break;  // uniform: read after the barrier
+    if (__syncthreads_or(*abort_flag != 0)) break;  // one decision for the CTA
     if (leader) {
       tc_fence_after();
       const uint32_t yh = sb + OFF_Y, yl = yh + 2 * ATOM;
@@ -2893,8 +2896,7 @@ __global__ void __launch_bounds__(r64::THREADS, 1)
         mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 69);
         tc_fence_after();
         if (et == 0) bulk_wait_read0();
-        named_bar_sync(1, 128);
-        if (*abort_flag) {
+        if (named_bar_or(1, 128, *abort_flag != 0)) {
           ok = false;
           break;
         }
@@ -3073,8 +3075,7 @@ __global__ void __launch_bounds__(h64::THREADS)
         }
       }
     }
-    __syncthreads();
-    if (*abort_flag) break;
+    if (__syncthreads_or(*abort_flag != 0)) break;  // one decision for the CTA
     if (leader) {
       if (store_sfr && tprev >= 0) store_tile(g.bh * a.T + tprev);
       if (store_sst) store_tile(g.bh * a.nseg + s);
@@ -3407,8 +3408,7 @@ __global__ void __launch_bounds__(rd2::threads(PRO), 1)
           const int dir = rnd >> 1, half = rnd & 1, buf = nstores & 1;
           // the store that last used this staging buffer has read it
           if (et == 0 && nstores >= 2) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-          named_bar_sync(1, 128);
-          if (*abort_flag) {
+          if (named_bar_or(1, 128, *abort_flag != 0)) {
             ok = false;
             break;
           }
@@ -3754,6 +3754,275 @@ __global__ void __launch_bounds__(c256::THREADS, 1)
   }
 }
 
+// D = 256 contraction on a CTA pair (a cluster of two CTAs, one tcgen05
+// MMA of M = 256 over both). Per frame-head and 64-token stage CTA r of the
+// pair loads only channels 128r .. 128r + 127 of K and of V (TMA, 128-byte
+// swizzle, evict-first) and scales its K half by beta; the even CTA then
+// issues, per 16 tokens,
+//     A += K^T (beta K),  U += V^T (beta K)        (M = 256, N = 256, K = 16)
+// with the A operands (K, V) split by rows and the B operand (beta K) split
+// by columns over the two CTAs' shared memory, so each byte of K and V is
+// read from memory once and multiplied once. CTA r's TMEM receives rows
+// 128r .. of A (columns 0-255) and of U (256-511); its eight epilogue warps
+// (four on A, four on U) write them as k_contract256_tc does. Barriers: stage
+// and beta*K slot releases are multicast MMA commits to both CTAs. The even
+// CTA's scalers arrive on its slot barrier directly; the odd CTA's arrive on
+// a local barrier, and a relay warp per slot forwards each completed use of
+// it with one cluster-scope arrival, so the scaler warps never wait on a
+// cluster-wide release and the releases of successive stages overlap. The epilogue warps of both CTAs arrive on the even
+// CTA's accumulator barrier. The MMA thread thus starts a stage once both
+// halves of its beta*K are written and a unit once both CTAs have drained
+// their accumulators.
+namespace cp256 {
+constexpr int D = 256;
+constexpr int TOK = 64;                 // tokens per stage
+constexpr int NST = 5;                  // stages
+constexpr int NBK = 4;                  // beta * K slots (each stage's slot waits for the
+                                        // pair's MMAs NBK stages back, across both CTAs)
+constexpr int BOX = TOK * 128;          // [64 tokens][64 channels]: 8 KiB
+constexpr int HT = 2 * BOX;             // this CTA's 128 channels of a stage: 16 KiB
+constexpr int OFF_K = 0;
+constexpr int OFF_V = OFF_K + NST * HT;
+constexpr int OFF_BK = OFF_V + NST * HT;
+constexpr int OFF_BETA = OFF_BK + NBK * HT;
+constexpr int OFF_BAR = OFF_BETA + NST * TOK * 4;
+constexpr int NBAR = 2 * NST + 3 * NBK + 3;  // full, empty; bk_full, bk_empty, bk_local; acc f/e, fin
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+static_assert(SMEM <= 232448, "D = 256 pair contraction shared memory");
+constexpr int NSC = 128;                // scaler threads
+constexpr int NEPI = 8;                 // epilogue warps
+constexpr int NRELAY = NBK;             // relay warps of the odd CTA, one per slot
+constexpr int THREADS = 64 + NSC + 32 * NEPI + 32 * NRELAY;
+constexpr uint32_t TMEM_COLS = 512;
+static_assert((HT / 16) % NSC == 0, "scaler chunks");
+}  // namespace cp256
+
+__global__ void __launch_bounds__(cp256::THREADS, 1)
+    k_contract256_pair_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                          const float* __restrict__ beta, float* __restrict__ A, float* __restrict__ U,
+                          int N, int S, float cA, float cU, int a_image) {
+  using namespace cp256;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the pair's MMAs
+  const uint32_t bar_full = sb + OFF_BAR;
+  const uint32_t bar_empty = bar_full + 8 * NST;
+  const uint32_t bar_bkf = bar_empty + 8 * NST;
+  const uint32_t bar_bke = bar_bkf + 8 * NBK;
+  const uint32_t bar_bkl = bar_bke + 8 * NBK;
+  const uint32_t bar_accf = bar_bkl + 8 * NBK;
+  const uint32_t bar_acce = bar_accf + 8;
+  const uint32_t bar_fin = bar_acce + 8;
+  uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bar_full + 8 * s, 33);  // expect_tx + 32 lanes' beta copies
+      mbar_init(bar_empty + 8 * s, 1);  // the pair's MMA commit
+    }
+    for (int s = 0; s < NBK; ++s) {
+      mbar_init(bar_bkf + 8 * s, NSC / 32 + 1);  // this CTA's scaler warps + the odd CTA's relay
+      mbar_init(bar_bke + 8 * s, 1);
+      mbar_init(bar_bkl + 8 * s, NSC / 32);      // the odd CTA's scaler warps
+    }
+    mbar_init(bar_accf, 1);
+    mbar_init(bar_acce, 2 * NEPI);  // the epilogue warps of both CTAs
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before either arrives on the other's
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int nst_frame = (S + TOK - 1) / TOK;
+  const int pair = (int)blockIdx.x >> 1, npair = (int)gridDim.x >> 1;
+  const int my_count = pair < N ? (N - 1 - pair) / npair + 1 : 0;
+
+  if (warp == 0) {
+    const uint64_t pol = l2_policy_evict_first();  // K and V are read once
+    int g = 0;
+    bool ok = true;
+    for (int i = 0; i < my_count && ok; ++i) {
+      const int n = pair + i * npair;
+      for (int st = 0; st < nst_frame; ++st, ++g) {
+        const int s = g % NST;
+        const uint32_t u = (uint32_t)(g / NST);
+        if (lane == 0) ok = mbar_wait(bar_empty + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 121);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar_full + 8 * s, 2 * HT);
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            const int ch = 128 * (int)rank + 64 * x;
+            tma_load_3d_hint(sb + OFF_K + s * HT + x * BOX, &tmK, bar_full + 8 * s, ch, st * TOK, n, pol);
+            tma_load_3d_hint(sb + OFF_V + s * HT + x * BOX, &tmV, bar_full + 8 * s, ch, st * TOK, n, pol);
+          }
+        }
+        const uint32_t bsa = sb + OFF_BETA + s * TOK * 4;
+#pragma unroll
+        for (int r = lane; r < TOK; r += 32) {
+          const int tok = st * TOK + r;
+          const bool in = tok < S;
+          cp_async_4(bsa + r * 4, beta + (size_t)n * S + (in ? tok : 0), in ? 4u : 0u);
+        }
+        cp_async_arrive_noinc(bar_full + 8 * s);
+      }
+    }
+    if (lane == 0)
+      for (int gg = (g > NST ? g - NST : 0); gg < g; ++gg)
+        mbar_wait(bar_full + 8 * (gg % NST), (uint32_t)(gg / NST) & 1, abort_flag, &g_tc_status, 122);
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(256, 256, true, true);
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; i < my_count && ok; ++i) {
+        ok = mbar_wait_cluster(bar_acce, ((uint32_t)i & 1) ^ 1, abort_flag, &g_tc_status, 123);
+        if (!ok) break;
+        tc_fence_after();
+        for (int st = 0; st < nst_frame; ++st, ++g) {
+          const int s = g % NST, kb = g % NBK;
+          ok = mbar_wait_cluster(bar_bkf + 8 * kb, (uint32_t)(g / NBK) & 1, abort_flag, &g_tc_status, 124);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t ka = sb + OFF_K + s * HT, va = sb + OFF_V + s * HT, ba = sb + OFF_BK + kb * HT;
+#pragma unroll
+          for (int kk = 0; kk < TOK / 16; ++kk) {
+            const uint64_t db = smem_desc_sw128(ba + kk * 2048, BOX, 1024);
+            const uint32_t acc = (st > 0 || kk > 0) ? 1u : 0u;
+            mma_bf16_pair(tmem, smem_desc_sw128(ka + kk * 2048, BOX, 1024), db, idesc, acc);
+            mma_bf16_pair(tmem + 256, smem_desc_sw128(va + kk * 2048, BOX, 1024), db, idesc, acc);
+          }
+          mma_commit_pair(bar_empty + 8 * s, 3);
+          mma_commit_pair(bar_bke + 8 * kb, 3);
+        }
+        if (!ok) break;
+        mma_commit_pair(bar_accf, 3);
+      }
+      mma_commit_pair(bar_fin, 3);
+    }
+    __syncwarp();
+  } else if (warp >= 2 + NSC / 32 + NEPI) {
+    // relay warp kb of the odd CTA: forwards each use of beta * K slot kb that
+    // this CTA's scalers completed to the even CTA's slot barrier
+    const int kb = warp - (2 + NSC / 32 + NEPI);
+    if (rank != 0 && lane == 0) {
+      const uint32_t bkf_lead = mapa_shared(bar_bkf + 8 * kb, 0);
+      const int total = my_count * nst_frame;  // stages kb, kb + NBK, ... of this CTA
+      for (int g = kb, u = 0; g < total; g += NBK, ++u) {
+        if (!mbar_wait(bar_bkl + 8 * kb, (uint32_t)u & 1, abort_flag, &g_tc_status, 129)) break;
+        mbar_arrive_cluster(bkf_lead);
+      }
+    }
+    __syncwarp();
+  } else if (warp < 2 + NSC / 32) {
+    const int t = threadIdx.x - 64;
+    const uint32_t bar_done = rank == 0 ? bar_bkf : bar_bkl;  // see the relay warps
+    int g = 0;
+    bool ok = true;
+    for (int i = 0; i < my_count && ok; ++i) {
+      for (int st = 0; st < nst_frame; ++st, ++g) {
+        const int s = g % NST, kb = g % NBK;
+        const uint32_t u = (uint32_t)(g / NST);
+        ok = mbar_wait(bar_full + 8 * s, u & 1, abort_flag, &g_tc_status, 125);
+        // the slot's previous beta * K has been consumed by the pair's MMAs
+        if (ok) ok = mbar_wait(bar_bke + 8 * kb, ((uint32_t)(g / NBK) & 1) ^ 1, abort_flag, &g_tc_status, 126);
+        if (!ok) break;
+        const uint8_t* kt = smem + OFF_K + s * HT;
+        uint8_t* bt = smem + OFF_BK + kb * HT;
+        const float* bs = (const float*)(smem + OFF_BETA) + s * TOK;
+#pragma unroll
+        for (int m = 0; m < (HT / 16) / NSC; ++m) {
+          const int c = t + NSC * m;
+          const float bv = bs[(c >> 3) & (TOK - 1)];
+          const uint4 x = *(const uint4*)(kt + c * 16);
+          uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
+            w[e] = pack_bf16x2(f.x * bv, f.y * bv);
+          }
+          *(uint4*)(bt + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async();
+        warp_arrive(bar_done + 8 * kb);
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int mat = (warp - 2 - NSC / 32) >> 2;  // 0: A, 1: U
+    const int row = q * 32 + lane;
+    const int k = 128 * (int)rank + row;
+    const uint32_t acce_lead = mapa_shared(bar_acce, 0);
+    const float sc = mat ? cU : cA;
+    for (int i = 0; i < my_count; ++i) {
+      const int n = pair + i * npair;
+      if (!mbar_wait(bar_accf, (uint32_t)i & 1, abort_flag, &g_tc_status, 127)) break;
+      tc_fence_after();
+      float* dst = (mat ? U : A) + ((size_t)n * D + k) * D;
+      uint8_t* img = (uint8_t*)A + (size_t)n * D * D * 4;
+      for (int c0 = 0; c0 < 256; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + mat * 256 + c0, r);
+        tmem_wait_ld();
+        if (mat == 0 && a_image) {
+          // row k of A_t into the operand image (hi, lo) of the D = 256 chains
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * j + e]) * sc;
+            uint4 hi, lo;
+            split_chunk(v, &hi, &lo);
+            const int off = img256_off(k, (c0 >> 3) + j);
+            *(uint4*)(img + off) = hi;
+            *(uint4*)(img + off + 8192) = lo;
+          }
+        } else if (mat == 1 && a_image) {
+          // U_t transposed for the D = 256 chains
+          float* ut = U + (size_t)n * D * D + k;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) ut[(size_t)(c0 + j) * D] = __uint_as_float(r[j]) * sc;
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *(float4*)(dst + c0 + 4 * j) =
+                make_float4(__uint_as_float(r[4 * j]) * sc, __uint_as_float(r[4 * j + 1]) * sc,
+                            __uint_as_float(r[4 * j + 2]) * sc, __uint_as_float(r[4 * j + 3]) * sc);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acce_lead);
+    }
+  }
+  // Teardown: every MMA of the pair has completed (bar_fin, multicast), and
+  // neither CTA leaves while the other may still arrive on its barriers.
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1 && lane == 0) {
+    volatile int keep_waiting = 0;
+    mbar_wait(bar_fin, 0, &keep_waiting, &g_tc_status, 128);
+  }
+  __syncwarp();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
 namespace r256 {
 constexpr int D = 256;
 constexpr int TOK = 128;
@@ -3905,8 +4174,7 @@ __global__ void __launch_bounds__(r256::THREADS, 1)
         mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 119);
         tc_fence_after();
         if (et == 0) bulk_wait_read0();
-        named_bar_sync(1, 128);
-        if (*abort_flag) {
+        if (named_bar_or(1, 128, *abort_flag != 0)) {
           ok = false;
           break;
         }
@@ -3947,9 +4215,305 @@ __global__ void __launch_bounds__(r256::THREADS, 1)
   }
 }
 
+// D = 256 readout on a CTA pair: tiles of 256 tokens, CTA r of the pair
+// loading tokens 128r .. 128r + 127 of each (all 256 channels, as four
+// 64-channel stages of a four-stage ring) and holding rows 128r .. of S_t
+// (hi, lo: 128 KiB). The even CTA issues O = Q S_hi^T + Q S_lo^T as M = 256
+// (tokens, split over the pair), N = 256 (columns of O, split over the pair's
+// S halves) MMAs, so each Q tile is read once; CTA r's TMEM receives its 128
+// tokens x 256 columns (double-buffered: 2 x 256 columns), read by its eight
+// epilogue warps (two per TMEM lane quarter, 128 columns each) in one batch
+// of TMEM loads, released to the MMA, then written back in four passes of
+// 64 columns through two 16 KiB staging boxes taken in turn, each pass one
+// TMA store. Both CTAs' Q and S loads complete their bytes on
+// the even CTA's barriers (the odd CTA's through the pair form of the TMA
+// load), which expect the bytes of both; stage and S releases are multicast
+// MMA commits; each CTA's epilogue signals the even CTA once per tile.
+namespace rp256 {
+constexpr int D = 256;
+constexpr int TOK = 128;                 // tokens per CTA and tile (256 per pair)
+constexpr int NQ = 4;                    // Q stages of 64 channels (four per tile)
+constexpr int BOX = TOK * 128;           // [128 rows][64 channels]: 16 KiB
+static_assert(4 * BOX == TOK * D * 2, "four stages hold a tile's D bf16 channels");
+constexpr int OFF_Q = 0;
+constexpr int OFF_S = OFF_Q + NQ * BOX;  // S rows half: hi 4 boxes, lo 4 boxes (128 KiB)
+constexpr int OFF_O = OFF_S + 8 * BOX;   // output staging: two boxes, used in turn
+constexpr int OFF_BAR = OFF_O + 2 * BOX;
+constexpr int NBAR = 2 * NQ + 2 + 4 + 1;  // qf, qe; sf, se; accf x2, acce x2; fin
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr int SMEM = OFF_MISC + 16 + 1024;
+static_assert(SMEM <= 232448, "D = 256 pair readout shared memory");
+constexpr int NEPI = 8;                  // epilogue warps
+constexpr int THREADS = 64 + 32 * NEPI;
+constexpr uint32_t TMEM_COLS = 512;
+}  // namespace rp256
+
+__global__ void __launch_bounds__(rp256::THREADS, 1)
+    k_readout256_pair_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
+                         const __grid_constant__ CUtensorMap tmO, int N, int S) {
+  using namespace rp256;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the pair's MMAs
+  const uint32_t bar_qf = sb + OFF_BAR;
+  const uint32_t bar_qe = bar_qf + 8 * NQ;
+  const uint32_t bar_sf = bar_qe + 8 * NQ;
+  const uint32_t bar_se = bar_sf + 8;
+  const uint32_t bar_accf = bar_se + 8;
+  const uint32_t bar_acce = bar_accf + 16;
+  const uint32_t bar_fin = bar_acce + 16;
+  uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
+  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NQ; ++s) {
+      mbar_init(bar_qf + 8 * s, 1);  // the even CTA's expect; the bytes of both CTAs
+      mbar_init(bar_qe + 8 * s, 1);
+    }
+    mbar_init(bar_sf, 1);
+    mbar_init(bar_se, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_accf + 8 * b, 1);
+      mbar_init(bar_acce + 8 * b, 2);  // one arrival per CTA
+    }
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before either arrives on the other's
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int ntile = (S + 2 * TOK - 1) / (2 * TOK);
+  const int pair = (int)blockIdx.x >> 1, npair = (int)gridDim.x >> 1;
+  const int my_count = pair < N ? (N - 1 - pair) / npair + 1 : 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // loads land in this CTA's shared memory; their bytes complete on the
+      // even CTA's barriers
+      const uint32_t qf_lead = mapa_shared(bar_qf, 0), sf_lead = mapa_shared(bar_sf, 0);
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; i < my_count && ok; ++i) {
+        const int n = pair + i * npair;
+        ok = mbar_wait(bar_se, ((uint32_t)i & 1) ^ 1, abort_flag, &g_tc_status, 131);
+        if (!ok) break;
+        if (rank == 0) mbar_arrive_expect_tx(bar_sf, 2 * 8 * BOX);
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+          for (int x = 0; x < 4; ++x)
+            tma_load_3d_pair(sb + OFF_S + (4 * hl + x) * BOX, &tmS, sf_lead, 64 * x, 128 * (int)rank,
+                             2 * n + hl);
+        for (int tl = 0; tl < ntile && ok; ++tl)
+          for (int qq = 0; qq < 4; ++qq, ++g) {
+            const int s = g % NQ;
+            const uint32_t u = (uint32_t)(g / NQ);
+            ok = mbar_wait(bar_qe + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 132);
+            if (!ok) break;
+            const int tok0 = 2 * TOK * tl + TOK * (int)rank;  // may lie past S: zero fill
+            if (rank == 0) mbar_arrive_expect_tx(bar_qf + 8 * s, 2 * BOX);
+            tma_load_3d_pair(sb + OFF_Q + s * BOX, &tmQ, qf_lead + 8 * s, 64 * qq, tok0, n);
+          }
+      }
+      // the even CTA's barriers count both CTAs' bytes: its drain covers the pair
+      if (rank == 0) {
+        for (int gg = (g > NQ ? g - NQ : 0); gg < g; ++gg)
+          mbar_wait(bar_qf + 8 * (gg % NQ), (uint32_t)(gg / NQ) & 1, abort_flag, &g_tc_status, 133);
+        if (my_count > 0) mbar_wait(bar_sf, (uint32_t)(my_count - 1) & 1, abort_flag, &g_tc_status, 134);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(256, 256, false, false);
+      int g = 0, gt = 0;
+      bool ok = true;
+      for (int i = 0; i < my_count && ok; ++i) {
+        ok = mbar_wait(bar_sf, (uint32_t)i & 1, abort_flag, &g_tc_status, 135);
+        if (!ok) break;
+        tc_fence_after();
+        for (int tl = 0; tl < ntile && ok; ++tl, ++gt) {
+          const int b = gt & 1;
+          const uint32_t ub = (uint32_t)(gt >> 1);
+          ok = mbar_wait_cluster(bar_acce + 8 * b, (ub & 1) ^ 1, abort_flag, &g_tc_status, 137);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t d = tmem + b * 256;
+          for (int qq = 0; qq < 4 && ok; ++qq, ++g) {
+            const int s = g % NQ;
+            ok = mbar_wait(bar_qf + 8 * s, (uint32_t)(g / NQ) & 1, abort_flag, &g_tc_status, 138);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t qa = sb + OFF_Q + s * BOX;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t soff = qq * BOX + kk * 32;
+              const uint64_t dq = smem_desc_sw128(qa + kk * 32, 16, 1024);
+              mma_bf16_pair(d, dq, smem_desc_sw128(sb + OFF_S + soff, 16, 1024), idesc,
+                            (qq > 0 || kk > 0) ? 1u : 0u);
+              mma_bf16_pair(d, dq, smem_desc_sw128(sb + OFF_S + 4 * BOX + soff, 16, 1024), idesc, 1u);
+            }
+            mma_commit_pair(bar_qe + 8 * s, 3);
+          }
+          if (!ok) break;
+          mma_commit_pair(bar_accf + 8 * b, 3);
+        }
+        if (!ok) break;
+        mma_commit_pair(bar_se, 3);
+      }
+      mma_commit_pair(bar_fin, 3);
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3;                // TMEM lane quarter
+    const int h = (warp - 2) >> 2;         // 32-column half of a pass
+    const int row = q * 32 + lane;
+    const int et = threadIdx.x - 64;
+    constexpr int NET = 32 * NEPI;
+    const uint32_t acce_lead = mapa_shared(bar_acce, 0);
+    int gt = 0, npass = 0;
+    bool ok = true;
+    for (int i = 0; i < my_count && ok; ++i) {
+      const int n = pair + i * npair;
+      for (int tl = 0; tl < ntile; ++tl, ++gt) {
+        const int b = gt & 1;
+        const uint32_t ub = (uint32_t)(gt >> 1);
+        const int tok0 = 2 * TOK * tl + TOK * (int)rank;
+        mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 142);
+        tc_fence_after();
+        // the thread's 128 columns (four passes of 32) in one batch of TMEM
+        // loads; the buffer is released to the MMA before any store
+        uint32_t r[4][32];
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 256 + p * 64 + 32 * h, r[p]);
+        tmem_wait_ld();
+        tc_fence_before();
+#pragma unroll
+        for (int p = 0; p < 4; ++p, ++npass) {
+          // the store that last used this staging box (two passes back) has read it
+          if (et == 0 && npass >= 2) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+          if (named_bar_or(1, NET, *abort_flag != 0)) {
+            ok = false;
+            break;
+          }
+          // every epilogue thread of this CTA has read the accumulator
+          if (p == 0 && et == 32) mbar_arrive_cluster(acce_lead + 8 * b);
+          uint8_t* ost = smem + OFF_O + (npass & 1) * BOX;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *(uint4*)(ost + row * 128 + (((4 * h + j) ^ (row & 7)) << 4)) = make_uint4(
+                pack_bf16x2(__uint_as_float(r[p][8 * j]), __uint_as_float(r[p][8 * j + 1])),
+                pack_bf16x2(__uint_as_float(r[p][8 * j + 2]), __uint_as_float(r[p][8 * j + 3])),
+                pack_bf16x2(__uint_as_float(r[p][8 * j + 4]), __uint_as_float(r[p][8 * j + 5])),
+                pack_bf16x2(__uint_as_float(r[p][8 * j + 6]), __uint_as_float(r[p][8 * j + 7])));
+          fence_proxy_async();
+          named_bar_sync(1, NET);
+          if (et == 0) {
+            if (tok0 < S) tma_store_3d(&tmO, smem_u32(ost), 64 * p, tok0, n);
+            bulk_commit();  // one group per pass, empty past S, so the waits above count passes
+          }
+        }
+        if (!ok) break;
+      }
+    }
+    if (et == 0) bulk_wait0();
+  }
+  // Teardown: every MMA of the pair has completed (bar_fin, multicast), and
+  // neither CTA leaves while the other may still arrive on its barriers.
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1 && lane == 0) {
+    volatile int keep_waiting = 0;
+    mbar_wait(bar_fin, 0, &keep_waiting, &g_tc_status, 143);
+  }
+  __syncwarp();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
+// Clusters of two CTAs of `kernel` (with `smem` bytes of dynamic shared
+// memory each) that can be resident at once; 0 if none.
+template <class K>
+static int max_active_pairs(K kernel, int threads, int smem) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * num_sms());
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+template <class K, class... Args>
+static cudaError_t launch_pairs(K kernel, int npair, int threads, int smem, cudaStream_t st,
+                                Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * npair);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 static cudaError_t tc_contract256(const void* k, const void* v, const float* beta, float* A,
                                   float* U, long long N, int S, float cA, float cU, int a_image,
                                   cudaStream_t st) {
+  {
+    // CTA pairs: each byte of K and V loaded and multiplied once
+    static DeviceOnce pair_once;
+    static int pairs_per_dev[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const cudaError_t pe = once_per_device(pair_once, [&]() -> cudaError_t {
+      cudaError_t e = cudaFuncSetAttribute(k_contract256_pair_tc,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, cp256::SMEM);
+      if (e != cudaSuccess) return e;
+      pairs_per_dev[dev & 63] = max_active_pairs(k_contract256_pair_tc, cp256::THREADS, cp256::SMEM);
+      return cudaSuccess;
+    });
+    if (pe != cudaSuccess) return pe;
+    const int maxp = pairs_per_dev[dev & 63];
+    if (maxp > 0) {
+      CUtensorMap mk, mv;
+      cudaError_t e = make_map_bf16_3d(&mk, k, 256, S, N, 64, cp256::TOK);
+      if (e == cudaSuccess) e = make_map_bf16_3d(&mv, v, 256, S, N, 64, cp256::TOK);
+      if (e != cudaSuccess) return e;
+      const int npair = (int)(N < maxp ? N : maxp);
+      e = launch_pairs(k_contract256_pair_tc, npair, cp256::THREADS, cp256::SMEM, st, mk, mv, beta,
+                       A, U, (int)N, S, cA, cU, a_image);
+      count_launch();
+      return e;
+    }
+  }
   CUtensorMap mk, mv;
   cudaError_t e = make_map_bf16_3d(&mk, k, 256, S, N, 64, c256::TOK);
   if (e != cudaSuccess) return e;
@@ -3971,6 +4535,34 @@ static cudaError_t tc_contract256(const void* k, const void* v, const float* bet
 
 static cudaError_t tc_readout256(const void* q, const void* Sfr_hilo, void* out, long long N, int S,
                                  cudaStream_t st) {
+  {
+    // CTA pairs: each Q tile loaded once
+    static DeviceOnce pair_once;
+    static int pairs_per_dev[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const cudaError_t pe = once_per_device(pair_once, [&]() -> cudaError_t {
+      cudaError_t e = cudaFuncSetAttribute(k_readout256_pair_tc,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, rp256::SMEM);
+      if (e != cudaSuccess) return e;
+      pairs_per_dev[dev & 63] = max_active_pairs(k_readout256_pair_tc, rp256::THREADS, rp256::SMEM);
+      return cudaSuccess;
+    });
+    if (pe != cudaSuccess) return pe;
+    const int maxp = pairs_per_dev[dev & 63];
+    if (maxp > 0) {
+      CUtensorMap mq, ms, mo;
+      cudaError_t e = make_map_bf16_3d(&mq, q, 256, S, N, 64, rp256::TOK);
+      if (e == cudaSuccess) e = make_map_bf16_3d(&ms, Sfr_hilo, 256, 256, 2 * N, 64, 128);
+      if (e == cudaSuccess) e = make_map_bf16_3d(&mo, out, 256, S, N, 64, rp256::TOK);
+      if (e != cudaSuccess) return e;
+      const int npair = (int)(N < maxp ? N : maxp);
+      e = launch_pairs(k_readout256_pair_tc, npair, rp256::THREADS, rp256::SMEM, st, mq, ms, mo,
+                       (int)N, S);
+      count_launch();
+      return e;
+    }
+  }
   CUtensorMap mq, ms, mo;
   cudaError_t e = make_map_bf16_3d(&mq, q, 256, S, N, 64, r256::TOK);
   if (e == cudaSuccess) e = make_map_bf16_3d(&ms, Sfr_hilo, 256, 256, 2 * N, 64, 128);

@@ -412,11 +412,12 @@ GDN_API int gdn_selftest_wait(int arrive, long long limit_ns, gdn_stream_t strea
  * for tests of their accuracy: for pair i < D/4 of an axis half and position
  * pos < npos, writes (cos, sin) of pos * rope_base^(-2i/(D/2)) to
  * cs[2 * (i * npos + pos)], cs[2 * (i * npos + pos) + 1] (device, fp32,
- * 16-byte aligned, 2 * npos * D/4 floats). reduced = 0: the table the
- * contraction and the one-direction readout copy into shared memory (full
- * precision sine/cosine of the fp32 angle); reduced = 1: the angle reduced to
- * [-pi, pi] by Cody-Waite reduction and the hardware sine/cosine, as the
- * bidirectional readout computes them per token. npos in [1, 2^20].
+ * 16-byte aligned, 2 * npos * D/4 floats). reduced = 1: the angle reduced to
+ * [-pi, pi] by Cody-Waite reduction, then the hardware sine/cosine, as every
+ * fused-prologue kernel computes them (the contraction and the one-direction
+ * readout into a shared table at start-up, the bidirectional readout per
+ * token); reduced = 0: the full-precision sine/cosine of the same fp32 angle,
+ * for comparison. npos in [1, 2^20].
  * Returns a status. */
 GDN_API int gdn_rope_eval(int npos, int D, float rope_base, int reduced, float* cs,
                           gdn_stream_t stream);
