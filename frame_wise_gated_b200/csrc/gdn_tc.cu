@@ -3517,242 +3517,11 @@ cudaError_t tc_readout2(const void* q, const void* sfr_f, const void* sfr_r, voi
 }
 
 // ============================================================================
-// D = 256 tensor-core contraction and readout.
-// Contraction: two CTAs per frame-head, one per 128-row half i of A and U:
-//   A[128i.., :] += K_i^T (beta K),  U[128i.., :] += V_i^T (beta K)
-// as M = 128, N = 256 MMAs (all 512 TMEM columns, no double buffer); the two
-// halves of a frame-head run on neighbouring CTAs, so K is read once from
-// HBM and once from L2. Readout: two CTAs per frame-head, one per 128-column
-// half j of O = Q S^T, holding rows 128j.. of S (hi, lo: 128 KiB) while Q
-// streams as [128 tokens][128 channels] half tiles (K split in two).
+// D = 256 tensor-core contraction and readout, each on CTA pairs (clusters of
+// two CTAs sharing one tcgen05 MMA of M = 256): every byte of K, V and Q is
+// loaded by one CTA only and multiplied once.
 // ============================================================================
-namespace c256 {
-constexpr int D = 256;
-constexpr int TOK = 32;                 // tokens per stage
-constexpr int NST = 8;                  // K/V stages
-constexpr int NBK = 2;                  // beta * K slots
-constexpr int BOX = TOK * 128;          // [32 tokens][64 channels]: 4 KiB
-constexpr int KT = 4 * BOX;             // K stage tile, all channels: 16 KiB
-constexpr int VT = 2 * BOX;             // V stage tile, one channel half: 8 KiB
-constexpr int OFF_K = 0;
-constexpr int OFF_V = OFF_K + NST * KT;
-constexpr int OFF_BK = OFF_V + NST * VT;
-constexpr int OFF_BETA = OFF_BK + NBK * KT;
-constexpr int OFF_BAR = OFF_BETA + NST * TOK * 4;
-constexpr int NBAR = 2 * NST + 2 * NBK + 3;  // full, empty; bk_full, bk_empty; acc_full, acc_empty, fin
-constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr int SMEM = OFF_MISC + 16 + 1024;
-static_assert(SMEM <= 232448, "D = 256 contraction shared memory");
-constexpr int NSC = 256;
-constexpr int THREADS = 64 + NSC + 128;
-constexpr uint32_t TMEM_COLS = 512;
-}  // namespace c256
-
 __device__ __forceinline__ int img256_off(int k, int n8);
-
-__global__ void __launch_bounds__(c256::THREADS, 1)
-    k_contract256_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                     const float* __restrict__ beta, float* __restrict__ A, float* __restrict__ U,
-                     int N, int S, float cA, float cU, int a_image) {
-  using namespace c256;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
-  const uint32_t sb = smem_u32(smem);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t bar_full = sb + OFF_BAR;
-  const uint32_t bar_empty = bar_full + 8 * NST;
-  const uint32_t bar_bkf = bar_empty + 8 * NST;
-  const uint32_t bar_bke = bar_bkf + 8 * NBK;
-  const uint32_t bar_accf = bar_bke + 8 * NBK;
-  const uint32_t bar_acce = bar_accf + 8;
-  const uint32_t bar_fin = bar_acce + 8;
-  uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
-  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < NST; ++s) {
-      mbar_init(bar_full + 8 * s, 33);
-      mbar_init(bar_empty + 8 * s, 1);
-    }
-    for (int s = 0; s < NBK; ++s) {
-      mbar_init(bar_bkf + 8 * s, NSC / 32);
-      mbar_init(bar_bke + 8 * s, 1);
-    }
-    mbar_init(bar_accf, 1);
-    mbar_init(bar_acce, 4);
-    mbar_init(bar_fin, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-  const int nst_frame = (S + TOK - 1) / TOK;
-  const int NU = 2 * N;
-  const int my_count = (int)blockIdx.x < NU ? (NU - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-
-  if (warp == 0) {
-    int g = 0;
-    bool ok = true;
-    for (int i = 0; i < my_count && ok; ++i) {
-      const int unit = blockIdx.x + i * gridDim.x, n = unit >> 1, half = unit & 1;
-      for (int st = 0; st < nst_frame; ++st, ++g) {
-        const int s = g % NST;
-        const uint32_t u = (uint32_t)(g / NST);
-        if (lane == 0) ok = mbar_wait(bar_empty + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 101);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(bar_full + 8 * s, KT + VT);
-#pragma unroll
-          for (int x = 0; x < 4; ++x)
-            tma_load_3d(sb + OFF_K + s * KT + x * BOX, &tmK, bar_full + 8 * s, 64 * x, st * TOK, n);
-#pragma unroll
-          for (int x = 0; x < 2; ++x)
-            tma_load_3d(sb + OFF_V + s * VT + x * BOX, &tmV, bar_full + 8 * s, 128 * half + 64 * x,
-                        st * TOK, n);
-        }
-        const uint32_t bsa = sb + OFF_BETA + s * TOK * 4;
-#pragma unroll
-        for (int r = lane; r < TOK; r += 32) {
-          const int tok = st * TOK + r;
-          const bool in = tok < S;
-          cp_async_4(bsa + r * 4, beta + (size_t)n * S + (in ? tok : 0), in ? 4u : 0u);
-        }
-        cp_async_arrive_noinc(bar_full + 8 * s);
-      }
-    }
-    if (lane == 0)
-      for (int gg = (g > NST ? g - NST : 0); gg < g; ++gg)
-        mbar_wait(bar_full + 8 * (gg % NST), (uint32_t)(gg / NST) & 1, abort_flag, &g_tc_status, 102);
-    __syncwarp();
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, 256, true, true);
-      int g = 0;
-      bool ok = true;
-      for (int i = 0; i < my_count && ok; ++i) {
-        const int half = (blockIdx.x + i * gridDim.x) & 1;
-        ok = mbar_wait(bar_acce, ((uint32_t)i & 1) ^ 1, abort_flag, &g_tc_status, 103);
-        if (!ok) break;
-        tc_fence_after();
-        for (int st = 0; st < nst_frame; ++st, ++g) {
-          const int s = g % NST, kb = g % NBK;
-          ok = mbar_wait(bar_bkf + 8 * kb, (uint32_t)(g / NBK) & 1, abort_flag, &g_tc_status, 104);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t ka = sb + OFF_K + s * KT + 2 * half * BOX, va = sb + OFF_V + s * VT,
-                         ba = sb + OFF_BK + kb * KT;
-#pragma unroll
-          for (int kk = 0; kk < TOK / 16; ++kk) {
-            const uint64_t db = smem_desc_sw128(ba + kk * 2048, BOX, 1024);
-            const uint32_t acc = (st > 0 || kk > 0) ? 1u : 0u;
-            mma_bf16(tmem, smem_desc_sw128(ka + kk * 2048, BOX, 1024), db, idesc, acc);
-            mma_bf16(tmem + 256, smem_desc_sw128(va + kk * 2048, BOX, 1024), db, idesc, acc);
-          }
-          mma_commit(bar_empty + 8 * s);
-          mma_commit(bar_bke + 8 * kb);
-        }
-        if (!ok) break;
-        mma_commit(bar_accf);
-      }
-      mma_commit(bar_fin);
-      mbar_wait(bar_fin, 0, abort_flag, &g_tc_status, 105);
-    }
-    __syncwarp();
-  } else if (warp < 2 + NSC / 32) {
-    const int t = threadIdx.x - 64;
-    int g = 0;
-    bool ok = true;
-    for (int i = 0; i < my_count && ok; ++i) {
-      for (int st = 0; st < nst_frame; ++st, ++g) {
-        const int s = g % NST, kb = g % NBK;
-        const uint32_t u = (uint32_t)(g / NST);
-        ok = mbar_wait(bar_full + 8 * s, u & 1, abort_flag, &g_tc_status, 106);
-        // the slot's previous beta * K has been consumed by its MMAs
-        if (ok) ok = mbar_wait(bar_bke + 8 * kb, ((uint32_t)(g / NBK) & 1) ^ 1, abort_flag, &g_tc_status, 108);
-        if (!ok) break;
-        const uint8_t* kt = smem + OFF_K + s * KT;
-        uint8_t* bt = smem + OFF_BK + kb * KT;
-        const float* bs = (const float*)(smem + OFF_BETA) + s * TOK;
-#pragma unroll
-        for (int m = 0; m < (KT / 16) / NSC; ++m) {
-          const int c = t + NSC * m;
-          const float bv = bs[(c >> 3) & (TOK - 1)];
-          uint4 x = *(const uint4*)(kt + c * 16);
-          uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
-            w[e] = pack_bf16x2(f.x * bv, f.y * bv);
-          }
-          *(uint4*)(bt + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        fence_proxy_async();
-        warp_arrive(bar_bkf + 8 * kb);
-      }
-    }
-  } else {
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
-    for (int i = 0; i < my_count; ++i) {
-      const int unit = blockIdx.x + i * gridDim.x, n = unit >> 1, half = unit & 1;
-      if (!mbar_wait(bar_accf, (uint32_t)i & 1, abort_flag, &g_tc_status, 107)) break;
-      tc_fence_after();
-#pragma unroll
-      for (int mat = 0; mat < 2; ++mat) {
-        float* dst = (mat ? U : A) + ((size_t)n * D + 128 * half + row) * D;
-        uint8_t* img = (uint8_t*)A + (size_t)n * D * D * 4;
-        const int k = 128 * half + row;
-        const float sc = mat ? cU : cA;
-        for (int c0 = 0; c0 < 256; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + mat * 256 + c0, r);
-          tmem_wait_ld();
-          if (mat == 0 && a_image) {
-            // row k of A_t into the operand image (hi, lo) of the D = 256 chains
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              float v[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(r[8 * j + e]) * sc;
-              uint4 hi, lo;
-              split_chunk(v, &hi, &lo);
-              const int off = img256_off(k, (c0 >> 3) + j);
-              *(uint4*)(img + off) = hi;
-              *(uint4*)(img + off + 8192) = lo;
-            }
-          } else if (mat == 1 && a_image) {
-            // U_t transposed for the D = 256 chains (their epilogue reads a
-            // column of U^T per row, 32 rows per warp: coalesced); each warp
-            // here writes 32 consecutive floats of a row of U^T
-            float* ut = U + (size_t)n * D * D + k;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) ut[(size_t)(c0 + j) * D] = __uint_as_float(r[j]) * sc;
-          } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              *(float4*)(dst + c0 + 4 * j) =
-                  make_float4(__uint_as_float(r[4 * j]) * sc, __uint_as_float(r[4 * j + 1]) * sc,
-                              __uint_as_float(r[4 * j + 2]) * sc, __uint_as_float(r[4 * j + 3]) * sc);
-          }
-        }
-      }
-      tc_fence_before();
-      warp_arrive(bar_acce);
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
-  }
-}
 
 // D = 256 contraction on a CTA pair (a cluster of two CTAs, one tcgen05
 // MMA of M = 256 over both). Per frame-head and 64-token stage CTA r of the
@@ -3764,7 +3533,9 @@ __global__ void __launch_bounds__(c256::THREADS, 1)
 // by columns over the two CTAs' shared memory, so each byte of K and V is
 // read from memory once and multiplied once. CTA r's TMEM receives rows
 // 128r .. of A (columns 0-255) and of U (256-511); its eight epilogue warps
-// (four on A, four on U) write them as k_contract256_tc does. Barriers: stage
+// (four on A, four on U) write rows 128r .. of A_t as the bf16 (hi, lo)
+// operand image of the D = 256 chains and of U_t transposed (or both in fp32
+// when no image is asked for). Barriers: stage
 // and beta*K slot releases are multicast MMA commits to both CTAs. The even
 // CTA's scalers arrive on its slot barrier directly; the odd CTA's arrive on
 // a local barrier, and a relay warp per slot forwards each completed use of
@@ -4020,198 +3791,6 @@ __global__ void __launch_bounds__(cp256::THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc_pair(tmem, TMEM_COLS);
-  }
-}
-
-namespace r256 {
-constexpr int D = 256;
-constexpr int TOK = 128;
-constexpr int NQ = 2;
-constexpr int BOX = TOK * 128;           // [128 rows][64 channels]: 16 KiB
-constexpr int QH = 2 * BOX;              // Q half tile (128 channels): 32 KiB
-static_assert(2 * QH == TOK * D * 2, "two half tiles hold a tile's D bf16 channels");
-constexpr int OFF_Q = 0;
-constexpr int OFF_S = OFF_Q + NQ * QH;   // S rows half: hi 4 atoms, lo 4 atoms (128 KiB)
-constexpr int OFF_O = OFF_S + 8 * BOX;   // output staging: 2 boxes
-constexpr int OFF_BAR = OFF_O + 2 * BOX;
-constexpr int NBAR = 2 * NQ + 2 + 4 + 1;
-constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr int SMEM = OFF_MISC + 16 + 1024;
-constexpr int THREADS = 192;
-constexpr uint32_t TMEM_COLS = 256;
-}  // namespace r256
-
-__global__ void __launch_bounds__(r256::THREADS, 1)
-    k_readout256_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
-                    const __grid_constant__ CUtensorMap tmO, int N, int S) {
-  using namespace r256;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
-  const uint32_t sb = smem_u32(smem);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t bar_qf = sb + OFF_BAR;
-  const uint32_t bar_qe = bar_qf + 8 * NQ;
-  const uint32_t bar_sf = bar_qe + 8 * NQ;
-  const uint32_t bar_se = bar_sf + 8;
-  const uint32_t bar_accf = bar_se + 8;
-  const uint32_t bar_acce = bar_accf + 16;
-  const uint32_t bar_fin = bar_acce + 16;
-  uint32_t* tmem_holder = (uint32_t*)(smem + OFF_MISC);
-  volatile int* abort_flag = (volatile int*)(smem + OFF_MISC + 4);
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < NQ; ++s) {
-      mbar_init(bar_qf + 8 * s, 1);
-      mbar_init(bar_qe + 8 * s, 1);
-    }
-    mbar_init(bar_sf, 1);
-    mbar_init(bar_se, 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar_accf + 8 * b, 1);
-      mbar_init(bar_acce + 8 * b, 4);
-    }
-    mbar_init(bar_fin, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-  const int ntile = (S + TOK - 1) / TOK;
-  const int NU = 2 * N;
-  const int my_count = (int)blockIdx.x < NU ? (NU - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      int g = 0;
-      bool ok = true;
-      for (int i = 0; i < my_count && ok; ++i) {
-        const int unit = blockIdx.x + i * gridDim.x, n = unit >> 1, half = unit & 1;
-        ok = mbar_wait(bar_se, ((uint32_t)i & 1) ^ 1, abort_flag, &g_tc_status, 111);
-        if (!ok) break;
-        mbar_arrive_expect_tx(bar_sf, 8 * BOX);
-#pragma unroll
-        for (int hl = 0; hl < 2; ++hl)
-#pragma unroll
-          for (int x = 0; x < 4; ++x)
-            tma_load_3d(sb + OFF_S + (4 * hl + x) * BOX, &tmS, bar_sf, 64 * x, 128 * half, 2 * n + hl);
-        for (int tl = 0; tl < ntile && ok; ++tl)
-          for (int kh = 0; kh < 2; ++kh, ++g) {
-            const int s = g % NQ;
-            const uint32_t u = (uint32_t)(g / NQ);
-            ok = mbar_wait(bar_qe + 8 * s, (u & 1) ^ 1, abort_flag, &g_tc_status, 112);
-            if (!ok) break;
-            const uint32_t qd = sb + OFF_Q + s * QH;
-            mbar_arrive_expect_tx(bar_qf + 8 * s, QH);
-            tma_load_3d(qd, &tmQ, bar_qf + 8 * s, 128 * kh, tl * TOK, n);
-            tma_load_3d(qd + BOX, &tmQ, bar_qf + 8 * s, 128 * kh + 64, tl * TOK, n);
-          }
-      }
-      for (int gg = (g > NQ ? g - NQ : 0); gg < g; ++gg)
-        mbar_wait(bar_qf + 8 * (gg % NQ), (uint32_t)(gg / NQ) & 1, abort_flag, &g_tc_status, 113);
-      if (my_count > 0) mbar_wait(bar_sf, (uint32_t)(my_count - 1) & 1, abort_flag, &g_tc_status, 114);
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
-      int g = 0, gt = 0;
-      bool ok = true;
-      for (int i = 0; i < my_count && ok; ++i) {
-        ok = mbar_wait(bar_sf, (uint32_t)i & 1, abort_flag, &g_tc_status, 115);
-        if (!ok) break;
-        tc_fence_after();
-        for (int tl = 0; tl < ntile && ok; ++tl, ++gt) {
-          const int b = gt & 1;
-          const uint32_t ub = (uint32_t)(gt >> 1);
-          ok = mbar_wait(bar_acce + 8 * b, (ub & 1) ^ 1, abort_flag, &g_tc_status, 116);
-          if (!ok) break;
-          const uint32_t d = tmem + b * 128;
-          for (int kh = 0; kh < 2 && ok; ++kh, ++g) {
-            const int s = g % NQ;
-            const uint32_t u = (uint32_t)(g / NQ);
-            ok = mbar_wait(bar_qf + 8 * s, u & 1, abort_flag, &g_tc_status, 117);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t qa = sb + OFF_Q + s * QH;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t qoff = (kk >> 2) * BOX + (kk & 3) * 32;
-              const uint32_t soff = (2 * kh + (kk >> 2)) * BOX + (kk & 3) * 32;
-              const uint64_t dq = smem_desc_sw128(qa + qoff, 16, 1024);
-              mma_bf16(d, dq, smem_desc_sw128(sb + OFF_S + soff, 16, 1024), idesc,
-                       (kh > 0 || kk > 0) ? 1u : 0u);
-              mma_bf16(d, dq, smem_desc_sw128(sb + OFF_S + 4 * BOX + soff, 16, 1024), idesc, 1u);
-            }
-            mma_commit(bar_qe + 8 * s);
-          }
-          if (!ok) break;
-          mma_commit(bar_accf + 8 * b);
-        }
-        if (!ok) break;
-        mma_commit(bar_se);
-      }
-      mma_commit(bar_fin);
-      mbar_wait(bar_fin, 0, abort_flag, &g_tc_status, 118);
-    }
-    __syncwarp();
-  } else {
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
-    const int et = threadIdx.x - 64;
-    uint8_t* ost = smem + OFF_O;
-    int gt = 0;
-    bool ok = true;
-    for (int i = 0; i < my_count && ok; ++i) {
-      const int unit = blockIdx.x + i * gridDim.x, n = unit >> 1, half = unit & 1;
-      for (int tl = 0; tl < ntile; ++tl, ++gt) {
-        const int b = gt & 1;
-        const uint32_t ub = (uint32_t)(gt >> 1);
-        mbar_wait(bar_accf + 8 * b, ub & 1, abort_flag, &g_tc_status, 119);
-        tc_fence_after();
-        if (et == 0) bulk_wait_read0();
-        if (named_bar_or(1, 128, *abort_flag != 0)) {
-          ok = false;
-          break;
-        }
-#pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-#pragma unroll
-          for (int c0 = 0; c0 < 64; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 128 + hb * 64 + c0, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              *(uint4*)(ost + hb * BOX + row * 128 + ((((c0 >> 3) + j) ^ (row & 7)) << 4)) = make_uint4(
-                  pack_bf16x2(__uint_as_float(r[8 * j]), __uint_as_float(r[8 * j + 1])),
-                  pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3])),
-                  pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5])),
-                  pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7])));
-          }
-        }
-        tc_fence_before();
-        warp_arrive(bar_acce + 8 * b);
-        fence_proxy_async();
-        named_bar_sync(1, 128);
-        if (et == 0) {
-          tma_store_3d(&tmO, sb + OFF_O, 128 * half, tl * TOK, n);
-          tma_store_3d(&tmO, sb + OFF_O + BOX, 128 * half + 64, tl * TOK, n);
-          bulk_commit();
-        }
-      }
-    }
-    if (et == 0) bulk_wait0();
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
@@ -4487,98 +4066,56 @@ static cudaError_t launch_pairs(K kernel, int npair, int threads, int smem, cuda
 static cudaError_t tc_contract256(const void* k, const void* v, const float* beta, float* A,
                                   float* U, long long N, int S, float cA, float cU, int a_image,
                                   cudaStream_t st) {
-  {
-    // CTA pairs: each byte of K and V loaded and multiplied once
-    static DeviceOnce pair_once;
-    static int pairs_per_dev[64];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    const cudaError_t pe = once_per_device(pair_once, [&]() -> cudaError_t {
-      cudaError_t e = cudaFuncSetAttribute(k_contract256_pair_tc,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, cp256::SMEM);
-      if (e != cudaSuccess) return e;
-      pairs_per_dev[dev & 63] = max_active_pairs(k_contract256_pair_tc, cp256::THREADS, cp256::SMEM);
-      return cudaSuccess;
-    });
-    if (pe != cudaSuccess) return pe;
-    const int maxp = pairs_per_dev[dev & 63];
-    if (maxp > 0) {
-      CUtensorMap mk, mv;
-      cudaError_t e = make_map_bf16_3d(&mk, k, 256, S, N, 64, cp256::TOK);
-      if (e == cudaSuccess) e = make_map_bf16_3d(&mv, v, 256, S, N, 64, cp256::TOK);
-      if (e != cudaSuccess) return e;
-      const int npair = (int)(N < maxp ? N : maxp);
-      e = launch_pairs(k_contract256_pair_tc, npair, cp256::THREADS, cp256::SMEM, st, mk, mv, beta,
-                       A, U, (int)N, S, cA, cU, a_image);
-      count_launch();
-      return e;
-    }
-  }
-  CUtensorMap mk, mv;
-  cudaError_t e = make_map_bf16_3d(&mk, k, 256, S, N, 64, c256::TOK);
-  if (e != cudaSuccess) return e;
-  e = make_map_bf16_3d(&mv, v, 256, S, N, 64, c256::TOK);
-  if (e != cudaSuccess) return e;
-  static DeviceOnce attr_once;
-  const cudaError_t attr_status = once_per_device(attr_once, [&]() -> cudaError_t {
-    cudaError_t e = cudaFuncSetAttribute(k_contract256_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, c256::SMEM);
-    return e;
+  static DeviceOnce pair_once;
+  static int pairs_per_dev[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const cudaError_t pe = once_per_device(pair_once, [&]() -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(k_contract256_pair_tc,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, cp256::SMEM);
+    if (e != cudaSuccess) return e;
+    pairs_per_dev[dev & 63] = max_active_pairs(k_contract256_pair_tc, cp256::THREADS, cp256::SMEM);
+    return cudaSuccess;
   });
-  if (attr_status != cudaSuccess) return attr_status;
-  const long long units = 2 * N;
-  const int grid = (int)(units < num_sms() ? units : num_sms());
-  k_contract256_tc<<<grid, c256::THREADS, c256::SMEM, st>>>(mk, mv, beta, A, U, (int)N, S, cA, cU,
-                                                            a_image);
+  if (pe != cudaSuccess) return pe;
+  const int maxp = pairs_per_dev[dev & 63];
+  if (maxp <= 0) return cudaErrorNotSupported;  // no cluster of two can be resident
+  CUtensorMap mk, mv;
+  cudaError_t e = make_map_bf16_3d(&mk, k, 256, S, N, 64, cp256::TOK);
+  if (e == cudaSuccess) e = make_map_bf16_3d(&mv, v, 256, S, N, 64, cp256::TOK);
+  if (e != cudaSuccess) return e;
+  const int npair = (int)(N < maxp ? N : maxp);
+  e = launch_pairs(k_contract256_pair_tc, npair, cp256::THREADS, cp256::SMEM, st, mk, mv, beta, A, U,
+                   (int)N, S, cA, cU, a_image);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 static cudaError_t tc_readout256(const void* q, const void* Sfr_hilo, void* out, long long N, int S,
                                  cudaStream_t st) {
-  {
-    // CTA pairs: each Q tile loaded once
-    static DeviceOnce pair_once;
-    static int pairs_per_dev[64];
-    int dev = 0;
-    cudaGetDevice(&dev);
-    const cudaError_t pe = once_per_device(pair_once, [&]() -> cudaError_t {
-      cudaError_t e = cudaFuncSetAttribute(k_readout256_pair_tc,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, rp256::SMEM);
-      if (e != cudaSuccess) return e;
-      pairs_per_dev[dev & 63] = max_active_pairs(k_readout256_pair_tc, rp256::THREADS, rp256::SMEM);
-      return cudaSuccess;
-    });
-    if (pe != cudaSuccess) return pe;
-    const int maxp = pairs_per_dev[dev & 63];
-    if (maxp > 0) {
-      CUtensorMap mq, ms, mo;
-      cudaError_t e = make_map_bf16_3d(&mq, q, 256, S, N, 64, rp256::TOK);
-      if (e == cudaSuccess) e = make_map_bf16_3d(&ms, Sfr_hilo, 256, 256, 2 * N, 64, 128);
-      if (e == cudaSuccess) e = make_map_bf16_3d(&mo, out, 256, S, N, 64, rp256::TOK);
-      if (e != cudaSuccess) return e;
-      const int npair = (int)(N < maxp ? N : maxp);
-      e = launch_pairs(k_readout256_pair_tc, npair, rp256::THREADS, rp256::SMEM, st, mq, ms, mo,
-                       (int)N, S);
-      count_launch();
-      return e;
-    }
-  }
-  CUtensorMap mq, ms, mo;
-  cudaError_t e = make_map_bf16_3d(&mq, q, 256, S, N, 64, r256::TOK);
-  if (e == cudaSuccess) e = make_map_bf16_3d(&ms, Sfr_hilo, 256, 256, 2 * N, 64, 128);
-  if (e == cudaSuccess) e = make_map_bf16_3d(&mo, out, 256, S, N, 64, r256::TOK);
-  if (e != cudaSuccess) return e;
-  static DeviceOnce attr_once;
-  const cudaError_t attr_status = once_per_device(attr_once, [&]() -> cudaError_t {
-    cudaError_t e = cudaFuncSetAttribute(k_readout256_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, r256::SMEM);
-    return e;
+  static DeviceOnce pair_once;
+  static int pairs_per_dev[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const cudaError_t pe = once_per_device(pair_once, [&]() -> cudaError_t {
+    cudaError_t e = cudaFuncSetAttribute(k_readout256_pair_tc,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, rp256::SMEM);
+    if (e != cudaSuccess) return e;
+    pairs_per_dev[dev & 63] = max_active_pairs(k_readout256_pair_tc, rp256::THREADS, rp256::SMEM);
+    return cudaSuccess;
   });
-  if (attr_status != cudaSuccess) return attr_status;
-  const long long units = 2 * N;
-  const int grid = (int)(units < num_sms() ? units : num_sms());
-  k_readout256_tc<<<grid, r256::THREADS, r256::SMEM, st>>>(mq, ms, mo, (int)N, S);
+  if (pe != cudaSuccess) return pe;
+  const int maxp = pairs_per_dev[dev & 63];
+  if (maxp <= 0) return cudaErrorNotSupported;  // no cluster of two can be resident
+  CUtensorMap mq, ms, mo;
+  cudaError_t e = make_map_bf16_3d(&mq, q, 256, S, N, 64, rp256::TOK);
+  if (e == cudaSuccess) e = make_map_bf16_3d(&ms, Sfr_hilo, 256, 256, 2 * N, 64, 128);
+  if (e == cudaSuccess) e = make_map_bf16_3d(&mo, out, 256, S, N, 64, rp256::TOK);
+  if (e != cudaSuccess) return e;
+  const int npair = (int)(N < maxp ? N : maxp);
+  e = launch_pairs(k_readout256_pair_tc, npair, rp256::THREADS, rp256::SMEM, st, mq, ms, mo, (int)N, S);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 // ============================================================================
