@@ -39,6 +39,12 @@
  *  - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *    stream); no entry point synchronises the host except
  *    gdn_check_device_status.
+ *  - Execution: the library is built for sm_100a (B200) only. bf16 inputs
+ *    at D in {64, 128, 256} run on the tensor cores (tcgen05, TMA); at
+ *    D = 256 the contraction and the readout launch clusters of two CTAs
+ *    that share one MMA, and a device that cannot hold such a cluster makes
+ *    those calls return GDN_ERR_CUDA. fp32 inputs, D in {16, 32} and
+ *    GDN_FORCE_SIMT run on CUDA cores.
  *  - Errors: argument errors return GDN_ERR_INVALID / GDN_ERR_UNSUPPORTED
  *    before anything is launched; a failed launch returns GDN_ERR_CUDA; a
  *    device-side bounded wait that ran out is reported by
