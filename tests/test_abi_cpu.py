@@ -74,6 +74,22 @@ def test_product_path_does_not_import_the_oracle():
                 assert "import oracle" not in txt and "from oracle" not in txt, f
 
 
+def test_kernel_loads_never_multicast():
+    """Every TMA or bulk load in the kernels writes only the issuing CTA's own
+    shared memory: the only PTX that multicasts across a cluster is the MMA
+    completion (tcgen05.commit) that releases a CTA pair's barriers."""
+    needle = "multicast" + "::" + "cluster"  # split so this file names no such load
+    csrc = os.path.join(ROOT, "frame_wise_gated_b200", "csrc")
+    found = 0
+    for f in sorted(os.listdir(csrc)):
+        txt = open(os.path.join(csrc, f), encoding="utf-8").read()
+        for line in re.findall(r'"([^"\n]*)"', txt):  # string literals: the inline PTX
+            if needle in line:
+                found += 1
+                assert line.lstrip().startswith("tcgen05.commit"), (f, line)
+    assert found >= 1  # the pair kernels' commits
+
+
 def test_fault_injection_fails_before_any_launch(lib):
     """The armed injection turns the next scan call, once its arguments pass
     the checks, into GDN_ERR_CUDA without a launch (no GPU needed: the
